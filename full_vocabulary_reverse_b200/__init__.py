@@ -1,0 +1,14 @@
+"""B200-native exact full-vocabulary reverse-KL distillation loss.
+
+The compute runs in ``librkl.so`` (hand-written sm_100a CUDA kernels behind a
+C ABI, see ``include/rkl.h``); this package only loads it and marshals
+arguments.  There is no CPU or PyTorch fallback: if the library is missing,
+every call raises.
+"""
+
+from .binding import (  # noqa: F401
+    RKLError, lib, compact_rows, forward_hidden, forward_logits, backward,
+    workspace_size, device_error, reverse_kl_hidden, reverse_kl_logits,
+    REDUCE_NONE, REDUCE_TOKEN_MEAN, REDUCE_SEQ_MEAN_NESTED,
+    PAYLOAD_HIDDEN, PAYLOAD_LOGITS,
+)

@@ -1,0 +1,231 @@
+"""ctypes binding of librkl.so (argument marshalling only).
+
+Every step of the loss runs in the CUDA library; this module allocates the
+caller-side tensors with PyTorch, passes raw device pointers and the current
+stream, and raises ``RKLError`` on any non-OK status.  There is no fallback:
+if ``librkl.so`` is missing or fails to load, every call raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "librkl.so")
+
+REDUCE_NONE = 0
+REDUCE_TOKEN_MEAN = 1
+REDUCE_SEQ_MEAN_NESTED = 2
+PAYLOAD_HIDDEN = 0
+PAYLOAD_LOGITS = 1
+DT_BF16 = 0
+DT_FP32 = 1
+
+_STATUS = {0: "RKL_OK", 1: "RKL_ERR_NULL", 2: "RKL_ERR_SHAPE", 3: "RKL_ERR_DTYPE",
+           4: "RKL_ERR_ALIGN", 5: "RKL_ERR_WORKSPACE", 6: "RKL_ERR_UNSUPPORTED",
+           7: "RKL_ERR_CUDA", 8: "RKL_ERR_DEVICE"}
+
+
+class RKLError(RuntimeError):
+    def __init__(self, status, msg):
+        super().__init__("%s: %s" % (_STATUS.get(status, status), msg))
+        self.status = status
+
+
+_lib = None
+
+_vp = ctypes.c_void_p
+_i64 = ctypes.c_int64
+_i32 = ctypes.c_int32
+_sz = ctypes.c_size_t
+
+_SIGS = {
+    "rkl_version": ([], ctypes.c_char_p),
+    "rkl_last_error": ([], ctypes.c_char_p),
+    "rkl_workspace_size": ([_i32, _i32, _i64, _i64, _i64, _i64, _i64, ctypes.POINTER(_sz)], _i32),
+    "rkl_compact_rows": ([_vp, _i64, _i64, _vp, _vp, _vp], _i32),
+    "rkl_forward_hidden": ([_vp, _vp, _vp, _vp, _i32, _i64, _i64, _i64, _i64, _vp, _i32, _i32,
+                            _vp, _vp, _vp, _vp, _sz, _vp], _i32),
+    "rkl_forward_logits": ([_vp, _vp, _vp, _i32, _i64, _i64, _i64, _i64, _vp, _i32, _i32,
+                            _vp, _vp, _vp, _vp, _sz, _vp], _i32),
+    "rkl_backward": ([_i32, _vp, _vp, _vp, _vp, _i32, _i64, _i64, _i64, _i64, _vp, _i32, _i32,
+                      _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp], _i32),
+    "rkl_device_error": ([ctypes.POINTER(_i32)], _i32),
+    "rkl_kernel_count": ([], _i32),
+    "rkl_kernel_name": ([_i32], ctypes.c_char_p),
+    "rkl_profile_enable": ([_i32], _i32),
+    "rkl_profile_reset": ([], _i32),
+    "rkl_profile_read": ([_i32, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_i64)], _i32),
+    "rkl_launch_count": ([], _i64),
+}
+
+
+def lib():
+    """The loaded librkl.so (raises if it was not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RKLError(7, "librkl.so is not built (python -m full_vocabulary_reverse_b200.build)")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (args, res) in _SIGS.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = L
+    return _lib
+
+
+def _check(status):
+    if status != 0:
+        raise RKLError(status, lib().rkl_last_error().decode())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _dtype_code(t):
+    if t.dtype == torch.bfloat16:
+        return DT_BF16
+    if t.dtype == torch.float32:
+        return DT_FP32
+    raise RKLError(3, "unsupported dtype %s" % (t.dtype,))
+
+
+def workspace_size(payload, dtype_code, n_max, B, Sm1, H, V):
+    out = ctypes.c_size_t(0)
+    _check(lib().rkl_workspace_size(payload, dtype_code, n_max, B, Sm1, H, V, ctypes.byref(out)))
+    return out.value
+
+
+def _workspace(payload, dtype_code, n_max, B, Sm1, H, V, device):
+    nbytes = workspace_size(payload, dtype_code, n_max, B, Sm1, H, V)
+    return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+
+
+def compact_rows(mask):
+    """S1: (row_idx int32 [B*Sm1] device, N host int)."""
+    B, Sm1 = mask.shape
+    mask = mask.contiguous()
+    if mask.dtype != torch.uint8:
+        mask = (mask != 0).to(torch.uint8)
+    row_idx = torch.empty(B * Sm1, dtype=torch.int32, device=mask.device)
+    n_dev = torch.empty(1, dtype=torch.int32, device=mask.device)
+    _check(lib().rkl_compact_rows(_ptr(mask), B, Sm1, _ptr(row_idx), _ptr(n_dev), _stream(mask.device)))
+    return row_idx, int(n_dev.item())
+
+
+def forward_hidden(h_s, h_t, W_s, W_t, B, Sm1, row_idx, N, reduction, workspace=None):
+    """S2-S4 on the hidden payload.  Returns (loss_tok [B,Sm1], loss [1], saved [N,3])."""
+    dev = h_s.device
+    T, H = h_s.shape
+    V = W_s.shape[0]
+    dt = _dtype_code(h_s)
+    loss_tok = torch.empty((B, Sm1), dtype=torch.float32, device=dev)
+    loss = torch.empty(1, dtype=torch.float32, device=dev)
+    saved = torch.empty((max(N, 1), 3), dtype=torch.float32, device=dev)
+    ws = workspace if workspace is not None else _workspace(PAYLOAD_HIDDEN, dt, max(N, 1), B, Sm1, H, V, dev)
+    _check(lib().rkl_forward_hidden(_ptr(h_s), _ptr(h_t), _ptr(W_s), _ptr(W_t), dt, B, Sm1, H, V,
+                                    _ptr(row_idx), N, reduction, _ptr(loss_tok), _ptr(loss), _ptr(saved),
+                                    _ptr(ws), ws.numel(), _stream(dev)))
+    return loss_tok, loss, saved
+
+
+def forward_logits(h_s, W_s, teacher_logits, B, Sm1, row_idx, N, reduction, workspace=None):
+    """S2-S4 + S8 on the logits payload.  Returns (loss_tok, loss, saved)."""
+    dev = h_s.device
+    T, H = h_s.shape
+    V = W_s.shape[0]
+    dt = _dtype_code(h_s)
+    loss_tok = torch.empty((B, Sm1), dtype=torch.float32, device=dev)
+    loss = torch.empty(1, dtype=torch.float32, device=dev)
+    saved = torch.empty((max(N, 1), 3), dtype=torch.float32, device=dev)
+    ws = workspace if workspace is not None else _workspace(PAYLOAD_LOGITS, dt, max(N, 1), B, Sm1, H, V, dev)
+    _check(lib().rkl_forward_logits(_ptr(h_s), _ptr(W_s), _ptr(teacher_logits), dt, B, Sm1, H, V,
+                                    _ptr(row_idx), N, reduction, _ptr(loss_tok), _ptr(loss), _ptr(saved),
+                                    _ptr(ws), ws.numel(), _stream(dev)))
+    return loss_tok, loss, saved
+
+
+def backward(payload, h_s, teacher, W_s, W_t, B, Sm1, row_idx, N, reduction, saved,
+             grad_loss=None, grad_tok=None, workspace=None, dH_s=None, dW_s=None):
+    """S5-S7.  Returns (dH_s [T,H] fp32, dW_s [V,H] fp32)."""
+    dev = h_s.device
+    T, H = h_s.shape
+    V = W_s.shape[0]
+    dt = _dtype_code(h_s)
+    if dH_s is None:
+        dH_s = torch.empty((T, H), dtype=torch.float32, device=dev)
+    if dW_s is None:
+        dW_s = torch.empty((V, H), dtype=torch.float32, device=dev)
+    if grad_loss is not None:
+        grad_loss = grad_loss.reshape(1).to(device=dev, dtype=torch.float32).contiguous()
+    if grad_tok is not None:
+        grad_tok = grad_tok.to(device=dev, dtype=torch.float32).contiguous()
+    ws = workspace if workspace is not None else _workspace(payload, dt, max(N, 1), B, Sm1, H, V, dev)
+    _check(lib().rkl_backward(payload, _ptr(h_s), _ptr(teacher), _ptr(W_s), _ptr(W_t), dt, B, Sm1, H, V,
+                              _ptr(row_idx), N, reduction, _ptr(saved), _ptr(grad_loss), _ptr(grad_tok),
+                              _ptr(dH_s), _ptr(dW_s), _ptr(ws), ws.numel(), _stream(dev)))
+    return dH_s, dW_s
+
+
+def device_error():
+    code = ctypes.c_int32(0)
+    lib().rkl_device_error(ctypes.byref(code))
+    return code.value
+
+
+class _RKLHidden(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, h_s, h_t, W_s, W_t, mask, reduction):
+        B, Sm1 = mask.shape
+        row_idx, N = compact_rows(mask)
+        loss_tok, loss, saved = forward_hidden(h_s, h_t, W_s, W_t, B, Sm1, row_idx, N, reduction)
+        ctx.save_for_backward(h_s, h_t, W_s, W_t, row_idx, saved)
+        ctx.meta = (B, Sm1, N, reduction)
+        return loss.reshape(()), loss_tok
+
+    @staticmethod
+    def backward(ctx, g_loss, g_tok):
+        h_s, h_t, W_s, W_t, row_idx, saved = ctx.saved_tensors
+        B, Sm1, N, reduction = ctx.meta
+        dH, dW = backward(PAYLOAD_HIDDEN, h_s, h_t, W_s, W_t, B, Sm1, row_idx, N, reduction, saved,
+                          grad_loss=g_loss, grad_tok=g_tok)
+        return dH.to(h_s.dtype), None, dW.to(W_s.dtype), None, None, None
+
+
+class _RKLLogits(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, h_s, W_s, teacher_logits, mask, reduction):
+        B, Sm1 = mask.shape
+        row_idx, N = compact_rows(mask)
+        loss_tok, loss, saved = forward_logits(h_s, W_s, teacher_logits, B, Sm1, row_idx, N, reduction)
+        ctx.save_for_backward(h_s, W_s, teacher_logits, row_idx, saved)
+        ctx.meta = (B, Sm1, N, reduction)
+        return loss.reshape(()), loss_tok
+
+    @staticmethod
+    def backward(ctx, g_loss, g_tok):
+        h_s, W_s, logits, row_idx, saved = ctx.saved_tensors
+        B, Sm1, N, reduction = ctx.meta
+        dH, dW = backward(PAYLOAD_LOGITS, h_s, logits, W_s, None, B, Sm1, row_idx, N, reduction, saved,
+                          grad_loss=g_loss, grad_tok=g_tok)
+        return dH.to(h_s.dtype), dW.to(W_s.dtype), None, None, None
+
+
+def reverse_kl_hidden(h_s, h_t, W_s, W_t, mask, reduction=REDUCE_TOKEN_MEAN):
+    """Differentiable (loss, loss_tok) of the hidden-state payload; grads to h_s and W_s."""
+    return _RKLHidden.apply(h_s.contiguous(), h_t.contiguous(), W_s.contiguous(), W_t.contiguous(),
+                            mask, reduction)
+
+
+def reverse_kl_logits(h_s, W_s, teacher_logits, mask, reduction=REDUCE_TOKEN_MEAN):
+    """Differentiable (loss, loss_tok) of the logits payload; grads to h_s and W_s."""
+    return _RKLLogits.apply(h_s.contiguous(), W_s.contiguous(), teacher_logits.contiguous(), mask, reduction)

@@ -1,0 +1,171 @@
+/*
+ * rkl.h -- C ABI of librkl.so: exact full-vocabulary reverse-KL distillation
+ * loss on NVIDIA B200 (sm_100a).
+ *
+ * The operation (NeMo RL PR #3978, "feat(mopd): add full-vocabulary on-policy
+ * distillation", description):
+ *
+ *     L_t = sum_v p_s(v) * (log p_s(v) - log p_t(v)),   p = softmax(z)
+ *
+ * for every trainable position t of a [B, S-1] batch, where the student logits
+ * are z_s = h_s W_s^T and the teacher logits are either z_t = h_t W_t^T
+ * (hidden-state payload) or shipped directly (logits payload) -- same page,
+ * payload bullets.  Only the N loss-masked rows are projected ("fix(megatron):
+ * compact actor logits before projection", slime PR #2310, Summary).  The
+ * backward is the shared one of PR #3978's first implementation note,
+ * dL/dz_s = p_s * (w - L) with w = log p_s - log p_t, recomputing the
+ * log-softmaxes instead of caching [N, V].
+ *
+ * Conventions for every entry point:
+ *  - Row-major tensors.  T = B * Sm1 token rows; row r = b * Sm1 + t predicts
+ *    token t + 1 of sequence b.  h_* are [T, H]; W_* are [V, H]; teacher logits
+ *    are [T, V]; the mask and the per-token loss are [B, Sm1].
+ *  - All pointers are DEVICE pointers unless stated, owned by the caller.  The
+ *    library never allocates device memory: scratch comes from the caller's
+ *    workspace (size from rkl_workspace_size).  Teacher inputs are read-only
+ *    and get no gradient (PR #3978: the teacher LM head is "a plain tensor").
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream).  All work is
+ *    enqueued on it; no entry point synchronises the host except
+ *    rkl_device_error.
+ *  - Errors are returned, never thrown or aborted on.  Arguments are checked
+ *    before any launch; on error nothing is enqueued and rkl_last_error()
+ *    (thread-local) describes the problem.
+ *  - Data pointers must be 16-byte aligned (RKL_ERR_ALIGN).  For RKL_BF16, H
+ *    must be a multiple of 64 and, on the logits payload, V a multiple of 8
+ *    (row pitch of 16 bytes); RKL_FP32 accepts any H and V >= 1.
+ *  - Results are deterministic: the same inputs give bitwise-equal outputs,
+ *    and a row's loss and dH row do not depend on which other rows are in the
+ *    batch.
+ */
+#ifndef RKL_H
+#define RKL_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum rkl_status {
+  RKL_OK = 0,
+  RKL_ERR_NULL = 1,        /* a required pointer is NULL */
+  RKL_ERR_SHAPE = 2,       /* a size is out of range or inconsistent */
+  RKL_ERR_DTYPE = 3,       /* unknown dtype / payload / reduction enum value */
+  RKL_ERR_ALIGN = 4,       /* a pointer is not 16-byte aligned */
+  RKL_ERR_WORKSPACE = 5,   /* workspace NULL or smaller than rkl_workspace_size */
+  RKL_ERR_UNSUPPORTED = 6, /* option with no code path (rejected, not ignored) */
+  RKL_ERR_CUDA = 7,        /* a CUDA runtime/driver call failed */
+  RKL_ERR_DEVICE = 8       /* a kernel's bounded wait ran out (rkl_device_error) */
+} rkl_status;
+
+typedef enum rkl_dtype { RKL_BF16 = 0, RKL_FP32 = 1 } rkl_dtype;
+
+/* PR #3978, second implementation note: token-level mean, or the nested
+ * per-sequence average under token_level_loss=false.  NONE returns only the
+ * per-token tensor. */
+typedef enum rkl_reduction {
+  RKL_REDUCE_NONE = 0,
+  RKL_REDUCE_TOKEN_MEAN = 1,        /* sum_k L_k / N            (0 when N = 0) */
+  RKL_REDUCE_SEQ_MEAN_NESTED = 2    /* mean over sequences with n_b > 0 of
+                                       sum_{t in b} L_t / n_b   (0 when N = 0) */
+} rkl_reduction;
+
+/* PR #3978, payload bullets: full.teacher_payload = hidden_states | logits. */
+typedef enum rkl_payload { RKL_PAYLOAD_HIDDEN = 0, RKL_PAYLOAD_LOGITS = 1 } rkl_payload;
+
+/* Library version string (static storage). */
+const char* rkl_version(void);
+
+/* Description of the last error on the calling thread ("" if none). */
+const char* rkl_last_error(void);
+
+/* Bytes of device workspace that rkl_forward_* and rkl_backward need for at
+ * most n_max trainable rows (n_max <= B*Sm1) of the given problem.  The same
+ * workspace may be reused by consecutive calls on one stream; calls that run
+ * concurrently need separate workspaces.  Content need not be initialised. */
+rkl_status rkl_workspace_size(rkl_payload payload, rkl_dtype dtype, int64_t n_max,
+                              int64_t B, int64_t Sm1, int64_t H, int64_t V,
+                              size_t* bytes /* host out */);
+
+/* S1, compaction (slime PR #2310, Summary: project only the N loss-masked
+ * rows).  row_idx[k] = flattened index b*Sm1+t of the k-th nonzero entry of
+ * mask [B, Sm1] (uint8, nonzero = trainable), strictly ascending; *n_dev = N.
+ * row_idx must hold B*Sm1 int32.  Bit-exact, deterministic.  The caller
+ * reads N back (one 4-byte device-to-host copy) to size the next calls. */
+rkl_status rkl_compact_rows(const uint8_t* mask, int64_t B, int64_t Sm1,
+                            int32_t* row_idx, int32_t* n_dev, void* stream);
+
+/* S2-S4, forward on the hidden-state payload (PR #3978, payload bullet 1).
+ * h_s, h_t [T, H]; W_s, W_t [V, H]; dtype of all four.  row_idx/N from
+ * rkl_compact_rows.  Outputs (fp32):
+ *   loss_tok [B, Sm1]  per-token loss, exact 0 at masked positions (nullable)
+ *   loss     [1]       reduced loss (nullable; ignored for RKL_REDUCE_NONE)
+ *   saved    [N, 3]    per-row (lse_s, lse_t, L) kept for rkl_backward
+ * N = 0 gives loss 0 and all-zero loss_tok without NaN (slime PR #2310: empty
+ * masks keep zero-gradient connections). */
+rkl_status rkl_forward_hidden(const void* h_s, const void* h_t,
+                              const void* W_s, const void* W_t, rkl_dtype dtype,
+                              int64_t B, int64_t Sm1, int64_t H, int64_t V,
+                              const int32_t* row_idx, int32_t N,
+                              rkl_reduction reduction,
+                              float* loss_tok, float* loss, float* saved,
+                              void* workspace, size_t workspace_bytes, void* stream);
+
+/* S2-S4 + S8, forward on the logits payload (PR #3978, payload bullet 2: the
+ * teacher ships full-vocabulary logits and needs no LM head).  teacher_logits
+ * [T, V] of `dtype`, used as given (only rows in row_idx are read).  Same
+ * outputs as rkl_forward_hidden. */
+rkl_status rkl_forward_logits(const void* h_s, const void* W_s,
+                              const void* teacher_logits, rkl_dtype dtype,
+                              int64_t B, int64_t Sm1, int64_t H, int64_t V,
+                              const int32_t* row_idx, int32_t N,
+                              rkl_reduction reduction,
+                              float* loss_tok, float* loss, float* saved,
+                              void* workspace, size_t workspace_bytes, void* stream);
+
+/* S5-S7, backward of either payload (PR #3978, first implementation note:
+ * dL/dz_s = p_s (w - L), log-softmaxes recomputed, nothing [N, V] kept).
+ *   payload   RKL_PAYLOAD_HIDDEN: teacher = h_t [T, H], W_t [V, H]
+ *             RKL_PAYLOAD_LOGITS: teacher = teacher logits [T, V], W_t NULL
+ *   saved     [N, 3] from the matching forward call on the same inputs
+ *   grad_loss [1] dLoss upstream gradient of the reduced loss (nullable = 0;
+ *             ignored for RKL_REDUCE_NONE)
+ *   grad_tok  [B, Sm1] upstream gradient of loss_tok (nullable = 0)
+ * Row weight of trainable row k: g_k = grad_tok[row] + grad_loss * w_k, with
+ * w_k = 1/N (token mean) or 1/(B_eff * n_b) (nested mean).  Outputs (fp32,
+ * overwritten): dH_s [T, H] with exact zero rows at masked positions, and
+ * dW_s [V, H].  No gradient is produced for the teacher inputs. */
+rkl_status rkl_backward(rkl_payload payload,
+                        const void* h_s, const void* teacher,
+                        const void* W_s, const void* W_t, rkl_dtype dtype,
+                        int64_t B, int64_t Sm1, int64_t H, int64_t V,
+                        const int32_t* row_idx, int32_t N,
+                        rkl_reduction reduction, const float* saved,
+                        const float* grad_loss, const float* grad_tok,
+                        float* dH_s, float* dW_s,
+                        void* workspace, size_t workspace_bytes, void* stream);
+
+/* Synchronises the current device, then reports and clears the library's
+ * device error word: *code = 0 if no kernel's bounded wait ran out since the
+ * last call, else a nonzero bit set naming the wait (the kernel returned
+ * early and its outputs are invalid).  Returns RKL_ERR_DEVICE when *code != 0. */
+rkl_status rkl_device_error(int32_t* code /* host out */);
+
+/* Measurement hooks (used by bench.py).  When enabled, every kernel launch of
+ * the library is bracketed by CUDA events on the launching stream;
+ * rkl_profile_read synchronises and returns, per kernel id, the summed device
+ * time and the launch count since the last rkl_profile_reset. */
+int32_t rkl_kernel_count(void);                 /* number of kernel ids */
+const char* rkl_kernel_name(int32_t kernel_id); /* NULL if out of range */
+rkl_status rkl_profile_enable(int32_t enable);
+rkl_status rkl_profile_reset(void);
+rkl_status rkl_profile_read(int32_t kernel_id, double* total_ms, int64_t* launches);
+/* Total kernel launches issued by the library since load (host counter). */
+int64_t rkl_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RKL_H */

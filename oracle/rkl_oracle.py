@@ -1,0 +1,223 @@
+"""Plain float64 CPU oracle for the exact full-vocabulary reverse-KL distillation loss.
+
+TEST INFRASTRUCTURE. This module is the correctness authority that the CUDA
+library is compared against. Only the test suite, ``__graft_entry__.smoke()``
+and the CPU-baseline / reference arm of ``bench.py`` may import it. The
+product path (the C-ABI library ``librkl.so`` and its Python binding) never
+imports, links or calls anything here, and this module imports nothing from
+the product package.
+
+What it computes, and where the pages define it:
+
+* "feat(mopd): add full-vocabulary on-policy distillation" (NeMo RL PR #3978),
+  description: the per-token objective
+      L_t = sum_v p_s(v) * (log p_s(v) - log p_t(v))
+  (reverse KL of student p_s from teacher p_t over the whole vocabulary).
+* same page, payload bullets: the teacher either ships pre-LM-head hidden
+  states that are projected with the teacher's own LM-head weight
+  (``hidden_states`` payload) or ships full-vocabulary logits (``logits``
+  payload).
+* same page, first implementation note: the shared backward
+  dL/dz_s = p_s * (w - L) with w = log p_s - log p_t; log-softmaxes are
+  recomputed in backward rather than cached.
+* same page, second implementation note: the loss receives a per-token
+  [B, S-1] tensor and reduces it either as a token-level mean or as the
+  nested per-sequence mean (``token_level_loss=false``).
+* "fix(megatron): compact actor logits before projection" (slime PR #2310),
+  Summary: only the N loss-masked rows are projected; scalar results are
+  scattered back to the [B, S-1] layout; empty masks keep zero-gradient
+  connections.
+
+Readings where the pages are silent (each is listed in the design doc):
+
+* Only the student gets gradients (the teacher LM head is "a plain tensor");
+  gradients flow to h_s and W_s.
+* The nested mean averages over sequences that have at least one trainable
+  position; with none at all the loss is 0.  The token mean with N = 0 is 0.
+* The mask is a per-position flag: nonzero = trainable.
+* Backward may keep three per-row scalars (lse_s, lse_t, L); it never keeps a
+  [N, V] tensor.
+
+Everything is float64.  Inputs may be float32 or float64 arrays (bf16 values
+are upcast exactly by the caller before they get here).  Rows are processed in
+chunks to bound memory; no other blocking, fusion or reordering is done.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+REDUCE_NONE = 0
+REDUCE_TOKEN_MEAN = 1
+REDUCE_SEQ_MEAN_NESTED = 2
+
+_ROW_CHUNK = 256
+
+
+def compact_rows(mask):
+    """Indices of the trainable rows of the flattened [B, S-1] mask, ascending.
+
+    slime PR #2310, Summary: project only the N loss-masked rows.
+    Returns (row_idx int64 [N], N).
+    """
+    flat = np.asarray(mask).reshape(-1) != 0
+    row_idx = np.flatnonzero(flat).astype(np.int64)
+    return row_idx, int(row_idx.shape[0])
+
+
+def log_softmax(z):
+    """Row-wise log-softmax with a max shift: z - (m + log sum exp(z - m))."""
+    m = np.max(z, axis=1, keepdims=True)
+    return z - (m + np.log(np.sum(np.exp(z - m), axis=1, keepdims=True)))
+
+
+def logsumexp(z):
+    m = np.max(z, axis=1)
+    return m + np.log(np.sum(np.exp(z - m[:, None]), axis=1))
+
+
+def _f64(a):
+    return np.asarray(a, dtype=np.float64)
+
+
+def _student_teacher_logits(rows, h_s, W_s64, teacher, W_t64):
+    """Logits of the selected rows.  NeMo RL PR #3978, payload bullets.
+
+    hidden_states payload: z_s = h_s W_s^T, z_t = h_t W_t^T.
+    logits payload (W_t64 is None): z_t is the shipped teacher logit row.
+    """
+    z_s = _f64(h_s[rows]) @ W_s64.T
+    if W_t64 is None:
+        z_t = _f64(teacher[rows])
+    else:
+        z_t = _f64(teacher[rows]) @ W_t64.T
+    return z_s, z_t
+
+
+def per_row_kl(z_s, z_t):
+    """L = sum_v p_s (log p_s - log p_t) per row, plus lse_s and lse_t.
+
+    NeMo RL PR #3978, description (the objective).
+    """
+    lp_s = log_softmax(z_s)
+    lp_t = log_softmax(z_t)
+    p_s = np.exp(lp_s)
+    L = np.sum(p_s * (lp_s - lp_t), axis=1)
+    return L, logsumexp(z_s), logsumexp(z_t)
+
+
+def reduce_loss(L_rows, row_idx, B, Sm1, reduction):
+    """Reduce the per-trainable-row losses to the scalar loss.
+
+    NeMo RL PR #3978, second implementation note: token-level mean, or the
+    nested per-sequence average under token_level_loss=false.
+    """
+    L_rows = _f64(L_rows)
+    N = L_rows.shape[0]
+    if reduction == REDUCE_NONE:
+        return None
+    if reduction == REDUCE_TOKEN_MEAN:
+        return float(np.sum(L_rows) / N) if N > 0 else 0.0
+    if reduction == REDUCE_SEQ_MEAN_NESTED:
+        seq = np.asarray(row_idx) // Sm1
+        per_seq = []
+        for b in range(B):
+            sel = seq == b
+            n_b = int(np.count_nonzero(sel))
+            if n_b > 0:
+                per_seq.append(np.sum(L_rows[sel]) / n_b)
+        return float(np.mean(per_seq)) if per_seq else 0.0
+    raise ValueError("unknown reduction %r" % (reduction,))
+
+
+def row_weights(row_idx, B, Sm1, reduction, grad_loss=1.0, grad_tok=None):
+    """g_k = dLoss/dL_k for each trainable row k (chain rule through the reduction).
+
+    token mean: grad_loss / N.  nested mean: grad_loss / (B_eff * n_b).  A
+    per-token upstream gradient grad_tok [B, S-1] (the gradient of the
+    per-token loss tensor itself) is added on top.
+    """
+    row_idx = np.asarray(row_idx)
+    N = row_idx.shape[0]
+    g = np.zeros(N, dtype=np.float64)
+    if reduction == REDUCE_TOKEN_MEAN and N > 0:
+        g += grad_loss / N
+    elif reduction == REDUCE_SEQ_MEAN_NESTED and N > 0:
+        seq = row_idx // Sm1
+        counts = np.bincount(seq, minlength=B)
+        b_eff = int(np.count_nonzero(counts))
+        g += grad_loss / (b_eff * counts[seq])
+    if grad_tok is not None:
+        g += _f64(grad_tok).reshape(-1)[row_idx]
+    return g
+
+
+def forward(h_s, W_s, teacher, W_t, mask, reduction):
+    """Full forward of either payload path.
+
+    h_s [T, H]; W_s [V, H]; teacher = h_t [T, H] with W_t [V, H] (hidden_states
+    payload) or teacher logits [T, V] with W_t None (logits payload);
+    mask [B, S-1].  Returns dict with loss_tok [B, S-1] (exact 0 at masked
+    positions), loss (scalar or None), and the saved per-row scalars
+    lse_s, lse_t, L [N], and row_idx.
+    """
+    mask = np.asarray(mask)
+    B, Sm1 = mask.shape
+    row_idx, N = compact_rows(mask)
+    W_s64 = _f64(W_s)
+    W_t64 = None if W_t is None else _f64(W_t)
+    L = np.zeros(N)
+    lse_s = np.zeros(N)
+    lse_t = np.zeros(N)
+    for c0 in range(0, N, _ROW_CHUNK):
+        rows = row_idx[c0:c0 + _ROW_CHUNK]
+        z_s, z_t = _student_teacher_logits(rows, h_s, W_s64, teacher, W_t64)
+        L[c0:c0 + len(rows)], lse_s[c0:c0 + len(rows)], lse_t[c0:c0 + len(rows)] = per_row_kl(z_s, z_t)
+    loss_tok = np.zeros(B * Sm1)
+    loss_tok[row_idx] = L
+    loss = reduce_loss(L, row_idx, B, Sm1, reduction)
+    return {"loss_tok": loss_tok.reshape(B, Sm1), "loss": loss, "L": L,
+            "lse_s": lse_s, "lse_t": lse_t, "row_idx": row_idx, "N": N}
+
+
+def backward(h_s, W_s, teacher, W_t, mask, reduction, grad_loss=1.0, grad_tok=None):
+    """Gradients of the loss with respect to h_s and W_s.
+
+    NeMo RL PR #3978, first implementation note: dL/dz_s = p_s * (w - L) with
+    w = log p_s - log p_t, log-softmaxes recomputed here (nothing [N, V] is
+    kept from the forward).  Chain rule through z_s = h_s W_s^T:
+        dH_s[rows] = dz W_s,   dW_s = dz^T h_s[rows].
+    Masked positions get exact zero rows in dH_s.
+    Returns (dH_s [T, H], dW_s [V, H]) in float64.
+    """
+    mask = np.asarray(mask)
+    B, Sm1 = mask.shape
+    row_idx, N = compact_rows(mask)
+    W_s64 = _f64(W_s)
+    W_t64 = None if W_t is None else _f64(W_t)
+    T, H = np.asarray(h_s).shape
+    g = row_weights(row_idx, B, Sm1, reduction, grad_loss, grad_tok)
+    dH = np.zeros((T, H))
+    dW = np.zeros(W_s64.shape)
+    for c0 in range(0, N, _ROW_CHUNK):
+        rows = row_idx[c0:c0 + _ROW_CHUNK]
+        z_s, z_t = _student_teacher_logits(rows, h_s, W_s64, teacher, W_t64)
+        lp_s = log_softmax(z_s)
+        lp_t = log_softmax(z_t)
+        p_s = np.exp(lp_s)
+        w = lp_s - lp_t
+        L = np.sum(p_s * w, axis=1)
+        dz = g[c0:c0 + len(rows), None] * p_s * (w - L[:, None])
+        dH[rows] = dz @ W_s64
+        dW += dz.T @ _f64(h_s[rows])
+    return dH, dW
+
+
+def dz_rows(z_s, z_t, g):
+    """dLoss/dz_s for given logit rows and row weights (for small pins)."""
+    lp_s = log_softmax(_f64(z_s))
+    lp_t = log_softmax(_f64(z_t))
+    p_s = np.exp(lp_s)
+    w = lp_s - lp_t
+    L = np.sum(p_s * w, axis=1)
+    return _f64(g)[:, None] * p_s * (w - L[:, None])

@@ -1,0 +1,255 @@
+"""Checks that pin the CPU oracle to facts fixed outside it.
+
+Each function takes the oracle module (so that the mutation tests can hand in
+a copy with a planted mistake) and returns the worst violation it found; the
+pin tests assert it is below a bound, the mutation tests assert that a planted
+mistake pushes it above.  The facts come from the mathematics of the objective
+in NeMo RL PR #3978 ("feat(mopd): add full-vocabulary on-policy distillation",
+description and first implementation note) and the masking rules of slime
+PR #2310 ("fix(megatron): compact actor logits before projection", Summary).
+"""
+
+import math
+
+import numpy as np
+import scipy.special
+import scipy.stats
+
+from oracle import brute
+
+
+def rand_problem(rs, B=2, Sm1=3, H=4, V=7, scale=1.0, mask=None, payload="hidden"):
+    T = B * Sm1
+    h_s = rs.normal(size=(T, H)) * scale
+    W_s = rs.normal(size=(V, H)) * scale
+    if payload == "hidden":
+        teacher = rs.normal(size=(T, H)) * scale
+        W_t = rs.normal(size=(V, H)) * scale
+    else:
+        teacher = rs.normal(size=(T, V)) * 2.0
+        W_t = None
+    if mask is None:
+        mask = (rs.uniform(size=(B, Sm1)) < 0.7).astype(np.uint8)
+        mask[0, -1] = 1
+    return h_s, W_s, teacher, W_t, mask
+
+
+def kl_vs_scipy(O, rs):
+    """L equals scipy.stats.entropy(p_s, p_t) = sum p_s log(p_s / p_t).
+
+    This is the Kullback-Leibler divergence of p_s from p_t, so a swapped
+    direction (forward KL) or a wrong log-softmax fails here."""
+    worst = 0.0
+    for V in (2, 5, 33, 1000):
+        z_s = rs.normal(size=(4, V)) * 3
+        z_t = rs.normal(size=(4, V)) * 3
+        L, _, _ = O.per_row_kl(z_s, z_t)
+        ref = scipy.stats.entropy(scipy.special.softmax(z_s, axis=1),
+                                  scipy.special.softmax(z_t, axis=1), axis=1)
+        worst = max(worst, float(np.max(np.abs(L - ref) / (1e-12 + np.abs(ref)))))
+    return worst
+
+
+def lse_vs_scipy(O, rs):
+    worst = 0.0
+    for V in (1, 3, 1000):
+        z = rs.normal(size=(5, V)) * 10 + 50
+        _, lse_s, lse_t = O.per_row_kl(z, z + 1.0)
+        ref = scipy.special.logsumexp(z, axis=1)
+        worst = max(worst, float(np.max(np.abs(lse_s - ref))), float(np.max(np.abs(lse_t - 1.0 - ref))))
+    return worst
+
+
+def uniform_teacher(O, rs):
+    """W_t = 0 -> p_t uniform -> L = log V - H(p_s), H from scipy.stats.entropy."""
+    worst = 0.0
+    for V in (3, 17, 512):
+        h_s, W_s, h_t, _, mask = rand_problem(rs, B=1, Sm1=4, H=5, V=V, mask=np.ones((1, 4), np.uint8))
+        W_t = np.zeros_like(W_s)
+        out = O.forward(h_s, W_s, h_t, W_t, mask, O.REDUCE_NONE)
+        p_s = scipy.special.softmax(h_s @ W_s.T, axis=1)
+        ref = math.log(V) - scipy.stats.entropy(p_s, axis=1)
+        worst = max(worst, float(np.max(np.abs(out["L"] - ref))))
+    return worst
+
+
+def one_logit_bump(O, rs):
+    """z_t = z_s + delta e_k -> L = -delta p_s(k) + log(1 + p_s(k)(e^delta - 1))."""
+    worst = 0.0
+    for delta in (-3.0, -0.5, 0.25, 2.0):
+        z_s = rs.normal(size=(3, 11)) * 2
+        k = 4
+        z_t = z_s.copy()
+        z_t[:, k] += delta
+        L, _, _ = O.per_row_kl(z_s, z_t)
+        p = scipy.special.softmax(z_s, axis=1)[:, k]
+        ref = -delta * p + np.log1p(p * math.expm1(delta))
+        worst = max(worst, float(np.max(np.abs(L - ref))))
+    return worst
+
+
+def binary_kl(O, rs):
+    """Two-token vocabulary: L = p log(p/q) + (1-p) log((1-p)/(1-q)), p = sigmoid."""
+    z_s = rs.normal(size=(6, 2)) * 2
+    z_t = rs.normal(size=(6, 2)) * 2
+    L, _, _ = O.per_row_kl(z_s, z_t)
+    p = scipy.special.expit(z_s[:, 1] - z_s[:, 0])
+    q = scipy.special.expit(z_t[:, 1] - z_t[:, 0])
+    ref = p * np.log(p / q) + (1 - p) * np.log((1 - p) / (1 - q))
+    return float(np.max(np.abs(L - ref)))
+
+
+def brute_force(O, rs):
+    """Per-token loss and both reductions against the pure-Python loops."""
+    worst = 0.0
+    for payload_seed in range(3):
+        h_s, W_s, h_t, W_t, mask = rand_problem(rs, B=3, Sm1=4, H=3, V=9)
+        ref_tok = np.array(brute.loss_tokens(h_s.tolist(), W_s.tolist(), h_t.tolist(), W_t.tolist(), mask.tolist()))
+        for red, ref_fn in ((O.REDUCE_TOKEN_MEAN, brute.token_mean), (O.REDUCE_SEQ_MEAN_NESTED, brute.nested_mean)):
+            out = O.forward(h_s, W_s, h_t, W_t, mask, red)
+            worst = max(worst, float(np.max(np.abs(out["loss_tok"] - ref_tok))))
+            worst = max(worst, abs(out["loss"] - ref_fn(ref_tok.tolist(), mask.tolist())))
+    return worst
+
+
+def compact_rows_brute(O, rs):
+    bad = 0
+    for kind in range(5):
+        mask = (rs.uniform(size=(3, 7)) < [0.0, 0.2, 0.5, 0.9, 1.0][kind]).astype(np.uint8)
+        idx, n = O.compact_rows(mask)
+        ref = brute.compact_rows(mask.tolist())
+        bad += int(n != len(ref) or list(idx) != ref)
+    return bad
+
+
+def _loss_fn(O, h_s, W_s, teacher, W_t, mask, red, grad_tok):
+    out = O.forward(h_s, W_s, teacher, W_t, mask, red)
+    val = 0.0 if out["loss"] is None else out["loss"]
+    if grad_tok is not None:
+        val += float(np.sum(grad_tok * out["loss_tok"]))
+    return val
+
+
+def finite_differences(O, rs, payload="hidden", red=None, with_grad_tok=False, grad_loss=1.0):
+    """Central differences of the scalar objective w.r.t. h_s and W_s.
+
+    Objective = grad_loss * loss + sum(grad_tok * loss_tok); backward must
+    return its gradient.  Returns the worst relative error."""
+    red = 1 if red is None else red
+    # unequal per-sequence counts and one empty sequence, so that the token
+    # mean and the nested mean have different row weights
+    mask = np.array([[1, 1, 1], [0, 1, 0], [0, 0, 0]], dtype=np.uint8)
+    h_s, W_s, teacher, W_t, mask = rand_problem(rs, B=3, Sm1=3, H=4, V=7, payload=payload, mask=mask)
+    grad_tok = rs.normal(size=mask.shape) if with_grad_tok else None
+
+    def f(hs, ws):
+        out = O.forward(hs, ws, teacher, W_t, mask, red)
+        val = 0.0 if out["loss"] is None else grad_loss * out["loss"]
+        if grad_tok is not None:
+            val += float(np.sum(grad_tok * out["loss_tok"]))
+        return val
+
+    dH, dW = O.backward(h_s, W_s, teacher, W_t, mask, red, grad_loss=grad_loss, grad_tok=grad_tok)
+    eps = 1e-6
+    num_H = np.zeros_like(h_s)
+    for i in range(h_s.shape[0]):
+        for j in range(h_s.shape[1]):
+            hp = h_s.copy(); hp[i, j] += eps
+            hm = h_s.copy(); hm[i, j] -= eps
+            num_H[i, j] = (f(hp, W_s) - f(hm, W_s)) / (2 * eps)
+    num_W = np.zeros_like(W_s)
+    for i in range(W_s.shape[0]):
+        for j in range(W_s.shape[1]):
+            wp = W_s.copy(); wp[i, j] += eps
+            wm = W_s.copy(); wm[i, j] -= eps
+            num_W[i, j] = (f(h_s, wp) - f(h_s, wm)) / (2 * eps)
+    scale_H = max(1e-12, float(np.max(np.abs(num_H))))
+    scale_W = max(1e-12, float(np.max(np.abs(num_W))))
+    return max(float(np.max(np.abs(dH - num_H))) / scale_H, float(np.max(np.abs(dW - num_W))) / scale_W)
+
+
+def self_distillation(O, rs):
+    """Teacher == student: L and every gradient exactly 0 (PR #3978 recipe)."""
+    h_s, W_s, _, _, mask = rand_problem(rs, B=2, Sm1=5, H=6, V=40)
+    out = O.forward(h_s, W_s, h_s.copy(), W_s.copy(), mask, O.REDUCE_SEQ_MEAN_NESTED)
+    dH, dW = O.backward(h_s, W_s, h_s.copy(), W_s.copy(), mask, O.REDUCE_SEQ_MEAN_NESTED)
+    return max(float(np.max(np.abs(out["loss_tok"]))), abs(out["loss"]),
+               float(np.max(np.abs(dH))), float(np.max(np.abs(dW))))
+
+
+def dz_sums_to_zero(O, rs):
+    """sum_v dL/dz_s = 0 per row (sum_v p_s (w - L) = L - L)."""
+    z_s = rs.normal(size=(8, 300)) * 3
+    z_t = z_s + rs.normal(size=(8, 300)) * 0.5
+    dz = O.dz_rows(z_s, z_t, np.ones(8))
+    return float(np.max(np.abs(dz.sum(axis=1)) / np.abs(dz).sum(axis=1)))
+
+
+def shift_invariance(O, rs):
+    """Adding a per-row constant to the teacher logits changes nothing."""
+    h_s, W_s, logits, _, mask = rand_problem(rs, B=2, Sm1=4, H=5, V=30, payload="logits")
+    shift = rs.uniform(-20, 20, size=(logits.shape[0], 1))
+    a = O.forward(h_s, W_s, logits, None, mask, 1)
+    b = O.forward(h_s, W_s, logits + shift, None, mask, 1)
+    dHa, dWa = O.backward(h_s, W_s, logits, None, mask, 1)
+    dHb, dWb = O.backward(h_s, W_s, logits + shift, None, mask, 1)
+    return max(float(np.max(np.abs(a["loss_tok"] - b["loss_tok"]))),
+               float(np.max(np.abs(dHa - dHb))), float(np.max(np.abs(dWa - dWb))))
+
+
+def masked_rows_exact_zero(O, rs):
+    """Masked positions: loss exactly 0 and dH row exactly 0 (slime PR #2310)."""
+    h_s, W_s, h_t, W_t, mask = rand_problem(rs, B=3, Sm1=5, H=4, V=9)
+    out = O.forward(h_s, W_s, h_t, W_t, mask, 1)
+    dH, _ = O.backward(h_s, W_s, h_t, W_t, mask, 1)
+    off = mask.reshape(-1) == 0
+    return float(np.max(np.abs(out["loss_tok"].reshape(-1)[off]), initial=0.0)) + \
+        float(np.max(np.abs(dH[off]), initial=0.0))
+
+
+def compact_equals_full(O, rs):
+    """Compact rows vs all rows then select (slime PR #2310 compact/full parity)."""
+    h_s, W_s, h_t, W_t, mask = rand_problem(rs, B=3, Sm1=6, H=5, V=21)
+    comp = O.forward(h_s, W_s, h_t, W_t, mask, 0)
+    full = O.forward(h_s, W_s, h_t, W_t, np.ones_like(mask), 0)
+    sel = mask.reshape(-1) != 0
+    return float(np.max(np.abs(comp["loss_tok"].reshape(-1)[sel] - full["loss_tok"].reshape(-1)[sel])))
+
+
+def empty_mask(O, rs):
+    """N = 0: loss 0, gradients 0, nothing NaN (slime PR #2310: empty masks)."""
+    h_s, W_s, h_t, W_t, _ = rand_problem(rs, B=2, Sm1=3, H=4, V=7)
+    mask = np.zeros((2, 3), np.uint8)
+    worst = 0.0
+    for red in (1, 2):
+        out = O.forward(h_s, W_s, h_t, W_t, mask, red)
+        dH, dW = O.backward(h_s, W_s, h_t, W_t, mask, red)
+        vals = np.concatenate([out["loss_tok"].ravel(), [out["loss"]], dH.ravel(), dW.ravel()])
+        if not np.all(np.isfinite(vals)):
+            return float("inf")
+        worst = max(worst, float(np.max(np.abs(vals))))
+    return worst
+
+
+def nested_vs_token_mean_equal_counts(O, rs):
+    """With equal per-sequence counts, the nested mean equals the token mean."""
+    h_s, W_s, h_t, W_t, _ = rand_problem(rs, B=3, Sm1=4, H=4, V=7)
+    mask = np.zeros((3, 4), np.uint8)
+    mask[0, [0, 2]] = 1
+    mask[1, [1, 3]] = 1
+    mask[2, [2, 3]] = 1
+    a = O.forward(h_s, W_s, h_t, W_t, mask, 1)["loss"]
+    b = O.forward(h_s, W_s, h_t, W_t, mask, 2)["loss"]
+    return abs(a - b)
+
+
+def nested_mean_by_hand(O, rs):
+    """Nested mean of a 2-sequence batch with an empty third sequence."""
+    h_s, W_s, h_t, W_t, _ = rand_problem(rs, B=3, Sm1=4, H=4, V=7)
+    mask = np.zeros((3, 4), np.uint8)
+    mask[0, [1]] = 1
+    mask[2, [0, 1, 3]] = 1
+    out = O.forward(h_s, W_s, h_t, W_t, mask, 2)
+    lt = out["loss_tok"]
+    ref = 0.5 * (lt[0, 1] + (lt[2, 0] + lt[2, 1] + lt[2, 3]) / 3.0)
+    return abs(out["loss"] - ref)

@@ -1,0 +1,185 @@
+"""Pins of the float64 CPU oracle (no GPU).
+
+Every check compares the oracle with something outside it: a library routine
+for a special case (scipy KL / entropy / logsumexp), a closed form, an
+invariant of the objective, a pure-Python brute force, or finite differences.
+The mutation tests plant plausible mistakes in a private copy of the oracle
+and show that at least one pin catches each.
+"""
+
+import json
+import os
+import types
+
+import numpy as np
+import pytest
+
+from oracle import rkl_oracle as O
+from tests import pins
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+@pytest.fixture
+def rs():
+    return np.random.RandomState(20261202)
+
+
+def test_kl_matches_scipy_entropy(rs):
+    assert pins.kl_vs_scipy(O, rs) < 1e-10
+
+
+def test_lse_matches_scipy(rs):
+    assert pins.lse_vs_scipy(O, rs) < 1e-10
+
+
+def test_kl_nonnegative(rs):
+    for V in (2, 10, 5000):
+        z_s = rs.normal(size=(16, V)) * 4
+        z_t = rs.normal(size=(16, V)) * 4
+        L, _, _ = O.per_row_kl(z_s, z_t)
+        assert np.all(L >= -1e-12)
+
+
+def test_uniform_teacher_closed_form(rs):
+    assert pins.uniform_teacher(O, rs) < 1e-10
+
+
+def test_one_logit_bump_closed_form(rs):
+    assert pins.one_logit_bump(O, rs) < 1e-12
+
+
+def test_binary_vocabulary_closed_form(rs):
+    assert pins.binary_kl(O, rs) < 1e-12
+
+
+def test_brute_force_loops(rs):
+    assert pins.brute_force(O, rs) < 1e-12
+
+
+def test_compact_rows_brute(rs):
+    assert pins.compact_rows_brute(O, rs) == 0
+
+
+@pytest.mark.parametrize("payload", ["hidden", "logits"])
+@pytest.mark.parametrize("red", [1, 2])
+def test_finite_differences(rs, payload, red):
+    assert pins.finite_differences(O, rs, payload=payload, red=red) < 1e-6
+
+
+def test_finite_differences_grad_tok(rs):
+    # reduction NONE: only the per-token upstream gradient drives backward
+    assert pins.finite_differences(O, rs, red=0, with_grad_tok=True) < 1e-6
+    # both a reduced-loss gradient and a per-token gradient at once
+    assert pins.finite_differences(O, rs, red=2, with_grad_tok=True, grad_loss=0.7) < 1e-6
+
+
+def test_self_distillation_exact_zero(rs):
+    assert pins.self_distillation(O, rs) == 0.0
+
+
+def test_dz_rows_sum_to_zero(rs):
+    assert pins.dz_sums_to_zero(O, rs) < 1e-13
+
+
+def test_teacher_shift_invariance(rs):
+    assert pins.shift_invariance(O, rs) < 1e-10
+
+
+def test_masked_rows_exact_zero(rs):
+    assert pins.masked_rows_exact_zero(O, rs) == 0.0
+
+
+def test_compact_equals_full(rs):
+    assert pins.compact_equals_full(O, rs) < 1e-12
+
+
+def test_empty_mask(rs):
+    assert pins.empty_mask(O, rs) == 0.0
+
+
+def test_nested_equals_token_mean_for_equal_counts(rs):
+    assert pins.nested_vs_token_mean_equal_counts(O, rs) < 1e-14
+
+
+def test_nested_mean_skips_empty_sequences(rs):
+    assert pins.nested_mean_by_hand(O, rs) < 1e-14
+
+
+def test_payload_ratio_golden():
+    """The logits payload is ~74x the hidden payload at 2k hidden / 152k vocab."""
+    with open(os.path.join(GOLDEN, "payload_ratio.json")) as f:
+        g = json.load(f)
+    ratio = g["V"] / g["H"]
+    assert round(ratio) == g["quoted_ratio"]
+    from full_vocabulary_reverse_b200.workloads import WORKLOADS
+    w = WORKLOADS["qwen_hidden"]
+    assert (w["H"], w["V"]) == (g["H"], g["V"])
+
+
+def test_golden_tiny_case():
+    """Stored oracle outputs of a tiny case (written by tests/golden/make_golden.py)."""
+    with open(os.path.join(GOLDEN, "tiny_case.json")) as f:
+        g = json.load(f)
+    a = {k: np.array(v) for k, v in g["inputs"].items()}
+    out = O.forward(a["h_s"], a["W_s"], a["h_t"], a["W_t"], a["mask"].astype(np.uint8), g["reduction"])
+    dH, dW = O.backward(a["h_s"], a["W_s"], a["h_t"], a["W_t"], a["mask"].astype(np.uint8), g["reduction"])
+    np.testing.assert_allclose(out["loss_tok"], np.array(g["loss_tok"]), rtol=1e-12, atol=1e-15)
+    np.testing.assert_allclose(out["loss"], g["loss"], rtol=1e-12)
+    np.testing.assert_allclose(dH, np.array(g["dH_s"]), rtol=1e-10, atol=1e-15)
+    np.testing.assert_allclose(dW, np.array(g["dW_s"]), rtol=1e-10, atol=1e-15)
+
+
+# --------------------------------------------------------------------------
+# Mutation tests: plant a mistake in a private copy of the oracle and check
+# that the pins notice.  The planted copy is built from the source text; the
+# real module is untouched.
+# --------------------------------------------------------------------------
+
+def _mutant(old, new):
+    src = open(O.__file__).read()
+    assert src.count(old) >= 1, old
+    mod = types.ModuleType("oracle_mutant")
+    exec(compile(src.replace(old, new), "oracle_mutant", "exec"), mod.__dict__)
+    return mod
+
+
+MUTATIONS = [
+    # dropped -L term in the shared backward
+    ("dz = g[c0:c0 + len(rows), None] * p_s * (w - L[:, None])",
+     "dz = g[c0:c0 + len(rows), None] * p_s * (w)", "fd"),
+    # forward KL instead of reverse KL
+    ("    p_s = np.exp(lp_s)\n    L = np.sum(p_s * (lp_s - lp_t), axis=1)",
+     "    p_s = np.exp(lp_t)\n    L = np.sum(p_s * (lp_t - lp_s), axis=1)", "kl"),
+    # wrong sign in the log-sum-exp
+    ("return z - (m + np.log(", "return z - (m - np.log(", "kl"),
+    # transposed / wrong operand in dW_s
+    ("dW += dz.T @ _f64(h_s[rows])", "dW += dz.T @ _f64(teacher[rows])", "fd"),
+    # wrong nested-mean weight
+    ("g += grad_loss / (b_eff * counts[seq])", "g += grad_loss / N", "fd_nested"),
+    # scatter to the wrong positions
+    ("loss_tok[row_idx] = L", "loss_tok[:N] = L", "masked"),
+    # off-by-one in compaction
+    ("row_idx = np.flatnonzero(flat).astype(np.int64)",
+     "row_idx = (np.flatnonzero(flat) + 1).astype(np.int64) % flat.size", "compact"),
+    # teacher max-shift applied to student lse in saved scalars
+    ("return m + np.log(np.sum(np.exp(z - m[:, None]), axis=1))",
+     "return m + np.log(np.sum(np.exp(z - m[:, None]), axis=1)) + 1e-3", "lse"),
+    # dH rows scattered to compact positions
+    ("dH[rows] = dz @ W_s64", "dH[c0:c0 + len(rows)] = dz @ W_s64", "masked"),
+]
+
+
+@pytest.mark.parametrize("old,new,kind", MUTATIONS)
+def test_pins_catch_planted_mistakes(old, new, kind):
+    M = _mutant(old, new)
+    rs = np.random.RandomState(7)
+    caught = {
+        "fd": lambda: pins.finite_differences(M, rs) > 1e-4,
+        "fd_nested": lambda: pins.finite_differences(M, rs, red=2) > 1e-4,
+        "kl": lambda: pins.kl_vs_scipy(M, rs) > 1e-6 or pins.brute_force(M, rs) > 1e-6,
+        "masked": lambda: pins.masked_rows_exact_zero(M, rs) > 0 or pins.brute_force(M, rs) > 1e-6,
+        "compact": lambda: pins.compact_rows_brute(M, rs) > 0,
+        "lse": lambda: pins.lse_vs_scipy(M, rs) > 1e-6,
+    }[kind]()
+    assert caught
