@@ -1,0 +1,592 @@
+// api.cu -- the C ABI of librkl.so (declared in include/rkl.h).
+//
+// Argument validation, workspace layout, TMA descriptor encoding, per-device
+// one-time setup and the launch sequence of each entry point.  Every numeric
+// step runs in the kernels of tc_kernels.cu / small_kernels.cu /
+// simt_kernels.cu; nothing here touches tensor data on the host.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "../../include/rkl.h"
+#include "kernels.h"
+
+namespace rkl {
+
+// ------------------------------------------------------------------ errors
+static thread_local std::string g_last_error;
+
+static rkl_status fail(rkl_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return s;
+}
+
+#define RKL_CUDA(call)                                                                          \
+  do {                                                                                          \
+    cudaError_t e__ = (call);                                                                   \
+    if (e__ != cudaSuccess) return fail(RKL_ERR_CUDA, "%s: %s", #call, cudaGetErrorString(e__)); \
+  } while (0)
+
+// ------------------------------------------------------------------ profiling
+static const char* const kKernelNames[K_COUNT] = {
+    "compact_rows", "gather_rows",   "fwd_dual_tc",  "fwd_single_tc", "teacher_lse", "combine_splits",
+    "scatter_loss", "reduce_loss",   "row_weights",  "dz_dual_tc",    "dz_single_tc", "grad_dw_dh_tc",
+    "scatter_dh",   "fwd_simt_fp32", "dz_simt_fp32", "grad_simt_fp32"};
+
+const char* kernel_name(int id) { return (id >= 0 && id < K_COUNT) ? kKernelNames[id] : nullptr; }
+
+struct ProfRec {
+  int id;
+  cudaEvent_t a, b;
+};
+static std::mutex g_prof_mu;
+static std::atomic<bool> g_profile{false};
+static std::atomic<long long> g_launches{0};
+static std::vector<ProfRec> g_prof_pending;
+static double g_prof_ms[K_COUNT];
+static long long g_prof_n[K_COUNT];
+
+LaunchScope::LaunchScope(int id_, cudaStream_t s) : id(id_), stream(s) {
+  g_launches.fetch_add(1);
+  if (g_profile.load()) {
+    if (cudaEventCreate(&ev0) == cudaSuccess && cudaEventCreate(&ev1) == cudaSuccess) {
+      cudaEventRecord(ev0, s);
+    } else {
+      ev0 = ev1 = nullptr;
+    }
+  }
+}
+
+LaunchScope::~LaunchScope() {
+  if (ev0 && ev1) {
+    cudaEventRecord(ev1, stream);
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    g_prof_pending.push_back({id, ev0, ev1});
+  }
+}
+
+// ------------------------------------------------------------------ devices
+struct DevState {
+  bool ready = false;
+  int sms = 0;
+};
+static std::mutex g_dev_mu;
+static DevState g_devs[64];
+
+static rkl_status device_setup(int* sms) {
+  int dev = 0;
+  RKL_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return fail(RKL_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DevState& d = g_devs[dev];
+  if (!d.ready) {
+    int major = 0, minor = 0;
+    RKL_CUDA(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev));
+    RKL_CUDA(cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev));
+    if (major != 10 || minor != 0)
+      return fail(RKL_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library is built for sm_100a (B200)", dev, major,
+                  minor);
+    RKL_CUDA(cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev));
+    RKL_CUDA(tc_setup(dev));
+    d.ready = true;
+  }
+  *sms = d.sms;
+  return RKL_OK;
+}
+
+// ------------------------------------------------------------------ TMA maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D row-major map: `inner` contiguous elements per row, `outer` rows,
+// `pitch` bytes between rows; 128-byte swizzle; out-of-bounds reads give 0.
+static rkl_status make_map(CUtensorMap* m, const void* ptr, bool f32, uint64_t inner, uint64_t outer,
+                           uint64_t pitch, uint32_t box_inner, uint32_t box_outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(RKL_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {pitch};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                  const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(RKL_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d) for %llux%llu pitch %llu box %ux%u", (int)r,
+                (unsigned long long)inner, (unsigned long long)outer, (unsigned long long)pitch, box_inner,
+                box_outer);
+  return RKL_OK;
+}
+
+// ------------------------------------------------------------------ plan
+constexpr int kVcBf16 = 4096;  // vocab chunk of the backward (multiple of kBN)
+constexpr int kVcF32 = 1024;
+
+struct Plan {
+  int n_pad = 0, es = 2, S = 1, VT = 1, Vc = 0;
+  size_t off_hcs = 0, off_hct = 0, off_part = 0, off_rowc = 0, off_lse = 0, off_dz = 0, off_dh = 0, total = 0;
+};
+
+static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+static Plan make_plan(rkl_payload payload, rkl_dtype dtype, int64_t n_max, int64_t H, int64_t V) {
+  Plan p;
+  const bool bf16 = dtype == RKL_BF16;
+  const int tile_m = bf16 ? kBM : kSimtBN;
+  const int tile_v = bf16 ? kBN : kSimtBN;
+  p.es = bf16 ? 2 : 4;
+  const int64_t n = n_max < 1 ? 1 : n_max;
+  p.n_pad = static_cast<int>(((n + kBM - 1) / kBM) * kBM);  // multiple of both tile heights
+  (void)tile_m;
+  p.VT = static_cast<int>((V + tile_v - 1) / tile_v);
+  p.S = p.VT < kSplits ? p.VT : kSplits;
+  const int vc = bf16 ? kVcBf16 : kVcF32;
+  const int64_t vround = ((V + kBN - 1) / kBN) * kBN;
+  p.Vc = static_cast<int>(vround < vc ? vround : vc);
+  size_t off = 256;  // header
+  p.off_hcs = off;
+  off = align256(off + size_t(p.n_pad) * H * p.es);
+  p.off_hct = off;
+  if (payload == RKL_PAYLOAD_HIDDEN) off = align256(off + size_t(p.n_pad) * H * p.es);
+  p.off_part = off;
+  off = align256(off + size_t(kSplits) * 5 * p.n_pad * sizeof(float));
+  p.off_rowc = off;
+  off = align256(off + size_t(3) * p.n_pad * sizeof(float));
+  p.off_lse = off;
+  off = align256(off + size_t(p.n_pad) * sizeof(float));
+  p.off_dz = off;
+  off = align256(off + size_t(p.n_pad) * p.Vc * p.es);
+  p.off_dh = off;
+  off = align256(off + size_t(p.n_pad) * H * sizeof(float));
+  p.total = off;
+  return p;
+}
+
+// ------------------------------------------------------------------ checks
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+static rkl_status check_common(rkl_payload payload, rkl_dtype dtype, int64_t B, int64_t Sm1, int64_t H, int64_t V,
+                               int32_t N, int reduction) {
+  if (dtype != RKL_BF16 && dtype != RKL_FP32) return fail(RKL_ERR_DTYPE, "unknown dtype %d", (int)dtype);
+  if (payload != RKL_PAYLOAD_HIDDEN && payload != RKL_PAYLOAD_LOGITS)
+    return fail(RKL_ERR_DTYPE, "unknown payload %d", (int)payload);
+  if (reduction < 0 || reduction > 2) return fail(RKL_ERR_DTYPE, "unknown reduction %d", reduction);
+  if (B < 1 || Sm1 < 1 || H < 1 || V < 1) return fail(RKL_ERR_SHAPE, "B, Sm1, H, V must be >= 1");
+  if (B * Sm1 >= (int64_t(1) << 31)) return fail(RKL_ERR_SHAPE, "B*Sm1 = %lld exceeds 2^31-1", (long long)(B * Sm1));
+  if (H > 65536) return fail(RKL_ERR_SHAPE, "H = %lld exceeds 65536", (long long)H);
+  if (V >= (int64_t(1) << 30)) return fail(RKL_ERR_SHAPE, "V = %lld too large", (long long)V);
+  if (N < 0 || N > B * Sm1) return fail(RKL_ERR_SHAPE, "N = %d outside [0, B*Sm1]", N);
+  if (dtype == RKL_BF16) {
+    if (H % 64 != 0) return fail(RKL_ERR_SHAPE, "bf16 requires H %% 64 == 0 (H = %lld)", (long long)H);
+    if (payload == RKL_PAYLOAD_LOGITS && V % 8 != 0)
+      return fail(RKL_ERR_SHAPE, "bf16 logits payload requires V %% 8 == 0 (V = %lld)", (long long)V);
+  }
+  return RKL_OK;
+}
+
+static rkl_status check_ptr(const void* p, const char* name, bool required = true) {
+  if (p == nullptr) return required ? fail(RKL_ERR_NULL, "%s is NULL", name) : RKL_OK;
+  if (!aligned16(p)) return fail(RKL_ERR_ALIGN, "%s is not 16-byte aligned", name);
+  return RKL_OK;
+}
+
+#define RKL_TRY(x)                   \
+  do {                               \
+    rkl_status s__ = (x);            \
+    if (s__ != RKL_OK) return s__;   \
+  } while (0)
+
+static uint8_t* ws_at(void* ws, size_t off) { return static_cast<uint8_t*>(ws) + off; }
+
+// ------------------------------------------------------------------ forward
+static rkl_status forward_impl(rkl_payload payload, const void* h_s, const void* teacher, const void* W_s,
+                               const void* W_t, rkl_dtype dtype, int64_t B, int64_t Sm1, int64_t H, int64_t V,
+                               const int32_t* row_idx, int32_t N, rkl_reduction reduction, float* loss_tok,
+                               float* loss, float* saved, void* workspace, size_t workspace_bytes, void* stream_) {
+  RKL_TRY(check_common(payload, dtype, B, Sm1, H, V, N, reduction));
+  RKL_TRY(check_ptr(h_s, "h_s"));
+  RKL_TRY(check_ptr(teacher, payload == RKL_PAYLOAD_HIDDEN ? "h_t" : "teacher_logits"));
+  RKL_TRY(check_ptr(W_s, "W_s"));
+  if (payload == RKL_PAYLOAD_HIDDEN) RKL_TRY(check_ptr(W_t, "W_t"));
+  RKL_TRY(check_ptr(row_idx, "row_idx"));
+  RKL_TRY(check_ptr(loss_tok, "loss_tok", false));
+  RKL_TRY(check_ptr(loss, "loss", false));
+  RKL_TRY(check_ptr(saved, "saved", N > 0));
+  RKL_TRY(check_ptr(workspace, "workspace"));
+  const Plan pl = make_plan(payload, dtype, N, H, V);
+  if (workspace_bytes < pl.total)
+    return fail(RKL_ERR_WORKSPACE, "workspace is %zu bytes, %zu needed", workspace_bytes, pl.total);
+  int sms = 0;
+  RKL_TRY(device_setup(&sms));
+  cudaStream_t s = static_cast<cudaStream_t>(stream_);
+  const long long T = B * Sm1;
+  const bool bf16 = dtype == RKL_BF16;
+  const bool hidden = payload == RKL_PAYLOAD_HIDDEN;
+
+  if (N > 0) {
+    float* part = reinterpret_cast<float*>(ws_at(workspace, pl.off_part));
+    float* lse_ext = reinterpret_cast<float*>(ws_at(workspace, pl.off_lse));
+    // S2: compact the rows (skipped when every row is trainable).
+    const void* as = h_s;
+    const void* at = teacher;
+    if (N < T) {
+      as = ws_at(workspace, pl.off_hcs);
+      at = hidden ? ws_at(workspace, pl.off_hct) : nullptr;
+      RKL_CUDA(launch_gather(h_s, hidden ? teacher : nullptr, const_cast<void*>(as), const_cast<void*>(at), row_idx,
+                             N, static_cast<int>(H * pl.es), s));
+    }
+    // S8: teacher log-sum-exp from the shipped logits.
+    if (!hidden) RKL_CUDA(launch_teacher_lse(teacher, bf16, row_idx, N, static_cast<int>(V), V, lse_ext, s));
+    const int ng = hidden ? 2 : 1;
+    if (bf16) {
+      FusedArgs a;
+      memset(&a, 0, sizeof(a));
+      RKL_TRY(make_map(&a.tm_as, as, false, H, N, H * 2, kBK, kBM));
+      RKL_TRY(make_map(&a.tm_bs, W_s, false, H, V, H * 2, kBK, kBN));
+      if (hidden) {
+        RKL_TRY(make_map(&a.tm_at, at, false, H, N, H * 2, kBK, kBM));
+        RKL_TRY(make_map(&a.tm_bt, W_t, false, H, V, H * 2, kBK, kBN));
+      } else {
+        a.teacher = static_cast<const uint16_t*>(teacher);
+        a.teacher_rows = N < T ? row_idx : nullptr;
+        a.teacher_pitch = V;
+      }
+      a.part = part;
+      a.N = N;
+      a.n_pad = pl.n_pad;
+      a.H = static_cast<int>(H);
+      a.V = static_cast<int>(V);
+      a.KB = static_cast<int>(H / kBK);
+      a.IT = pl.VT;
+      a.vt_base = 0;
+      a.S = pl.S;
+      const int MT = (N + kBM - 1) / kBM;
+      RKL_CUDA(launch_fused(ng, false, a, dim3(MT, pl.S), s));
+    } else {
+      SimtArgs a;
+      memset(&a, 0, sizeof(a));
+      a.as = static_cast<const float*>(as);
+      a.bs = static_cast<const float*>(W_s);
+      if (hidden) {
+        a.at = static_cast<const float*>(at);
+        a.bt = static_cast<const float*>(W_t);
+      } else {
+        a.teacher = static_cast<const float*>(teacher);
+        a.teacher_rows = N < T ? row_idx : nullptr;
+        a.teacher_pitch = V;
+      }
+      a.part = part;
+      a.N = N;
+      a.n_pad = pl.n_pad;
+      a.H = static_cast<int>(H);
+      a.V = static_cast<int>(V);
+      a.IT = pl.VT;
+      a.S = pl.S;
+      a.ng = ng;
+      const int MT = (N + kSimtBN - 1) / kSimtBN;
+      RKL_CUDA(launch_simt_fused(false, a, dim3(MT, pl.S), s));
+    }
+    // S4
+    RKL_CUDA(launch_combine(part, pl.S, pl.n_pad, N, hidden, lse_ext, saved, s));
+  }
+  if (loss_tok) RKL_CUDA(launch_scatter_loss(saved, row_idx, N, T, loss_tok, s));
+  if (loss && reduction != RKL_REDUCE_NONE)
+    RKL_CUDA(launch_reduce(saved, row_idx, N, static_cast<int>(B), static_cast<int>(Sm1), reduction, loss, s));
+  return RKL_OK;
+}
+
+// ------------------------------------------------------------------ backward
+static rkl_status backward_impl(rkl_payload payload, const void* h_s, const void* teacher, const void* W_s,
+                                const void* W_t, rkl_dtype dtype, int64_t B, int64_t Sm1, int64_t H, int64_t V,
+                                const int32_t* row_idx, int32_t N, rkl_reduction reduction, const float* saved,
+                                const float* grad_loss, const float* grad_tok, float* dH_s, float* dW_s,
+                                void* workspace, size_t workspace_bytes, void* stream_) {
+  RKL_TRY(check_common(payload, dtype, B, Sm1, H, V, N, reduction));
+  RKL_TRY(check_ptr(h_s, "h_s"));
+  RKL_TRY(check_ptr(teacher, payload == RKL_PAYLOAD_HIDDEN ? "h_t" : "teacher_logits"));
+  RKL_TRY(check_ptr(W_s, "W_s"));
+  if (payload == RKL_PAYLOAD_HIDDEN) RKL_TRY(check_ptr(W_t, "W_t"));
+  RKL_TRY(check_ptr(row_idx, "row_idx"));
+  RKL_TRY(check_ptr(saved, "saved", N > 0));
+  RKL_TRY(check_ptr(grad_loss, "grad_loss", false));
+  RKL_TRY(check_ptr(grad_tok, "grad_tok", false));
+  RKL_TRY(check_ptr(dH_s, "dH_s"));
+  RKL_TRY(check_ptr(dW_s, "dW_s"));
+  RKL_TRY(check_ptr(workspace, "workspace"));
+  const Plan pl = make_plan(payload, dtype, N, H, V);
+  if (workspace_bytes < pl.total)
+    return fail(RKL_ERR_WORKSPACE, "workspace is %zu bytes, %zu needed", workspace_bytes, pl.total);
+  int sms = 0;
+  RKL_TRY(device_setup(&sms));
+  cudaStream_t s = static_cast<cudaStream_t>(stream_);
+  const long long T = B * Sm1;
+  const bool bf16 = dtype == RKL_BF16;
+  const bool hidden = payload == RKL_PAYLOAD_HIDDEN;
+  float* dHc = reinterpret_cast<float*>(ws_at(workspace, pl.off_dh));
+
+  if (N == 0) {
+    RKL_CUDA(cudaMemsetAsync(dW_s, 0, size_t(V) * H * sizeof(float), s));
+    RKL_CUDA(launch_scatter_dh(dHc, row_idx, 0, T, static_cast<int>(H), dH_s, s));
+    return RKL_OK;
+  }
+  const void* as = h_s;
+  const void* at = teacher;
+  if (N < T) {
+    as = ws_at(workspace, pl.off_hcs);
+    at = hidden ? ws_at(workspace, pl.off_hct) : nullptr;
+    RKL_CUDA(launch_gather(h_s, hidden ? teacher : nullptr, const_cast<void*>(as), const_cast<void*>(at), row_idx, N,
+                           static_cast<int>(H * pl.es), s));
+  }
+  float* rowc = reinterpret_cast<float*>(ws_at(workspace, pl.off_rowc));
+  RKL_CUDA(launch_row_weights(saved, row_idx, N, pl.n_pad, static_cast<int>(B), static_cast<int>(Sm1), reduction,
+                              grad_loss, grad_tok, rowc, s));
+  void* dz = ws_at(workspace, pl.off_dz);
+  const int ng = hidden ? 2 : 1;
+  const int nchunks = static_cast<int>((V + pl.Vc - 1) / pl.Vc);
+
+  if (bf16) {
+    FusedArgs a;
+    memset(&a, 0, sizeof(a));
+    RKL_TRY(make_map(&a.tm_as, as, false, H, N, H * 2, kBK, kBM));
+    RKL_TRY(make_map(&a.tm_bs, W_s, false, H, V, H * 2, kBK, kBN));
+    if (hidden) {
+      RKL_TRY(make_map(&a.tm_at, at, false, H, N, H * 2, kBK, kBM));
+      RKL_TRY(make_map(&a.tm_bt, W_t, false, H, V, H * 2, kBK, kBN));
+    } else {
+      a.teacher = static_cast<const uint16_t*>(teacher);
+      a.teacher_rows = N < T ? row_idx : nullptr;
+      a.teacher_pitch = V;
+    }
+    a.rowc = rowc;
+    a.N = N;
+    a.n_pad = pl.n_pad;
+    a.H = static_cast<int>(H);
+    a.V = static_cast<int>(V);
+    a.KB = static_cast<int>(H / kBK);
+    const int MT = (N + kBM - 1) / kBM;
+
+    GradArgs g;
+    memset(&g, 0, sizeof(g));
+    RKL_TRY(make_map(&g.tm_hs_mn, as, false, H, N, H * 2, 64, 64));
+    RKL_TRY(make_map(&g.tm_ws_mn, W_s, false, H, V, H * 2, 64, 64));
+    RKL_TRY(make_map(&g.tm_dw, dW_s, true, H, V, H * 4, 32, 32));
+    RKL_TRY(make_map(&g.tm_dh, dHc, true, H, N, H * 4, 32, 32));
+    g.N = N;
+    g.H = static_cast<int>(H);
+    g.NT = static_cast<int>(H / kGradBN) + (H % kGradBN ? 1 : 0);
+    g.MTH = MT;
+    g.nH = g.MTH * g.NT;
+    g.KBW = (N + kBK - 1) / kBK;
+
+    for (int c = 0; c < nchunks; ++c) {
+      const int cv0 = c * pl.Vc;
+      const int cw = static_cast<int>((V - cv0) < pl.Vc ? (V - cv0) : pl.Vc);
+      // S6: recompute the logits of this chunk and write dz (bf16) [N, cw].
+      RKL_TRY(make_map(&a.tm_dz, dz, false, cw, N, size_t(pl.Vc) * 2, 64, 32));
+      a.IT = (cw + kBN - 1) / kBN;
+      a.vt_base = cv0 / kBN;
+      a.chunk_v0 = cv0;
+      a.items_total = MT * a.IT;
+      const int grid = a.items_total < sms ? a.items_total : sms;
+      RKL_CUDA(launch_fused(ng, true, a, dim3(grid), s));
+      // S7: dW_s[chunk] = dz^T hc_s and dHc (+)= dz W_s[chunk].
+      RKL_TRY(make_map(&g.tm_dz_k, dz, false, cw, N, size_t(pl.Vc) * 2, 64, 128));
+      RKL_TRY(make_map(&g.tm_dz_mn, dz, false, cw, N, size_t(pl.Vc) * 2, 64, 64));
+      g.cw = cw;
+      g.cv0 = cv0;
+      g.MTW = (cw + kBM - 1) / kBM;
+      g.nW = g.MTW * g.NT;
+      g.KBH = (cw + kBK - 1) / kBK;
+      g.dh_accumulate = c > 0;
+      const int tiles = g.nW + g.nH;
+      RKL_CUDA(launch_grad(g, tiles < sms ? tiles : sms, s));
+    }
+  } else {
+    SimtArgs a;
+    memset(&a, 0, sizeof(a));
+    a.as = static_cast<const float*>(as);
+    a.bs = static_cast<const float*>(W_s);
+    if (hidden) {
+      a.at = static_cast<const float*>(at);
+      a.bt = static_cast<const float*>(W_t);
+    } else {
+      a.teacher = static_cast<const float*>(teacher);
+      a.teacher_rows = N < T ? row_idx : nullptr;
+      a.teacher_pitch = V;
+    }
+    a.rowc = rowc;
+    a.dz = static_cast<float*>(dz);
+    a.N = N;
+    a.n_pad = pl.n_pad;
+    a.H = static_cast<int>(H);
+    a.V = static_cast<int>(V);
+    a.ng = ng;
+    const int MT = (N + kSimtBN - 1) / kSimtBN;
+    for (int c = 0; c < nchunks; ++c) {
+      const int cv0 = c * pl.Vc;
+      const int cw = static_cast<int>((V - cv0) < pl.Vc ? (V - cv0) : pl.Vc);
+      a.cw = cw;
+      a.IT = (cw + kSimtBN - 1) / kSimtBN;
+      a.vt_base = cv0 / kSimtBN;
+      a.chunk_v0 = cv0;
+      const int items = MT * a.IT;
+      RKL_CUDA(launch_simt_fused(true, a, dim3(items < 4 * sms ? items : 4 * sms), s));
+      const float* dzf = static_cast<const float*>(dz);
+      // dW_s[cv0 + m, n] = sum_k dz[k, m] hc_s[k, n]
+      RKL_CUDA(launch_simt_gemm(dzf, 1, cw, a.as, H, 1, dW_s + size_t(cv0) * H, H, cw, static_cast<int>(H), N, 0,
+                                s));
+      // dHc[m, n] (+)= sum_k dz[m, k] W_s[cv0 + k, n]
+      RKL_CUDA(launch_simt_gemm(dzf, cw, 1, a.bs + size_t(cv0) * H, H, 1, dHc, H, N, static_cast<int>(H), cw,
+                                c > 0, s));
+    }
+  }
+  RKL_CUDA(launch_scatter_dh(dHc, row_idx, N, T, static_cast<int>(H), dH_s, s));
+  return RKL_OK;
+}
+
+}  // namespace rkl
+
+// ====================================================================== C ABI
+using namespace rkl;
+
+extern "C" {
+
+const char* rkl_version(void) { return "rkl 0.1 (sm_100a)"; }
+
+const char* rkl_last_error(void) { return g_last_error.c_str(); }
+
+rkl_status rkl_workspace_size(rkl_payload payload, rkl_dtype dtype, int64_t n_max, int64_t B, int64_t Sm1, int64_t H,
+                              int64_t V, size_t* bytes) {
+  if (bytes == nullptr) return fail(RKL_ERR_NULL, "bytes is NULL");
+  RKL_TRY(check_common(payload, dtype, B, Sm1, H, V, 0, 0));
+  if (n_max < 0 || n_max > B * Sm1) return fail(RKL_ERR_SHAPE, "n_max outside [0, B*Sm1]");
+  *bytes = make_plan(payload, dtype, n_max, H, V).total;
+  return RKL_OK;
+}
+
+rkl_status rkl_compact_rows(const uint8_t* mask, int64_t B, int64_t Sm1, int32_t* row_idx, int32_t* n_dev,
+                            void* stream) {
+  if (mask == nullptr || row_idx == nullptr || n_dev == nullptr)
+    return fail(RKL_ERR_NULL, "mask, row_idx and n_dev must be non-NULL");
+  if (!aligned16(row_idx)) return fail(RKL_ERR_ALIGN, "row_idx is not 16-byte aligned");
+  if (B < 1 || Sm1 < 1) return fail(RKL_ERR_SHAPE, "B and Sm1 must be >= 1");
+  if (B * Sm1 >= (int64_t(1) << 31)) return fail(RKL_ERR_SHAPE, "B*Sm1 exceeds 2^31-1");
+  int sms = 0;
+  RKL_TRY(device_setup(&sms));
+  RKL_CUDA(launch_compact(mask, B * Sm1, row_idx, n_dev, static_cast<cudaStream_t>(stream)));
+  return RKL_OK;
+}
+
+rkl_status rkl_forward_hidden(const void* h_s, const void* h_t, const void* W_s, const void* W_t, rkl_dtype dtype,
+                              int64_t B, int64_t Sm1, int64_t H, int64_t V, const int32_t* row_idx, int32_t N,
+                              rkl_reduction reduction, float* loss_tok, float* loss, float* saved, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+  return forward_impl(RKL_PAYLOAD_HIDDEN, h_s, h_t, W_s, W_t, dtype, B, Sm1, H, V, row_idx, N, reduction, loss_tok,
+                      loss, saved, workspace, workspace_bytes, stream);
+}
+
+rkl_status rkl_forward_logits(const void* h_s, const void* W_s, const void* teacher_logits, rkl_dtype dtype,
+                              int64_t B, int64_t Sm1, int64_t H, int64_t V, const int32_t* row_idx, int32_t N,
+                              rkl_reduction reduction, float* loss_tok, float* loss, float* saved, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+  return forward_impl(RKL_PAYLOAD_LOGITS, h_s, teacher_logits, W_s, nullptr, dtype, B, Sm1, H, V, row_idx, N,
+                      reduction, loss_tok, loss, saved, workspace, workspace_bytes, stream);
+}
+
+rkl_status rkl_backward(rkl_payload payload, const void* h_s, const void* teacher, const void* W_s, const void* W_t,
+                        rkl_dtype dtype, int64_t B, int64_t Sm1, int64_t H, int64_t V, const int32_t* row_idx,
+                        int32_t N, rkl_reduction reduction, const float* saved, const float* grad_loss,
+                        const float* grad_tok, float* dH_s, float* dW_s, void* workspace, size_t workspace_bytes,
+                        void* stream) {
+  return backward_impl(payload, h_s, teacher, W_s, W_t, dtype, B, Sm1, H, V, row_idx, N, reduction, saved, grad_loss,
+                       grad_tok, dH_s, dW_s, workspace, workspace_bytes, stream);
+}
+
+rkl_status rkl_device_error(int32_t* code) {
+  if (code == nullptr) return fail(RKL_ERR_NULL, "code is NULL");
+  RKL_CUDA(cudaDeviceSynchronize());
+  int v = 0;
+  RKL_CUDA(read_and_clear_device_error(&v));
+  *code = v;
+  if (v != 0) return fail(RKL_ERR_DEVICE, "a kernel wait ran out (bits 0x%x); its outputs are invalid", v);
+  return RKL_OK;
+}
+
+int32_t rkl_kernel_count(void) { return K_COUNT; }
+
+const char* rkl_kernel_name(int32_t kernel_id) { return kernel_name(kernel_id); }
+
+rkl_status rkl_profile_enable(int32_t enable) {
+  g_profile.store(enable != 0);
+  return RKL_OK;
+}
+
+static rkl_status drain_profile() {
+  std::vector<ProfRec> pend;
+  {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    pend.swap(g_prof_pending);
+  }
+  for (const ProfRec& r : pend) {
+    float ms = 0.f;
+    cudaError_t e = cudaEventSynchronize(r.b);
+    if (e == cudaSuccess) e = cudaEventElapsedTime(&ms, r.a, r.b);
+    cudaEventDestroy(r.a);
+    cudaEventDestroy(r.b);
+    if (e != cudaSuccess) return fail(RKL_ERR_CUDA, "profile event: %s", cudaGetErrorString(e));
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    g_prof_ms[r.id] += ms;
+    g_prof_n[r.id] += 1;
+  }
+  return RKL_OK;
+}
+
+rkl_status rkl_profile_reset(void) {
+  RKL_TRY(drain_profile());
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  for (int i = 0; i < K_COUNT; ++i) {
+    g_prof_ms[i] = 0.0;
+    g_prof_n[i] = 0;
+  }
+  return RKL_OK;
+}
+
+rkl_status rkl_profile_read(int32_t kernel_id, double* total_ms, int64_t* launches) {
+  if (kernel_id < 0 || kernel_id >= K_COUNT) return fail(RKL_ERR_SHAPE, "kernel id %d out of range", kernel_id);
+  if (total_ms == nullptr || launches == nullptr) return fail(RKL_ERR_NULL, "outputs are NULL");
+  RKL_TRY(drain_profile());
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  *total_ms = g_prof_ms[kernel_id];
+  *launches = g_prof_n[kernel_id];
+  return RKL_OK;
+}
+
+int64_t rkl_launch_count(void) { return g_launches.load(); }
+
+}  // extern "C"

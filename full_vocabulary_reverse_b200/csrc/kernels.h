@@ -1,0 +1,124 @@
+// kernels.h -- launcher interface between the C-ABI layer (api.cu) and the
+// kernel translation units.  Host-only declarations; no torch types.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace rkl {
+
+// Kernel ids for the measurement hooks (rkl_profile_*).
+enum KernelId : int {
+  K_COMPACT = 0,
+  K_GATHER,
+  K_FWD_DUAL_TC,      // S3 hidden payload, tcgen05 (z_s and z_t, online stats)
+  K_FWD_SINGLE_TC,    // S3 logits payload, tcgen05 (z_s, teacher rows loaded)
+  K_TEACHER_LSE,      // S8 teacher log-sum-exp, bandwidth bound
+  K_COMBINE,          // S4 merge split statistics
+  K_SCATTER_LOSS,     // S4 loss_tok scatter
+  K_REDUCE,           // S4 scalar loss
+  K_ROW_WEIGHTS,      // S5
+  K_DZ_DUAL_TC,       // S6 hidden payload, tcgen05 recompute + dz
+  K_DZ_SINGLE_TC,     // S6 logits payload
+  K_GRAD_TC,          // S7 dW_s and dH_s tiles (grouped), tcgen05
+  K_SCATTER_DH,       // S7 dH scatter to [T, H]
+  K_FWD_SIMT,         // fp32 S3 (CUDA cores)
+  K_DZ_SIMT,          // fp32 S6
+  K_GRAD_SIMT,        // fp32 S7
+  K_COUNT
+};
+
+const char* kernel_name(int id);
+
+// Records (optionally timed) launches; implemented in api.cu.
+struct LaunchScope {
+  LaunchScope(int id, cudaStream_t s);
+  ~LaunchScope();
+  int id;
+  cudaStream_t stream;
+  cudaEvent_t ev0 = nullptr, ev1 = nullptr;
+};
+
+constexpr int kBM = 128;       // rows per tile (TMEM lanes)
+constexpr int kBN = 128;       // vocab columns per fused tile
+constexpr int kBK = 64;        // K per pipeline stage (128 B of bf16)
+constexpr int kGradBN = 256;   // H columns per gradient tile
+constexpr int kSplits = 37;    // vocab splits of the forward (148 SMs = 4 x 37)
+
+// ---------------------------------------------------------------- tcgen05
+struct FusedArgs {
+  // operand maps (bf16, 128-byte swizzle, box {64, 128})
+  CUtensorMap tm_as, tm_at, tm_bs, tm_bt;
+  CUtensorMap tm_dz;                 // dz chunk output [N, cw] bf16, box {64, 32}
+  const uint16_t* teacher;           // logits payload: teacher logits [T, V] bf16
+  const int32_t* teacher_rows;       // logits payload: row_idx (nullptr = identity)
+  long long teacher_pitch;           // elements per teacher row
+  float* part;                       // stats: [S][5][n_pad]
+  const float* rowc;                 // dz: [3][n_pad]: lse_s*log2e, cst, g
+  int N, n_pad, H, V, KB;
+  int IT;                            // vocab tiles per m-tile covered by this launch
+  int vt_base;                       // first vocab tile of this launch
+  int S;                             // stats: number of vocab splits
+  int items_total;                   // dz: m-tiles * IT
+  int chunk_v0;                      // dz: first vocab column of the chunk
+};
+
+struct GradArgs {
+  CUtensorMap tm_dz_k;    // dz chunk [N, cw] bf16 as K-major A (box {64, 128})
+  CUtensorMap tm_dz_mn;   // dz chunk as MN-major A (box {64, 64})
+  CUtensorMap tm_hs_mn;   // hc_s [N, H] bf16 as MN-major B (box {64, 64})
+  CUtensorMap tm_ws_mn;   // W_s [V, H] bf16 as MN-major B (box {64, 64})
+  CUtensorMap tm_dw;      // dW_s [V, H] fp32 output (box {32, 32})
+  CUtensorMap tm_dh;      // dHc [N, H] fp32 output (box {32, 32})
+  int N, H, cw, cv0;
+  int MTW, MTH, NT, nW, nH, KBW, KBH;
+  int dh_accumulate;
+};
+
+size_t fused_smem_bytes(int ng, bool dz);
+size_t grad_smem_bytes();
+cudaError_t tc_setup(int device);  // one-time cudaFuncSetAttribute per device
+cudaError_t launch_fused(int ng, bool dz, const FusedArgs& a, dim3 grid, cudaStream_t s);
+cudaError_t launch_grad(const GradArgs& a, int grid, cudaStream_t s);
+cudaError_t read_and_clear_device_error(int* code);
+
+// ---------------------------------------------------------------- small kernels
+cudaError_t launch_compact(const uint8_t* mask, long long T, int32_t* row_idx, int32_t* n_dev, cudaStream_t s);
+cudaError_t launch_gather(const void* h_s, const void* h_t, void* hc_s, void* hc_t, const int32_t* row_idx, int N,
+                          int row_bytes, cudaStream_t s);
+cudaError_t launch_teacher_lse(const void* logits, bool bf16, const int32_t* row_idx, int N, int V,
+                               long long pitch, float* lse_t, cudaStream_t s);
+cudaError_t launch_combine(const float* part, int S, int n_pad, int N, bool teacher_from_part,
+                           const float* lse_t_ext, float* saved, cudaStream_t s);
+cudaError_t launch_scatter_loss(const float* saved, const int32_t* row_idx, int N, long long T, float* loss_tok,
+                                cudaStream_t s);
+cudaError_t launch_reduce(const float* saved, const int32_t* row_idx, int N, int B, int Sm1, int reduction,
+                          float* loss, cudaStream_t s);
+cudaError_t launch_row_weights(const float* saved, const int32_t* row_idx, int N, int n_pad, int B, int Sm1,
+                               int reduction, const float* grad_loss, const float* grad_tok, float* rowc,
+                               cudaStream_t s);
+cudaError_t launch_scatter_dh(const float* dHc, const int32_t* row_idx, int N, long long T, int H, float* dH_s,
+                              cudaStream_t s);
+
+// ---------------------------------------------------------------- fp32 CUDA-core path
+struct SimtArgs {
+  const float* as; const float* at;   // compact rows [N, H] (at: hidden payload)
+  const float* bs; const float* bt;   // W [V, H] (bt: hidden payload)
+  const float* teacher;               // logits payload: [T, V] fp32
+  const int32_t* teacher_rows;
+  long long teacher_pitch;
+  float* part; const float* rowc;
+  float* dz;                          // dz chunk [N, cw] fp32
+  int N, n_pad, H, V, S, IT, vt_base, chunk_v0, cw;
+  int ng;
+};
+constexpr int kSimtBN = 32;
+cudaError_t launch_simt_fused(bool dz, const SimtArgs& a, dim3 grid, cudaStream_t s);
+// C[M, Nc] (+)= sum_k A(m, k) B(k, n); A(m,k) = A[m*sam + k*sak], B(k,n) = B[k*sbk + n*sbn]
+cudaError_t launch_simt_gemm(const float* A, long long sam, long long sak, const float* B, long long sbk,
+                             long long sbn, float* C, long long ldc, int M, int Nc, int K, int accumulate,
+                             cudaStream_t s);
+
+}  // namespace rkl

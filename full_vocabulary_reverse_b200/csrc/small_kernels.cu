@@ -1,0 +1,463 @@
+// small_kernels.cu -- the bandwidth-bound and bookkeeping steps of the loss:
+//   S1 compaction of the trainable rows, S2 row gather, S8 teacher
+//   log-sum-exp over shipped logits, S4 split merge / scatter / reduction,
+//   S5 per-row backward weights, and the final dH scatter.
+// Sources: "fix(megatron): compact actor logits before projection" (slime PR
+// #2310, Summary: project only the N loss-masked rows, scatter scalars back,
+// empty masks keep zero gradients) and "feat(mopd): add full-vocabulary
+// on-policy distillation" (NeMo RL PR #3978: the objective, the logits
+// payload, the token-level / nested per-sequence reduction).
+#include <cuda_bf16.h>
+
+#include <cfloat>
+
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace rkl {
+namespace {
+
+__device__ __forceinline__ int lower_bound_i32(const int32_t* a, int n, long long key) {
+  int lo = 0, hi = n;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (static_cast<long long>(a[mid]) < key)
+      lo = mid + 1;
+    else
+      hi = mid;
+  }
+  return lo;
+}
+
+// --------------------------------------------------------------------- S1
+// One CTA, 1024 threads; tiles of 8 mask bytes per thread; block-wide
+// exclusive scan; ascending row indices by construction.
+__global__ void __launch_bounds__(1024) compact_kernel(const uint8_t* __restrict__ mask, long long T,
+                                                       int32_t* __restrict__ row_idx, int32_t* __restrict__ n_dev) {
+  constexpr int ITEMS = 8;
+  __shared__ int warp_incl[32];
+  __shared__ int carry;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid == 0) carry = 0;
+  __syncthreads();
+  for (long long base = 0; base < T; base += 1024LL * ITEMS) {
+    const long long i0 = base + static_cast<long long>(tid) * ITEMS;
+    int flags = 0, cnt = 0;
+#pragma unroll
+    for (int k = 0; k < ITEMS; ++k) {
+      const bool f = (i0 + k < T) && mask[i0 + k] != 0;
+      flags |= static_cast<int>(f) << k;
+      cnt += f;
+    }
+    int x = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) warp_incl[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+      int w = warp_incl[lane];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, w, o);
+        if (lane >= o) w += y;
+      }
+      warp_incl[lane] = w;
+    }
+    __syncthreads();
+    int pos = carry + (warp ? warp_incl[warp - 1] : 0) + x - cnt;
+#pragma unroll
+    for (int k = 0; k < ITEMS; ++k)
+      if (flags & (1 << k)) row_idx[pos++] = static_cast<int32_t>(i0 + k);
+    __syncthreads();
+    if (tid == 0) carry += warp_incl[31];
+    __syncthreads();
+  }
+  if (tid == 0) *n_dev = carry;
+}
+
+// --------------------------------------------------------------------- S2
+// hc[k] = h[row_idx[k]] for k < N; blockIdx.y selects student / teacher.
+__global__ void __launch_bounds__(256) gather_kernel(const uint8_t* __restrict__ h_s, const uint8_t* __restrict__ h_t,
+                                                     uint8_t* __restrict__ hc_s, uint8_t* __restrict__ hc_t,
+                                                     const int32_t* __restrict__ row_idx, int N, int row_bytes) {
+  const uint8_t* src = blockIdx.y == 0 ? h_s : h_t;
+  uint8_t* dst = blockIdx.y == 0 ? hc_s : hc_t;
+  for (int k = blockIdx.x; k < N; k += gridDim.x) {
+    const uint8_t* s = src + static_cast<long long>(row_idx[k]) * row_bytes;
+    uint8_t* d = dst + static_cast<long long>(k) * row_bytes;
+    if ((row_bytes & 15) == 0) {
+      const uint4* s4 = reinterpret_cast<const uint4*>(s);
+      uint4* d4 = reinterpret_cast<uint4*>(d);
+      for (int i = threadIdx.x; i < row_bytes / 16; i += blockDim.x) d4[i] = __ldg(s4 + i);
+    } else {
+      const uint32_t* s1 = reinterpret_cast<const uint32_t*>(s);
+      uint32_t* d1 = reinterpret_cast<uint32_t*>(d);
+      for (int i = threadIdx.x; i < row_bytes / 4; i += blockDim.x) d1[i] = __ldg(s1 + i);
+    }
+  }
+}
+
+// --------------------------------------------------------------------- S8
+// lse_t[k] = log sum_v exp(z_t[row_idx[k], v]) over the shipped teacher
+// logits.  One CTA per row, 16-byte streaming loads, four in flight per
+// thread, per-thread online (max, sum), then a block merge.
+__device__ __forceinline__ void lse_merge(float& m, float& s, float m2, float s2) {
+  const float nm = fmaxf(m, m2);
+  if (nm == -INFINITY) return;
+  s = s * ex2((m - nm) * kLog2e) + s2 * ex2((m2 - nm) * kLog2e);
+  m = nm;
+}
+
+__device__ __forceinline__ uint4 ldg_stream_v4(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+template <typename T>
+__device__ __forceinline__ void vec_to_float(const uint4& w, float* out);
+
+template <>
+__device__ __forceinline__ void vec_to_float<__nv_bfloat16>(const uint4& w, float* out) {
+  const uint32_t a[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    out[2 * i] = __uint_as_float(a[i] << 16);
+    out[2 * i + 1] = __uint_as_float(a[i] & 0xFFFF0000u);
+  }
+}
+
+template <>
+__device__ __forceinline__ void vec_to_float<float>(const uint4& w, float* out) {
+  out[0] = __uint_as_float(w.x);
+  out[1] = __uint_as_float(w.y);
+  out[2] = __uint_as_float(w.z);
+  out[3] = __uint_as_float(w.w);
+}
+
+template <typename T>
+__device__ __forceinline__ float to_f(T x);
+template <>
+__device__ __forceinline__ float to_f<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T>
+__global__ void __launch_bounds__(256) teacher_lse_kernel(const T* __restrict__ logits,
+                                                          const int32_t* __restrict__ row_idx, int N, int V,
+                                                          long long pitch, float* __restrict__ lse_t) {
+  constexpr int VEC = 16 / sizeof(T);
+  constexpr int UNROLL = 4;
+  const int k = blockIdx.x;
+  if (k >= N) return;
+  const long long r = row_idx ? row_idx[k] : k;
+  const T* row = logits + r * pitch;
+  float m = -INFINITY, s = 0.f;
+  const bool vec_ok = ((reinterpret_cast<uintptr_t>(row) & 15) == 0);
+  int done = 0;
+  if (vec_ok) {
+    const int nvec = V / VEC;
+    const uint4* rv = reinterpret_cast<const uint4*>(row);
+    int i = threadIdx.x;
+    for (; i + (UNROLL - 1) * 256 < nvec; i += UNROLL * 256) {
+      uint4 w[UNROLL];
+#pragma unroll
+      for (int u = 0; u < UNROLL; ++u) w[u] = ldg_stream_v4(rv + i + u * 256);
+#pragma unroll
+      for (int u = 0; u < UNROLL; ++u) {
+        float x[VEC];
+        vec_to_float<T>(w[u], x);
+        float vm = x[0];
+#pragma unroll
+        for (int j = 1; j < VEC; ++j) vm = fmaxf(vm, x[j]);
+        if (vm > m) {
+          s *= ex2((m - vm) * kLog2e);
+          m = vm;
+        }
+        const float m2 = m * kLog2e;
+        float acc = 0.f;
+#pragma unroll
+        for (int j = 0; j < VEC; ++j) acc += ex2(fmaf(x[j], kLog2e, -m2));
+        s += acc;
+      }
+    }
+    for (; i < nvec; i += 256) {
+      float x[VEC];
+      vec_to_float<T>(ldg_stream_v4(rv + i), x);
+#pragma unroll
+      for (int j = 0; j < VEC; ++j) {
+        if (x[j] > m) {
+          s *= ex2((m - x[j]) * kLog2e);
+          m = x[j];
+        }
+        s += ex2((x[j] - m) * kLog2e);
+      }
+    }
+    done = nvec * VEC;
+  }
+  for (int v = done + threadIdx.x; v < V; v += 256) {
+    const float x = to_f<T>(row[v]);
+    if (x > m) {
+      s *= ex2((m - x) * kLog2e);
+      m = x;
+    }
+    s += ex2((x - m) * kLog2e);
+  }
+  // block merge (fixed order)
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
+    const float s2 = __shfl_xor_sync(0xffffffffu, s, o);
+    lse_merge(m, s, m2, s2);
+  }
+  __shared__ float sm[8], ss[8];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) {
+    sm[warp] = m;
+    ss[warp] = s;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float M = sm[0], Ssum = ss[0];
+    for (int w = 1; w < 8; ++w) lse_merge(M, Ssum, sm[w], ss[w]);
+    lse_t[k] = M + logf(Ssum);
+  }
+}
+
+// --------------------------------------------------------------------- S4
+// Merge the per-split statistics of each row in split order; L = A/S_s -
+// lse_s + lse_t.  The student and teacher statistics go through the same
+// operations, so teacher == student gives L = 0 exactly.
+__global__ void combine_kernel(const float* __restrict__ part, int S, int n_pad, int N, int teacher_from_part,
+                               const float* __restrict__ lse_ext, float* __restrict__ saved) {
+  const int k = blockIdx.x * blockDim.x + threadIdx.x;
+  if (k >= N) return;
+  float m_s = -INFINITY, S_s = 0.f, A = 0.f, m_t = -INFINITY, S_t = 0.f;
+  for (int s = 0; s < S; ++s) {
+    const float* b = part + static_cast<size_t>(s) * 5 * n_pad + k;
+    const float ms = b[0], Ss = b[n_pad], As = b[2 * n_pad], mt = b[3 * n_pad], St = b[4 * n_pad];
+    if (ms != -INFINITY) {
+      const float nm = fmaxf(m_s, ms);
+      const float a = expf(m_s - nm), c = expf(ms - nm);
+      S_s = S_s * a + Ss * c;
+      A = A * a + As * c;
+      m_s = nm;
+    }
+    if (teacher_from_part && mt != -INFINITY) {
+      const float nm = fmaxf(m_t, mt);
+      const float a = expf(m_t - nm), c = expf(mt - nm);
+      S_t = S_t * a + St * c;
+      m_t = nm;
+    }
+  }
+  const float lse_s = m_s + logf(S_s);
+  const float lse_t = teacher_from_part ? m_t + logf(S_t) : lse_ext[k];
+  const float L = A / S_s - lse_s + lse_t;
+  saved[3 * k + 0] = lse_s;
+  saved[3 * k + 1] = lse_t;
+  saved[3 * k + 2] = L;
+}
+
+// loss_tok[t] = L of t if t is trainable else exactly 0.
+__global__ void scatter_loss_kernel(const float* __restrict__ saved, const int32_t* __restrict__ row_idx, int N,
+                                    long long T, float* __restrict__ loss_tok) {
+  const long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (t >= T) return;
+  const int k = lower_bound_i32(row_idx, N, t);
+  loss_tok[t] = (k < N && row_idx[k] == t) ? saved[3 * k + 2] : 0.f;
+}
+
+__device__ __forceinline__ double block_sum_1024(double v, double* sh) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  if (lane == 0) sh[warp] = v;
+  __syncthreads();
+  double r = 0.0;
+  if (threadIdx.x == 0)
+    for (int w = 0; w < 32; ++w) r += sh[w];
+  __syncthreads();
+  return r;
+}
+
+// Scalar loss: token mean sum_k L_k / N, or nested mean over sequences with
+// n_b > 0 of sum_{k in b} L_k / n_b.  Fixed summation order (deterministic).
+__global__ void __launch_bounds__(1024) reduce_kernel(const float* __restrict__ saved,
+                                                      const int32_t* __restrict__ row_idx, int N, int B, int Sm1,
+                                                      int reduction, float* __restrict__ loss) {
+  __shared__ double sh[32];
+  if (reduction == 1) {
+    double acc = 0.0;
+    for (int k = threadIdx.x; k < N; k += 1024) acc += saved[3 * k + 2];
+    const double tot = block_sum_1024(acc, sh);
+    if (threadIdx.x == 0) *loss = N > 0 ? static_cast<float>(tot / N) : 0.f;
+  } else {
+    double acc = 0.0, cnt = 0.0;
+    for (int b = threadIdx.x; b < B; b += 1024) {
+      const int lo = lower_bound_i32(row_idx, N, static_cast<long long>(b) * Sm1);
+      const int hi = lower_bound_i32(row_idx, N, static_cast<long long>(b + 1) * Sm1);
+      if (hi > lo) {
+        double sb = 0.0;
+        for (int k = lo; k < hi; ++k) sb += saved[3 * k + 2];
+        acc += sb / (hi - lo);
+        cnt += 1.0;
+      }
+    }
+    const double tot = block_sum_1024(acc, sh);
+    const double c = block_sum_1024(cnt, sh);
+    if (threadIdx.x == 0) *loss = c > 0 ? static_cast<float>(tot / c) : 0.f;
+  }
+}
+
+// --------------------------------------------------------------------- S5
+// Row constants of the recompute pass: rowc[0] = lse_s*log2(e),
+// rowc[1] = lse_t - lse_s - L, rowc[2] = g = dLoss/dL_k.  Padding rows get 0.
+__global__ void __launch_bounds__(256) row_weights_kernel(const float* __restrict__ saved,
+                                                          const int32_t* __restrict__ row_idx, int N, int n_pad,
+                                                          int B, int Sm1, int reduction,
+                                                          const float* __restrict__ grad_loss,
+                                                          const float* __restrict__ grad_tok,
+                                                          float* __restrict__ rowc) {
+  __shared__ int b_eff_sh;
+  if (threadIdx.x == 0) b_eff_sh = 0;
+  __syncthreads();
+  if (reduction == 2) {
+    int local = 0;
+    for (int b = threadIdx.x; b < B; b += blockDim.x) {
+      const int lo = lower_bound_i32(row_idx, N, static_cast<long long>(b) * Sm1);
+      const int hi = lower_bound_i32(row_idx, N, static_cast<long long>(b + 1) * Sm1);
+      local += hi > lo;
+    }
+    atomicAdd(&b_eff_sh, local);
+  }
+  __syncthreads();
+  const int k = blockIdx.x * blockDim.x + threadIdx.x;
+  if (k >= n_pad) return;
+  float c0 = 0.f, c1 = 0.f, c2 = 0.f;
+  if (k < N) {
+    const int row = row_idx[k];
+    const float lse_s = saved[3 * k], lse_t = saved[3 * k + 1], L = saved[3 * k + 2];
+    float w = 0.f;
+    if (reduction == 1) {
+      w = 1.f / static_cast<float>(N);
+    } else if (reduction == 2) {
+      const int b = row / Sm1;
+      const int lo = lower_bound_i32(row_idx, N, static_cast<long long>(b) * Sm1);
+      const int hi = lower_bound_i32(row_idx, N, static_cast<long long>(b + 1) * Sm1);
+      w = 1.f / (static_cast<float>(b_eff_sh) * static_cast<float>(hi - lo));
+    }
+    float g = 0.f;
+    if (reduction != 0 && grad_loss != nullptr) g = grad_loss[0] * w;
+    if (grad_tok != nullptr) g += grad_tok[row];
+    c0 = lse_s * kLog2e;
+    c1 = lse_t - lse_s - L;
+    c2 = g;
+  }
+  rowc[k] = c0;
+  rowc[n_pad + k] = c1;
+  rowc[2 * n_pad + k] = c2;
+}
+
+// dH_s[t] = dHc[k] if t = row_idx[k], else exact zeros.
+__global__ void __launch_bounds__(256) scatter_dh_kernel(const float* __restrict__ dHc,
+                                                         const int32_t* __restrict__ row_idx, int N, long long T,
+                                                         int H, float* __restrict__ dH_s) {
+  for (long long t = blockIdx.x; t < T; t += gridDim.x) {
+    const int k = lower_bound_i32(row_idx, N, t);
+    const bool hit = k < N && row_idx[k] == t;
+    float* d = dH_s + t * H;
+    if (hit) {
+      const float* s = dHc + static_cast<long long>(k) * H;
+      if ((H & 3) == 0) {
+        float4* d4 = reinterpret_cast<float4*>(d);
+        const float4* s4 = reinterpret_cast<const float4*>(s);
+        for (int i = threadIdx.x; i < H / 4; i += blockDim.x) d4[i] = s4[i];
+      } else {
+        for (int i = threadIdx.x; i < H; i += blockDim.x) d[i] = s[i];
+      }
+    } else {
+      if ((H & 3) == 0) {
+        float4* d4 = reinterpret_cast<float4*>(d);
+        for (int i = threadIdx.x; i < H / 4; i += blockDim.x) d4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      } else {
+        for (int i = threadIdx.x; i < H; i += blockDim.x) d[i] = 0.f;
+      }
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_compact(const uint8_t* mask, long long T, int32_t* row_idx, int32_t* n_dev, cudaStream_t s) {
+  LaunchScope scope(K_COMPACT, s);
+  compact_kernel<<<1, 1024, 0, s>>>(mask, T, row_idx, n_dev);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gather(const void* h_s, const void* h_t, void* hc_s, void* hc_t, const int32_t* row_idx, int N,
+                          int row_bytes, cudaStream_t s) {
+  if (N <= 0) return cudaSuccess;
+  LaunchScope scope(K_GATHER, s);
+  dim3 grid(N < 65535 ? N : 65535, h_t ? 2 : 1);
+  gather_kernel<<<grid, 256, 0, s>>>(static_cast<const uint8_t*>(h_s), static_cast<const uint8_t*>(h_t),
+                                     static_cast<uint8_t*>(hc_s), static_cast<uint8_t*>(hc_t), row_idx, N, row_bytes);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_teacher_lse(const void* logits, bool bf16, const int32_t* row_idx, int N, int V, long long pitch,
+                               float* lse_t, cudaStream_t s) {
+  if (N <= 0) return cudaSuccess;
+  LaunchScope scope(K_TEACHER_LSE, s);
+  if (bf16)
+    teacher_lse_kernel<__nv_bfloat16><<<N, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(logits), row_idx, N, V,
+                                                         pitch, lse_t);
+  else
+    teacher_lse_kernel<float><<<N, 256, 0, s>>>(static_cast<const float*>(logits), row_idx, N, V, pitch, lse_t);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const float* part, int S, int n_pad, int N, bool teacher_from_part, const float* lse_ext,
+                           float* saved, cudaStream_t s) {
+  if (N <= 0) return cudaSuccess;
+  LaunchScope scope(K_COMBINE, s);
+  combine_kernel<<<(N + 255) / 256, 256, 0, s>>>(part, S, n_pad, N, teacher_from_part ? 1 : 0, lse_ext, saved);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_scatter_loss(const float* saved, const int32_t* row_idx, int N, long long T, float* loss_tok,
+                                cudaStream_t s) {
+  LaunchScope scope(K_SCATTER_LOSS, s);
+  scatter_loss_kernel<<<static_cast<unsigned>((T + 255) / 256), 256, 0, s>>>(saved, row_idx, N, T, loss_tok);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_reduce(const float* saved, const int32_t* row_idx, int N, int B, int Sm1, int reduction,
+                          float* loss, cudaStream_t s) {
+  LaunchScope scope(K_REDUCE, s);
+  reduce_kernel<<<1, 1024, 0, s>>>(saved, row_idx, N, B, Sm1, reduction, loss);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_row_weights(const float* saved, const int32_t* row_idx, int N, int n_pad, int B, int Sm1,
+                               int reduction, const float* grad_loss, const float* grad_tok, float* rowc,
+                               cudaStream_t s) {
+  LaunchScope scope(K_ROW_WEIGHTS, s);
+  row_weights_kernel<<<(n_pad + 255) / 256, 256, 0, s>>>(saved, row_idx, N, n_pad, B, Sm1, reduction, grad_loss,
+                                                         grad_tok, rowc);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_scatter_dh(const float* dHc, const int32_t* row_idx, int N, long long T, int H, float* dH_s,
+                              cudaStream_t s) {
+  LaunchScope scope(K_SCATTER_DH, s);
+  const long long blocks = T < 65535 * 8 ? T : 65535 * 8;
+  scatter_dh_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(dHc, row_idx, N, T, H, dH_s);
+  return cudaGetLastError();
+}
+
+}  // namespace rkl

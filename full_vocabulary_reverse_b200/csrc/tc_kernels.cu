@@ -1,0 +1,738 @@
+// tc_kernels.cu -- tcgen05 (5th-generation tensor core) kernels of the loss.
+//
+// fused_kernel<NG, DZ>   S3 / S6: per 128-row tile of the compacted rows,
+//   stream 128-wide vocab tiles of the LM head(s) through TMA -> shared memory
+//   -> tcgen05.mma -> TMEM, and reduce each tile in the epilogue without ever
+//   writing logits to global memory.
+//     NG = 2: hidden-state payload, z_s = h_s W_s^T and z_t = h_t W_t^T in two
+//             TMEM accumulators ("feat(mopd): add full-vocabulary on-policy
+//             distillation", NeMo RL PR #3978, payload bullet 1).
+//     NG = 1: logits payload, z_s from the tensor core, z_t read from the
+//             shipped teacher logits (payload bullet 2).
+//     DZ = false: online per-row statistics m_s, sum e^(z_s-m_s),
+//             A = sum e^(z_s-m_s)(z_s-z_t), m_t, sum e^(z_t-m_t) for one vocab
+//             split -> L = A/S_s - lse_s + lse_t after the splits are merged.
+//     DZ = true: the shared backward of the same page's first implementation
+//             note, dL/dz_s = g p_s ((z_s - z_t) + lse_t - lse_s - L), written
+//             as a bf16 [N, cw] chunk for the gradient GEMMs.
+//
+// grad_kernel  S7: grouped persistent GEMM over one vocab chunk,
+//     dW_s[chunk] = dz^T hc_s  and  dHc += dz W_s[chunk]
+//   (chain rule through z_s = h_s W_s^T), fp32 accumulators in TMEM,
+//   TMA store / TMA reduce-add epilogue.
+//
+// Warp roles (192 threads): warp 0 = TMA producer, warp 1 = MMA issuer,
+// warps 2..5 = epilogue (warp w reads TMEM lanes 32*(w%4) .. +31, i.e. one
+// tile row per thread).  Warp 2 also allocates / frees TMEM.  TMEM holds two
+// accumulator slots so the epilogue of tile i overlaps the MMAs of tile i+1.
+#include <cuda_bf16.h>
+
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace rkl {
+
+__device__ int g_dev_err = 0;
+
+namespace {
+
+constexpr int kThreads = 192;
+constexpr int kStgBoxBytes = 4096;  // one 32-row staging box per epilogue warp
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+__device__ __forceinline__ void raise_abort(volatile int* abort_flag, int bit) {
+  atomicOr(&g_dev_err, bit);
+  *abort_flag = 1;
+}
+
+template <int NG>
+struct FusedCfg {
+  static constexpr int A_BYTES = kBM * kBK * 2;
+  static constexpr int B_BYTES = kBN * kBK * 2;
+  static constexpr int STAGE_BYTES = NG * (A_BYTES + B_BYTES);
+  static constexpr int STAGES = NG == 2 ? 3 : 6;
+  static constexpr int ACC_COLS = NG * kBN;
+  static constexpr int TMEM_COLS = 2 * ACC_COLS;
+};
+
+// Bytes: 1024 alignment slack + stages + epilogue staging + barriers.
+template <int NG, bool DZ>
+constexpr size_t fused_smem() {
+  return 1024 + size_t(FusedCfg<NG>::STAGES) * FusedCfg<NG>::STAGE_BYTES + (DZ ? 4 * 2 * kStgBoxBytes : 0) + 256;
+}
+
+// ---- online statistics of one 32-column chunk (all columns valid)
+struct RowStats {
+  float m_s, S_s, A, m_t, S_t;
+};
+
+__device__ __forceinline__ void stats_chunk(RowStats& st, const float* zs, const float* zt) {
+  float cm_s = zs[0], cm_t = zt[0];
+#pragma unroll
+  for (int j = 1; j < 32; ++j) {
+    cm_s = fmaxf(cm_s, zs[j]);
+    cm_t = fmaxf(cm_t, zt[j]);
+  }
+  const float nm_s = fmaxf(st.m_s, cm_s), nm_t = fmaxf(st.m_t, cm_t);
+  const float a_s = ex2((st.m_s - nm_s) * kLog2e), a_t = ex2((st.m_t - nm_t) * kLog2e);
+  st.S_s *= a_s;
+  st.A *= a_s;
+  st.S_t *= a_t;
+  st.m_s = nm_s;
+  st.m_t = nm_t;
+  const float ms2 = nm_s * kLog2e, mt2 = nm_t * kLog2e;
+  float s0 = 0.f, s1 = 0.f, t0 = 0.f, t1 = 0.f, q0 = 0.f, q1 = 0.f;
+#pragma unroll
+  for (int j = 0; j < 32; j += 2) {
+    const float e0 = ex2(fmaf(zs[j], kLog2e, -ms2));
+    const float f0 = ex2(fmaf(zt[j], kLog2e, -mt2));
+    const float e1 = ex2(fmaf(zs[j + 1], kLog2e, -ms2));
+    const float f1 = ex2(fmaf(zt[j + 1], kLog2e, -mt2));
+    s0 += e0;
+    t0 += f0;
+    q0 = fmaf(e0, zs[j] - zt[j], q0);
+    s1 += e1;
+    t1 += f1;
+    q1 = fmaf(e1, zs[j + 1] - zt[j + 1], q1);
+  }
+  st.S_s += s0 + s1;
+  st.S_t += t0 + t1;
+  st.A += q0 + q1;
+}
+
+// Same for a chunk whose first nv (< 32) columns are inside the vocabulary
+// (fully unrolled with predicates so that zs / zt stay in registers).
+__device__ __forceinline__ void stats_chunk_tail(RowStats& st, const float* zs, const float* zt, int nv) {
+  float cm_s = -INFINITY, cm_t = -INFINITY;
+#pragma unroll
+  for (int j = 0; j < 32; ++j)
+    if (j < nv) {
+      cm_s = fmaxf(cm_s, zs[j]);
+      cm_t = fmaxf(cm_t, zt[j]);
+    }
+  const float nm_s = fmaxf(st.m_s, cm_s), nm_t = fmaxf(st.m_t, cm_t);
+  const float a_s = ex2((st.m_s - nm_s) * kLog2e), a_t = ex2((st.m_t - nm_t) * kLog2e);
+  st.S_s *= a_s;
+  st.A *= a_s;
+  st.S_t *= a_t;
+  st.m_s = nm_s;
+  st.m_t = nm_t;
+  const float ms2 = nm_s * kLog2e, mt2 = nm_t * kLog2e;
+#pragma unroll
+  for (int j = 0; j < 32; ++j)
+    if (j < nv) {
+      const float e = ex2(fmaf(zs[j], kLog2e, -ms2));
+      const float f = ex2(fmaf(zt[j], kLog2e, -mt2));
+      st.S_s += e;
+      st.S_t += f;
+      st.A = fmaf(e, zs[j] - zt[j], st.A);
+    }
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+__device__ __forceinline__ uint4 ldg_nc_v4(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
+}  // namespace
+
+// ============================================================================
+// Fused forward-statistics / dz kernel.
+// ============================================================================
+template <int NG, bool DZ>
+__global__ void __launch_bounds__(kThreads, 1) fused_kernel(const __grid_constant__ FusedArgs p) {
+  using Cfg = FusedCfg<NG>;
+  constexpr int STAGES = Cfg::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* stg = smem + STAGES * Cfg::STAGE_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(stg + (DZ ? 4 * 2 * kStgBoxBytes : 0));
+  uint64_t* full = bars;
+  uint64_t* empty = bars + STAGES;
+  uint64_t* acc_full = bars + 2 * STAGES;
+  uint64_t* acc_empty = acc_full + 2;
+  uint64_t* tear = acc_empty + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(tear + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // Work range of this CTA: items u in [u0, u1), u -> (m-tile u / IT, vocab
+  // tile vt_base + u % IT).
+  int u0, u1, split = 0;
+  if (!DZ) {
+    const int mt = blockIdx.x;
+    split = blockIdx.y;
+    const int vb = static_cast<int>((static_cast<long long>(split) * p.IT) / p.S);
+    const int ve = static_cast<int>((static_cast<long long>(split + 1) * p.IT) / p.S);
+    u0 = mt * p.IT + vb;
+    u1 = mt * p.IT + ve;
+  } else {
+    u0 = static_cast<int>((static_cast<long long>(blockIdx.x) * p.items_total) / gridDim.x);
+    u1 = static_cast<int>((static_cast<long long>(blockIdx.x + 1) * p.items_total) / gridDim.x);
+  }
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < STAGES; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], 4);
+    }
+    mbar_init(tear, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 2) {
+    tmem_alloc(tmem_holder, Cfg::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&p.tm_as);
+      tma_prefetch_desc(&p.tm_bs);
+      if (NG == 2) {
+        tma_prefetch_desc(&p.tm_at);
+        tma_prefetch_desc(&p.tm_bt);
+      }
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t armed = 0;  // bit i: stage i has been armed at least once
+      uint32_t last_par = 0;
+      bool ok = true;
+      for (int u = u0; u < u1 && ok; ++u) {
+        const int m0 = (u / p.IT) * kBM;
+        const int v0 = (p.vt_base + u % p.IT) * kBN;
+        for (int kb = 0; kb < p.KB; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) {
+            raise_abort(abort_flag, ERR_WAIT_TMA_EMPTY);
+            ok = false;
+            break;
+          }
+          uint8_t* sa = smem + stage * Cfg::STAGE_BYTES;
+          mbar_arrive_expect_tx(&full[stage], Cfg::STAGE_BYTES);
+          tma_load_2d(sa, &p.tm_as, &full[stage], kb * kBK, m0);
+          tma_load_2d(sa + Cfg::A_BYTES, &p.tm_bs, &full[stage], kb * kBK, v0);
+          if (NG == 2) {
+            tma_load_2d(sa + 2 * Cfg::A_BYTES, &p.tm_at, &full[stage], kb * kBK, m0);
+            tma_load_2d(sa + 2 * Cfg::A_BYTES + Cfg::B_BYTES, &p.tm_bt, &full[stage], kb * kBK, v0);
+          }
+          armed |= 1u << stage;
+          last_par = (last_par & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      // Drain: every armed stage's last phase must have landed before exit.
+      for (int i = 0; i < STAGES; ++i)
+        if (armed & (1u << i)) {
+          volatile int never = 0;
+          if (!mbar_wait(&full[i], (last_par >> i) & 1, &never)) atomicOr(&g_dev_err, ERR_WAIT_TEARDOWN);
+        }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16(kBM, kBN, 0, 0);
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      int it = 0;
+      for (int u = u0; u < u1 && ok; ++u, ++it) {
+        const int acc = it & 1;
+        const uint32_t ap = (it >> 1) & 1;
+        if (!mbar_wait(&acc_empty[acc], ap ^ 1, abort_flag)) {
+          raise_abort(abort_flag, ERR_WAIT_ACC_EMPTY);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_s = tmem_base + acc * Cfg::ACC_COLS;
+        const uint32_t d_t = d_s + kBN;
+        for (int kb = 0; kb < p.KB; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag)) {
+            raise_abort(abort_flag, ERR_WAIT_TMA_FULL);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + stage * Cfg::STAGE_BYTES);
+#pragma unroll
+          for (int k = 0; k < kBK / 16; ++k) {
+            const uint32_t acc_flag = (kb | k) != 0;
+            umma_bf16(d_s, sdesc_sw128(sa + 32 * k, 16, 1024), sdesc_sw128(sa + Cfg::A_BYTES + 32 * k, 16, 1024),
+                      idesc, acc_flag);
+            if (NG == 2)
+              umma_bf16(d_t, sdesc_sw128(sa + 2 * Cfg::A_BYTES + 32 * k, 16, 1024),
+                        sdesc_sw128(sa + 2 * Cfg::A_BYTES + Cfg::B_BYTES + 32 * k, 16, 1024), idesc, acc_flag);
+          }
+          umma_commit(&empty[stage]);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (ok) umma_commit(&acc_full[acc]);
+      }
+      // All issued MMAs must finish before TMEM is released.
+      umma_commit(tear);
+      volatile int never = 0;
+      if (!mbar_wait(tear, 0, &never)) atomicOr(&g_dev_err, ERR_WAIT_TEARDOWN);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
+    RowStats st{-INFINITY, 0.f, 0.f, -INFINITY, 0.f};
+    int cur_mt = -1;
+    float lse2 = 0.f, cst = 0.f, g = 0.f;
+    const uint16_t* trow = nullptr;
+    int box = 0;
+    int it = 0;
+    for (int u = u0; u < u1; ++u, ++it) {
+      const int mt = u / p.IT;
+      const int m0 = mt * kBM;
+      const int v0 = (p.vt_base + u % p.IT) * kBN;
+      if (mt != cur_mt) {
+        cur_mt = mt;
+        const int r = m0 + row;
+        if (DZ) {
+          lse2 = p.rowc[r];
+          cst = p.rowc[p.n_pad + r];
+          g = p.rowc[2 * p.n_pad + r];
+        }
+        if (NG == 1) {
+          trow = nullptr;
+          if (r < p.N) {
+            const long long tr = p.teacher_rows ? p.teacher_rows[r] : r;
+            trow = p.teacher + tr * p.teacher_pitch;
+          }
+        }
+      }
+      // Teacher logits of this row for the tile (logits payload): 128 bf16.
+      uint4 tv[NG == 1 ? 16 : 1];
+      if (NG == 1) {
+        if (trow != nullptr) {
+          const uint16_t* src = trow + v0;
+          const int nvalid = p.V - v0;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            if (i * 8 < nvalid)
+              tv[i] = ldg_nc_v4(src + i * 8);
+            else
+              tv[i] = make_uint4(0, 0, 0, 0);
+          }
+          // warm L2 for the next tile of this row
+          if (u + 1 < u1 && (u + 1) / p.IT == mt) {
+            const int nv0 = (p.vt_base + (u + 1) % p.IT) * kBN;
+            if (nv0 < p.V) prefetch_l2(trow + nv0);
+            if (nv0 + 64 < p.V) prefetch_l2(trow + nv0 + 64);
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) tv[i] = make_uint4(0, 0, 0, 0);
+        }
+      }
+      const int acc = it & 1;
+      const uint32_t ap = (it >> 1) & 1;
+      bool ok = mbar_wait(&acc_full[acc], ap, abort_flag);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) {
+        if (lane == 0) raise_abort(abort_flag, ERR_WAIT_ACC_FULL);
+        break;
+      }
+      tc_fence_after();
+      const uint32_t tb = tmem_base + lane_off + acc * Cfg::ACC_COLS;
+#pragma unroll
+      for (int c = 0; c < kBN / 32; ++c) {
+        float zs[32], zt[32];
+        tmem_ld_32x32(tb + c * 32, zs);
+        if (NG == 2) tmem_ld_32x32(tb + kBN + c * 32, zt);
+        tmem_wait_ld();
+        if (c == kBN / 32 - 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc_empty[acc]);
+        }
+        if (NG == 1) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const uint4 w = tv[c * 4 + i];
+            zt[8 * i + 0] = bf16_lo(w.x);
+            zt[8 * i + 1] = bf16_hi(w.x);
+            zt[8 * i + 2] = bf16_lo(w.y);
+            zt[8 * i + 3] = bf16_hi(w.y);
+            zt[8 * i + 4] = bf16_lo(w.z);
+            zt[8 * i + 5] = bf16_hi(w.z);
+            zt[8 * i + 6] = bf16_lo(w.w);
+            zt[8 * i + 7] = bf16_hi(w.w);
+          }
+        }
+        if (!DZ) {
+          const int nv = p.V - (v0 + c * 32);
+          if (nv >= 32)
+            stats_chunk(st, zs, zt);
+          else if (nv > 0)
+            stats_chunk_tail(st, zs, zt, nv);
+        } else {
+          // dz = g * p_s * ((z_s - z_t) + cst); columns past the chunk end are
+          // clipped by the TMA store.
+          uint32_t pk[16];
+#pragma unroll
+          for (int j = 0; j < 32; j += 2) {
+            const float p0 = ex2(fmaf(zs[j], kLog2e, -lse2));
+            const float p1 = ex2(fmaf(zs[j + 1], kLog2e, -lse2));
+            const float d0 = g * p0 * ((zs[j] - zt[j]) + cst);
+            const float d1 = g * p1 * ((zs[j + 1] - zt[j + 1]) + cst);
+            pk[j / 2] = pack_bf16x2(d0, d1);
+          }
+          uint8_t* buf = stg + (q * 2 + (box & 1)) * kStgBoxBytes;
+          if ((c & 1) == 0) {
+            if (lane == 0) bulk_wait_read<1>();
+            __syncwarp();
+          }
+          const uint32_t rbase = smem_u32(buf) + lane * 128;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int chunk16 = (c & 1) * 4 + i;
+            st_shared_v4(rbase + ((chunk16 ^ (lane & 7)) << 4), pk[4 * i], pk[4 * i + 1], pk[4 * i + 2],
+                         pk[4 * i + 3]);
+          }
+          if (c & 1) {
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&p.tm_dz, buf, v0 - p.chunk_v0 + (c - 1) * 32, m0 + q * 32);
+              bulk_commit();
+            }
+            ++box;
+          }
+        }
+      }
+    }
+    if (!DZ) {
+      if (u1 > u0) {
+        float* base = p.part + static_cast<size_t>(split) * 5 * p.n_pad + (u0 / p.IT) * kBM + row;
+        base[0] = st.m_s;
+        base[p.n_pad] = st.S_s;
+        base[2 * p.n_pad] = st.A;
+        base[3 * p.n_pad] = st.m_t;
+        base[4 * p.n_pad] = st.S_t;
+      }
+    } else {
+      if (lane == 0) bulk_wait<0>();
+      __syncwarp();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+  }
+}
+
+// ============================================================================
+// Grouped gradient GEMM: dW_s tiles (A = dz^T, MN-major; B = hc_s, MN-major)
+// then dH tiles (A = dz, K-major; B = W_s, MN-major).  128 x 256 tiles.
+// ============================================================================
+namespace {
+constexpr int kGA = kBM * kBK * 2;       // 16 KB
+constexpr int kGB = kGradBN * kBK * 2;   // 32 KB
+constexpr int kGStage = kGA + kGB;       // 48 KB
+constexpr int kGStages = 4;
+constexpr int kGTmemCols = 2 * kGradBN;  // 512
+}  // namespace
+
+__global__ void __launch_bounds__(kThreads, 1) grad_kernel(const __grid_constant__ GradArgs p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* stg = smem + kGStages * kGStage;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(stg + 4 * 2 * kStgBoxBytes);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + kGStages;
+  uint64_t* acc_full = bars + 2 * kGStages;
+  uint64_t* acc_empty = acc_full + 2;
+  uint64_t* tear = acc_empty + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(tear + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_tiles = p.nW + p.nH;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kGStages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], 4);
+    }
+    mbar_init(tear, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 2) {
+    tmem_alloc(tmem_holder, kGTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tma_prefetch_desc(&p.tm_dz_k);
+      tma_prefetch_desc(&p.tm_dz_mn);
+      tma_prefetch_desc(&p.tm_hs_mn);
+      tma_prefetch_desc(&p.tm_ws_mn);
+      int stage = 0;
+      uint32_t phase = 0, armed = 0, last_par = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+        const bool is_w = t < p.nW;
+        const int tt = is_w ? t : t - p.nW;
+        const int mtile = is_w ? tt % p.MTW : tt % p.MTH;
+        const int n0 = (is_w ? tt / p.MTW : tt / p.MTH) * kGradBN;
+        const int KB = is_w ? p.KBW : p.KBH;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) {
+            raise_abort(abort_flag, ERR_WAIT_TMA_EMPTY);
+            ok = false;
+            break;
+          }
+          uint8_t* sa = smem + stage * kGStage;
+          uint8_t* sb = sa + kGA;
+          mbar_arrive_expect_tx(&full[stage], kGStage);
+          if (is_w) {
+            // A = dz^T: two 64-wide vocab blocks x 64 rows (K)
+            tma_load_2d(sa, &p.tm_dz_mn, &full[stage], mtile * kBM, kb * kBK);
+            tma_load_2d(sa + kGA / 2, &p.tm_dz_mn, &full[stage], mtile * kBM + 64, kb * kBK);
+#pragma unroll
+            for (int i = 0; i < kGradBN / 64; ++i)
+              tma_load_2d(sb + i * (kGB / 4), &p.tm_hs_mn, &full[stage], n0 + 64 * i, kb * kBK);
+          } else {
+            tma_load_2d(sa, &p.tm_dz_k, &full[stage], kb * kBK, mtile * kBM);
+#pragma unroll
+            for (int i = 0; i < kGradBN / 64; ++i)
+              tma_load_2d(sb + i * (kGB / 4), &p.tm_ws_mn, &full[stage], n0 + 64 * i, p.cv0 + kb * kBK);
+          }
+          armed |= 1u << stage;
+          last_par = (last_par & ~(1u << stage)) | (phase << stage);
+          if (++stage == kGStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      for (int i = 0; i < kGStages; ++i)
+        if (armed & (1u << i)) {
+          volatile int never = 0;
+          if (!mbar_wait(&full[i], (last_par >> i) & 1, &never)) atomicOr(&g_dev_err, ERR_WAIT_TEARDOWN);
+        }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc_w = idesc_bf16(kBM, kGradBN, 1, 1);
+      constexpr uint32_t idesc_h = idesc_bf16(kBM, kGradBN, 0, 1);
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      int it = 0;
+      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++it) {
+        const bool is_w = t < p.nW;
+        const int KB = is_w ? p.KBW : p.KBH;
+        const int acc = it & 1;
+        const uint32_t ap = (it >> 1) & 1;
+        if (!mbar_wait(&acc_empty[acc], ap ^ 1, abort_flag)) {
+          raise_abort(abort_flag, ERR_WAIT_ACC_EMPTY);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d = tmem_base + acc * kGradBN;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag)) {
+            raise_abort(abort_flag, ERR_WAIT_TMA_FULL);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + stage * kGStage);
+          const uint32_t sb = sa + kGA;
+#pragma unroll
+          for (int k = 0; k < kBK / 16; ++k) {
+            const uint32_t acc_flag = (kb | k) != 0;
+            if (is_w)
+              umma_bf16(d, sdesc_sw128(sa + 2048 * k, kGA / 2, 1024), sdesc_sw128(sb + 2048 * k, kGB / 4, 1024),
+                        idesc_w, acc_flag);
+            else
+              umma_bf16(d, sdesc_sw128(sa + 32 * k, 16, 1024), sdesc_sw128(sb + 2048 * k, kGB / 4, 1024), idesc_h,
+                        acc_flag);
+          }
+          umma_commit(&empty[stage]);
+          if (++stage == kGStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (ok) umma_commit(&acc_full[acc]);
+      }
+      umma_commit(tear);
+      volatile int never = 0;
+      if (!mbar_wait(tear, 0, &never)) atomicOr(&g_dev_err, ERR_WAIT_TEARDOWN);
+    }
+  } else {
+    const int q = warp & 3;
+    const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
+    int box = 0;
+    int it = 0;
+    for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++it) {
+      const bool is_w = t < p.nW;
+      const int tt = is_w ? t : t - p.nW;
+      const int mtile = is_w ? tt % p.MTW : tt % p.MTH;
+      const int n0 = (is_w ? tt / p.MTW : tt / p.MTH) * kGradBN;
+      const int acc = it & 1;
+      const uint32_t ap = (it >> 1) & 1;
+      bool ok = mbar_wait(&acc_full[acc], ap, abort_flag);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) {
+        if (lane == 0) raise_abort(abort_flag, ERR_WAIT_ACC_FULL);
+        break;
+      }
+      tc_fence_after();
+      const uint32_t tb = tmem_base + lane_off + acc * kGradBN;
+      const int row0 = is_w ? p.cv0 + mtile * kBM + q * 32 : mtile * kBM + q * 32;
+#pragma unroll 1
+      for (int c = 0; c < kGradBN / 32; ++c) {
+        float v[32];
+        tmem_ld_32x32(tb + c * 32, v);
+        tmem_wait_ld();
+        if (c == kGradBN / 32 - 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc_empty[acc]);
+        }
+        uint8_t* buf = stg + (q * 2 + (box & 1)) * kStgBoxBytes;
+        if (lane == 0) bulk_wait_read<1>();
+        __syncwarp();
+        const uint32_t rbase = smem_u32(buf) + lane * 128;
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          st_shared_v4(rbase + ((i ^ (lane & 7)) << 4), __float_as_uint(v[4 * i]), __float_as_uint(v[4 * i + 1]),
+                       __float_as_uint(v[4 * i + 2]), __float_as_uint(v[4 * i + 3]));
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          if (is_w)
+            tma_store_2d(&p.tm_dw, buf, n0 + c * 32, row0);
+          else if (p.dh_accumulate)
+            tma_reduce_add_2d(&p.tm_dh, buf, n0 + c * 32, row0);
+          else
+            tma_store_2d(&p.tm_dh, buf, n0 + c * 32, row0);
+          bulk_commit();
+        }
+        ++box;
+      }
+    }
+    if (lane == 0) bulk_wait<0>();
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kGTmemCols);
+  }
+}
+
+// ============================================================================
+// Host launchers
+// ============================================================================
+size_t fused_smem_bytes(int ng, bool dz) {
+  if (ng == 2) return dz ? fused_smem<2, true>() : fused_smem<2, false>();
+  return dz ? fused_smem<1, true>() : fused_smem<1, false>();
+}
+
+size_t grad_smem_bytes() { return 1024 + size_t(kGStages) * kGStage + 4 * 2 * kStgBoxBytes + 256; }
+
+cudaError_t tc_setup(int /*device*/) {
+  cudaError_t e;
+  if ((e = cudaFuncSetAttribute(fused_kernel<2, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)fused_smem<2, false>())) != cudaSuccess)
+    return e;
+  if ((e = cudaFuncSetAttribute(fused_kernel<2, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)fused_smem<2, true>())) != cudaSuccess)
+    return e;
+  if ((e = cudaFuncSetAttribute(fused_kernel<1, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)fused_smem<1, false>())) != cudaSuccess)
+    return e;
+  if ((e = cudaFuncSetAttribute(fused_kernel<1, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)fused_smem<1, true>())) != cudaSuccess)
+    return e;
+  return cudaFuncSetAttribute(grad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)grad_smem_bytes());
+}
+
+cudaError_t launch_fused(int ng, bool dz, const FusedArgs& a, dim3 grid, cudaStream_t s) {
+  const size_t smem = fused_smem_bytes(ng, dz);
+  const int id = ng == 2 ? (dz ? K_DZ_DUAL_TC : K_FWD_DUAL_TC) : (dz ? K_DZ_SINGLE_TC : K_FWD_SINGLE_TC);
+  LaunchScope scope(id, s);
+  if (ng == 2) {
+    if (dz)
+      fused_kernel<2, true><<<grid, kThreads, smem, s>>>(a);
+    else
+      fused_kernel<2, false><<<grid, kThreads, smem, s>>>(a);
+  } else {
+    if (dz)
+      fused_kernel<1, true><<<grid, kThreads, smem, s>>>(a);
+    else
+      fused_kernel<1, false><<<grid, kThreads, smem, s>>>(a);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_grad(const GradArgs& a, int grid, cudaStream_t s) {
+  LaunchScope scope(K_GRAD_TC, s);
+  grad_kernel<<<grid, kThreads, grad_smem_bytes(), s>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t read_and_clear_device_error(int* code) {
+  int v = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(&v, g_dev_err, sizeof(int));
+  if (e != cudaSuccess) return e;
+  *code = v;
+  if (v != 0) {
+    const int zero = 0;
+    e = cudaMemcpyToSymbol(g_dev_err, &zero, sizeof(int));
+  }
+  return e;
+}
+
+}  // namespace rkl
