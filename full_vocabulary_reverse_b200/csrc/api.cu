@@ -145,37 +145,41 @@ static rkl_status make_map(CUtensorMap* m, const void* ptr, bool f32, uint64_t i
 }
 
 // ------------------------------------------------------------------ plan
-constexpr int kVcBf16 = 4096;  // vocab chunk of the backward (multiple of kBN)
+constexpr int kVcBf16 = 8192;  // vocab chunk of the backward (multiple of kBN)
 constexpr int kVcF32 = 1024;
+constexpr int kSimtSplits = 37;
 
 struct Plan {
-  int n_pad = 0, es = 2, S = 1, VT = 1, Vc = 0;
-  size_t off_hcs = 0, off_hct = 0, off_part = 0, off_rowc = 0, off_lse = 0, off_dz = 0, off_dh = 0, total = 0;
+  int n_pad = 0, es = 2, S = 1, VT = 1, Vc = 0, nchunks = 1;
+  size_t off_hcs = 0, off_hct = 0, off_part = 0, off_rowc = 0, off_lse = 0, off_dz = 0, off_dh = 0, off_cnt = 0,
+         total = 0;
 };
 
 static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// Workspace layout.  S = number of partial-statistics groups of the forward:
+// groups of kGroupTiles vocab tiles on the tensor-core path, kSimtSplits
+// vocab splits on the fp32 path -- both depend on V only.
 static Plan make_plan(rkl_payload payload, rkl_dtype dtype, int64_t n_max, int64_t H, int64_t V) {
   Plan p;
   const bool bf16 = dtype == RKL_BF16;
-  const int tile_m = bf16 ? kBM : kSimtBN;
   const int tile_v = bf16 ? kBN : kSimtBN;
   p.es = bf16 ? 2 : 4;
   const int64_t n = n_max < 1 ? 1 : n_max;
   p.n_pad = static_cast<int>(((n + kBM - 1) / kBM) * kBM);  // multiple of both tile heights
-  (void)tile_m;
   p.VT = static_cast<int>((V + tile_v - 1) / tile_v);
-  p.S = p.VT < kSplits ? p.VT : kSplits;
+  p.S = bf16 ? (p.VT + kGroupTiles - 1) / kGroupTiles : (p.VT < kSimtSplits ? p.VT : kSimtSplits);
   const int vc = bf16 ? kVcBf16 : kVcF32;
   const int64_t vround = ((V + kBN - 1) / kBN) * kBN;
   p.Vc = static_cast<int>(vround < vc ? vround : vc);
+  p.nchunks = static_cast<int>((V + p.Vc - 1) / p.Vc);
   size_t off = 256;  // header
   p.off_hcs = off;
   off = align256(off + size_t(p.n_pad) * H * p.es);
   p.off_hct = off;
   if (payload == RKL_PAYLOAD_HIDDEN) off = align256(off + size_t(p.n_pad) * H * p.es);
   p.off_part = off;
-  off = align256(off + size_t(kSplits) * 5 * p.n_pad * sizeof(float));
+  off = align256(off + size_t(p.S) * 5 * p.n_pad * sizeof(float));
   p.off_rowc = off;
   off = align256(off + size_t(3) * p.n_pad * sizeof(float));
   p.off_lse = off;
@@ -184,6 +188,8 @@ static Plan make_plan(rkl_payload payload, rkl_dtype dtype, int64_t n_max, int64
   off = align256(off + size_t(p.n_pad) * p.Vc * p.es);
   p.off_dh = off;
   off = align256(off + size_t(p.n_pad) * H * sizeof(float));
+  p.off_cnt = off;
+  off = align256(off + size_t(p.nchunks) * sizeof(int));
   p.total = off;
   return p;
 }
@@ -285,9 +291,12 @@ static rkl_status forward_impl(rkl_payload payload, const void* h_s, const void*
       a.KB = static_cast<int>(H / kBK);
       a.IT = pl.VT;
       a.vt_base = 0;
-      a.S = pl.S;
+      a.GT = kGroupTiles;
+      a.G = pl.S;
       const int MT = (N + kBM - 1) / kBM;
-      RKL_CUDA(launch_fused(ng, false, a, dim3(MT, pl.S), s));
+      a.MT = MT;
+      a.units_total = MT * a.G;
+      RKL_CUDA(launch_fused(ng, false, a, dim3(a.units_total < sms ? a.units_total : sms), s));
     } else {
       SimtArgs a;
       memset(&a, 0, sizeof(a));
@@ -390,7 +399,10 @@ static rkl_status backward_impl(rkl_payload payload, const void* h_s, const void
     a.V = static_cast<int>(V);
     a.KB = static_cast<int>(H / kBK);
     const int MT = (N + kBM - 1) / kBM;
+    a.MT = MT;
 
+    int* counters = reinterpret_cast<int*>(ws_at(workspace, pl.off_cnt));
+    RKL_CUDA(cudaMemsetAsync(counters, 0, size_t(nchunks) * sizeof(int), s));
     GradArgs g;
     memset(&g, 0, sizeof(g));
     RKL_TRY(make_map(&g.tm_hs_mn, as, false, H, N, H * 2, 64, 64));
@@ -400,7 +412,7 @@ static rkl_status backward_impl(rkl_payload payload, const void* h_s, const void
     g.N = N;
     g.H = static_cast<int>(H);
     g.NT = static_cast<int>(H / kGradBN) + (H % kGradBN ? 1 : 0);
-    g.MTH = MT;
+    g.MTH = (N + 2 * kBM - 1) / (2 * kBM);  // 256-row pair tiles
     g.nH = g.MTH * g.NT;
     g.KBW = (N + kBK - 1) / kBK;
 
@@ -412,20 +424,23 @@ static rkl_status backward_impl(rkl_payload payload, const void* h_s, const void
       a.IT = (cw + kBN - 1) / kBN;
       a.vt_base = cv0 / kBN;
       a.chunk_v0 = cv0;
-      a.items_total = MT * a.IT;
-      const int grid = a.items_total < sms ? a.items_total : sms;
+      a.GT = 1;
+      a.G = a.IT;
+      a.units_total = MT * a.IT;
+      const int grid = a.units_total < sms ? a.units_total : sms;
       RKL_CUDA(launch_fused(ng, true, a, dim3(grid), s));
       // S7: dW_s[chunk] = dz^T hc_s and dHc (+)= dz W_s[chunk].
       RKL_TRY(make_map(&g.tm_dz_k, dz, false, cw, N, size_t(pl.Vc) * 2, 64, 128));
       RKL_TRY(make_map(&g.tm_dz_mn, dz, false, cw, N, size_t(pl.Vc) * 2, 64, 64));
       g.cw = cw;
       g.cv0 = cv0;
-      g.MTW = (cw + kBM - 1) / kBM;
+      g.MTW = (cw + 2 * kBM - 1) / (2 * kBM);
       g.nW = g.MTW * g.NT;
       g.KBH = (cw + kBK - 1) / kBK;
       g.dh_accumulate = c > 0;
-      const int tiles = g.nW + g.nH;
-      RKL_CUDA(launch_grad(g, tiles < sms ? tiles : sms, s));
+      g.tile_counter = counters + c;
+      const int pairs = g.nW + g.nH;
+      RKL_CUDA(launch_grad(g, 2 * pairs < sms ? 2 * pairs : sms, s));
     }
   } else {
     SimtArgs a;

@@ -45,7 +45,7 @@ constexpr int kBM = 128;       // rows per tile (TMEM lanes)
 constexpr int kBN = 128;       // vocab columns per fused tile
 constexpr int kBK = 64;        // K per pipeline stage (128 B of bf16)
 constexpr int kGradBN = 256;   // H columns per gradient tile
-constexpr int kSplits = 37;    // vocab splits of the forward (148 SMs = 4 x 37)
+constexpr int kGroupTiles = 8;  // vocab tiles per forward statistics group
 
 // ---------------------------------------------------------------- tcgen05
 struct FusedArgs {
@@ -55,13 +55,15 @@ struct FusedArgs {
   const uint16_t* teacher;           // logits payload: teacher logits [T, V] bf16
   const int32_t* teacher_rows;       // logits payload: row_idx (nullptr = identity)
   long long teacher_pitch;           // elements per teacher row
-  float* part;                       // stats: [S][5][n_pad]
+  float* part;                       // stats: [G][5][n_pad]
   const float* rowc;                 // dz: [3][n_pad]: lse_s*log2e, cst, g
   int N, n_pad, H, V, KB;
   int IT;                            // vocab tiles per m-tile covered by this launch
   int vt_base;                       // first vocab tile of this launch
-  int S;                             // stats: number of vocab splits
-  int items_total;                   // dz: m-tiles * IT
+  int GT;                            // vocab tiles per unit (group)
+  int G;                             // units per m-tile = ceil(IT / GT)
+  int MT;                            // m-tiles (128 rows each)
+  int units_total;                   // MT * G
   int chunk_v0;                      // dz: first vocab column of the chunk
 };
 
@@ -72,6 +74,7 @@ struct GradArgs {
   CUtensorMap tm_ws_mn;   // W_s [V, H] bf16 as MN-major B (box {64, 64})
   CUtensorMap tm_dw;      // dW_s [V, H] fp32 output (box {32, 32})
   CUtensorMap tm_dh;      // dHc [N, H] fp32 output (box {32, 32})
+  int* tile_counter;      // zeroed before the launch; dynamic tile scheduler
   int N, H, cw, cv0;
   int MTW, MTH, NT, nW, nH, KBW, KBH;
   int dh_accumulate;

@@ -230,37 +230,51 @@ __global__ void __launch_bounds__(256) teacher_lse_kernel(const T* __restrict__ 
 }
 
 // --------------------------------------------------------------------- S4
-// Merge the per-split statistics of each row in split order; L = A/S_s -
-// lse_s + lse_t.  The student and teacher statistics go through the same
-// operations, so teacher == student gives L = 0 exactly.
-__global__ void combine_kernel(const float* __restrict__ part, int S, int n_pad, int N, int teacher_from_part,
-                               const float* __restrict__ lse_ext, float* __restrict__ saved) {
-  const int k = blockIdx.x * blockDim.x + threadIdx.x;
+// Merge the per-group statistics of each row; L = A/S_s - lse_s + lse_t.
+// One warp per row: lane l merges groups l, l+32, ..., then a fixed
+// butterfly merges the lanes (same order on every run).  Student and teacher
+// statistics go through identical operations, so teacher == student gives
+// L = 0 exactly.
+struct Stat3 {
+  float m, S, A;
+};
+
+__device__ __forceinline__ void merge3(Stat3& a, const Stat3& b) {
+  const float nm = fmaxf(a.m, b.m);
+  if (nm == -INFINITY) return;
+  const float ea = expf(a.m - nm), eb = expf(b.m - nm);
+  a.S = a.S * ea + b.S * eb;
+  a.A = a.A * ea + b.A * eb;
+  a.m = nm;
+}
+
+__global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ part, int S, int n_pad, int N,
+                                                      int teacher_from_part, const float* __restrict__ lse_ext,
+                                                      float* __restrict__ saved) {
+  const int lane = threadIdx.x & 31;
+  const int k = blockIdx.x * 8 + (threadIdx.x >> 5);
   if (k >= N) return;
-  float m_s = -INFINITY, S_s = 0.f, A = 0.f, m_t = -INFINITY, S_t = 0.f;
-  for (int s = 0; s < S; ++s) {
-    const float* b = part + static_cast<size_t>(s) * 5 * n_pad + k;
-    const float ms = b[0], Ss = b[n_pad], As = b[2 * n_pad], mt = b[3 * n_pad], St = b[4 * n_pad];
-    if (ms != -INFINITY) {
-      const float nm = fmaxf(m_s, ms);
-      const float a = expf(m_s - nm), c = expf(ms - nm);
-      S_s = S_s * a + Ss * c;
-      A = A * a + As * c;
-      m_s = nm;
-    }
-    if (teacher_from_part && mt != -INFINITY) {
-      const float nm = fmaxf(m_t, mt);
-      const float a = expf(m_t - nm), c = expf(mt - nm);
-      S_t = S_t * a + St * c;
-      m_t = nm;
-    }
+  Stat3 s{-INFINITY, 0.f, 0.f}, t{-INFINITY, 0.f, 0.f};
+  for (int g = lane; g < S; g += 32) {
+    const float* b = part + static_cast<size_t>(g) * 5 * n_pad + k;
+    merge3(s, Stat3{b[0], b[n_pad], b[2 * n_pad]});
+    if (teacher_from_part) merge3(t, Stat3{b[3 * n_pad], b[4 * n_pad], 0.f});
   }
-  const float lse_s = m_s + logf(S_s);
-  const float lse_t = teacher_from_part ? m_t + logf(S_t) : lse_ext[k];
-  const float L = A / S_s - lse_s + lse_t;
-  saved[3 * k + 0] = lse_s;
-  saved[3 * k + 1] = lse_t;
-  saved[3 * k + 2] = L;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    merge3(s, Stat3{__shfl_xor_sync(0xffffffffu, s.m, o), __shfl_xor_sync(0xffffffffu, s.S, o),
+                    __shfl_xor_sync(0xffffffffu, s.A, o)});
+    merge3(t, Stat3{__shfl_xor_sync(0xffffffffu, t.m, o), __shfl_xor_sync(0xffffffffu, t.S, o),
+                    __shfl_xor_sync(0xffffffffu, t.A, o)});
+  }
+  if (lane == 0) {
+    const float lse_s = s.m + logf(s.S);
+    const float lse_t = teacher_from_part ? t.m + logf(t.S) : lse_ext[k];
+    const float L = s.A / s.S - lse_s + lse_t;
+    saved[3 * k + 0] = lse_s;
+    saved[3 * k + 1] = lse_t;
+    saved[3 * k + 2] = L;
+  }
 }
 
 // loss_tok[t] = L of t if t is trainable else exactly 0.
@@ -425,7 +439,7 @@ cudaError_t launch_combine(const float* part, int S, int n_pad, int N, bool teac
                            float* saved, cudaStream_t s) {
   if (N <= 0) return cudaSuccess;
   LaunchScope scope(K_COMBINE, s);
-  combine_kernel<<<(N + 255) / 256, 256, 0, s>>>(part, S, n_pad, N, teacher_from_part ? 1 : 0, lse_ext, saved);
+  combine_kernel<<<(N + 7) / 8, 256, 0, s>>>(part, S, n_pad, N, teacher_from_part ? 1 : 0, lse_ext, saved);
   return cudaGetLastError();
 }
 

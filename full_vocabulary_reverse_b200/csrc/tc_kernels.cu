@@ -170,20 +170,14 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const __grid_constan
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // Work range of this CTA: items u in [u0, u1), u -> (m-tile u / IT, vocab
-  // tile vt_base + u % IT).
-  int u0, u1, split = 0;
-  if (!DZ) {
-    const int mt = blockIdx.x;
-    split = blockIdx.y;
-    const int vb = static_cast<int>((static_cast<long long>(split) * p.IT) / p.S);
-    const int ve = static_cast<int>((static_cast<long long>(split + 1) * p.IT) / p.S);
-    u0 = mt * p.IT + vb;
-    u1 = mt * p.IT + ve;
-  } else {
-    u0 = static_cast<int>((static_cast<long long>(blockIdx.x) * p.items_total) / gridDim.x);
-    u1 = static_cast<int>((static_cast<long long>(blockIdx.x + 1) * p.items_total) / gridDim.x);
-  }
+  // Work of this CTA: units u = blockIdx.x, blockIdx.x + gridDim.x, ...
+  // Unit u = (m-tile u % MT, vocab group u / MT); group g covers the vocab
+  // tiles vt_base + [g*GT, min(g*GT + GT, IT)).  With the m-tile as the fast
+  // index, the CTAs running at any moment share a few vocab groups, so each
+  // LM-head tile is fetched from HBM once and re-served from L2 to every
+  // m-tile.  Forward statistics are flushed per unit, so their grouping
+  // depends on V only -- never on N or on the grid -- and a row's loss does
+  // not depend on the rest of the batch.
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < STAGES; ++i) {
@@ -221,28 +215,32 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const __grid_constan
       uint32_t armed = 0;  // bit i: stage i has been armed at least once
       uint32_t last_par = 0;
       bool ok = true;
-      for (int u = u0; u < u1 && ok; ++u) {
-        const int m0 = (u / p.IT) * kBM;
-        const int v0 = (p.vt_base + u % p.IT) * kBN;
-        for (int kb = 0; kb < p.KB; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) {
-            raise_abort(abort_flag, ERR_WAIT_TMA_EMPTY);
-            ok = false;
-            break;
-          }
-          uint8_t* sa = smem + stage * Cfg::STAGE_BYTES;
-          mbar_arrive_expect_tx(&full[stage], Cfg::STAGE_BYTES);
-          tma_load_2d(sa, &p.tm_as, &full[stage], kb * kBK, m0);
-          tma_load_2d(sa + Cfg::A_BYTES, &p.tm_bs, &full[stage], kb * kBK, v0);
-          if (NG == 2) {
-            tma_load_2d(sa + 2 * Cfg::A_BYTES, &p.tm_at, &full[stage], kb * kBK, m0);
-            tma_load_2d(sa + 2 * Cfg::A_BYTES + Cfg::B_BYTES, &p.tm_bt, &full[stage], kb * kBK, v0);
-          }
-          armed |= 1u << stage;
-          last_par = (last_par & ~(1u << stage)) | (phase << stage);
-          if (++stage == STAGES) {
-            stage = 0;
-            phase ^= 1;
+      for (int u = blockIdx.x; u < p.units_total && ok; u += gridDim.x) {
+        const int m0 = (u % p.MT) * kBM;
+        const int g = u / p.MT;
+        const int vt_end = min(g * p.GT + p.GT, p.IT);
+        for (int vt = g * p.GT; vt < vt_end && ok; ++vt) {
+          const int v0 = (p.vt_base + vt) * kBN;
+          for (int kb = 0; kb < p.KB; ++kb) {
+            if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) {
+              raise_abort(abort_flag, ERR_WAIT_TMA_EMPTY);
+              ok = false;
+              break;
+            }
+            uint8_t* sa = smem + stage * Cfg::STAGE_BYTES;
+            mbar_arrive_expect_tx(&full[stage], Cfg::STAGE_BYTES);
+            tma_load_2d(sa, &p.tm_as, &full[stage], kb * kBK, m0);
+            tma_load_2d(sa + Cfg::A_BYTES, &p.tm_bs, &full[stage], kb * kBK, v0);
+            if (NG == 2) {
+              tma_load_2d(sa + 2 * Cfg::A_BYTES, &p.tm_at, &full[stage], kb * kBK, m0);
+              tma_load_2d(sa + 2 * Cfg::A_BYTES + Cfg::B_BYTES, &p.tm_bt, &full[stage], kb * kBK, v0);
+            }
+            armed |= 1u << stage;
+            last_par = (last_par & ~(1u << stage)) | (phase << stage);
+            if (++stage == STAGES) {
+              stage = 0;
+              phase ^= 1;
+            }
           }
         }
       }
@@ -261,40 +259,45 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const __grid_constan
       uint32_t phase = 0;
       bool ok = true;
       int it = 0;
-      for (int u = u0; u < u1 && ok; ++u, ++it) {
-        const int acc = it & 1;
-        const uint32_t ap = (it >> 1) & 1;
-        if (!mbar_wait(&acc_empty[acc], ap ^ 1, abort_flag)) {
-          raise_abort(abort_flag, ERR_WAIT_ACC_EMPTY);
-          break;
-        }
-        tc_fence_after();
-        const uint32_t d_s = tmem_base + acc * Cfg::ACC_COLS;
-        const uint32_t d_t = d_s + kBN;
-        for (int kb = 0; kb < p.KB; ++kb) {
-          if (!mbar_wait(&full[stage], phase, abort_flag)) {
-            raise_abort(abort_flag, ERR_WAIT_TMA_FULL);
+      for (int u = blockIdx.x; u < p.units_total && ok; u += gridDim.x) {
+        const int g = u / p.MT;
+        const int vt_end = min(g * p.GT + p.GT, p.IT);
+        for (int vt = g * p.GT; vt < vt_end && ok; ++vt, ++it) {
+          const int acc = it & 1;
+          const uint32_t ap = (it >> 1) & 1;
+          if (!mbar_wait(&acc_empty[acc], ap ^ 1, abort_flag)) {
+            raise_abort(abort_flag, ERR_WAIT_ACC_EMPTY);
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t sa = smem_u32(smem + stage * Cfg::STAGE_BYTES);
+          const uint32_t d_s = tmem_base + acc * Cfg::ACC_COLS;
+          const uint32_t d_t = d_s + kBN;
+          for (int kb = 0; kb < p.KB; ++kb) {
+            if (!mbar_wait(&full[stage], phase, abort_flag)) {
+              raise_abort(abort_flag, ERR_WAIT_TMA_FULL);
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t sa = smem_u32(smem + stage * Cfg::STAGE_BYTES);
 #pragma unroll
-          for (int k = 0; k < kBK / 16; ++k) {
-            const uint32_t acc_flag = (kb | k) != 0;
-            umma_bf16(d_s, sdesc_sw128(sa + 32 * k, 16, 1024), sdesc_sw128(sa + Cfg::A_BYTES + 32 * k, 16, 1024),
-                      idesc, acc_flag);
-            if (NG == 2)
-              umma_bf16(d_t, sdesc_sw128(sa + 2 * Cfg::A_BYTES + 32 * k, 16, 1024),
-                        sdesc_sw128(sa + 2 * Cfg::A_BYTES + Cfg::B_BYTES + 32 * k, 16, 1024), idesc, acc_flag);
+            for (int k = 0; k < kBK / 16; ++k) {
+              const uint32_t acc_flag = (kb | k) != 0;
+              umma_bf16(d_s, sdesc_sw128(sa + 32 * k, 16, 1024),
+                        sdesc_sw128(sa + Cfg::A_BYTES + 32 * k, 16, 1024), idesc, acc_flag);
+              if (NG == 2)
+                umma_bf16(d_t, sdesc_sw128(sa + 2 * Cfg::A_BYTES + 32 * k, 16, 1024),
+                          sdesc_sw128(sa + 2 * Cfg::A_BYTES + Cfg::B_BYTES + 32 * k, 16, 1024), idesc, acc_flag);
+            }
+            umma_commit(&empty[stage]);
+            if (++stage == STAGES) {
+              stage = 0;
+              phase ^= 1;
+            }
           }
-          umma_commit(&empty[stage]);
-          if (++stage == STAGES) {
-            stage = 0;
-            phase ^= 1;
-          }
+          if (ok) umma_commit(&acc_full[acc]);
         }
-        if (ok) umma_commit(&acc_full[acc]);
       }
       // All issued MMAs must finish before TMEM is released.
       umma_commit(tear);
@@ -306,23 +309,24 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const __grid_constan
     const int q = warp & 3;
     const int row = q * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
-    RowStats st{-INFINITY, 0.f, 0.f, -INFINITY, 0.f};
     int cur_mt = -1;
-    float lse2 = 0.f, cst = 0.f, g = 0.f;
+    float lse2 = 0.f, cst = 0.f, g_row = 0.f;
     const uint16_t* trow = nullptr;
     int box = 0;
     int it = 0;
-    for (int u = u0; u < u1; ++u, ++it) {
-      const int mt = u / p.IT;
+    bool ok = true;
+    for (int u = blockIdx.x; u < p.units_total && ok; u += gridDim.x) {
+      const int mt = u % p.MT;
       const int m0 = mt * kBM;
-      const int v0 = (p.vt_base + u % p.IT) * kBN;
+      const int g = u / p.MT;
+      const int vt_end = min(g * p.GT + p.GT, p.IT);
       if (mt != cur_mt) {
         cur_mt = mt;
         const int r = m0 + row;
         if (DZ) {
           lse2 = p.rowc[r];
           cst = p.rowc[p.n_pad + r];
-          g = p.rowc[2 * p.n_pad + r];
+          g_row = p.rowc[2 * p.n_pad + r];
         }
         if (NG == 1) {
           trow = nullptr;
@@ -332,117 +336,121 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const __grid_constan
           }
         }
       }
-      // Teacher logits of this row for the tile (logits payload): 128 bf16.
-      uint4 tv[NG == 1 ? 16 : 1];
-      if (NG == 1) {
-        if (trow != nullptr) {
-          const uint16_t* src = trow + v0;
-          const int nvalid = p.V - v0;
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            if (i * 8 < nvalid)
-              tv[i] = ldg_nc_v4(src + i * 8);
-            else
-              tv[i] = make_uint4(0, 0, 0, 0);
-          }
-          // warm L2 for the next tile of this row
-          if (u + 1 < u1 && (u + 1) / p.IT == mt) {
-            const int nv0 = (p.vt_base + (u + 1) % p.IT) * kBN;
-            if (nv0 < p.V) prefetch_l2(trow + nv0);
-            if (nv0 + 64 < p.V) prefetch_l2(trow + nv0 + 64);
-          }
-        } else {
-#pragma unroll
-          for (int i = 0; i < 16; ++i) tv[i] = make_uint4(0, 0, 0, 0);
-        }
-      }
-      const int acc = it & 1;
-      const uint32_t ap = (it >> 1) & 1;
-      bool ok = mbar_wait(&acc_full[acc], ap, abort_flag);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) {
-        if (lane == 0) raise_abort(abort_flag, ERR_WAIT_ACC_FULL);
-        break;
-      }
-      tc_fence_after();
-      const uint32_t tb = tmem_base + lane_off + acc * Cfg::ACC_COLS;
-#pragma unroll
-      for (int c = 0; c < kBN / 32; ++c) {
-        float zs[32], zt[32];
-        tmem_ld_32x32(tb + c * 32, zs);
-        if (NG == 2) tmem_ld_32x32(tb + kBN + c * 32, zt);
-        tmem_wait_ld();
-        if (c == kBN / 32 - 1) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&acc_empty[acc]);
-        }
+      RowStats st{-INFINITY, 0.f, 0.f, -INFINITY, 0.f};
+      for (int vt = g * p.GT; vt < vt_end; ++vt, ++it) {
+        const int v0 = (p.vt_base + vt) * kBN;
+        // Teacher logits of this row for the tile (logits payload): 128 bf16.
+        uint4 tv[NG == 1 ? 16 : 1];
         if (NG == 1) {
+          if (trow != nullptr) {
+            const uint16_t* src = trow + v0;
+            const int nvalid = p.V - v0;
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const uint4 w = tv[c * 4 + i];
-            zt[8 * i + 0] = bf16_lo(w.x);
-            zt[8 * i + 1] = bf16_hi(w.x);
-            zt[8 * i + 2] = bf16_lo(w.y);
-            zt[8 * i + 3] = bf16_hi(w.y);
-            zt[8 * i + 4] = bf16_lo(w.z);
-            zt[8 * i + 5] = bf16_hi(w.z);
-            zt[8 * i + 6] = bf16_lo(w.w);
-            zt[8 * i + 7] = bf16_hi(w.w);
+            for (int i = 0; i < 16; ++i) {
+              if (i * 8 < nvalid)
+                tv[i] = ldg_nc_v4(src + i * 8);
+              else
+                tv[i] = make_uint4(0, 0, 0, 0);
+            }
+            // warm L2 for the next tile of this row
+            const int nv0 = v0 + kBN;
+            if (vt + 1 < vt_end) {
+              if (nv0 < p.V) prefetch_l2(trow + nv0);
+              if (nv0 + 64 < p.V) prefetch_l2(trow + nv0 + 64);
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) tv[i] = make_uint4(0, 0, 0, 0);
           }
         }
-        if (!DZ) {
-          const int nv = p.V - (v0 + c * 32);
-          if (nv >= 32)
-            stats_chunk(st, zs, zt);
-          else if (nv > 0)
-            stats_chunk_tail(st, zs, zt, nv);
-        } else {
-          // dz = g * p_s * ((z_s - z_t) + cst); columns past the chunk end are
-          // clipped by the TMA store.
-          uint32_t pk[16];
+        const int acc = it & 1;
+        const uint32_t ap = (it >> 1) & 1;
+        bool w_ok = mbar_wait(&acc_full[acc], ap, abort_flag);
+        w_ok = __all_sync(0xffffffffu, w_ok);
+        if (!w_ok) {
+          if (lane == 0) raise_abort(abort_flag, ERR_WAIT_ACC_FULL);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t tb = tmem_base + lane_off + acc * Cfg::ACC_COLS;
 #pragma unroll
-          for (int j = 0; j < 32; j += 2) {
-            const float p0 = ex2(fmaf(zs[j], kLog2e, -lse2));
-            const float p1 = ex2(fmaf(zs[j + 1], kLog2e, -lse2));
-            const float d0 = g * p0 * ((zs[j] - zt[j]) + cst);
-            const float d1 = g * p1 * ((zs[j + 1] - zt[j + 1]) + cst);
-            pk[j / 2] = pack_bf16x2(d0, d1);
-          }
-          uint8_t* buf = stg + (q * 2 + (box & 1)) * kStgBoxBytes;
-          if ((c & 1) == 0) {
-            if (lane == 0) bulk_wait_read<1>();
+        for (int c = 0; c < kBN / 32; ++c) {
+          float zs[32], zt[32];
+          tmem_ld_32x32(tb + c * 32, zs);
+          if (NG == 2) tmem_ld_32x32(tb + kBN + c * 32, zt);
+          tmem_wait_ld();
+          if (c == kBN / 32 - 1) {
+            tc_fence_before();
             __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[acc]);
           }
-          const uint32_t rbase = smem_u32(buf) + lane * 128;
+          if (NG == 1) {
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int chunk16 = (c & 1) * 4 + i;
-            st_shared_v4(rbase + ((chunk16 ^ (lane & 7)) << 4), pk[4 * i], pk[4 * i + 1], pk[4 * i + 2],
-                         pk[4 * i + 3]);
-          }
-          if (c & 1) {
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-              tma_store_2d(&p.tm_dz, buf, v0 - p.chunk_v0 + (c - 1) * 32, m0 + q * 32);
-              bulk_commit();
+            for (int i = 0; i < 4; ++i) {
+              const uint4 w = tv[c * 4 + i];
+              zt[8 * i + 0] = bf16_lo(w.x);
+              zt[8 * i + 1] = bf16_hi(w.x);
+              zt[8 * i + 2] = bf16_lo(w.y);
+              zt[8 * i + 3] = bf16_hi(w.y);
+              zt[8 * i + 4] = bf16_lo(w.z);
+              zt[8 * i + 5] = bf16_hi(w.z);
+              zt[8 * i + 6] = bf16_lo(w.w);
+              zt[8 * i + 7] = bf16_hi(w.w);
             }
-            ++box;
+          }
+          if (!DZ) {
+            const int nv = p.V - (v0 + c * 32);
+            if (nv >= 32)
+              stats_chunk(st, zs, zt);
+            else if (nv > 0)
+              stats_chunk_tail(st, zs, zt, nv);
+          } else {
+            // dz = g * p_s * ((z_s - z_t) + cst); columns past the chunk end
+            // are clipped by the TMA store.
+            uint32_t pk[16];
+#pragma unroll
+            for (int j = 0; j < 32; j += 2) {
+              const float p0 = ex2(fmaf(zs[j], kLog2e, -lse2));
+              const float p1 = ex2(fmaf(zs[j + 1], kLog2e, -lse2));
+              const float d0 = g_row * p0 * ((zs[j] - zt[j]) + cst);
+              const float d1 = g_row * p1 * ((zs[j + 1] - zt[j + 1]) + cst);
+              pk[j / 2] = pack_bf16x2(d0, d1);
+            }
+            uint8_t* buf = stg + (q * 2 + (box & 1)) * kStgBoxBytes;
+            if ((c & 1) == 0) {
+              if (lane == 0) bulk_wait_read<1>();
+              __syncwarp();
+            }
+            const uint32_t rbase = smem_u32(buf) + lane * 128;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int chunk16 = (c & 1) * 4 + i;
+              st_shared_v4(rbase + ((chunk16 ^ (lane & 7)) << 4), pk[4 * i], pk[4 * i + 1], pk[4 * i + 2],
+                           pk[4 * i + 3]);
+            }
+            if (c & 1) {
+              fence_proxy_async_smem();
+              __syncwarp();
+              if (lane == 0) {
+                tma_store_2d(&p.tm_dz, buf, v0 - p.chunk_v0 + (c - 1) * 32, m0 + q * 32);
+                bulk_commit();
+              }
+              ++box;
+            }
           }
         }
       }
-    }
-    if (!DZ) {
-      if (u1 > u0) {
-        float* base = p.part + static_cast<size_t>(split) * 5 * p.n_pad + (u0 / p.IT) * kBM + row;
+      if (!DZ && ok) {
+        float* base = p.part + static_cast<size_t>(g) * 5 * p.n_pad + m0 + row;
         base[0] = st.m_s;
         base[p.n_pad] = st.S_s;
         base[2 * p.n_pad] = st.A;
         base[3 * p.n_pad] = st.m_t;
         base[4 * p.n_pad] = st.S_t;
       }
-    } else {
+    }
+    if (DZ) {
       if (lane == 0) bulk_wait<0>();
       __syncwarp();
     }
@@ -461,13 +469,24 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const __grid_constan
 // then dH tiles (A = dz, K-major; B = W_s, MN-major).  128 x 256 tiles.
 // ============================================================================
 namespace {
-constexpr int kGA = kBM * kBK * 2;       // 16 KB
-constexpr int kGB = kGradBN * kBK * 2;   // 32 KB
-constexpr int kGStage = kGA + kGB;       // 48 KB
-constexpr int kGStages = 4;
+constexpr int kGA = kBM * kBK * 2;             // 16 KB: this CTA's 128 rows of A
+constexpr int kGB = (kGradBN / 2) * kBK * 2;   // 16 KB: this CTA's half of B
+constexpr int kGStage = kGA + kGB;             // 32 KB
+constexpr int kGStages = 6;
 constexpr int kGTmemCols = 2 * kGradBN;  // 512
+constexpr int kSched = 2;                // tile-index broadcast ring depth
 }  // namespace
 
+// One 2-CTA cluster computes a 256 x 256 tile with tcgen05.mma.cta_group::2:
+// CTA rank r holds rows [128 r, 128 r + 128) of A and columns
+// [128 r, 128 r + 128) of B in its own shared memory, and receives rows
+// [128 r, 128 r + 128) of D in its own TMEM.  Each CTA therefore streams only
+// half of the B operand, halving the L2 -> shared-memory bytes per flop of a
+// single-CTA 128 x 256 tile.  The leader (rank 0) issues the MMAs and owns
+// the operand-full barriers (both CTAs' TMA loads count on them), the
+// accumulator-empty barriers (both CTAs' epilogues arrive) and the tile
+// scheduler (it claims tiles with an atomic counter and writes each index
+// into both CTAs' rings).
 __global__ void __launch_bounds__(kThreads, 1) grad_kernel(const __grid_constant__ GradArgs p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -478,10 +497,15 @@ __global__ void __launch_bounds__(kThreads, 1) grad_kernel(const __grid_constant
   uint64_t* acc_full = bars + 2 * kGStages;
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* tear = acc_empty + 2;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(tear + 1);
+  uint64_t* sched_full = tear + 1;             // [kSched]
+  uint64_t* sched_empty = sched_full + kSched;  // [kSched]
+  int* sched_tile = reinterpret_cast<int*>(sched_empty + kSched);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sched_tile + kSched);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
   const int n_tiles = p.nW + p.nH;
 
   if (threadIdx.x == 0) {
@@ -491,18 +515,22 @@ __global__ void __launch_bounds__(kThreads, 1) grad_kernel(const __grid_constant
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&acc_full[i], 1);
-      mbar_init(&acc_empty[i], 4);
+      mbar_init(&acc_empty[i], 8);  // 4 epilogue warps in each CTA of the pair
+    }
+    for (int i = 0; i < kSched; ++i) {
+      mbar_init(&sched_full[i], 1);
+      mbar_init(&sched_empty[i], 1 + 4 + 1 + 4);  // leader MMA + epilogues, peer producer + epilogues
     }
     mbar_init(tear, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
   if (warp == 2) {
-    tmem_alloc(tmem_holder, kGTmemCols);
-    tmem_relinquish();
+    tmem_alloc_pair(tmem_holder, kGTmemCols);
+    tmem_relinquish_pair();
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
 
@@ -512,36 +540,60 @@ __global__ void __launch_bounds__(kThreads, 1) grad_kernel(const __grid_constant
       tma_prefetch_desc(&p.tm_dz_mn);
       tma_prefetch_desc(&p.tm_hs_mn);
       tma_prefetch_desc(&p.tm_ws_mn);
+      const uint32_t full0 = mapa_shared(smem_u32(full), 0);  // leader's full[0]
       int stage = 0;
       uint32_t phase = 0, armed = 0, last_par = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
-        const bool is_w = t < p.nW;
-        const int tt = is_w ? t : t - p.nW;
-        const int mtile = is_w ? tt % p.MTW : tt % p.MTH;
-        const int n0 = (is_w ? tt / p.MTW : tt / p.MTH) * kGradBN;
-        const int KB = is_w ? p.KBW : p.KBH;
+      for (int i = 0; ok; ++i) {
+        const int slot = i % kSched;
+        const uint32_t sp = (i / kSched) & 1;
+        int t;
+        if (leader) {
+          if (!mbar_wait_cluster(&sched_empty[slot], sp ^ 1, abort_flag)) {
+            raise_abort(abort_flag, ERR_WAIT_AUX);
+            break;
+          }
+          t = atomicAdd(p.tile_counter, 1);
+          if (t >= n_tiles) t = -1;
+          sched_tile[slot] = t;
+          st_cluster_u32(mapa_shared(smem_u32(&sched_tile[slot]), 1), static_cast<uint32_t>(t));
+          mbar_arrive(&sched_full[slot]);
+          mbar_arrive_cluster(mapa_shared(smem_u32(&sched_full[slot]), 1));
+        } else {
+          if (!mbar_wait_cluster(&sched_full[slot], sp, abort_flag)) {
+            raise_abort(abort_flag, ERR_WAIT_AUX);
+            break;
+          }
+          t = sched_tile[slot];
+          mbar_arrive_cluster(mapa_shared(smem_u32(&sched_empty[slot]), 0));
+        }
+        if (t < 0) break;
+        const bool is_h = t < p.nH;
+        const int tt = is_h ? t : t - p.nH;
+        const int m0 = (is_h ? tt % p.MTH : tt % p.MTW) * 2 * kBM + rank * kBM;  // this CTA's A rows
+        const int n0 = (is_h ? tt / p.MTH : tt / p.MTW) * kGradBN + rank * (kGradBN / 2);  // this CTA's B half
+        const int KB = is_h ? p.KBH : p.KBW;
         for (int kb = 0; kb < KB; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) {
+          if (!mbar_wait_cluster(&empty[stage], phase ^ 1, abort_flag)) {
             raise_abort(abort_flag, ERR_WAIT_TMA_EMPTY);
             ok = false;
             break;
           }
           uint8_t* sa = smem + stage * kGStage;
           uint8_t* sb = sa + kGA;
-          mbar_arrive_expect_tx(&full[stage], kGStage);
-          if (is_w) {
-            // A = dz^T: two 64-wide vocab blocks x 64 rows (K)
-            tma_load_2d(sa, &p.tm_dz_mn, &full[stage], mtile * kBM, kb * kBK);
-            tma_load_2d(sa + kGA / 2, &p.tm_dz_mn, &full[stage], mtile * kBM + 64, kb * kBK);
-#pragma unroll
-            for (int i = 0; i < kGradBN / 64; ++i)
-              tma_load_2d(sb + i * (kGB / 4), &p.tm_hs_mn, &full[stage], n0 + 64 * i, kb * kBK);
+          const uint32_t fb = full0 + stage * 8;
+          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * kGStage);
+          if (!is_h) {
+            // A = dz^T: two 64-wide vocab blocks x 64 rows (K); B = hc_s.
+            tma_load_2d_pair(sa, &p.tm_dz_mn, fb, m0, kb * kBK);
+            tma_load_2d_pair(sa + kGA / 2, &p.tm_dz_mn, fb, m0 + 64, kb * kBK);
+            tma_load_2d_pair(sb, &p.tm_hs_mn, fb, n0, kb * kBK);
+            tma_load_2d_pair(sb + kGB / 2, &p.tm_hs_mn, fb, n0 + 64, kb * kBK);
           } else {
-            tma_load_2d(sa, &p.tm_dz_k, &full[stage], kb * kBK, mtile * kBM);
-#pragma unroll
-            for (int i = 0; i < kGradBN / 64; ++i)
-              tma_load_2d(sb + i * (kGB / 4), &p.tm_ws_mn, &full[stage], n0 + 64 * i, p.cv0 + kb * kBK);
+            // A = dz (K-major); B = W_s rows of the chunk.
+            tma_load_2d_pair(sa, &p.tm_dz_k, fb, kb * kBK, m0);
+            tma_load_2d_pair(sb, &p.tm_ws_mn, fb, n0, p.cv0 + kb * kBK);
+            tma_load_2d_pair(sb + kGB / 2, &p.tm_ws_mn, fb, n0 + 64, p.cv0 + kb * kBK);
           }
           armed |= 1u << stage;
           last_par = (last_par & ~(1u << stage)) | (phase << stage);
@@ -551,26 +603,36 @@ __global__ void __launch_bounds__(kThreads, 1) grad_kernel(const __grid_constant
           }
         }
       }
-      for (int i = 0; i < kGStages; ++i)
-        if (armed & (1u << i)) {
-          volatile int never = 0;
-          if (!mbar_wait(&full[i], (last_par >> i) & 1, &never)) atomicOr(&g_dev_err, ERR_WAIT_TEARDOWN);
-        }
+      // The leader's full barriers count both CTAs' loads: drain them there.
+      if (leader)
+        for (int i = 0; i < kGStages; ++i)
+          if (armed & (1u << i)) {
+            volatile int never = 0;
+            if (!mbar_wait(&full[i], (last_par >> i) & 1, &never)) atomicOr(&g_dev_err, ERR_WAIT_TEARDOWN);
+          }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      constexpr uint32_t idesc_w = idesc_bf16(kBM, kGradBN, 1, 1);
-      constexpr uint32_t idesc_h = idesc_bf16(kBM, kGradBN, 0, 1);
+    if (leader && lane == 0) {
+      constexpr uint32_t idesc_w = idesc_bf16(2 * kBM, kGradBN, 1, 1);
+      constexpr uint32_t idesc_h = idesc_bf16(2 * kBM, kGradBN, 0, 1);
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      int it = 0;
-      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++it) {
-        const bool is_w = t < p.nW;
-        const int KB = is_w ? p.KBW : p.KBH;
-        const int acc = it & 1;
-        const uint32_t ap = (it >> 1) & 1;
-        if (!mbar_wait(&acc_empty[acc], ap ^ 1, abort_flag)) {
+      for (int i = 0; ok; ++i) {
+        const int slot = i % kSched;
+        const uint32_t sp = (i / kSched) & 1;
+        if (!mbar_wait(&sched_full[slot], sp, abort_flag)) {
+          raise_abort(abort_flag, ERR_WAIT_AUX);
+          break;
+        }
+        const int t = sched_tile[slot];
+        mbar_arrive(&sched_empty[slot]);
+        if (t < 0) break;
+        const bool is_h = t < p.nH;
+        const int KB = is_h ? p.KBH : p.KBW;
+        const int acc = i & 1;
+        const uint32_t ap = (i >> 1) & 1;
+        if (!mbar_wait_cluster(&acc_empty[acc], ap ^ 1, abort_flag)) {
           raise_abort(abort_flag, ERR_WAIT_ACC_EMPTY);
           break;
         }
@@ -588,38 +650,51 @@ __global__ void __launch_bounds__(kThreads, 1) grad_kernel(const __grid_constant
 #pragma unroll
           for (int k = 0; k < kBK / 16; ++k) {
             const uint32_t acc_flag = (kb | k) != 0;
-            if (is_w)
-              umma_bf16(d, sdesc_sw128(sa + 2048 * k, kGA / 2, 1024), sdesc_sw128(sb + 2048 * k, kGB / 4, 1024),
-                        idesc_w, acc_flag);
+            if (!is_h)
+              umma_bf16_pair(d, sdesc_sw128(sa + 2048 * k, kGA / 2, 1024), sdesc_sw128(sb + 2048 * k, kGB / 2, 1024),
+                             idesc_w, acc_flag);
             else
-              umma_bf16(d, sdesc_sw128(sa + 32 * k, 16, 1024), sdesc_sw128(sb + 2048 * k, kGB / 4, 1024), idesc_h,
-                        acc_flag);
+              umma_bf16_pair(d, sdesc_sw128(sa + 32 * k, 16, 1024), sdesc_sw128(sb + 2048 * k, kGB / 2, 1024),
+                             idesc_h, acc_flag);
           }
-          umma_commit(&empty[stage]);
+          umma_commit_pair(&empty[stage], 0x3);
           if (++stage == kGStages) {
             stage = 0;
             phase ^= 1;
           }
         }
-        if (ok) umma_commit(&acc_full[acc]);
+        if (ok) umma_commit_pair(&acc_full[acc], 0x3);
       }
-      umma_commit(tear);
+      umma_commit_pair(tear, 0x1);
       volatile int never = 0;
       if (!mbar_wait(tear, 0, &never)) atomicOr(&g_dev_err, ERR_WAIT_TEARDOWN);
     }
   } else {
     const int q = warp & 3;
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
+    const uint32_t sched_empty0 = mapa_shared(smem_u32(sched_empty), 0);
+    const uint32_t acc_empty0 = mapa_shared(smem_u32(acc_empty), 0);
     int box = 0;
-    int it = 0;
-    for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++it) {
-      const bool is_w = t < p.nW;
-      const int tt = is_w ? t : t - p.nW;
-      const int mtile = is_w ? tt % p.MTW : tt % p.MTH;
-      const int n0 = (is_w ? tt / p.MTW : tt / p.MTH) * kGradBN;
-      const int acc = it & 1;
-      const uint32_t ap = (it >> 1) & 1;
-      bool ok = mbar_wait(&acc_full[acc], ap, abort_flag);
+    for (int i = 0;; ++i) {
+      const int slot = i % kSched;
+      const uint32_t sp = (i / kSched) & 1;
+      bool ok = mbar_wait_cluster(&sched_full[slot], sp, abort_flag);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) {
+        if (lane == 0) raise_abort(abort_flag, ERR_WAIT_AUX);
+        break;
+      }
+      const int t = sched_tile[slot];
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(sched_empty0 + slot * 8);
+      if (t < 0) break;
+      const bool is_h = t < p.nH;
+      const int tt = is_h ? t : t - p.nH;
+      const int mtile = is_h ? tt % p.MTH : tt % p.MTW;
+      const int n0 = (is_h ? tt / p.MTH : tt / p.MTW) * kGradBN;
+      const int acc = i & 1;
+      const uint32_t ap = (i >> 1) & 1;
+      ok = mbar_wait_cluster(&acc_full[acc], ap, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) {
         if (lane == 0) raise_abort(abort_flag, ERR_WAIT_ACC_FULL);
@@ -627,7 +702,8 @@ __global__ void __launch_bounds__(kThreads, 1) grad_kernel(const __grid_constant
       }
       tc_fence_after();
       const uint32_t tb = tmem_base + lane_off + acc * kGradBN;
-      const int row0 = is_w ? p.cv0 + mtile * kBM + q * 32 : mtile * kBM + q * 32;
+      const int rows = mtile * 2 * kBM + rank * kBM + q * 32;
+      const int row0 = is_h ? rows : p.cv0 + rows;
 #pragma unroll 1
       for (int c = 0; c < kGradBN / 32; ++c) {
         float v[32];
@@ -636,20 +712,20 @@ __global__ void __launch_bounds__(kThreads, 1) grad_kernel(const __grid_constant
         if (c == kGradBN / 32 - 1) {
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&acc_empty[acc]);
+          if (lane == 0) mbar_arrive_cluster(acc_empty0 + acc * 8);
         }
         uint8_t* buf = stg + (q * 2 + (box & 1)) * kStgBoxBytes;
         if (lane == 0) bulk_wait_read<1>();
         __syncwarp();
         const uint32_t rbase = smem_u32(buf) + lane * 128;
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-          st_shared_v4(rbase + ((i ^ (lane & 7)) << 4), __float_as_uint(v[4 * i]), __float_as_uint(v[4 * i + 1]),
-                       __float_as_uint(v[4 * i + 2]), __float_as_uint(v[4 * i + 3]));
+        for (int j = 0; j < 8; ++j)
+          st_shared_v4(rbase + ((j ^ (lane & 7)) << 4), __float_as_uint(v[4 * j]), __float_as_uint(v[4 * j + 1]),
+                       __float_as_uint(v[4 * j + 2]), __float_as_uint(v[4 * j + 3]));
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          if (is_w)
+          if (!is_h)
             tma_store_2d(&p.tm_dw, buf, n0 + c * 32, row0);
           else if (p.dh_accumulate)
             tma_reduce_add_2d(&p.tm_dh, buf, n0 + c * 32, row0);
@@ -664,11 +740,13 @@ __global__ void __launch_bounds__(kThreads, 1) grad_kernel(const __grid_constant
     __syncwarp();
   }
 
+  // Neither CTA may release its TMEM or shared memory while the pair MMAs or
+  // the other CTA can still touch them.
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();
   if (warp == 2) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, kGTmemCols);
+    tmem_dealloc_pair(tmem_base, kGTmemCols);
   }
 }
 
@@ -680,7 +758,7 @@ size_t fused_smem_bytes(int ng, bool dz) {
   return dz ? fused_smem<1, true>() : fused_smem<1, false>();
 }
 
-size_t grad_smem_bytes() { return 1024 + size_t(kGStages) * kGStage + 4 * 2 * kStgBoxBytes + 256; }
+size_t grad_smem_bytes() { return 1024 + size_t(kGStages) * kGStage + 4 * 2 * kStgBoxBytes + 512; }
 
 cudaError_t tc_setup(int /*device*/) {
   cudaError_t e;
@@ -719,8 +797,19 @@ cudaError_t launch_fused(int ng, bool dz, const FusedArgs& a, dim3 grid, cudaStr
 
 cudaError_t launch_grad(const GradArgs& a, int grid, cudaStream_t s) {
   LaunchScope scope(K_GRAD_TC, s);
-  grad_kernel<<<grid, kThreads, grad_smem_bytes(), s>>>(a);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid & ~1);  // whole CTA pairs
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = grad_smem_bytes();
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, grad_kernel, a);
 }
 
 cudaError_t read_and_clear_device_error(int* code) {
