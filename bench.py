@@ -172,6 +172,16 @@ class Problem:
         return N
 
 
+def reduce_over_ranks(ms, tokens, dist, device):
+    """(max over ranks of the device-timed milliseconds, sum over ranks of the tokens)."""
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    n = torch.tensor([float(tokens)], dtype=torch.float64, device=device)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        dist.all_reduce(n, op=dist.ReduceOp.SUM)
+    return float(t[0]), float(n[0])
+
+
 def kernel_profile():
     L = rb.lib()
     out = {}
@@ -302,14 +312,8 @@ def run_gpu(args, rank, world, dist):
     rb._check(L.rkl_profile_enable(0))
     prof = kernel_profile()
     ms = e0.elapsed_time(e1)
-    t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if dist is not None:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_max = float(t[0])
-    n_tot = torch.tensor([float(N * args.steps)], dtype=torch.float64, device=dev)
-    if dist is not None:
-        dist.all_reduce(n_tot)
-    value = float(n_tot[0]) / (ms_max / 1000.0)
+    ms_max, n_tot = reduce_over_ranks(ms, N * args.steps, dist, dev)
+    value = n_tot / (ms_max / 1000.0)
 
     # ---- end to end through the C ABI with host buffers
     h_pin = prob.inp["h_s"].cpu().pin_memory()
@@ -336,10 +340,8 @@ def run_gpu(args, rank, world, dist):
         e2e_step()
     f1.record(stream)
     torch.cuda.synchronize()
-    t2 = torch.tensor([f0.elapsed_time(f1)], dtype=torch.float64, device=dev)
-    if dist is not None:
-        dist.all_reduce(t2, op=dist.ReduceOp.MAX)
-    e2e_value = float(n_tot[0]) / (float(t2[0]) / 1000.0)
+    ms_e2e, _ = reduce_over_ranks(f0.elapsed_time(f1), 0, dist, dev)
+    e2e_value = n_tot / (ms_e2e / 1000.0)
     h2d = h_pin.numel() * h_pin.element_size() + t_pin.numel() * t_pin.element_size() + m_pin.numel()
     d2h = 4 + 4  # loss scalar + N (the compaction count read back to size the launches)
 
