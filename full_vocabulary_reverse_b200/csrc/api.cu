@@ -15,7 +15,7 @@
 #include <string>
 #include <vector>
 
-#include "../../include/rkl.h"
+#include "rkl.h"
 #include "kernels.h"
 
 namespace rkl {
@@ -145,7 +145,7 @@ static rkl_status make_map(CUtensorMap* m, const void* ptr, bool f32, uint64_t i
 }
 
 // ------------------------------------------------------------------ plan
-constexpr int kVcBf16 = 8192;  // vocab chunk of the backward (multiple of kBN)
+constexpr int kVcBf16 = 8192;  // vocab chunk of the backward (multiple of kFBN)
 constexpr int kVcF32 = 1024;
 constexpr int kSimtSplits = 37;
 
@@ -163,14 +163,14 @@ static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 static Plan make_plan(rkl_payload payload, rkl_dtype dtype, int64_t n_max, int64_t H, int64_t V) {
   Plan p;
   const bool bf16 = dtype == RKL_BF16;
-  const int tile_v = bf16 ? kBN : kSimtBN;
+  const int tile_v = bf16 ? kFBN : kSimtBN;
   p.es = bf16 ? 2 : 4;
   const int64_t n = n_max < 1 ? 1 : n_max;
-  p.n_pad = static_cast<int>(((n + kBM - 1) / kBM) * kBM);  // multiple of both tile heights
+  p.n_pad = static_cast<int>(((n + 2 * kBM - 1) / (2 * kBM)) * (2 * kBM));  // whole 256-row pair tiles
   p.VT = static_cast<int>((V + tile_v - 1) / tile_v);
   p.S = bf16 ? (p.VT + kGroupTiles - 1) / kGroupTiles : (p.VT < kSimtSplits ? p.VT : kSimtSplits);
   const int vc = bf16 ? kVcBf16 : kVcF32;
-  const int64_t vround = ((V + kBN - 1) / kBN) * kBN;
+  const int64_t vround = ((V + kFBN - 1) / kFBN) * kFBN;
   p.Vc = static_cast<int>(vround < vc ? vround : vc);
   p.nchunks = static_cast<int>((V + p.Vc - 1) / p.Vc);
   size_t off = 256;  // header
@@ -274,10 +274,10 @@ static rkl_status forward_impl(rkl_payload payload, const void* h_s, const void*
       FusedArgs a;
       memset(&a, 0, sizeof(a));
       RKL_TRY(make_map(&a.tm_as, as, false, H, N, H * 2, kBK, kBM));
-      RKL_TRY(make_map(&a.tm_bs, W_s, false, H, V, H * 2, kBK, kBN));
+      RKL_TRY(make_map(&a.tm_bs, W_s, false, H, V, H * 2, kBK, kFBN / 2));
       if (hidden) {
         RKL_TRY(make_map(&a.tm_at, at, false, H, N, H * 2, kBK, kBM));
-        RKL_TRY(make_map(&a.tm_bt, W_t, false, H, V, H * 2, kBK, kBN));
+        RKL_TRY(make_map(&a.tm_bt, W_t, false, H, V, H * 2, kBK, kFBN / 2));
       } else {
         a.teacher = static_cast<const uint16_t*>(teacher);
         a.teacher_rows = N < T ? row_idx : nullptr;
@@ -293,10 +293,10 @@ static rkl_status forward_impl(rkl_payload payload, const void* h_s, const void*
       a.vt_base = 0;
       a.GT = kGroupTiles;
       a.G = pl.S;
-      const int MT = (N + kBM - 1) / kBM;
+      const int MT = (N + 2 * kBM - 1) / (2 * kBM);
       a.MT = MT;
       a.units_total = MT * a.G;
-      RKL_CUDA(launch_fused(ng, false, a, dim3(a.units_total < sms ? a.units_total : sms), s));
+      RKL_CUDA(launch_fused(ng, false, a, 2 * a.units_total < sms ? 2 * a.units_total : sms, s));
     } else {
       SimtArgs a;
       memset(&a, 0, sizeof(a));
@@ -383,10 +383,10 @@ static rkl_status backward_impl(rkl_payload payload, const void* h_s, const void
     FusedArgs a;
     memset(&a, 0, sizeof(a));
     RKL_TRY(make_map(&a.tm_as, as, false, H, N, H * 2, kBK, kBM));
-    RKL_TRY(make_map(&a.tm_bs, W_s, false, H, V, H * 2, kBK, kBN));
+    RKL_TRY(make_map(&a.tm_bs, W_s, false, H, V, H * 2, kBK, kFBN / 2));
     if (hidden) {
       RKL_TRY(make_map(&a.tm_at, at, false, H, N, H * 2, kBK, kBM));
-      RKL_TRY(make_map(&a.tm_bt, W_t, false, H, V, H * 2, kBK, kBN));
+      RKL_TRY(make_map(&a.tm_bt, W_t, false, H, V, H * 2, kBK, kFBN / 2));
     } else {
       a.teacher = static_cast<const uint16_t*>(teacher);
       a.teacher_rows = N < T ? row_idx : nullptr;
@@ -398,7 +398,7 @@ static rkl_status backward_impl(rkl_payload payload, const void* h_s, const void
     a.H = static_cast<int>(H);
     a.V = static_cast<int>(V);
     a.KB = static_cast<int>(H / kBK);
-    const int MT = (N + kBM - 1) / kBM;
+    const int MT = (N + 2 * kBM - 1) / (2 * kBM);
     a.MT = MT;
 
     int* counters = reinterpret_cast<int*>(ws_at(workspace, pl.off_cnt));
@@ -421,14 +421,13 @@ static rkl_status backward_impl(rkl_payload payload, const void* h_s, const void
       const int cw = static_cast<int>((V - cv0) < pl.Vc ? (V - cv0) : pl.Vc);
       // S6: recompute the logits of this chunk and write dz (bf16) [N, cw].
       RKL_TRY(make_map(&a.tm_dz, dz, false, cw, N, size_t(pl.Vc) * 2, 64, 32));
-      a.IT = (cw + kBN - 1) / kBN;
-      a.vt_base = cv0 / kBN;
+      a.IT = (cw + kFBN - 1) / kFBN;
+      a.vt_base = cv0 / kFBN;
       a.chunk_v0 = cv0;
       a.GT = 1;
       a.G = a.IT;
       a.units_total = MT * a.IT;
-      const int grid = a.units_total < sms ? a.units_total : sms;
-      RKL_CUDA(launch_fused(ng, true, a, dim3(grid), s));
+      RKL_CUDA(launch_fused(ng, true, a, 2 * a.units_total < sms ? 2 * a.units_total : sms, s));
       // S7: dW_s[chunk] = dz^T hc_s and dHc (+)= dz W_s[chunk].
       RKL_TRY(make_map(&g.tm_dz_k, dz, false, cw, N, size_t(pl.Vc) * 2, 64, 128));
       RKL_TRY(make_map(&g.tm_dz_mn, dz, false, cw, N, size_t(pl.Vc) * 2, 64, 64));

@@ -42,14 +42,15 @@ struct LaunchScope {
 };
 
 constexpr int kBM = 128;       // rows per tile (TMEM lanes)
-constexpr int kBN = 128;       // vocab columns per fused tile
+constexpr int kBN = 128;       // vocab tile granularity of the statistics groups / chunks
+constexpr int kFBN = 256;      // vocab columns per fused pair tile
 constexpr int kBK = 64;        // K per pipeline stage (128 B of bf16)
 constexpr int kGradBN = 256;   // H columns per gradient tile
-constexpr int kGroupTiles = 8;  // vocab tiles per forward statistics group
+constexpr int kGroupTiles = 4;  // 256-column vocab tiles per forward statistics group (1024 columns)
 
 // ---------------------------------------------------------------- tcgen05
 struct FusedArgs {
-  // operand maps (bf16, 128-byte swizzle, box {64, 128})
+  // operand maps (bf16, 128-byte swizzle): A box {64, 128}, B box {64, 128}
   CUtensorMap tm_as, tm_at, tm_bs, tm_bt;
   CUtensorMap tm_dz;                 // dz chunk output [N, cw] bf16, box {64, 32}
   const uint16_t* teacher;           // logits payload: teacher logits [T, V] bf16
@@ -58,11 +59,11 @@ struct FusedArgs {
   float* part;                       // stats: [G][5][n_pad]
   const float* rowc;                 // dz: [3][n_pad]: lse_s*log2e, cst, g
   int N, n_pad, H, V, KB;
-  int IT;                            // vocab tiles per m-tile covered by this launch
-  int vt_base;                       // first vocab tile of this launch
+  int IT;                            // 256-column vocab tiles per row tile in this launch
+  int vt_base;                       // first 256-column vocab tile of this launch
   int GT;                            // vocab tiles per unit (group)
   int G;                             // units per m-tile = ceil(IT / GT)
-  int MT;                            // m-tiles (128 rows each)
+  int MT;                            // row tiles (256 rows each, one per CTA pair)
   int units_total;                   // MT * G
   int chunk_v0;                      // dz: first vocab column of the chunk
 };
@@ -83,7 +84,7 @@ struct GradArgs {
 size_t fused_smem_bytes(int ng, bool dz);
 size_t grad_smem_bytes();
 cudaError_t tc_setup(int device);  // one-time cudaFuncSetAttribute per device
-cudaError_t launch_fused(int ng, bool dz, const FusedArgs& a, dim3 grid, cudaStream_t s);
+cudaError_t launch_fused(int ng, bool dz, const FusedArgs& a, int grid, cudaStream_t s);  // grid: CTAs, even
 cudaError_t launch_grad(const GradArgs& a, int grid, cudaStream_t s);
 cudaError_t read_and_clear_device_error(int* code);
 

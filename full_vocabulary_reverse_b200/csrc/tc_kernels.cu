@@ -48,14 +48,20 @@ __device__ __forceinline__ void raise_abort(volatile int* abort_flag, int bit) {
   *abort_flag = 1;
 }
 
+// Per-CTA shared-memory layout of one pipeline stage of the pair kernel: this
+// CTA's 128 rows of A (the compacted hidden rows of z_s and, for NG = 2, of
+// z_t) and its half (128 rows) of the 256-row LM-head tile(s).  TMEM holds
+// z_s (and z_t) for 256 vocab columns: one accumulator slot of 512 columns
+// for NG = 2, two slots of 256 for NG = 1.
 template <int NG>
 struct FusedCfg {
-  static constexpr int A_BYTES = kBM * kBK * 2;
-  static constexpr int B_BYTES = kBN * kBK * 2;
+  static constexpr int A_BYTES = kBM * kBK * 2;          // 16 KB
+  static constexpr int B_BYTES = (kFBN / 2) * kBK * 2;   // 16 KB
   static constexpr int STAGE_BYTES = NG * (A_BYTES + B_BYTES);
   static constexpr int STAGES = NG == 2 ? 3 : 6;
-  static constexpr int ACC_COLS = NG * kBN;
-  static constexpr int TMEM_COLS = 2 * ACC_COLS;
+  static constexpr int ACC_COLS = NG * kFBN;
+  static constexpr int NUM_ACC = NG == 2 ? 1 : 2;
+  static constexpr int TMEM_COLS = NUM_ACC * ACC_COLS;   // 512
 };
 
 // Bytes: 1024 alignment slack + stages + epilogue staging + barriers.
@@ -150,7 +156,18 @@ __device__ __forceinline__ void prefetch_l2(const void* p) {
 }  // namespace
 
 // ============================================================================
-// Fused forward-statistics / dz kernel.
+// Fused forward-statistics / dz kernel on CTA pairs.
+//
+// A 2-CTA cluster computes a 256-row x 256-column tile of z_s (and z_t) with
+// tcgen05.mma.cta_group::2 (M = 256, N = 256): CTA rank r stages rows
+// [128 r, 128 r + 128) of the compacted hidden rows and rows
+// [128 r, 128 r + 128) of the 256-row LM-head tile, and receives its 128 rows
+// of the logits in its own TMEM.  Each staged hidden-row tile feeds 256
+// vocab columns, which keeps the operand bytes per flop -- the limit of
+// these kernels -- at 1/3 below a 128-column tile.  The
+// leader (rank 0) issues the MMAs and owns the operand-full and
+// accumulator-empty barriers; both CTAs run the same producer and epilogue
+// code on their own rows.
 // ============================================================================
 template <int NG, bool DZ>
 __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const __grid_constant__ FusedArgs p) {
@@ -169,15 +186,19 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const __grid_constan
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  static_assert(Cfg::TMEM_COLS <= 512, "TMEM has 512 columns");
 
-  // Work of this CTA: units u = blockIdx.x, blockIdx.x + gridDim.x, ...
-  // Unit u = (m-tile u % MT, vocab group u / MT); group g covers the vocab
-  // tiles vt_base + [g*GT, min(g*GT + GT, IT)).  With the m-tile as the fast
-  // index, the CTAs running at any moment share a few vocab groups, so each
-  // LM-head tile is fetched from HBM once and re-served from L2 to every
-  // m-tile.  Forward statistics are flushed per unit, so their grouping
-  // depends on V only -- never on N or on the grid -- and a row's loss does
-  // not depend on the rest of the batch.
+  // Work of this pair: units u = pair, pair + npairs, ...
+  // Unit u = (256-row tile u % MT, vocab group u / MT); group g covers the
+  // vocab tiles vt_base + [g*GT, min(g*GT + GT, IT)).  With the row tile as
+  // the fast index, the pairs running at any moment share a few vocab groups,
+  // so each LM-head tile is fetched from HBM once and re-served from L2 to
+  // every row tile.  Forward statistics are flushed per unit, so their
+  // grouping depends on V only -- never on N or on the grid -- and a row's
+  // loss does not depend on the rest of the batch.
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < STAGES; ++i) {
@@ -186,18 +207,18 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const __grid_constan
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&acc_full[i], 1);
-      mbar_init(&acc_empty[i], 4);
+      mbar_init(&acc_empty[i], 8);  // 4 epilogue warps in each CTA of the pair
     }
     mbar_init(tear, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
   if (warp == 2) {
-    tmem_alloc(tmem_holder, Cfg::TMEM_COLS);
-    tmem_relinquish();
+    tmem_alloc_pair(tmem_holder, Cfg::TMEM_COLS);
+    tmem_relinquish_pair();
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
 
@@ -210,30 +231,32 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const __grid_constan
         tma_prefetch_desc(&p.tm_at);
         tma_prefetch_desc(&p.tm_bt);
       }
+      const uint32_t full0 = mapa_shared(smem_u32(full), 0);  // leader's full[0]
       int stage = 0;
       uint32_t phase = 0;
       uint32_t armed = 0;  // bit i: stage i has been armed at least once
       uint32_t last_par = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < p.units_total && ok; u += gridDim.x) {
-        const int m0 = (u % p.MT) * kBM;
+      for (int u = pair; u < p.units_total && ok; u += npairs) {
+        const int m0 = (u % p.MT) * 2 * kBM + rank * kBM;
         const int g = u / p.MT;
         const int vt_end = min(g * p.GT + p.GT, p.IT);
         for (int vt = g * p.GT; vt < vt_end && ok; ++vt) {
-          const int v0 = (p.vt_base + vt) * kBN;
+          const int v0 = (p.vt_base + vt) * kFBN + rank * (kFBN / 2);
           for (int kb = 0; kb < p.KB; ++kb) {
-            if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) {
+            if (!mbar_wait_cluster(&empty[stage], phase ^ 1, abort_flag)) {
               raise_abort(abort_flag, ERR_WAIT_TMA_EMPTY);
               ok = false;
               break;
             }
             uint8_t* sa = smem + stage * Cfg::STAGE_BYTES;
-            mbar_arrive_expect_tx(&full[stage], Cfg::STAGE_BYTES);
-            tma_load_2d(sa, &p.tm_as, &full[stage], kb * kBK, m0);
-            tma_load_2d(sa + Cfg::A_BYTES, &p.tm_bs, &full[stage], kb * kBK, v0);
+            const uint32_t fb = full0 + stage * 8;
+            if (leader) mbar_arrive_expect_tx(&full[stage], 2 * Cfg::STAGE_BYTES);
+            tma_load_2d_pair(sa, &p.tm_as, fb, kb * kBK, m0);
+            tma_load_2d_pair(sa + Cfg::A_BYTES, &p.tm_bs, fb, kb * kBK, v0);
             if (NG == 2) {
-              tma_load_2d(sa + 2 * Cfg::A_BYTES, &p.tm_at, &full[stage], kb * kBK, m0);
-              tma_load_2d(sa + 2 * Cfg::A_BYTES + Cfg::B_BYTES, &p.tm_bt, &full[stage], kb * kBK, v0);
+              tma_load_2d_pair(sa + Cfg::A_BYTES + Cfg::B_BYTES, &p.tm_at, fb, kb * kBK, m0);
+              tma_load_2d_pair(sa + 2 * Cfg::A_BYTES + Cfg::B_BYTES, &p.tm_bt, fb, kb * kBK, v0);
             }
             armed |= 1u << stage;
             last_par = (last_par & ~(1u << stage)) | (phase << stage);
@@ -244,35 +267,36 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const __grid_constan
           }
         }
       }
-      // Drain: every armed stage's last phase must have landed before exit.
-      for (int i = 0; i < STAGES; ++i)
-        if (armed & (1u << i)) {
-          volatile int never = 0;
-          if (!mbar_wait(&full[i], (last_par >> i) & 1, &never)) atomicOr(&g_dev_err, ERR_WAIT_TEARDOWN);
-        }
+      // The leader's full barriers count both CTAs' loads: drain them there.
+      if (leader)
+        for (int i = 0; i < STAGES; ++i)
+          if (armed & (1u << i)) {
+            volatile int never = 0;
+            if (!mbar_wait(&full[i], (last_par >> i) & 1, &never)) atomicOr(&g_dev_err, ERR_WAIT_TEARDOWN);
+          }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16(kBM, kBN, 0, 0);
+    // ------------------------------------------------------------ MMA issuer (leader)
+    if (leader && lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16(2 * kBM, kFBN, 0, 0);
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
       int it = 0;
-      for (int u = blockIdx.x; u < p.units_total && ok; u += gridDim.x) {
+      for (int u = pair; u < p.units_total && ok; u += npairs) {
         const int g = u / p.MT;
         const int vt_end = min(g * p.GT + p.GT, p.IT);
         for (int vt = g * p.GT; vt < vt_end && ok; ++vt, ++it) {
-          const int acc = it & 1;
-          const uint32_t ap = (it >> 1) & 1;
-          if (!mbar_wait(&acc_empty[acc], ap ^ 1, abort_flag)) {
+          const int acc = it % Cfg::NUM_ACC;
+          const uint32_t ap = (it / Cfg::NUM_ACC) & 1;
+          if (!mbar_wait_cluster(&acc_empty[acc], ap ^ 1, abort_flag)) {
             raise_abort(abort_flag, ERR_WAIT_ACC_EMPTY);
             ok = false;
             break;
           }
           tc_fence_after();
           const uint32_t d_s = tmem_base + acc * Cfg::ACC_COLS;
-          const uint32_t d_t = d_s + kBN;
+          const uint32_t d_t = d_s + kFBN;
           for (int kb = 0; kb < p.KB; ++kb) {
             if (!mbar_wait(&full[stage], phase, abort_flag)) {
               raise_abort(abort_flag, ERR_WAIT_TMA_FULL);
@@ -281,26 +305,29 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const __grid_constan
             }
             tc_fence_after();
             const uint32_t sa = smem_u32(smem + stage * Cfg::STAGE_BYTES);
+            const uint32_t sb = sa + Cfg::A_BYTES;
+            const uint32_t sat = sb + Cfg::B_BYTES;
+            const uint32_t sbt = sat + Cfg::A_BYTES;
 #pragma unroll
             for (int k = 0; k < kBK / 16; ++k) {
               const uint32_t acc_flag = (kb | k) != 0;
-              umma_bf16(d_s, sdesc_sw128(sa + 32 * k, 16, 1024),
-                        sdesc_sw128(sa + Cfg::A_BYTES + 32 * k, 16, 1024), idesc, acc_flag);
+              umma_bf16_pair(d_s, sdesc_sw128(sa + 32 * k, 16, 1024), sdesc_sw128(sb + 32 * k, 16, 1024), idesc,
+                             acc_flag);
               if (NG == 2)
-                umma_bf16(d_t, sdesc_sw128(sa + 2 * Cfg::A_BYTES + 32 * k, 16, 1024),
-                          sdesc_sw128(sa + 2 * Cfg::A_BYTES + Cfg::B_BYTES + 32 * k, 16, 1024), idesc, acc_flag);
+                umma_bf16_pair(d_t, sdesc_sw128(sat + 32 * k, 16, 1024), sdesc_sw128(sbt + 32 * k, 16, 1024),
+                               idesc, acc_flag);
             }
-            umma_commit(&empty[stage]);
+            umma_commit_pair(&empty[stage], 0x3);
             if (++stage == STAGES) {
               stage = 0;
               phase ^= 1;
             }
           }
-          if (ok) umma_commit(&acc_full[acc]);
+          if (ok) umma_commit_pair(&acc_full[acc], 0x3);
         }
       }
       // All issued MMAs must finish before TMEM is released.
-      umma_commit(tear);
+      umma_commit_pair(tear, 0x1);
       volatile int never = 0;
       if (!mbar_wait(tear, 0, &never)) atomicOr(&g_dev_err, ERR_WAIT_TEARDOWN);
     }
@@ -309,19 +336,19 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const __grid_constan
     const int q = warp & 3;
     const int row = q * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
-    int cur_mt = -1;
+    const uint32_t acc_empty0 = mapa_shared(smem_u32(acc_empty), 0);
+    int cur_m0 = -1;
     float lse2 = 0.f, cst = 0.f, g_row = 0.f;
     const uint16_t* trow = nullptr;
     int box = 0;
     int it = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < p.units_total && ok; u += gridDim.x) {
-      const int mt = u % p.MT;
-      const int m0 = mt * kBM;
+    for (int u = pair; u < p.units_total && ok; u += npairs) {
+      const int m0 = (u % p.MT) * 2 * kBM + rank * kBM;  // this CTA's first row
       const int g = u / p.MT;
       const int vt_end = min(g * p.GT + p.GT, p.IT);
-      if (mt != cur_mt) {
-        cur_mt = mt;
+      if (m0 != cur_m0) {
+        cur_m0 = m0;
         const int r = m0 + row;
         if (DZ) {
           lse2 = p.rowc[r];
@@ -338,34 +365,19 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const __grid_constan
       }
       RowStats st{-INFINITY, 0.f, 0.f, -INFINITY, 0.f};
       for (int vt = g * p.GT; vt < vt_end; ++vt, ++it) {
-        const int v0 = (p.vt_base + vt) * kBN;
-        // Teacher logits of this row for the tile (logits payload): 128 bf16.
-        uint4 tv[NG == 1 ? 16 : 1];
+        const int v0 = (p.vt_base + vt) * kFBN;
+        // Teacher logits of this row (logits payload): 32 bf16 per chunk,
+        // loaded one chunk ahead.
+        uint4 tcur[NG == 1 ? 4 : 1], tnxt[NG == 1 ? 4 : 1];
         if (NG == 1) {
-          if (trow != nullptr) {
-            const uint16_t* src = trow + v0;
-            const int nvalid = p.V - v0;
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              if (i * 8 < nvalid)
-                tv[i] = ldg_nc_v4(src + i * 8);
-              else
-                tv[i] = make_uint4(0, 0, 0, 0);
-            }
-            // warm L2 for the next tile of this row
-            const int nv0 = v0 + kBN;
-            if (vt + 1 < vt_end) {
-              if (nv0 < p.V) prefetch_l2(trow + nv0);
-              if (nv0 + 64 < p.V) prefetch_l2(trow + nv0 + 64);
-            }
-          } else {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) tv[i] = make_uint4(0, 0, 0, 0);
+          for (int i = 0; i < 4; ++i) {
+            tcur[i] = (trow != nullptr && i * 8 < p.V - v0) ? ldg_nc_v4(trow + v0 + i * 8) : make_uint4(0, 0, 0, 0);
           }
         }
-        const int acc = it & 1;
-        const uint32_t ap = (it >> 1) & 1;
-        bool w_ok = mbar_wait(&acc_full[acc], ap, abort_flag);
+        const int acc = it % Cfg::NUM_ACC;
+        const uint32_t ap = (it / Cfg::NUM_ACC) & 1;
+        bool w_ok = mbar_wait_cluster(&acc_full[acc], ap, abort_flag);
         w_ok = __all_sync(0xffffffffu, w_ok);
         if (!w_ok) {
           if (lane == 0) raise_abort(abort_flag, ERR_WAIT_ACC_FULL);
@@ -375,20 +387,26 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const __grid_constan
         tc_fence_after();
         const uint32_t tb = tmem_base + lane_off + acc * Cfg::ACC_COLS;
 #pragma unroll
-        for (int c = 0; c < kBN / 32; ++c) {
+        for (int c = 0; c < kFBN / 32; ++c) {
           float zs[32], zt[32];
+          if (NG == 1 && c + 1 < kFBN / 32) {
+            const int vn = v0 + (c + 1) * 32;
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              tnxt[i] = (trow != nullptr && i * 8 < p.V - vn) ? ldg_nc_v4(trow + vn + i * 8) : make_uint4(0, 0, 0, 0);
+          }
           tmem_ld_32x32(tb + c * 32, zs);
-          if (NG == 2) tmem_ld_32x32(tb + kBN + c * 32, zt);
+          if (NG == 2) tmem_ld_32x32(tb + kFBN + c * 32, zt);
           tmem_wait_ld();
-          if (c == kBN / 32 - 1) {
+          if (c == kFBN / 32 - 1) {
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&acc_empty[acc]);
+            if (lane == 0) mbar_arrive_cluster(acc_empty0 + acc * 8);
           }
           if (NG == 1) {
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-              const uint4 w = tv[c * 4 + i];
+              const uint4 w = tcur[i];
               zt[8 * i + 0] = bf16_lo(w.x);
               zt[8 * i + 1] = bf16_hi(w.x);
               zt[8 * i + 2] = bf16_lo(w.y);
@@ -398,6 +416,8 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const __grid_constan
               zt[8 * i + 6] = bf16_lo(w.w);
               zt[8 * i + 7] = bf16_hi(w.w);
             }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) tcur[i] = tnxt[i];
           }
           if (!DZ) {
             const int nv = p.V - (v0 + c * 32);
@@ -456,11 +476,13 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const __grid_constan
     }
   }
 
+  // Neither CTA may release its TMEM or shared memory while the pair MMAs or
+  // the other CTA can still touch them.
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();
   if (warp == 2) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+    tmem_dealloc_pair(tmem_base, Cfg::TMEM_COLS);
   }
 }
 
@@ -777,22 +799,30 @@ cudaError_t tc_setup(int /*device*/) {
   return cudaFuncSetAttribute(grad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)grad_smem_bytes());
 }
 
-cudaError_t launch_fused(int ng, bool dz, const FusedArgs& a, dim3 grid, cudaStream_t s) {
+template <typename K>
+static cudaError_t launch_pair(K kernel, int grid, size_t smem, cudaStream_t s, const FusedArgs& a) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid & ~1);  // whole CTA pairs
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, a);
+}
+
+cudaError_t launch_fused(int ng, bool dz, const FusedArgs& a, int grid, cudaStream_t s) {
   const size_t smem = fused_smem_bytes(ng, dz);
   const int id = ng == 2 ? (dz ? K_DZ_DUAL_TC : K_FWD_DUAL_TC) : (dz ? K_DZ_SINGLE_TC : K_FWD_SINGLE_TC);
   LaunchScope scope(id, s);
-  if (ng == 2) {
-    if (dz)
-      fused_kernel<2, true><<<grid, kThreads, smem, s>>>(a);
-    else
-      fused_kernel<2, false><<<grid, kThreads, smem, s>>>(a);
-  } else {
-    if (dz)
-      fused_kernel<1, true><<<grid, kThreads, smem, s>>>(a);
-    else
-      fused_kernel<1, false><<<grid, kThreads, smem, s>>>(a);
-  }
-  return cudaGetLastError();
+  if (ng == 2) return dz ? launch_pair(fused_kernel<2, true>, grid, smem, s, a)
+                         : launch_pair(fused_kernel<2, false>, grid, smem, s, a);
+  return dz ? launch_pair(fused_kernel<1, true>, grid, smem, s, a) : launch_pair(fused_kernel<1, false>, grid, smem, s, a);
 }
 
 cudaError_t launch_grad(const GradArgs& a, int grid, cudaStream_t s) {
