@@ -53,6 +53,8 @@ _SIGS = {
                             _vp, _vp, _vp, _vp, _sz, _vp], _i32),
     "rkl_backward": ([_i32, _vp, _vp, _vp, _vp, _i32, _i64, _i64, _i64, _i64, _vp, _i32, _i32,
                       _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp], _i32),
+    "rkl_forward_hidden_noalloc": ([_vp, _vp, _vp, _vp, _i32, _i64, _i64, _i64, _i64, _vp, _i32, _i32,
+                                    _vp, _vp, _vp, _vp], _i32),
     "rkl_device_error": ([ctypes.POINTER(_i32)], _i32),
     "rkl_kernel_count": ([], _i32),
     "rkl_kernel_name": ([_i32], ctypes.c_char_p),

@@ -234,7 +234,8 @@ static uint8_t* ws_at(void* ws, size_t off) { return static_cast<uint8_t*>(ws) +
 static rkl_status forward_impl(rkl_payload payload, const void* h_s, const void* teacher, const void* W_s,
                                const void* W_t, rkl_dtype dtype, int64_t B, int64_t Sm1, int64_t H, int64_t V,
                                const int32_t* row_idx, int32_t N, rkl_reduction reduction, float* loss_tok,
-                               float* loss, float* saved, void* workspace, size_t workspace_bytes, void* stream_) {
+                               float* loss, float* saved, void* workspace, size_t workspace_bytes, void* stream_,
+                               bool forward_only_workspace = false) {
   RKL_TRY(check_common(payload, dtype, B, Sm1, H, V, N, reduction));
   RKL_TRY(check_ptr(h_s, "h_s"));
   RKL_TRY(check_ptr(teacher, payload == RKL_PAYLOAD_HIDDEN ? "h_t" : "teacher_logits"));
@@ -246,8 +247,10 @@ static rkl_status forward_impl(rkl_payload payload, const void* h_s, const void*
   RKL_TRY(check_ptr(saved, "saved", N > 0));
   RKL_TRY(check_ptr(workspace, "workspace"));
   const Plan pl = make_plan(payload, dtype, N, H, V);
-  if (workspace_bytes < pl.total)
-    return fail(RKL_ERR_WORKSPACE, "workspace is %zu bytes, %zu needed", workspace_bytes, pl.total);
+  // The forward touches only the regions in front of the dz chunk.
+  const size_t needed = forward_only_workspace ? pl.off_dz : pl.total;
+  if (workspace_bytes < needed)
+    return fail(RKL_ERR_WORKSPACE, "workspace is %zu bytes, %zu needed", workspace_bytes, needed);
   int sms = 0;
   RKL_TRY(device_setup(&sms));
   cudaStream_t s = static_cast<cudaStream_t>(stream_);
@@ -604,3 +607,57 @@ rkl_status rkl_profile_read(int32_t kernel_id, double* total_ms, int64_t* launch
 int64_t rkl_launch_count(void) { return g_launches.load(); }
 
 }  // extern "C"
+
+// ====================================================================== no-allocation forward
+// Scratch of rkl_forward_hidden_noalloc: one array in the library's device
+// image.  Every GPU on which the library's kernels are loaded holds these
+// bytes until the process exits, whether or not it ever calls that entry
+// point.  Host code only sees a stand-in symbol for it; the device address is
+// looked up per device below.
+namespace rkl {
+constexpr size_t kStaticScratchBytes = size_t(32) << 20;  // 32 MiB
+static __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
+
+static std::mutex g_static_mu;
+static void* g_static_ptr[64];  // device address of g_static_scratch, per device
+
+// Looks up (once per device, with that device current) the device address of
+// the static scratch array.
+static rkl_status static_scratch_ptr(void** out) {
+  int dev = 0;
+  RKL_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return fail(RKL_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lk(g_static_mu);
+  if (g_static_ptr[dev] == nullptr) {
+    void* ptr = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&ptr, g_static_scratch);
+    if (e != cudaSuccess || ptr == nullptr)
+      return fail(RKL_ERR_CUDA, "cudaGetSymbolAddress(static scratch) failed on device %d: %s", dev,
+                  cudaGetErrorString(e));
+    g_static_ptr[dev] = ptr;
+  }
+  *out = g_static_ptr[dev];
+  return RKL_OK;
+}
+}  // namespace rkl
+
+extern "C" rkl_status rkl_forward_hidden_noalloc(const void* h_s, const void* h_t, const void* W_s, const void* W_t,
+                                                 rkl_dtype dtype, int64_t B, int64_t Sm1, int64_t H, int64_t V,
+                                                 const int32_t* row_idx, int32_t N, rkl_reduction reduction,
+                                                 float* loss_tok, float* loss, float* saved, void* stream) {
+  // Size check first, from the same layout the workspace path uses; nothing
+  // on the device is touched when the problem does not fit.
+  RKL_TRY(check_common(RKL_PAYLOAD_HIDDEN, dtype, B, Sm1, H, V, N, reduction));
+  const Plan pl = make_plan(RKL_PAYLOAD_HIDDEN, dtype, N, H, V);
+  if (pl.off_dz > kStaticScratchBytes)
+    return fail(RKL_ERR_WORKSPACE,
+                "rkl_forward_hidden_noalloc: this problem needs %zu bytes of scratch, the static limit is %zu "
+                "bytes (%zu MiB); use rkl_forward_hidden with a caller workspace",
+                pl.off_dz, kStaticScratchBytes, kStaticScratchBytes >> 20);
+  void* scratch = nullptr;
+  RKL_TRY(static_scratch_ptr(&scratch));
+  // Every region of the scratch that the forward reads is written earlier in
+  // the same call, so nothing needs clearing between calls.
+  return forward_impl(RKL_PAYLOAD_HIDDEN, h_s, h_t, W_s, W_t, dtype, B, Sm1, H, V, row_idx, N, reduction, loss_tok,
+                      loss, saved, scratch, kStaticScratchBytes, stream, /*forward_only_workspace=*/true);
+}

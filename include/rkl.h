@@ -146,6 +146,34 @@ rkl_status rkl_backward(rkl_payload payload,
                         float* dH_s, float* dW_s,
                         void* workspace, size_t workspace_bytes, void* stream);
 
+/* rkl_forward_hidden without a caller workspace, for callers that cannot
+ * allocate device memory when they call: a runtime that plans all device
+ * memory up front and forbids allocation afterwards, code that runs where
+ * cudaMalloc is not allowed or would stall (it can synchronise the device and
+ * can fail under memory pressure), or a host with no device allocator of its
+ * own.  The pages have no counterpart to this entry point; it is a packaging
+ * convenience of this library.
+ *
+ * Arguments and outputs are those of rkl_forward_hidden.  The scratch is a
+ * fixed 32 MiB array inside the library's device image: every GPU on which
+ * the library is loaded holds it until the process exits.  A problem whose
+ * forward needs more scratch (rows x hidden x dtype of the compacted student
+ * and teacher rows, plus the partial statistics) is rejected with
+ * RKL_ERR_WORKSPACE and a message giving both sizes; nothing is enqueued.
+ * The first call on each device looks up the array's device address (with
+ * that device current); make that first call before any stream capture.
+ * This entry point allocates nothing: no cudaMalloc, no cudaFree, no
+ * allocating library call.  All calls share the one array and each call
+ * overwrites what it uses, so calls whose work can overlap on the GPU (other
+ * streams, other host threads) race and must be serialised by the caller. */
+rkl_status rkl_forward_hidden_noalloc(const void* h_s, const void* h_t,
+                                      const void* W_s, const void* W_t, rkl_dtype dtype,
+                                      int64_t B, int64_t Sm1, int64_t H, int64_t V,
+                                      const int32_t* row_idx, int32_t N,
+                                      rkl_reduction reduction,
+                                      float* loss_tok, float* loss, float* saved,
+                                      void* stream);
+
 /* Synchronises the current device, then reports and clears the library's
  * device error word: *code = 0 if no kernel's bounded wait ran out since the
  * last call, else a nonzero bit set naming the wait (the kernel returned
