@@ -145,7 +145,7 @@ static rkl_status make_map(CUtensorMap* m, const void* ptr, bool f32, uint64_t i
 }
 
 // ------------------------------------------------------------------ plan
-constexpr int kVcBf16 = 8192;  // vocab chunk of the backward (multiple of kFBN)
+constexpr int kVcBf16 = 16384;  // vocab chunk of the backward (multiple of kFBN)
 constexpr int kVcF32 = 1024;
 constexpr int kSimtSplits = 37;
 
@@ -168,7 +168,8 @@ static Plan make_plan(rkl_payload payload, rkl_dtype dtype, int64_t n_max, int64
   const int64_t n = n_max < 1 ? 1 : n_max;
   p.n_pad = static_cast<int>(((n + 2 * kBM - 1) / (2 * kBM)) * (2 * kBM));  // whole 256-row pair tiles
   p.VT = static_cast<int>((V + tile_v - 1) / tile_v);
-  p.S = bf16 ? (p.VT + kGroupTiles - 1) / kGroupTiles : (p.VT < kSimtSplits ? p.VT : kSimtSplits);
+  // tensor-core path: two statistics slots (column halves) per group
+  p.S = bf16 ? 2 * ((p.VT + kGroupTiles - 1) / kGroupTiles) : (p.VT < kSimtSplits ? p.VT : kSimtSplits);
   const int vc = bf16 ? kVcBf16 : kVcF32;
   const int64_t vround = ((V + kFBN - 1) / kFBN) * kFBN;
   p.Vc = static_cast<int>(vround < vc ? vround : vc);
@@ -295,7 +296,7 @@ static rkl_status forward_impl(rkl_payload payload, const void* h_s, const void*
       a.IT = pl.VT;
       a.vt_base = 0;
       a.GT = kGroupTiles;
-      a.G = pl.S;
+      a.G = pl.S / 2;
       const int MT = (N + 2 * kBM - 1) / (2 * kBM);
       a.MT = MT;
       a.units_total = MT * a.G;

@@ -36,7 +36,9 @@ __device__ int g_dev_err = 0;
 
 namespace {
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 192;       // gradient kernel: producer, MMA, 4 epilogue warps
+constexpr int kFusedEpi = 8;        // fused kernels: 2 epilogue warps per TMEM lane quarter
+constexpr int kFusedThreads = 64 + 32 * kFusedEpi;
 constexpr int kStgBoxBytes = 4096;  // one 32-row staging box per epilogue warp
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
@@ -67,7 +69,7 @@ struct FusedCfg {
 // Bytes: 1024 alignment slack + stages + epilogue staging + barriers.
 template <int NG, bool DZ>
 constexpr size_t fused_smem() {
-  return 1024 + size_t(FusedCfg<NG>::STAGES) * FusedCfg<NG>::STAGE_BYTES + (DZ ? 4 * 2 * kStgBoxBytes : 0) + 256;
+  return 1024 + size_t(FusedCfg<NG>::STAGES) * FusedCfg<NG>::STAGE_BYTES + (DZ ? kFusedEpi * kStgBoxBytes : 0) + 256;
 }
 
 // ---- online statistics of one 32-column chunk (all columns valid)
@@ -170,13 +172,13 @@ __device__ __forceinline__ void prefetch_l2(const void* p) {
 // code on their own rows.
 // ============================================================================
 template <int NG, bool DZ>
-__global__ void __launch_bounds__(kThreads, 1) fused_kernel(const __grid_constant__ FusedArgs p) {
+__global__ void __launch_bounds__(kFusedThreads, 1) fused_kernel(const __grid_constant__ FusedArgs p) {
   using Cfg = FusedCfg<NG>;
   constexpr int STAGES = Cfg::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* stg = smem + STAGES * Cfg::STAGE_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(stg + (DZ ? 4 * 2 * kStgBoxBytes : 0));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(stg + (DZ ? kFusedEpi * kStgBoxBytes : 0));
   uint64_t* full = bars;
   uint64_t* empty = bars + STAGES;
   uint64_t* acc_full = bars + 2 * STAGES;
@@ -207,7 +209,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const __grid_constan
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&acc_full[i], 1);
-      mbar_init(&acc_empty[i], 8);  // 4 epilogue warps in each CTA of the pair
+      mbar_init(&acc_empty[i], 2 * kFusedEpi);  // every epilogue warp of both CTAs
     }
     mbar_init(tear, 1);
     *abort_flag = 0;
@@ -333,7 +335,10 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const __grid_constan
     }
   } else {
     // ------------------------------------------------------------ epilogue
+    // Warp w reads TMEM lane quarter q = w % 4 (tile rows 32 q .. 32 q + 31)
+    // and columns [128 h, 128 h + 128) of the 256-column tile, h = (w-2) / 4.
     const int q = warp & 3;
+    const int half = (warp - 2) >> 2;
     const int row = q * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
     const uint32_t acc_empty0 = mapa_shared(smem_u32(acc_empty), 0);
@@ -365,7 +370,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const __grid_constan
       }
       RowStats st{-INFINITY, 0.f, 0.f, -INFINITY, 0.f};
       for (int vt = g * p.GT; vt < vt_end; ++vt, ++it) {
-        const int v0 = (p.vt_base + vt) * kFBN;
+        const int v0 = (p.vt_base + vt) * kFBN + half * (kFBN / 2);  // this warp's first column
         // Teacher logits of this row (logits payload): 32 bf16 per chunk,
         // loaded one chunk ahead.
         uint4 tcur[NG == 1 ? 4 : 1], tnxt[NG == 1 ? 4 : 1];
@@ -385,11 +390,12 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const __grid_constan
           break;
         }
         tc_fence_after();
-        const uint32_t tb = tmem_base + lane_off + acc * Cfg::ACC_COLS;
+        const uint32_t tb = tmem_base + lane_off + acc * Cfg::ACC_COLS + half * (kFBN / 2);
+        constexpr int kChunks = kFBN / 2 / 32;
 #pragma unroll
-        for (int c = 0; c < kFBN / 32; ++c) {
+        for (int c = 0; c < kChunks; ++c) {
           float zs[32], zt[32];
-          if (NG == 1 && c + 1 < kFBN / 32) {
+          if (NG == 1 && c + 1 < kChunks) {
             const int vn = v0 + (c + 1) * 32;
 #pragma unroll
             for (int i = 0; i < 4; ++i)
@@ -398,7 +404,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const __grid_constan
           tmem_ld_32x32(tb + c * 32, zs);
           if (NG == 2) tmem_ld_32x32(tb + kFBN + c * 32, zt);
           tmem_wait_ld();
-          if (c == kFBN / 32 - 1) {
+          if (c == kChunks - 1) {
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(acc_empty0 + acc * 8);
@@ -437,9 +443,9 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const __grid_constan
               const float d1 = g_row * p1 * ((zs[j + 1] - zt[j + 1]) + cst);
               pk[j / 2] = pack_bf16x2(d0, d1);
             }
-            uint8_t* buf = stg + (q * 2 + (box & 1)) * kStgBoxBytes;
+            uint8_t* buf = stg + (warp - 2) * kStgBoxBytes;  // one staging box per warp
             if ((c & 1) == 0) {
-              if (lane == 0) bulk_wait_read<1>();
+              if (lane == 0) bulk_wait_read<0>();
               __syncwarp();
             }
             const uint32_t rbase = smem_u32(buf) + lane * 128;
@@ -462,7 +468,8 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const __grid_constan
         }
       }
       if (!DZ && ok) {
-        float* base = p.part + static_cast<size_t>(g) * 5 * p.n_pad + m0 + row;
+        // statistics slot (group, column half): 2 slots per group
+        float* base = p.part + static_cast<size_t>(2 * g + half) * 5 * p.n_pad + m0 + row;
         base[0] = st.m_s;
         base[p.n_pad] = st.S_s;
         base[2 * p.n_pad] = st.A;
@@ -803,7 +810,7 @@ template <typename K>
 static cudaError_t launch_pair(K kernel, int grid, size_t smem, cudaStream_t s, const FusedArgs& a) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid & ~1);  // whole CTA pairs
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3(kFusedThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
