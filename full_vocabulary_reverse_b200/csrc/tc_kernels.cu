@@ -599,8 +599,11 @@ __global__ void __launch_bounds__(kThreads, 1) grad_kernel(const __grid_constant
         if (t < 0) break;
         const bool is_h = t < p.nH;
         const int tt = is_h ? t : t - p.nH;
-        const int m0 = (is_h ? tt % p.MTH : tt % p.MTW) * 2 * kBM + rank * kBM;  // this CTA's A rows
-        const int n0 = (is_h ? tt / p.MTH : tt / p.MTW) * kGradBN + rank * (kGradBN / 2);  // this CTA's B half
+        // tile tt = (row / vocab block tt / NT, H block tt % NT): the H block is
+        // the fast index, so the tiles running together share their A block
+        // (a slice of dz) in L2 and each slice of dz is read from memory once.
+        const int m0 = (tt / p.NT) * 2 * kBM + rank * kBM;                 // this CTA's A rows
+        const int n0 = (tt % p.NT) * kGradBN + rank * (kGradBN / 2);       // this CTA's B half
         const int KB = is_h ? p.KBH : p.KBW;
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait_cluster(&empty[stage], phase ^ 1, abort_flag)) {
@@ -719,8 +722,8 @@ __global__ void __launch_bounds__(kThreads, 1) grad_kernel(const __grid_constant
       if (t < 0) break;
       const bool is_h = t < p.nH;
       const int tt = is_h ? t : t - p.nH;
-      const int mtile = is_h ? tt % p.MTH : tt % p.MTW;
-      const int n0 = (is_h ? tt / p.MTH : tt / p.MTW) * kGradBN;
+      const int mtile = tt / p.NT;
+      const int n0 = (tt % p.NT) * kGradBN;
       const int acc = i & 1;
       const uint32_t ap = (i >> 1) & 1;
       ok = mbar_wait_cluster(&acc_full[acc], ap, abort_flag);
