@@ -221,3 +221,43 @@ def dz_rows(z_s, z_t, g):
     w = lp_s - lp_t
     L = np.sum(p_s * w, axis=1)
     return _f64(g)[:, None] * p_s * (w - L[:, None])
+
+
+# ---------------------------------------------------------------------------
+# Both sides as logits.  NeMo RL PR #3978, payload bullet 2 calls the logits
+# payload the numerical-reference path; when the student's logits are also
+# given as a [T, V] tensor the loss and its gradient w.r.t. those logits are
+# the same objective and the same shared backward, with no LM head.
+# ---------------------------------------------------------------------------
+
+def forward_logits_pair(z_s, z_t, mask, reduction):
+    """Loss of student logits z_s [T, V] against teacher logits z_t [T, V]."""
+    mask = np.asarray(mask)
+    B, Sm1 = mask.shape
+    row_idx, N = compact_rows(mask)
+    L = np.zeros(N)
+    lse_s = np.zeros(N)
+    lse_t = np.zeros(N)
+    for c0 in range(0, N, _ROW_CHUNK):
+        rows = row_idx[c0:c0 + _ROW_CHUNK]
+        n = len(rows)
+        L[c0:c0 + n], lse_s[c0:c0 + n], lse_t[c0:c0 + n] = per_row_kl(_f64(z_s[rows]), _f64(z_t[rows]))
+    loss_tok = np.zeros(B * Sm1)
+    loss_tok[row_idx] = L
+    loss = reduce_loss(L, row_idx, B, Sm1, reduction)
+    return {"loss_tok": loss_tok.reshape(B, Sm1), "loss": loss, "L": L,
+            "lse_s": lse_s, "lse_t": lse_t, "row_idx": row_idx, "N": N}
+
+
+def backward_logits_pair(z_s, z_t, mask, reduction, grad_loss=1.0, grad_tok=None):
+    """dLoss/dz_s [T, V]: the shared backward p_s (w - L) times the row weight;
+    exact zero rows at masked positions."""
+    mask = np.asarray(mask)
+    B, Sm1 = mask.shape
+    row_idx, N = compact_rows(mask)
+    g = row_weights(row_idx, B, Sm1, reduction, grad_loss, grad_tok)
+    dz = np.zeros(np.asarray(z_s).shape)
+    for c0 in range(0, N, _ROW_CHUNK):
+        rows = row_idx[c0:c0 + _ROW_CHUNK]
+        dz[rows] = dz_rows(_f64(z_s[rows]), _f64(z_t[rows]), g[c0:c0 + len(rows)])
+    return dz

@@ -253,3 +253,41 @@ def nested_mean_by_hand(O, rs):
     lt = out["loss_tok"]
     ref = 0.5 * (lt[0, 1] + (lt[2, 0] + lt[2, 1] + lt[2, 3]) / 3.0)
     return abs(out["loss"] - ref)
+
+
+def logits_pair_finite_differences(O, rs, red=1, with_grad_tok=False):
+    """Central differences of the objective w.r.t. the student logits."""
+    mask = np.array([[1, 1, 0], [0, 1, 0], [0, 0, 0]], dtype=np.uint8)
+    z_s = rs.normal(size=(9, 6)) * 2
+    z_t = rs.normal(size=(9, 6)) * 2
+    grad_tok = rs.normal(size=mask.shape) if with_grad_tok else None
+
+    def f(zs):
+        out = O.forward_logits_pair(zs, z_t, mask, red)
+        val = 0.0 if out["loss"] is None else out["loss"]
+        if grad_tok is not None:
+            val += float(np.sum(grad_tok * out["loss_tok"]))
+        return val
+
+    dz = O.backward_logits_pair(z_s, z_t, mask, red, grad_tok=grad_tok)
+    eps = 1e-6
+    num = np.zeros_like(z_s)
+    for i in range(z_s.shape[0]):
+        for j in range(z_s.shape[1]):
+            zp = z_s.copy(); zp[i, j] += eps
+            zm = z_s.copy(); zm[i, j] -= eps
+            num[i, j] = (f(zp) - f(zm)) / (2 * eps)
+    return float(np.max(np.abs(dz - num)) / max(1e-12, np.max(np.abs(num))))
+
+
+def logits_pair_matches_hidden_chain_rule(O, rs):
+    """With z_s = h_s W_s^T and z_t = h_t W_t^T, the logits-pair loss equals the
+    hidden-payload loss and dH_s = dz W_s, dW_s = dz^T h_s (chain rule)."""
+    h_s, W_s, h_t, W_t, mask = rand_problem(rs, B=2, Sm1=4, H=3, V=8)
+    z_s, z_t = h_s @ W_s.T, h_t @ W_t.T
+    a = O.forward(h_s, W_s, h_t, W_t, mask, 2)
+    b = O.forward_logits_pair(z_s, z_t, mask, 2)
+    dH, dW = O.backward(h_s, W_s, h_t, W_t, mask, 2)
+    dz = O.backward_logits_pair(z_s, z_t, mask, 2)
+    return max(float(np.max(np.abs(a["loss_tok"] - b["loss_tok"]))), abs(a["loss"] - b["loss"]),
+               float(np.max(np.abs(dH - dz @ W_s))), float(np.max(np.abs(dW - dz.T @ h_s))))

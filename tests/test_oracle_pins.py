@@ -183,3 +183,32 @@ def test_pins_catch_planted_mistakes(old, new, kind):
         "lse": lambda: pins.lse_vs_scipy(M, rs) > 1e-6,
     }[kind]()
     assert caught
+
+
+@pytest.mark.parametrize("red", [1, 2])
+def test_logits_pair_finite_differences(rs, red):
+    assert pins.logits_pair_finite_differences(O, rs, red=red) < 1e-6
+    assert pins.logits_pair_finite_differences(O, rs, red=0, with_grad_tok=True) < 1e-6
+
+
+def test_logits_pair_kl_matches_scipy(rs):
+    import scipy.special
+    import scipy.stats
+    z_s = rs.normal(size=(6, 50)) * 3
+    z_t = rs.normal(size=(6, 50)) * 3
+    out = O.forward_logits_pair(z_s, z_t, np.ones((2, 3), np.uint8), 0)
+    ref = scipy.stats.entropy(scipy.special.softmax(z_s, axis=1), scipy.special.softmax(z_t, axis=1), axis=1)
+    assert np.max(np.abs(out["L"] - ref)) < 1e-10
+
+
+def test_logits_pair_chain_rule_to_hidden_payload(rs):
+    assert pins.logits_pair_matches_hidden_chain_rule(O, rs) < 1e-12
+
+
+def test_logits_pair_masked_rows_zero_and_self_distill(rs):
+    z = rs.normal(size=(6, 40)) * 3
+    mask = np.array([[1, 0, 1], [0, 0, 1]], np.uint8)
+    dz = O.backward_logits_pair(z, rs.normal(size=(6, 40)), mask, 1)
+    assert np.all(dz[mask.reshape(-1) == 0] == 0)
+    assert np.all(O.backward_logits_pair(z, z.copy(), mask, 1) == 0)
+    assert O.forward_logits_pair(z, z.copy(), mask, 1)["loss"] == 0.0
