@@ -120,25 +120,31 @@ class Problem:
         self.dev = device
         self.B, self.Sm1 = inp["mask"].shape
         self.T = self.B * self.Sm1
-        self.H = inp["h_s"].shape[1]
-        self.V = inp["W_s"].shape[0]
-        self.logits = "teacher_logits" in inp
-        self.payload = rb.PAYLOAD_LOGITS if self.logits else rb.PAYLOAD_HIDDEN
-        self.dt = rb._dtype_code(inp["h_s"])
-        self.teacher = inp["teacher_logits"] if self.logits else inp["h_t"]
-        self.W_t = None if self.logits else inp["W_t"]
+        self.pair = "student_logits" in inp
+        self.logits = "teacher_logits" in inp and not self.pair
+        self.student = inp["student_logits"] if self.pair else inp["h_s"]
+        self.H = 0 if self.pair else inp["h_s"].shape[1]
+        self.V = inp["student_logits"].shape[1] if self.pair else inp["W_s"].shape[0]
+        self.payload = rb.PAYLOAD_LOGITS_PAIR if self.pair else (rb.PAYLOAD_LOGITS if self.logits else
+                                                                 rb.PAYLOAD_HIDDEN)
+        self.dt = rb._dtype_code(self.student)
+        self.teacher = inp["teacher_logits"] if (self.logits or self.pair) else inp["h_t"]
+        self.W_t = None if (self.logits or self.pair) else inp["W_t"]
         L = rb.lib()
         self.L = L
         self.row_idx = torch.empty(self.T, dtype=torch.int32, device=device)
         self.n_dev = torch.empty(1, dtype=torch.int32, device=device)
         self.n_host = torch.empty(1, dtype=torch.int32).pin_memory()
-        nbytes = rb.workspace_size(self.payload, self.dt, self.T, self.B, self.Sm1, self.H, self.V)
+        nbytes = rb.workspace_size(self.payload, self.dt, self.T, self.B, self.Sm1, max(self.H, 64), self.V)
         self.ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
         self.loss_tok = torch.empty((self.B, self.Sm1), dtype=torch.float32, device=device)
         self.loss = torch.empty(1, dtype=torch.float32, device=device)
         self.saved = torch.empty((self.T, 3), dtype=torch.float32, device=device)
-        self.dH = torch.empty((self.T, self.H), dtype=torch.float32, device=device)
-        self.dW = torch.empty((self.V, self.H), dtype=torch.float32, device=device)
+        if self.pair:
+            self.dz = torch.empty_like(self.student)
+        else:
+            self.dH = torch.empty((self.T, self.H), dtype=torch.float32, device=device)
+            self.dW = torch.empty((self.V, self.H), dtype=torch.float32, device=device)
         self.grad_loss = torch.ones(1, dtype=torch.float32, device=device)
         self.N = None
 
@@ -148,7 +154,7 @@ class Problem:
     def step(self, h_s=None, teacher=None, mask=None):
         """S1..S7 for one batch; returns N.  Inputs default to the resident ones."""
         L, p = self.L, self._p
-        h_s = self.inp["h_s"] if h_s is None else h_s
+        h_s = self.student if h_s is None else h_s
         teacher = self.teacher if teacher is None else teacher
         mask = self.inp["mask"] if mask is None else mask
         s = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
@@ -156,6 +162,15 @@ class Problem:
         self.n_host.copy_(self.n_dev, non_blocking=True)
         torch.cuda.current_stream().synchronize()
         N = int(self.n_host[0])
+        if self.pair:
+            rb._check(L.rkl_forward_logits_pair(p(h_s), p(teacher), self.dt, self.B, self.Sm1, self.V,
+                                                p(self.row_idx), N, self.reduction, p(self.loss_tok), p(self.loss),
+                                                p(self.saved), p(self.ws), self.ws.numel(), s))
+            rb._check(L.rkl_backward_logits_pair(p(h_s), p(teacher), self.dt, self.B, self.Sm1, self.V,
+                                                 p(self.row_idx), N, self.reduction, p(self.saved),
+                                                 p(self.grad_loss), None, p(self.dz), p(self.ws), self.ws.numel(), s))
+            self.N = N
+            return N
         if self.logits:
             rb._check(L.rkl_forward_logits(p(h_s), p(self.inp["W_s"]), p(teacher), self.dt, self.B, self.Sm1, self.H,
                                            self.V, p(self.row_idx), N, self.reduction, p(self.loss_tok), p(self.loss),
@@ -196,6 +211,9 @@ def kernel_profile():
 def algorithmic_work(prob, N):
     """Per-kernel algorithmic flops (tensor kernels) or bytes (bandwidth kernels) of one step."""
     H, V = prob.H, prob.V
+    if prob.pair:
+        return {"pair_fwd": ("hbm", 4.0 * N * V + 16.0 * N),
+                "pair_bwd": ("hbm", 4.0 * N * V + 2.0 * prob.T * V)}
     if prob.logits:
         return {"fwd_single_tc": ("tensor", 2.0 * N * H * V), "dz_single_tc": ("tensor", 2.0 * N * H * V),
                 "grad_dw_dh_tc": ("tensor", 4.0 * N * H * V), "teacher_lse": ("hbm", 2.0 * N * V + 4.0 * N)}
@@ -236,15 +254,22 @@ def cpu_oracle_sample(inp, reduction, name, rows=CPU_SAMPLE_ROWS):
     sub[flat] = 1
     sub = sub.reshape(mask.shape)
     f64 = lambda t: None if t is None else t.float().cpu().numpy()  # noqa: E731
-    h_s, W_s = f64(inp["h_s"]), f64(inp["W_s"])
-    if "teacher_logits" in inp:
-        teacher, W_t = f64(inp["teacher_logits"]), None
+    if "student_logits" in inp:
+        zs, zt = f64(inp["student_logits"]), f64(inp["teacher_logits"])
+        t0 = time.perf_counter()
+        O.forward_logits_pair(zs, zt, sub, reduction)
+        O.backward_logits_pair(zs, zt, sub, reduction)
+        dt = time.perf_counter() - t0
     else:
-        teacher, W_t = f64(inp["h_t"]), f64(inp["W_t"])
-    t0 = time.perf_counter()
-    O.forward(h_s, W_s, teacher, W_t, sub, reduction)
-    O.backward(h_s, W_s, teacher, W_t, sub, reduction)
-    dt = time.perf_counter() - t0
+        h_s, W_s = f64(inp["h_s"]), f64(inp["W_s"])
+        if "teacher_logits" in inp:
+            teacher, W_t = f64(inp["teacher_logits"]), None
+        else:
+            teacher, W_t = f64(inp["h_t"]), f64(inp["W_t"])
+        t0 = time.perf_counter()
+        O.forward(h_s, W_s, teacher, W_t, sub, reduction)
+        O.backward(h_s, W_s, teacher, W_t, sub, reduction)
+        dt = time.perf_counter() - t0
     threads = max([d.get("num_threads", 1) for d in threadpool_info()] or [1])
     return {"value": len(flat) / dt, "unit": UNIT, "cores": threads, "kind": "oracle",
             "sample": "%d trainable rows of the %s workload (float64 NumPy forward+backward incl. weight upcast), "
@@ -270,8 +295,10 @@ def run_reference(args, rank, world):
     out = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": world, "steps": len(vals),
            "warmup": args.warmup, "ms_per_step": 1000.0 * secs / max(1, len(vals)), "higher_is_better": True,
            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-           "config": {"workload": args.workload, "B": B, "Sm1": Sm1, "H": inp["h_s"].shape[1],
-                      "V": inp["W_s"].shape[0], "sample_rows": vals[-1]["rows"]},
+           "config": {"workload": args.workload, "B": B, "Sm1": Sm1,
+                      "H": inp["h_s"].shape[1] if "h_s" in inp else 0,
+                      "V": inp["W_s"].shape[0] if "W_s" in inp else inp["student_logits"].shape[1],
+                      "sample_rows": vals[-1]["rows"]},
            "cpu_baseline": {"value": v, "unit": UNIT, "cores": vals[-1]["cores"], "kind": "oracle",
                             "sample": vals[-1]["sample"]},
            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -321,11 +348,11 @@ def run_gpu(args, rank, world, dist):
     # stream while step i computes (two device buffers), as a training loop
     # with a prefetching data loader would do.  All copies are inside the
     # timed region.
-    h_pin = prob.inp["h_s"].cpu().pin_memory()
+    h_pin = prob.student.cpu().pin_memory()
     t_pin = prob.teacher.cpu().pin_memory()
     m_pin = prob.inp["mask"].cpu().pin_memory()
     loss_host = torch.empty(1, dtype=torch.float32).pin_memory()
-    bufs = [(torch.empty_like(prob.inp["h_s"]), torch.empty_like(prob.teacher), torch.empty_like(prob.inp["mask"]))
+    bufs = [(torch.empty_like(prob.student), torch.empty_like(prob.teacher), torch.empty_like(prob.inp["mask"]))
             for _ in range(2)]
     copy_stream = torch.cuda.Stream(dev)
     ready = [torch.cuda.Event(), torch.cuda.Event()]
@@ -392,22 +419,26 @@ def run_gpu(args, rank, world, dist):
                         "frac": ach / pk["hbm_gbs"], "traffic": traffic_for(k)}
     step_flops = sum(w for b, w in work.values() if b == "tensor")
     step_tflops = step_flops * args.steps / (ms / 1000.0) / 1e12
+    step_bytes = sum(w for b, w in work.values() if b == "hbm")
     total_ms = sum(v["ms"] for v in prof.values())
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16" if prob.dt == 0 else "fp32", "data": "synthetic",
         "config": {"workload": args.workload, "B": prob.B, "Sm1": prob.Sm1, "H": prob.H, "V": prob.V,
-                   "trainable_rows": N, "tokens_T": prob.T, "payload": "logits" if prob.logits else "hidden",
+                   "trainable_rows": N, "tokens_T": prob.T,
+                   "payload": "logits_pair" if prob.pair else ("logits" if prob.logits else "hidden"),
                    "parallelism": "replicas" if world > 1 else "single",
-                   "l2": "inputs larger than L2 (LM-head weights %.2f GB per pass > 126 MB); no flush" % (
-                       (2 if not prob.logits else 1) * prob.V * prob.H * 2 / 1e9)},
+                   "l2": "inputs larger than L2 (%.2f GB streamed per pass > 126 MB); no flush" % (
+                       (2 * prob.T * prob.V * 2 if prob.pair else (2 if not prob.logits else 1) * prob.V * prob.H * 2)
+                       / 1e9)},
         "roofline": {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
                      "frac": achieved / peak, "traffic": traffic_for(dom),
                      "peak_source": "%s %s" % (pk["source"], "bf16 sustained" if bound == "tensor" else "hbm copy"),
                      "frac_of_burst": achieved / pk["bf16_tflops"] if bound == "tensor" else None},
         "roofline_hbm_kernels": extra or None,
         "step_tflops": step_tflops, "step_tc_frac_sustained": step_tflops / pk["bf16_tflops_sustained"],
+        "step_hbm_gbs": step_bytes * args.steps / (ms / 1000.0) / 1e9,
         "tokens_T_per_s": value * prob.T / N,
         "kernels": {k: {"ms_per_step": v["ms"] / args.steps, "launches_per_step": v["launches"] / args.steps,
                         "share": v["ms"] / total_ms} for k, v in sorted(prof.items(), key=lambda x: -x[1]["ms"])},

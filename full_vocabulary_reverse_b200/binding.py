@@ -21,6 +21,7 @@ REDUCE_TOKEN_MEAN = 1
 REDUCE_SEQ_MEAN_NESTED = 2
 PAYLOAD_HIDDEN = 0
 PAYLOAD_LOGITS = 1
+PAYLOAD_LOGITS_PAIR = 2
 DT_BF16 = 0
 DT_FP32 = 1
 
@@ -53,6 +54,10 @@ _SIGS = {
                             _vp, _vp, _vp, _vp, _sz, _vp], _i32),
     "rkl_backward": ([_i32, _vp, _vp, _vp, _vp, _i32, _i64, _i64, _i64, _i64, _vp, _i32, _i32,
                       _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp], _i32),
+    "rkl_forward_logits_pair": ([_vp, _vp, _i32, _i64, _i64, _i64, _vp, _i32, _i32, _vp, _vp, _vp, _vp, _sz, _vp],
+                                _i32),
+    "rkl_backward_logits_pair": ([_vp, _vp, _i32, _i64, _i64, _i64, _vp, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _sz,
+                                  _vp], _i32),
     "rkl_forward_hidden_noalloc": ([_vp, _vp, _vp, _vp, _i32, _i64, _i64, _i64, _i64, _vp, _i32, _i32,
                                     _vp, _vp, _vp, _vp], _i32),
     "rkl_device_error": ([ctypes.POINTER(_i32)], _i32),
@@ -178,6 +183,40 @@ def backward(payload, h_s, teacher, W_s, W_t, B, Sm1, row_idx, N, reduction, sav
     return dH_s, dW_s
 
 
+def forward_logits_pair(student_logits, teacher_logits, B, Sm1, row_idx, N, reduction, workspace=None):
+    """Both sides as logits.  Returns (loss_tok [B,Sm1], loss [1], saved [N,3])."""
+    dev = student_logits.device
+    V = student_logits.shape[1]
+    dt = _dtype_code(student_logits)
+    loss_tok = torch.empty((B, Sm1), dtype=torch.float32, device=dev)
+    loss = torch.empty(1, dtype=torch.float32, device=dev)
+    saved = torch.empty((max(N, 1), 3), dtype=torch.float32, device=dev)
+    ws = workspace if workspace is not None else _workspace(PAYLOAD_LOGITS_PAIR, dt, max(N, 1), B, Sm1, 64, V, dev)
+    _check(lib().rkl_forward_logits_pair(_ptr(student_logits), _ptr(teacher_logits), dt, B, Sm1, V, _ptr(row_idx), N,
+                                         reduction, _ptr(loss_tok), _ptr(loss), _ptr(saved), _ptr(ws), ws.numel(),
+                                         _stream(dev)))
+    return loss_tok, loss, saved
+
+
+def backward_logits_pair(student_logits, teacher_logits, B, Sm1, row_idx, N, reduction, saved, grad_loss=None,
+                         grad_tok=None, workspace=None, dz=None):
+    """dLoss/dz_s [T, V] in the dtype of the logits."""
+    dev = student_logits.device
+    V = student_logits.shape[1]
+    dt = _dtype_code(student_logits)
+    if dz is None:
+        dz = torch.empty_like(student_logits)
+    if grad_loss is not None:
+        grad_loss = grad_loss.reshape(1).to(device=dev, dtype=torch.float32).contiguous()
+    if grad_tok is not None:
+        grad_tok = grad_tok.to(device=dev, dtype=torch.float32).contiguous()
+    ws = workspace if workspace is not None else _workspace(PAYLOAD_LOGITS_PAIR, dt, max(N, 1), B, Sm1, 64, V, dev)
+    _check(lib().rkl_backward_logits_pair(_ptr(student_logits), _ptr(teacher_logits), dt, B, Sm1, V, _ptr(row_idx),
+                                          N, reduction, _ptr(saved), _ptr(grad_loss), _ptr(grad_tok), _ptr(dz),
+                                          _ptr(ws), ws.numel(), _stream(dev)))
+    return dz
+
+
 def device_error():
     code = ctypes.c_int32(0)
     lib().rkl_device_error(ctypes.byref(code))
@@ -220,6 +259,29 @@ class _RKLLogits(torch.autograd.Function):
         dH, dW = backward(PAYLOAD_LOGITS, h_s, logits, W_s, None, B, Sm1, row_idx, N, reduction, saved,
                           grad_loss=g_loss, grad_tok=g_tok)
         return dH.to(h_s.dtype), dW.to(W_s.dtype), None, None, None
+
+
+class _RKLLogitsPair(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, student_logits, teacher_logits, mask, reduction):
+        B, Sm1 = mask.shape
+        row_idx, N = compact_rows(mask)
+        loss_tok, loss, saved = forward_logits_pair(student_logits, teacher_logits, B, Sm1, row_idx, N, reduction)
+        ctx.save_for_backward(student_logits, teacher_logits, row_idx, saved)
+        ctx.meta = (B, Sm1, N, reduction)
+        return loss.reshape(()), loss_tok
+
+    @staticmethod
+    def backward(ctx, g_loss, g_tok):
+        zs, zt, row_idx, saved = ctx.saved_tensors
+        B, Sm1, N, reduction = ctx.meta
+        dz = backward_logits_pair(zs, zt, B, Sm1, row_idx, N, reduction, saved, grad_loss=g_loss, grad_tok=g_tok)
+        return dz, None, None, None
+
+
+def reverse_kl_logits_pair(student_logits, teacher_logits, mask, reduction=REDUCE_TOKEN_MEAN):
+    """Differentiable (loss, loss_tok) with both sides given as [T, V] logits; grad to the student logits."""
+    return _RKLLogitsPair.apply(student_logits.contiguous(), teacher_logits.contiguous(), mask, reduction)
 
 
 def reverse_kl_hidden(h_s, h_t, W_s, W_t, mask, reduction=REDUCE_TOKEN_MEAN):

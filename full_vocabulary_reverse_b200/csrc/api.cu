@@ -43,7 +43,7 @@ static rkl_status fail(rkl_status s, const char* fmt, ...) {
 static const char* const kKernelNames[K_COUNT] = {
     "compact_rows", "gather_rows",   "fwd_dual_tc",  "fwd_single_tc", "teacher_lse", "combine_splits",
     "scatter_loss", "reduce_loss",   "row_weights",  "dz_dual_tc",    "dz_single_tc", "grad_dw_dh_tc",
-    "scatter_dh",   "fwd_simt_fp32", "dz_simt_fp32", "grad_simt_fp32"};
+    "scatter_dh",   "fwd_simt_fp32", "dz_simt_fp32", "grad_simt_fp32", "pair_fwd",   "pair_bwd"};
 
 const char* kernel_name(int id) { return (id >= 0 && id < K_COUNT) ? kKernelNames[id] : nullptr; }
 
@@ -201,8 +201,9 @@ static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 static rkl_status check_common(rkl_payload payload, rkl_dtype dtype, int64_t B, int64_t Sm1, int64_t H, int64_t V,
                                int32_t N, int reduction) {
   if (dtype != RKL_BF16 && dtype != RKL_FP32) return fail(RKL_ERR_DTYPE, "unknown dtype %d", (int)dtype);
-  if (payload != RKL_PAYLOAD_HIDDEN && payload != RKL_PAYLOAD_LOGITS)
+  if (payload != RKL_PAYLOAD_HIDDEN && payload != RKL_PAYLOAD_LOGITS && payload != RKL_PAYLOAD_LOGITS_PAIR)
     return fail(RKL_ERR_DTYPE, "unknown payload %d", (int)payload);
+  if (payload == RKL_PAYLOAD_LOGITS_PAIR) H = 64;  // no hidden dimension in this mode
   if (reduction < 0 || reduction > 2) return fail(RKL_ERR_DTYPE, "unknown reduction %d", reduction);
   if (B < 1 || Sm1 < 1 || H < 1 || V < 1) return fail(RKL_ERR_SHAPE, "B, Sm1, H, V must be >= 1");
   if (B * Sm1 >= (int64_t(1) << 31)) return fail(RKL_ERR_SHAPE, "B*Sm1 = %lld exceeds 2^31-1", (long long)(B * Sm1));
@@ -499,12 +500,76 @@ const char* rkl_version(void) { return "rkl 0.1 (sm_100a)"; }
 
 const char* rkl_last_error(void) { return g_last_error.c_str(); }
 
+// Workspace of the logits-pair mode: only the per-row constants of the backward.
+static size_t pair_workspace_bytes(int64_t n_max) {
+  const int64_t n = n_max < 1 ? 1 : n_max;
+  const size_t n_pad = size_t(((n + 255) / 256) * 256);
+  return 256 + align256(3 * n_pad * sizeof(float));
+}
+
 rkl_status rkl_workspace_size(rkl_payload payload, rkl_dtype dtype, int64_t n_max, int64_t B, int64_t Sm1, int64_t H,
                               int64_t V, size_t* bytes) {
   if (bytes == nullptr) return fail(RKL_ERR_NULL, "bytes is NULL");
   RKL_TRY(check_common(payload, dtype, B, Sm1, H, V, 0, 0));
   if (n_max < 0 || n_max > B * Sm1) return fail(RKL_ERR_SHAPE, "n_max outside [0, B*Sm1]");
-  *bytes = make_plan(payload, dtype, n_max, H, V).total;
+  *bytes = payload == RKL_PAYLOAD_LOGITS_PAIR ? pair_workspace_bytes(n_max) : make_plan(payload, dtype, n_max, H, V).total;
+  return RKL_OK;
+}
+
+rkl_status rkl_forward_logits_pair(const void* student_logits, const void* teacher_logits, rkl_dtype dtype, int64_t B,
+                                   int64_t Sm1, int64_t V, const int32_t* row_idx, int32_t N, rkl_reduction reduction,
+                                   float* loss_tok, float* loss, float* saved, void* workspace,
+                                   size_t workspace_bytes, void* stream) {
+  RKL_TRY(check_common(RKL_PAYLOAD_LOGITS_PAIR, dtype, B, Sm1, 64, V, N, reduction));
+  RKL_TRY(check_ptr(student_logits, "student_logits"));
+  RKL_TRY(check_ptr(teacher_logits, "teacher_logits"));
+  RKL_TRY(check_ptr(row_idx, "row_idx"));
+  RKL_TRY(check_ptr(loss_tok, "loss_tok", false));
+  RKL_TRY(check_ptr(loss, "loss", false));
+  RKL_TRY(check_ptr(saved, "saved", N > 0));
+  RKL_TRY(check_ptr(workspace, "workspace"));
+  if (workspace_bytes < pair_workspace_bytes(N))
+    return fail(RKL_ERR_WORKSPACE, "workspace is %zu bytes, %zu needed", workspace_bytes, pair_workspace_bytes(N));
+  int sms = 0;
+  RKL_TRY(device_setup(&sms));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const long long T = B * Sm1;
+  RKL_CUDA(launch_pair_fwd(student_logits, teacher_logits, dtype == RKL_BF16, row_idx, N, static_cast<int>(V), saved,
+                           s));
+  if (loss_tok) RKL_CUDA(launch_scatter_loss(saved, row_idx, N, T, loss_tok, s));
+  if (loss && reduction != RKL_REDUCE_NONE)
+    RKL_CUDA(launch_reduce(saved, row_idx, N, static_cast<int>(B), static_cast<int>(Sm1), reduction, loss, s));
+  return RKL_OK;
+}
+
+rkl_status rkl_backward_logits_pair(const void* student_logits, const void* teacher_logits, rkl_dtype dtype,
+                                    int64_t B, int64_t Sm1, int64_t V, const int32_t* row_idx, int32_t N,
+                                    rkl_reduction reduction, const float* saved, const float* grad_loss,
+                                    const float* grad_tok, void* dz, void* workspace, size_t workspace_bytes,
+                                    void* stream) {
+  RKL_TRY(check_common(RKL_PAYLOAD_LOGITS_PAIR, dtype, B, Sm1, 64, V, N, reduction));
+  RKL_TRY(check_ptr(student_logits, "student_logits"));
+  RKL_TRY(check_ptr(teacher_logits, "teacher_logits"));
+  RKL_TRY(check_ptr(row_idx, "row_idx"));
+  RKL_TRY(check_ptr(saved, "saved", N > 0));
+  RKL_TRY(check_ptr(grad_loss, "grad_loss", false));
+  RKL_TRY(check_ptr(grad_tok, "grad_tok", false));
+  RKL_TRY(check_ptr(dz, "dz"));
+  RKL_TRY(check_ptr(workspace, "workspace"));
+  if (workspace_bytes < pair_workspace_bytes(N))
+    return fail(RKL_ERR_WORKSPACE, "workspace is %zu bytes, %zu needed", workspace_bytes, pair_workspace_bytes(N));
+  int sms = 0;
+  RKL_TRY(device_setup(&sms));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const long long T = B * Sm1;
+  const int64_t n = N < 1 ? 1 : N;
+  const int n_pad = static_cast<int>(((n + 255) / 256) * 256);
+  float* rowc = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + 256);
+  if (N > 0)
+    RKL_CUDA(launch_row_weights(saved, row_idx, N, n_pad, static_cast<int>(B), static_cast<int>(Sm1), reduction,
+                                grad_loss, grad_tok, rowc, s));
+  RKL_CUDA(launch_pair_bwd(student_logits, teacher_logits, dtype == RKL_BF16, row_idx, N, n_pad, T,
+                           static_cast<int>(V), rowc, dz, s));
   return RKL_OK;
 }
 

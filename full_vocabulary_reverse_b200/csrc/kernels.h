@@ -27,6 +27,8 @@ enum KernelId : int {
   K_FWD_SIMT,         // fp32 S3 (CUDA cores)
   K_DZ_SIMT,          // fp32 S6
   K_GRAD_SIMT,        // fp32 S7
+  K_PAIR_FWD,         // both sides as logits: forward statistics, bandwidth bound
+  K_PAIR_BWD,         // both sides as logits: dL/dz_s rows, bandwidth bound
   K_COUNT
 };
 
@@ -105,6 +107,10 @@ cudaError_t launch_row_weights(const float* saved, const int32_t* row_idx, int N
                                cudaStream_t s);
 cudaError_t launch_scatter_dh(const float* dHc, const int32_t* row_idx, int N, long long T, int H, float* dH_s,
                               cudaStream_t s);
+cudaError_t launch_pair_fwd(const void* zs, const void* zt, bool bf16, const int32_t* row_idx, int N, int V,
+                            float* saved, cudaStream_t s);
+cudaError_t launch_pair_bwd(const void* zs, const void* zt, bool bf16, const int32_t* row_idx, int N, int n_pad,
+                            long long T, int V, const float* rowc, void* dz, cudaStream_t s);
 
 // ---------------------------------------------------------------- fp32 CUDA-core path
 struct SimtArgs {

@@ -405,6 +405,184 @@ __global__ void __launch_bounds__(256) scatter_dh_kernel(const float* __restrict
   }
 }
 
+// ------------------------------------------------------------ logits pair
+// Both sides as [T, V] logits (NeMo RL PR #3978, payload bullet 2: the logits
+// path as the numerical reference).  Forward: one CTA per trainable row
+// streams z_s and z_t once with 16-byte loads and keeps online
+// (m_s, S_s, A, m_t, S_t) per thread, then merges them in a fixed order.
+// Backward: one CTA per token row writes dL/dz_s for the whole row (exact
+// zeros at masked rows).  Both are pure HBM streams.
+struct PairStat {
+  float m_s, S_s, A, m_t, S_t;
+};
+
+__device__ __forceinline__ void pair_merge(PairStat& a, const PairStat& b) {
+  const float ns = fmaxf(a.m_s, b.m_s), nt = fmaxf(a.m_t, b.m_t);
+  if (ns != -INFINITY) {
+    const float ea = ex2((a.m_s - ns) * kLog2e), eb = ex2((b.m_s - ns) * kLog2e);
+    a.S_s = a.S_s * ea + b.S_s * eb;
+    a.A = a.A * ea + b.A * eb;
+    a.m_s = ns;
+  }
+  if (nt != -INFINITY) {
+    const float ea = ex2((a.m_t - nt) * kLog2e), eb = ex2((b.m_t - nt) * kLog2e);
+    a.S_t = a.S_t * ea + b.S_t * eb;
+    a.m_t = nt;
+  }
+}
+
+// Online update with VEC values of each side.
+template <int VEC>
+__device__ __forceinline__ void pair_update(PairStat& st, const float* xs, const float* xt) {
+  float cs = xs[0], ct = xt[0];
+#pragma unroll
+  for (int j = 1; j < VEC; ++j) {
+    cs = fmaxf(cs, xs[j]);
+    ct = fmaxf(ct, xt[j]);
+  }
+  if (cs > st.m_s) {
+    const float a = ex2((st.m_s - cs) * kLog2e);
+    st.S_s *= a;
+    st.A *= a;
+    st.m_s = cs;
+  }
+  if (ct > st.m_t) {
+    st.S_t *= ex2((st.m_t - ct) * kLog2e);
+    st.m_t = ct;
+  }
+  const float ms2 = st.m_s * kLog2e, mt2 = st.m_t * kLog2e;
+#pragma unroll
+  for (int j = 0; j < VEC; ++j) {
+    const float e = ex2(fmaf(xs[j], kLog2e, -ms2));
+    const float f = ex2(fmaf(xt[j], kLog2e, -mt2));
+    st.S_s += e;
+    st.S_t += f;
+    st.A = fmaf(e, xs[j] - xt[j], st.A);
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) pair_fwd_kernel(const T* __restrict__ zs_all, const T* __restrict__ zt_all,
+                                                       const int32_t* __restrict__ row_idx, int N, int V,
+                                                       float* __restrict__ saved) {
+  constexpr int VEC = 16 / sizeof(T);
+  const int k = blockIdx.x;
+  if (k >= N) return;
+  const long long r = row_idx[k];
+  const T* zs = zs_all + r * V;
+  const T* zt = zt_all + r * V;
+  PairStat st{-INFINITY, 0.f, 0.f, -INFINITY, 0.f};
+  int done = 0;
+  if (((reinterpret_cast<uintptr_t>(zs) | reinterpret_cast<uintptr_t>(zt)) & 15) == 0) {
+    const int nvec = V / VEC;
+    const uint4* vs = reinterpret_cast<const uint4*>(zs);
+    const uint4* vt = reinterpret_cast<const uint4*>(zt);
+    int i = threadIdx.x;
+    for (; i + 256 < nvec; i += 512) {
+      const uint4 a0 = ldg_stream_v4(vs + i), b0 = ldg_stream_v4(vt + i);
+      const uint4 a1 = ldg_stream_v4(vs + i + 256), b1 = ldg_stream_v4(vt + i + 256);
+      float xs[VEC], xt[VEC];
+      vec_to_float<T>(a0, xs);
+      vec_to_float<T>(b0, xt);
+      pair_update<VEC>(st, xs, xt);
+      vec_to_float<T>(a1, xs);
+      vec_to_float<T>(b1, xt);
+      pair_update<VEC>(st, xs, xt);
+    }
+    for (; i < nvec; i += 256) {
+      float xs[VEC], xt[VEC];
+      vec_to_float<T>(ldg_stream_v4(vs + i), xs);
+      vec_to_float<T>(ldg_stream_v4(vt + i), xt);
+      pair_update<VEC>(st, xs, xt);
+    }
+    done = nvec * VEC;
+  }
+  for (int v = done + threadIdx.x; v < V; v += 256) {
+    const float xs = to_f<T>(zs[v]), xt = to_f<T>(zt[v]);
+    pair_update<1>(st, &xs, &xt);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    PairStat b{__shfl_xor_sync(0xffffffffu, st.m_s, o), __shfl_xor_sync(0xffffffffu, st.S_s, o),
+               __shfl_xor_sync(0xffffffffu, st.A, o), __shfl_xor_sync(0xffffffffu, st.m_t, o),
+               __shfl_xor_sync(0xffffffffu, st.S_t, o)};
+    pair_merge(st, b);
+  }
+  __shared__ PairStat sh[8];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) sh[warp] = st;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    PairStat t = sh[0];
+    for (int w = 1; w < 8; ++w) pair_merge(t, sh[w]);
+    const float lse_s = t.m_s + logf(t.S_s);
+    const float lse_t = t.m_t + logf(t.S_t);
+    saved[3 * k + 0] = lse_s;
+    saved[3 * k + 1] = lse_t;
+    saved[3 * k + 2] = t.A / t.S_s - lse_s + lse_t;
+  }
+}
+
+template <typename T>
+__device__ __forceinline__ uint4 float_to_vec(const float* d);
+
+template <>
+__device__ __forceinline__ uint4 float_to_vec<__nv_bfloat16>(const float* d) {
+  return make_uint4(pack_bf16x2(d[0], d[1]), pack_bf16x2(d[2], d[3]), pack_bf16x2(d[4], d[5]),
+                    pack_bf16x2(d[6], d[7]));
+}
+
+template <>
+__device__ __forceinline__ uint4 float_to_vec<float>(const float* d) {
+  return make_uint4(__float_as_uint(d[0]), __float_as_uint(d[1]), __float_as_uint(d[2]), __float_as_uint(d[3]));
+}
+
+template <typename T>
+__device__ __forceinline__ T from_f(float x);
+template <>
+__device__ __forceinline__ float from_f<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
+
+// dz[t, :] = g p_s ((z_s - z_t) + lse_t - lse_s - L) for trainable t, else 0.
+template <typename T>
+__global__ void __launch_bounds__(256) pair_bwd_kernel(const T* __restrict__ zs_all, const T* __restrict__ zt_all,
+                                                       const int32_t* __restrict__ row_idx, int N, int n_pad, int V,
+                                                       const float* __restrict__ rowc, T* __restrict__ dz_all) {
+  constexpr int VEC = 16 / sizeof(T);
+  const long long t = blockIdx.x;
+  const int k = lower_bound_i32(row_idx, N, t);
+  const bool hit = k < N && row_idx[k] == t;
+  const T* zs = zs_all + t * V;
+  const T* zt = zt_all + t * V;
+  T* dz = dz_all + t * V;
+  const bool vec_ok = ((reinterpret_cast<uintptr_t>(zs) | reinterpret_cast<uintptr_t>(zt) |
+                        reinterpret_cast<uintptr_t>(dz)) & 15) == 0;
+  const int nvec = vec_ok ? V / VEC : 0;
+  if (!hit) {
+    uint4* d4 = reinterpret_cast<uint4*>(dz);
+    for (int i = threadIdx.x; i < nvec; i += 256) d4[i] = make_uint4(0, 0, 0, 0);
+    for (int v = nvec * VEC + threadIdx.x; v < V; v += 256) dz[v] = from_f<T>(0.f);
+    return;
+  }
+  const float lse2 = rowc[k], cst = rowc[n_pad + k], g = rowc[2 * n_pad + k];
+  const uint4* vs = reinterpret_cast<const uint4*>(zs);
+  const uint4* vt = reinterpret_cast<const uint4*>(zt);
+  uint4* vd = reinterpret_cast<uint4*>(dz);
+  for (int i = threadIdx.x; i < nvec; i += 256) {
+    float xs[VEC], xt[VEC], d[VEC];
+    vec_to_float<T>(ldg_stream_v4(vs + i), xs);
+    vec_to_float<T>(ldg_stream_v4(vt + i), xt);
+#pragma unroll
+    for (int j = 0; j < VEC; ++j) d[j] = g * ex2(fmaf(xs[j], kLog2e, -lse2)) * ((xs[j] - xt[j]) + cst);
+    vd[i] = float_to_vec<T>(d);
+  }
+  for (int v = nvec * VEC + threadIdx.x; v < V; v += 256) {
+    const float xs = to_f<T>(zs[v]), xt = to_f<T>(zt[v]);
+    dz[v] = from_f<T>(g * ex2(fmaf(xs, kLog2e, -lse2)) * ((xs - xt) + cst));
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_compact(const uint8_t* mask, long long T, int32_t* row_idx, int32_t* n_dev, cudaStream_t s) {
@@ -471,6 +649,38 @@ cudaError_t launch_scatter_dh(const float* dHc, const int32_t* row_idx, int N, l
   LaunchScope scope(K_SCATTER_DH, s);
   const long long blocks = T < 65535 * 8 ? T : 65535 * 8;
   scatter_dh_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(dHc, row_idx, N, T, H, dH_s);
+  return cudaGetLastError();
+}
+
+}  // namespace rkl
+
+namespace rkl {
+
+cudaError_t launch_pair_fwd(const void* zs, const void* zt, bool bf16, const int32_t* row_idx, int N, int V,
+                            float* saved, cudaStream_t s) {
+  if (N <= 0) return cudaSuccess;
+  LaunchScope scope(K_PAIR_FWD, s);
+  if (bf16)
+    pair_fwd_kernel<__nv_bfloat16><<<N, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(zs),
+                                                      static_cast<const __nv_bfloat16*>(zt), row_idx, N, V, saved);
+  else
+    pair_fwd_kernel<float><<<N, 256, 0, s>>>(static_cast<const float*>(zs), static_cast<const float*>(zt), row_idx,
+                                             N, V, saved);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pair_bwd(const void* zs, const void* zt, bool bf16, const int32_t* row_idx, int N, int n_pad,
+                            long long T, int V, const float* rowc, void* dz, cudaStream_t s) {
+  if (T <= 0) return cudaSuccess;
+  LaunchScope scope(K_PAIR_BWD, s);
+  if (bf16)
+    pair_bwd_kernel<__nv_bfloat16><<<static_cast<unsigned>(T), 256, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(zs), static_cast<const __nv_bfloat16*>(zt), row_idx, N, n_pad, V, rowc,
+        static_cast<__nv_bfloat16*>(dz));
+  else
+    pair_bwd_kernel<float><<<static_cast<unsigned>(T), 256, 0, s>>>(static_cast<const float*>(zs),
+                                                                    static_cast<const float*>(zt), row_idx, N, n_pad,
+                                                                    V, rowc, static_cast<float*>(dz));
   return cudaGetLastError();
 }
 

@@ -20,6 +20,9 @@ Named workloads:
   long_prompt     bf16, B=8, S-1=4096 (T=32768), H=4096, V=151936, W as
                   qwen_hidden at H=4096, last 256 positions of each sequence
                   trainable (N=2048), token mean.
+  logits_pair     both sides as bf16 logits [8192, 151936]: student ~ N(0,9),
+                  teacher = student + N(0, 0.5^2) + per-row shift U(-20,20);
+                  all rows trainable; token mean.
 """
 
 from __future__ import annotations
@@ -45,6 +48,8 @@ WORKLOADS = {
                            reduction=REDUCE_TOKEN_MEAN, mask="all", weights="perturbed", seed=1238),
     "long_prompt": dict(dtype="bf16", B=8, Sm1=4096, H=4096, V=151936, payload="hidden",
                         reduction=REDUCE_TOKEN_MEAN, mask="suffix256", weights="perturbed", seed=1239),
+    "logits_pair": dict(dtype="bf16", B=4, Sm1=2048, H=0, V=151936, payload="logits_pair",
+                        reduction=REDUCE_TOKEN_MEAN, mask="all", weights="perturbed", seed=1240),
 }
 
 TORCH_DTYPES = {"bf16": torch.bfloat16, "fp32": torch.float32}
@@ -95,6 +100,19 @@ def make_inputs(B, Sm1, H, V, dtype="bf16", payload="hidden", mask="prefix",
     gen = torch.Generator(device=device)
     gen.manual_seed(seed)
     out = {}
+    if payload == "logits_pair":
+        zs = torch.empty((T, V), dtype=tdt, device=device)
+        zt = torch.empty((T, V), dtype=tdt, device=device)
+        shift = torch.rand((T, 1), generator=gen, device=device) * 40.0 - 20.0
+        for r0 in range(0, T, 512):
+            r1 = min(T, r0 + 512)
+            a = torch.randn((r1 - r0, V), generator=gen, device=device) * logit_std
+            zs[r0:r1] = a.to(tdt)
+            b = a + torch.randn((r1 - r0, V), generator=gen, device=device) * 0.5 + shift[r0:r1]
+            zt[r0:r1] = (b if weights != "same" else a).to(tdt)
+        out["student_logits"], out["teacher_logits"] = zs, zt
+        out["mask"] = torch.from_numpy(make_mask(mask, B, Sm1, seed if mask_seed is None else mask_seed)).to(device)
+        return out
     out["h_s"] = _randn((T, H), gen, device).to(tdt)
     w_scale = logit_std / math.sqrt(H)
     W_s32 = _randn((V, H), gen, device, scale=w_scale)

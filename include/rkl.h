@@ -71,8 +71,13 @@ typedef enum rkl_reduction {
                                        sum_{t in b} L_t / n_b   (0 when N = 0) */
 } rkl_reduction;
 
-/* PR #3978, payload bullets: full.teacher_payload = hidden_states | logits. */
-typedef enum rkl_payload { RKL_PAYLOAD_HIDDEN = 0, RKL_PAYLOAD_LOGITS = 1 } rkl_payload;
+/* PR #3978, payload bullets: full.teacher_payload = hidden_states | logits.
+ * LOGITS_PAIR: the student's logits are given too (rkl_*_logits_pair). */
+typedef enum rkl_payload {
+  RKL_PAYLOAD_HIDDEN = 0,
+  RKL_PAYLOAD_LOGITS = 1,
+  RKL_PAYLOAD_LOGITS_PAIR = 2
+} rkl_payload;
 
 /* Library version string (static storage). */
 const char* rkl_version(void);
@@ -145,6 +150,31 @@ rkl_status rkl_backward(rkl_payload payload,
                         const float* grad_loss, const float* grad_tok,
                         float* dH_s, float* dW_s,
                         void* workspace, size_t workspace_bytes, void* stream);
+
+/* Both sides as logits: the student's logits [T, V] are given as well as the
+ * teacher's (the logits payload of PR #3978's payload bullet 2 used as the
+ * numerical reference, with the student side also materialised).  Same loss
+ * and saved scalars as rkl_forward_logits; bandwidth bound (reads 2 N V
+ * elements).  Any V >= 1; rows are read with 16-byte loads when the row
+ * pitch allows.  Workspace: rkl_workspace_size(RKL_PAYLOAD_LOGITS_PAIR, ...)
+ * (H is ignored). */
+rkl_status rkl_forward_logits_pair(const void* student_logits, const void* teacher_logits,
+                                   rkl_dtype dtype, int64_t B, int64_t Sm1, int64_t V,
+                                   const int32_t* row_idx, int32_t N,
+                                   rkl_reduction reduction,
+                                   float* loss_tok, float* loss, float* saved,
+                                   void* workspace, size_t workspace_bytes, void* stream);
+
+/* Backward of rkl_forward_logits_pair: dz [T, V] of `dtype` (overwritten) =
+ * dLoss/dz_s = g_k p_s (w - L) on trainable rows (row weight g_k as in
+ * rkl_backward), exact zeros on masked rows.  Reads 2 N V and writes T V
+ * elements. */
+rkl_status rkl_backward_logits_pair(const void* student_logits, const void* teacher_logits,
+                                    rkl_dtype dtype, int64_t B, int64_t Sm1, int64_t V,
+                                    const int32_t* row_idx, int32_t N,
+                                    rkl_reduction reduction, const float* saved,
+                                    const float* grad_loss, const float* grad_tok, void* dz,
+                                    void* workspace, size_t workspace_bytes, void* stream);
 
 /* rkl_forward_hidden without a caller workspace, for callers that cannot
  * allocate device memory when they call: a runtime that plans all device

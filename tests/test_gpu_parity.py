@@ -176,3 +176,63 @@ def test_autograd_wrapper():
     assert abs(float(loss) - r["loss"]) <= 1e-4 + 1e-3 * abs(r["loss"])
     assert grad_rel_err(h_s.grad.float(), r["dH_s"]) < GRAD_RTOL
     assert grad_rel_err(W_s.grad.float(), r["dW_s"]) < GRAD_RTOL
+
+
+# ---------------------------------------------------------------- logits pair
+def _pair_case(B, Sm1, V, dtype="bf16", mask="random", seed=0, same=False):
+    from full_vocabulary_reverse_b200.workloads import make_inputs
+    return make_inputs(B, Sm1, 0, V, dtype=dtype, payload="logits_pair", mask=mask,
+                       weights="same" if same else "perturbed", seed=seed, device="cuda")
+
+
+def _pair_run(inp, red, grad_tok=None):
+    mask = inp["mask"]
+    B, Sm1 = mask.shape
+    row_idx, N = rb.compact_rows(mask)
+    lt, loss, saved = rb.forward_logits_pair(inp["student_logits"], inp["teacher_logits"], B, Sm1, row_idx, N, red)
+    gl = torch.ones(1, device="cuda")
+    gt = None if grad_tok is None else torch.as_tensor(grad_tok, dtype=torch.float32).cuda()
+    dz = rb.backward_logits_pair(inp["student_logits"], inp["teacher_logits"], B, Sm1, row_idx, N, red, saved,
+                                 grad_loss=gl, grad_tok=gt)
+    torch.cuda.synchronize()
+    assert rb.device_error() == 0
+    return lt, loss, saved[:N], dz, N
+
+
+@pytest.mark.parametrize("V,dtype,red", [(1000, "bf16", 1), (1003, "bf16", 2), (777, "fp32", 1), (4096, "fp32", 2)])
+def test_logits_pair_small(V, dtype, red):
+    inp = _pair_case(3, 70, V, dtype=dtype, seed=V)
+    lt, loss, saved, dz, N = _pair_run(inp, red)
+    m = inp["mask"].cpu().numpy()
+    zs, zt = to_np(inp["student_logits"]), to_np(inp["teacher_logits"])
+    ref = O.forward_logits_pair(zs, zt, m, red)
+    rdz = O.backward_logits_pair(zs, zt, m, red)
+    assert_tok_close(lt, ref["loss_tok"])
+    assert abs(float(loss) - ref["loss"]) <= 1e-4 + 1e-3 * abs(ref["loss"])
+    # dz is rounded to the logits' dtype: bf16 relative error ~2^-8 per element
+    tol = 2e-2 if dtype == "bf16" else 1e-4
+    assert grad_rel_err(dz, rdz) < tol
+    off = m.reshape(-1) == 0
+    assert float(torch.count_nonzero(dz[torch.as_tensor(off).cuda()])) == 0
+
+
+def test_logits_pair_self_distill_and_empty():
+    inp = _pair_case(2, 50, 999, seed=3, same=True)
+    lt, loss, saved, dz, N = _pair_run(inp, 2)
+    assert float(torch.count_nonzero(lt)) == 0 and float(loss) == 0.0 and float(torch.count_nonzero(dz)) == 0
+    inp = _pair_case(2, 50, 999, seed=4, mask="none")
+    lt, loss, saved, dz, N = _pair_run(inp, 1)
+    assert N == 0 and float(loss) == 0.0 and float(torch.count_nonzero(dz)) == 0
+    assert bool(torch.isfinite(dz.float()).all())
+
+
+def test_logits_pair_matches_logits_payload_forward():
+    # the logits-pair forward and the LM-head forward agree when z_s = h_s W_s^T is given explicitly
+    inp = small_case(B=2, Sm1=64, H=128, V=640, payload="logits", mask="random", seed=31)
+    h_s, W_s = inp["h_s"].cuda(), inp["W_s"].cuda()
+    zs = (h_s.double() @ W_s.double().t()).to(torch.bfloat16)
+    mask = inp["mask"].cuda()
+    row_idx, N = rb.compact_rows(mask)
+    a = rb.forward_logits_pair(zs, inp["teacher_logits"].cuda(), 2, 64, row_idx, N, 1)[0]
+    ref = O.forward_logits_pair(to_np(zs), to_np(inp["teacher_logits"]), inp["mask"].numpy(), 1)
+    assert_tok_close(a, ref["loss_tok"])

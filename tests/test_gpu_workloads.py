@@ -178,3 +178,29 @@ def test_long_prompt_compact_equals_full():
     g_dH = to_np(out["dH"][torch.as_tensor(rows, device=out["dH"].device)])
     r_dH = np.stack([dH_ref[int(r)] for r in rows])
     assert np.max(np.abs(g_dH - r_dH)) / np.max(np.abs(r_dH)) < GRAD_RTOL
+
+
+def test_logits_pair_full_size():
+    inp = make_workload("logits_pair", device="cuda")
+    mask = inp["mask"]
+    B, Sm1 = mask.shape
+    row_idx, N = rb.compact_rows(mask)
+    lt, loss, saved = rb.forward_logits_pair(inp["student_logits"], inp["teacher_logits"], B, Sm1, row_idx, N, 1)
+    dz = rb.backward_logits_pair(inp["student_logits"], inp["teacher_logits"], B, Sm1, row_idx, N, 1, saved,
+                                 grad_loss=torch.ones(1, device="cuda"))
+    torch.cuda.synchronize()
+    assert rb.device_error() == 0 and N == B * Sm1
+    rows = np.unique(np.concatenate([[0, N - 1], np.random.RandomState(9).choice(N, 10, replace=False)]))
+    rt = torch.as_tensor(rows, device="cuda")
+    zs = to_np(inp["student_logits"][rt])
+    zt = to_np(inp["teacher_logits"][rt])
+    one = np.ones((1, len(rows)), np.uint8)
+    ref = O.forward_logits_pair(zs, zt, one, O.REDUCE_NONE)
+    rdz = O.backward_logits_pair(zs, zt, one, O.REDUCE_NONE, grad_tok=np.full((1, len(rows)), 1.0 / N))
+    g_tok = to_np(lt.reshape(-1)[rt])
+    assert np.all(np.abs(g_tok - ref["L"]) <= TOK_ATOL + TOK_RTOL * np.abs(ref["L"]))
+    assert np.max(np.abs(to_np(dz[rt]) - rdz)) / np.max(np.abs(rdz)) < 2e-2
+    # every dz row sums to ~0 (sum_v p_s (w - L) = 0), at every size
+    s = dz.float().sum(dim=1).abs()
+    a = dz.float().abs().sum(dim=1)
+    assert float((s / a.clamp_min(1e-30)).max()) < 2e-2
