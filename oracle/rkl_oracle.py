@@ -261,3 +261,45 @@ def backward_logits_pair(z_s, z_t, mask, reduction, grad_loss=1.0, grad_tok=None
         rows = row_idx[c0:c0 + _ROW_CHUNK]
         dz[rows] = dz_rows(_f64(z_s[rows]), _f64(z_t[rows]), g[c0:c0 + len(rows)])
     return dz
+
+
+# ---------------------------------------------------------------------------
+# Student statistics from the same pass.  NeMo RL PR #3978, first
+# implementation note (the kernels sit beside a chunked entropy kernel) and
+# slime PR #2310, Summary (log-probability / entropy computed on the [N, V]
+# compacted rows and scattered back):
+#   entropy        H(p_s) = -sum_v p_s(v) log p_s(v)
+#   target log-p   log p_s(y) for the target token y of the position
+# Both are 0 at masked positions.
+# ---------------------------------------------------------------------------
+
+def student_stats_rows(z_s, targets=None):
+    """(entropy [n], target log-prob [n] or None) of logit rows z_s [n, V]."""
+    lp = log_softmax(_f64(z_s))
+    ent = -np.sum(np.exp(lp) * lp, axis=1)
+    tlp = None
+    if targets is not None:
+        tlp = lp[np.arange(lp.shape[0]), np.asarray(targets)]
+    return ent, tlp
+
+
+def student_stats(h_s, W_s, mask, targets=None, student_logits=None):
+    """Per-position [B, S-1] entropy and target log-prob of the student.
+
+    The student logits are h_s W_s^T, or `student_logits` [T, V] when given
+    (then h_s and W_s are ignored).  targets: [B, S-1] token ids or None."""
+    mask = np.asarray(mask)
+    B, Sm1 = mask.shape
+    row_idx, N = compact_rows(mask)
+    W_s64 = None if student_logits is not None else _f64(W_s)
+    ent = np.zeros(B * Sm1)
+    tlp = np.zeros(B * Sm1)
+    tflat = None if targets is None else np.asarray(targets).reshape(-1)
+    for c0 in range(0, N, _ROW_CHUNK):
+        rows = row_idx[c0:c0 + _ROW_CHUNK]
+        z = _f64(student_logits[rows]) if student_logits is not None else _f64(h_s[rows]) @ W_s64.T
+        e, t = student_stats_rows(z, None if tflat is None else tflat[rows])
+        ent[rows] = e
+        if t is not None:
+            tlp[rows] = t
+    return ent.reshape(B, Sm1), (tlp.reshape(B, Sm1) if targets is not None else None)

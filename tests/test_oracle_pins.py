@@ -212,3 +212,40 @@ def test_logits_pair_masked_rows_zero_and_self_distill(rs):
     assert np.all(dz[mask.reshape(-1) == 0] == 0)
     assert np.all(O.backward_logits_pair(z, z.copy(), mask, 1) == 0)
     assert O.forward_logits_pair(z, z.copy(), mask, 1)["loss"] == 0.0
+
+
+def test_student_entropy_and_logprob_match_scipy(rs):
+    import scipy.special
+    import scipy.stats
+    h_s, W_s, _, _, mask = rand_problem_for_stats(rs)
+    targets = rs.randint(0, W_s.shape[0], size=mask.shape)
+    ent, tlp = O.student_stats(h_s, W_s, mask, targets)
+    z = h_s @ W_s.T
+    ref_ent = scipy.stats.entropy(scipy.special.softmax(z, axis=1), axis=1)
+    ref_lp = scipy.special.log_softmax(z, axis=1)[np.arange(z.shape[0]), targets.reshape(-1)]
+    on = mask.reshape(-1) != 0
+    assert np.max(np.abs(ent.reshape(-1)[on] - ref_ent[on])) < 1e-10
+    assert np.max(np.abs(tlp.reshape(-1)[on] - ref_lp[on])) < 1e-10
+    assert np.all(ent.reshape(-1)[~on] == 0) and np.all(tlp.reshape(-1)[~on] == 0)
+
+
+def test_student_entropy_closed_forms(rs):
+    # uniform student logits: entropy = log V; one-hot limit: entropy -> 0
+    ent, _ = O.student_stats_rows(np.zeros((2, 37)))
+    assert np.max(np.abs(ent - np.log(37))) < 1e-12
+    z = np.full((1, 10), -1e3)
+    z[0, 3] = 0.0
+    ent, tlp = O.student_stats_rows(z, [3])
+    assert abs(ent[0]) < 1e-12 and abs(tlp[0]) < 1e-12
+
+
+def test_student_stats_from_logits_equal_hidden(rs):
+    h_s, W_s, _, _, mask = rand_problem_for_stats(rs)
+    targets = rs.randint(0, W_s.shape[0], size=mask.shape)
+    a = O.student_stats(h_s, W_s, mask, targets)
+    b = O.student_stats(None, None, mask, targets, student_logits=h_s @ W_s.T)
+    assert np.max(np.abs(a[0] - b[0])) < 1e-12 and np.max(np.abs(a[1] - b[1])) < 1e-12
+
+
+def rand_problem_for_stats(rs):
+    return pins.rand_problem(rs, B=3, Sm1=5, H=4, V=23)
