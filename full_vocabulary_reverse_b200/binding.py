@@ -54,6 +54,10 @@ _SIGS = {
                             _vp, _vp, _vp, _vp, _sz, _vp], _i32),
     "rkl_backward": ([_i32, _vp, _vp, _vp, _vp, _i32, _i64, _i64, _i64, _i64, _vp, _i32, _i32,
                       _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp], _i32),
+    "rkl_forward_hidden_ex": ([_vp, _vp, _vp, _vp, _i32, _i64, _i64, _i64, _i64, _vp, _i32, _i32,
+                               _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp], _i32),
+    "rkl_forward_logits_ex": ([_vp, _vp, _vp, _i32, _i64, _i64, _i64, _i64, _vp, _i32, _i32,
+                               _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp], _i32),
     "rkl_forward_logits_pair": ([_vp, _vp, _i32, _i64, _i64, _i64, _vp, _i32, _i32, _vp, _vp, _vp, _vp, _sz, _vp],
                                 _i32),
     "rkl_backward_logits_pair": ([_vp, _vp, _i32, _i64, _i64, _i64, _vp, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _sz,
@@ -143,6 +147,35 @@ def forward_hidden(h_s, h_t, W_s, W_t, B, Sm1, row_idx, N, reduction, workspace=
                                     _ptr(row_idx), N, reduction, _ptr(loss_tok), _ptr(loss), _ptr(saved),
                                     _ptr(ws), ws.numel(), _stream(dev)))
     return loss_tok, loss, saved
+
+
+def forward_with_stats(h_s, teacher, W_s, W_t, B, Sm1, row_idx, N, reduction, targets=None, workspace=None):
+    """Forward of the hidden payload (W_t given) or the logits payload (W_t None)
+    plus the student's per-token entropy and target log-prob.
+    Returns (loss_tok, loss, saved, entropy [B,Sm1], target_logprob [B,Sm1] or None)."""
+    dev = h_s.device
+    T, H = h_s.shape
+    V = W_s.shape[0]
+    dt = _dtype_code(h_s)
+    payload = PAYLOAD_HIDDEN if W_t is not None else PAYLOAD_LOGITS
+    loss_tok = torch.empty((B, Sm1), dtype=torch.float32, device=dev)
+    loss = torch.empty(1, dtype=torch.float32, device=dev)
+    saved = torch.empty((max(N, 1), 3), dtype=torch.float32, device=dev)
+    ent = torch.empty((B, Sm1), dtype=torch.float32, device=dev)
+    tlp = torch.empty((B, Sm1), dtype=torch.float32, device=dev) if targets is not None else None
+    if targets is not None:
+        targets = targets.to(device=dev, dtype=torch.int32).contiguous()
+    ws = workspace if workspace is not None else _workspace(payload, dt, max(N, 1), B, Sm1, H, V, dev)
+    if payload == PAYLOAD_HIDDEN:
+        st = lib().rkl_forward_hidden_ex(_ptr(h_s), _ptr(teacher), _ptr(W_s), _ptr(W_t), dt, B, Sm1, H, V,
+                                         _ptr(row_idx), N, reduction, _ptr(loss_tok), _ptr(loss), _ptr(saved),
+                                         _ptr(targets), _ptr(ent), _ptr(tlp), _ptr(ws), ws.numel(), _stream(dev))
+    else:
+        st = lib().rkl_forward_logits_ex(_ptr(h_s), _ptr(W_s), _ptr(teacher), dt, B, Sm1, H, V, _ptr(row_idx), N,
+                                         reduction, _ptr(loss_tok), _ptr(loss), _ptr(saved), _ptr(targets),
+                                         _ptr(ent), _ptr(tlp), _ptr(ws), ws.numel(), _stream(dev))
+    _check(st)
+    return loss_tok, loss, saved, ent, tlp
 
 
 def forward_logits(h_s, W_s, teacher_logits, B, Sm1, row_idx, N, reduction, workspace=None):

@@ -180,7 +180,7 @@ static Plan make_plan(rkl_payload payload, rkl_dtype dtype, int64_t n_max, int64
   p.off_hct = off;
   if (payload == RKL_PAYLOAD_HIDDEN) off = align256(off + size_t(p.n_pad) * H * p.es);
   p.off_part = off;
-  off = align256(off + size_t(p.S) * 5 * p.n_pad * sizeof(float));
+  off = align256(off + size_t(p.S) * kStatVals * p.n_pad * sizeof(float));
   p.off_rowc = off;
   off = align256(off + size_t(3) * p.n_pad * sizeof(float));
   p.off_lse = off;
@@ -237,7 +237,8 @@ static rkl_status forward_impl(rkl_payload payload, const void* h_s, const void*
                                const void* W_t, rkl_dtype dtype, int64_t B, int64_t Sm1, int64_t H, int64_t V,
                                const int32_t* row_idx, int32_t N, rkl_reduction reduction, float* loss_tok,
                                float* loss, float* saved, void* workspace, size_t workspace_bytes, void* stream_,
-                               bool forward_only_workspace = false) {
+                               bool forward_only_workspace = false, const int32_t* targets = nullptr,
+                               float* entropy = nullptr, float* target_logprob = nullptr) {
   RKL_TRY(check_common(payload, dtype, B, Sm1, H, V, N, reduction));
   RKL_TRY(check_ptr(h_s, "h_s"));
   RKL_TRY(check_ptr(teacher, payload == RKL_PAYLOAD_HIDDEN ? "h_t" : "teacher_logits"));
@@ -248,6 +249,10 @@ static rkl_status forward_impl(rkl_payload payload, const void* h_s, const void*
   RKL_TRY(check_ptr(loss, "loss", false));
   RKL_TRY(check_ptr(saved, "saved", N > 0));
   RKL_TRY(check_ptr(workspace, "workspace"));
+  RKL_TRY(check_ptr(targets, "targets", false));
+  RKL_TRY(check_ptr(entropy, "entropy", false));
+  RKL_TRY(check_ptr(target_logprob, "target_logprob", false));
+  if (target_logprob && !targets) return fail(RKL_ERR_NULL, "target_logprob needs targets");
   const Plan pl = make_plan(payload, dtype, N, H, V);
   // The forward touches only the regions in front of the dz chunk.
   const size_t needed = forward_only_workspace ? pl.off_dz : pl.total;
@@ -260,6 +265,15 @@ static rkl_status forward_impl(rkl_payload payload, const void* h_s, const void*
   const bool bf16 = dtype == RKL_BF16;
   const bool hidden = payload == RKL_PAYLOAD_HIDDEN;
 
+  // Per-row entropy / target log-prob reuse regions of the backward's row
+  // constants (3 x n_pad floats), which the forward does not otherwise use.
+  float* rowc = reinterpret_cast<float*>(ws_at(workspace, pl.off_rowc));
+  float* tlogit = targets ? rowc : nullptr;
+  float* ent_rows = entropy ? rowc + pl.n_pad : nullptr;
+  float* lp_rows = target_logprob ? rowc + 2 * pl.n_pad : nullptr;
+  // A target id outside [0, V) is never found by the kernels: its log-prob
+  // reads back the NaN written here.
+  if (tlogit && N > 0) RKL_CUDA(cudaMemsetAsync(tlogit, 0xFF, size_t(pl.n_pad) * sizeof(float), s));
   if (N > 0) {
     float* part = reinterpret_cast<float*>(ws_at(workspace, pl.off_part));
     float* lse_ext = reinterpret_cast<float*>(ws_at(workspace, pl.off_lse));
@@ -289,6 +303,9 @@ static rkl_status forward_impl(rkl_payload payload, const void* h_s, const void*
         a.teacher_pitch = V;
       }
       a.part = part;
+      a.row_idx = row_idx;
+      a.targets = targets;
+      a.tlogit = tlogit;
       a.N = N;
       a.n_pad = pl.n_pad;
       a.H = static_cast<int>(H);
@@ -316,6 +333,9 @@ static rkl_status forward_impl(rkl_payload payload, const void* h_s, const void*
         a.teacher_pitch = V;
       }
       a.part = part;
+      a.row_idx = row_idx;
+      a.targets = targets;
+      a.tlogit = tlogit;
       a.N = N;
       a.n_pad = pl.n_pad;
       a.H = static_cast<int>(H);
@@ -327,9 +347,11 @@ static rkl_status forward_impl(rkl_payload payload, const void* h_s, const void*
       RKL_CUDA(launch_simt_fused(false, a, dim3(MT, pl.S), s));
     }
     // S4
-    RKL_CUDA(launch_combine(part, pl.S, pl.n_pad, N, hidden, lse_ext, saved, s));
+    RKL_CUDA(launch_combine(part, pl.S, pl.n_pad, N, hidden, lse_ext, tlogit, saved, ent_rows, lp_rows, s));
   }
   if (loss_tok) RKL_CUDA(launch_scatter_loss(saved, row_idx, N, T, loss_tok, s));
+  if (entropy) RKL_CUDA(launch_scatter_rows(ent_rows, row_idx, N, T, entropy, s));
+  if (target_logprob) RKL_CUDA(launch_scatter_rows(lp_rows, row_idx, N, T, target_logprob, s));
   if (loss && reduction != RKL_REDUCE_NONE)
     RKL_CUDA(launch_reduce(saved, row_idx, N, static_cast<int>(B), static_cast<int>(Sm1), reduction, loss, s));
   return RKL_OK;
@@ -600,6 +622,25 @@ rkl_status rkl_forward_logits(const void* h_s, const void* W_s, const void* teac
                               size_t workspace_bytes, void* stream) {
   return forward_impl(RKL_PAYLOAD_LOGITS, h_s, teacher_logits, W_s, nullptr, dtype, B, Sm1, H, V, row_idx, N,
                       reduction, loss_tok, loss, saved, workspace, workspace_bytes, stream);
+}
+
+rkl_status rkl_forward_hidden_ex(const void* h_s, const void* h_t, const void* W_s, const void* W_t, rkl_dtype dtype,
+                                 int64_t B, int64_t Sm1, int64_t H, int64_t V, const int32_t* row_idx, int32_t N,
+                                 rkl_reduction reduction, float* loss_tok, float* loss, float* saved,
+                                 const int32_t* targets, float* entropy, float* target_logprob, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+  return forward_impl(RKL_PAYLOAD_HIDDEN, h_s, h_t, W_s, W_t, dtype, B, Sm1, H, V, row_idx, N, reduction, loss_tok,
+                      loss, saved, workspace, workspace_bytes, stream, false, targets, entropy, target_logprob);
+}
+
+rkl_status rkl_forward_logits_ex(const void* h_s, const void* W_s, const void* teacher_logits, rkl_dtype dtype,
+                                 int64_t B, int64_t Sm1, int64_t H, int64_t V, const int32_t* row_idx, int32_t N,
+                                 rkl_reduction reduction, float* loss_tok, float* loss, float* saved,
+                                 const int32_t* targets, float* entropy, float* target_logprob, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+  return forward_impl(RKL_PAYLOAD_LOGITS, h_s, teacher_logits, W_s, nullptr, dtype, B, Sm1, H, V, row_idx, N,
+                      reduction, loss_tok, loss, saved, workspace, workspace_bytes, stream, false, targets, entropy,
+                      target_logprob);
 }
 
 rkl_status rkl_backward(rkl_payload payload, const void* h_s, const void* teacher, const void* W_s, const void* W_t,

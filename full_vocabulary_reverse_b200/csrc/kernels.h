@@ -49,6 +49,7 @@ constexpr int kFBN = 256;      // vocab columns per fused pair tile
 constexpr int kBK = 64;        // K per pipeline stage (128 B of bf16)
 constexpr int kGradBN = 256;   // H columns per gradient tile
 constexpr int kGroupTiles = 4;  // 256-column vocab tiles per forward statistics group (1024 columns)
+constexpr int kStatVals = 6;    // per slot: m_s, S_s, A, m_t, S_t, sum e^(z_s-m_s) z_s
 
 // ---------------------------------------------------------------- tcgen05
 struct FusedArgs {
@@ -58,8 +59,11 @@ struct FusedArgs {
   const uint16_t* teacher;           // logits payload: teacher logits [T, V] bf16
   const int32_t* teacher_rows;       // logits payload: row_idx (nullptr = identity)
   long long teacher_pitch;           // elements per teacher row
-  float* part;                       // stats: [G][5][n_pad]
+  float* part;                       // stats: [2G][kStatVals][n_pad]
   const float* rowc;                 // dz: [3][n_pad]: lse_s*log2e, cst, g
+  const int32_t* row_idx;            // stats: compacted row -> token position
+  const int32_t* targets;            // stats: target token id per position (nullable)
+  float* tlogit;                     // stats: z_s at the target column [n_pad]
   int N, n_pad, H, V, KB;
   int IT;                            // 256-column vocab tiles per row tile in this launch
   int vt_base;                       // first 256-column vocab tile of this launch
@@ -97,8 +101,12 @@ cudaError_t launch_gather(const void* h_s, const void* h_t, void* hc_s, void* hc
 cudaError_t launch_teacher_lse(const void* logits, bool bf16, const int32_t* row_idx, int N, int V,
                                long long pitch, float* lse_t, cudaStream_t s);
 cudaError_t launch_combine(const float* part, int S, int n_pad, int N, bool teacher_from_part,
-                           const float* lse_t_ext, float* saved, cudaStream_t s);
+                           const float* lse_t_ext, const float* tlogit, float* saved, float* ent_rows,
+                           float* lp_rows, cudaStream_t s);
 cudaError_t launch_scatter_loss(const float* saved, const int32_t* row_idx, int N, long long T, float* loss_tok,
+                                cudaStream_t s);
+// out[t] = rows[k] where t = row_idx[k], else 0 (per-token [B, S-1] scatter)
+cudaError_t launch_scatter_rows(const float* rows, const int32_t* row_idx, int N, long long T, float* out,
                                 cudaStream_t s);
 cudaError_t launch_reduce(const float* saved, const int32_t* row_idx, int N, int B, int Sm1, int reduction,
                           float* loss, cudaStream_t s);
@@ -120,6 +128,7 @@ struct SimtArgs {
   const int32_t* teacher_rows;
   long long teacher_pitch;
   float* part; const float* rowc;
+  const int32_t* row_idx; const int32_t* targets; float* tlogit;
   float* dz;                          // dz chunk [N, cw] fp32
   int N, n_pad, H, V, S, IT, vt_base, chunk_v0, cw;
   int ng;

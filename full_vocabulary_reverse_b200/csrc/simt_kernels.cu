@@ -33,7 +33,12 @@ __global__ void __launch_bounds__(256) simt_fused_kernel(const SimtArgs a) {
     u1 = static_cast<int>((static_cast<long long>(blockIdx.x + 1) * total) / gridDim.x);
   }
 
-  float m_s = -INFINITY, S_s = 0.f, A = 0.f, m_t = -INFINITY, S_t = 0.f;
+  float m_s = -INFINITY, S_s = 0.f, A = 0.f, m_t = -INFINITY, S_t = 0.f, Bz = 0.f;
+  int tgt = -1;
+  if (!DZ && tid < TB && a.targets != nullptr) {
+    const int r = (u0 / a.IT) * TB + tid;
+    if (r < a.N) tgt = a.targets[a.row_idx[r]];
+  }
   for (int u = u0; u < u1; ++u) {
     const int m0 = (u / a.IT) * TB;
     const int v0 = (a.vt_base + u % a.IT) * TB;
@@ -90,6 +95,7 @@ __global__ void __launch_bounds__(256) simt_fused_kernel(const SimtArgs a) {
         const float sc_s = ex2((m_s - nm_s) * kLog2e), sc_t = ex2((m_t - nm_t) * kLog2e);
         S_s *= sc_s;
         A *= sc_s;
+        Bz *= sc_s;
         S_t *= sc_t;
         m_s = nm_s;
         m_t = nm_t;
@@ -99,7 +105,10 @@ __global__ void __launch_bounds__(256) simt_fused_kernel(const SimtArgs a) {
           S_s += e;
           S_t += f;
           A = fmaf(e, Zs[r][j] - Zt[r][j], A);
+          Bz = fmaf(e, Zs[r][j], Bz);
         }
+        const unsigned d = static_cast<unsigned>(tgt - v0);
+        if (tgt >= 0 && d < static_cast<unsigned>(TB)) a.tlogit[m0 + r] = Zs[r][d];
       } else if (m0 + r < a.N) {
         const float lse2 = a.rowc[m0 + r], cst = a.rowc[a.n_pad + m0 + r], g = a.rowc[2 * a.n_pad + m0 + r];
         float* out = a.dz + static_cast<long long>(m0 + r) * a.cw + (v0 - a.chunk_v0);
@@ -112,12 +121,13 @@ __global__ void __launch_bounds__(256) simt_fused_kernel(const SimtArgs a) {
     __syncthreads();
   }
   if (!DZ && tid < TB && u1 > u0) {
-    float* base = a.part + static_cast<size_t>(split) * 5 * a.n_pad + (u0 / a.IT) * TB + tid;
+    float* base = a.part + static_cast<size_t>(split) * kStatVals * a.n_pad + (u0 / a.IT) * TB + tid;
     base[0] = m_s;
     base[a.n_pad] = S_s;
     base[2 * a.n_pad] = A;
     base[3 * a.n_pad] = m_t;
     base[4 * a.n_pad] = S_t;
+    base[5 * a.n_pad] = Bz;
   }
 }
 

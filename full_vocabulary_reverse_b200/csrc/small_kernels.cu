@@ -236,7 +236,7 @@ __global__ void __launch_bounds__(256) teacher_lse_kernel(const T* __restrict__ 
 // statistics go through identical operations, so teacher == student gives
 // L = 0 exactly.
 struct Stat3 {
-  float m, S, A;
+  float m, S, A, Bz;
 };
 
 __device__ __forceinline__ void merge3(Stat3& a, const Stat3& b) {
@@ -245,27 +245,31 @@ __device__ __forceinline__ void merge3(Stat3& a, const Stat3& b) {
   const float ea = expf(a.m - nm), eb = expf(b.m - nm);
   a.S = a.S * ea + b.S * eb;
   a.A = a.A * ea + b.A * eb;
+  a.Bz = a.Bz * ea + b.Bz * eb;
   a.m = nm;
 }
 
+// Optional student statistics of row k (nullable outputs): entropy
+// lse_s - sum p_s z_s = lse_s - Bz / S_s, and target log-prob tlogit - lse_s.
 __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ part, int S, int n_pad, int N,
                                                       int teacher_from_part, const float* __restrict__ lse_ext,
-                                                      float* __restrict__ saved) {
+                                                      const float* __restrict__ tlogit, float* __restrict__ saved,
+                                                      float* __restrict__ ent_rows, float* __restrict__ lp_rows) {
   const int lane = threadIdx.x & 31;
   const int k = blockIdx.x * 8 + (threadIdx.x >> 5);
   if (k >= N) return;
-  Stat3 s{-INFINITY, 0.f, 0.f}, t{-INFINITY, 0.f, 0.f};
+  Stat3 s{-INFINITY, 0.f, 0.f, 0.f}, t{-INFINITY, 0.f, 0.f, 0.f};
   for (int g = lane; g < S; g += 32) {
-    const float* b = part + static_cast<size_t>(g) * 5 * n_pad + k;
-    merge3(s, Stat3{b[0], b[n_pad], b[2 * n_pad]});
-    if (teacher_from_part) merge3(t, Stat3{b[3 * n_pad], b[4 * n_pad], 0.f});
+    const float* b = part + static_cast<size_t>(g) * kStatVals * n_pad + k;
+    merge3(s, Stat3{b[0], b[n_pad], b[2 * n_pad], b[5 * n_pad]});
+    if (teacher_from_part) merge3(t, Stat3{b[3 * n_pad], b[4 * n_pad], 0.f, 0.f});
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     merge3(s, Stat3{__shfl_xor_sync(0xffffffffu, s.m, o), __shfl_xor_sync(0xffffffffu, s.S, o),
-                    __shfl_xor_sync(0xffffffffu, s.A, o)});
+                    __shfl_xor_sync(0xffffffffu, s.A, o), __shfl_xor_sync(0xffffffffu, s.Bz, o)});
     merge3(t, Stat3{__shfl_xor_sync(0xffffffffu, t.m, o), __shfl_xor_sync(0xffffffffu, t.S, o),
-                    __shfl_xor_sync(0xffffffffu, t.A, o)});
+                    __shfl_xor_sync(0xffffffffu, t.A, o), __shfl_xor_sync(0xffffffffu, t.Bz, o)});
   }
   if (lane == 0) {
     const float lse_s = s.m + logf(s.S);
@@ -274,7 +278,18 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
     saved[3 * k + 0] = lse_s;
     saved[3 * k + 1] = lse_t;
     saved[3 * k + 2] = L;
+    if (ent_rows) ent_rows[k] = lse_s - s.Bz / s.S;
+    if (lp_rows) lp_rows[k] = tlogit[k] - lse_s;
   }
+}
+
+// out[t] = rows[k] if t = row_idx[k] else exactly 0.
+__global__ void scatter_rows_kernel(const float* __restrict__ rows, const int32_t* __restrict__ row_idx, int N,
+                                    long long T, float* __restrict__ out) {
+  const long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (t >= T) return;
+  const int k = lower_bound_i32(row_idx, N, t);
+  out[t] = (k < N && row_idx[k] == t) ? rows[k] : 0.f;
 }
 
 // loss_tok[t] = L of t if t is trainable else exactly 0.
@@ -614,10 +629,18 @@ cudaError_t launch_teacher_lse(const void* logits, bool bf16, const int32_t* row
 }
 
 cudaError_t launch_combine(const float* part, int S, int n_pad, int N, bool teacher_from_part, const float* lse_ext,
-                           float* saved, cudaStream_t s) {
+                           const float* tlogit, float* saved, float* ent_rows, float* lp_rows, cudaStream_t s) {
   if (N <= 0) return cudaSuccess;
   LaunchScope scope(K_COMBINE, s);
-  combine_kernel<<<(N + 7) / 8, 256, 0, s>>>(part, S, n_pad, N, teacher_from_part ? 1 : 0, lse_ext, saved);
+  combine_kernel<<<(N + 7) / 8, 256, 0, s>>>(part, S, n_pad, N, teacher_from_part ? 1 : 0, lse_ext, tlogit, saved,
+                                             ent_rows, lp_rows);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_scatter_rows(const float* rows, const int32_t* row_idx, int N, long long T, float* out,
+                                cudaStream_t s) {
+  LaunchScope scope(K_SCATTER_LOSS, s);
+  scatter_rows_kernel<<<static_cast<unsigned>((T + 255) / 256), 256, 0, s>>>(rows, row_idx, N, T, out);
   return cudaGetLastError();
 }
 

@@ -74,7 +74,7 @@ constexpr size_t fused_smem() {
 
 // ---- online statistics of one 32-column chunk (all columns valid)
 struct RowStats {
-  float m_s, S_s, A, m_t, S_t;
+  float m_s, S_s, A, m_t, S_t, Bz;  // Bz = sum e^(z_s - m_s) z_s (student entropy)
 };
 
 __device__ __forceinline__ void stats_chunk(RowStats& st, const float* zs, const float* zt) {
@@ -88,11 +88,12 @@ __device__ __forceinline__ void stats_chunk(RowStats& st, const float* zs, const
   const float a_s = ex2((st.m_s - nm_s) * kLog2e), a_t = ex2((st.m_t - nm_t) * kLog2e);
   st.S_s *= a_s;
   st.A *= a_s;
+  st.Bz *= a_s;
   st.S_t *= a_t;
   st.m_s = nm_s;
   st.m_t = nm_t;
   const float ms2 = nm_s * kLog2e, mt2 = nm_t * kLog2e;
-  float s0 = 0.f, s1 = 0.f, t0 = 0.f, t1 = 0.f, q0 = 0.f, q1 = 0.f;
+  float s0 = 0.f, s1 = 0.f, t0 = 0.f, t1 = 0.f, q0 = 0.f, q1 = 0.f, b0 = 0.f, b1 = 0.f;
 #pragma unroll
   for (int j = 0; j < 32; j += 2) {
     const float e0 = ex2(fmaf(zs[j], kLog2e, -ms2));
@@ -102,13 +103,16 @@ __device__ __forceinline__ void stats_chunk(RowStats& st, const float* zs, const
     s0 += e0;
     t0 += f0;
     q0 = fmaf(e0, zs[j] - zt[j], q0);
+    b0 = fmaf(e0, zs[j], b0);
     s1 += e1;
     t1 += f1;
     q1 = fmaf(e1, zs[j + 1] - zt[j + 1], q1);
+    b1 = fmaf(e1, zs[j + 1], b1);
   }
   st.S_s += s0 + s1;
   st.S_t += t0 + t1;
   st.A += q0 + q1;
+  st.Bz += b0 + b1;
 }
 
 // Same for a chunk whose first nv (< 32) columns are inside the vocabulary
@@ -125,6 +129,7 @@ __device__ __forceinline__ void stats_chunk_tail(RowStats& st, const float* zs, 
   const float a_s = ex2((st.m_s - nm_s) * kLog2e), a_t = ex2((st.m_t - nm_t) * kLog2e);
   st.S_s *= a_s;
   st.A *= a_s;
+  st.Bz *= a_s;
   st.S_t *= a_t;
   st.m_s = nm_s;
   st.m_t = nm_t;
@@ -137,7 +142,20 @@ __device__ __forceinline__ void stats_chunk_tail(RowStats& st, const float* zs, 
       st.S_s += e;
       st.S_t += f;
       st.A = fmaf(e, zs[j] - zt[j], st.A);
+      st.Bz = fmaf(e, zs[j], st.Bz);
     }
+}
+
+// z_s of the target column if it falls in this 32-column chunk (rare: one
+// chunk per row), written once per row.
+__device__ __forceinline__ void pick_target(const float* zs, int tgt, int col0, float* out) {
+  const unsigned d = static_cast<unsigned>(tgt - col0);
+  if (d < 32u) {
+    float v = 0.f;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v = (d == static_cast<unsigned>(j)) ? zs[j] : v;
+    *out = v;
+  }
 }
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
@@ -344,6 +362,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_kernel(const __grid_co
     const uint32_t acc_empty0 = mapa_shared(smem_u32(acc_empty), 0);
     int cur_m0 = -1;
     float lse2 = 0.f, cst = 0.f, g_row = 0.f;
+    int tgt = -1;  // target column of this row (forward with targets), else -1
     const uint16_t* trow = nullptr;
     int box = 0;
     int it = 0;
@@ -359,6 +378,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_kernel(const __grid_co
           lse2 = p.rowc[r];
           cst = p.rowc[p.n_pad + r];
           g_row = p.rowc[2 * p.n_pad + r];
+        } else {
+          tgt = (p.targets != nullptr && r < p.N) ? p.targets[p.row_idx[r]] : -1;
         }
         if (NG == 1) {
           trow = nullptr;
@@ -368,7 +389,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_kernel(const __grid_co
           }
         }
       }
-      RowStats st{-INFINITY, 0.f, 0.f, -INFINITY, 0.f};
+      RowStats st{-INFINITY, 0.f, 0.f, -INFINITY, 0.f, 0.f};
       for (int vt = g * p.GT; vt < vt_end; ++vt, ++it) {
         const int v0 = (p.vt_base + vt) * kFBN + half * (kFBN / 2);  // this warp's first column
         // Teacher logits of this row (logits payload): 32 bf16 per chunk,
@@ -431,6 +452,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_kernel(const __grid_co
               stats_chunk(st, zs, zt);
             else if (nv > 0)
               stats_chunk_tail(st, zs, zt, nv);
+            if (tgt >= 0) pick_target(zs, tgt, v0 + c * 32, p.tlogit + m0 + row);
           } else {
             // dz = g * p_s * ((z_s - z_t) + cst); columns past the chunk end
             // are clipped by the TMA store.
@@ -469,12 +491,13 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_kernel(const __grid_co
       }
       if (!DZ && ok) {
         // statistics slot (group, column half): 2 slots per group
-        float* base = p.part + static_cast<size_t>(2 * g + half) * 5 * p.n_pad + m0 + row;
+        float* base = p.part + static_cast<size_t>(2 * g + half) * kStatVals * p.n_pad + m0 + row;
         base[0] = st.m_s;
         base[p.n_pad] = st.S_s;
         base[2 * p.n_pad] = st.A;
         base[3 * p.n_pad] = st.m_t;
         base[4 * p.n_pad] = st.S_t;
+        base[5 * p.n_pad] = st.Bz;
       }
     }
     if (DZ) {

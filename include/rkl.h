@@ -129,6 +129,33 @@ rkl_status rkl_forward_logits(const void* h_s, const void* W_s,
                               float* loss_tok, float* loss, float* saved,
                               void* workspace, size_t workspace_bytes, void* stream);
 
+/* rkl_forward_hidden / rkl_forward_logits plus per-token statistics of the
+ * student distribution from the same pass (PR #3978, implementation note 1:
+ * the kernels sit beside a chunked entropy kernel; slime PR #2310, Summary:
+ * log-probability / entropy on the compacted rows, scattered back):
+ *   targets        [B, Sm1] int32 target token id per position (nullable;
+ *                  required for target_logprob; ids outside [0, V) give NaN)
+ *   entropy        [B, Sm1] fp32 H(p_s) = -sum_v p_s log p_s (nullable)
+ *   target_logprob [B, Sm1] fp32 log p_s(targets) (nullable)
+ * Both outputs are exactly 0 at masked positions.  The loss outputs are
+ * identical to those of the plain entry points. */
+rkl_status rkl_forward_hidden_ex(const void* h_s, const void* h_t,
+                                 const void* W_s, const void* W_t, rkl_dtype dtype,
+                                 int64_t B, int64_t Sm1, int64_t H, int64_t V,
+                                 const int32_t* row_idx, int32_t N,
+                                 rkl_reduction reduction,
+                                 float* loss_tok, float* loss, float* saved,
+                                 const int32_t* targets, float* entropy, float* target_logprob,
+                                 void* workspace, size_t workspace_bytes, void* stream);
+rkl_status rkl_forward_logits_ex(const void* h_s, const void* W_s,
+                                 const void* teacher_logits, rkl_dtype dtype,
+                                 int64_t B, int64_t Sm1, int64_t H, int64_t V,
+                                 const int32_t* row_idx, int32_t N,
+                                 rkl_reduction reduction,
+                                 float* loss_tok, float* loss, float* saved,
+                                 const int32_t* targets, float* entropy, float* target_logprob,
+                                 void* workspace, size_t workspace_bytes, void* stream);
+
 /* S5-S7, backward of either payload (PR #3978, first implementation note:
  * dL/dz_s = p_s (w - L), log-softmaxes recomputed, nothing [N, V] kept).
  *   payload   RKL_PAYLOAD_HIDDEN: teacher = h_t [T, H], W_t [V, H]

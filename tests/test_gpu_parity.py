@@ -236,3 +236,31 @@ def test_logits_pair_matches_logits_payload_forward():
     a = rb.forward_logits_pair(zs, inp["teacher_logits"].cuda(), 2, 64, row_idx, N, 1)[0]
     ref = O.forward_logits_pair(to_np(zs), to_np(inp["teacher_logits"]), inp["mask"].numpy(), 1)
     assert_tok_close(a, ref["loss_tok"])
+
+
+# ---------------------------------------------------------------- student entropy / target log-prob
+@pytest.mark.parametrize("payload,dtype,V", [("hidden", "bf16", 1000), ("logits", "bf16", 1200),
+                                             ("hidden", "fp32", 333), ("logits", "fp32", 520)])
+def test_student_entropy_and_target_logprob(payload, dtype, V):
+    H = 128 if dtype == "bf16" else 40
+    inp = small_case(B=3, Sm1=90, H=H, V=V, dtype=dtype, payload=payload, mask="random", seed=V + 7)
+    rs = np.random.RandomState(V)
+    targets = torch.from_numpy(rs.randint(0, V, size=(3, 90)).astype(np.int32))
+    mask = inp["mask"].cuda()
+    row_idx, N = rb.compact_rows(mask)
+    teacher = inp["h_t"].cuda() if payload == "hidden" else inp["teacher_logits"].cuda()
+    W_t = inp["W_t"].cuda() if payload == "hidden" else None
+    lt, loss, saved, ent, tlp = rb.forward_with_stats(inp["h_s"].cuda(), teacher, inp["W_s"].cuda(), W_t, 3, 90,
+                                                      row_idx, N, 1, targets=targets)
+    torch.cuda.synchronize()
+    assert rb.device_error() == 0
+    h_s, W_s = to_np(inp["h_s"]), to_np(inp["W_s"])
+    m = inp["mask"].numpy()
+    r_ent, r_tlp = O.student_stats(h_s, W_s, m, targets.numpy())
+    # the loss outputs are unchanged by the extra statistics
+    assert_tok_close(lt, run_oracle(inp, 1, backward=False)["loss_tok"])
+    assert np.max(np.abs(to_np(ent) - r_ent)) <= 1e-4 + 1e-3 * np.max(np.abs(r_ent))
+    assert np.all(np.abs(to_np(tlp) - r_tlp) <= 1e-4 + 1e-3 * np.abs(r_tlp))
+    off = torch.as_tensor(m.reshape(-1) == 0)
+    assert float(torch.count_nonzero(ent.reshape(-1).cpu()[off])) == 0
+    assert float(torch.count_nonzero(tlp.reshape(-1).cpu()[off])) == 0
