@@ -36,7 +36,7 @@ __device__ int g_dev_err = 0;
 
 namespace {
 
-constexpr int kThreads = 192;       // gradient kernel: producer, MMA, 4 epilogue warps
+constexpr int kThreads = 64 + 32 * 8;  // gradient kernel: producer, MMA, 8 epilogue warps
 constexpr int kFusedEpi = 8;        // fused kernels: 2 epilogue warps per TMEM lane quarter
 constexpr int kFusedThreads = 64 + 32 * kFusedEpi;
 constexpr int kStgBoxBytes = 4096;  // one 32-row staging box per epilogue warp
@@ -567,11 +567,11 @@ __global__ void __launch_bounds__(kThreads, 1) grad_kernel(const __grid_constant
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&acc_full[i], 1);
-      mbar_init(&acc_empty[i], 8);  // 4 epilogue warps in each CTA of the pair
+      mbar_init(&acc_empty[i], 16);  // 8 epilogue warps in each CTA of the pair
     }
     for (int i = 0; i < kSched; ++i) {
       mbar_init(&sched_full[i], 1);
-      mbar_init(&sched_empty[i], 1 + 4 + 1 + 4);  // leader MMA + epilogues, peer producer + epilogues
+      mbar_init(&sched_empty[i], 1 + 8 + 1 + 8);  // leader MMA + epilogues, peer producer + epilogues
     }
     mbar_init(tear, 1);
     *abort_flag = 0;
@@ -725,7 +725,10 @@ __global__ void __launch_bounds__(kThreads, 1) grad_kernel(const __grid_constant
       if (!mbar_wait(tear, 0, &never)) atomicOr(&g_dev_err, ERR_WAIT_TEARDOWN);
     }
   } else {
+    // Warp w reads TMEM lane quarter w % 4 and columns [128 h, 128 h + 128)
+    // of the 256-column accumulator, h = (w - 2) / 4.
     const int q = warp & 3;
+    const int half = (warp - 2) >> 2;
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
     const uint32_t sched_empty0 = mapa_shared(smem_u32(sched_empty), 0);
     const uint32_t acc_empty0 = mapa_shared(smem_u32(acc_empty), 0);
@@ -756,21 +759,22 @@ __global__ void __launch_bounds__(kThreads, 1) grad_kernel(const __grid_constant
         break;
       }
       tc_fence_after();
-      const uint32_t tb = tmem_base + lane_off + acc * kGradBN;
+      const uint32_t tb = tmem_base + lane_off + acc * kGradBN + half * (kGradBN / 2);
       const int rows = mtile * 2 * kBM + rank * kBM + q * 32;
       const int row0 = is_h ? rows : p.cv0 + rows;
+      const int c0 = n0 + half * (kGradBN / 2);
 #pragma unroll 1
-      for (int c = 0; c < kGradBN / 32; ++c) {
+      for (int c = 0; c < kGradBN / 2 / 32; ++c) {
         float v[32];
         tmem_ld_32x32(tb + c * 32, v);
         tmem_wait_ld();
-        if (c == kGradBN / 32 - 1) {
+        if (c == kGradBN / 2 / 32 - 1) {
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive_cluster(acc_empty0 + acc * 8);
         }
-        uint8_t* buf = stg + (q * 2 + (box & 1)) * kStgBoxBytes;
-        if (lane == 0) bulk_wait_read<1>();
+        uint8_t* buf = stg + (warp - 2) * kStgBoxBytes;  // one staging box per warp
+        if (lane == 0) bulk_wait_read<0>();
         __syncwarp();
         const uint32_t rbase = smem_u32(buf) + lane * 128;
 #pragma unroll
@@ -781,11 +785,11 @@ __global__ void __launch_bounds__(kThreads, 1) grad_kernel(const __grid_constant
         __syncwarp();
         if (lane == 0) {
           if (!is_h)
-            tma_store_2d(&p.tm_dw, buf, n0 + c * 32, row0);
+            tma_store_2d(&p.tm_dw, buf, c0 + c * 32, row0);
           else if (p.dh_accumulate)
-            tma_reduce_add_2d(&p.tm_dh, buf, n0 + c * 32, row0);
+            tma_reduce_add_2d(&p.tm_dh, buf, c0 + c * 32, row0);
           else
-            tma_store_2d(&p.tm_dh, buf, n0 + c * 32, row0);
+            tma_store_2d(&p.tm_dh, buf, c0 + c * 32, row0);
           bulk_commit();
         }
         ++box;
