@@ -23,7 +23,8 @@
  *  - All pointers are DEVICE pointers unless stated, owned by the caller.  The
  *    library never allocates device memory: scratch comes from the caller's
  *    workspace (size from rkl_workspace_size).  Teacher inputs are read-only
- *    and get no gradient (PR #3978: the teacher LM head is "a plain tensor").
+ *    and get no gradient (PR #3978, implementation note 5: the teacher LM head
+ *    is held outside the trained parameters).
  *  - `stream` is a cudaStream_t (NULL = legacy default stream).  All work is
  *    enqueued on it; no entry point synchronises the host except
  *    rkl_device_error.
@@ -107,8 +108,8 @@ rkl_status rkl_compact_rows(const uint8_t* mask, int64_t B, int64_t Sm1,
  *   loss_tok [B, Sm1]  per-token loss, exact 0 at masked positions (nullable)
  *   loss     [1]       reduced loss (nullable; ignored for RKL_REDUCE_NONE)
  *   saved    [N, 3]    per-row (lse_s, lse_t, L) kept for rkl_backward
- * N = 0 gives loss 0 and all-zero loss_tok without NaN (slime PR #2310: empty
- * masks keep zero-gradient connections). */
+ * N = 0 gives loss 0 and all-zero loss_tok without NaN (slime PR #2310, Summary:
+ * an empty mask still yields a well-defined zero gradient). */
 rkl_status rkl_forward_hidden(const void* h_s, const void* h_t,
                               const void* W_s, const void* W_t, rkl_dtype dtype,
                               int64_t B, int64_t Sm1, int64_t H, int64_t V,

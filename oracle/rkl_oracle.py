@@ -25,12 +25,13 @@ What it computes, and where the pages define it:
   nested per-sequence mean (``token_level_loss=false``).
 * "fix(megatron): compact actor logits before projection" (slime PR #2310),
   Summary: only the N loss-masked rows are projected; scalar results are
-  scattered back to the [B, S-1] layout; empty masks keep zero-gradient
-  connections.
+  scattered back to the [B, S-1] layout; an empty mask still yields a
+  well-defined zero gradient.
 
 Readings where the pages are silent (each is listed in the design doc):
 
-* Only the student gets gradients (the teacher LM head is "a plain tensor");
+* Only the student gets gradients (the teacher LM head is held as an ordinary
+  tensor outside the trained parameters);
   gradients flow to h_s and W_s.
 * The nested mean averages over sequences that have at least one trainable
   position; with none at all the loss is 0.  The token mean with N = 0 is 0.
@@ -224,10 +225,11 @@ def dz_rows(z_s, z_t, g):
 
 
 # ---------------------------------------------------------------------------
-# Both sides as logits.  NeMo RL PR #3978, payload bullet 2 calls the logits
-# payload the numerical-reference path; when the student's logits are also
-# given as a [T, V] tensor the loss and its gradient w.r.t. those logits are
-# the same objective and the same shared backward, with no LM head.
+# Both sides as logits.  NeMo RL PR #3978, payload bullet 2 presents the
+# logits payload as a path for numerical checks and fallback, not production;
+# when the student's logits are also given as a [T, V] tensor the loss and its
+# gradient w.r.t. those logits are the same objective and the same shared
+# backward, with no LM head.
 # ---------------------------------------------------------------------------
 
 def forward_logits_pair(z_s, z_t, mask, reduction):
