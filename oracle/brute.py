@@ -79,3 +79,31 @@ def compact_rows(mask):
                 out.append(k)
             k += 1
     return out
+
+
+def loss_tokens_multi(h_s, W_s, h_t, W_t_list, teacher_idx, mask):
+    """Per-position loss [B][S-1] with the teacher head W_t_list[k] chosen by
+    the position's teacher index k; masked positions are 0."""
+    B = len(mask)
+    Sm1 = len(mask[0])
+    out = [[0.0] * Sm1 for _ in range(B)]
+    for b in range(B):
+        for t in range(Sm1):
+            if mask[b][t]:
+                r = b * Sm1 + t
+                W_t = W_t_list[teacher_idx[b][t]]
+                out[b][t] = kl_row(logits_row(h_s[r], W_s), logits_row(h_t[r], W_t))
+    return out
+
+
+def count_rows_per_teacher(mask, teacher_idx, n_teachers):
+    counts = [0] * n_teachers
+    bad = 0
+    for mrow, trow in zip(mask, teacher_idx):
+        for m, k in zip(mrow, trow):
+            if m:
+                if 0 <= k < n_teachers:
+                    counts[k] += 1
+                else:
+                    bad += 1
+    return counts, bad

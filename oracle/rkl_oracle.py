@@ -305,3 +305,82 @@ def student_stats(h_s, W_s, mask, targets=None, student_logits=None):
         if t is not None:
             tlp[rows] = t
     return ent.reshape(B, Sm1), (tlp.reshape(B, Sm1) if targets is not None else None)
+
+
+# ---------------------------------------------------------------------------
+# Several teachers, one per row.  NeMo RL PR #3978, first-version limits: the
+# first version takes exactly one teacher checkpoint, and the payload is laid
+# out so that a per-row teacher index can be added.  Reading: every position
+# carries an index k in [0, n_teachers); the teacher logits of a trainable
+# row r are z_t = h_t[r] W_t[k_r]^T with W_t[k] the LM head of teacher k (all
+# teachers share the vocabulary and the width of h_t); the per-row objective,
+# its backward and the reductions are unchanged.  The index of a masked
+# position is never read.
+# ---------------------------------------------------------------------------
+
+def count_rows_per_teacher(mask, teacher_idx, n_teachers):
+    """(counts [n_teachers], n_bad): trainable rows per teacher, and trainable
+    rows whose teacher index lies outside [0, n_teachers)."""
+    flat = np.asarray(mask).reshape(-1) != 0
+    tid = np.asarray(teacher_idx).reshape(-1)[flat]
+    ok = (tid >= 0) & (tid < n_teachers)
+    counts = np.bincount(tid[ok], minlength=n_teachers)[:n_teachers]
+    return counts.astype(np.int64), int(np.count_nonzero(~ok))
+
+
+def _multi_teacher_logits(rows, h_t, W_t64, tid_flat):
+    """z_t of the selected rows, each projected with its own teacher's head."""
+    k = tid_flat[rows]
+    z_t = np.zeros((len(rows), W_t64.shape[1]))
+    for g in np.unique(k):
+        sel = k == g
+        z_t[sel] = _f64(h_t[rows[sel]]) @ W_t64[g].T
+    return z_t
+
+
+def forward_multi(h_s, W_s, h_t, W_t, teacher_idx, mask, reduction):
+    """Forward with a teacher per row.  W_t [n_teachers, V, H]; teacher_idx
+    [B, S-1] ints.  Same outputs as forward()."""
+    mask = np.asarray(mask)
+    B, Sm1 = mask.shape
+    row_idx, N = compact_rows(mask)
+    W_s64 = _f64(W_s)
+    W_t64 = _f64(W_t)
+    tid = np.asarray(teacher_idx).reshape(-1)
+    L = np.zeros(N)
+    lse_s = np.zeros(N)
+    lse_t = np.zeros(N)
+    for c0 in range(0, N, _ROW_CHUNK):
+        rows = row_idx[c0:c0 + _ROW_CHUNK]
+        n = len(rows)
+        z_s = _f64(h_s[rows]) @ W_s64.T
+        z_t = _multi_teacher_logits(rows, h_t, W_t64, tid)
+        L[c0:c0 + n], lse_s[c0:c0 + n], lse_t[c0:c0 + n] = per_row_kl(z_s, z_t)
+    loss_tok = np.zeros(B * Sm1)
+    loss_tok[row_idx] = L
+    loss = reduce_loss(L, row_idx, B, Sm1, reduction)
+    return {"loss_tok": loss_tok.reshape(B, Sm1), "loss": loss, "L": L,
+            "lse_s": lse_s, "lse_t": lse_t, "row_idx": row_idx, "N": N}
+
+
+def backward_multi(h_s, W_s, h_t, W_t, teacher_idx, mask, reduction, grad_loss=1.0, grad_tok=None):
+    """(dH_s [T, H], dW_s [V, H]) with a teacher per row; the student side of
+    the chain rule is that of backward()."""
+    mask = np.asarray(mask)
+    B, Sm1 = mask.shape
+    row_idx, N = compact_rows(mask)
+    W_s64 = _f64(W_s)
+    W_t64 = _f64(W_t)
+    tid = np.asarray(teacher_idx).reshape(-1)
+    T, H = np.asarray(h_s).shape
+    g = row_weights(row_idx, B, Sm1, reduction, grad_loss, grad_tok)
+    dH = np.zeros((T, H))
+    dW = np.zeros(W_s64.shape)
+    for c0 in range(0, N, _ROW_CHUNK):
+        rows = row_idx[c0:c0 + _ROW_CHUNK]
+        z_s = _f64(h_s[rows]) @ W_s64.T
+        z_t = _multi_teacher_logits(rows, h_t, W_t64, tid)
+        dz = dz_rows(z_s, z_t, g[c0:c0 + len(rows)])
+        dH[rows] = dz @ W_s64
+        dW += dz.T @ _f64(h_s[rows])
+    return dH, dW

@@ -291,3 +291,86 @@ def logits_pair_matches_hidden_chain_rule(O, rs):
     dz = O.backward_logits_pair(z_s, z_t, mask, 2)
     return max(float(np.max(np.abs(a["loss_tok"] - b["loss_tok"]))), abs(a["loss"] - b["loss"]),
                float(np.max(np.abs(dH - dz @ W_s))), float(np.max(np.abs(dW - dz.T @ h_s))))
+
+
+# ----------------------------------------------------------------- several teachers
+
+def rand_multi_problem(rs, B=3, Sm1=4, H=3, V=9, n_teachers=3):
+    T = B * Sm1
+    h_s = rs.normal(size=(T, H))
+    W_s = rs.normal(size=(V, H))
+    h_t = rs.normal(size=(T, H))
+    W_t = rs.normal(size=(n_teachers, V, H))
+    tid = rs.randint(0, n_teachers, size=(B, Sm1))
+    mask = (rs.uniform(size=(B, Sm1)) < 0.7).astype(np.uint8)
+    mask[0, -1] = 1
+    return h_s, W_s, h_t, W_t, tid, mask
+
+
+def multi_teacher_brute_force(O, rs):
+    """Per-token loss and both reductions with a teacher per row, against the
+    pure-Python loops that pick each position's teacher head."""
+    worst = 0.0
+    for _ in range(3):
+        h_s, W_s, h_t, W_t, tid, mask = rand_multi_problem(rs)
+        ref_tok = np.array(brute.loss_tokens_multi(h_s.tolist(), W_s.tolist(), h_t.tolist(),
+                                                   [w.tolist() for w in W_t], tid.tolist(), mask.tolist()))
+        for red, ref_fn in ((O.REDUCE_TOKEN_MEAN, brute.token_mean), (O.REDUCE_SEQ_MEAN_NESTED, brute.nested_mean)):
+            out = O.forward_multi(h_s, W_s, h_t, W_t, tid, mask, red)
+            worst = max(worst, float(np.max(np.abs(out["loss_tok"] - ref_tok))))
+            worst = max(worst, abs(out["loss"] - ref_fn(ref_tok.tolist(), mask.tolist())))
+    return worst
+
+
+def multi_teacher_kl_vs_scipy(O, rs):
+    """Each row's loss is scipy's KL of softmax(z_s) from softmax(z_t) with
+    z_t built from that row's own teacher head."""
+    h_s, W_s, h_t, W_t, tid, mask = rand_multi_problem(rs, B=4, Sm1=5, H=6, V=50, n_teachers=4)
+    out = O.forward_multi(h_s, W_s, h_t, W_t, tid, mask, O.REDUCE_NONE)
+    worst = 0.0
+    for r in np.flatnonzero(mask.reshape(-1)):
+        z_s = h_s[r] @ W_s.T
+        z_t = h_t[r] @ W_t[tid.reshape(-1)[r]].T
+        ref = scipy.stats.entropy(scipy.special.softmax(z_s), scipy.special.softmax(z_t))
+        worst = max(worst, abs(out["loss_tok"].reshape(-1)[r] - ref))
+    return worst
+
+
+def multi_teacher_finite_differences(O, rs, red=1):
+    """Central differences of the objective w.r.t. h_s and W_s, teacher per row."""
+    mask = np.array([[1, 1, 1], [0, 1, 0], [0, 0, 0]], dtype=np.uint8)
+    h_s, W_s, h_t, W_t, tid, _ = rand_multi_problem(rs, B=3, Sm1=3, H=4, V=7, n_teachers=2)
+    tid[0] = [0, 1, 1]
+
+    def f(hs, ws):
+        return O.forward_multi(hs, ws, h_t, W_t, tid, mask, red)["loss"]
+
+    dH, dW = O.backward_multi(h_s, W_s, h_t, W_t, tid, mask, red)
+    eps = 1e-6
+    num_H = np.zeros_like(h_s)
+    for i in range(h_s.shape[0]):
+        for j in range(h_s.shape[1]):
+            hp = h_s.copy(); hp[i, j] += eps
+            hm = h_s.copy(); hm[i, j] -= eps
+            num_H[i, j] = (f(hp, W_s) - f(hm, W_s)) / (2 * eps)
+    num_W = np.zeros_like(W_s)
+    for i in range(W_s.shape[0]):
+        for j in range(W_s.shape[1]):
+            wp = W_s.copy(); wp[i, j] += eps
+            wm = W_s.copy(); wm[i, j] -= eps
+            num_W[i, j] = (f(h_s, wp) - f(h_s, wm)) / (2 * eps)
+    return max(float(np.max(np.abs(dH - num_H))) / max(1e-12, float(np.max(np.abs(num_H)))),
+               float(np.max(np.abs(dW - num_W))) / max(1e-12, float(np.max(np.abs(num_W)))))
+
+
+def multi_teacher_counts_brute(O, rs):
+    """Rows per teacher and out-of-range indices, against loops.  Masked
+    positions may hold any index (never read)."""
+    bad = 0
+    for _ in range(5):
+        mask = (rs.uniform(size=(3, 8)) < 0.6).astype(np.uint8)
+        tid = rs.randint(-1, 5, size=(3, 8))
+        counts, n_bad = O.count_rows_per_teacher(mask, tid, 4)
+        ref_counts, ref_bad = brute.count_rows_per_teacher(mask.tolist(), tid.tolist(), 4)
+        bad += int(list(counts) != ref_counts or n_bad != ref_bad)
+    return bad

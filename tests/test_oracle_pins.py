@@ -249,3 +249,59 @@ def test_student_stats_from_logits_equal_hidden(rs):
 
 def rand_problem_for_stats(rs):
     return pins.rand_problem(rs, B=3, Sm1=5, H=4, V=23)
+
+
+# ------------------------------------------------------------ several teachers
+
+def test_multi_teacher_brute_force(rs):
+    assert pins.multi_teacher_brute_force(O, rs) < 1e-12
+
+
+def test_multi_teacher_kl_vs_scipy(rs):
+    assert pins.multi_teacher_kl_vs_scipy(O, rs) < 1e-10
+
+
+@pytest.mark.parametrize("red", [1, 2])
+def test_multi_teacher_finite_differences(rs, red):
+    assert pins.multi_teacher_finite_differences(O, rs, red=red) < 1e-6
+
+
+def test_multi_teacher_counts_brute(rs):
+    assert pins.multi_teacher_counts_brute(O, rs) == 0
+
+
+def test_multi_teacher_single_teacher_reduces(rs):
+    # every row on teacher g: the single-teacher forward/backward with W_t[g]
+    h_s, W_s, h_t, W_t, _, mask = pins.rand_multi_problem(rs)
+    for g in range(W_t.shape[0]):
+        tid = np.full(mask.shape, g)
+        a = O.forward_multi(h_s, W_s, h_t, W_t, tid, mask, 2)
+        b = O.forward(h_s, W_s, h_t, W_t[g], mask, 2)
+        assert np.max(np.abs(a["loss_tok"] - b["loss_tok"])) < 1e-14 and abs(a["loss"] - b["loss"]) < 1e-14
+        dHa, dWa = O.backward_multi(h_s, W_s, h_t, W_t, tid, mask, 2)
+        dHb, dWb = O.backward(h_s, W_s, h_t, W_t[g], mask, 2)
+        assert np.max(np.abs(dHa - dHb)) < 1e-14 and np.max(np.abs(dWa - dWb)) < 1e-14
+
+
+MULTI_MUTATIONS = [
+    # every row projected with the first teacher's head
+    ("z_t[sel] = _f64(h_t[rows[sel]]) @ W_t64[g].T", "z_t[sel] = _f64(h_t[rows[sel]]) @ W_t64[0].T", "brute"),
+    # teacher index read at the compact position instead of the token position
+    ("    k = tid_flat[rows]\n", "    k = tid_flat[np.arange(len(rows))]\n", "brute"),
+    # teacher indices off by one
+    ("z_t[sel] = _f64(h_t[rows[sel]]) @ W_t64[g].T",
+     "z_t[sel] = _f64(h_t[rows[sel]]) @ W_t64[(g + 1) % W_t64.shape[0]].T", "brute"),
+    # masked rows counted per teacher
+    ("    tid = np.asarray(teacher_idx).reshape(-1)[flat]\n", "    tid = np.asarray(teacher_idx).reshape(-1)\n",
+     "counts"),
+]
+
+
+@pytest.mark.parametrize("old,new,kind", MULTI_MUTATIONS)
+def test_multi_teacher_pins_catch_planted_mistakes(old, new, kind):
+    M = _mutant(old, new)
+    rs = np.random.RandomState(11)
+    if kind == "brute":
+        assert pins.multi_teacher_brute_force(M, rs) > 1e-6
+    else:
+        assert pins.multi_teacher_counts_brute(M, rs) > 0
