@@ -122,6 +122,8 @@ class Problem:
         self.T = self.B * self.Sm1
         self.pair = "student_logits" in inp
         self.logits = "teacher_logits" in inp and not self.pair
+        self.multi = "teacher_idx" in inp
+        self.n_teachers = inp["W_t"].shape[0] if self.multi else 1
         self.student = inp["student_logits"] if self.pair else inp["h_s"]
         self.H = 0 if self.pair else inp["h_s"].shape[1]
         self.V = inp["student_logits"].shape[1] if self.pair else inp["W_s"].shape[0]
@@ -135,7 +137,12 @@ class Problem:
         self.row_idx = torch.empty(self.T, dtype=torch.int32, device=device)
         self.n_dev = torch.empty(1, dtype=torch.int32, device=device)
         self.n_host = torch.empty(1, dtype=torch.int32).pin_memory()
-        nbytes = rb.workspace_size(self.payload, self.dt, self.T, self.B, self.Sm1, max(self.H, 64), self.V)
+        if self.multi:
+            nbytes = rb.workspace_size_multi(self.dt, self.T, self.n_teachers, self.B, self.Sm1, self.H, self.V)
+            self.counts_dev = torch.empty(self.n_teachers + 1, dtype=torch.int32, device=device)
+            self.counts_host = torch.empty(self.n_teachers + 1, dtype=torch.int32).pin_memory()
+        else:
+            nbytes = rb.workspace_size(self.payload, self.dt, self.T, self.B, self.Sm1, max(self.H, 64), self.V)
         self.ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
         self.loss_tok = torch.empty((self.B, self.Sm1), dtype=torch.float32, device=device)
         self.loss = torch.empty(1, dtype=torch.float32, device=device)
@@ -151,13 +158,23 @@ class Problem:
     def _p(self, t):
         return None if t is None else ctypes.c_void_p(t.data_ptr())
 
-    def step(self, h_s=None, teacher=None, mask=None):
+    def inputs(self):
+        """The per-batch input tensors (what a data loader would deliver each step)."""
+        out = [self.student, self.teacher, self.inp["mask"]]
+        if self.multi:
+            out.append(self.inp["teacher_idx"])
+        return out
+
+    def step(self, h_s=None, teacher=None, mask=None, teacher_idx=None):
         """S1..S7 for one batch; returns N.  Inputs default to the resident ones."""
         L, p = self.L, self._p
         h_s = self.student if h_s is None else h_s
         teacher = self.teacher if teacher is None else teacher
         mask = self.inp["mask"] if mask is None else mask
         s = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+        if self.multi:
+            tid = self.inp["teacher_idx"] if teacher_idx is None else teacher_idx
+            return self._step_multi(h_s, teacher, mask, tid, s)
         rb._check(L.rkl_compact_rows(p(mask), self.B, self.Sm1, p(self.row_idx), p(self.n_dev), s))
         self.n_host.copy_(self.n_dev, non_blocking=True)
         torch.cuda.current_stream().synchronize()
@@ -183,6 +200,27 @@ class Problem:
         rb._check(L.rkl_backward(self.payload, p(h_s), p(teacher), p(self.inp["W_s"]), p(self.W_t), self.dt, self.B,
                                  self.Sm1, self.H, self.V, p(self.row_idx), N, self.reduction, p(self.saved),
                                  p(self.grad_loss), None, p(self.dH), p(self.dW), p(self.ws), self.ws.numel(), s))
+        self.N = N
+        return N
+
+    def _step_multi(self, h_s, h_t, mask, tid, s):
+        L, p = self.L, self._p
+        nt = self.n_teachers
+        rb._check(L.rkl_compact_rows_multi(p(mask), p(tid), self.B, self.Sm1, nt, p(self.row_idx), p(self.n_dev),
+                                           p(self.counts_dev), s))
+        self.n_host.copy_(self.n_dev, non_blocking=True)
+        self.counts_host.copy_(self.counts_dev, non_blocking=True)
+        torch.cuda.current_stream().synchronize()
+        N = int(self.n_host[0])
+        counts = (ctypes.c_int32 * nt)(*self.counts_host[:nt].tolist())
+        rb._check(L.rkl_forward_hidden_multi(p(h_s), p(h_t), p(self.inp["W_s"]), p(self.W_t), nt, p(tid), counts,
+                                             self.dt, self.B, self.Sm1, self.H, self.V, p(self.row_idx), N,
+                                             self.reduction, p(self.loss_tok), p(self.loss), p(self.saved),
+                                             p(self.ws), self.ws.numel(), s))
+        rb._check(L.rkl_backward_hidden_multi(p(h_s), p(h_t), p(self.inp["W_s"]), p(self.W_t), nt, p(tid), counts,
+                                              self.dt, self.B, self.Sm1, self.H, self.V, p(self.row_idx), N,
+                                              self.reduction, p(self.saved), p(self.grad_loss), None, p(self.dH),
+                                              p(self.dW), p(self.ws), self.ws.numel(), s))
         self.N = N
         return N
 
@@ -267,8 +305,13 @@ def cpu_oracle_sample(inp, reduction, name, rows=CPU_SAMPLE_ROWS):
         else:
             teacher, W_t = f64(inp["h_t"]), f64(inp["W_t"])
         t0 = time.perf_counter()
-        O.forward(h_s, W_s, teacher, W_t, sub, reduction)
-        O.backward(h_s, W_s, teacher, W_t, sub, reduction)
+        if "teacher_idx" in inp:
+            tid = inp["teacher_idx"].cpu().numpy()
+            O.forward_multi(h_s, W_s, teacher, W_t, tid, sub, reduction)
+            O.backward_multi(h_s, W_s, teacher, W_t, tid, sub, reduction)
+        else:
+            O.forward(h_s, W_s, teacher, W_t, sub, reduction)
+            O.backward(h_s, W_s, teacher, W_t, sub, reduction)
         dt = time.perf_counter() - t0
     threads = max([d.get("num_threads", 1) for d in threadpool_info()] or [1])
     return {"value": len(flat) / dt, "unit": UNIT, "cores": threads, "kind": "oracle",
@@ -348,12 +391,9 @@ def run_gpu(args, rank, world, dist):
     # stream while step i computes (two device buffers), as a training loop
     # with a prefetching data loader would do.  All copies are inside the
     # timed region.
-    h_pin = prob.student.cpu().pin_memory()
-    t_pin = prob.teacher.cpu().pin_memory()
-    m_pin = prob.inp["mask"].cpu().pin_memory()
+    pins = [t.cpu().pin_memory() for t in prob.inputs()]
     loss_host = torch.empty(1, dtype=torch.float32).pin_memory()
-    bufs = [(torch.empty_like(prob.student), torch.empty_like(prob.teacher), torch.empty_like(prob.inp["mask"]))
-            for _ in range(2)]
+    bufs = [[torch.empty_like(t) for t in prob.inputs()] for _ in range(2)]
     copy_stream = torch.cuda.Stream(dev)
     ready = [torch.cuda.Event(), torch.cuda.Event()]
     consumed = [torch.cuda.Event(), torch.cuda.Event()]
@@ -362,9 +402,8 @@ def run_gpu(args, rank, world, dist):
         b = bufs[i % 2]
         with torch.cuda.stream(copy_stream):
             copy_stream.wait_event(consumed[i % 2])
-            b[0].copy_(h_pin, non_blocking=True)
-            b[1].copy_(t_pin, non_blocking=True)
-            b[2].copy_(m_pin, non_blocking=True)
+            for dst, src in zip(b, pins):
+                dst.copy_(src, non_blocking=True)
             ready[i % 2].record(copy_stream)
 
     def e2e_run(n):
@@ -375,8 +414,7 @@ def run_gpu(args, rank, world, dist):
             if i + 1 < n:
                 issue_copy(i + 1)
             stream.wait_event(ready[i % 2])
-            b = bufs[i % 2]
-            prob.step(b[0], b[1], b[2])
+            prob.step(*bufs[i % 2])
             consumed[i % 2].record(stream)
             loss_host.copy_(prob.loss, non_blocking=True)
 
@@ -390,8 +428,10 @@ def run_gpu(args, rank, world, dist):
     torch.cuda.synchronize()
     ms_e2e, _ = reduce_over_ranks(f0.elapsed_time(f1), 0, dist, dev)
     e2e_value = n_tot / (ms_e2e / 1000.0)
-    h2d = h_pin.numel() * h_pin.element_size() + t_pin.numel() * t_pin.element_size() + m_pin.numel()
-    d2h = 4 + 4  # loss scalar + N (the compaction count read back to size the launches)
+    h2d = sum(t.numel() * t.element_size() for t in pins)
+    # loss scalar + N (the compaction count read back to size the launches)
+    # + the per-teacher row counts of the teacher-per-row mode
+    d2h = 4 + 4 + (4 * (prob.n_teachers + 1) if prob.multi else 0)
 
     if rank != 0:
         return
@@ -427,10 +467,13 @@ def run_gpu(args, rank, world, dist):
         "vs_baseline": None, "dtype": "bf16" if prob.dt == 0 else "fp32", "data": "synthetic",
         "config": {"workload": args.workload, "B": prob.B, "Sm1": prob.Sm1, "H": prob.H, "V": prob.V,
                    "trainable_rows": N, "tokens_T": prob.T,
-                   "payload": "logits_pair" if prob.pair else ("logits" if prob.logits else "hidden"),
+                   "payload": "logits_pair" if prob.pair else ("logits" if prob.logits else
+                                                                 ("hidden, %d teachers" % prob.n_teachers
+                                                                  if prob.multi else "hidden")),
                    "parallelism": "replicas" if world > 1 else "single",
                    "l2": "inputs larger than L2 (%.2f GB streamed per pass > 126 MB); no flush" % (
-                       (2 * prob.T * prob.V * 2 if prob.pair else (2 if not prob.logits else 1) * prob.V * prob.H * 2)
+                       (2 * prob.T * prob.V * 2 if prob.pair else
+                        ((1 + prob.n_teachers) if not prob.logits else 1) * prob.V * prob.H * 2)
                        / 1e9)},
         "roofline": {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
                      "frac": achieved / peak, "traffic": traffic_for(dom),

@@ -64,6 +64,12 @@ _SIGS = {
                                   _vp], _i32),
     "rkl_forward_hidden_noalloc": ([_vp, _vp, _vp, _vp, _i32, _i64, _i64, _i64, _i64, _vp, _i32, _i32,
                                     _vp, _vp, _vp, _vp], _i32),
+    "rkl_compact_rows_multi": ([_vp, _vp, _i64, _i64, _i32, _vp, _vp, _vp, _vp], _i32),
+    "rkl_workspace_size_multi": ([_i32, _i64, _i32, _i64, _i64, _i64, _i64, ctypes.POINTER(_sz)], _i32),
+    "rkl_forward_hidden_multi": ([_vp, _vp, _vp, _vp, _i32, _vp, _vp, _i32, _i64, _i64, _i64, _i64, _vp, _i32, _i32,
+                                  _vp, _vp, _vp, _vp, _sz, _vp], _i32),
+    "rkl_backward_hidden_multi": ([_vp, _vp, _vp, _vp, _i32, _vp, _vp, _i32, _i64, _i64, _i64, _i64, _vp, _i32, _i32,
+                                   _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp], _i32),
     "rkl_device_error": ([ctypes.POINTER(_i32)], _i32),
     "rkl_kernel_count": ([], _i32),
     "rkl_kernel_name": ([_i32], ctypes.c_char_p),
@@ -248,6 +254,116 @@ def backward_logits_pair(student_logits, teacher_logits, B, Sm1, row_idx, N, red
                                           N, reduction, _ptr(saved), _ptr(grad_loss), _ptr(grad_tok), _ptr(dz),
                                           _ptr(ws), ws.numel(), _stream(dev)))
     return dz
+
+
+# ------------------------------------------------------------ teacher per row
+
+def compact_rows_multi(mask, teacher_idx, n_teachers):
+    """S1 with per-teacher counts: (row_idx int32 [B*Sm1] device, N, counts list
+    of n_teachers ints).  Raises if a trainable row's teacher index is out of
+    range."""
+    B, Sm1 = mask.shape
+    mask = mask.contiguous()
+    if mask.dtype != torch.uint8:
+        mask = (mask != 0).to(torch.uint8)
+    tid = teacher_idx.to(device=mask.device, dtype=torch.int32).contiguous()
+    row_idx = torch.empty(B * Sm1, dtype=torch.int32, device=mask.device)
+    n_dev = torch.empty(1, dtype=torch.int32, device=mask.device)
+    counts = torch.empty(n_teachers + 1, dtype=torch.int32, device=mask.device)
+    _check(lib().rkl_compact_rows_multi(_ptr(mask), _ptr(tid), B, Sm1, n_teachers, _ptr(row_idx), _ptr(n_dev),
+                                        _ptr(counts), _stream(mask.device)))
+    host = counts.cpu().tolist()
+    if host[n_teachers] != 0:
+        raise RKLError(2, "%d trainable rows have a teacher index outside [0, %d)" % (host[n_teachers], n_teachers))
+    return row_idx, int(n_dev.item()), host[:n_teachers]
+
+
+def workspace_size_multi(dtype_code, n_max, n_teachers, B, Sm1, H, V):
+    out = ctypes.c_size_t(0)
+    _check(lib().rkl_workspace_size_multi(dtype_code, n_max, n_teachers, B, Sm1, H, V, ctypes.byref(out)))
+    return out.value
+
+
+def _counts_host(counts):
+    arr = (ctypes.c_int32 * len(counts))(*[int(c) for c in counts])
+    return arr
+
+
+def forward_hidden_multi(h_s, h_t, W_s, W_t, teacher_idx, counts, B, Sm1, row_idx, N, reduction, workspace=None):
+    """Forward with a teacher per row.  W_t [n_teachers, V, H]; teacher_idx
+    [B, Sm1] int32 device; counts from compact_rows_multi.
+    Returns (loss_tok [B,Sm1], loss [1], saved [N,3])."""
+    dev = h_s.device
+    T, H = h_s.shape
+    V = W_s.shape[0]
+    nt = W_t.shape[0]
+    dt = _dtype_code(h_s)
+    tid = teacher_idx.to(device=dev, dtype=torch.int32).contiguous()
+    loss_tok = torch.empty((B, Sm1), dtype=torch.float32, device=dev)
+    loss = torch.empty(1, dtype=torch.float32, device=dev)
+    saved = torch.empty((max(N, 1), 3), dtype=torch.float32, device=dev)
+    if workspace is None:
+        nbytes = workspace_size_multi(dt, max(N, 1), nt, B, Sm1, H, V)
+        workspace = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=dev)
+    _check(lib().rkl_forward_hidden_multi(_ptr(h_s), _ptr(h_t), _ptr(W_s), _ptr(W_t), nt, _ptr(tid),
+                                          _counts_host(counts), dt, B, Sm1, H, V, _ptr(row_idx), N, reduction,
+                                          _ptr(loss_tok), _ptr(loss), _ptr(saved), _ptr(workspace), workspace.numel(),
+                                          _stream(dev)))
+    return loss_tok, loss, saved
+
+
+def backward_hidden_multi(h_s, h_t, W_s, W_t, teacher_idx, counts, B, Sm1, row_idx, N, reduction, saved,
+                          grad_loss=None, grad_tok=None, workspace=None, dH_s=None, dW_s=None):
+    """Backward with a teacher per row.  Returns (dH_s [T,H] fp32, dW_s [V,H] fp32)."""
+    dev = h_s.device
+    T, H = h_s.shape
+    V = W_s.shape[0]
+    nt = W_t.shape[0]
+    dt = _dtype_code(h_s)
+    tid = teacher_idx.to(device=dev, dtype=torch.int32).contiguous()
+    if dH_s is None:
+        dH_s = torch.empty((T, H), dtype=torch.float32, device=dev)
+    if dW_s is None:
+        dW_s = torch.empty((V, H), dtype=torch.float32, device=dev)
+    if grad_loss is not None:
+        grad_loss = grad_loss.reshape(1).to(device=dev, dtype=torch.float32).contiguous()
+    if grad_tok is not None:
+        grad_tok = grad_tok.to(device=dev, dtype=torch.float32).contiguous()
+    if workspace is None:
+        nbytes = workspace_size_multi(dt, max(N, 1), nt, B, Sm1, H, V)
+        workspace = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=dev)
+    _check(lib().rkl_backward_hidden_multi(_ptr(h_s), _ptr(h_t), _ptr(W_s), _ptr(W_t), nt, _ptr(tid),
+                                           _counts_host(counts), dt, B, Sm1, H, V, _ptr(row_idx), N, reduction,
+                                           _ptr(saved), _ptr(grad_loss), _ptr(grad_tok), _ptr(dH_s), _ptr(dW_s),
+                                           _ptr(workspace), workspace.numel(), _stream(dev)))
+    return dH_s, dW_s
+
+
+class _RKLHiddenMulti(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, h_s, h_t, W_s, W_t, teacher_idx, mask, reduction):
+        B, Sm1 = mask.shape
+        row_idx, N, counts = compact_rows_multi(mask, teacher_idx, W_t.shape[0])
+        tid = teacher_idx.to(device=h_s.device, dtype=torch.int32).contiguous()
+        loss_tok, loss, saved = forward_hidden_multi(h_s, h_t, W_s, W_t, tid, counts, B, Sm1, row_idx, N, reduction)
+        ctx.save_for_backward(h_s, h_t, W_s, W_t, tid, row_idx, saved)
+        ctx.meta = (B, Sm1, N, reduction, counts)
+        return loss.reshape(()), loss_tok
+
+    @staticmethod
+    def backward(ctx, g_loss, g_tok):
+        h_s, h_t, W_s, W_t, tid, row_idx, saved = ctx.saved_tensors
+        B, Sm1, N, reduction, counts = ctx.meta
+        dH, dW = backward_hidden_multi(h_s, h_t, W_s, W_t, tid, counts, B, Sm1, row_idx, N, reduction, saved,
+                                       grad_loss=g_loss, grad_tok=g_tok)
+        return dH.to(h_s.dtype), None, dW.to(W_s.dtype), None, None, None, None
+
+
+def reverse_kl_hidden_multi(h_s, h_t, W_s, W_t, teacher_idx, mask, reduction=REDUCE_TOKEN_MEAN):
+    """Differentiable (loss, loss_tok) with a teacher per row: W_t [n_teachers, V, H]
+    stacked heads, teacher_idx [B, S-1]; grads to h_s and W_s."""
+    return _RKLHiddenMulti.apply(h_s.contiguous(), h_t.contiguous(), W_s.contiguous(), W_t.contiguous(),
+                                 teacher_idx, mask, reduction)
 
 
 def device_error():

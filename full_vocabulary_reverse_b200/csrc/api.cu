@@ -43,7 +43,8 @@ static rkl_status fail(rkl_status s, const char* fmt, ...) {
 static const char* const kKernelNames[K_COUNT] = {
     "compact_rows", "gather_rows",   "fwd_dual_tc",  "fwd_single_tc", "teacher_lse", "combine_splits",
     "scatter_loss", "reduce_loss",   "row_weights",  "dz_dual_tc",    "dz_single_tc", "grad_dw_dh_tc",
-    "scatter_dh",   "fwd_simt_fp32", "dz_simt_fp32", "grad_simt_fp32", "pair_fwd",   "pair_bwd"};
+    "scatter_dh",   "fwd_simt_fp32", "dz_simt_fp32", "grad_simt_fp32", "pair_fwd",   "pair_bwd",
+    "count_teachers", "build_slots"};
 
 const char* kernel_name(int id) { return (id >= 0 && id < K_COUNT) ? kKernelNames[id] : nullptr; }
 
@@ -152,21 +153,26 @@ constexpr int kSimtSplits = 37;
 struct Plan {
   int n_pad = 0, es = 2, S = 1, VT = 1, Vc = 0, nchunks = 1;
   size_t off_hcs = 0, off_hct = 0, off_part = 0, off_rowc = 0, off_lse = 0, off_dz = 0, off_dh = 0, off_cnt = 0,
-         total = 0;
+         off_slot = 0, off_kslot = 0, total = 0;
 };
 
 static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 // Workspace layout.  S = number of partial-statistics groups of the forward:
 // groups of kGroupTiles vocab tiles on the tensor-core path, kSimtSplits
-// vocab splits on the fp32 path -- both depend on V only.
-static Plan make_plan(rkl_payload payload, rkl_dtype dtype, int64_t n_max, int64_t H, int64_t V) {
+// vocab splits on the fp32 path -- both depend on V only.  With a teacher per
+// row (n_teachers > 1) the rows are regrouped by teacher into whole 256-row
+// tiles: sum_g ceil(n_g / 256) <= ceil(N / 256) + n_teachers - 1 tiles, plus
+// the slot maps.
+static Plan make_plan(rkl_payload payload, rkl_dtype dtype, int64_t n_max, int64_t H, int64_t V,
+                      int n_teachers = 1) {
   Plan p;
   const bool bf16 = dtype == RKL_BF16;
   const int tile_v = bf16 ? kFBN : kSimtBN;
   p.es = bf16 ? 2 : 4;
   const int64_t n = n_max < 1 ? 1 : n_max;
   p.n_pad = static_cast<int>(((n + 2 * kBM - 1) / (2 * kBM)) * (2 * kBM));  // whole 256-row pair tiles
+  if (n_teachers > 1) p.n_pad += 2 * kBM * (n_teachers - 1);
   p.VT = static_cast<int>((V + tile_v - 1) / tile_v);
   // tensor-core path: two statistics slots (column halves) per group
   p.S = bf16 ? 2 * ((p.VT + kGroupTiles - 1) / kGroupTiles) : (p.VT < kSimtSplits ? p.VT : kSimtSplits);
@@ -191,8 +197,54 @@ static Plan make_plan(rkl_payload payload, rkl_dtype dtype, int64_t n_max, int64
   off = align256(off + size_t(p.n_pad) * H * sizeof(float));
   p.off_cnt = off;
   off = align256(off + size_t(p.nchunks) * sizeof(int));
+  if (n_teachers > 1) {
+    p.off_slot = off;
+    off = align256(off + size_t(p.n_pad) * sizeof(int32_t));
+    p.off_kslot = off;
+    off = align256(off + size_t(n) * sizeof(int32_t));
+  }
   p.total = off;
   return p;
+}
+
+// Teacher-grouped row layout of the per-row-teacher mode (host side).
+struct MultiTeacher {
+  int n = 0;                         // teachers (> 1)
+  const int32_t* teacher_idx = nullptr;  // [B, Sm1] device
+  const void* W_t = nullptr;         // stacked heads [n, V, H]
+  TeacherSlots ts{};
+  int n_rows = 0;                    // slots in use (sum of 256-rounded counts)
+  int group_row_end[kMaxTeachers] = {};
+};
+
+static rkl_status make_multi(int n_teachers, const int32_t* teacher_idx, const int32_t* counts, int32_t N,
+                             MultiTeacher* mt) {
+  if (n_teachers < 1 || n_teachers > kMaxTeachers)
+    return fail(RKL_ERR_SHAPE, "n_teachers = %d outside [1, %d]", n_teachers, kMaxTeachers);
+  if (teacher_idx == nullptr || counts == nullptr) return fail(RKL_ERR_NULL, "teacher_idx and counts must be non-NULL");
+  if ((reinterpret_cast<uintptr_t>(teacher_idx) & 15) != 0)
+    return fail(RKL_ERR_ALIGN, "teacher_idx is not 16-byte aligned");
+  mt->n = n_teachers;
+  mt->teacher_idx = teacher_idx;
+  mt->ts.n = n_teachers;
+  long long sum = 0;
+  int base = 0;
+  for (int g = 0; g < n_teachers; ++g) {
+    if (counts[g] < 0) return fail(RKL_ERR_SHAPE, "counts[%d] = %d is negative", g, counts[g]);
+    sum += counts[g];
+    mt->ts.count[g] = counts[g];
+    mt->ts.base[g] = base;
+    if (sum > N) break;
+    base += ((counts[g] + 2 * kBM - 1) / (2 * kBM)) * (2 * kBM);
+    mt->group_row_end[g] = base;
+  }
+  if (sum != N)
+    return fail(RKL_ERR_SHAPE,
+                "per-teacher counts add up to %lld but N = %d (a trainable row has a teacher index outside "
+                "[0, n_teachers), or the counts belong to another mask)",
+                sum, N);
+  mt->n_rows = base;
+  return RKL_OK;
 }
 
 // ------------------------------------------------------------------ checks
@@ -238,7 +290,8 @@ static rkl_status forward_impl(rkl_payload payload, const void* h_s, const void*
                                const int32_t* row_idx, int32_t N, rkl_reduction reduction, float* loss_tok,
                                float* loss, float* saved, void* workspace, size_t workspace_bytes, void* stream_,
                                bool forward_only_workspace = false, const int32_t* targets = nullptr,
-                               float* entropy = nullptr, float* target_logprob = nullptr) {
+                               float* entropy = nullptr, float* target_logprob = nullptr,
+                               const MultiTeacher* mt = nullptr) {
   RKL_TRY(check_common(payload, dtype, B, Sm1, H, V, N, reduction));
   RKL_TRY(check_ptr(h_s, "h_s"));
   RKL_TRY(check_ptr(teacher, payload == RKL_PAYLOAD_HIDDEN ? "h_t" : "teacher_logits"));
@@ -253,7 +306,7 @@ static rkl_status forward_impl(rkl_payload payload, const void* h_s, const void*
   RKL_TRY(check_ptr(entropy, "entropy", false));
   RKL_TRY(check_ptr(target_logprob, "target_logprob", false));
   if (target_logprob && !targets) return fail(RKL_ERR_NULL, "target_logprob needs targets");
-  const Plan pl = make_plan(payload, dtype, N, H, V);
+  const Plan pl = make_plan(payload, dtype, N, H, V, mt ? mt->n : 1);
   // The forward touches only the regions in front of the dz chunk.
   const size_t needed = forward_only_workspace ? pl.off_dz : pl.total;
   if (workspace_bytes < needed)
@@ -277,14 +330,24 @@ static rkl_status forward_impl(rkl_payload payload, const void* h_s, const void*
   if (N > 0) {
     float* part = reinterpret_cast<float*>(ws_at(workspace, pl.off_part));
     float* lse_ext = reinterpret_cast<float*>(ws_at(workspace, pl.off_lse));
+    // Teacher per row: rows regrouped by teacher into whole pair tiles.
+    int32_t* slot_k = nullptr;
+    int n_rows = N;
+    if (mt) {
+      slot_k = reinterpret_cast<int32_t*>(ws_at(workspace, pl.off_slot));
+      n_rows = mt->n_rows;
+      RKL_CUDA(cudaMemsetAsync(slot_k, 0xFF, size_t(n_rows) * sizeof(int32_t), s));
+      RKL_CUDA(launch_build_slots(row_idx, mt->teacher_idx, N, mt->ts, slot_k,
+                                  reinterpret_cast<int32_t*>(ws_at(workspace, pl.off_kslot)), s));
+    }
     // S2: compact the rows (skipped when every row is trainable).
     const void* as = h_s;
     const void* at = teacher;
-    if (N < T) {
+    if (N < T || mt) {
       as = ws_at(workspace, pl.off_hcs);
       at = hidden ? ws_at(workspace, pl.off_hct) : nullptr;
       RKL_CUDA(launch_gather(h_s, hidden ? teacher : nullptr, const_cast<void*>(as), const_cast<void*>(at), row_idx,
-                             N, static_cast<int>(H * pl.es), s));
+                             slot_k, n_rows, static_cast<int>(H * pl.es), s));
     }
     // S8: teacher log-sum-exp from the shipped logits.
     if (!hidden) RKL_CUDA(launch_teacher_lse(teacher, bf16, row_idx, N, static_cast<int>(V), V, lse_ext, s));
@@ -292,11 +355,15 @@ static rkl_status forward_impl(rkl_payload payload, const void* h_s, const void*
     if (bf16) {
       FusedArgs a;
       memset(&a, 0, sizeof(a));
-      RKL_TRY(make_map(&a.tm_as, as, false, H, N, H * 2, kBK, kBM));
+      RKL_TRY(make_map(&a.tm_as, as, false, H, n_rows, H * 2, kBK, kBM));
       RKL_TRY(make_map(&a.tm_bs, W_s, false, H, V, H * 2, kBK, kFBN / 2));
       if (hidden) {
-        RKL_TRY(make_map(&a.tm_at, at, false, H, N, H * 2, kBK, kBM));
-        RKL_TRY(make_map(&a.tm_bt, W_t, false, H, V, H * 2, kBK, kFBN / 2));
+        RKL_TRY(make_map(&a.tm_at, at, false, H, n_rows, H * 2, kBK, kBM));
+        RKL_TRY(make_map(&a.tm_bt, W_t, false, H, V * (mt ? mt->n : 1), H * 2, kBK, kFBN / 2));
+        if (mt) {
+          a.tgroups = mt->n;
+          for (int g = 0; g < mt->n; ++g) a.group_row_end[g] = mt->group_row_end[g];
+        }
       } else {
         a.teacher = static_cast<const uint16_t*>(teacher);
         a.teacher_rows = N < T ? row_idx : nullptr;
@@ -306,7 +373,7 @@ static rkl_status forward_impl(rkl_payload payload, const void* h_s, const void*
       a.row_idx = row_idx;
       a.targets = targets;
       a.tlogit = tlogit;
-      a.N = N;
+      a.N = n_rows;
       a.n_pad = pl.n_pad;
       a.H = static_cast<int>(H);
       a.V = static_cast<int>(V);
@@ -315,7 +382,7 @@ static rkl_status forward_impl(rkl_payload payload, const void* h_s, const void*
       a.vt_base = 0;
       a.GT = kGroupTiles;
       a.G = pl.S / 2;
-      const int MT = (N + 2 * kBM - 1) / (2 * kBM);
+      const int MT = (n_rows + 2 * kBM - 1) / (2 * kBM);
       a.MT = MT;
       a.units_total = MT * a.G;
       RKL_CUDA(launch_fused(ng, false, a, 2 * a.units_total < sms ? 2 * a.units_total : sms, s));
@@ -327,6 +394,10 @@ static rkl_status forward_impl(rkl_payload payload, const void* h_s, const void*
       if (hidden) {
         a.at = static_cast<const float*>(at);
         a.bt = static_cast<const float*>(W_t);
+        if (mt) {
+          a.tgroups = mt->n;
+          for (int g = 0; g < mt->n; ++g) a.group_row_end[g] = mt->group_row_end[g];
+        }
       } else {
         a.teacher = static_cast<const float*>(teacher);
         a.teacher_rows = N < T ? row_idx : nullptr;
@@ -336,18 +407,19 @@ static rkl_status forward_impl(rkl_payload payload, const void* h_s, const void*
       a.row_idx = row_idx;
       a.targets = targets;
       a.tlogit = tlogit;
-      a.N = N;
+      a.N = n_rows;
       a.n_pad = pl.n_pad;
       a.H = static_cast<int>(H);
       a.V = static_cast<int>(V);
       a.IT = pl.VT;
       a.S = pl.S;
       a.ng = ng;
-      const int MT = (N + kSimtBN - 1) / kSimtBN;
+      const int MT = (n_rows + kSimtBN - 1) / kSimtBN;
       RKL_CUDA(launch_simt_fused(false, a, dim3(MT, pl.S), s));
     }
     // S4
-    RKL_CUDA(launch_combine(part, pl.S, pl.n_pad, N, hidden, lse_ext, tlogit, saved, ent_rows, lp_rows, s));
+    RKL_CUDA(launch_combine(part, pl.S, pl.n_pad, n_rows, hidden, lse_ext, tlogit, saved, ent_rows, lp_rows, slot_k,
+                            s));
   }
   if (loss_tok) RKL_CUDA(launch_scatter_loss(saved, row_idx, N, T, loss_tok, s));
   if (entropy) RKL_CUDA(launch_scatter_rows(ent_rows, row_idx, N, T, entropy, s));
@@ -362,7 +434,8 @@ static rkl_status backward_impl(rkl_payload payload, const void* h_s, const void
                                 const void* W_t, rkl_dtype dtype, int64_t B, int64_t Sm1, int64_t H, int64_t V,
                                 const int32_t* row_idx, int32_t N, rkl_reduction reduction, const float* saved,
                                 const float* grad_loss, const float* grad_tok, float* dH_s, float* dW_s,
-                                void* workspace, size_t workspace_bytes, void* stream_) {
+                                void* workspace, size_t workspace_bytes, void* stream_,
+                                const MultiTeacher* mt = nullptr) {
   RKL_TRY(check_common(payload, dtype, B, Sm1, H, V, N, reduction));
   RKL_TRY(check_ptr(h_s, "h_s"));
   RKL_TRY(check_ptr(teacher, payload == RKL_PAYLOAD_HIDDEN ? "h_t" : "teacher_logits"));
@@ -375,7 +448,7 @@ static rkl_status backward_impl(rkl_payload payload, const void* h_s, const void
   RKL_TRY(check_ptr(dH_s, "dH_s"));
   RKL_TRY(check_ptr(dW_s, "dW_s"));
   RKL_TRY(check_ptr(workspace, "workspace"));
-  const Plan pl = make_plan(payload, dtype, N, H, V);
+  const Plan pl = make_plan(payload, dtype, N, H, V, mt ? mt->n : 1);
   if (workspace_bytes < pl.total)
     return fail(RKL_ERR_WORKSPACE, "workspace is %zu bytes, %zu needed", workspace_bytes, pl.total);
   int sms = 0;
@@ -388,20 +461,31 @@ static rkl_status backward_impl(rkl_payload payload, const void* h_s, const void
 
   if (N == 0) {
     RKL_CUDA(cudaMemsetAsync(dW_s, 0, size_t(V) * H * sizeof(float), s));
-    RKL_CUDA(launch_scatter_dh(dHc, row_idx, 0, T, static_cast<int>(H), dH_s, s));
+    RKL_CUDA(launch_scatter_dh(dHc, row_idx, nullptr, 0, T, static_cast<int>(H), dH_s, s));
     return RKL_OK;
+  }
+  // Teacher per row: rows regrouped by teacher into whole pair tiles.
+  int32_t* slot_k = nullptr;
+  int32_t* k_slot = nullptr;
+  int n_rows = N;
+  if (mt) {
+    slot_k = reinterpret_cast<int32_t*>(ws_at(workspace, pl.off_slot));
+    k_slot = reinterpret_cast<int32_t*>(ws_at(workspace, pl.off_kslot));
+    n_rows = mt->n_rows;
+    RKL_CUDA(cudaMemsetAsync(slot_k, 0xFF, size_t(n_rows) * sizeof(int32_t), s));
+    RKL_CUDA(launch_build_slots(row_idx, mt->teacher_idx, N, mt->ts, slot_k, k_slot, s));
   }
   const void* as = h_s;
   const void* at = teacher;
-  if (N < T) {
+  if (N < T || mt) {
     as = ws_at(workspace, pl.off_hcs);
     at = hidden ? ws_at(workspace, pl.off_hct) : nullptr;
-    RKL_CUDA(launch_gather(h_s, hidden ? teacher : nullptr, const_cast<void*>(as), const_cast<void*>(at), row_idx, N,
-                           static_cast<int>(H * pl.es), s));
+    RKL_CUDA(launch_gather(h_s, hidden ? teacher : nullptr, const_cast<void*>(as), const_cast<void*>(at), row_idx,
+                           slot_k, n_rows, static_cast<int>(H * pl.es), s));
   }
   float* rowc = reinterpret_cast<float*>(ws_at(workspace, pl.off_rowc));
   RKL_CUDA(launch_row_weights(saved, row_idx, N, pl.n_pad, static_cast<int>(B), static_cast<int>(Sm1), reduction,
-                              grad_loss, grad_tok, rowc, s));
+                              grad_loss, grad_tok, rowc, slot_k, s));
   void* dz = ws_at(workspace, pl.off_dz);
   const int ng = hidden ? 2 : 1;
   const int nchunks = static_cast<int>((V + pl.Vc - 1) / pl.Vc);
@@ -409,45 +493,49 @@ static rkl_status backward_impl(rkl_payload payload, const void* h_s, const void
   if (bf16) {
     FusedArgs a;
     memset(&a, 0, sizeof(a));
-    RKL_TRY(make_map(&a.tm_as, as, false, H, N, H * 2, kBK, kBM));
+    RKL_TRY(make_map(&a.tm_as, as, false, H, n_rows, H * 2, kBK, kBM));
     RKL_TRY(make_map(&a.tm_bs, W_s, false, H, V, H * 2, kBK, kFBN / 2));
     if (hidden) {
-      RKL_TRY(make_map(&a.tm_at, at, false, H, N, H * 2, kBK, kBM));
-      RKL_TRY(make_map(&a.tm_bt, W_t, false, H, V, H * 2, kBK, kFBN / 2));
+      RKL_TRY(make_map(&a.tm_at, at, false, H, n_rows, H * 2, kBK, kBM));
+      RKL_TRY(make_map(&a.tm_bt, W_t, false, H, V * (mt ? mt->n : 1), H * 2, kBK, kFBN / 2));
+      if (mt) {
+        a.tgroups = mt->n;
+        for (int g = 0; g < mt->n; ++g) a.group_row_end[g] = mt->group_row_end[g];
+      }
     } else {
       a.teacher = static_cast<const uint16_t*>(teacher);
       a.teacher_rows = N < T ? row_idx : nullptr;
       a.teacher_pitch = V;
     }
     a.rowc = rowc;
-    a.N = N;
+    a.N = n_rows;
     a.n_pad = pl.n_pad;
     a.H = static_cast<int>(H);
     a.V = static_cast<int>(V);
     a.KB = static_cast<int>(H / kBK);
-    const int MT = (N + 2 * kBM - 1) / (2 * kBM);
+    const int MT = (n_rows + 2 * kBM - 1) / (2 * kBM);
     a.MT = MT;
 
     int* counters = reinterpret_cast<int*>(ws_at(workspace, pl.off_cnt));
     RKL_CUDA(cudaMemsetAsync(counters, 0, size_t(nchunks) * sizeof(int), s));
     GradArgs g;
     memset(&g, 0, sizeof(g));
-    RKL_TRY(make_map(&g.tm_hs_mn, as, false, H, N, H * 2, 64, 64));
+    RKL_TRY(make_map(&g.tm_hs_mn, as, false, H, n_rows, H * 2, 64, 64));
     RKL_TRY(make_map(&g.tm_ws_mn, W_s, false, H, V, H * 2, 64, 64));
     RKL_TRY(make_map(&g.tm_dw, dW_s, true, H, V, H * 4, 32, 32));
-    RKL_TRY(make_map(&g.tm_dh, dHc, true, H, N, H * 4, 32, 32));
-    g.N = N;
+    RKL_TRY(make_map(&g.tm_dh, dHc, true, H, n_rows, H * 4, 32, 32));
+    g.N = n_rows;
     g.H = static_cast<int>(H);
     g.NT = static_cast<int>(H / kGradBN) + (H % kGradBN ? 1 : 0);
-    g.MTH = (N + 2 * kBM - 1) / (2 * kBM);  // 256-row pair tiles
+    g.MTH = (n_rows + 2 * kBM - 1) / (2 * kBM);  // 256-row pair tiles
     g.nH = g.MTH * g.NT;
-    g.KBW = (N + kBK - 1) / kBK;
+    g.KBW = (n_rows + kBK - 1) / kBK;
 
     for (int c = 0; c < nchunks; ++c) {
       const int cv0 = c * pl.Vc;
       const int cw = static_cast<int>((V - cv0) < pl.Vc ? (V - cv0) : pl.Vc);
       // S6: recompute the logits of this chunk and write dz (bf16) [N, cw].
-      RKL_TRY(make_map(&a.tm_dz, dz, false, cw, N, size_t(pl.Vc) * 2, 64, 32));
+      RKL_TRY(make_map(&a.tm_dz, dz, false, cw, n_rows, size_t(pl.Vc) * 2, 64, 32));
       a.IT = (cw + kFBN - 1) / kFBN;
       a.vt_base = cv0 / kFBN;
       a.chunk_v0 = cv0;
@@ -456,8 +544,8 @@ static rkl_status backward_impl(rkl_payload payload, const void* h_s, const void
       a.units_total = MT * a.IT;
       RKL_CUDA(launch_fused(ng, true, a, 2 * a.units_total < sms ? 2 * a.units_total : sms, s));
       // S7: dW_s[chunk] = dz^T hc_s and dHc (+)= dz W_s[chunk].
-      RKL_TRY(make_map(&g.tm_dz_k, dz, false, cw, N, size_t(pl.Vc) * 2, 64, 128));
-      RKL_TRY(make_map(&g.tm_dz_mn, dz, false, cw, N, size_t(pl.Vc) * 2, 64, 64));
+      RKL_TRY(make_map(&g.tm_dz_k, dz, false, cw, n_rows, size_t(pl.Vc) * 2, 64, 128));
+      RKL_TRY(make_map(&g.tm_dz_mn, dz, false, cw, n_rows, size_t(pl.Vc) * 2, 64, 64));
       g.cw = cw;
       g.cv0 = cv0;
       g.MTW = (cw + 2 * kBM - 1) / (2 * kBM);
@@ -476,6 +564,10 @@ static rkl_status backward_impl(rkl_payload payload, const void* h_s, const void
     if (hidden) {
       a.at = static_cast<const float*>(at);
       a.bt = static_cast<const float*>(W_t);
+      if (mt) {
+        a.tgroups = mt->n;
+        for (int g = 0; g < mt->n; ++g) a.group_row_end[g] = mt->group_row_end[g];
+      }
     } else {
       a.teacher = static_cast<const float*>(teacher);
       a.teacher_rows = N < T ? row_idx : nullptr;
@@ -483,12 +575,12 @@ static rkl_status backward_impl(rkl_payload payload, const void* h_s, const void
     }
     a.rowc = rowc;
     a.dz = static_cast<float*>(dz);
-    a.N = N;
+    a.N = n_rows;
     a.n_pad = pl.n_pad;
     a.H = static_cast<int>(H);
     a.V = static_cast<int>(V);
     a.ng = ng;
-    const int MT = (N + kSimtBN - 1) / kSimtBN;
+    const int MT = (n_rows + kSimtBN - 1) / kSimtBN;
     for (int c = 0; c < nchunks; ++c) {
       const int cv0 = c * pl.Vc;
       const int cw = static_cast<int>((V - cv0) < pl.Vc ? (V - cv0) : pl.Vc);
@@ -500,14 +592,14 @@ static rkl_status backward_impl(rkl_payload payload, const void* h_s, const void
       RKL_CUDA(launch_simt_fused(true, a, dim3(items < 4 * sms ? items : 4 * sms), s));
       const float* dzf = static_cast<const float*>(dz);
       // dW_s[cv0 + m, n] = sum_k dz[k, m] hc_s[k, n]
-      RKL_CUDA(launch_simt_gemm(dzf, 1, cw, a.as, H, 1, dW_s + size_t(cv0) * H, H, cw, static_cast<int>(H), N, 0,
-                                s));
+      RKL_CUDA(launch_simt_gemm(dzf, 1, cw, a.as, H, 1, dW_s + size_t(cv0) * H, H, cw, static_cast<int>(H), n_rows,
+                                0, s));
       // dHc[m, n] (+)= sum_k dz[m, k] W_s[cv0 + k, n]
-      RKL_CUDA(launch_simt_gemm(dzf, cw, 1, a.bs + size_t(cv0) * H, H, 1, dHc, H, N, static_cast<int>(H), cw,
+      RKL_CUDA(launch_simt_gemm(dzf, cw, 1, a.bs + size_t(cv0) * H, H, 1, dHc, H, n_rows, static_cast<int>(H), cw,
                                 c > 0, s));
     }
   }
-  RKL_CUDA(launch_scatter_dh(dHc, row_idx, N, T, static_cast<int>(H), dH_s, s));
+  RKL_CUDA(launch_scatter_dh(dHc, row_idx, k_slot, N, T, static_cast<int>(H), dH_s, s));
   return RKL_OK;
 }
 
@@ -589,7 +681,7 @@ rkl_status rkl_backward_logits_pair(const void* student_logits, const void* teac
   float* rowc = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + 256);
   if (N > 0)
     RKL_CUDA(launch_row_weights(saved, row_idx, N, n_pad, static_cast<int>(B), static_cast<int>(Sm1), reduction,
-                                grad_loss, grad_tok, rowc, s));
+                                grad_loss, grad_tok, rowc, nullptr, s));
   RKL_CUDA(launch_pair_bwd(student_logits, teacher_logits, dtype == RKL_BF16, row_idx, N, n_pad, T,
                            static_cast<int>(V), rowc, dz, s));
   return RKL_OK;
@@ -650,6 +742,64 @@ rkl_status rkl_backward(rkl_payload payload, const void* h_s, const void* teache
                         void* stream) {
   return backward_impl(payload, h_s, teacher, W_s, W_t, dtype, B, Sm1, H, V, row_idx, N, reduction, saved, grad_loss,
                        grad_tok, dH_s, dW_s, workspace, workspace_bytes, stream);
+}
+
+// ---------------------------------------------------------------- teacher per row
+rkl_status rkl_compact_rows_multi(const uint8_t* mask, const int32_t* teacher_idx, int64_t B, int64_t Sm1,
+                                  int32_t n_teachers, int32_t* row_idx, int32_t* n_dev, int32_t* counts,
+                                  void* stream) {
+  if (mask == nullptr || teacher_idx == nullptr || row_idx == nullptr || n_dev == nullptr || counts == nullptr)
+    return fail(RKL_ERR_NULL, "mask, teacher_idx, row_idx, n_dev and counts must be non-NULL");
+  if (!aligned16(row_idx) || !aligned16(teacher_idx))
+    return fail(RKL_ERR_ALIGN, "row_idx and teacher_idx must be 16-byte aligned");
+  if (B < 1 || Sm1 < 1) return fail(RKL_ERR_SHAPE, "B and Sm1 must be >= 1");
+  if (B * Sm1 >= (int64_t(1) << 31)) return fail(RKL_ERR_SHAPE, "B*Sm1 exceeds 2^31-1");
+  if (n_teachers < 1 || n_teachers > kMaxTeachers)
+    return fail(RKL_ERR_SHAPE, "n_teachers = %d outside [1, %d]", n_teachers, kMaxTeachers);
+  int sms = 0;
+  RKL_TRY(device_setup(&sms));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  RKL_CUDA(cudaMemsetAsync(counts, 0, size_t(n_teachers + 1) * sizeof(int32_t), s));
+  RKL_CUDA(launch_compact(mask, B * Sm1, row_idx, n_dev, s));
+  RKL_CUDA(launch_count_teachers(mask, teacher_idx, B * Sm1, n_teachers, counts, s));
+  return RKL_OK;
+}
+
+rkl_status rkl_workspace_size_multi(rkl_dtype dtype, int64_t n_max, int32_t n_teachers, int64_t B, int64_t Sm1,
+                                    int64_t H, int64_t V, size_t* bytes) {
+  if (bytes == nullptr) return fail(RKL_ERR_NULL, "bytes is NULL");
+  RKL_TRY(check_common(RKL_PAYLOAD_HIDDEN, dtype, B, Sm1, H, V, 0, 0));
+  if (n_max < 0 || n_max > B * Sm1) return fail(RKL_ERR_SHAPE, "n_max outside [0, B*Sm1]");
+  if (n_teachers < 1 || n_teachers > kMaxTeachers)
+    return fail(RKL_ERR_SHAPE, "n_teachers = %d outside [1, %d]", n_teachers, kMaxTeachers);
+  *bytes = make_plan(RKL_PAYLOAD_HIDDEN, dtype, n_max, H, V, n_teachers).total;
+  return RKL_OK;
+}
+
+rkl_status rkl_forward_hidden_multi(const void* h_s, const void* h_t, const void* W_s, const void* W_t,
+                                   int32_t n_teachers, const int32_t* teacher_idx, const int32_t* counts,
+                                   rkl_dtype dtype, int64_t B, int64_t Sm1, int64_t H, int64_t V,
+                                   const int32_t* row_idx, int32_t N, rkl_reduction reduction, float* loss_tok,
+                                   float* loss, float* saved, void* workspace, size_t workspace_bytes,
+                                   void* stream) {
+  MultiTeacher mt;
+  RKL_TRY(make_multi(n_teachers, teacher_idx, counts, N, &mt));
+  return forward_impl(RKL_PAYLOAD_HIDDEN, h_s, h_t, W_s, W_t, dtype, B, Sm1, H, V, row_idx, N, reduction, loss_tok,
+                      loss, saved, workspace, workspace_bytes, stream, false, nullptr, nullptr, nullptr,
+                      n_teachers > 1 ? &mt : nullptr);
+}
+
+rkl_status rkl_backward_hidden_multi(const void* h_s, const void* h_t, const void* W_s, const void* W_t,
+                                    int32_t n_teachers, const int32_t* teacher_idx, const int32_t* counts,
+                                    rkl_dtype dtype, int64_t B, int64_t Sm1, int64_t H, int64_t V,
+                                    const int32_t* row_idx, int32_t N, rkl_reduction reduction, const float* saved,
+                                    const float* grad_loss, const float* grad_tok, float* dH_s, float* dW_s,
+                                    void* workspace, size_t workspace_bytes, void* stream) {
+  MultiTeacher mt;
+  RKL_TRY(make_multi(n_teachers, teacher_idx, counts, N, &mt));
+  return backward_impl(RKL_PAYLOAD_HIDDEN, h_s, h_t, W_s, W_t, dtype, B, Sm1, H, V, row_idx, N, reduction, saved,
+                       grad_loss, grad_tok, dH_s, dW_s, workspace, workspace_bytes, stream,
+                       n_teachers > 1 ? &mt : nullptr);
 }
 
 rkl_status rkl_device_error(int32_t* code) {

@@ -29,6 +29,8 @@ enum KernelId : int {
   K_GRAD_SIMT,        // fp32 S7
   K_PAIR_FWD,         // both sides as logits: forward statistics, bandwidth bound
   K_PAIR_BWD,         // both sides as logits: dL/dz_s rows, bandwidth bound
+  K_COUNT_TEACHERS,   // per-row teachers: trainable rows per teacher
+  K_BUILD_SLOTS,      // per-row teachers: teacher-grouped row slots
   K_COUNT
 };
 
@@ -50,6 +52,7 @@ constexpr int kBK = 64;        // K per pipeline stage (128 B of bf16)
 constexpr int kGradBN = 256;   // H columns per gradient tile
 constexpr int kGroupTiles = 4;  // 256-column vocab tiles per forward statistics group (1024 columns)
 constexpr int kStatVals = 6;    // per slot: m_s, S_s, A, m_t, S_t, sum e^(z_s-m_s) z_s
+constexpr int kMaxTeachers = 16;  // teacher heads of the per-row-teacher mode
 
 // ---------------------------------------------------------------- tcgen05
 struct FusedArgs {
@@ -72,6 +75,11 @@ struct FusedArgs {
   int MT;                            // row tiles (256 rows each, one per CTA pair)
   int units_total;                   // MT * G
   int chunk_v0;                      // dz: first vocab column of the chunk
+  // Teacher per row: tm_bt covers the stacked heads [tgroups * V, H] and the
+  // rows of teacher g occupy [group_row_end[g-1], group_row_end[g]) (whole
+  // 256-row pair tiles).  tgroups <= 1: one teacher head.
+  int tgroups;
+  int group_row_end[kMaxTeachers];
 };
 
 struct GradArgs {
@@ -96,13 +104,15 @@ cudaError_t read_and_clear_device_error(int* code);
 
 // ---------------------------------------------------------------- small kernels
 cudaError_t launch_compact(const uint8_t* mask, long long T, int32_t* row_idx, int32_t* n_dev, cudaStream_t s);
-cudaError_t launch_gather(const void* h_s, const void* h_t, void* hc_s, void* hc_t, const int32_t* row_idx, int N,
-                          int row_bytes, cudaStream_t s);
+// hc[p] = h[row_idx[k]] with k = slot_k[p] (slot_k nullptr: k = p); k < 0 gives a zero row.
+cudaError_t launch_gather(const void* h_s, const void* h_t, void* hc_s, void* hc_t, const int32_t* row_idx,
+                          const int32_t* slot_k, int n_rows, int row_bytes, cudaStream_t s);
 cudaError_t launch_teacher_lse(const void* logits, bool bf16, const int32_t* row_idx, int N, int V,
                                long long pitch, float* lse_t, cudaStream_t s);
-cudaError_t launch_combine(const float* part, int S, int n_pad, int N, bool teacher_from_part,
+// Statistics rows p < n_rows are written to compact row slot_k[p] (nullptr: p; < 0: skipped).
+cudaError_t launch_combine(const float* part, int S, int n_pad, int n_rows, bool teacher_from_part,
                            const float* lse_t_ext, const float* tlogit, float* saved, float* ent_rows,
-                           float* lp_rows, cudaStream_t s);
+                           float* lp_rows, const int32_t* slot_k, cudaStream_t s);
 cudaError_t launch_scatter_loss(const float* saved, const int32_t* row_idx, int N, long long T, float* loss_tok,
                                 cudaStream_t s);
 // out[t] = rows[k] where t = row_idx[k], else 0 (per-token [B, S-1] scatter)
@@ -112,9 +122,23 @@ cudaError_t launch_reduce(const float* saved, const int32_t* row_idx, int N, int
                           float* loss, cudaStream_t s);
 cudaError_t launch_row_weights(const float* saved, const int32_t* row_idx, int N, int n_pad, int B, int Sm1,
                                int reduction, const float* grad_loss, const float* grad_tok, float* rowc,
-                               cudaStream_t s);
-cudaError_t launch_scatter_dh(const float* dHc, const int32_t* row_idx, int N, long long T, int H, float* dH_s,
-                              cudaStream_t s);
+                               const int32_t* slot_k, cudaStream_t s);
+// dH_s[row_idx[k]] = dHc[k_slot[k]] (k_slot nullptr: k), all other rows 0.
+cudaError_t launch_scatter_dh(const float* dHc, const int32_t* row_idx, const int32_t* k_slot, int N, long long T,
+                              int H, float* dH_s, cudaStream_t s);
+// Trainable rows per teacher: counts[g] for g < n_teachers, counts[n_teachers] =
+// trainable rows whose index is outside [0, n_teachers).  counts must be zeroed.
+cudaError_t launch_count_teachers(const uint8_t* mask, const int32_t* teacher_idx, long long T, int n_teachers,
+                                  int32_t* counts, cudaStream_t s);
+struct TeacherSlots {
+  int n;                      // teachers
+  int count[kMaxTeachers];    // trainable rows of each teacher
+  int base[kMaxTeachers];     // first slot of each teacher (multiples of 256)
+};
+// Slot of every compact row k (teacher-grouped, ascending within a teacher):
+// slot_k[p] = k (slot_k pre-filled with -1 for padding), k_slot[k] = p.
+cudaError_t launch_build_slots(const int32_t* row_idx, const int32_t* teacher_idx, int N, const TeacherSlots& ts,
+                               int32_t* slot_k, int32_t* k_slot, cudaStream_t s);
 cudaError_t launch_pair_fwd(const void* zs, const void* zt, bool bf16, const int32_t* row_idx, int N, int V,
                             float* saved, cudaStream_t s);
 cudaError_t launch_pair_bwd(const void* zs, const void* zt, bool bf16, const int32_t* row_idx, int N, int n_pad,
@@ -132,6 +156,8 @@ struct SimtArgs {
   float* dz;                          // dz chunk [N, cw] fp32
   int N, n_pad, H, V, S, IT, vt_base, chunk_v0, cw;
   int ng;
+  int tgroups;                        // > 1: bt is the stacked teacher heads [tgroups, V, H]
+  int group_row_end[kMaxTeachers];    // rows of teacher g end here (multiples of 32)
 };
 constexpr int kSimtBN = 32;
 cudaError_t launch_simt_fused(bool dz, const SimtArgs& a, dim3 grid, cudaStream_t s);

@@ -42,6 +42,13 @@ __global__ void __launch_bounds__(256) simt_fused_kernel(const SimtArgs a) {
   for (int u = u0; u < u1; ++u) {
     const int m0 = (u / a.IT) * TB;
     const int v0 = (a.vt_base + u % a.IT) * TB;
+    // teacher per row: rows of teacher g end at group_row_end[g]
+    const float* bt = a.bt;
+    if (a.tgroups > 1) {
+      int tg = 0;
+      while (tg + 1 < a.tgroups && m0 >= a.group_row_end[tg]) ++tg;
+      bt += static_cast<long long>(tg) * a.V * a.H;
+    }
     float cs[4] = {0.f, 0.f, 0.f, 0.f}, ct[4] = {0.f, 0.f, 0.f, 0.f};
     for (int k0 = 0; k0 < a.H; k0 += TB) {
       for (int e = tid; e < TB * TB; e += 256) {
@@ -51,7 +58,7 @@ __global__ void __launch_bounds__(256) simt_fused_kernel(const SimtArgs a) {
         Bs[r][kk] = (v0 + r < a.V && kin) ? a.bs[static_cast<long long>(v0 + r) * a.H + k0 + kk] : 0.f;
         if (a.ng == 2) {
           At[r][kk] = (m0 + r < a.N && kin) ? a.at[static_cast<long long>(m0 + r) * a.H + k0 + kk] : 0.f;
-          Bt[r][kk] = (v0 + r < a.V && kin) ? a.bt[static_cast<long long>(v0 + r) * a.H + k0 + kk] : 0.f;
+          Bt[r][kk] = (v0 + r < a.V && kin) ? bt[static_cast<long long>(v0 + r) * a.H + k0 + kk] : 0.f;
         }
       }
       __syncthreads();

@@ -79,15 +79,23 @@ __global__ void __launch_bounds__(1024) compact_kernel(const uint8_t* __restrict
 }
 
 // --------------------------------------------------------------------- S2
-// hc[k] = h[row_idx[k]] for k < N; blockIdx.y selects student / teacher.
+// hc[p] = h[row_idx[k]] for p < n_rows, k = slot_k[p] (or p without a slot
+// map); a slot with k < 0 (padding between teacher groups) becomes a zero
+// row.  blockIdx.y selects student / teacher.
 __global__ void __launch_bounds__(256) gather_kernel(const uint8_t* __restrict__ h_s, const uint8_t* __restrict__ h_t,
                                                      uint8_t* __restrict__ hc_s, uint8_t* __restrict__ hc_t,
-                                                     const int32_t* __restrict__ row_idx, int N, int row_bytes) {
+                                                     const int32_t* __restrict__ row_idx,
+                                                     const int32_t* __restrict__ slot_k, int n_rows, int row_bytes) {
   const uint8_t* src = blockIdx.y == 0 ? h_s : h_t;
   uint8_t* dst = blockIdx.y == 0 ? hc_s : hc_t;
-  for (int k = blockIdx.x; k < N; k += gridDim.x) {
+  for (int p = blockIdx.x; p < n_rows; p += gridDim.x) {
+    const int k = slot_k ? slot_k[p] : p;
+    uint8_t* d = dst + static_cast<long long>(p) * row_bytes;
+    if (k < 0) {
+      for (int i = threadIdx.x; i < row_bytes / 4; i += blockDim.x) reinterpret_cast<uint32_t*>(d)[i] = 0u;
+      continue;
+    }
     const uint8_t* s = src + static_cast<long long>(row_idx[k]) * row_bytes;
-    uint8_t* d = dst + static_cast<long long>(k) * row_bytes;
     if ((row_bytes & 15) == 0) {
       const uint4* s4 = reinterpret_cast<const uint4*>(s);
       uint4* d4 = reinterpret_cast<uint4*>(d);
@@ -251,13 +259,18 @@ __device__ __forceinline__ void merge3(Stat3& a, const Stat3& b) {
 
 // Optional student statistics of row k (nullable outputs): entropy
 // lse_s - sum p_s z_s = lse_s - Bz / S_s, and target log-prob tlogit - lse_s.
-__global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ part, int S, int n_pad, int N,
+// Statistics row k (a slot of the teacher-grouped layout when slot_k is
+// given) is written to compact row out = slot_k[k]; padding slots are skipped.
+__global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ part, int S, int n_pad, int n_rows,
                                                       int teacher_from_part, const float* __restrict__ lse_ext,
                                                       const float* __restrict__ tlogit, float* __restrict__ saved,
-                                                      float* __restrict__ ent_rows, float* __restrict__ lp_rows) {
+                                                      float* __restrict__ ent_rows, float* __restrict__ lp_rows,
+                                                      const int32_t* __restrict__ slot_k) {
   const int lane = threadIdx.x & 31;
   const int k = blockIdx.x * 8 + (threadIdx.x >> 5);
-  if (k >= N) return;
+  if (k >= n_rows) return;
+  const int out = slot_k ? slot_k[k] : k;
+  if (out < 0) return;
   Stat3 s{-INFINITY, 0.f, 0.f, 0.f}, t{-INFINITY, 0.f, 0.f, 0.f};
   for (int g = lane; g < S; g += 32) {
     const float* b = part + static_cast<size_t>(g) * kStatVals * n_pad + k;
@@ -275,11 +288,11 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
     const float lse_s = s.m + logf(s.S);
     const float lse_t = teacher_from_part ? t.m + logf(t.S) : lse_ext[k];
     const float L = s.A / s.S - lse_s + lse_t;
-    saved[3 * k + 0] = lse_s;
-    saved[3 * k + 1] = lse_t;
-    saved[3 * k + 2] = L;
-    if (ent_rows) ent_rows[k] = lse_s - s.Bz / s.S;
-    if (lp_rows) lp_rows[k] = tlogit[k] - lse_s;
+    saved[3 * out + 0] = lse_s;
+    saved[3 * out + 1] = lse_t;
+    saved[3 * out + 2] = L;
+    if (ent_rows) ent_rows[out] = lse_s - s.Bz / s.S;
+    if (lp_rows) lp_rows[out] = tlogit[k] - lse_s;
   }
 }
 
@@ -346,12 +359,14 @@ __global__ void __launch_bounds__(1024) reduce_kernel(const float* __restrict__ 
 // --------------------------------------------------------------------- S5
 // Row constants of the recompute pass: rowc[0] = lse_s*log2(e),
 // rowc[1] = lse_t - lse_s - L, rowc[2] = g = dLoss/dL_k.  Padding rows get 0.
+// With a slot map, row p of rowc belongs to compact row slot_k[p].
 __global__ void __launch_bounds__(256) row_weights_kernel(const float* __restrict__ saved,
                                                           const int32_t* __restrict__ row_idx, int N, int n_pad,
                                                           int B, int Sm1, int reduction,
                                                           const float* __restrict__ grad_loss,
                                                           const float* __restrict__ grad_tok,
-                                                          float* __restrict__ rowc) {
+                                                          float* __restrict__ rowc,
+                                                          const int32_t* __restrict__ slot_k) {
   __shared__ int b_eff_sh;
   if (threadIdx.x == 0) b_eff_sh = 0;
   __syncthreads();
@@ -365,10 +380,11 @@ __global__ void __launch_bounds__(256) row_weights_kernel(const float* __restric
     atomicAdd(&b_eff_sh, local);
   }
   __syncthreads();
-  const int k = blockIdx.x * blockDim.x + threadIdx.x;
-  if (k >= n_pad) return;
+  const int p = blockIdx.x * blockDim.x + threadIdx.x;
+  if (p >= n_pad) return;
+  const int k = slot_k ? slot_k[p] : p;
   float c0 = 0.f, c1 = 0.f, c2 = 0.f;
-  if (k < N) {
+  if (k >= 0 && k < N) {
     const int row = row_idx[k];
     const float lse_s = saved[3 * k], lse_t = saved[3 * k + 1], L = saved[3 * k + 2];
     float w = 0.f;
@@ -387,21 +403,23 @@ __global__ void __launch_bounds__(256) row_weights_kernel(const float* __restric
     c1 = lse_t - lse_s - L;
     c2 = g;
   }
-  rowc[k] = c0;
-  rowc[n_pad + k] = c1;
-  rowc[2 * n_pad + k] = c2;
+  rowc[p] = c0;
+  rowc[n_pad + p] = c1;
+  rowc[2 * n_pad + p] = c2;
 }
 
-// dH_s[t] = dHc[k] if t = row_idx[k], else exact zeros.
+// dH_s[t] = dHc[k_slot[k]] (dHc[k] without a slot map) if t = row_idx[k],
+// else exact zeros.
 __global__ void __launch_bounds__(256) scatter_dh_kernel(const float* __restrict__ dHc,
-                                                         const int32_t* __restrict__ row_idx, int N, long long T,
+                                                         const int32_t* __restrict__ row_idx,
+                                                         const int32_t* __restrict__ k_slot, int N, long long T,
                                                          int H, float* __restrict__ dH_s) {
   for (long long t = blockIdx.x; t < T; t += gridDim.x) {
     const int k = lower_bound_i32(row_idx, N, t);
-    const bool hit = k < N && row_idx[k] == t;
+    const int src = (k < N && row_idx[k] == t) ? (k_slot ? k_slot[k] : k) : -1;
     float* d = dH_s + t * H;
-    if (hit) {
-      const float* s = dHc + static_cast<long long>(k) * H;
+    if (src >= 0) {
+      const float* s = dHc + static_cast<long long>(src) * H;
       if ((H & 3) == 0) {
         float4* d4 = reinterpret_cast<float4*>(d);
         const float4* s4 = reinterpret_cast<const float4*>(s);
@@ -417,6 +435,91 @@ __global__ void __launch_bounds__(256) scatter_dh_kernel(const float* __restrict
         for (int i = threadIdx.x; i < H; i += blockDim.x) d[i] = 0.f;
       }
     }
+  }
+}
+
+// ------------------------------------------------------- teacher per row
+// NeMo RL PR #3978, first-version limits: one teacher in the first version,
+// with the payload laid out for a per-row teacher index.  Each trainable row
+// carries the index of its teacher; rows are regrouped by teacher into whole
+// 256-row tiles so that every tile of the tensor-core kernels projects with
+// one teacher head.
+
+// counts[g] += trainable rows of teacher g; counts[n] += trainable rows whose
+// index is outside [0, n).  Shared-memory histogram, then one global add per
+// bin and block (integer adds: the result does not depend on their order).
+__global__ void __launch_bounds__(1024) count_teachers_kernel(const uint8_t* __restrict__ mask,
+                                                              const int32_t* __restrict__ teacher_idx, long long T,
+                                                              int n, int32_t* __restrict__ counts) {
+  __shared__ int hist[kMaxTeachers + 1];
+  if (threadIdx.x <= kMaxTeachers) hist[threadIdx.x] = 0;
+  __syncthreads();
+  for (long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; t < T;
+       t += static_cast<long long>(gridDim.x) * blockDim.x) {
+    if (mask[t] != 0) {
+      const int g = teacher_idx[t];
+      atomicAdd(&hist[(g >= 0 && g < n) ? g : n], 1);
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x <= n && hist[threadIdx.x] != 0) atomicAdd(&counts[threadIdx.x], hist[threadIdx.x]);
+}
+
+// Teacher-grouped slots.  Compact rows k are taken in ascending order, 1024 at
+// a time; a row of teacher g gets slot base[g] + (rows of teacher g before
+// it).  Within a warp the rank comes from __match_any_sync, across warps from
+// an exclusive scan of the per-warp counts (warp g of the block scans the
+// counts of teacher g).  A row whose index is out of range, or whose rank
+// exceeds the count given for its teacher, gets no slot (k_slot = -1), so
+// every store stays inside the layout even for inconsistent counts.
+__global__ void __launch_bounds__(1024) build_slots_kernel(const int32_t* __restrict__ row_idx,
+                                                           const int32_t* __restrict__ teacher_idx, int N,
+                                                           const TeacherSlots ts, int32_t* __restrict__ slot_k,
+                                                           int32_t* __restrict__ k_slot) {
+  __shared__ int wcnt[32][kMaxTeachers];  // per warp and teacher; then its exclusive prefix
+  __shared__ int total[kMaxTeachers];
+  __shared__ int carry[kMaxTeachers];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid < kMaxTeachers) carry[tid] = 0;
+  for (int c0 = 0; c0 < N; c0 += 1024) {
+    for (int i = tid; i < 32 * kMaxTeachers; i += 1024) (&wcnt[0][0])[i] = 0;
+    __syncthreads();
+    const int k = c0 + tid;
+    int g = -1;
+    if (k < N) {
+      g = teacher_idx[row_idx[k]];
+      if (g < 0 || g >= ts.n) g = -1;
+    }
+    const unsigned peers = __match_any_sync(0xffffffffu, g);
+    const int rank_w = __popc(peers & ((1u << lane) - 1u));
+    if (g >= 0 && rank_w == 0) wcnt[warp][g] = __popc(peers);
+    __syncthreads();
+    if (warp < ts.n) {
+      const int x = wcnt[lane][warp];
+      int incl = x;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      wcnt[lane][warp] = incl - x;
+      if (lane == 31) total[warp] = incl;
+    }
+    __syncthreads();
+    if (k < N) {
+      int slot = -1;
+      if (g >= 0) {
+        const int r = carry[g] + wcnt[warp][g] + rank_w;
+        if (r < ts.count[g]) {
+          slot = ts.base[g] + r;
+          slot_k[slot] = k;
+        }
+      }
+      k_slot[k] = slot;
+    }
+    __syncthreads();
+    if (tid < ts.n) carry[tid] += total[tid];
+    __syncthreads();
   }
 }
 
@@ -606,13 +709,14 @@ cudaError_t launch_compact(const uint8_t* mask, long long T, int32_t* row_idx, i
   return cudaGetLastError();
 }
 
-cudaError_t launch_gather(const void* h_s, const void* h_t, void* hc_s, void* hc_t, const int32_t* row_idx, int N,
-                          int row_bytes, cudaStream_t s) {
-  if (N <= 0) return cudaSuccess;
+cudaError_t launch_gather(const void* h_s, const void* h_t, void* hc_s, void* hc_t, const int32_t* row_idx,
+                          const int32_t* slot_k, int n_rows, int row_bytes, cudaStream_t s) {
+  if (n_rows <= 0) return cudaSuccess;
   LaunchScope scope(K_GATHER, s);
-  dim3 grid(N < 65535 ? N : 65535, h_t ? 2 : 1);
+  dim3 grid(n_rows < 65535 ? n_rows : 65535, h_t ? 2 : 1);
   gather_kernel<<<grid, 256, 0, s>>>(static_cast<const uint8_t*>(h_s), static_cast<const uint8_t*>(h_t),
-                                     static_cast<uint8_t*>(hc_s), static_cast<uint8_t*>(hc_t), row_idx, N, row_bytes);
+                                     static_cast<uint8_t*>(hc_s), static_cast<uint8_t*>(hc_t), row_idx, slot_k,
+                                     n_rows, row_bytes);
   return cudaGetLastError();
 }
 
@@ -628,12 +732,13 @@ cudaError_t launch_teacher_lse(const void* logits, bool bf16, const int32_t* row
   return cudaGetLastError();
 }
 
-cudaError_t launch_combine(const float* part, int S, int n_pad, int N, bool teacher_from_part, const float* lse_ext,
-                           const float* tlogit, float* saved, float* ent_rows, float* lp_rows, cudaStream_t s) {
-  if (N <= 0) return cudaSuccess;
+cudaError_t launch_combine(const float* part, int S, int n_pad, int n_rows, bool teacher_from_part,
+                           const float* lse_ext, const float* tlogit, float* saved, float* ent_rows, float* lp_rows,
+                           const int32_t* slot_k, cudaStream_t s) {
+  if (n_rows <= 0) return cudaSuccess;
   LaunchScope scope(K_COMBINE, s);
-  combine_kernel<<<(N + 7) / 8, 256, 0, s>>>(part, S, n_pad, N, teacher_from_part ? 1 : 0, lse_ext, tlogit, saved,
-                                             ent_rows, lp_rows);
+  combine_kernel<<<(n_rows + 7) / 8, 256, 0, s>>>(part, S, n_pad, n_rows, teacher_from_part ? 1 : 0, lse_ext, tlogit,
+                                                  saved, ent_rows, lp_rows, slot_k);
   return cudaGetLastError();
 }
 
@@ -660,18 +765,35 @@ cudaError_t launch_reduce(const float* saved, const int32_t* row_idx, int N, int
 
 cudaError_t launch_row_weights(const float* saved, const int32_t* row_idx, int N, int n_pad, int B, int Sm1,
                                int reduction, const float* grad_loss, const float* grad_tok, float* rowc,
-                               cudaStream_t s) {
+                               const int32_t* slot_k, cudaStream_t s) {
   LaunchScope scope(K_ROW_WEIGHTS, s);
   row_weights_kernel<<<(n_pad + 255) / 256, 256, 0, s>>>(saved, row_idx, N, n_pad, B, Sm1, reduction, grad_loss,
-                                                         grad_tok, rowc);
+                                                         grad_tok, rowc, slot_k);
   return cudaGetLastError();
 }
 
-cudaError_t launch_scatter_dh(const float* dHc, const int32_t* row_idx, int N, long long T, int H, float* dH_s,
-                              cudaStream_t s) {
+cudaError_t launch_scatter_dh(const float* dHc, const int32_t* row_idx, const int32_t* k_slot, int N, long long T,
+                              int H, float* dH_s, cudaStream_t s) {
   LaunchScope scope(K_SCATTER_DH, s);
   const long long blocks = T < 65535 * 8 ? T : 65535 * 8;
-  scatter_dh_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(dHc, row_idx, N, T, H, dH_s);
+  scatter_dh_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(dHc, row_idx, k_slot, N, T, H, dH_s);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_count_teachers(const uint8_t* mask, const int32_t* teacher_idx, long long T, int n_teachers,
+                                  int32_t* counts, cudaStream_t s) {
+  LaunchScope scope(K_COUNT_TEACHERS, s);
+  const long long blocks = (T + 1023) / 1024;
+  count_teachers_kernel<<<static_cast<unsigned>(blocks < 1024 ? blocks : 1024), 1024, 0, s>>>(mask, teacher_idx, T,
+                                                                                               n_teachers, counts);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_build_slots(const int32_t* row_idx, const int32_t* teacher_idx, int N, const TeacherSlots& ts,
+                               int32_t* slot_k, int32_t* k_slot, cudaStream_t s) {
+  if (N <= 0) return cudaSuccess;
+  LaunchScope scope(K_BUILD_SLOTS, s);
+  build_slots_kernel<<<1, 1024, 0, s>>>(row_idx, teacher_idx, N, ts, slot_k, k_slot);
   return cudaGetLastError();
 }
 

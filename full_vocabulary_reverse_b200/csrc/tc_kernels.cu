@@ -261,6 +261,17 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_kernel(const __grid_co
         const int m0 = (u % p.MT) * 2 * kBM + rank * kBM;
         const int g = u / p.MT;
         const int vt_end = min(g * p.GT + p.GT, p.IT);
+        // Teacher per row: the head of this tile's teacher starts at row
+        // teacher * V of the stacked heads.  Columns at or past V of a tile
+        // then read the next head's rows instead of zeros; the epilogue never
+        // uses them (statistics stop at V, the dz store is clipped at V).
+        int tv_off = 0;
+        if (NG == 2 && p.tgroups > 1) {
+          const int tile_row = (u % p.MT) * 2 * kBM;
+          int tg = 0;
+          while (tg + 1 < p.tgroups && tile_row >= p.group_row_end[tg]) ++tg;
+          tv_off = tg * p.V;
+        }
         for (int vt = g * p.GT; vt < vt_end && ok; ++vt) {
           const int v0 = (p.vt_base + vt) * kFBN + rank * (kFBN / 2);
           for (int kb = 0; kb < p.KB; ++kb) {
@@ -276,7 +287,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_kernel(const __grid_co
             tma_load_2d_pair(sa + Cfg::A_BYTES, &p.tm_bs, fb, kb * kBK, v0);
             if (NG == 2) {
               tma_load_2d_pair(sa + Cfg::A_BYTES + Cfg::B_BYTES, &p.tm_at, fb, kb * kBK, m0);
-              tma_load_2d_pair(sa + 2 * Cfg::A_BYTES + Cfg::B_BYTES, &p.tm_bt, fb, kb * kBK, v0);
+              tma_load_2d_pair(sa + 2 * Cfg::A_BYTES + Cfg::B_BYTES, &p.tm_bt, fb, kb * kBK, v0 + tv_off);
             }
             armed |= 1u << stage;
             last_par = (last_par & ~(1u << stage)) | (phase << stage);

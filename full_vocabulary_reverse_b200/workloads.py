@@ -23,6 +23,9 @@ Named workloads:
   logits_pair     both sides as bf16 logits [8192, 151936]: student ~ N(0,9),
                   teacher = student + N(0, 0.5^2) + per-row shift U(-20,20);
                   all rows trainable; token mean.
+  multi_teacher   qwen_hidden shapes and mask with two teacher heads
+                  W_t[g] = W_s + N(0, 0.004^2) (independent draws), teacher
+                  of sequence b = b mod 2; token mean.
 """
 
 from __future__ import annotations
@@ -50,6 +53,9 @@ WORKLOADS = {
                         reduction=REDUCE_TOKEN_MEAN, mask="suffix256", weights="perturbed", seed=1239),
     "logits_pair": dict(dtype="bf16", B=4, Sm1=2048, H=0, V=151936, payload="logits_pair",
                         reduction=REDUCE_TOKEN_MEAN, mask="all", weights="perturbed", seed=1240),
+    "multi_teacher": dict(dtype="bf16", B=4, Sm1=2048, H=2048, V=151936, payload="hidden_multi",
+                          reduction=REDUCE_TOKEN_MEAN, mask="prefix", weights="perturbed", seed=1241,
+                          mask_seed=1236, n_teachers=2, teacher_assign="sequence"),
 }
 
 TORCH_DTYPES = {"bf16": torch.bfloat16, "fp32": torch.float32}
@@ -89,12 +95,26 @@ def _randn(shape, gen, device, scale=1.0, chunk_rows=8192):
     return out
 
 
+def make_teacher_idx(assign, B, Sm1, n_teachers, seed):
+    """int32 [B, Sm1] teacher index of every position: per sequence
+    (b mod n_teachers) or drawn uniformly per position."""
+    if assign == "sequence":
+        idx = np.repeat((np.arange(B) % n_teachers)[:, None], Sm1, axis=1)
+    elif assign == "random":
+        idx = np.random.RandomState(seed + 7).randint(0, n_teachers, size=(B, Sm1))
+    else:
+        raise ValueError(assign)
+    return torch.from_numpy(idx.astype(np.int32))
+
+
 def make_inputs(B, Sm1, H, V, dtype="bf16", payload="hidden", mask="prefix",
                 weights="perturbed", seed=0, device="cpu", mask_seed=None,
-                logit_std=3.0, teacher_noise=0.004):
+                logit_std=3.0, teacher_noise=0.004, n_teachers=1, teacher_assign="sequence"):
     """Draw one problem.  Returns a dict of torch tensors on `device`:
     h_s [T,H], W_s [V,H], mask uint8 [B,Sm1], and h_t [T,H] + W_t [V,H]
-    (hidden payload) or teacher_logits [T,V] (logits payload)."""
+    (hidden payload) or teacher_logits [T,V] (logits payload).  The
+    hidden_multi payload gives W_t [n_teachers, V, H] and teacher_idx
+    [B, Sm1] int32 instead."""
     T = B * Sm1
     tdt = TORCH_DTYPES[dtype]
     gen = torch.Generator(device=device)
@@ -117,6 +137,16 @@ def make_inputs(B, Sm1, H, V, dtype="bf16", payload="hidden", mask="prefix",
     w_scale = logit_std / math.sqrt(H)
     W_s32 = _randn((V, H), gen, device, scale=w_scale)
     out["W_s"] = W_s32.to(tdt)
+    if payload == "hidden_multi":
+        out["h_t"] = _randn((T, H), gen, device).to(tdt)
+        W_t = torch.empty((n_teachers, V, H), dtype=tdt, device=device)
+        for g in range(n_teachers):
+            W_t[g] = (W_s32 + _randn((V, H), gen, device, scale=teacher_noise)).to(tdt)
+        out["W_t"] = W_t
+        out["teacher_idx"] = make_teacher_idx(teacher_assign, B, Sm1, n_teachers, seed).to(device)
+        del W_s32
+        out["mask"] = torch.from_numpy(make_mask(mask, B, Sm1, seed if mask_seed is None else mask_seed)).to(device)
+        return out
     if payload == "hidden":
         if weights == "same":
             out["h_t"] = out["h_s"].clone()
@@ -155,7 +185,8 @@ def make_workload(name, device="cpu", **overrides):
     red = cfg.pop("reduction")
     inp = make_inputs(cfg["B"], cfg["Sm1"], cfg["H"], cfg["V"], dtype=cfg["dtype"],
                       payload=cfg["payload"], mask=cfg["mask"], weights=cfg["weights"],
-                      seed=cfg["seed"], device=device, mask_seed=cfg.get("mask_seed"))
+                      seed=cfg["seed"], device=device, mask_seed=cfg.get("mask_seed"),
+                      n_teachers=cfg.get("n_teachers", 1), teacher_assign=cfg.get("teacher_assign", "sequence"))
     inp["reduction"] = red
     inp["cfg"] = cfg
     return inp

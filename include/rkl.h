@@ -180,8 +180,8 @@ rkl_status rkl_backward(rkl_payload payload,
                         void* workspace, size_t workspace_bytes, void* stream);
 
 /* Both sides as logits: the student's logits [T, V] are given as well as the
- * teacher's (the logits payload of PR #3978's payload bullet 2 used as the
- * numerical reference, with the student side also materialised).  Same loss
+ * teacher's (the logits payload of PR #3978's payload bullet 2, meant for
+ * numerical checks, with the student side also materialised).  Same loss
  * and saved scalars as rkl_forward_logits; bandwidth bound (reads 2 N V
  * elements).  Any V >= 1; rows are read with 16-byte loads when the row
  * pitch allows.  Workspace: rkl_workspace_size(RKL_PAYLOAD_LOGITS_PAIR, ...)
@@ -202,6 +202,70 @@ rkl_status rkl_backward_logits_pair(const void* student_logits, const void* teac
                                     const int32_t* row_idx, int32_t N,
                                     rkl_reduction reduction, const float* saved,
                                     const float* grad_loss, const float* grad_tok, void* dz,
+                                    void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * A teacher per row (hidden-state payload).  PR #3978, first-version limits:
+ * the first version takes one teacher checkpoint and lays out the payload so
+ * that a per-row teacher index can be added.  Here every position carries
+ * the index k in [0, n_teachers) of its teacher, and the teacher logits of a
+ * trainable row r are z_t = h_t[r] W_t[k_r]^T, with W_t the stacked teacher
+ * heads [n_teachers, V, H] (all teachers share V and H).  The loss, the saved
+ * scalars, the reductions and the gradients are those of the one-teacher
+ * entry points.  1 <= n_teachers <= 16.
+ *
+ * Internally the compacted rows are regrouped by teacher into whole 256-row
+ * tiles (padding rows between groups cost at most 255 rows per teacher of
+ * extra tensor-core work), so every tile projects with one teacher head.
+ * ------------------------------------------------------------------------ */
+
+/* S1 with teacher counts.  teacher_idx [B, Sm1] int32 (device; entries at
+ * masked positions are never read).  Writes row_idx / *n_dev exactly as
+ * rkl_compact_rows, and counts [n_teachers + 1] (device): counts[g] = number
+ * of trainable rows of teacher g, counts[n_teachers] = number of trainable
+ * rows whose index lies outside [0, n_teachers) (such rows make the forward
+ * and backward fail with RKL_ERR_SHAPE).  The caller reads counts back (a
+ * (n_teachers + 1)-int copy) together with N. */
+rkl_status rkl_compact_rows_multi(const uint8_t* mask, const int32_t* teacher_idx,
+                                  int64_t B, int64_t Sm1, int32_t n_teachers,
+                                  int32_t* row_idx, int32_t* n_dev, int32_t* counts, void* stream);
+
+/* Workspace bytes of rkl_forward_hidden_multi / rkl_backward_hidden_multi
+ * for up to n_max trainable rows. */
+rkl_status rkl_workspace_size_multi(rkl_dtype dtype, int64_t n_max, int32_t n_teachers,
+                                    int64_t B, int64_t Sm1, int64_t H, int64_t V, size_t* bytes);
+
+/* Forward with a teacher per row.  Arguments as rkl_forward_hidden, plus:
+ *   W_t          [n_teachers, V, H] stacked teacher heads (device)
+ *   teacher_idx  [B, Sm1] int32 (device), the array given to compaction
+ *   counts       [n_teachers] int32, HOST copy of the counts written by
+ *                rkl_compact_rows_multi; they must add up to N
+ *                (RKL_ERR_SHAPE otherwise).  Counts that do not belong to
+ *                teacher_idx and the mask give unspecified (memory-safe)
+ *                results.
+ * Per-row entropy / target log-prob outputs are not offered in this mode. */
+rkl_status rkl_forward_hidden_multi(const void* h_s, const void* h_t,
+                                   const void* W_s, const void* W_t,
+                                   int32_t n_teachers, const int32_t* teacher_idx,
+                                   const int32_t* counts, rkl_dtype dtype,
+                                   int64_t B, int64_t Sm1, int64_t H, int64_t V,
+                                   const int32_t* row_idx, int32_t N,
+                                   rkl_reduction reduction,
+                                   float* loss_tok, float* loss, float* saved,
+                                   void* workspace, size_t workspace_bytes, void* stream);
+
+/* Backward with a teacher per row; arguments as rkl_backward (hidden
+ * payload) plus those of rkl_forward_hidden_multi.  dH_s [T, H] and dW_s
+ * [V, H] as rkl_backward; no gradient for any teacher input. */
+rkl_status rkl_backward_hidden_multi(const void* h_s, const void* h_t,
+                                    const void* W_s, const void* W_t,
+                                    int32_t n_teachers, const int32_t* teacher_idx,
+                                    const int32_t* counts, rkl_dtype dtype,
+                                    int64_t B, int64_t Sm1, int64_t H, int64_t V,
+                                    const int32_t* row_idx, int32_t N,
+                                    rkl_reduction reduction, const float* saved,
+                                    const float* grad_loss, const float* grad_tok,
+                                    float* dH_s, float* dW_s,
                                     void* workspace, size_t workspace_bytes, void* stream);
 
 /* rkl_forward_hidden without a caller workspace, for callers that cannot

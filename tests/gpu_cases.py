@@ -21,6 +21,8 @@ def run_gpu(inp, reduction, backward=True, grad_loss=1.0, grad_tok=None):
     """Forward (+ backward) of one problem through librkl.so."""
     mask = inp["mask"].cuda()
     B, Sm1 = mask.shape
+    if "teacher_idx" in inp:
+        return _run_gpu_multi(inp, reduction, backward, grad_loss, grad_tok)
     row_idx, N = rb.compact_rows(mask)
     payload = rb.PAYLOAD_LOGITS if "teacher_logits" in inp else rb.PAYLOAD_HIDDEN
     h_s = inp["h_s"].cuda()
@@ -43,10 +45,37 @@ def run_gpu(inp, reduction, backward=True, grad_loss=1.0, grad_tok=None):
     return out
 
 
+def _run_gpu_multi(inp, reduction, backward, grad_loss, grad_tok):
+    mask = inp["mask"].cuda()
+    B, Sm1 = mask.shape
+    h_s, h_t, W_s, W_t = (inp[k].cuda() for k in ("h_s", "h_t", "W_s", "W_t"))
+    tid = inp["teacher_idx"].cuda()
+    row_idx, N, counts = rb.compact_rows_multi(mask, tid, W_t.shape[0])
+    loss_tok, loss, saved = rb.forward_hidden_multi(h_s, h_t, W_s, W_t, tid, counts, B, Sm1, row_idx, N, reduction)
+    out = {"row_idx": row_idx[:N].cpu().numpy(), "N": N, "counts": counts, "loss_tok": loss_tok, "loss": loss,
+           "saved": saved[:N]}
+    if backward:
+        gl = torch.tensor([grad_loss], dtype=torch.float32, device="cuda")
+        gt = None if grad_tok is None else torch.as_tensor(grad_tok, dtype=torch.float32).cuda()
+        out["dH_s"], out["dW_s"] = rb.backward_hidden_multi(h_s, h_t, W_s, W_t, tid, counts, B, Sm1, row_idx, N,
+                                                            reduction, saved, grad_loss=gl, grad_tok=gt)
+    torch.cuda.synchronize()
+    assert rb.device_error() == 0
+    return out
+
+
 def run_oracle(inp, reduction, backward=True, grad_loss=1.0, grad_tok=None):
     h_s = to_np(inp["h_s"])
     W_s = to_np(inp["W_s"])
     mask = inp["mask"].cpu().numpy()
+    if "teacher_idx" in inp:
+        h_t, W_t = to_np(inp["h_t"]), to_np(inp["W_t"])
+        tid = inp["teacher_idx"].cpu().numpy()
+        out = O.forward_multi(h_s, W_s, h_t, W_t, tid, mask, reduction)
+        if backward:
+            out["dH_s"], out["dW_s"] = O.backward_multi(h_s, W_s, h_t, W_t, tid, mask, reduction,
+                                                        grad_loss=grad_loss, grad_tok=grad_tok)
+        return out
     if "teacher_logits" in inp:
         teacher, W_t = to_np(inp["teacher_logits"]), None
     else:
@@ -78,6 +107,7 @@ def grad_rel_err(gpu, ref):
 
 
 def small_case(B=2, Sm1=100, H=128, V=1000, dtype="bf16", payload="hidden", mask="random", weights="perturbed",
-               seed=0, teacher_noise=0.05):
+               seed=0, teacher_noise=0.05, n_teachers=1, teacher_assign="sequence"):
     return make_inputs(B, Sm1, H, V, dtype=dtype, payload=payload, mask=mask, weights=weights, seed=seed,
-                       device="cpu", teacher_noise=teacher_noise)
+                       device="cpu", teacher_noise=teacher_noise, n_teachers=n_teachers,
+                       teacher_assign=teacher_assign)

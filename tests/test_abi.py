@@ -128,3 +128,28 @@ def test_binding_raises_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(binding, "_lib", None)
     with pytest.raises(binding.RKLError):
         binding.lib()
+
+
+def test_multi_teacher_argument_errors(L):
+    sz = ctypes.c_size_t()
+    assert L.rkl_workspace_size_multi(0, 4096, 2, 4, 2048, 2048, 151936, ctypes.byref(sz)) == 0
+    two = sz.value
+    assert L.rkl_workspace_size_multi(0, 4096, 1, 4, 2048, 2048, 151936, ctypes.byref(sz)) == 0
+    assert sz.value < two              # one extra pair tile of rows per extra teacher, plus slot maps
+    assert L.rkl_workspace_size_multi(0, 4096, 0, 4, 2048, 2048, 151936, ctypes.byref(sz)) == 2
+    assert L.rkl_workspace_size_multi(0, 4096, 17, 4, 2048, 2048, 151936, ctypes.byref(sz)) == 2
+
+    def fwd(counts, n_teachers=2, N=4, tid=GOOD):
+        arr = (ctypes.c_int32 * len(counts))(*counts)
+        return L.rkl_forward_hidden_multi(_fake(GOOD), _fake(GOOD), _fake(GOOD), _fake(GOOD), n_teachers,
+                                          _fake(tid) if tid else None, arr, 0, 2, 3, 64, 128, _fake(GOOD), N, 1,
+                                          _fake(GOOD), _fake(GOOD), _fake(GOOD), _fake(GOOD), 1 << 40, None)
+    assert fwd([1, 2]) == 2            # counts add up to 3, N = 4
+    assert b"counts" in L.rkl_last_error()
+    assert fwd([1, -1, 4], n_teachers=3) == 2
+    assert fwd([2, 2], n_teachers=20) == 2
+    assert fwd([2, 2], tid=0) == 1
+    assert fwd([2, 2], tid=GOOD + 4) == 4
+    assert L.rkl_compact_rows_multi(_fake(GOOD), None, 2, 3, 2, _fake(GOOD), _fake(GOOD), _fake(GOOD), None) == 1
+    assert L.rkl_compact_rows_multi(_fake(GOOD), _fake(GOOD), 2, 3, 0, _fake(GOOD), _fake(GOOD), _fake(GOOD),
+                                    None) == 2
