@@ -49,7 +49,7 @@ constexpr int kBM = 128;       // rows per tile (TMEM lanes)
 constexpr int kBN = 128;       // vocab tile granularity of the statistics groups / chunks
 constexpr int kFBN = 256;      // vocab columns per fused pair tile
 constexpr int kBK = 64;        // K per pipeline stage (128 B of bf16)
-constexpr int kGradBN = 256;   // H columns per gradient tile
+constexpr int kGradBN = 512;   // H columns per gradient pair tile (two N = 256 halves)
 constexpr int kGroupTiles = 4;  // 256-column vocab tiles per forward statistics group (1024 columns)
 constexpr int kStatVals = 6;    // per slot: m_s, S_s, A, m_t, S_t, sum e^(z_s-m_s) z_s
 constexpr int kMaxTeachers = 16;  // teacher heads of the per-row-teacher mode

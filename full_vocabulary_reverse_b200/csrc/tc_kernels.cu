@@ -1,9 +1,9 @@
 // tc_kernels.cu -- tcgen05 (5th-generation tensor core) kernels of the loss.
 //
-// fused_kernel<NG, DZ>   S3 / S6: per 128-row tile of the compacted rows,
-//   stream 128-wide vocab tiles of the LM head(s) through TMA -> shared memory
-//   -> tcgen05.mma -> TMEM, and reduce each tile in the epilogue without ever
-//   writing logits to global memory.
+// fused_kernel<NG, DZ>   S3 / S6: per 256-row tile of the compacted rows (one
+//   CTA pair), stream 256-wide vocab tiles of the LM head(s) through TMA ->
+//   shared memory -> tcgen05.mma -> TMEM, and reduce each tile in the epilogue
+//   without ever writing logits to global memory.
 //     NG = 2: hidden-state payload, z_s = h_s W_s^T and z_t = h_t W_t^T in two
 //             TMEM accumulators ("feat(mopd): add full-vocabulary on-policy
 //             distillation", NeMo RL PR #3978, payload bullet 1).
@@ -18,13 +18,14 @@
 //
 // grad_kernel  S7: grouped persistent GEMM over one vocab chunk,
 //     dW_s[chunk] = dz^T hc_s  and  dHc += dz W_s[chunk]
-//   (chain rule through z_s = h_s W_s^T), fp32 accumulators in TMEM,
-//   TMA store / TMA reduce-add epilogue.
+//   (chain rule through z_s = h_s W_s^T), 256 x 512 tiles per CTA pair, fp32
+//   accumulators in TMEM, TMA store / TMA reduce-add epilogue.
 //
-// Warp roles (192 threads): warp 0 = TMA producer, warp 1 = MMA issuer,
-// warps 2..5 = epilogue (warp w reads TMEM lanes 32*(w%4) .. +31, i.e. one
-// tile row per thread).  Warp 2 also allocates / frees TMEM.  TMEM holds two
-// accumulator slots so the epilogue of tile i overlaps the MMAs of tile i+1.
+// All kernels run on 2-CTA clusters with tcgen05.mma.cta_group::2 issued by
+// one thread of the leader CTA.  Warp roles (320 threads): warp 0 = TMA
+// producer, warp 1 = MMA issuer, warps 2..9 = epilogue (warp w reads TMEM
+// lanes 32*(w%4) .. +31, i.e. one tile row per thread, and half of the
+// columns).  Warp 2 also allocates / frees TMEM.
 #include <cuda_bf16.h>
 
 #include "kernels.h"
@@ -529,36 +530,42 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_kernel(const __grid_co
 
 // ============================================================================
 // Grouped gradient GEMM: dW_s tiles (A = dz^T, MN-major; B = hc_s, MN-major)
-// then dH tiles (A = dz, K-major; B = W_s, MN-major).  128 x 256 tiles.
+// then dH tiles (A = dz, K-major; B = W_s, MN-major).  256 x 512 pair tiles.
 // ============================================================================
 namespace {
-constexpr int kGA = kBM * kBK * 2;             // 16 KB: this CTA's 128 rows of A
-constexpr int kGB = (kGradBN / 2) * kBK * 2;   // 16 KB: this CTA's half of B
-constexpr int kGStage = kGA + kGB;             // 32 KB
-constexpr int kGStages = 6;
-constexpr int kGTmemCols = 2 * kGradBN;  // 512
-constexpr int kSched = 2;                // tile-index broadcast ring depth
+constexpr int kGA = kBM * kBK * 2;           // 16 KB: this CTA's 128 rows of A
+constexpr int kGBP = 128 * kBK * 2;          // 16 KB: one 128-column piece of B
+constexpr int kGStage = kGA + 2 * kGBP;      // 48 KB: A + this CTA's two B pieces
+constexpr int kGStages = 4;
+constexpr int kGTmemCols = kGradBN;          // 512: one 256 x 512 accumulator (two N = 256 halves)
+constexpr int kSched = 2;                    // tile-index broadcast ring depth
 }  // namespace
 
-// One 2-CTA cluster computes a 256 x 256 tile with tcgen05.mma.cta_group::2:
-// CTA rank r holds rows [128 r, 128 r + 128) of A and columns
-// [128 r, 128 r + 128) of B in its own shared memory, and receives rows
-// [128 r, 128 r + 128) of D in its own TMEM.  Each CTA therefore streams only
-// half of the B operand, halving the L2 -> shared-memory bytes per flop of a
-// single-CTA 128 x 256 tile.  The leader (rank 0) issues the MMAs and owns
-// the operand-full barriers (both CTAs' TMA loads count on them), the
-// accumulator-empty barriers (both CTAs' epilogues arrive) and the tile
-// scheduler (it claims tiles with an atomic counter and writes each index
-// into both CTAs' rings).
+// One 2-CTA cluster computes a 256 x 512 tile as two tcgen05.mma.cta_group::2
+// products of N = 256 that share the A operand: CTA rank r holds rows
+// [128 r, 128 r + 128) of A, and for half j = 0, 1 the columns
+// [256 j + 128 r, 256 j + 128 r + 128) of B, and receives rows
+// [128 r, 128 r + 128) of D in its own TMEM (columns [256 j, 256 j + 256) =
+// half j).  Per 64-deep K step a CTA streams 48 KB (16 KB of A, 32 KB of B)
+// for 2 x 256 x 256 x 64 x 2 flop, a third fewer bytes per flop than a
+// 256 x 256 tile; that matters because these kernels are bound by the
+// L2 -> shared-memory operand feed.  TMEM holds the whole 512-column tile, so
+// the epilogue drains it in two halves: half 0 (all eight epilogue warps)
+// first, then half 1, and the next tile's first MMA into a half waits only
+// for that half.  The leader (rank 0) issues the MMAs and owns the
+// operand-full barriers (both CTAs' TMA loads count on them), the
+// accumulator barriers (both CTAs' epilogues arrive) and the tile scheduler
+// (it claims tiles with an atomic counter and writes each index into both
+// CTAs' rings).
 __global__ void __launch_bounds__(kThreads, 1) grad_kernel(const __grid_constant__ GradArgs p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* stg = smem + kGStages * kGStage;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(stg + 4 * 2 * kStgBoxBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(stg + 8 * kStgBoxBytes);
   uint64_t* full = bars;
   uint64_t* empty = bars + kGStages;
   uint64_t* acc_full = bars + 2 * kGStages;
-  uint64_t* acc_empty = acc_full + 2;
+  uint64_t* acc_empty = acc_full + 1;  // [2]: one per accumulator half
   uint64_t* tear = acc_empty + 2;
   uint64_t* sched_full = tear + 1;             // [kSched]
   uint64_t* sched_empty = sched_full + kSched;  // [kSched]
@@ -576,10 +583,8 @@ __global__ void __launch_bounds__(kThreads, 1) grad_kernel(const __grid_constant
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&acc_full[i], 1);
-      mbar_init(&acc_empty[i], 16);  // 8 epilogue warps in each CTA of the pair
-    }
+    mbar_init(acc_full, 1);
+    for (int i = 0; i < 2; ++i) mbar_init(&acc_empty[i], 16);  // 8 epilogue warps in each CTA of the pair
     for (int i = 0; i < kSched; ++i) {
       mbar_init(&sched_full[i], 1);
       mbar_init(&sched_empty[i], 1 + 8 + 1 + 8);  // leader MMA + epilogues, peer producer + epilogues
@@ -636,8 +641,8 @@ __global__ void __launch_bounds__(kThreads, 1) grad_kernel(const __grid_constant
         // tile tt = (row / vocab block tt / NT, H block tt % NT): the H block is
         // the fast index, so the tiles running together share their A block
         // (a slice of dz) in L2 and each slice of dz is read from memory once.
-        const int m0 = (tt / p.NT) * 2 * kBM + rank * kBM;                 // this CTA's A rows
-        const int n0 = (tt % p.NT) * kGradBN + rank * (kGradBN / 2);       // this CTA's B half
+        const int m0 = (tt / p.NT) * 2 * kBM + rank * kBM;   // this CTA's A rows
+        const int nb = (tt % p.NT) * kGradBN + rank * 128;   // this CTA's first B piece
         const int KB = is_h ? p.KBH : p.KBW;
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait_cluster(&empty[stage], phase ^ 1, abort_flag)) {
@@ -653,13 +658,21 @@ __global__ void __launch_bounds__(kThreads, 1) grad_kernel(const __grid_constant
             // A = dz^T: two 64-wide vocab blocks x 64 rows (K); B = hc_s.
             tma_load_2d_pair(sa, &p.tm_dz_mn, fb, m0, kb * kBK);
             tma_load_2d_pair(sa + kGA / 2, &p.tm_dz_mn, fb, m0 + 64, kb * kBK);
-            tma_load_2d_pair(sb, &p.tm_hs_mn, fb, n0, kb * kBK);
-            tma_load_2d_pair(sb + kGB / 2, &p.tm_hs_mn, fb, n0 + 64, kb * kBK);
           } else {
             // A = dz (K-major); B = W_s rows of the chunk.
             tma_load_2d_pair(sa, &p.tm_dz_k, fb, kb * kBK, m0);
-            tma_load_2d_pair(sb, &p.tm_ws_mn, fb, n0, p.cv0 + kb * kBK);
-            tma_load_2d_pair(sb + kGB / 2, &p.tm_ws_mn, fb, n0 + 64, p.cv0 + kb * kBK);
+          }
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            uint8_t* bp = sb + j * kGBP;
+            const int n = nb + j * (kGradBN / 2);
+            if (!is_h) {
+              tma_load_2d_pair(bp, &p.tm_hs_mn, fb, n, kb * kBK);
+              tma_load_2d_pair(bp + kGBP / 2, &p.tm_hs_mn, fb, n + 64, kb * kBK);
+            } else {
+              tma_load_2d_pair(bp, &p.tm_ws_mn, fb, n, p.cv0 + kb * kBK);
+              tma_load_2d_pair(bp + kGBP / 2, &p.tm_ws_mn, fb, n + 64, p.cv0 + kb * kBK);
+            }
           }
           armed |= 1u << stage;
           last_par = (last_par & ~(1u << stage)) | (phase << stage);
@@ -679,8 +692,8 @@ __global__ void __launch_bounds__(kThreads, 1) grad_kernel(const __grid_constant
     }
   } else if (warp == 1) {
     if (leader && lane == 0) {
-      constexpr uint32_t idesc_w = idesc_bf16(2 * kBM, kGradBN, 1, 1);
-      constexpr uint32_t idesc_h = idesc_bf16(2 * kBM, kGradBN, 0, 1);
+      constexpr uint32_t idesc_w = idesc_bf16(2 * kBM, kGradBN / 2, 1, 1);
+      constexpr uint32_t idesc_h = idesc_bf16(2 * kBM, kGradBN / 2, 0, 1);
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
@@ -696,14 +709,7 @@ __global__ void __launch_bounds__(kThreads, 1) grad_kernel(const __grid_constant
         if (t < 0) break;
         const bool is_h = t < p.nH;
         const int KB = is_h ? p.KBH : p.KBW;
-        const int acc = i & 1;
-        const uint32_t ap = (i >> 1) & 1;
-        if (!mbar_wait_cluster(&acc_empty[acc], ap ^ 1, abort_flag)) {
-          raise_abort(abort_flag, ERR_WAIT_ACC_EMPTY);
-          break;
-        }
-        tc_fence_after();
-        const uint32_t d = tmem_base + acc * kGradBN;
+        const uint32_t ap = i & 1;  // the accumulator is drained once per tile
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(&full[stage], phase, abort_flag)) {
             raise_abort(abort_flag, ERR_WAIT_TMA_FULL);
@@ -714,36 +720,52 @@ __global__ void __launch_bounds__(kThreads, 1) grad_kernel(const __grid_constant
           const uint32_t sa = smem_u32(smem + stage * kGStage);
           const uint32_t sb = sa + kGA;
 #pragma unroll
-          for (int k = 0; k < kBK / 16; ++k) {
-            const uint32_t acc_flag = (kb | k) != 0;
-            if (!is_h)
-              umma_bf16_pair(d, sdesc_sw128(sa + 2048 * k, kGA / 2, 1024), sdesc_sw128(sb + 2048 * k, kGB / 2, 1024),
-                             idesc_w, acc_flag);
-            else
-              umma_bf16_pair(d, sdesc_sw128(sa + 32 * k, 16, 1024), sdesc_sw128(sb + 2048 * k, kGB / 2, 1024),
-                             idesc_h, acc_flag);
+          for (int j = 0; j < 2; ++j) {
+            if (kb == 0) {
+              // the previous tile's epilogue must have read this half out
+              if (!mbar_wait_cluster(&acc_empty[j], ap ^ 1, abort_flag)) {
+                raise_abort(abort_flag, ERR_WAIT_ACC_EMPTY);
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+            }
+            const uint32_t d = tmem_base + j * (kGradBN / 2);
+            const uint32_t bj = sb + j * kGBP;
+#pragma unroll
+            for (int k = 0; k < kBK / 16; ++k) {
+              const uint32_t acc_flag = (kb | k) != 0;
+              if (!is_h)
+                umma_bf16_pair(d, sdesc_sw128(sa + 2048 * k, kGA / 2, 1024), sdesc_sw128(bj + 2048 * k, kGBP / 2, 1024),
+                               idesc_w, acc_flag);
+              else
+                umma_bf16_pair(d, sdesc_sw128(sa + 32 * k, 16, 1024), sdesc_sw128(bj + 2048 * k, kGBP / 2, 1024),
+                               idesc_h, acc_flag);
+            }
           }
+          if (!ok) break;
           umma_commit_pair(&empty[stage], 0x3);
           if (++stage == kGStages) {
             stage = 0;
             phase ^= 1;
           }
         }
-        if (ok) umma_commit_pair(&acc_full[acc], 0x3);
+        if (ok) umma_commit_pair(acc_full, 0x3);
       }
       umma_commit_pair(tear, 0x1);
       volatile int never = 0;
       if (!mbar_wait(tear, 0, &never)) atomicOr(&g_dev_err, ERR_WAIT_TEARDOWN);
     }
   } else {
-    // Warp w reads TMEM lane quarter w % 4 and columns [128 h, 128 h + 128)
-    // of the 256-column accumulator, h = (w - 2) / 4.
+    // Warp w reads TMEM lane quarter w % 4.  Half 0 of the accumulator is
+    // drained first by all eight warps (warp w takes columns
+    // [128 s, 128 s + 128) of the half, s = (w - 2) / 4), then half 1.
     const int q = warp & 3;
-    const int half = (warp - 2) >> 2;
+    const int sub = (warp - 2) >> 2;
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
     const uint32_t sched_empty0 = mapa_shared(smem_u32(sched_empty), 0);
     const uint32_t acc_empty0 = mapa_shared(smem_u32(acc_empty), 0);
-    int box = 0;
+    uint8_t* buf = stg + (warp - 2) * kStgBoxBytes;  // one staging box per warp
     for (int i = 0;; ++i) {
       const int slot = i % kSched;
       const uint32_t sp = (i / kSched) & 1;
@@ -761,49 +783,49 @@ __global__ void __launch_bounds__(kThreads, 1) grad_kernel(const __grid_constant
       const int tt = is_h ? t : t - p.nH;
       const int mtile = tt / p.NT;
       const int n0 = (tt % p.NT) * kGradBN;
-      const int acc = i & 1;
-      const uint32_t ap = (i >> 1) & 1;
-      ok = mbar_wait_cluster(&acc_full[acc], ap, abort_flag);
+      ok = mbar_wait_cluster(acc_full, i & 1, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) {
         if (lane == 0) raise_abort(abort_flag, ERR_WAIT_ACC_FULL);
         break;
       }
       tc_fence_after();
-      const uint32_t tb = tmem_base + lane_off + acc * kGradBN + half * (kGradBN / 2);
       const int rows = mtile * 2 * kBM + rank * kBM + q * 32;
       const int row0 = is_h ? rows : p.cv0 + rows;
-      const int c0 = n0 + half * (kGradBN / 2);
 #pragma unroll 1
-      for (int c = 0; c < kGradBN / 2 / 32; ++c) {
-        float v[32];
-        tmem_ld_32x32(tb + c * 32, v);
-        tmem_wait_ld();
-        if (c == kGradBN / 2 / 32 - 1) {
-          tc_fence_before();
+      for (int j = 0; j < 2; ++j) {
+        const int col = j * (kGradBN / 2) + sub * 128;  // first column of this warp in the tile
+        const uint32_t tb = tmem_base + lane_off + col;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          float v[32];
+          tmem_ld_32x32(tb + c * 32, v);
+          tmem_wait_ld();
+          if (c == 3) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(acc_empty0 + j * 8);
+          }
+          if (lane == 0) bulk_wait_read<0>();
           __syncwarp();
-          if (lane == 0) mbar_arrive_cluster(acc_empty0 + acc * 8);
-        }
-        uint8_t* buf = stg + (warp - 2) * kStgBoxBytes;  // one staging box per warp
-        if (lane == 0) bulk_wait_read<0>();
-        __syncwarp();
-        const uint32_t rbase = smem_u32(buf) + lane * 128;
+          const uint32_t rbase = smem_u32(buf) + lane * 128;
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-          st_shared_v4(rbase + ((j ^ (lane & 7)) << 4), __float_as_uint(v[4 * j]), __float_as_uint(v[4 * j + 1]),
-                       __float_as_uint(v[4 * j + 2]), __float_as_uint(v[4 * j + 3]));
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          if (!is_h)
-            tma_store_2d(&p.tm_dw, buf, c0 + c * 32, row0);
-          else if (p.dh_accumulate)
-            tma_reduce_add_2d(&p.tm_dh, buf, c0 + c * 32, row0);
-          else
-            tma_store_2d(&p.tm_dh, buf, c0 + c * 32, row0);
-          bulk_commit();
+          for (int e = 0; e < 8; ++e)
+            st_shared_v4(rbase + ((e ^ (lane & 7)) << 4), __float_as_uint(v[4 * e]), __float_as_uint(v[4 * e + 1]),
+                         __float_as_uint(v[4 * e + 2]), __float_as_uint(v[4 * e + 3]));
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            const int cx = n0 + col + c * 32;
+            if (!is_h)
+              tma_store_2d(&p.tm_dw, buf, cx, row0);
+            else if (p.dh_accumulate)
+              tma_reduce_add_2d(&p.tm_dh, buf, cx, row0);
+            else
+              tma_store_2d(&p.tm_dh, buf, cx, row0);
+            bulk_commit();
+          }
         }
-        ++box;
       }
     }
     if (lane == 0) bulk_wait<0>();
@@ -828,7 +850,7 @@ size_t fused_smem_bytes(int ng, bool dz) {
   return dz ? fused_smem<1, true>() : fused_smem<1, false>();
 }
 
-size_t grad_smem_bytes() { return 1024 + size_t(kGStages) * kGStage + 4 * 2 * kStgBoxBytes + 512; }
+size_t grad_smem_bytes() { return 1024 + size_t(kGStages) * kGStage + 8 * kStgBoxBytes + 512; }
 
 cudaError_t tc_setup(int /*device*/) {
   cudaError_t e;
