@@ -146,7 +146,7 @@ static rkl_status make_map(CUtensorMap* m, const void* ptr, bool f32, uint64_t i
 }
 
 // ------------------------------------------------------------------ plan
-constexpr int kVcBf16 = 16384;  // vocab chunk of the backward (multiple of kFBN)
+constexpr int kVcBf16 = 65536;  // widest vocab chunk of the backward (multiple of kFBN)
 constexpr int kVcF32 = 1024;
 constexpr int kSimtSplits = 37;
 
@@ -176,9 +176,18 @@ static Plan make_plan(rkl_payload payload, rkl_dtype dtype, int64_t n_max, int64
   p.VT = static_cast<int>((V + tile_v - 1) / tile_v);
   // tensor-core path: two statistics slots (column halves) per group
   p.S = bf16 ? 2 * ((p.VT + kGroupTiles - 1) / kGroupTiles) : (p.VT < kSimtSplits ? p.VT : kSimtSplits);
+  // Backward vocab chunks: as few as the widest chunk allows, of equal width
+  // (a multiple of the 256-column tile), so that every gradient launch has the
+  // same work and the tails of the persistent kernels are paid few times.
   const int vc = bf16 ? kVcBf16 : kVcF32;
   const int64_t vround = ((V + kFBN - 1) / kFBN) * kFBN;
-  p.Vc = static_cast<int>(vround < vc ? vround : vc);
+  if (bf16) {
+    const int64_t nch = (vround + vc - 1) / vc;
+    const int64_t w = (vround + nch - 1) / nch;
+    p.Vc = static_cast<int>(((w + kFBN - 1) / kFBN) * kFBN);
+  } else {
+    p.Vc = static_cast<int>(vround < vc ? vround : vc);
+  }
   p.nchunks = static_cast<int>((V + p.Vc - 1) / p.Vc);
   size_t off = 256;  // header
   p.off_hcs = off;

@@ -50,7 +50,7 @@ def test_three_teachers_random_rows(red):
 def test_teacher_without_rows_and_several_chunks():
     # four teachers by sequence over three sequences: teacher 3 has no rows;
     # V spans two backward vocab chunks with a ragged tail
-    inp = small_case(B=3, Sm1=200, H=128, V=20000 + 72, payload="hidden_multi", mask="random", seed=32,
+    inp = small_case(B=3, Sm1=200, H=128, V=65536 + 2072, payload="hidden_multi", mask="random", seed=32,
                      n_teachers=4, teacher_assign="sequence")
     g = _check(inp, 1)
     assert g["counts"][3] == 0

@@ -42,9 +42,9 @@ def test_hidden_bf16_forward_backward(red):
 
 
 def test_hidden_bf16_multi_chunk_ragged():
-    # V spans three backward chunks (4096 wide) with a ragged last tile;
-    # N = 300ish rows: three 128-row tiles, the last one partial.
-    inp = small_case(B=2, Sm1=200, H=256, V=9000 + 40, mask="random", seed=5)
+    # V spans three backward chunks (equal widths of at most 65536 columns)
+    # with a ragged last tile; N = 200ish rows: one partial 256-row pair tile.
+    inp = small_case(B=2, Sm1=200, H=256, V=131072 + 1040, mask="random", seed=5)
     g = run_gpu(inp, 1)
     r = run_oracle(inp, 1)
     assert_tok_close(g["loss_tok"], r["loss_tok"])
