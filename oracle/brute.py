@@ -107,3 +107,19 @@ def count_rows_per_teacher(mask, teacher_idx, n_teachers):
                 else:
                     bad += 1
     return counts, bad
+
+
+def topk_estimate_row(z_s, z_t, y, k):
+    """Top-k estimate of one row by loops: the exact reverse-KL terms of the k
+    largest student logits (ties: lower token id first) plus w(y) when the
+    sampled token y is outside them."""
+    p_s = _softmax(z_s)
+    p_t = _softmax(z_t)
+    ranked = sorted(range(len(z_s)), key=lambda v: (-z_s[v], v))
+    S = set(ranked[:max(0, min(k, len(z_s)))])
+    total = 0.0
+    for v in S:
+        total += p_s[v] * (math.log(p_s[v]) - math.log(p_t[v]))
+    if y not in S:
+        total += math.log(p_s[y]) - math.log(p_t[y])
+    return total

@@ -384,3 +384,91 @@ def backward_multi(h_s, W_s, h_t, W_t, teacher_idx, mask, reduction, grad_loss=1
         dH[rows] = dz @ W_s64
         dW += dz.T @ _f64(h_s[rows])
     return dH, dW
+
+
+# ---------------------------------------------------------------------------
+# Top-k estimator.  NeMo RL PR #3978, description: the exact objective is the
+# K = V limit of the top-k MOPD estimator; once the support spans the whole
+# vocabulary the estimator's score-function tail term vanishes.  The page
+# does not write the estimator out; the reading used here:
+#   * support S = the k tokens of largest student logit (ties: lower token id
+#     first) -- the student is the sampling policy of on-policy distillation;
+#   * per-token estimate  L_hat = sum_{v in S} p_s(v) w(v) + [y not in S] w(y),
+#     w = log p_s - log p_t, y = the sampled (target) token of the position:
+#     the exact part over S plus a one-sample estimate of the tail
+#     sum_{v not in S} p_s(v) w(v) (y ~ p_s makes it unbiased);
+#   * gradient estimate w.r.t. z_s, S held fixed:
+#       p_s(v) ([v in S](w(v) + 1) - (L_S + P_S))            (exact part)
+#       + [y not in S](w(y) + 1)(e_y - p_s)(v)                (score function)
+#     with L_S = sum_S p_s w, P_S = sum_S p_s.
+# k = 0 gives the sampled-token gap w(y) that the page's objective replaces;
+# k >= V gives the exact loss and dL/dz = p_s (w - L).
+# ---------------------------------------------------------------------------
+
+def topk_support(z_s, k):
+    """Boolean [n, V] mask of each row's top-k student logits (ties by lower id)."""
+    z_s = _f64(z_s)
+    n, V = z_s.shape
+    mask = np.zeros((n, V), dtype=bool)
+    kk = min(max(int(k), 0), V)
+    for i in range(n):
+        order = np.argsort(-z_s[i], kind="stable")
+        mask[i, order[:kk]] = True
+    return mask
+
+
+def topk_rows(z_s, z_t, y, k, g=None):
+    """Per-row top-k estimate (and its z_s-gradient when row weights g are
+    given) for logit rows z_s, z_t [n, V] and sampled tokens y [n].
+    Returns (L_hat [n], dz [n, V] or None)."""
+    lp_s = log_softmax(_f64(z_s))
+    lp_t = log_softmax(_f64(z_t))
+    p_s = np.exp(lp_s)
+    w = lp_s - lp_t
+    S = topk_support(z_s, k)
+    rows = np.arange(lp_s.shape[0])
+    y = np.asarray(y)
+    L_S = np.sum(np.where(S, p_s * w, 0.0), axis=1)
+    P_S = np.sum(np.where(S, p_s, 0.0), axis=1)
+    out_y = ~S[rows, y]
+    w_y = w[rows, y]
+    L_hat = L_S + np.where(out_y, w_y, 0.0)
+    if g is None:
+        return L_hat, None
+    a = np.where(out_y, w_y + 1.0, 0.0)
+    dz = p_s * (np.where(S, w + 1.0, 0.0) - (L_S + P_S)[:, None])
+    dz -= a[:, None] * p_s
+    dz[rows, y] += a
+    return L_hat, _f64(g)[:, None] * dz
+
+
+def forward_topk_pair(z_s, z_t, targets, k, mask, reduction):
+    """Top-k estimate with both sides as [T, V] logits; targets [B, S-1] are
+    the sampled tokens.  Same outputs as forward_logits_pair (L = L_hat)."""
+    mask = np.asarray(mask)
+    B, Sm1 = mask.shape
+    row_idx, N = compact_rows(mask)
+    yflat = np.asarray(targets).reshape(-1)
+    L = np.zeros(N)
+    for c0 in range(0, N, _ROW_CHUNK):
+        rows = row_idx[c0:c0 + _ROW_CHUNK]
+        L[c0:c0 + len(rows)], _ = topk_rows(z_s[rows], z_t[rows], yflat[rows], k)
+    loss_tok = np.zeros(B * Sm1)
+    loss_tok[row_idx] = L
+    loss = reduce_loss(L, row_idx, B, Sm1, reduction)
+    return {"loss_tok": loss_tok.reshape(B, Sm1), "loss": loss, "L": L, "row_idx": row_idx, "N": N}
+
+
+def backward_topk_pair(z_s, z_t, targets, k, mask, reduction, grad_loss=1.0, grad_tok=None):
+    """Gradient estimate dLoss/dz_s [T, V] of the top-k estimator; exact zero
+    rows at masked positions."""
+    mask = np.asarray(mask)
+    B, Sm1 = mask.shape
+    row_idx, N = compact_rows(mask)
+    g = row_weights(row_idx, B, Sm1, reduction, grad_loss, grad_tok)
+    yflat = np.asarray(targets).reshape(-1)
+    dz = np.zeros(np.asarray(z_s).shape)
+    for c0 in range(0, N, _ROW_CHUNK):
+        rows = row_idx[c0:c0 + _ROW_CHUNK]
+        _, dz[rows] = topk_rows(z_s[rows], z_t[rows], yflat[rows], k, g[c0:c0 + len(rows)])
+    return dz

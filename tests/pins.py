@@ -374,3 +374,100 @@ def multi_teacher_counts_brute(O, rs):
         ref_counts, ref_bad = brute.count_rows_per_teacher(mask.tolist(), tid.tolist(), 4)
         bad += int(list(counts) != ref_counts or n_bad != ref_bad)
     return bad
+
+
+# ----------------------------------------------------------------- top-k estimator
+
+def topk_limits(O, rs):
+    """k >= V: the exact loss and dL/dz = p_s (w - L).  k = 0: the
+    sampled-token gap log p_s(y) - log p_t(y) (scipy) and its score-function
+    gradient (w(y) + 1)(e_y - p_s)."""
+    worst = 0.0
+    n, V = 5, 23
+    z_s = rs.normal(size=(n, V)) * 3
+    z_t = rs.normal(size=(n, V)) * 3
+    y = rs.randint(0, V, size=n)
+    g = rs.uniform(0.5, 2.0, size=n)
+    L, _, _ = O.per_row_kl(z_s, z_t)
+    for k in (V, V + 7):
+        Lk, dz = O.topk_rows(z_s, z_t, y, k, g)
+        worst = max(worst, float(np.max(np.abs(Lk - L))), float(np.max(np.abs(dz - O.dz_rows(z_s, z_t, g)))))
+    L0, dz0 = O.topk_rows(z_s, z_t, y, 0, g)
+    ls = scipy.special.log_softmax(z_s, axis=1)
+    lt = scipy.special.log_softmax(z_t, axis=1)
+    wy = ls[np.arange(n), y] - lt[np.arange(n), y]
+    ref = -np.exp(ls) * (wy + 1.0)[:, None]
+    ref[np.arange(n), y] += wy + 1.0
+    worst = max(worst, float(np.max(np.abs(L0 - wy))), float(np.max(np.abs(dz0 - g[:, None] * ref))))
+    return worst
+
+
+def topk_unbiased(O, rs):
+    """Averaging the estimate and its gradient over the sampled token
+    y ~ p_s gives the exact loss and the exact gradient, for every k."""
+    worst = 0.0
+    V = 17
+    z_s = rs.normal(size=(1, V)) * 2
+    z_t = rs.normal(size=(1, V)) * 2
+    p = scipy.special.softmax(z_s[0])
+    L, _, _ = O.per_row_kl(z_s, z_t)
+    dz_exact = O.dz_rows(z_s, z_t, np.ones(1))
+    for k in (1, 2, 5, 11, 16):
+        EL = 0.0
+        Edz = np.zeros(V)
+        for yy in range(V):
+            Lk, dz = O.topk_rows(z_s, z_t, np.array([yy]), k, np.ones(1))
+            EL += p[yy] * Lk[0]
+            Edz += p[yy] * dz[0]
+        worst = max(worst, abs(EL - L[0]), float(np.max(np.abs(Edz - dz_exact[0]))))
+    return worst
+
+
+def topk_brute(O, rs):
+    """Estimate against the pure-Python loop, on rows with tied logits."""
+    worst = 0.0
+    for _ in range(4):
+        V = 9
+        z_s = rs.randint(-2, 3, size=(3, V)).astype(float)  # many ties
+        z_t = rs.normal(size=(3, V))
+        y = rs.randint(0, V, size=3)
+        for k in (0, 1, 3, 4, 8, 9):
+            Lk, _ = O.topk_rows(z_s, z_t, y, k)
+            for i in range(3):
+                ref = brute.topk_estimate_row(z_s[i].tolist(), z_t[i].tolist(), int(y[i]), k)
+                worst = max(worst, abs(Lk[i] - ref))
+    return worst
+
+
+def topk_support_ties(O, rs):
+    """The support takes the k largest student logits, lower token id first
+    among equal logits (compared with a sort by (-z, id))."""
+    bad = 0
+    for _ in range(5):
+        z = rs.randint(-1, 2, size=(2, 12)).astype(float)
+        for k in (0, 1, 4, 7, 12):
+            S = O.topk_support(z, k)
+            for i in range(2):
+                ranked = sorted(range(12), key=lambda v: (-z[i, v], v))
+                bad += int(sorted(np.flatnonzero(S[i]).tolist()) != sorted(ranked[:k]))
+    return bad
+
+
+def topk_finite_differences(O, rs):
+    """With the sampled token inside the support, the estimate is the exact
+    reverse-KL sum over S; its gradient (S held fixed) against central
+    differences (logits well separated, so S does not move)."""
+    V, k = 10, 4
+    z_s = np.sort(rs.uniform(-3, 3, size=V))[::-1].copy() + np.arange(V)[::-1] * 0.3
+    z_s = z_s[rs.permutation(V)][None, :]
+    z_t = rs.normal(size=(1, V))
+    S = O.topk_support(z_s, k)[0]
+    y = np.array([int(np.flatnonzero(S)[0])])
+    _, dz = O.topk_rows(z_s, z_t, y, k, np.ones(1))
+    eps = 1e-6
+    num = np.zeros(V)
+    for j in range(V):
+        zp = z_s.copy(); zp[0, j] += eps
+        zm = z_s.copy(); zm[0, j] -= eps
+        num[j] = (O.topk_rows(zp, z_t, y, k)[0][0] - O.topk_rows(zm, z_t, y, k)[0][0]) / (2 * eps)
+    return float(np.max(np.abs(dz[0] - num)) / np.max(np.abs(num)))

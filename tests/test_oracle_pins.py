@@ -14,6 +14,7 @@ import types
 import numpy as np
 import pytest
 
+from oracle import brute
 from oracle import rkl_oracle as O
 from tests import pins
 
@@ -305,3 +306,67 @@ def test_multi_teacher_pins_catch_planted_mistakes(old, new, kind):
         assert pins.multi_teacher_brute_force(M, rs) > 1e-6
     else:
         assert pins.multi_teacher_counts_brute(M, rs) > 0
+
+
+# ------------------------------------------------------------ top-k estimator
+
+def test_topk_limits(rs):
+    assert pins.topk_limits(O, rs) < 1e-12
+
+
+def test_topk_unbiased_over_sampled_token(rs):
+    assert pins.topk_unbiased(O, rs) < 1e-12
+
+
+def test_topk_brute_force_with_ties(rs):
+    assert pins.topk_brute(O, rs) < 1e-12
+
+
+def test_topk_support_ties(rs):
+    assert pins.topk_support_ties(O, rs) == 0
+
+
+def test_topk_finite_differences(rs):
+    assert pins.topk_finite_differences(O, rs) < 1e-6
+
+
+def test_topk_pair_masked_rows_and_reduction(rs):
+    z_s = rs.normal(size=(6, 30)) * 2
+    z_t = rs.normal(size=(6, 30)) * 2
+    y = rs.randint(0, 30, size=(2, 3))
+    mask = np.array([[1, 0, 1], [0, 1, 1]], np.uint8)
+    out = O.forward_topk_pair(z_s, z_t, y, 5, mask, 2)
+    assert np.all(out["loss_tok"][mask == 0] == 0)
+    assert abs(out["loss"] - brute.nested_mean(out["loss_tok"].tolist(), mask.tolist())) < 1e-14
+    dz = O.backward_topk_pair(z_s, z_t, y, 5, mask, 2)
+    assert np.all(dz[mask.reshape(-1) == 0] == 0)
+    # k = V reduces to the logits-pair path
+    a = O.forward_topk_pair(z_s, z_t, y, 30, mask, 1)
+    b = O.forward_logits_pair(z_s, z_t, mask, 1)
+    assert np.max(np.abs(a["loss_tok"] - b["loss_tok"])) < 1e-12
+    assert np.max(np.abs(O.backward_topk_pair(z_s, z_t, y, 30, mask, 1) - O.backward_logits_pair(z_s, z_t, mask, 1))) < 1e-12
+
+
+TOPK_MUTATIONS = [
+    # ties broken by higher id
+    ("order = np.argsort(-z_s[i], kind=\"stable\")", "order = V - 1 - np.argsort(-z_s[i][::-1], kind=\"stable\")", "support"),
+    # score-function term without the +1
+    ("a = np.where(out_y, w_y + 1.0, 0.0)", "a = np.where(out_y, w_y, 0.0)", "unbiased"),
+    # tail estimate applied even when y is inside the support
+    ("L_hat = L_S + np.where(out_y, w_y, 0.0)", "L_hat = L_S + w_y", "brute"),
+    # support mass missing from the gradient constant
+    ("- (L_S + P_S)[:, None])", "- (L_S)[:, None])", "limits"),
+]
+
+
+@pytest.mark.parametrize("old,new,kind", TOPK_MUTATIONS)
+def test_topk_pins_catch_planted_mistakes(old, new, kind):
+    M = _mutant(old, new)
+    rs = np.random.RandomState(13)
+    caught = {
+        "support": lambda: pins.topk_support_ties(M, rs) > 0 or pins.topk_brute(M, rs) > 1e-6,
+        "unbiased": lambda: pins.topk_unbiased(M, rs) > 1e-6,
+        "brute": lambda: pins.topk_brute(M, rs) > 1e-6,
+        "limits": lambda: pins.topk_limits(M, rs) > 1e-6,
+    }[kind]()
+    assert caught
