@@ -124,6 +124,8 @@ class Problem:
         self.logits = "teacher_logits" in inp and not self.pair
         self.multi = "teacher_idx" in inp
         self.n_teachers = inp["W_t"].shape[0] if self.multi else 1
+        self.topk = self.pair and "targets" in inp
+        self.k = int(self.cfg.get("k", 0)) if self.topk else None
         self.student = inp["student_logits"] if self.pair else inp["h_s"]
         self.H = 0 if self.pair else inp["h_s"].shape[1]
         self.V = inp["student_logits"].shape[1] if self.pair else inp["W_s"].shape[0]
@@ -146,7 +148,7 @@ class Problem:
         self.ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
         self.loss_tok = torch.empty((self.B, self.Sm1), dtype=torch.float32, device=device)
         self.loss = torch.empty(1, dtype=torch.float32, device=device)
-        self.saved = torch.empty((self.T, 3), dtype=torch.float32, device=device)
+        self.saved = torch.empty(7 * self.T, dtype=torch.float32, device=device)
         if self.pair:
             self.dz = torch.empty_like(self.student)
         else:
@@ -163,9 +165,11 @@ class Problem:
         out = [self.student, self.teacher, self.inp["mask"]]
         if self.multi:
             out.append(self.inp["teacher_idx"])
+        if self.topk:
+            out.append(self.inp["targets"])
         return out
 
-    def step(self, h_s=None, teacher=None, mask=None, teacher_idx=None):
+    def step(self, h_s=None, teacher=None, mask=None, extra=None):
         """S1..S7 for one batch; returns N.  Inputs default to the resident ones."""
         L, p = self.L, self._p
         h_s = self.student if h_s is None else h_s
@@ -173,12 +177,22 @@ class Problem:
         mask = self.inp["mask"] if mask is None else mask
         s = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
         if self.multi:
-            tid = self.inp["teacher_idx"] if teacher_idx is None else teacher_idx
+            tid = self.inp["teacher_idx"] if extra is None else extra
             return self._step_multi(h_s, teacher, mask, tid, s)
         rb._check(L.rkl_compact_rows(p(mask), self.B, self.Sm1, p(self.row_idx), p(self.n_dev), s))
         self.n_host.copy_(self.n_dev, non_blocking=True)
         torch.cuda.current_stream().synchronize()
         N = int(self.n_host[0])
+        if self.topk:
+            tg = self.inp["targets"] if extra is None else extra
+            rb._check(L.rkl_forward_topk_pair(p(h_s), p(teacher), self.dt, self.B, self.Sm1, self.V, p(self.row_idx), N,
+                                              self.k, p(tg), self.reduction, p(self.loss_tok), p(self.loss),
+                                              p(self.saved), p(self.ws), self.ws.numel(), s))
+            rb._check(L.rkl_backward_topk_pair(p(h_s), p(teacher), self.dt, self.B, self.Sm1, self.V, p(self.row_idx),
+                                               N, p(tg), self.reduction, p(self.saved), p(self.grad_loss), None,
+                                               p(self.dz), p(self.ws), self.ws.numel(), s))
+            self.N = N
+            return N
         if self.pair:
             rb._check(L.rkl_forward_logits_pair(p(h_s), p(teacher), self.dt, self.B, self.Sm1, self.V,
                                                 p(self.row_idx), N, self.reduction, p(self.loss_tok), p(self.loss),
@@ -249,6 +263,10 @@ def kernel_profile():
 def algorithmic_work(prob, N):
     """Per-kernel algorithmic flops (tensor kernels) or bytes (bandwidth kernels) of one step."""
     H, V = prob.H, prob.V
+    if prob.topk:
+        # the estimator must read both logit rows once and write dz once
+        return {"topk_fwd": ("hbm", 4.0 * N * V + 28.0 * N),
+                "topk_bwd": ("hbm", 4.0 * N * V + 2.0 * prob.T * V)}
     if prob.pair:
         return {"pair_fwd": ("hbm", 4.0 * N * V + 16.0 * N),
                 "pair_bwd": ("hbm", 4.0 * N * V + 2.0 * prob.T * V)}
@@ -261,7 +279,7 @@ def algorithmic_work(prob, N):
 
 def source_sha():
     h = hashlib.sha256()
-    for f in ("tc_kernels.cu", "small_kernels.cu", "sm100.cuh", "kernels.h", "api.cu"):
+    for f in ("tc_kernels.cu", "small_kernels.cu", "topk_kernels.cu", "sm100.cuh", "kernels.h", "api.cu"):
         with open(os.path.join(ROOT, "full_vocabulary_reverse_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -281,7 +299,7 @@ def traffic_for(kernel):
 
 
 # ----------------------------------------------------------------- arms
-def cpu_oracle_sample(inp, reduction, name, rows=CPU_SAMPLE_ROWS):
+def cpu_oracle_sample(inp, reduction, name, rows=CPU_SAMPLE_ROWS, k=None):
     """Time the float64 oracle (as it stands) on the first `rows` trainable rows."""
     from threadpoolctl import threadpool_info
     from oracle import rkl_oracle as O
@@ -295,8 +313,13 @@ def cpu_oracle_sample(inp, reduction, name, rows=CPU_SAMPLE_ROWS):
     if "student_logits" in inp:
         zs, zt = f64(inp["student_logits"]), f64(inp["teacher_logits"])
         t0 = time.perf_counter()
-        O.forward_logits_pair(zs, zt, sub, reduction)
-        O.backward_logits_pair(zs, zt, sub, reduction)
+        if "targets" in inp:
+            y = inp["targets"].cpu().numpy()
+            O.forward_topk_pair(zs, zt, y, k, sub, reduction)
+            O.backward_topk_pair(zs, zt, y, k, sub, reduction)
+        else:
+            O.forward_logits_pair(zs, zt, sub, reduction)
+            O.backward_logits_pair(zs, zt, sub, reduction)
         dt = time.perf_counter() - t0
     else:
         h_s, W_s = f64(inp["h_s"]), f64(inp["W_s"])
@@ -325,11 +348,11 @@ def run_reference(args, rank, world):
     if rank != 0:
         return
     inp = make_workload(args.workload, device="cpu", **shape_overrides(args))
-    inp.pop("cfg")
+    cfg = inp.pop("cfg")
     red = inp.pop("reduction")
     vals = []
     for i in range(args.warmup + args.steps):
-        r = cpu_oracle_sample(inp, red, args.workload, rows=args.ref_rows)
+        r = cpu_oracle_sample(inp, red, args.workload, rows=args.ref_rows, k=cfg.get("k"))
         if i >= args.warmup:
             vals.append(r)
     v = statistics.median([x["value"] for x in vals])
@@ -467,7 +490,8 @@ def run_gpu(args, rank, world, dist):
         "vs_baseline": None, "dtype": "bf16" if prob.dt == 0 else "fp32", "data": "synthetic",
         "config": {"workload": args.workload, "B": prob.B, "Sm1": prob.Sm1, "H": prob.H, "V": prob.V,
                    "trainable_rows": N, "tokens_T": prob.T,
-                   "payload": "logits_pair" if prob.pair else ("logits" if prob.logits else
+                   "payload": ("logits_pair, top-k estimator k=%d" % prob.k if prob.topk else "logits_pair")
+                   if prob.pair else ("logits" if prob.logits else
                                                                  ("hidden, %d teachers" % prob.n_teachers
                                                                   if prob.multi else "hidden")),
                    "parallelism": "replicas" if world > 1 else "single",
@@ -491,7 +515,7 @@ def run_gpu(args, rank, world, dist):
     }
     if world == 1 and not args.no_cpu_baseline:
         inp = dict(prob.inp)
-        out["cpu_baseline"] = {k: v for k, v in cpu_oracle_sample(inp, prob.reduction, prob.name).items()
+        out["cpu_baseline"] = {k: v for k, v in cpu_oracle_sample(inp, prob.reduction, prob.name, k=prob.k).items()
                                if k not in ("seconds", "rows")}
     print(json.dumps(out), flush=True)
 

@@ -70,6 +70,10 @@ _SIGS = {
                                   _vp, _vp, _vp, _vp, _sz, _vp], _i32),
     "rkl_backward_hidden_multi": ([_vp, _vp, _vp, _vp, _i32, _vp, _vp, _i32, _i64, _i64, _i64, _i64, _vp, _i32, _i32,
                                    _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp], _i32),
+    "rkl_forward_topk_pair": ([_vp, _vp, _i32, _i64, _i64, _i64, _vp, _i32, _i64, _vp, _i32, _vp, _vp, _vp, _vp, _sz,
+                               _vp], _i32),
+    "rkl_backward_topk_pair": ([_vp, _vp, _i32, _i64, _i64, _i64, _vp, _i32, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _sz,
+                                _vp], _i32),
     "rkl_device_error": ([ctypes.POINTER(_i32)], _i32),
     "rkl_kernel_count": ([], _i32),
     "rkl_kernel_name": ([_i32], ctypes.c_char_p),
@@ -254,6 +258,72 @@ def backward_logits_pair(student_logits, teacher_logits, B, Sm1, row_idx, N, red
                                           N, reduction, _ptr(saved), _ptr(grad_loss), _ptr(grad_tok), _ptr(dz),
                                           _ptr(ws), ws.numel(), _stream(dev)))
     return dz
+
+
+# ------------------------------------------------------------ top-k estimator
+
+def forward_topk_pair(student_logits, teacher_logits, targets, k, B, Sm1, row_idx, N, reduction, workspace=None):
+    """Top-k estimator with both sides as logits; targets [B, Sm1] are the
+    sampled tokens.  Returns (loss_tok [B,Sm1], loss [1], saved [7N])."""
+    dev = student_logits.device
+    V = student_logits.shape[1]
+    dt = _dtype_code(student_logits)
+    tg = targets.to(device=dev, dtype=torch.int32).contiguous()
+    loss_tok = torch.empty((B, Sm1), dtype=torch.float32, device=dev)
+    loss = torch.empty(1, dtype=torch.float32, device=dev)
+    saved = torch.empty(7 * max(N, 1), dtype=torch.float32, device=dev)
+    ws = workspace if workspace is not None else _workspace(PAYLOAD_LOGITS_PAIR, dt, max(N, 1), B, Sm1, 64, V, dev)
+    _check(lib().rkl_forward_topk_pair(_ptr(student_logits), _ptr(teacher_logits), dt, B, Sm1, V, _ptr(row_idx), N,
+                                       int(k), _ptr(tg), reduction, _ptr(loss_tok), _ptr(loss), _ptr(saved),
+                                       _ptr(ws), ws.numel(), _stream(dev)))
+    return loss_tok, loss, saved
+
+
+def backward_topk_pair(student_logits, teacher_logits, targets, B, Sm1, row_idx, N, reduction, saved,
+                       grad_loss=None, grad_tok=None, workspace=None, dz=None):
+    """Gradient estimate dLoss/dz_s [T, V] of the top-k estimator."""
+    dev = student_logits.device
+    V = student_logits.shape[1]
+    dt = _dtype_code(student_logits)
+    tg = targets.to(device=dev, dtype=torch.int32).contiguous()
+    if dz is None:
+        dz = torch.empty_like(student_logits)
+    if grad_loss is not None:
+        grad_loss = grad_loss.reshape(1).to(device=dev, dtype=torch.float32).contiguous()
+    if grad_tok is not None:
+        grad_tok = grad_tok.to(device=dev, dtype=torch.float32).contiguous()
+    ws = workspace if workspace is not None else _workspace(PAYLOAD_LOGITS_PAIR, dt, max(N, 1), B, Sm1, 64, V, dev)
+    _check(lib().rkl_backward_topk_pair(_ptr(student_logits), _ptr(teacher_logits), dt, B, Sm1, V, _ptr(row_idx), N,
+                                        _ptr(tg), reduction, _ptr(saved), _ptr(grad_loss), _ptr(grad_tok), _ptr(dz),
+                                        _ptr(ws), ws.numel(), _stream(dev)))
+    return dz
+
+
+class _RKLTopkPair(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, student_logits, teacher_logits, targets, mask, k, reduction):
+        B, Sm1 = mask.shape
+        row_idx, N = compact_rows(mask)
+        loss_tok, loss, saved = forward_topk_pair(student_logits, teacher_logits, targets, k, B, Sm1, row_idx, N,
+                                                  reduction)
+        tg = targets.to(device=student_logits.device, dtype=torch.int32).contiguous()
+        ctx.save_for_backward(student_logits, teacher_logits, tg, row_idx, saved)
+        ctx.meta = (B, Sm1, N, reduction)
+        return loss.reshape(()), loss_tok
+
+    @staticmethod
+    def backward(ctx, g_loss, g_tok):
+        zs, zt, tg, row_idx, saved = ctx.saved_tensors
+        B, Sm1, N, reduction = ctx.meta
+        dz = backward_topk_pair(zs, zt, tg, B, Sm1, row_idx, N, reduction, saved, grad_loss=g_loss, grad_tok=g_tok)
+        return dz, None, None, None, None, None
+
+
+def topk_estimator_logits_pair(student_logits, teacher_logits, targets, mask, k, reduction=REDUCE_TOKEN_MEAN):
+    """Differentiable (loss, loss_tok) of the top-k estimator (both sides as
+    [T, V] logits, targets = sampled tokens); grad to the student logits."""
+    return _RKLTopkPair.apply(student_logits.contiguous(), teacher_logits.contiguous(), targets, mask, int(k),
+                              reduction)
 
 
 # ------------------------------------------------------------ teacher per row

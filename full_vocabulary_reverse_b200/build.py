@@ -19,7 +19,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "librkl.so")
-SOURCES = ["api.cu", "tc_kernels.cu", "small_kernels.cu", "simt_kernels.cu"]
+SOURCES = ["api.cu", "tc_kernels.cu", "small_kernels.cu", "simt_kernels.cu", "topk_kernels.cu"]
 HEADERS = ["kernels.h", "sm100.cuh"]
 
 

@@ -44,7 +44,7 @@ static const char* const kKernelNames[K_COUNT] = {
     "compact_rows", "gather_rows",   "fwd_dual_tc",  "fwd_single_tc", "teacher_lse", "combine_splits",
     "scatter_loss", "reduce_loss",   "row_weights",  "dz_dual_tc",    "dz_single_tc", "grad_dw_dh_tc",
     "scatter_dh",   "fwd_simt_fp32", "dz_simt_fp32", "grad_simt_fp32", "pair_fwd",   "pair_bwd",
-    "count_teachers", "build_slots"};
+    "count_teachers", "build_slots", "topk_fwd", "topk_bwd"};
 
 const char* kernel_name(int id) { return (id >= 0 && id < K_COUNT) ? kKernelNames[id] : nullptr; }
 
@@ -693,6 +693,69 @@ rkl_status rkl_backward_logits_pair(const void* student_logits, const void* teac
                                 grad_loss, grad_tok, rowc, nullptr, s));
   RKL_CUDA(launch_pair_bwd(student_logits, teacher_logits, dtype == RKL_BF16, row_idx, N, n_pad, T,
                            static_cast<int>(V), rowc, dz, s));
+  return RKL_OK;
+}
+
+// ---------------------------------------------------------------- top-k estimator
+static rkl_status check_topk(const void* zs, const void* zt, rkl_dtype dtype, int64_t B, int64_t Sm1, int64_t V,
+                             const int32_t* row_idx, int32_t N, int64_t k, const int32_t* targets, int reduction,
+                             void* workspace, size_t workspace_bytes) {
+  RKL_TRY(check_common(RKL_PAYLOAD_LOGITS_PAIR, dtype, B, Sm1, 64, V, N, reduction));
+  RKL_TRY(check_ptr(zs, "student_logits"));
+  RKL_TRY(check_ptr(zt, "teacher_logits"));
+  RKL_TRY(check_ptr(row_idx, "row_idx"));
+  RKL_TRY(check_ptr(targets, "targets"));
+  RKL_TRY(check_ptr(workspace, "workspace"));
+  if (k < 0) return fail(RKL_ERR_SHAPE, "k = %lld is negative", (long long)k);
+  if (workspace_bytes < pair_workspace_bytes(N))
+    return fail(RKL_ERR_WORKSPACE, "workspace is %zu bytes, %zu needed", workspace_bytes, pair_workspace_bytes(N));
+  return RKL_OK;
+}
+
+rkl_status rkl_forward_topk_pair(const void* student_logits, const void* teacher_logits, rkl_dtype dtype, int64_t B,
+                                 int64_t Sm1, int64_t V, const int32_t* row_idx, int32_t N, int64_t k,
+                                 const int32_t* targets, rkl_reduction reduction, float* loss_tok, float* loss,
+                                 float* saved, void* workspace, size_t workspace_bytes, void* stream) {
+  RKL_TRY(check_topk(student_logits, teacher_logits, dtype, B, Sm1, V, row_idx, N, k, targets, reduction, workspace,
+                     workspace_bytes));
+  RKL_TRY(check_ptr(loss_tok, "loss_tok", false));
+  RKL_TRY(check_ptr(loss, "loss", false));
+  RKL_TRY(check_ptr(saved, "saved", N > 0));
+  int sms = 0;
+  RKL_TRY(device_setup(&sms));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const long long T = B * Sm1;
+  RKL_CUDA(launch_topk_fwd(student_logits, teacher_logits, dtype == RKL_BF16, row_idx, targets, N,
+                           static_cast<int>(V), k, saved, saved + 3 * size_t(N), s));
+  if (loss_tok) RKL_CUDA(launch_scatter_loss(saved, row_idx, N, T, loss_tok, s));
+  if (loss && reduction != RKL_REDUCE_NONE)
+    RKL_CUDA(launch_reduce(saved, row_idx, N, static_cast<int>(B), static_cast<int>(Sm1), reduction, loss, s));
+  return RKL_OK;
+}
+
+rkl_status rkl_backward_topk_pair(const void* student_logits, const void* teacher_logits, rkl_dtype dtype,
+                                  int64_t B, int64_t Sm1, int64_t V, const int32_t* row_idx, int32_t N,
+                                  const int32_t* targets, rkl_reduction reduction, const float* saved,
+                                  const float* grad_loss, const float* grad_tok, void* dz, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
+  RKL_TRY(check_topk(student_logits, teacher_logits, dtype, B, Sm1, V, row_idx, N, 0, targets, reduction, workspace,
+                     workspace_bytes));
+  RKL_TRY(check_ptr(saved, "saved", N > 0));
+  RKL_TRY(check_ptr(grad_loss, "grad_loss", false));
+  RKL_TRY(check_ptr(grad_tok, "grad_tok", false));
+  RKL_TRY(check_ptr(dz, "dz"));
+  int sms = 0;
+  RKL_TRY(device_setup(&sms));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const long long T = B * Sm1;
+  const int64_t n = N < 1 ? 1 : N;
+  const int n_pad = static_cast<int>(((n + 255) / 256) * 256);
+  float* rowc = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + 256);
+  if (N > 0)
+    RKL_CUDA(launch_row_weights(saved, row_idx, N, n_pad, static_cast<int>(B), static_cast<int>(Sm1), reduction,
+                                grad_loss, grad_tok, rowc, nullptr, s));
+  RKL_CUDA(launch_topk_bwd(student_logits, teacher_logits, dtype == RKL_BF16, row_idx, targets, N, n_pad, T,
+                           static_cast<int>(V), saved, N > 0 ? saved + 3 * size_t(N) : nullptr, rowc, dz, s));
   return RKL_OK;
 }
 

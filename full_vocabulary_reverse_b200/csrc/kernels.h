@@ -31,6 +31,8 @@ enum KernelId : int {
   K_PAIR_BWD,         // both sides as logits: dL/dz_s rows, bandwidth bound
   K_COUNT_TEACHERS,   // per-row teachers: trainable rows per teacher
   K_BUILD_SLOTS,      // per-row teachers: teacher-grouped row slots
+  K_TOPK_FWD,         // top-k estimator, both sides as logits: selection + estimate
+  K_TOPK_BWD,         // top-k estimator: gradient estimate rows
   K_COUNT
 };
 
@@ -143,6 +145,15 @@ cudaError_t launch_pair_fwd(const void* zs, const void* zt, bool bf16, const int
                             float* saved, cudaStream_t s);
 cudaError_t launch_pair_bwd(const void* zs, const void* zt, bool bf16, const int32_t* row_idx, int N, int n_pad,
                             long long T, int V, const float* rowc, void* dz, cudaStream_t s);
+
+// Top-k estimator with both sides as logits (topk_kernels.cu).  saved [N, 3]
+// (lse_s, lse_t, estimate), saved_tk [N, 4] (C, a, K* bits, v_last bits).
+cudaError_t launch_topk_fwd(const void* zs, const void* zt, bool bf16, const int32_t* row_idx,
+                            const int32_t* targets, int N, int V, long long k, float* saved, float* saved_tk,
+                            cudaStream_t s);
+cudaError_t launch_topk_bwd(const void* zs, const void* zt, bool bf16, const int32_t* row_idx,
+                            const int32_t* targets, int N, int n_pad, long long T, int V, const float* saved,
+                            const float* saved_tk, const float* rowc, void* dz, cudaStream_t s);
 
 // ---------------------------------------------------------------- fp32 CUDA-core path
 struct SimtArgs {

@@ -23,6 +23,9 @@ Named workloads:
   logits_pair     both sides as bf16 logits [8192, 151936]: student ~ N(0,9),
                   teacher = student + N(0, 0.5^2) + per-row shift U(-20,20);
                   all rows trainable; token mean.
+  logits_pair_topk  logits_pair inputs, top-k estimator with k = 64 and the
+                  sampled token of each position drawn from the student's
+                  softmax (on-policy sample).
   multi_teacher   qwen_hidden shapes and mask with two teacher heads
                   W_t[g] = W_s + N(0, 0.004^2) (independent draws), teacher
                   of sequence b = b mod 2; token mean.
@@ -53,6 +56,9 @@ WORKLOADS = {
                         reduction=REDUCE_TOKEN_MEAN, mask="suffix256", weights="perturbed", seed=1239),
     "logits_pair": dict(dtype="bf16", B=4, Sm1=2048, H=0, V=151936, payload="logits_pair",
                         reduction=REDUCE_TOKEN_MEAN, mask="all", weights="perturbed", seed=1240),
+    "logits_pair_topk": dict(dtype="bf16", B=4, Sm1=2048, H=0, V=151936, payload="logits_pair",
+                             reduction=REDUCE_TOKEN_MEAN, mask="all", weights="perturbed", seed=1242,
+                             targets="sampled", k=64),
     "multi_teacher": dict(dtype="bf16", B=4, Sm1=2048, H=2048, V=151936, payload="hidden_multi",
                           reduction=REDUCE_TOKEN_MEAN, mask="prefix", weights="perturbed", seed=1241,
                           mask_seed=1236, n_teachers=2, teacher_assign="sequence"),
@@ -109,7 +115,7 @@ def make_teacher_idx(assign, B, Sm1, n_teachers, seed):
 
 def make_inputs(B, Sm1, H, V, dtype="bf16", payload="hidden", mask="prefix",
                 weights="perturbed", seed=0, device="cpu", mask_seed=None,
-                logit_std=3.0, teacher_noise=0.004, n_teachers=1, teacher_assign="sequence"):
+                logit_std=3.0, teacher_noise=0.004, n_teachers=1, teacher_assign="sequence", targets=None):
     """Draw one problem.  Returns a dict of torch tensors on `device`:
     h_s [T,H], W_s [V,H], mask uint8 [B,Sm1], and h_t [T,H] + W_t [V,H]
     (hidden payload) or teacher_logits [T,V] (logits payload).  The
@@ -131,6 +137,14 @@ def make_inputs(B, Sm1, H, V, dtype="bf16", payload="hidden", mask="prefix",
             b = a + torch.randn((r1 - r0, V), generator=gen, device=device) * 0.5 + shift[r0:r1]
             zt[r0:r1] = (b if weights != "same" else a).to(tdt)
         out["student_logits"], out["teacher_logits"] = zs, zt
+        if targets == "sampled":
+            # the sampled token of each position, drawn from the student's softmax
+            y = torch.empty(T, dtype=torch.int64, device=device)
+            for r0 in range(0, T, 512):
+                r1 = min(T, r0 + 512)
+                p = torch.softmax(zs[r0:r1].float(), dim=1)
+                y[r0:r1] = torch.multinomial(p, 1, generator=gen).reshape(-1)
+            out["targets"] = y.to(torch.int32).reshape(B, Sm1)
         out["mask"] = torch.from_numpy(make_mask(mask, B, Sm1, seed if mask_seed is None else mask_seed)).to(device)
         return out
     out["h_s"] = _randn((T, H), gen, device).to(tdt)
@@ -186,7 +200,8 @@ def make_workload(name, device="cpu", **overrides):
     inp = make_inputs(cfg["B"], cfg["Sm1"], cfg["H"], cfg["V"], dtype=cfg["dtype"],
                       payload=cfg["payload"], mask=cfg["mask"], weights=cfg["weights"],
                       seed=cfg["seed"], device=device, mask_seed=cfg.get("mask_seed"),
-                      n_teachers=cfg.get("n_teachers", 1), teacher_assign=cfg.get("teacher_assign", "sequence"))
+                      n_teachers=cfg.get("n_teachers", 1), teacher_assign=cfg.get("teacher_assign", "sequence"),
+                      targets=cfg.get("targets"))
     inp["reduction"] = red
     inp["cfg"] = cfg
     return inp

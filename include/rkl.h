@@ -205,6 +205,49 @@ rkl_status rkl_backward_logits_pair(const void* student_logits, const void* teac
                                     void* workspace, size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
+ * Top-k estimator, both sides as [T, V] logits.  PR #3978, description: the
+ * exact objective is the K = V limit of the top-k MOPD estimator, whose
+ * score-function tail term vanishes when the support spans the vocabulary.
+ * The page does not write the estimator out; this library's reading:
+ *   S      = the k largest student logits of the row (ties: lower token id
+ *            first); k = 0 gives an empty support, k >= V the whole row;
+ *   L_hat  = sum_{v in S} p_s(v) w(v) + [y not in S] w(y), w = log p_s -
+ *            log p_t, y = the position's sampled token (targets);
+ *   dz_s   = g (p_s ([v in S](w + 1) - C) + [v = y] a), a = [y not in S]
+ *            (w(y) + 1), C = sum_S p_s w + sum_S p_s + a.
+ * Averaged over y ~ p_s, L_hat and dz_s are the exact loss and gradient; at
+ * k = 0, L_hat is the sampled-token gap w(y); at k >= V they are the exact
+ * ones.  Bandwidth bound: the forward reads the student row 3 (bf16) or 5
+ * (fp32) times and the teacher row once; the backward reads both rows once
+ * and writes dz once.
+ * ------------------------------------------------------------------------ */
+
+/* Forward of the top-k estimator.  targets [B, Sm1] int32 (device): the
+ * sampled token of every position (only trainable positions are read; an id
+ * outside [0, V) gives NaN for that row).  loss_tok / loss as
+ * rkl_forward_logits_pair with L = L_hat.  saved [7 N] floats: [N, 3]
+ * (lse_s, lse_t, L_hat) followed by [N, 4] (C, a, and the bit patterns of
+ * the k-th key and of the last tied token id taken into S), for
+ * rkl_backward_topk_pair.  k >= 0 (RKL_ERR_SHAPE otherwise).  Workspace:
+ * rkl_workspace_size(RKL_PAYLOAD_LOGITS_PAIR, ...). */
+rkl_status rkl_forward_topk_pair(const void* student_logits, const void* teacher_logits,
+                                 rkl_dtype dtype, int64_t B, int64_t Sm1, int64_t V,
+                                 const int32_t* row_idx, int32_t N, int64_t k,
+                                 const int32_t* targets, rkl_reduction reduction,
+                                 float* loss_tok, float* loss, float* saved,
+                                 void* workspace, size_t workspace_bytes, void* stream);
+
+/* Backward of the top-k estimator: dz [T, V] of `dtype` (overwritten) with
+ * exact zero rows at masked positions; row weights g as rkl_backward; saved
+ * and targets from the matching forward call. */
+rkl_status rkl_backward_topk_pair(const void* student_logits, const void* teacher_logits,
+                                  rkl_dtype dtype, int64_t B, int64_t Sm1, int64_t V,
+                                  const int32_t* row_idx, int32_t N, const int32_t* targets,
+                                  rkl_reduction reduction, const float* saved,
+                                  const float* grad_loss, const float* grad_tok, void* dz,
+                                  void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
  * A teacher per row (hidden-state payload).  PR #3978, first-version limits:
  * the first version takes one teacher checkpoint and lays out the payload so
  * that a per-row teacher index can be added.  Here every position carries
