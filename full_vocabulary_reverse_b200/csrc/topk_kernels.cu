@@ -16,18 +16,19 @@
 //
 // Forward, one CTA per trainable row:
 //   pass A  streams z_s and z_t once: online log-sum-exp of both sides and a
-//           256-bin histogram of the top byte of an order-preserving integer
-//           key of z_s;
-//   pass B  (one per further key byte: 1 for bf16, 3 for fp32) histograms the
-//           next byte among the elements whose key matches the bytes chosen
-//           so far; after the last level the key K* of the k-th largest
-//           logit and the number r of elements of key K* that S takes are
-//           known exactly (radix select);
-//   pass C  streams z_s in index order, 2048 (bf16) or 1024 (fp32) elements
-//           per round: elements of key > K* are in S, and elements of key
-//           K* are ranked in index order by a block scan so that the first r
-//           join S (this fixes v_last, the last of them); z_t is read only at
-//           the members of S, which give L_S and P_S.
+//           4096-bin histogram of the top 12 bits of an order-preserving
+//           integer key of z_s; a block scan from the top finds the bin of
+//           the k-th largest key;
+//   pass B  streams z_s once more: keys above that bin are members of S (z_t
+//           is gathered at them), keys in the bin are appended to a list in
+//           shared memory (key, token id); a bitonic sort of the list orders
+//           it by key, lower token id first, and its first r entries (r = k -
+//           members above the bin) complete S, fixing the k-th key K* and
+//           v_last, the last token id of key K* taken.
+//   If the bin holds more than 4096 entries (long runs of tied logits), the
+//   selection finishes exactly instead: radix passes over the remaining key
+//   bits give K*, and an index-ordered pass ranks the ties of key K* by a
+//   block scan.
 // Backward, one CTA per token row: dz_s in one stream over z_s and z_t, S
 // decided by (key > K*) or (key = K* and v <= v_last), exact zero rows at
 // masked positions.
@@ -162,6 +163,39 @@ __device__ __forceinline__ void pick_bin(const int* hist, int need, int* bin, in
   *above = acc;
 }
 
+constexpr int kTopShift = 20;            // first-level histogram: the top 12 key bits
+constexpr int kTopBins = 1 << (32 - kTopShift);
+constexpr int kCap = 4096;               // candidates sorted in shared memory
+
+// Descending bitonic sort of n (a power of two, <= kCap) 64-bit entries in
+// shared memory by the whole block.
+__device__ __forceinline__ void bitonic_desc(unsigned long long* a, int n) {
+  for (int size = 2; size <= n; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int i = threadIdx.x; i < n / 2; i += kTkThreads) {
+        const int lo = 2 * stride * (i / stride) + (i % stride);
+        const int hi = lo + stride;
+        const unsigned long long x = a[lo], y = a[hi];
+        if ((x < y) == ((lo & size) == 0)) {
+          a[lo] = y;
+          a[hi] = x;
+        }
+      }
+      __syncthreads();
+    }
+  }
+}
+
+// One student row's contribution to the sums over S: p_s(v) w(v) and p_s(v).
+template <typename T>
+__device__ __forceinline__ void add_member(float zs_v, const T* zt, int v, float lse_s, float lse_t, float& L_S,
+                                           float& P_S) {
+  const float ls = zs_v - lse_s;
+  const float p = ex2(ls * kLog2e);
+  L_S = fmaf(p, ls - (TkIo<T>::one(zt, v) - lse_t), L_S);
+  P_S += p;
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kTkThreads) topk_fwd_kernel(const T* __restrict__ zs_all,
                                                               const T* __restrict__ zt_all,
@@ -171,11 +205,14 @@ __global__ void __launch_bounds__(kTkThreads) topk_fwd_kernel(const T* __restric
                                                               float* __restrict__ saved_tk) {
   using Io = TkIo<T>;
   constexpr int VEC = Io::VEC;
-  __shared__ int hist[256];
+  // 32 KB: the 4096-bin histogram of pass A, then the candidate list
+  __shared__ unsigned long long buf[kCap];
+  int* hist = reinterpret_cast<int*>(buf);
+  __shared__ int hist2[256];
   __shared__ int scan_sh[32];
   __shared__ float red_sh[4][kTkThreads / 32];
-  __shared__ uint32_t s_prefix;
-  __shared__ int s_need, s_vlast;
+  __shared__ uint32_t s_kstar;
+  __shared__ int s_need, s_vlast, s_ncand, s_bin;
   __shared__ float s_lse[2];
 
   const int kr = blockIdx.x;
@@ -188,29 +225,50 @@ __global__ void __launch_bounds__(kTkThreads) topk_fwd_kernel(const T* __restric
   const int nvec = vec_ok ? V / VEC : 0;
   const uint4* vs = reinterpret_cast<const uint4*>(zs);
   const uint4* vt = reinterpret_cast<const uint4*>(zt);
-  const bool select = k_sel > 0 && k_sel < V;  // else S is empty or the whole row
+  // 0: empty support, 1: the whole row, 2: a proper subset to select
+  const int mode = k_sel <= 0 ? 0 : (k_sel >= V ? 1 : 2);
 
-  for (int i = tid; i < 256; i += kTkThreads) hist[i] = 0;
+  for (int i = tid; i < kTopBins; i += kTkThreads) hist[i] = 0;
+  if (tid == 0) {
+    s_ncand = 0;
+    s_kstar = mode == 0 ? 0xFFFFFFFFu : 0u;  // above every key / below every key
+    s_vlast = mode == 0 ? -1 : INT_MAX;
+  }
   __syncthreads();
 
-  // ---- pass A: both log-sum-exps and the top-byte histogram of z_s
+  // ---- pass A: both log-sum-exps and the 12-bit histogram of the z_s keys
   float m_s = -INFINITY, S_s = 0.f, m_t = -INFINITY, S_t = 0.f;
   for (int i = tid; i < nvec; i += kTkThreads) {
     float xs[VEC], xt[VEC];
     Io::unpack(tk_ldg_v4(vs + i), xs);
     Io::unpack(tk_ldg_v4(vt + i), xt);
+    float cs = xs[0], ct = xt[0];
+#pragma unroll
+    for (int j = 1; j < VEC; ++j) {
+      cs = fmaxf(cs, xs[j]);
+      ct = fmaxf(ct, xt[j]);
+    }
+    if (cs > m_s) {
+      S_s *= ex2((m_s - cs) * kLog2e);
+      m_s = cs;
+    }
+    if (ct > m_t) {
+      S_t *= ex2((m_t - ct) * kLog2e);
+      m_t = ct;
+    }
+    const float ms2 = m_s * kLog2e, mt2 = m_t * kLog2e;
 #pragma unroll
     for (int j = 0; j < VEC; ++j) {
-      lse_add(m_s, S_s, xs[j]);
-      lse_add(m_t, S_t, xt[j]);
-      if (select) atomicAdd(&hist[(Io::KMASK & fkey_raw(xs[j])) >> 24], 1);
+      S_s += ex2(fmaf(xs[j], kLog2e, -ms2));
+      S_t += ex2(fmaf(xt[j], kLog2e, -mt2));
+      if (mode == 2) atomicAdd(&hist[(Io::KMASK & fkey_raw(xs[j])) >> kTopShift], 1);
     }
   }
   for (int v = nvec * VEC + tid; v < V; v += kTkThreads) {
     const float xs = Io::one(zs, v), xt = Io::one(zt, v);
     lse_add(m_s, S_s, xs);
     lse_add(m_t, S_t, xt);
-    if (select) atomicAdd(&hist[(Io::KMASK & fkey_raw(xs)) >> 24], 1);
+    if (mode == 2) atomicAdd(&hist[(Io::KMASK & fkey_raw(xs)) >> kTopShift], 1);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
@@ -232,107 +290,159 @@ __global__ void __launch_bounds__(kTkThreads) topk_fwd_kernel(const T* __restric
     }
     s_lse[0] = a + logf(b);
     s_lse[1] = c + logf(d);
-    if (select) {
-      int bin, above;
-      pick_bin(hist, static_cast<int>(k_sel), &bin, &above);
-      s_prefix = static_cast<uint32_t>(bin) << 24;
-      s_need = static_cast<int>(k_sel) - above;
-    } else {
-      // empty support: a key above every value; whole row: key 0 and no index cap
-      s_prefix = k_sel <= 0 ? 0xFFFFFFFFu : 0u;
-      s_need = 0;
+  }
+  if (mode == 2) {
+    // the bin of the k-th largest key: thread tid owns bins [16 g, 16 g + 16),
+    // g = 255 - tid, so an inclusive scan in thread order counts from the top
+    constexpr int PER = kTopBins / kTkThreads;
+    const int g = kTkThreads - 1 - tid;
+    int sg = 0;
+#pragma unroll
+    for (int j = 0; j < PER; ++j) sg += hist[PER * g + j];
+    int tot;
+    const int incl = block_incl_scan(sg, scan_sh, &tot);
+    const int above = incl - sg;
+    if (above < k_sel && k_sel <= incl) {
+      int acc = above;
+      for (int j = PER - 1; j >= 0; --j) {
+        const int bn = PER * g + j;
+        if (acc + hist[bn] >= k_sel) {
+          s_bin = bn;
+          s_need = static_cast<int>(k_sel) - acc;
+          break;
+        }
+        acc += hist[bn];
+      }
     }
   }
   __syncthreads();
-
-  // ---- pass B: the remaining key bytes of the k-th largest logit
-  if (select) {
-    for (int level = 1; level < Io::LEVELS; ++level) {
-      const int shift = 24 - 8 * level;
-      const uint32_t hi_mask = 0xFFFFFFFFu << (shift + 8);
-      const uint32_t prefix = s_prefix;
-      for (int i = tid; i < 256; i += kTkThreads) hist[i] = 0;
-      __syncthreads();
-      for (int i = tid; i < nvec; i += kTkThreads) {
-        float xs[VEC];
-        Io::unpack(tk_ldg_v4(vs + i), xs);
-#pragma unroll
-        for (int j = 0; j < VEC; ++j) {
-          const uint32_t key = (Io::KMASK & fkey_raw(xs[j]));
-          if ((key & hi_mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1);
-        }
-      }
-      for (int v = nvec * VEC + tid; v < V; v += kTkThreads) {
-        const uint32_t key = (Io::KMASK & fkey_raw(Io::one(zs, v)));
-        if ((key & hi_mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1);
-      }
-      __syncthreads();
-      if (tid == 0) {
-        int bin, above;
-        pick_bin(hist, s_need, &bin, &above);
-        s_prefix = prefix | (static_cast<uint32_t>(bin) << shift);
-        s_need -= above;
-      }
-      __syncthreads();
-    }
-  }
-  // Keys of bf16 values keep only their top 16 bits (KMASK), so after the two
-  // levels s_prefix is the full key K*.
-  const uint32_t kstar = s_prefix;
-  const int need = s_need;  // members of key K*, taken lowest index first
   const float lse_s = s_lse[0], lse_t = s_lse[1];
-
-  // ---- pass C: tie ranks in index order, and the sums over S
   float L_S = 0.f, P_S = 0.f;
-  int carry = 0;
-  if (tid == 0) s_vlast = select ? -1 : (k_sel <= 0 ? -1 : INT_MAX);
-  constexpr int CH = VEC * kTkThreads;
-  for (int c0 = 0; c0 < V; c0 += CH) {
-    const int v0 = c0 + tid * VEC;
-    float xs[VEC];
-    if (vec_ok && v0 + VEC <= V) {
-      Io::unpack(tk_ldg_v4(zs + v0), xs);
-    } else {
+
+  if (mode == 1) {
+    // ---- the whole row is the support
+    for (int i = tid; i < nvec; i += kTkThreads) {
+      float xs[VEC], xt[VEC];
+      Io::unpack(tk_ldg_v4(vs + i), xs);
+      Io::unpack(tk_ldg_v4(vt + i), xt);
 #pragma unroll
-      for (int j = 0; j < VEC; ++j) xs[j] = v0 + j < V ? Io::one(zs, v0 + j) : -INFINITY;
-    }
-    uint32_t keys[VEC];
-    int eq = 0;
-#pragma unroll
-    for (int j = 0; j < VEC; ++j) {
-      keys[j] = v0 + j < V ? (Io::KMASK & fkey_raw(xs[j])) : 0u;
-      eq += (select && v0 + j < V && keys[j] == kstar) ? 1 : 0;
-    }
-    int total = 0;
-    int rank = carry;
-    if (select) {
-      const int incl = block_incl_scan(eq, scan_sh, &total);
-      rank = carry + incl - eq;
-    }
-#pragma unroll
-    for (int j = 0; j < VEC; ++j) {
-      const int v = v0 + j;
-      if (v >= V) continue;
-      bool in;
-      if (select) {
-        in = keys[j] > kstar;
-        if (keys[j] == kstar) {
-          in = rank < need;
-          if (rank == need - 1) s_vlast = v;
-          ++rank;
-        }
-      } else {
-        in = k_sel > 0;
-      }
-      if (in) {
+      for (int j = 0; j < VEC; ++j) {
         const float ls = xs[j] - lse_s;
         const float p = ex2(ls * kLog2e);
-        const float w = ls - (Io::one(zt, v) - lse_t);
-        L_S = fmaf(p, w, L_S);
+        L_S = fmaf(p, ls - (xt[j] - lse_t), L_S);
         P_S += p;
       }
     }
-    carry += total;
+    for (int v = nvec * VEC + tid; v < V; v += kTkThreads) add_member<T>(Io::one(zs, v), zt, v, lse_s, lse_t, L_S, P_S);
+  } else if (mode == 2) {
+    // ---- pass B: keys above the bin are members; keys in the bin are candidates
+    const uint32_t bin = static_cast<uint32_t>(s_bin);
+    const int need = s_need;
+    for (int i = tid; i < nvec; i += kTkThreads) {
+      float xs[VEC];
+      Io::unpack(tk_ldg_v4(vs + i), xs);
+#pragma unroll
+      for (int j = 0; j < VEC; ++j) {
+        const uint32_t key = Io::KMASK & fkey_raw(xs[j]);
+        const uint32_t kb = key >> kTopShift;
+        if (kb > bin) {
+          add_member<T>(xs[j], zt, i * VEC + j, lse_s, lse_t, L_S, P_S);
+        } else if (kb == bin) {
+          const int slot = atomicAdd(&s_ncand, 1);
+          if (slot < kCap) buf[slot] = (static_cast<unsigned long long>(key) << 32) | (~static_cast<uint32_t>(i * VEC + j));
+        }
+      }
+    }
+    for (int v = nvec * VEC + tid; v < V; v += kTkThreads) {
+      const float x = Io::one(zs, v);
+      const uint32_t key = Io::KMASK & fkey_raw(x);
+      const uint32_t kb = key >> kTopShift;
+      if (kb > bin) {
+        add_member<T>(x, zt, v, lse_s, lse_t, L_S, P_S);
+      } else if (kb == bin) {
+        const int slot = atomicAdd(&s_ncand, 1);
+        if (slot < kCap) buf[slot] = (static_cast<unsigned long long>(key) << 32) | (~static_cast<uint32_t>(v));
+      }
+    }
+    __syncthreads();
+    const int nc = s_ncand;
+    if (nc <= kCap) {
+      // ---- the candidates in key order (lower token id first on equal keys)
+      int n2 = 2;
+      while (n2 < nc) n2 <<= 1;
+      for (int i = nc + tid; i < n2; i += kTkThreads) buf[i] = 0ull;
+      __syncthreads();
+      bitonic_desc(buf, n2);
+      for (int j = tid; j < need; j += kTkThreads) {
+        const int v = static_cast<int>(~static_cast<uint32_t>(buf[j]));
+        add_member<T>(Io::one(zs, v), zt, v, lse_s, lse_t, L_S, P_S);
+      }
+      if (tid == 0) {
+        const unsigned long long e = buf[need - 1];
+        s_kstar = static_cast<uint32_t>(e >> 32);
+        s_vlast = static_cast<int>(~static_cast<uint32_t>(e));
+      }
+    } else {
+      // ---- too many candidates: finish the radix select on the lower key
+      // bits, then rank the ties of key K* in index order
+      const int lo_end = Io::KMASK == 0xFFFF0000u ? 16 : 0;
+      uint32_t prefix = bin << kTopShift;
+      int rem = need;
+      for (int hi = kTopShift; hi > lo_end;) {
+        const int width = hi - lo_end < 8 ? hi - lo_end : 8;
+        const int sh = hi - width;
+        for (int i = tid; i < 256; i += kTkThreads) hist2[i] = 0;
+        __syncthreads();
+        for (int v = tid; v < V; v += kTkThreads) {
+          const uint32_t key = Io::KMASK & fkey_raw(Io::one(zs, v));
+          if ((key >> hi) == (prefix >> hi)) atomicAdd(&hist2[(key >> sh) & ((1u << width) - 1u)], 1);
+        }
+        __syncthreads();
+        if (tid == 0) {
+          int bn, ab;
+          pick_bin(hist2, rem, &bn, &ab);
+          s_bin = bn;
+          s_need = rem - ab;
+        }
+        __syncthreads();
+        prefix |= static_cast<uint32_t>(s_bin) << sh;
+        rem = s_need;
+        hi = sh;
+        __syncthreads();
+      }
+      const uint32_t kstar = prefix;
+      int carry = 0;
+      constexpr int CH = VEC * kTkThreads;
+      for (int c0 = 0; c0 < V; c0 += CH) {
+        const int v0 = c0 + tid * VEC;
+        float xs[VEC];
+        uint32_t keys[VEC];
+        int eq = 0;
+#pragma unroll
+        for (int j = 0; j < VEC; ++j) {
+          xs[j] = v0 + j < V ? Io::one(zs, v0 + j) : -INFINITY;
+          keys[j] = v0 + j < V ? (Io::KMASK & fkey_raw(xs[j])) : 0u;
+          eq += (v0 + j < V && keys[j] == kstar) ? 1 : 0;
+        }
+        int total;
+        const int incl = block_incl_scan(eq, scan_sh, &total);
+        int rank = carry + incl - eq;
+#pragma unroll
+        for (int j = 0; j < VEC; ++j) {
+          const int v = v0 + j;
+          if (v >= V || (keys[j] >> kTopShift) != bin) continue;  // keys above the bin are counted
+          bool in = keys[j] > kstar;
+          if (keys[j] == kstar) {
+            in = rank < rem;
+            if (rank == rem - 1) s_vlast = v;
+            ++rank;
+          }
+          if (in) add_member<T>(xs[j], zt, v, lse_s, lse_t, L_S, P_S);
+        }
+        carry += total;
+      }
+      if (tid == 0) s_kstar = kstar;
+    }
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
@@ -351,6 +461,7 @@ __global__ void __launch_bounds__(kTkThreads) topk_fwd_kernel(const T* __restric
       ls += red_sh[0][w];
       ps += red_sh[1][w];
     }
+    const uint32_t kstar = s_kstar;
     const int vlast = s_vlast;
     const int y = targets[r];
     float Lh, a;
@@ -359,7 +470,7 @@ __global__ void __launch_bounds__(kTkThreads) topk_fwd_kernel(const T* __restric
       a = Lh;
     } else {
       const float zy = Io::one(zs, y);
-      const uint32_t ky = (Io::KMASK & fkey_raw(zy));
+      const uint32_t ky = Io::KMASK & fkey_raw(zy);
       const bool y_in = ky > kstar || (ky == kstar && y <= vlast);
       const float wy = (zy - lse_s) - (Io::one(zt, y) - lse_t);
       Lh = ls + (y_in ? 0.f : wy);

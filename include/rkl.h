@@ -217,9 +217,10 @@ rkl_status rkl_backward_logits_pair(const void* student_logits, const void* teac
  *            (w(y) + 1), C = sum_S p_s w + sum_S p_s + a.
  * Averaged over y ~ p_s, L_hat and dz_s are the exact loss and gradient; at
  * k = 0, L_hat is the sampled-token gap w(y); at k >= V they are the exact
- * ones.  Bandwidth bound: the forward reads the student row 3 (bf16) or 5
- * (fp32) times and the teacher row once; the backward reads both rows once
- * and writes dz once.
+ * ones.  Bandwidth bound: the forward reads the student row twice and the
+ * teacher row once (plus the few teacher entries of S); rows whose k-th
+ * logit sits in a run of more than 4096 near-equal logits take extra exact
+ * passes.  The backward reads both rows once and writes dz once.
  * ------------------------------------------------------------------------ */
 
 /* Forward of the top-k estimator.  targets [B, Sm1] int32 (device): the

@@ -146,3 +146,19 @@ def test_topk_full_size():
     assert np.max(np.abs(g_dz - dz_ref)) / np.max(np.abs(dz_ref)) < GRAD_RTOL
     rs_ = dz.double().sum(dim=1).abs()
     assert float((rs_ / dz.double().abs().sum(dim=1)).max()) < 1e-2
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+@pytest.mark.parametrize("k", [100, 3000, 8999])
+def test_topk_many_ties_take_the_exact_path(dtype, k):
+    # student logits drawn from three values: the bin of the k-th logit holds
+    # thousands of tied entries, more than the shared-memory candidate list,
+    # so the selection finishes with the exact radix / index-order path
+    inp, y = _case(2, 20, 9000, dtype=dtype, seed=k)
+    rs = np.random.RandomState(k)
+    vals = rs.choice([-1.0, 0.5, 2.0], size=inp["student_logits"].shape, p=[0.2, 0.5, 0.3])
+    inp["student_logits"] = torch.from_numpy(vals).to(inp["student_logits"].dtype)
+    lt, loss, dz, N = _run(inp, y, k, 1)
+    ref, dz_ref = _ref(inp, y, k, 1)
+    assert_tok_close(lt, ref["loss_tok"])
+    assert grad_rel_err(dz, dz_ref) < (GRAD_RTOL if dtype == "bf16" else 1e-4)
