@@ -162,3 +162,18 @@ def test_multi_teacher_full_size():
     off = ~inp["mask"].reshape(-1).bool()
     assert float(torch.count_nonzero(lt.reshape(-1)[off])) == 0
     assert float(torch.count_nonzero(dH[off])) == 0
+
+
+def test_autograd_wrapper_several_teachers():
+    inp = small_case(B=2, Sm1=100, H=128, V=700, payload="hidden_multi", mask="random", seed=39, n_teachers=3,
+                     teacher_assign="random")
+    h_s = inp["h_s"].cuda().requires_grad_(True)
+    W_s = inp["W_s"].cuda().requires_grad_(True)
+    loss, loss_tok = rb.reverse_kl_hidden_multi(h_s, inp["h_t"].cuda(), W_s, inp["W_t"].cuda(),
+                                                inp["teacher_idx"].cuda(), inp["mask"].cuda(), 2)
+    (loss + 0.5 * loss_tok.sum()).backward()
+    gt = np.full(inp["mask"].shape, 0.5)
+    r = run_oracle(inp, 2, grad_tok=gt)
+    assert abs(float(loss.detach()) - r["loss"]) <= 1e-4 + 1e-3 * abs(r["loss"])
+    assert grad_rel_err(h_s.grad.float(), r["dH_s"]) < GRAD_RTOL
+    assert grad_rel_err(W_s.grad.float(), r["dW_s"]) < GRAD_RTOL

@@ -162,3 +162,14 @@ def test_topk_many_ties_take_the_exact_path(dtype, k):
     ref, dz_ref = _ref(inp, y, k, 1)
     assert_tok_close(lt, ref["loss_tok"])
     assert grad_rel_err(dz, dz_ref) < (GRAD_RTOL if dtype == "bf16" else 1e-4)
+
+
+def test_topk_autograd_wrapper():
+    inp, y = _case(2, 50, 1024, seed=21)
+    zs = inp["student_logits"].cuda().requires_grad_(True)
+    loss, loss_tok = rb.topk_estimator_logits_pair(zs, inp["teacher_logits"].cuda(), y.cuda(), inp["mask"].cuda(),
+                                                   32, 1)
+    loss.backward()
+    ref, dz_ref = _ref(inp, y, 32, 1)
+    assert abs(float(loss.detach()) - ref["loss"]) <= 1e-4 + 1e-3 * abs(ref["loss"])
+    assert grad_rel_err(zs.grad.float(), dz_ref) < GRAD_RTOL
