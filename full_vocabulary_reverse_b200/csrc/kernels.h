@@ -48,7 +48,6 @@ struct LaunchScope {
 };
 
 constexpr int kBM = 128;       // rows per tile (TMEM lanes)
-constexpr int kBN = 128;       // vocab tile granularity of the statistics groups / chunks
 constexpr int kFBN = 256;      // vocab columns per fused pair tile
 constexpr int kBK = 64;        // K per pipeline stage (128 B of bf16)
 constexpr int kGradBN = 512;   // H columns per gradient pair tile (two N = 256 halves)

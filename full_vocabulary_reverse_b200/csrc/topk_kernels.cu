@@ -103,10 +103,6 @@ struct TkIo<float> {
   __device__ static float cvt(float x) { return x; }
 };
 
-struct Lse2 {
-  float m_s, S_s, m_t, S_t;
-};
-
 __device__ __forceinline__ void lse_add(float& m, float& S, float x) {
   if (x > m) {
     S = S * ex2((m - x) * kLog2e) + 1.f;
