@@ -35,6 +35,7 @@
 #include <cuda_bf16.h>
 
 #include <climits>
+#include <type_traits>
 
 #include "kernels.h"
 #include "sm100.cuh"
@@ -59,6 +60,18 @@ __device__ __forceinline__ uint4 tk_ldg_v4(const void* p) {
 __device__ __forceinline__ uint32_t fkey_raw(float x) {
   const uint32_t u = x == 0.f ? 0u : __float_as_uint(x);
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Keys of the two bf16 values packed in a 32-bit word, each in its half of the
+// result (the same order-preserving map, applied to both halves at once: a
+// positive value's sign bit is set, a negative value's bits are inverted, and
+// -0 takes the key of +0).
+__device__ __forceinline__ uint32_t bf16_pair_keys(uint32_t w) {
+  const uint32_t neg = ((w >> 15) & 0x00010001u) * 0x7FFFu;
+  uint32_t key = (w ^ 0x80008000u) ^ neg;
+  if ((key & 0xFFFFu) == 0x7FFFu) key += 1u;
+  if ((key >> 16) == 0x7FFFu) key += 0x10000u;
+  return key;
 }
 
 template <typename T>
@@ -236,8 +249,23 @@ __global__ void __launch_bounds__(kTkThreads) topk_fwd_kernel(const T* __restric
   float m_s = -INFINITY, S_s = 0.f, m_t = -INFINITY, S_t = 0.f;
   for (int i = tid; i < nvec; i += kTkThreads) {
     float xs[VEC], xt[VEC];
-    Io::unpack(tk_ldg_v4(vs + i), xs);
+    const uint4 ws = tk_ldg_v4(vs + i);
+    Io::unpack(ws, xs);
     Io::unpack(tk_ldg_v4(vt + i), xt);
+    if (mode == 2) {
+      if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+        const uint32_t wz[4] = {ws.x, ws.y, ws.z, ws.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint32_t kp = bf16_pair_keys(wz[q]);
+          atomicAdd(&hist[(kp >> (kTopShift - 16)) & (kTopBins - 1)], 1);
+          atomicAdd(&hist[kp >> kTopShift], 1);
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < VEC; ++j) atomicAdd(&hist[(Io::KMASK & fkey_raw(xs[j])) >> kTopShift], 1);
+      }
+    }
     float cs = xs[0], ct = xt[0];
 #pragma unroll
     for (int j = 1; j < VEC; ++j) {
@@ -257,7 +285,6 @@ __global__ void __launch_bounds__(kTkThreads) topk_fwd_kernel(const T* __restric
     for (int j = 0; j < VEC; ++j) {
       S_s += ex2(fmaf(xs[j], kLog2e, -ms2));
       S_t += ex2(fmaf(xt[j], kLog2e, -mt2));
-      if (mode == 2) atomicAdd(&hist[(Io::KMASK & fkey_raw(xs[j])) >> kTopShift], 1);
     }
   }
   for (int v = nvec * VEC + tid; v < V; v += kTkThreads) {
@@ -336,10 +363,27 @@ __global__ void __launch_bounds__(kTkThreads) topk_fwd_kernel(const T* __restric
     const int need = s_need;
     for (int i = tid; i < nvec; i += kTkThreads) {
       float xs[VEC];
-      Io::unpack(tk_ldg_v4(vs + i), xs);
+      const uint4 ws = tk_ldg_v4(vs + i);
+      Io::unpack(ws, xs);
+      uint32_t keys[VEC];
+      if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+        const uint32_t wz[4] = {ws.x, ws.y, ws.z, ws.w};
+        bool any = false;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint32_t kp = bf16_pair_keys(wz[q]);
+          keys[2 * q] = kp << 16;
+          keys[2 * q + 1] = kp & 0xFFFF0000u;
+          any |= ((kp >> (kTopShift - 16)) & (kTopBins - 1)) >= bin || (kp >> kTopShift) >= bin;
+        }
+        if (!any) continue;  // no key of these 8 reaches the bin (the common case)
+      } else {
+#pragma unroll
+        for (int j = 0; j < VEC; ++j) keys[j] = Io::KMASK & fkey_raw(xs[j]);
+      }
 #pragma unroll
       for (int j = 0; j < VEC; ++j) {
-        const uint32_t key = Io::KMASK & fkey_raw(xs[j]);
+        const uint32_t key = keys[j];
         const uint32_t kb = key >> kTopShift;
         if (kb > bin) {
           add_member<T>(xs[j], zt, i * VEC + j, lse_s, lse_t, L_S, P_S);
