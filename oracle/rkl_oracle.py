@@ -28,7 +28,7 @@ What it computes, and where the pages define it:
   scattered back to the [B, S-1] layout; an empty mask still yields a
   well-defined zero gradient.
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings where the pages are silent (the project's design notes list each):
 
 * Only the student gets gradients (the teacher LM head is held as an ordinary
   tensor outside the trained parameters);

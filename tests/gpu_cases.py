@@ -8,7 +8,7 @@ from full_vocabulary_reverse_b200 import binding as rb
 from full_vocabulary_reverse_b200.workloads import make_inputs
 from oracle import rkl_oracle as O
 
-# Tolerances (stated by the benchmark spec for bf16 inputs with fp32 accumulation):
+# Tolerances for bf16 inputs with fp32 accumulation:
 #   per-token loss |dL| <= 1e-4 + 1e-3 |L|; gradients max-norm relative 2e-2.
 TOK_ATOL, TOK_RTOL, GRAD_RTOL = 1e-4, 1e-3, 2e-2
 
