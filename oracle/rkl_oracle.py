@@ -472,3 +472,43 @@ def backward_topk_pair(z_s, z_t, targets, k, mask, reduction, grad_loss=1.0, gra
         rows = row_idx[c0:c0 + _ROW_CHUNK]
         _, dz[rows] = topk_rows(z_s[rows], z_t[rows], yflat[rows], k, g[c0:c0 + len(rows)])
     return dz
+
+
+def forward_topk_hidden(h_s, W_s, h_t, W_t, targets, k, mask, reduction):
+    """Top-k estimate on the hidden-state payload: the estimator of
+    forward_topk_pair with z_s = h_s W_s^T and z_t = h_t W_t^T."""
+    mask = np.asarray(mask)
+    B, Sm1 = mask.shape
+    row_idx, N = compact_rows(mask)
+    W_s64, W_t64 = _f64(W_s), _f64(W_t)
+    yflat = np.asarray(targets).reshape(-1)
+    L = np.zeros(N)
+    for c0 in range(0, N, _ROW_CHUNK):
+        rows = row_idx[c0:c0 + _ROW_CHUNK]
+        z_s, z_t = _student_teacher_logits(rows, h_s, W_s64, h_t, W_t64)
+        L[c0:c0 + len(rows)], _ = topk_rows(z_s, z_t, yflat[rows], k)
+    loss_tok = np.zeros(B * Sm1)
+    loss_tok[row_idx] = L
+    loss = reduce_loss(L, row_idx, B, Sm1, reduction)
+    return {"loss_tok": loss_tok.reshape(B, Sm1), "loss": loss, "L": L, "row_idx": row_idx, "N": N}
+
+
+def backward_topk_hidden(h_s, W_s, h_t, W_t, targets, k, mask, reduction, grad_loss=1.0, grad_tok=None):
+    """(dH_s [T, H], dW_s [V, H]) of the top-k estimate: its z_s-gradient
+    (topk_rows) through z_s = h_s W_s^T."""
+    mask = np.asarray(mask)
+    B, Sm1 = mask.shape
+    row_idx, N = compact_rows(mask)
+    W_s64, W_t64 = _f64(W_s), _f64(W_t)
+    g = row_weights(row_idx, B, Sm1, reduction, grad_loss, grad_tok)
+    yflat = np.asarray(targets).reshape(-1)
+    T, H = np.asarray(h_s).shape
+    dH = np.zeros((T, H))
+    dW = np.zeros(W_s64.shape)
+    for c0 in range(0, N, _ROW_CHUNK):
+        rows = row_idx[c0:c0 + _ROW_CHUNK]
+        z_s, z_t = _student_teacher_logits(rows, h_s, W_s64, h_t, W_t64)
+        _, dz = topk_rows(z_s, z_t, yflat[rows], k, g[c0:c0 + len(rows)])
+        dH[rows] = dz @ W_s64
+        dW += dz.T @ _f64(h_s[rows])
+    return dH, dW

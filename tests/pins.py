@@ -471,3 +471,51 @@ def topk_finite_differences(O, rs):
         zm = z_s.copy(); zm[0, j] -= eps
         num[j] = (O.topk_rows(zp, z_t, y, k)[0][0] - O.topk_rows(zm, z_t, y, k)[0][0]) / (2 * eps)
     return float(np.max(np.abs(dz[0] - num)) / np.max(np.abs(num)))
+
+
+def topk_hidden_chain_rule(O, rs):
+    """The hidden-payload top-k estimate equals the logits-pair one on
+    z = h W^T, and its gradients are dz W_s and dz^T h_s (chain rule)."""
+    h_s, W_s, h_t, W_t, mask = rand_problem(rs, B=2, Sm1=4, H=3, V=11)
+    y = rs.randint(0, 11, size=mask.shape)
+    z_s, z_t = h_s @ W_s.T, h_t @ W_t.T
+    worst = 0.0
+    for k in (0, 3, 11):
+        a = O.forward_topk_hidden(h_s, W_s, h_t, W_t, y, k, mask, 2)
+        b = O.forward_topk_pair(z_s, z_t, y, k, mask, 2)
+        dH, dW = O.backward_topk_hidden(h_s, W_s, h_t, W_t, y, k, mask, 2)
+        dz = O.backward_topk_pair(z_s, z_t, y, k, mask, 2)
+        worst = max(worst, float(np.max(np.abs(a["loss_tok"] - b["loss_tok"]))), abs(a["loss"] - b["loss"]),
+                    float(np.max(np.abs(dH - dz @ W_s))), float(np.max(np.abs(dW - dz.T @ h_s))))
+    return worst
+
+
+def topk_hidden_finite_differences(O, rs):
+    """Central differences of the top-k objective w.r.t. h_s and W_s when the
+    sampled tokens lie in the support (no score-function term) and the
+    support does not move under the perturbation."""
+    B, Sm1, H, V, k = 1, 3, 3, 9, 4
+    h_s = rs.normal(size=(3, H))
+    W_s = rs.normal(size=(V, H)) * 2
+    h_t = rs.normal(size=(3, H))
+    W_t = rs.normal(size=(V, H))
+    mask = np.ones((B, Sm1), np.uint8)
+    S = O.topk_support(h_s @ W_s.T, k)
+    y = np.array([[int(np.flatnonzero(S[i])[0]) for i in range(3)]])
+    f = lambda hs, ws: O.forward_topk_hidden(hs, ws, h_t, W_t, y, k, mask, 1)["loss"]  # noqa: E731
+    dH, dW = O.backward_topk_hidden(h_s, W_s, h_t, W_t, y, k, mask, 1)
+    eps = 1e-6
+    num_H = np.zeros_like(h_s)
+    for i in range(h_s.shape[0]):
+        for j in range(H):
+            hp = h_s.copy(); hp[i, j] += eps
+            hm = h_s.copy(); hm[i, j] -= eps
+            num_H[i, j] = (f(hp, W_s) - f(hm, W_s)) / (2 * eps)
+    num_W = np.zeros_like(W_s)
+    for i in range(V):
+        for j in range(H):
+            wp = W_s.copy(); wp[i, j] += eps
+            wm = W_s.copy(); wm[i, j] -= eps
+            num_W[i, j] = (f(h_s, wp) - f(h_s, wm)) / (2 * eps)
+    return max(float(np.max(np.abs(dH - num_H))) / float(np.max(np.abs(num_H))),
+               float(np.max(np.abs(dW - num_W))) / float(np.max(np.abs(num_W))))

@@ -370,3 +370,11 @@ def test_topk_pins_catch_planted_mistakes(old, new, kind):
         "limits": lambda: pins.topk_limits(M, rs) > 1e-6,
     }[kind]()
     assert caught
+
+
+def test_topk_hidden_chain_rule(rs):
+    assert pins.topk_hidden_chain_rule(O, rs) < 1e-12
+
+
+def test_topk_hidden_finite_differences(rs):
+    assert pins.topk_hidden_finite_differences(O, rs) < 1e-6
