@@ -11,6 +11,7 @@ from .binding import (  # noqa: F401
     forward_logits_pair, backward_logits_pair, forward_with_stats,
     workspace_size, device_error, reverse_kl_hidden, reverse_kl_logits, reverse_kl_logits_pair,
     forward_topk_pair, backward_topk_pair, topk_estimator_logits_pair,
+    forward_topk_hidden, backward_topk_hidden, topk_estimator_hidden,
     compact_rows_multi, forward_hidden_multi, backward_hidden_multi, workspace_size_multi, reverse_kl_hidden_multi,
     REDUCE_NONE, REDUCE_TOKEN_MEAN, REDUCE_SEQ_MEAN_NESTED,
     PAYLOAD_HIDDEN, PAYLOAD_LOGITS, PAYLOAD_LOGITS_PAIR,

@@ -44,7 +44,7 @@ static const char* const kKernelNames[K_COUNT] = {
     "compact_rows", "gather_rows",   "fwd_dual_tc",  "fwd_single_tc", "teacher_lse", "combine_splits",
     "scatter_loss", "reduce_loss",   "row_weights",  "dz_dual_tc",    "dz_single_tc", "grad_dw_dh_tc",
     "scatter_dh",   "fwd_simt_fp32", "dz_simt_fp32", "grad_simt_fp32", "pair_fwd",   "pair_bwd",
-    "count_teachers", "build_slots", "topk_fwd", "topk_bwd"};
+    "count_teachers", "build_slots", "topk_fwd", "topk_bwd", "zw_dual_tc", "dz_topk_tc", "topk_rowk"};
 
 const char* kernel_name(int id) { return (id >= 0 && id < K_COUNT) ? kKernelNames[id] : nullptr; }
 
@@ -153,8 +153,12 @@ constexpr int kSimtSplits = 37;
 struct Plan {
   int n_pad = 0, es = 2, S = 1, VT = 1, Vc = 0, nchunks = 1;
   size_t off_hcs = 0, off_hct = 0, off_part = 0, off_rowc = 0, off_lse = 0, off_dz = 0, off_dh = 0, off_cnt = 0,
-         off_slot = 0, off_kslot = 0, total = 0;
+         off_slot = 0, off_kslot = 0, off_rowk = 0, off_z = 0, total = 0;
+  int zrows = 0;      // top-k, hidden payload: rows of a logit block
+  long long zpitch = 0;  // its row pitch (floats)
 };
+
+constexpr int kTopkBlockRows = 512;  // top-k, hidden payload: rows whose logits are written at a time
 
 static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -193,7 +197,8 @@ static Plan make_plan(rkl_payload payload, rkl_dtype dtype, int64_t n_max, int64
   p.off_hcs = off;
   off = align256(off + size_t(p.n_pad) * H * p.es);
   p.off_hct = off;
-  if (payload == RKL_PAYLOAD_HIDDEN) off = align256(off + size_t(p.n_pad) * H * p.es);
+  if (payload == RKL_PAYLOAD_HIDDEN || payload == RKL_PAYLOAD_TOPK_HIDDEN)
+    off = align256(off + size_t(p.n_pad) * H * p.es);
   p.off_part = off;
   off = align256(off + size_t(p.S) * kStatVals * p.n_pad * sizeof(float));
   p.off_rowc = off;
@@ -211,6 +216,16 @@ static Plan make_plan(rkl_payload payload, rkl_dtype dtype, int64_t n_max, int64
     off = align256(off + size_t(p.n_pad) * sizeof(int32_t));
     p.off_kslot = off;
     off = align256(off + size_t(n) * sizeof(int32_t));
+  }
+  if (payload == RKL_PAYLOAD_TOPK_HIDDEN) {
+    // per-row constants of the top-k dz pass, and z_s, z_t (fp32) of one
+    // block of rows: never more than kTopkBlockRows rows of logits at a time
+    p.off_rowk = off;
+    off = align256(off + size_t(6) * p.n_pad * sizeof(float));
+    p.zrows = p.n_pad < kTopkBlockRows ? p.n_pad : kTopkBlockRows;
+    p.zpitch = ((V + 3) / 4) * 4;
+    p.off_z = off;
+    off = align256(off + size_t(2) * p.zrows * p.zpitch * sizeof(float));
   }
   p.total = off;
   return p;
@@ -262,7 +277,8 @@ static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 static rkl_status check_common(rkl_payload payload, rkl_dtype dtype, int64_t B, int64_t Sm1, int64_t H, int64_t V,
                                int32_t N, int reduction) {
   if (dtype != RKL_BF16 && dtype != RKL_FP32) return fail(RKL_ERR_DTYPE, "unknown dtype %d", (int)dtype);
-  if (payload != RKL_PAYLOAD_HIDDEN && payload != RKL_PAYLOAD_LOGITS && payload != RKL_PAYLOAD_LOGITS_PAIR)
+  if (payload != RKL_PAYLOAD_HIDDEN && payload != RKL_PAYLOAD_LOGITS && payload != RKL_PAYLOAD_LOGITS_PAIR &&
+      payload != RKL_PAYLOAD_TOPK_HIDDEN)
     return fail(RKL_ERR_DTYPE, "unknown payload %d", (int)payload);
   if (payload == RKL_PAYLOAD_LOGITS_PAIR) H = 64;  // no hidden dimension in this mode
   if (reduction < 0 || reduction > 2) return fail(RKL_ERR_DTYPE, "unknown reduction %d", reduction);
@@ -444,12 +460,16 @@ static rkl_status backward_impl(rkl_payload payload, const void* h_s, const void
                                 const int32_t* row_idx, int32_t N, rkl_reduction reduction, const float* saved,
                                 const float* grad_loss, const float* grad_tok, float* dH_s, float* dW_s,
                                 void* workspace, size_t workspace_bytes, void* stream_,
-                                const MultiTeacher* mt = nullptr) {
+                                const MultiTeacher* mt = nullptr, const int32_t* topk_targets = nullptr) {
   RKL_TRY(check_common(payload, dtype, B, Sm1, H, V, N, reduction));
   RKL_TRY(check_ptr(h_s, "h_s"));
-  RKL_TRY(check_ptr(teacher, payload == RKL_PAYLOAD_HIDDEN ? "h_t" : "teacher_logits"));
+  RKL_TRY(check_ptr(teacher, payload != RKL_PAYLOAD_LOGITS ? "h_t" : "teacher_logits"));
   RKL_TRY(check_ptr(W_s, "W_s"));
-  if (payload == RKL_PAYLOAD_HIDDEN) RKL_TRY(check_ptr(W_t, "W_t"));
+  if (payload != RKL_PAYLOAD_LOGITS) RKL_TRY(check_ptr(W_t, "W_t"));
+  const bool topk = payload == RKL_PAYLOAD_TOPK_HIDDEN;
+  if (topk && dtype != RKL_BF16)
+    return fail(RKL_ERR_UNSUPPORTED, "the top-k estimator on the hidden payload needs bf16 inputs");
+  if (topk) RKL_TRY(check_ptr(topk_targets, "targets"));
   RKL_TRY(check_ptr(row_idx, "row_idx"));
   RKL_TRY(check_ptr(saved, "saved", N > 0));
   RKL_TRY(check_ptr(grad_loss, "grad_loss", false));
@@ -465,7 +485,7 @@ static rkl_status backward_impl(rkl_payload payload, const void* h_s, const void
   cudaStream_t s = static_cast<cudaStream_t>(stream_);
   const long long T = B * Sm1;
   const bool bf16 = dtype == RKL_BF16;
-  const bool hidden = payload == RKL_PAYLOAD_HIDDEN;
+  const bool hidden = payload != RKL_PAYLOAD_LOGITS;
   float* dHc = reinterpret_cast<float*>(ws_at(workspace, pl.off_dh));
 
   if (N == 0) {
@@ -495,6 +515,11 @@ static rkl_status backward_impl(rkl_payload payload, const void* h_s, const void
   float* rowc = reinterpret_cast<float*>(ws_at(workspace, pl.off_rowc));
   RKL_CUDA(launch_row_weights(saved, row_idx, N, pl.n_pad, static_cast<int>(B), static_cast<int>(Sm1), reduction,
                               grad_loss, grad_tok, rowc, slot_k, s));
+  float* rowk = nullptr;
+  if (topk) {
+    rowk = reinterpret_cast<float*>(ws_at(workspace, pl.off_rowk));
+    RKL_CUDA(launch_topk_rowk(saved, saved + 3 * size_t(N), row_idx, topk_targets, N, pl.n_pad, rowk, s));
+  }
   void* dz = ws_at(workspace, pl.off_dz);
   const int ng = hidden ? 2 : 1;
   const int nchunks = static_cast<int>((V + pl.Vc - 1) / pl.Vc);
@@ -517,6 +542,7 @@ static rkl_status backward_impl(rkl_payload payload, const void* h_s, const void
       a.teacher_pitch = V;
     }
     a.rowc = rowc;
+    a.rowk = rowk;
     a.N = n_rows;
     a.n_pad = pl.n_pad;
     a.H = static_cast<int>(H);
@@ -551,7 +577,11 @@ static rkl_status backward_impl(rkl_payload payload, const void* h_s, const void
       a.GT = 1;
       a.G = a.IT;
       a.units_total = MT * a.IT;
-      RKL_CUDA(launch_fused(ng, true, a, 2 * a.units_total < sms ? 2 * a.units_total : sms, s));
+      const int fgrid = 2 * a.units_total < sms ? 2 * a.units_total : sms;
+      if (topk)
+        RKL_CUDA(launch_fused_topk(2, a, fgrid, s));
+      else
+        RKL_CUDA(launch_fused(ng, true, a, fgrid, s));
       // S7: dW_s[chunk] = dz^T hc_s and dHc (+)= dz W_s[chunk].
       RKL_TRY(make_map(&g.tm_dz_k, dz, false, cw, n_rows, size_t(pl.Vc) * 2, 64, 128));
       RKL_TRY(make_map(&g.tm_dz_mn, dz, false, cw, n_rows, size_t(pl.Vc) * 2, 64, 64));
@@ -726,7 +756,7 @@ rkl_status rkl_forward_topk_pair(const void* student_logits, const void* teacher
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const long long T = B * Sm1;
   RKL_CUDA(launch_topk_fwd(student_logits, teacher_logits, dtype == RKL_BF16, row_idx, targets, N,
-                           static_cast<int>(V), k, saved, saved + 3 * size_t(N), s));
+                           static_cast<int>(V), k, saved, saved + 3 * size_t(N), V, false, s));
   if (loss_tok) RKL_CUDA(launch_scatter_loss(saved, row_idx, N, T, loss_tok, s));
   if (loss && reduction != RKL_REDUCE_NONE)
     RKL_CUDA(launch_reduce(saved, row_idx, N, static_cast<int>(B), static_cast<int>(Sm1), reduction, loss, s));
@@ -757,6 +787,91 @@ rkl_status rkl_backward_topk_pair(const void* student_logits, const void* teache
   RKL_CUDA(launch_topk_bwd(student_logits, teacher_logits, dtype == RKL_BF16, row_idx, targets, N, n_pad, T,
                            static_cast<int>(V), saved, N > 0 ? saved + 3 * size_t(N) : nullptr, rowc, dz, s));
   return RKL_OK;
+}
+
+// Top-k estimator on the hidden payload.  Forward: per block of up to
+// kTopkBlockRows compacted rows, the tcgen05 kernel writes z_s and z_t (fp32)
+// of the block, and the selection / estimate kernel of the logits-pair form
+// runs on those rows.  Backward: the recompute + dz kernel with the top-k
+// formula (membership from the same fp32 logits, bit for bit), then the
+// gradient GEMMs of the exact path.
+rkl_status rkl_forward_topk_hidden(const void* h_s, const void* h_t, const void* W_s, const void* W_t,
+                                   rkl_dtype dtype, int64_t B, int64_t Sm1, int64_t H, int64_t V,
+                                   const int32_t* row_idx, int32_t N, int64_t k, const int32_t* targets,
+                                   rkl_reduction reduction, float* loss_tok, float* loss, float* saved,
+                                   void* workspace, size_t workspace_bytes, void* stream) {
+  RKL_TRY(check_common(RKL_PAYLOAD_TOPK_HIDDEN, dtype, B, Sm1, H, V, N, reduction));
+  if (dtype != RKL_BF16)
+    return fail(RKL_ERR_UNSUPPORTED, "the top-k estimator on the hidden payload needs bf16 inputs");
+  if (k < 0) return fail(RKL_ERR_SHAPE, "k = %lld is negative", (long long)k);
+  RKL_TRY(check_ptr(h_s, "h_s"));
+  RKL_TRY(check_ptr(h_t, "h_t"));
+  RKL_TRY(check_ptr(W_s, "W_s"));
+  RKL_TRY(check_ptr(W_t, "W_t"));
+  RKL_TRY(check_ptr(row_idx, "row_idx"));
+  RKL_TRY(check_ptr(targets, "targets"));
+  RKL_TRY(check_ptr(loss_tok, "loss_tok", false));
+  RKL_TRY(check_ptr(loss, "loss", false));
+  RKL_TRY(check_ptr(saved, "saved", N > 0));
+  RKL_TRY(check_ptr(workspace, "workspace"));
+  const Plan pl = make_plan(RKL_PAYLOAD_TOPK_HIDDEN, dtype, N, H, V);
+  if (workspace_bytes < pl.total)
+    return fail(RKL_ERR_WORKSPACE, "workspace is %zu bytes, %zu needed", workspace_bytes, pl.total);
+  int sms = 0;
+  RKL_TRY(device_setup(&sms));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const long long T = B * Sm1;
+  if (N > 0) {
+    const uint8_t* as = static_cast<const uint8_t*>(h_s);
+    const uint8_t* at = static_cast<const uint8_t*>(h_t);
+    if (N < T) {
+      as = ws_at(workspace, pl.off_hcs);
+      at = ws_at(workspace, pl.off_hct);
+      RKL_CUDA(launch_gather(h_s, h_t, const_cast<uint8_t*>(as), const_cast<uint8_t*>(at), row_idx, nullptr, N,
+                             static_cast<int>(H * 2), s));
+    }
+    float* zs = reinterpret_cast<float*>(ws_at(workspace, pl.off_z));
+    float* zt = zs + size_t(pl.zrows) * pl.zpitch;
+    for (int r0 = 0; r0 < N; r0 += pl.zrows) {
+      const int nb = (N - r0) < pl.zrows ? (N - r0) : pl.zrows;
+      FusedArgs a;
+      memset(&a, 0, sizeof(a));
+      RKL_TRY(make_map(&a.tm_as, as + size_t(r0) * H * 2, false, H, nb, H * 2, kBK, kBM));
+      RKL_TRY(make_map(&a.tm_at, at + size_t(r0) * H * 2, false, H, nb, H * 2, kBK, kBM));
+      RKL_TRY(make_map(&a.tm_bs, W_s, false, H, V, H * 2, kBK, kFBN / 2));
+      RKL_TRY(make_map(&a.tm_bt, W_t, false, H, V, H * 2, kBK, kFBN / 2));
+      RKL_TRY(make_map(&a.tm_zs, zs, true, V, nb, size_t(pl.zpitch) * 4, 32, 32));
+      RKL_TRY(make_map(&a.tm_zt, zt, true, V, nb, size_t(pl.zpitch) * 4, 32, 32));
+      a.N = nb;
+      a.n_pad = pl.n_pad;
+      a.H = static_cast<int>(H);
+      a.V = static_cast<int>(V);
+      a.KB = static_cast<int>(H / kBK);
+      a.IT = pl.VT;
+      a.vt_base = 0;
+      a.GT = 1;
+      a.G = pl.VT;
+      a.MT = (nb + 2 * kBM - 1) / (2 * kBM);
+      a.units_total = a.MT * a.G;
+      RKL_CUDA(launch_fused_topk(1, a, 2 * a.units_total < sms ? 2 * a.units_total : sms, s));
+      RKL_CUDA(launch_topk_fwd(zs, zt, false, row_idx + r0, targets, nb, static_cast<int>(V), k, saved + 3 * size_t(r0),
+                               saved + 3 * size_t(N) + 4 * size_t(r0), pl.zpitch, true, s));
+    }
+  }
+  if (loss_tok) RKL_CUDA(launch_scatter_loss(saved, row_idx, N, T, loss_tok, s));
+  if (loss && reduction != RKL_REDUCE_NONE)
+    RKL_CUDA(launch_reduce(saved, row_idx, N, static_cast<int>(B), static_cast<int>(Sm1), reduction, loss, s));
+  return RKL_OK;
+}
+
+rkl_status rkl_backward_topk_hidden(const void* h_s, const void* h_t, const void* W_s, const void* W_t,
+                                    rkl_dtype dtype, int64_t B, int64_t Sm1, int64_t H, int64_t V,
+                                    const int32_t* row_idx, int32_t N, const int32_t* targets,
+                                    rkl_reduction reduction, const float* saved, const float* grad_loss,
+                                    const float* grad_tok, float* dH_s, float* dW_s, void* workspace,
+                                    size_t workspace_bytes, void* stream) {
+  return backward_impl(RKL_PAYLOAD_TOPK_HIDDEN, h_s, h_t, W_s, W_t, dtype, B, Sm1, H, V, row_idx, N, reduction,
+                       saved, grad_loss, grad_tok, dH_s, dW_s, workspace, workspace_bytes, stream, nullptr, targets);
 }
 
 rkl_status rkl_compact_rows(const uint8_t* mask, int64_t B, int64_t Sm1, int32_t* row_idx, int32_t* n_dev,

@@ -33,6 +33,9 @@ enum KernelId : int {
   K_BUILD_SLOTS,      // per-row teachers: teacher-grouped row slots
   K_TOPK_FWD,         // top-k estimator, both sides as logits: selection + estimate
   K_TOPK_BWD,         // top-k estimator: gradient estimate rows
+  K_ZW_DUAL_TC,       // top-k, hidden payload: z_s and z_t of a row block written by tcgen05
+  K_DZ_TOPK_TC,       // top-k, hidden payload: recompute + top-k dz chunk
+  K_TOPK_ROWK,        // top-k, hidden payload: per-row constants of the dz pass
   K_COUNT
 };
 
@@ -81,6 +84,12 @@ struct FusedArgs {
   // 256-row pair tiles).  tgroups <= 1: one teacher head.
   int tgroups;
   int group_row_end[kMaxTeachers];
+  // Top-k estimator on the hidden payload.  Logit writer: z_s, z_t fp32
+  // [rows, V] outputs (box {32, 32}).  Top-k dz: per-row constants
+  // rowk [6][n_pad] = (lse_t - lse_s, C, a, bits of K*, bits of v_last,
+  // bits of the sampled token id).
+  CUtensorMap tm_zs, tm_zt;
+  const float* rowk;
 };
 
 struct GradArgs {
@@ -100,6 +109,9 @@ size_t fused_smem_bytes(int ng, bool dz);
 size_t grad_smem_bytes();
 cudaError_t tc_setup(int device);  // one-time cudaFuncSetAttribute per device
 cudaError_t launch_fused(int ng, bool dz, const FusedArgs& a, int grid, cudaStream_t s);  // grid: CTAs, even
+// Hidden-payload top-k: write z_s and z_t (fp32) of the rows of a (variant 1),
+// or the top-k dz chunk (variant 2); both on the NG = 2 dz configuration.
+cudaError_t launch_fused_topk(int variant, const FusedArgs& a, int grid, cudaStream_t s);
 cudaError_t launch_grad(const GradArgs& a, int grid, cudaStream_t s);
 cudaError_t read_and_clear_device_error(int* code);
 
@@ -147,9 +159,13 @@ cudaError_t launch_pair_bwd(const void* zs, const void* zt, bool bf16, const int
 
 // Top-k estimator with both sides as logits (topk_kernels.cu).  saved [N, 3]
 // (lse_s, lse_t, estimate), saved_tk [N, 4] (C, a, K* bits, v_last bits).
+// Logit rows: zs + row * zpitch with row = row_idx[k] (local = false) or the
+// block-local k (local = true); the sampled token is targets[row_idx[k]].
 cudaError_t launch_topk_fwd(const void* zs, const void* zt, bool bf16, const int32_t* row_idx,
                             const int32_t* targets, int N, int V, long long k, float* saved, float* saved_tk,
-                            cudaStream_t s);
+                            long long zpitch, bool local, cudaStream_t s);
+cudaError_t launch_topk_rowk(const float* saved, const float* saved_tk, const int32_t* row_idx,
+                             const int32_t* targets, int N, int n_pad, float* rowk, cudaStream_t s);
 cudaError_t launch_topk_bwd(const void* zs, const void* zt, bool bf16, const int32_t* row_idx,
                             const int32_t* targets, int N, int n_pad, long long T, int V, const float* saved,
                             const float* saved_tk, const float* rowc, void* dz, cudaStream_t s);

@@ -190,7 +190,11 @@ __device__ __forceinline__ void prefetch_l2(const void* p) {
 // accumulator-empty barriers; both CTAs run the same producer and epilogue
 // code on their own rows.
 // ============================================================================
-template <int NG, bool DZ>
+// VAR (with NG = 2, DZ = true) selects the epilogue of the hidden-payload
+// top-k estimator: 1 writes the z_s and z_t tiles (fp32), 2 writes the top-k
+// dz  g (p_s ([v in S](w + 1) - C) + [v = y] a),  S = {key(z_s) > K*, or
+// key(z_s) = K* and v <= v_last} with the order-preserving float key.
+template <int NG, bool DZ, int VAR = 0>
 __global__ void __launch_bounds__(kFusedThreads, 1) fused_kernel(const __grid_constant__ FusedArgs p) {
   using Cfg = FusedCfg<NG>;
   constexpr int STAGES = Cfg::STAGES;
@@ -374,6 +378,9 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_kernel(const __grid_co
     const uint32_t acc_empty0 = mapa_shared(smem_u32(acc_empty), 0);
     int cur_m0 = -1;
     float lse2 = 0.f, cst = 0.f, g_row = 0.f;
+    float tk_C = 0.f, tk_ga = 0.f;     // top-k dz: C and g a
+    uint32_t tk_kstar = 0u;
+    int tk_vlast = -1, tk_y = -1;
     int tgt = -1;  // target column of this row (forward with targets), else -1
     const uint16_t* trow = nullptr;
     int box = 0;
@@ -386,11 +393,20 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_kernel(const __grid_co
       if (m0 != cur_m0) {
         cur_m0 = m0;
         const int r = m0 + row;
-        if (DZ) {
+        if (DZ && VAR == 2) {
+          lse2 = p.rowc[r];
+          g_row = p.rowc[2 * p.n_pad + r];
+          cst = p.rowk[r];
+          tk_C = p.rowk[p.n_pad + r];
+          tk_ga = g_row * p.rowk[2 * p.n_pad + r];
+          tk_kstar = __float_as_uint(p.rowk[3 * p.n_pad + r]);
+          tk_vlast = __float_as_int(p.rowk[4 * p.n_pad + r]);
+          tk_y = __float_as_int(p.rowk[5 * p.n_pad + r]);
+        } else if (DZ && VAR == 0) {
           lse2 = p.rowc[r];
           cst = p.rowc[p.n_pad + r];
           g_row = p.rowc[2 * p.n_pad + r];
-        } else {
+        } else if (!DZ) {
           tgt = (p.targets != nullptr && r < p.N) ? p.targets[p.row_idx[r]] : -1;
         }
         if (NG == 1) {
@@ -465,17 +481,60 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_kernel(const __grid_co
             else if (nv > 0)
               stats_chunk_tail(st, zs, zt, nv);
             if (tgt >= 0) pick_target(zs, tgt, v0 + c * 32, p.tlogit + m0 + row);
+          } else if (VAR == 1) {
+            // z_s and z_t of this 32-column chunk, fp32, one 32 x 32 box each
+            // (columns past V are clipped by the TMA store)
+            uint8_t* buf = stg + (warp - 2) * kStgBoxBytes;  // one staging box per warp
+#pragma unroll
+            for (int which = 0; which < 2; ++which) {
+              const float* src = which == 0 ? zs : zt;
+              if (lane == 0) bulk_wait_read<0>();
+              __syncwarp();
+              const uint32_t rbase = smem_u32(buf) + lane * 128;
+#pragma unroll
+              for (int e = 0; e < 8; ++e)
+                st_shared_v4(rbase + ((e ^ (lane & 7)) << 4), __float_as_uint(src[4 * e]),
+                             __float_as_uint(src[4 * e + 1]), __float_as_uint(src[4 * e + 2]),
+                             __float_as_uint(src[4 * e + 3]));
+              fence_proxy_async_smem();
+              __syncwarp();
+              if (lane == 0) {
+                tma_store_2d(which == 0 ? &p.tm_zs : &p.tm_zt, buf, v0 + c * 32, m0 + q * 32);
+                bulk_commit();
+              }
+            }
           } else {
             // dz = g * p_s * ((z_s - z_t) + cst); columns past the chunk end
             // are clipped by the TMA store.
             uint32_t pk[16];
+            if (VAR == 2) {
+              // top-k: dz = g p_s ([v in S](w + 1) - C) + [v = y] g a
+              const int col0 = v0 + c * 32;
 #pragma unroll
-            for (int j = 0; j < 32; j += 2) {
-              const float p0 = ex2(fmaf(zs[j], kLog2e, -lse2));
-              const float p1 = ex2(fmaf(zs[j + 1], kLog2e, -lse2));
-              const float d0 = g_row * p0 * ((zs[j] - zt[j]) + cst);
-              const float d1 = g_row * p1 * ((zs[j + 1] - zt[j + 1]) + cst);
-              pk[j / 2] = pack_bf16x2(d0, d1);
+              for (int j = 0; j < 32; j += 2) {
+                float d[2];
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                  const float x = zs[j + h];
+                  const uint32_t u = x == 0.f ? 0u : __float_as_uint(x);
+                  const uint32_t key = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+                  const int v = col0 + j + h;
+                  const bool in = key > tk_kstar || (key == tk_kstar && v <= tk_vlast);
+                  const float pr = ex2(fmaf(x, kLog2e, -lse2));
+                  const float coef = (in ? (x - zt[j + h]) + cst + 1.f : 0.f) - tk_C;
+                  d[h] = g_row * pr * coef + (v == tk_y ? tk_ga : 0.f);
+                }
+                pk[j / 2] = pack_bf16x2(d[0], d[1]);
+              }
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; j += 2) {
+                const float p0 = ex2(fmaf(zs[j], kLog2e, -lse2));
+                const float p1 = ex2(fmaf(zs[j + 1], kLog2e, -lse2));
+                const float d0 = g_row * p0 * ((zs[j] - zt[j]) + cst);
+                const float d1 = g_row * p1 * ((zs[j + 1] - zt[j + 1]) + cst);
+                pk[j / 2] = pack_bf16x2(d0, d1);
+              }
             }
             uint8_t* buf = stg + (warp - 2) * kStgBoxBytes;  // one staging box per warp
             if ((c & 1) == 0) {
@@ -866,6 +925,12 @@ cudaError_t tc_setup(int /*device*/) {
   if ((e = cudaFuncSetAttribute(fused_kernel<1, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)fused_smem<1, true>())) != cudaSuccess)
     return e;
+  if ((e = cudaFuncSetAttribute(fused_kernel<2, true, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)fused_smem<2, true>())) != cudaSuccess)
+    return e;
+  if ((e = cudaFuncSetAttribute(fused_kernel<2, true, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)fused_smem<2, true>())) != cudaSuccess)
+    return e;
   return cudaFuncSetAttribute(grad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)grad_smem_bytes());
 }
 
@@ -893,6 +958,13 @@ cudaError_t launch_fused(int ng, bool dz, const FusedArgs& a, int grid, cudaStre
   if (ng == 2) return dz ? launch_pair(fused_kernel<2, true>, grid, smem, s, a)
                          : launch_pair(fused_kernel<2, false>, grid, smem, s, a);
   return dz ? launch_pair(fused_kernel<1, true>, grid, smem, s, a) : launch_pair(fused_kernel<1, false>, grid, smem, s, a);
+}
+
+cudaError_t launch_fused_topk(int variant, const FusedArgs& a, int grid, cudaStream_t s) {
+  const size_t smem = fused_smem_bytes(2, true);
+  LaunchScope scope(variant == 1 ? K_ZW_DUAL_TC : K_DZ_TOPK_TC, s);
+  return variant == 1 ? launch_pair(fused_kernel<2, true, 1>, grid, smem, s, a)
+                      : launch_pair(fused_kernel<2, true, 2>, grid, smem, s, a);
 }
 
 cudaError_t launch_grad(const GradArgs& a, int grid, cudaStream_t s) {

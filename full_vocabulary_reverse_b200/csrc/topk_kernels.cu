@@ -211,7 +211,8 @@ __global__ void __launch_bounds__(kTkThreads) topk_fwd_kernel(const T* __restric
                                                               const int32_t* __restrict__ row_idx,
                                                               const int32_t* __restrict__ targets, int N, int V,
                                                               long long k_sel, float* __restrict__ saved,
-                                                              float* __restrict__ saved_tk) {
+                                                              float* __restrict__ saved_tk, long long zpitch,
+                                                              int local) {
   using Io = TkIo<T>;
   constexpr int VEC = Io::VEC;
   // 32 KB: the 4096-bin histogram of pass A, then the candidate list
@@ -227,9 +228,10 @@ __global__ void __launch_bounds__(kTkThreads) topk_fwd_kernel(const T* __restric
   const int kr = blockIdx.x;
   if (kr >= N) return;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const long long r = row_idx[kr];
-  const T* zs = zs_all + r * V;
-  const T* zt = zt_all + r * V;
+  const long long r = row_idx[kr];  // token position (sampled token)
+  const long long zr = local ? kr : r;  // logit row: a block-local row, or the token position
+  const T* zs = zs_all + zr * zpitch;
+  const T* zt = zt_all + zr * zpitch;
   const bool vec_ok = ((reinterpret_cast<uintptr_t>(zs) | reinterpret_cast<uintptr_t>(zt)) & 15) == 0;
   const int nvec = vec_ok ? V / VEC : 0;
   const uint4* vs = reinterpret_cast<const uint4*>(zs);
@@ -596,20 +598,51 @@ __global__ void __launch_bounds__(kTkThreads) topk_bwd_kernel(const T* __restric
   }
 }
 
+// Per-row constants of the hidden-payload top-k dz pass, [6][n_pad]:
+// lse_t - lse_s, C, a, and the bit patterns of K*, v_last and the sampled
+// token id; padding rows get values that select nothing.
+__global__ void __launch_bounds__(256) topk_rowk_kernel(const float* __restrict__ saved,
+                                                        const float* __restrict__ saved_tk,
+                                                        const int32_t* __restrict__ row_idx,
+                                                        const int32_t* __restrict__ targets, int N, int n_pad,
+                                                        float* __restrict__ rowk) {
+  const int p = blockIdx.x * blockDim.x + threadIdx.x;
+  if (p >= n_pad) return;
+  float v[6] = {0.f, 0.f, 0.f, __uint_as_float(0xFFFFFFFFu), __int_as_float(-1), __int_as_float(-1)};
+  if (p < N) {
+    v[0] = saved[3 * p + 1] - saved[3 * p];
+    v[1] = saved_tk[4 * p];
+    v[2] = saved_tk[4 * p + 1];
+    v[3] = saved_tk[4 * p + 2];
+    v[4] = saved_tk[4 * p + 3];
+    v[5] = __int_as_float(targets[row_idx[p]]);
+  }
+#pragma unroll
+  for (int i = 0; i < 6; ++i) rowk[static_cast<size_t>(i) * n_pad + p] = v[i];
+}
+
 }  // namespace
 
 cudaError_t launch_topk_fwd(const void* zs, const void* zt, bool bf16, const int32_t* row_idx,
                             const int32_t* targets, int N, int V, long long k, float* saved, float* saved_tk,
-                            cudaStream_t s) {
+                            long long zpitch, bool local, cudaStream_t s) {
   if (N <= 0) return cudaSuccess;
   LaunchScope scope(K_TOPK_FWD, s);
   if (bf16)
     topk_fwd_kernel<__nv_bfloat16><<<N, kTkThreads, 0, s>>>(static_cast<const __nv_bfloat16*>(zs),
                                                             static_cast<const __nv_bfloat16*>(zt), row_idx, targets,
-                                                            N, V, k, saved, saved_tk);
+                                                            N, V, k, saved, saved_tk, zpitch, local ? 1 : 0);
   else
     topk_fwd_kernel<float><<<N, kTkThreads, 0, s>>>(static_cast<const float*>(zs), static_cast<const float*>(zt),
-                                                    row_idx, targets, N, V, k, saved, saved_tk);
+                                                    row_idx, targets, N, V, k, saved, saved_tk, zpitch,
+                                                    local ? 1 : 0);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_topk_rowk(const float* saved, const float* saved_tk, const int32_t* row_idx,
+                             const int32_t* targets, int N, int n_pad, float* rowk, cudaStream_t s) {
+  LaunchScope scope(K_TOPK_ROWK, s);
+  topk_rowk_kernel<<<(n_pad + 255) / 256, 256, 0, s>>>(saved, saved_tk, row_idx, targets, N, n_pad, rowk);
   return cudaGetLastError();
 }
 

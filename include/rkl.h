@@ -73,11 +73,14 @@ typedef enum rkl_reduction {
 } rkl_reduction;
 
 /* PR #3978, payload bullets: full.teacher_payload = hidden_states | logits.
- * LOGITS_PAIR: the student's logits are given too (rkl_*_logits_pair). */
+ * LOGITS_PAIR: the student's logits are given too (rkl_*_logits_pair).
+ * TOPK_HIDDEN: only for rkl_workspace_size, the workspace of
+ * rkl_forward_topk_hidden / rkl_backward_topk_hidden. */
 typedef enum rkl_payload {
   RKL_PAYLOAD_HIDDEN = 0,
   RKL_PAYLOAD_LOGITS = 1,
-  RKL_PAYLOAD_LOGITS_PAIR = 2
+  RKL_PAYLOAD_LOGITS_PAIR = 2,
+  RKL_PAYLOAD_TOPK_HIDDEN = 3
 } rkl_payload;
 
 /* Library version string (static storage). */
@@ -237,6 +240,33 @@ rkl_status rkl_forward_topk_pair(const void* student_logits, const void* teacher
                                  const int32_t* targets, rkl_reduction reduction,
                                  float* loss_tok, float* loss, float* saved,
                                  void* workspace, size_t workspace_bytes, void* stream);
+
+/* The same estimator on the hidden-state payload (bf16 only; RKL_FP32 gives
+ * RKL_ERR_UNSUPPORTED): z_s = h_s W_s^T and z_t = h_t W_t^T as in
+ * rkl_forward_hidden.  The forward writes the fp32 logits of at most 512
+ * compacted rows at a time into the workspace and selects / estimates on
+ * them; the backward recomputes the logits tile by tile (bitwise the same
+ * fp32 values, so the support is the forward's) and runs the gradient GEMMs
+ * of rkl_backward.  Arguments as rkl_forward_hidden / rkl_backward plus k and
+ * targets as rkl_forward_topk_pair; saved [7 N] as there; workspace:
+ * rkl_workspace_size(RKL_PAYLOAD_TOPK_HIDDEN, ...).  Outputs dH_s [T, H] and
+ * dW_s [V, H] as rkl_backward. */
+rkl_status rkl_forward_topk_hidden(const void* h_s, const void* h_t,
+                                   const void* W_s, const void* W_t, rkl_dtype dtype,
+                                   int64_t B, int64_t Sm1, int64_t H, int64_t V,
+                                   const int32_t* row_idx, int32_t N, int64_t k,
+                                   const int32_t* targets, rkl_reduction reduction,
+                                   float* loss_tok, float* loss, float* saved,
+                                   void* workspace, size_t workspace_bytes, void* stream);
+
+rkl_status rkl_backward_topk_hidden(const void* h_s, const void* h_t,
+                                    const void* W_s, const void* W_t, rkl_dtype dtype,
+                                    int64_t B, int64_t Sm1, int64_t H, int64_t V,
+                                    const int32_t* row_idx, int32_t N, const int32_t* targets,
+                                    rkl_reduction reduction, const float* saved,
+                                    const float* grad_loss, const float* grad_tok,
+                                    float* dH_s, float* dW_s,
+                                    void* workspace, size_t workspace_bytes, void* stream);
 
 /* Backward of the top-k estimator: dz [T, V] of `dtype` (overwritten) with
  * exact zero rows at masked positions; row weights g as rkl_backward; saved

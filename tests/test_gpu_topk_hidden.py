@@ -1,0 +1,137 @@
+"""GPU parity of the top-k estimator on the hidden-state payload against the
+float64 oracle.
+
+The support is decided on the kernels' fp32 logits and on the oracle's
+float64 logits; the two can disagree only where the k-th and (k+1)-th
+student logits (or the sampled token's logit and the k-th) lie within fp32
+rounding of each other.  Such rows are listed by the oracle side and left out
+of the per-token comparison (their results are valid for either order); the
+test requires them to be rare.  Covers several k from the empty support to
+the whole row, more than one 512-row logit block, ragged vocabularies, both
+reductions, masked rows, the autograd wrapper and the full-size workload.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from full_vocabulary_reverse_b200 import binding as rb
+from full_vocabulary_reverse_b200.workloads import make_inputs
+from oracle import rkl_oracle as O
+from tests.gpu_cases import GRAD_RTOL, TOK_ATOL, TOK_RTOL, grad_rel_err, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+def _case(B, Sm1, H, V, seed, mask="random"):
+    inp = make_inputs(B, Sm1, H, V, dtype="bf16", payload="hidden", mask=mask, weights="perturbed", seed=seed,
+                      device="cpu", teacher_noise=0.05)
+    y = torch.from_numpy(np.random.RandomState(seed + 5).randint(0, V, size=(B, Sm1)).astype(np.int32))
+    return inp, y
+
+
+def _ambiguous(inp, y, k):
+    """Flattened positions whose support or tail decision is within fp32 reach."""
+    h_s = to_np(inp["h_s"])
+    W_s = to_np(inp["W_s"])
+    z = h_s @ W_s.T
+    V = z.shape[1]
+    out = set()
+    if k <= 0 or k >= V:
+        return out
+    zs = -np.sort(-z, axis=1)
+    yflat = y.numpy().reshape(-1)
+    trainable = inp["mask"].numpy().reshape(-1) != 0
+    for r in range(z.shape[0]):
+        if not trainable[r]:
+            continue
+        thr = zs[r, k - 1]
+        # fp32 logits of H bf16 products are within ~1e-6 |z| of the float64 ones
+        tol = 2e-5 * max(1.0, abs(thr))
+        if zs[r, k - 1] - zs[r, k] < tol or abs(z[r, yflat[r]] - thr) < tol:
+            out.add(r)
+    return out
+
+
+def _run(inp, y, k, red, grad_tok=None):
+    h_s, h_t, W_s, W_t = (inp[n].cuda() for n in ("h_s", "h_t", "W_s", "W_t"))
+    mask = inp["mask"].cuda()
+    B, Sm1 = mask.shape
+    row_idx, N = rb.compact_rows(mask)
+    lt, loss, saved = rb.forward_topk_hidden(h_s, h_t, W_s, W_t, y.cuda(), k, B, Sm1, row_idx, N, red)
+    gt = None if grad_tok is None else torch.as_tensor(grad_tok, dtype=torch.float32).cuda()
+    dH, dW = rb.backward_topk_hidden(h_s, h_t, W_s, W_t, y.cuda(), B, Sm1, row_idx, N, red, saved,
+                                     grad_loss=torch.ones(1, device="cuda"), grad_tok=gt)
+    torch.cuda.synchronize()
+    assert rb.device_error() == 0
+    return lt, loss, dH, dW, N
+
+
+def _check(inp, y, k, red, grad_tok=None):
+    lt, loss, dH, dW, N = _run(inp, y, k, red, grad_tok)
+    args = (to_np(inp["h_s"]), to_np(inp["W_s"]), to_np(inp["h_t"]), to_np(inp["W_t"]), y.numpy(), k,
+            inp["mask"].numpy(), red)
+    ref = O.forward_topk_hidden(*args)
+    dH_ref, dW_ref = O.backward_topk_hidden(*args, grad_tok=grad_tok)
+    amb = _ambiguous(inp, y, k)
+    assert len(amb) <= max(2, N // 50)
+    keep = np.array([r not in amb for r in range(lt.numel())])
+    g = to_np(lt).reshape(-1)[keep]
+    r = ref["loss_tok"].reshape(-1)[keep]
+    bad = np.abs(g - r) > TOK_ATOL + TOK_RTOL * np.abs(r)
+    assert not bad.any(), (np.flatnonzero(bad)[:5], g[bad][:5], r[bad][:5])
+    assert grad_rel_err(dH, dH_ref) < GRAD_RTOL
+    assert grad_rel_err(dW, dW_ref) < GRAD_RTOL
+    off = inp["mask"].reshape(-1).numpy() == 0
+    assert np.all(to_np(lt).reshape(-1)[off] == 0) and np.all(to_np(dH)[off] == 0)
+    return N
+
+
+@pytest.mark.parametrize("k", [0, 1, 64, 1040])
+def test_topk_hidden_two_blocks(k):
+    # about 600 trainable rows: two 512-row logit blocks, the second partial
+    inp, y = _case(3, 400, 128, 1040, seed=60 + k)
+    assert _check(inp, y, k, 1) > 512
+
+
+@pytest.mark.parametrize("red", [0, 2])
+def test_topk_hidden_reductions_and_chunks(red):
+    # V spans two backward vocab chunks; per-token upstream gradient or nested mean
+    inp, y = _case(2, 100, 64, 65536 + 904, seed=70 + red)
+    gt = np.random.RandomState(3).normal(size=inp["mask"].shape) if red == 0 else None
+    _check(inp, y, 32, red, grad_tok=gt)
+
+
+def test_topk_hidden_whole_row_equals_exact_loss():
+    inp, y = _case(2, 120, 128, 777, seed=80)
+    lt, loss, dH, dW, N = _run(inp, y, 777, 1)
+    h_s, h_t, W_s, W_t = (inp[n].cuda() for n in ("h_s", "h_t", "W_s", "W_t"))
+    row_idx, N2 = rb.compact_rows(inp["mask"].cuda())
+    lt2, _, saved = rb.forward_hidden(h_s, h_t, W_s, W_t, 2, 120, row_idx, N2, 1)
+    dH2, dW2 = rb.backward(rb.PAYLOAD_HIDDEN, h_s, h_t, W_s, W_t, 2, 120, row_idx, N2, 1, saved,
+                           grad_loss=torch.ones(1, device="cuda"))
+    assert np.max(np.abs(to_np(lt) - to_np(lt2))) < 1e-4
+    assert grad_rel_err(dH, to_np(dH2)) < 1e-2 and grad_rel_err(dW, to_np(dW2)) < 1e-2
+
+
+def test_topk_hidden_autograd_wrapper():
+    inp, y = _case(2, 80, 128, 600, seed=90)
+    h_s = inp["h_s"].cuda().requires_grad_(True)
+    W_s = inp["W_s"].cuda().requires_grad_(True)
+    loss, _ = rb.topk_estimator_hidden(h_s, inp["h_t"].cuda(), W_s, inp["W_t"].cuda(), y.cuda(), inp["mask"].cuda(),
+                                       16, 1)
+    loss.backward()
+    args = (to_np(inp["h_s"]), to_np(inp["W_s"]), to_np(inp["h_t"]), to_np(inp["W_t"]), y.numpy(), 16,
+            inp["mask"].numpy(), 1)
+    dH_ref, dW_ref = O.backward_topk_hidden(*args)
+    assert grad_rel_err(h_s.grad.float(), dH_ref) < GRAD_RTOL
+    assert grad_rel_err(W_s.grad.float(), dW_ref) < GRAD_RTOL
+
+
+def test_topk_hidden_fp32_is_rejected():
+    inp, y = _case(1, 8, 64, 100, seed=91)
+    h = inp["h_s"].float().cuda()
+    W = inp["W_s"].float().cuda()
+    row_idx, N = rb.compact_rows(torch.ones((1, 8), dtype=torch.uint8).cuda())
+    with pytest.raises(rb.RKLError):
+        rb.forward_topk_hidden(h, h, W, W, y.cuda(), 4, 1, 8, row_idx, N, 1)
