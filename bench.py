@@ -125,7 +125,8 @@ class Problem:
         self.multi = "teacher_idx" in inp
         self.n_teachers = inp["W_t"].shape[0] if self.multi else 1
         self.topk = self.pair and "targets" in inp
-        self.k = int(self.cfg.get("k", 0)) if self.topk else None
+        self.topk_hidden = (not self.pair) and "targets" in inp
+        self.k = int(self.cfg.get("k", 0)) if (self.topk or self.topk_hidden) else None
         self.student = inp["student_logits"] if self.pair else inp["h_s"]
         self.H = 0 if self.pair else inp["h_s"].shape[1]
         self.V = inp["student_logits"].shape[1] if self.pair else inp["W_s"].shape[0]
@@ -143,6 +144,8 @@ class Problem:
             nbytes = rb.workspace_size_multi(self.dt, self.T, self.n_teachers, self.B, self.Sm1, self.H, self.V)
             self.counts_dev = torch.empty(self.n_teachers + 1, dtype=torch.int32, device=device)
             self.counts_host = torch.empty(self.n_teachers + 1, dtype=torch.int32).pin_memory()
+        elif self.topk_hidden:
+            nbytes = rb.workspace_size(rb.PAYLOAD_TOPK_HIDDEN, self.dt, self.T, self.B, self.Sm1, self.H, self.V)
         else:
             nbytes = rb.workspace_size(self.payload, self.dt, self.T, self.B, self.Sm1, max(self.H, 64), self.V)
         self.ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
@@ -165,7 +168,7 @@ class Problem:
         out = [self.student, self.teacher, self.inp["mask"]]
         if self.multi:
             out.append(self.inp["teacher_idx"])
-        if self.topk:
+        if self.topk or self.topk_hidden:
             out.append(self.inp["targets"])
         return out
 
@@ -200,6 +203,18 @@ class Problem:
             rb._check(L.rkl_backward_logits_pair(p(h_s), p(teacher), self.dt, self.B, self.Sm1, self.V,
                                                  p(self.row_idx), N, self.reduction, p(self.saved),
                                                  p(self.grad_loss), None, p(self.dz), p(self.ws), self.ws.numel(), s))
+            self.N = N
+            return N
+        if self.topk_hidden:
+            tg = self.inp["targets"] if extra is None else extra
+            rb._check(L.rkl_forward_topk_hidden(p(h_s), p(teacher), p(self.inp["W_s"]), p(self.W_t), self.dt, self.B,
+                                                self.Sm1, self.H, self.V, p(self.row_idx), N, self.k, p(tg),
+                                                self.reduction, p(self.loss_tok), p(self.loss), p(self.saved),
+                                                p(self.ws), self.ws.numel(), s))
+            rb._check(L.rkl_backward_topk_hidden(p(h_s), p(teacher), p(self.inp["W_s"]), p(self.W_t), self.dt,
+                                                 self.B, self.Sm1, self.H, self.V, p(self.row_idx), N, p(tg),
+                                                 self.reduction, p(self.saved), p(self.grad_loss), None, p(self.dH),
+                                                 p(self.dW), p(self.ws), self.ws.numel(), s))
             self.N = N
             return N
         if self.logits:
@@ -270,6 +285,11 @@ def algorithmic_work(prob, N):
     if prob.pair:
         return {"pair_fwd": ("hbm", 4.0 * N * V + 16.0 * N),
                 "pair_bwd": ("hbm", 4.0 * N * V + 2.0 * prob.T * V)}
+    if prob.topk_hidden:
+        # writer 4 N H V (z_s and z_t), selection/estimate over the written fp32
+        # logits (read 2 x 4 N V bytes once), dz recompute 4 N H V, grad 4 N H V
+        return {"zw_dual_tc": ("tensor", 4.0 * N * H * V), "topk_fwd": ("hbm", 8.0 * N * V),
+                "dz_topk_tc": ("tensor", 4.0 * N * H * V), "grad_dw_dh_tc": ("tensor", 4.0 * N * H * V)}
     if prob.logits:
         return {"fwd_single_tc": ("tensor", 2.0 * N * H * V), "dz_single_tc": ("tensor", 2.0 * N * H * V),
                 "grad_dw_dh_tc": ("tensor", 4.0 * N * H * V), "teacher_lse": ("hbm", 2.0 * N * V + 4.0 * N)}
@@ -332,6 +352,10 @@ def cpu_oracle_sample(inp, reduction, name, rows=CPU_SAMPLE_ROWS, k=None):
             tid = inp["teacher_idx"].cpu().numpy()
             O.forward_multi(h_s, W_s, teacher, W_t, tid, sub, reduction)
             O.backward_multi(h_s, W_s, teacher, W_t, tid, sub, reduction)
+        elif "targets" in inp:
+            y = inp["targets"].cpu().numpy()
+            O.forward_topk_hidden(h_s, W_s, teacher, W_t, y, k, sub, reduction)
+            O.backward_topk_hidden(h_s, W_s, teacher, W_t, y, k, sub, reduction)
         else:
             O.forward(h_s, W_s, teacher, W_t, sub, reduction)
             O.backward(h_s, W_s, teacher, W_t, sub, reduction)
@@ -491,7 +515,8 @@ def run_gpu(args, rank, world, dist):
         "config": {"workload": args.workload, "B": prob.B, "Sm1": prob.Sm1, "H": prob.H, "V": prob.V,
                    "trainable_rows": N, "tokens_T": prob.T,
                    "payload": ("logits_pair, top-k estimator k=%d" % prob.k if prob.topk else "logits_pair")
-                   if prob.pair else ("logits" if prob.logits else
+                   if prob.pair else ("hidden, top-k estimator k=%d" % prob.k if prob.topk_hidden else
+                                      "logits" if prob.logits else
                                                                  ("hidden, %d teachers" % prob.n_teachers
                                                                   if prob.multi else "hidden")),
                    "parallelism": "replicas" if world > 1 else "single",

@@ -26,6 +26,9 @@ Named workloads:
   logits_pair_topk  logits_pair inputs, top-k estimator with k = 64 and the
                   sampled token of each position drawn from the student's
                   softmax (on-policy sample).
+  topk_hidden     qwen_hidden inputs, top-k estimator with k = 64 and a
+                  sampled token per position drawn uniformly (the estimator's
+                  cost does not depend on how the tokens were drawn).
   multi_teacher   qwen_hidden shapes and mask with two teacher heads
                   W_t[g] = W_s + N(0, 0.004^2) (independent draws), teacher
                   of sequence b = b mod 2; token mean.
@@ -59,6 +62,9 @@ WORKLOADS = {
     "logits_pair_topk": dict(dtype="bf16", B=4, Sm1=2048, H=0, V=151936, payload="logits_pair",
                              reduction=REDUCE_TOKEN_MEAN, mask="all", weights="perturbed", seed=1242,
                              targets="sampled", k=64),
+    "topk_hidden": dict(dtype="bf16", B=4, Sm1=2048, H=2048, V=151936, payload="hidden",
+                        reduction=REDUCE_TOKEN_MEAN, mask="prefix", weights="perturbed", seed=1236,
+                        targets="uniform", k=64),
     "multi_teacher": dict(dtype="bf16", B=4, Sm1=2048, H=2048, V=151936, payload="hidden_multi",
                           reduction=REDUCE_TOKEN_MEAN, mask="prefix", weights="perturbed", seed=1241,
                           mask_seed=1236, n_teachers=2, teacher_assign="sequence"),
@@ -188,6 +194,9 @@ def make_inputs(B, Sm1, H, V, dtype="bf16", payload="hidden", mask="prefix",
     else:
         raise ValueError(payload)
     del W_s32
+    if targets == "uniform":
+        y = np.random.RandomState(seed + 11).randint(0, V, size=(B, Sm1)).astype(np.int32)
+        out["targets"] = torch.from_numpy(y).to(device)
     out["mask"] = torch.from_numpy(make_mask(mask, B, Sm1, seed if mask_seed is None else mask_seed)).to(device)
     return out
 

@@ -135,3 +135,46 @@ def test_topk_hidden_fp32_is_rejected():
     row_idx, N = rb.compact_rows(torch.ones((1, 8), dtype=torch.uint8).cuda())
     with pytest.raises(rb.RKLError):
         rb.forward_topk_hidden(h, h, W, W, y.cuda(), 4, 1, 8, row_idx, N, 1)
+
+
+@pytest.mark.slow
+def test_topk_hidden_full_size():
+    # topk_hidden: the qwen_hidden problem (N = 3635, H = 2048, V = 151936),
+    # k = 64; sampled rows against the oracle (rows whose support is within
+    # fp32 reach of a tie are skipped), and two identities over the whole
+    # problem: sum_v dW_s = 0 and <dW_s, W_s> = <dH_s, h_s>
+    from full_vocabulary_reverse_b200.workloads import make_workload
+    inp = make_workload("topk_hidden", device="cuda")
+    k, red = inp["cfg"]["k"], inp["reduction"]
+    mask = inp["mask"]
+    B, Sm1 = mask.shape
+    row_idx, N = rb.compact_rows(mask)
+    y = inp["targets"]
+    lt, loss, saved = rb.forward_topk_hidden(inp["h_s"], inp["h_t"], inp["W_s"], inp["W_t"], y, k, B, Sm1, row_idx,
+                                             N, red)
+    dH, dW = rb.backward_topk_hidden(inp["h_s"], inp["h_t"], inp["W_s"], inp["W_t"], y, B, Sm1, row_idx, N, red,
+                                     saved, grad_loss=torch.ones(1, device="cuda"))
+    torch.cuda.synchronize()
+    assert rb.device_error() == 0
+    ridx = row_idx[:N].cpu().numpy()
+    pick = np.unique(np.concatenate([[0, N - 1], np.random.RandomState(8).choice(N, 14, replace=False)]))
+    rows = ridx[pick]
+    rt = torch.as_tensor(rows, device="cuda")
+    f = lambda t: t.float().cpu().numpy().astype(np.float64)  # noqa: E731
+    z_s = f(inp["h_s"][rt]) @ f(inp["W_s"]).T
+    z_t = f(inp["h_t"][rt]) @ f(inp["W_t"]).T
+    yy = y.reshape(-1)[rt].cpu().numpy()
+    L_ref, dz_ref = O.topk_rows(z_s, z_t, yy, k, np.full(len(rows), 1.0 / N))
+    zs_sorted = -np.sort(-z_s, axis=1)
+    clear = (zs_sorted[:, k - 1] - zs_sorted[:, k] > 2e-5 * np.abs(zs_sorted[:, k - 1])) & \
+            (np.abs(z_s[np.arange(len(rows)), yy] - zs_sorted[:, k - 1]) > 2e-5 * np.abs(zs_sorted[:, k - 1]))
+    g_tok = to_np(lt.reshape(-1)[rt])
+    assert np.all(np.abs(g_tok - L_ref)[clear] <= (TOK_ATOL + TOK_RTOL * np.abs(L_ref))[clear])
+    g_dH = to_np(dH[rt])
+    r_dH = dz_ref @ f(inp["W_s"])
+    assert np.max(np.abs(g_dH - r_dH)[clear]) / np.max(np.abs(r_dH)) < GRAD_RTOL
+    dWd, dHd = dW.double(), dH.double()
+    assert dWd.sum(dim=0).abs().max().item() <= 2e-2 * dWd.abs().sum(dim=0).max().item()
+    a = (dWd * inp["W_s"].double()).sum().item()
+    b = (dHd * inp["h_s"].double()).sum().item()
+    assert abs(a - b) <= 1e-3 * (dWd * inp["W_s"].double()).abs().sum().item()
