@@ -158,7 +158,7 @@ struct Plan {
   long long zpitch = 0;  // its row pitch (floats)
 };
 
-constexpr int kTopkBlockRows = 512;  // top-k, hidden payload: rows whose logits are written at a time
+constexpr int kTopkBlockRows = 2048;  // top-k, hidden payload: rows whose logits are written at a time
 
 static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 

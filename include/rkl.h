@@ -243,7 +243,7 @@ rkl_status rkl_forward_topk_pair(const void* student_logits, const void* teacher
 
 /* The same estimator on the hidden-state payload (bf16 only; RKL_FP32 gives
  * RKL_ERR_UNSUPPORTED): z_s = h_s W_s^T and z_t = h_t W_t^T as in
- * rkl_forward_hidden.  The forward writes the fp32 logits of at most 512
+ * rkl_forward_hidden.  The forward writes the fp32 logits of at most 2048
  * compacted rows at a time into the workspace and selects / estimates on
  * them; the backward recomputes the logits tile by tile (bitwise the same
  * fp32 values, so the support is the forward's) and runs the gradient GEMMs

@@ -7,7 +7,7 @@ student logits (or the sampled token's logit and the k-th) lie within fp32
 rounding of each other.  Such rows are listed by the oracle side and left out
 of the per-token comparison (their results are valid for either order); the
 test requires them to be rare.  Covers several k from the empty support to
-the whole row, more than one 512-row logit block, ragged vocabularies, both
+the whole row, more than one 2048-row logit block, ragged vocabularies, both
 reductions, masked rows, the autograd wrapper and the full-size workload.
 """
 
@@ -89,9 +89,9 @@ def _check(inp, y, k, red, grad_tok=None):
 
 @pytest.mark.parametrize("k", [0, 1, 64, 1040])
 def test_topk_hidden_two_blocks(k):
-    # about 600 trainable rows: two 512-row logit blocks, the second partial
-    inp, y = _case(3, 400, 128, 1040, seed=60 + k)
-    assert _check(inp, y, k, 1) > 512
+    # about 2400 trainable rows: two 2048-row logit blocks, the second partial
+    inp, y = _case(6, 800, 128, 1040, seed=60 + k)
+    assert _check(inp, y, k, 1) > 2048
 
 
 @pytest.mark.parametrize("red", [0, 2])
