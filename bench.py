@@ -305,8 +305,9 @@ def source_sha():
     return h.hexdigest()[:16]
 
 
-def traffic_for(kernel):
-    """DRAM bytes per launch from the committed ncu summary, or None if stale."""
+def traffic_for(kernel, workload):
+    """DRAM bytes per launch of `kernel` on `workload` from the committed ncu
+    summary, or None if there is none or the kernel sources changed since."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.json")
     if not os.path.exists(path):
         return None
@@ -314,7 +315,7 @@ def traffic_for(kernel):
         d = json.load(f)
     if d.get("source_sha") != source_sha():
         return None
-    k = d.get("kernels", {}).get(kernel)
+    k = d.get("kernels", {}).get("%s@%s" % (kernel, workload))
     return None if k is None else k.get("dram_bytes_per_launch")
 
 
@@ -503,7 +504,7 @@ def run_gpu(args, rank, world, dist):
             per_l = w * args.steps / prof[k]["launches"]
             ach = per_l / (prof[k]["ms"] / prof[k]["launches"] / 1000.0) / 1e9
             extra[k] = {"bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                        "frac": ach / pk["hbm_gbs"], "traffic": traffic_for(k)}
+                        "frac": ach / pk["hbm_gbs"], "traffic": traffic_for(k, prob.name)}
     step_flops = sum(w for b, w in work.values() if b == "tensor")
     step_tflops = step_flops * args.steps / (ms / 1000.0) / 1e12
     step_bytes = sum(w for b, w in work.values() if b == "hbm")
@@ -525,7 +526,7 @@ def run_gpu(args, rank, world, dist):
                         ((1 + prob.n_teachers) if not prob.logits else 1) * prob.V * prob.H * 2)
                        / 1e9)},
         "roofline": {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
-                     "frac": achieved / peak, "traffic": traffic_for(dom),
+                     "frac": achieved / peak, "traffic": traffic_for(dom, prob.name),
                      "peak_source": "%s %s" % (pk["source"], "bf16 sustained" if bound == "tensor" else "hbm copy"),
                      "frac_of_burst": achieved / pk["bf16_tflops"] if bound == "tensor" else None},
         "roofline_hbm_kernels": extra or None,
