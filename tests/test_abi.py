@@ -153,3 +153,37 @@ def test_multi_teacher_argument_errors(L):
     assert L.rkl_compact_rows_multi(_fake(GOOD), None, 2, 3, 2, _fake(GOOD), _fake(GOOD), _fake(GOOD), None) == 1
     assert L.rkl_compact_rows_multi(_fake(GOOD), _fake(GOOD), 2, 3, 0, _fake(GOOD), _fake(GOOD), _fake(GOOD),
                                     None) == 2
+
+
+def test_topk_argument_errors(L):
+    def fwd_pair(k=8, targets=GOOD, ws_bytes=1 << 40):
+        return L.rkl_forward_topk_pair(_fake(GOOD), _fake(GOOD), 0, 2, 3, 1000, _fake(GOOD), 4, k,
+                                       _fake(targets) if targets else None, 1, _fake(GOOD), _fake(GOOD), _fake(GOOD),
+                                       _fake(GOOD), ws_bytes, None)
+    assert fwd_pair(k=-1) == 2
+    assert fwd_pair(targets=0) == 1
+    assert fwd_pair(targets=GOOD + 4) == 4
+    assert fwd_pair(ws_bytes=8) == 5
+
+    def fwd_hidden(dtype=0, k=8, targets=GOOD, H=64):
+        return L.rkl_forward_topk_hidden(_fake(GOOD), _fake(GOOD), _fake(GOOD), _fake(GOOD), dtype, 2, 3, H, 1000,
+                                         _fake(GOOD), 4, k, _fake(targets) if targets else None, 1, _fake(GOOD),
+                                         _fake(GOOD), _fake(GOOD), _fake(GOOD), 1 << 40, None)
+    assert fwd_hidden(dtype=1) == 6          # fp32: unsupported on this path
+    assert fwd_hidden(k=-3) == 2
+    assert fwd_hidden(targets=0) == 1
+    assert fwd_hidden(H=100) == 2            # bf16 needs H % 64 == 0
+
+
+def test_workspace_sizes_follow_the_layout(L):
+    def size(payload, n, H=2048, V=151936, B=4, Sm1=2048):
+        sz = ctypes.c_size_t()
+        assert L.rkl_workspace_size(payload, 0, n, B, Sm1, H, V, ctypes.byref(sz)) == 0
+        return sz.value
+    # grows with the rows; the top-k hidden workspace adds the logit block and row constants
+    assert size(0, 1) < size(0, 1000) < size(0, 8192)
+    assert size(3, 4096) > size(0, 4096) + 2 * 2048 * 151936 * 4 - 1
+    # the logits-pair workspace holds only per-row constants
+    assert size(2, 8192) < 1 << 20
+    # rows round up to whole 256-row pair tiles
+    assert size(0, 1) == size(0, 256) and size(0, 257) > size(0, 256)
