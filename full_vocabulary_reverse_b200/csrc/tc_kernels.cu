@@ -855,16 +855,18 @@ __global__ void __launch_bounds__(kThreads, 1) grad_kernel(const __grid_constant
       for (int j = 0; j < 2; ++j) {
         const int col = j * (kGradBN / 2) + sub * 128;  // first column of this warp in the tile
         const uint32_t tb = tmem_base + lane_off + col;
-#pragma unroll 1
+        // all 128 columns of this warp's part of the half in one burst, so the
+        // half is released to the next tile's MMAs before any staging work
+        float vv[4][32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld_32x32(tb + c * 32, vv[c]);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(acc_empty0 + j * 8);
+#pragma unroll
         for (int c = 0; c < 4; ++c) {
-          float v[32];
-          tmem_ld_32x32(tb + c * 32, v);
-          tmem_wait_ld();
-          if (c == 3) {
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(acc_empty0 + j * 8);
-          }
+          const float* v = vv[c];
           if (lane == 0) bulk_wait_read<0>();
           __syncwarp();
           const uint32_t rbase = smem_u32(buf) + lane * 128;
