@@ -297,9 +297,24 @@ def algorithmic_work(prob, N):
             "grad_dw_dh_tc": ("tensor", 4.0 * N * H * V)}
 
 
-def source_sha():
+# the sources each kernel family is built from: a family's stored DRAM traffic
+# stays valid while these files are unchanged
+SOURCE_GROUPS = {
+    "tc": ("tc_kernels.cu", "sm100.cuh", "kernels.h", "api.cu"),
+    "small": ("small_kernels.cu", "kernels.h", "api.cu"),
+    "topk": ("topk_kernels.cu", "sm100.cuh", "kernels.h", "api.cu"),
+}
+
+
+def kernel_group(kernel):
+    if kernel.startswith("topk_"):
+        return "topk"
+    return "tc" if kernel.endswith("_tc") else "small"
+
+
+def source_sha(group):
     h = hashlib.sha256()
-    for f in ("tc_kernels.cu", "small_kernels.cu", "topk_kernels.cu", "sm100.cuh", "kernels.h", "api.cu"):
+    for f in SOURCE_GROUPS[group]:
         with open(os.path.join(ROOT, "full_vocabulary_reverse_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -307,13 +322,14 @@ def source_sha():
 
 def traffic_for(kernel, workload):
     """DRAM bytes per launch of `kernel` on `workload` from the committed ncu
-    summary, or None if there is none or the kernel sources changed since."""
+    summary, or None if there is none or the kernel's sources changed since."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
         d = json.load(f)
-    if d.get("source_sha") != source_sha():
+    group = kernel_group(kernel)
+    if d.get("source_sha", {}).get(group) != source_sha(group):
         return None
     k = d.get("kernels", {}).get("%s@%s" % (kernel, workload))
     return None if k is None else k.get("dram_bytes_per_launch")

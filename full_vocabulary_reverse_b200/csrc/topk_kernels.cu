@@ -15,20 +15,25 @@
 //            L_S = sum_S p_s w, P_S = sum_S p_s.
 //
 // Forward, one CTA per trainable row:
-//   pass A  streams z_s and z_t once: online log-sum-exp of both sides and a
-//           4096-bin histogram of the top 12 bits of an order-preserving
-//           integer key of z_s; a block scan from the top finds the bin of
-//           the k-th largest key;
-//   pass B  streams z_s once more: keys above that bin are members of S (z_t
-//           is gathered at them), keys in the bin are appended to a list in
-//           shared memory (key, token id); a bitonic sort of the list orders
-//           it by key, lower token id first, and its first r entries (r = k -
-//           members above the bin) complete S, fixing the k-th key K* and
-//           v_last, the last token id of key K* taken.
-//   If the bin holds more than 4096 entries (long runs of tied logits), the
-//   selection finishes exactly instead: radix passes over the remaining key
-//   bits give K*, and an index-ordered pass ranks the ties of key K* by a
-//   block scan.
+//   pass A  streams z_s and z_t once: online log-sum-exp of both sides.  For
+//           k <= 256 (every thread owning logits) each thread's running
+//           maximum comes for free; the k-th largest of the 256 maxima, tau,
+//           is a lower bound of the k-th largest logit (k distinct logits
+//           reach it).  Otherwise pass A also builds a 4096-bin histogram of
+//           the top 12 bits of an order-preserving integer key of z_s, and a
+//           block scan from the top finds the bin of the k-th largest key.
+//   pass B  streams z_s once more.  Threshold path: keys >= tau go to a
+//           candidate list (key, token id) in shared memory; about 70 for
+//           k = 64 on i.i.d. logits.  Histogram path: keys above the bin are
+//           members of S (z_t is gathered at them), keys in the bin are
+//           candidates.  A bitonic sort orders the list by key, lower token id
+//           first, and its first r entries (r = k - members found in pass B)
+//           complete S, fixing the k-th key K* and v_last, the last token id
+//           of key K* taken.
+//   If the list would exceed 4096 entries (long runs of tied logits), the
+//   selection finishes exactly instead: radix passes over the key bits not
+//   yet fixed give K*, and an index-ordered pass ranks the ties of key K* by
+//   a block scan.
 // Backward, one CTA per token row: dz_s in one stream over z_s and z_t, S
 // decided by (key > K*) or (key = K* and v <= v_last), exact zero rows at
 // masked positions.
@@ -63,15 +68,16 @@ __device__ __forceinline__ uint32_t fkey_raw(float x) {
 }
 
 // Keys of the two bf16 values packed in a 32-bit word, each in its half of the
-// result (the same order-preserving map, applied to both halves at once: a
-// positive value's sign bit is set, a negative value's bits are inverted, and
-// -0 takes the key of +0).
+// result (the same order-preserving map, applied to both halves at once).  A
+// packed bf16 add of +0 turns -0 into +0 (a zero sum of opposite-signed zeros
+// is +0 under round-to-nearest) and leaves every other value as it is; prmt
+// with sign replication spreads each half's sign bit over the half; then a
+// negative half is inverted and a positive one gets its sign bit set.
 __device__ __forceinline__ uint32_t bf16_pair_keys(uint32_t w) {
-  const uint32_t neg = ((w >> 15) & 0x00010001u) * 0x7FFFu;
-  uint32_t key = (w ^ 0x80008000u) ^ neg;
-  if ((key & 0xFFFFu) == 0x7FFFu) key += 1u;
-  if ((key >> 16) == 0x7FFFu) key += 0x10000u;
-  return key;
+  uint32_t c, s;
+  asm("add.rn.bf16x2 %0, %1, %2;" : "=r"(c) : "r"(w), "r"(0u));
+  asm("prmt.b32 %0, %1, 0, 0xBB99;" : "=r"(s) : "r"(c));
+  return c ^ (s | 0x80008000u);
 }
 
 template <typename T>
@@ -205,6 +211,27 @@ __device__ __forceinline__ void add_member(float zs_v, const T* zt, int v, float
   P_S += p;
 }
 
+// Pass B's decision for one logit (key, value x, token id v): on the threshold
+// path keys >= tau become candidates; on the histogram path keys above the
+// bin are members and keys in the bin candidates.
+template <typename T>
+__device__ __forceinline__ void classify(bool thr, uint32_t key, float x, int v, uint32_t tau, uint32_t bin,
+                                         const T* zt, float lse_s, float lse_t, float& L_S, float& P_S,
+                                         unsigned long long* cand, int* ncand) {
+  bool take = false;
+  if (thr) {
+    take = key >= tau;
+  } else {
+    const uint32_t kb = key >> kTopShift;
+    if (kb > bin) add_member<T>(x, zt, v, lse_s, lse_t, L_S, P_S);
+    take = kb == bin;
+  }
+  if (take) {
+    const int slot = atomicAdd(ncand, 1);
+    if (slot < kCap) cand[slot] = (static_cast<unsigned long long>(key) << 32) | (~static_cast<uint32_t>(v));
+  }
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kTkThreads) topk_fwd_kernel(const T* __restrict__ zs_all,
                                                               const T* __restrict__ zt_all,
@@ -221,7 +248,7 @@ __global__ void __launch_bounds__(kTkThreads) topk_fwd_kernel(const T* __restric
   __shared__ int hist2[256];
   __shared__ int scan_sh[32];
   __shared__ float red_sh[4][kTkThreads / 32];
-  __shared__ uint32_t s_kstar;
+  __shared__ uint32_t s_kstar, s_tau;
   __shared__ int s_need, s_vlast, s_ncand, s_bin;
   __shared__ float s_lse[2];
 
@@ -238,8 +265,13 @@ __global__ void __launch_bounds__(kTkThreads) topk_fwd_kernel(const T* __restric
   const uint4* vt = reinterpret_cast<const uint4*>(zt);
   // 0: empty support, 1: the whole row, 2: a proper subset to select
   const int mode = k_sel <= 0 ? 0 : (k_sel >= V ? 1 : 2);
+  // small k with every thread owning logits: the k-th largest of the
+  // threads' maxima bounds the k-th largest logit from below, and no
+  // histogram is needed
+  const bool thr = mode == 2 && k_sel <= kTkThreads && nvec >= kTkThreads;
 
-  for (int i = tid; i < kTopBins; i += kTkThreads) hist[i] = 0;
+  if (mode == 2 && !thr)
+    for (int i = tid; i < kTopBins; i += kTkThreads) hist[i] = 0;
   if (tid == 0) {
     s_ncand = 0;
     s_kstar = mode == 0 ? 0xFFFFFFFFu : 0u;  // above every key / below every key
@@ -254,7 +286,7 @@ __global__ void __launch_bounds__(kTkThreads) topk_fwd_kernel(const T* __restric
     const uint4 ws = tk_ldg_v4(vs + i);
     Io::unpack(ws, xs);
     Io::unpack(tk_ldg_v4(vt + i), xt);
-    if (mode == 2) {
+    if (mode == 2 && !thr) {
       if constexpr (std::is_same<T, __nv_bfloat16>::value) {
         const uint32_t wz[4] = {ws.x, ws.y, ws.z, ws.w};
 #pragma unroll
@@ -293,8 +325,9 @@ __global__ void __launch_bounds__(kTkThreads) topk_fwd_kernel(const T* __restric
     const float xs = Io::one(zs, v), xt = Io::one(zt, v);
     lse_add(m_s, S_s, xs);
     lse_add(m_t, S_t, xt);
-    if (mode == 2) atomicAdd(&hist[(Io::KMASK & fkey_raw(xs)) >> kTopShift], 1);
+    if (mode == 2 && !thr) atomicAdd(&hist[(Io::KMASK & fkey_raw(xs)) >> kTopShift], 1);
   }
+  const float thread_max = m_s;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     lse_join(m_s, S_s, __shfl_xor_sync(0xffffffffu, m_s, o), __shfl_xor_sync(0xffffffffu, S_s, o));
@@ -316,7 +349,17 @@ __global__ void __launch_bounds__(kTkThreads) topk_fwd_kernel(const T* __restric
     s_lse[0] = a + logf(b);
     s_lse[1] = c + logf(d);
   }
-  if (mode == 2) {
+  if (thr) {
+    // tau = the k-th largest of the threads' maximum keys: k distinct logits
+    // reach it, so every logit of the top k does too
+    buf[tid] = (static_cast<unsigned long long>(Io::KMASK & fkey_raw(thread_max)) << 32) | tid;
+    __syncthreads();
+    bitonic_desc(buf, kTkThreads);
+    if (tid == 0) {
+      s_tau = static_cast<uint32_t>(buf[k_sel - 1] >> 32);
+      s_need = static_cast<int>(k_sel);
+    }
+  } else if (mode == 2) {
     // the bin of the k-th largest key: thread tid owns bins [16 g, 16 g + 16),
     // g = 255 - tid, so an inclusive scan in thread order counts from the top
     constexpr int PER = kTopBins / kTkThreads;
@@ -360,56 +403,53 @@ __global__ void __launch_bounds__(kTkThreads) topk_fwd_kernel(const T* __restric
     }
     for (int v = nvec * VEC + tid; v < V; v += kTkThreads) add_member<T>(Io::one(zs, v), zt, v, lse_s, lse_t, L_S, P_S);
   } else if (mode == 2) {
-    // ---- pass B: keys above the bin are members; keys in the bin are candidates
+    // ---- pass B.  Histogram path: keys above the bin are members, keys in
+    // the bin are candidates.  Threshold path: keys >= tau are candidates.
     const uint32_t bin = static_cast<uint32_t>(s_bin);
+    const uint32_t tau = s_tau;
     const int need = s_need;
+    // 16-bit (bf16) keys sit in the top half: a low-half key reaches the
+    // bound iff it is >= lo_thr, a high-half key iff the pair key is >= hi_thr
+    const uint32_t lo_thr = thr ? tau >> 16 : bin << (kTopShift - 16);
+    const uint32_t hi_thr = thr ? tau : bin << kTopShift;
     for (int i = tid; i < nvec; i += kTkThreads) {
       float xs[VEC];
       const uint4 ws = tk_ldg_v4(vs + i);
-      Io::unpack(ws, xs);
       uint32_t keys[VEC];
       if constexpr (std::is_same<T, __nv_bfloat16>::value) {
         const uint32_t wz[4] = {ws.x, ws.y, ws.z, ws.w};
+        uint32_t kp[4];
         bool any = false;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          const uint32_t kp = bf16_pair_keys(wz[q]);
-          keys[2 * q] = kp << 16;
-          keys[2 * q + 1] = kp & 0xFFFF0000u;
-          any |= ((kp >> (kTopShift - 16)) & (kTopBins - 1)) >= bin || (kp >> kTopShift) >= bin;
+          kp[q] = bf16_pair_keys(wz[q]);
+          any |= (kp[q] & 0xFFFFu) >= lo_thr || kp[q] >= hi_thr;
         }
-        if (!any) continue;  // no key of these 8 reaches the bin (the common case)
+        if (!any) continue;  // no key of these 8 reaches the bound (the common case)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          keys[2 * q] = kp[q] << 16;
+          keys[2 * q + 1] = kp[q] & 0xFFFF0000u;
+        }
+        Io::unpack(ws, xs);
       } else {
+        Io::unpack(ws, xs);
 #pragma unroll
         for (int j = 0; j < VEC; ++j) keys[j] = Io::KMASK & fkey_raw(xs[j]);
       }
 #pragma unroll
-      for (int j = 0; j < VEC; ++j) {
-        const uint32_t key = keys[j];
-        const uint32_t kb = key >> kTopShift;
-        if (kb > bin) {
-          add_member<T>(xs[j], zt, i * VEC + j, lse_s, lse_t, L_S, P_S);
-        } else if (kb == bin) {
-          const int slot = atomicAdd(&s_ncand, 1);
-          if (slot < kCap) buf[slot] = (static_cast<unsigned long long>(key) << 32) | (~static_cast<uint32_t>(i * VEC + j));
-        }
-      }
+      for (int j = 0; j < VEC; ++j)
+        classify<T>(thr, keys[j], xs[j], i * VEC + j, tau, bin, zt, lse_s, lse_t, L_S, P_S, buf, &s_ncand);
     }
     for (int v = nvec * VEC + tid; v < V; v += kTkThreads) {
       const float x = Io::one(zs, v);
-      const uint32_t key = Io::KMASK & fkey_raw(x);
-      const uint32_t kb = key >> kTopShift;
-      if (kb > bin) {
-        add_member<T>(x, zt, v, lse_s, lse_t, L_S, P_S);
-      } else if (kb == bin) {
-        const int slot = atomicAdd(&s_ncand, 1);
-        if (slot < kCap) buf[slot] = (static_cast<unsigned long long>(key) << 32) | (~static_cast<uint32_t>(v));
-      }
+      classify<T>(thr, Io::KMASK & fkey_raw(x), x, v, tau, bin, zt, lse_s, lse_t, L_S, P_S, buf, &s_ncand);
     }
     __syncthreads();
     const int nc = s_ncand;
     if (nc <= kCap) {
-      // ---- the candidates in key order (lower token id first on equal keys)
+      // ---- the candidates in key order (lower token id first on equal keys);
+      // the first `need` of them complete the support
       int n2 = 2;
       while (n2 < nc) n2 <<= 1;
       for (int i = nc + tid; i < n2; i += kTkThreads) buf[i] = 0ull;
@@ -425,19 +465,25 @@ __global__ void __launch_bounds__(kTkThreads) topk_fwd_kernel(const T* __restric
         s_vlast = static_cast<int>(~static_cast<uint32_t>(e));
       }
     } else {
-      // ---- too many candidates: finish the radix select on the lower key
-      // bits, then rank the ties of key K* in index order
+      // ---- too many candidates: a radix select over the key bits below the
+      // ones already fixed (the bin's 12, or none on the threshold path) gives
+      // K*, then the ties of key K* are ranked in index order.  Keys whose
+      // fixed bits are above the prefix are members added in pass B.
       const int lo_end = Io::KMASK == 0xFFFF0000u ? 16 : 0;
-      uint32_t prefix = bin << kTopShift;
+      const int hi0 = thr ? 32 : kTopShift;
+      const uint32_t fixed = thr ? 0u : ~0u << kTopShift;  // the key bits fixed before the radix passes
+      const uint32_t prefix0 = thr ? 0u : bin << kTopShift;
+      uint32_t prefix = prefix0;
       int rem = need;
-      for (int hi = kTopShift; hi > lo_end;) {
+      for (int hi = hi0; hi > lo_end;) {
         const int width = hi - lo_end < 8 ? hi - lo_end : 8;
         const int sh = hi - width;
+        const uint32_t hmask = hi >= 32 ? 0u : ~0u << hi;
         for (int i = tid; i < 256; i += kTkThreads) hist2[i] = 0;
         __syncthreads();
         for (int v = tid; v < V; v += kTkThreads) {
           const uint32_t key = Io::KMASK & fkey_raw(Io::one(zs, v));
-          if ((key >> hi) == (prefix >> hi)) atomicAdd(&hist2[(key >> sh) & ((1u << width) - 1u)], 1);
+          if ((key & hmask) == (prefix & hmask)) atomicAdd(&hist2[(key >> sh) & ((1u << width) - 1u)], 1);
         }
         __syncthreads();
         if (tid == 0) {
@@ -472,7 +518,7 @@ __global__ void __launch_bounds__(kTkThreads) topk_fwd_kernel(const T* __restric
 #pragma unroll
         for (int j = 0; j < VEC; ++j) {
           const int v = v0 + j;
-          if (v >= V || (keys[j] >> kTopShift) != bin) continue;  // keys above the bin are counted
+          if (v >= V || (keys[j] & fixed) != prefix0) continue;  // members added in pass B, or below
           bool in = keys[j] > kstar;
           if (keys[j] == kstar) {
             in = rank < rem;

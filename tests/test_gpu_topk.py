@@ -149,19 +149,73 @@ def test_topk_full_size():
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "fp32"])
-@pytest.mark.parametrize("k", [100, 3000, 8999])
-def test_topk_many_ties_take_the_exact_path(dtype, k):
-    # student logits drawn from three values: the bin of the k-th logit holds
-    # thousands of tied entries, more than the shared-memory candidate list,
-    # so the selection finishes with the exact radix / index-order path
+@pytest.mark.parametrize("k,probs", [(100, [0.2, 0.5, 0.3]), (3000, [0.2, 0.5, 0.3]), (8999, [0.2, 0.5, 0.3]),
+                                     (1, [0.2, 0.3, 0.5]), (100, [0.2, 0.3, 0.5]), (256, [0.2, 0.3, 0.5])])
+def test_topk_many_ties_take_the_exact_path(dtype, k, probs):
+    # student logits drawn from three values: the bin of the k-th logit (or,
+    # for k <= 256, the bound from the threads' maxima) admits thousands of
+    # tied entries; above 4096, more than the shared-memory candidate list,
+    # the selection finishes with the exact radix / index-order path
     inp, y = _case(2, 20, 9000, dtype=dtype, seed=k)
     rs = np.random.RandomState(k)
-    vals = rs.choice([-1.0, 0.5, 2.0], size=inp["student_logits"].shape, p=[0.2, 0.5, 0.3])
+    vals = rs.choice([-1.0, 0.5, 2.0], size=inp["student_logits"].shape, p=probs)
     inp["student_logits"] = torch.from_numpy(vals).to(inp["student_logits"].dtype)
     lt, loss, dz, N = _run(inp, y, k, 1)
     ref, dz_ref = _ref(inp, y, k, 1)
     assert_tok_close(lt, ref["loss_tok"])
     assert grad_rel_err(dz, dz_ref) < (GRAD_RTOL if dtype == "bf16" else 1e-4)
+
+
+def _key(x, dtype):
+    # order-preserving integer key of a logit, -0 and +0 sharing one key; a
+    # bf16 logit keeps only its 16 significant bits
+    u = np.float32(x).view(np.uint32) if x != 0 else np.uint32(0)
+    k = (~u if u & np.uint32(0x80000000) else u | np.uint32(0x80000000)) & np.uint32(0xFFFFFFFF)
+    return int(k) & (0xFFFF0000 if dtype == "bf16" else 0xFFFFFFFF)
+
+
+# logit values: -1, -0, +0, 1e-39, -1e-39, 3e-39 (subnormal), 0.5
+_ZERO_MIXES = [
+    # k-th logit inside a run of ~1600 zeros (candidate list, histogram path)
+    (4103, [0.25, 0.2, 0.2, 0.05, 0.05, 0.05, 0.2], 2051),
+    # a run of ~4900 keys in the bin of zero: more than the list holds (exact path)
+    (9000, [0.25, 0.25, 0.25, 0.05, 0.05, 0.05, 0.1], 4050),
+    # k <= 256: the bound from the threads' maxima is zero, ~3760 candidates
+    (9000, [0.55, 0.2, 0.2, 0.01, 0.03, 0.005, 0.005], 250),
+    # k <= 256 with ~5570 logits at or above the bound (exact path from the top)
+    (9000, [0.35, 0.3, 0.3, 0.01, 0.03, 0.005, 0.005], 250),
+]
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+@pytest.mark.parametrize("V,probs,k", _ZERO_MIXES)
+def test_topk_signed_zeros_and_subnormals(dtype, V, probs, k):
+    # -0 and +0 are one logit value (ties ranked by token id) and subnormal
+    # logits keep their order, with the k-th logit of every row a zero
+    inp, y = _case(2, 10, V, dtype=dtype, seed=V + k)
+    rs = np.random.RandomState(V + k + 1)
+    vals = np.array([-1.0, -0.0, 0.0, 1e-39, -1e-39, 3e-39, 0.5])
+    inp["student_logits"] = torch.from_numpy(rs.choice(vals, size=inp["student_logits"].shape, p=probs)).to(
+        inp["student_logits"].dtype)
+    zs, zt, mask = inp["student_logits"].cuda(), inp["teacher_logits"].cuda(), inp["mask"].cuda()
+    B, Sm1 = mask.shape
+    row_idx, N = rb.compact_rows(mask)
+    lt, loss, saved = rb.forward_topk_pair(zs, zt, y.cuda(), k, B, Sm1, row_idx, N, 1)
+    dz = rb.backward_topk_pair(zs, zt, y.cuda(), B, Sm1, row_idx, N, 1, saved, grad_loss=torch.ones(1, device="cuda"))
+    torch.cuda.synchronize()
+    ref, dz_ref = _ref(inp, y, k, 1)
+    assert_tok_close(lt, ref["loss_tok"])
+    assert grad_rel_err(dz, dz_ref) < (GRAD_RTOL if dtype == "bf16" else 1e-4)
+    # the k-th key K* and the last token id taken at it, exactly
+    z = to_np(inp["student_logits"].reshape(-1, V))
+    rows = row_idx[:N].cpu().numpy()
+    S = O.topk_support(z[rows], k)
+    tk = saved[3 * N:].reshape(N, 4).cpu().numpy()
+    for i in range(N):
+        zmin = z[rows[i]][S[i]].min()
+        assert zmin == 0.0  # the boundary falls in the zero run
+        assert int(tk[i, 2:3].view(np.uint32)[0]) == _key(zmin, dtype)
+        assert int(tk[i, 3:4].view(np.int32)[0]) == int(np.flatnonzero(S[i] & (z[rows[i]] == zmin)).max())
 
 
 def test_topk_autograd_wrapper():
