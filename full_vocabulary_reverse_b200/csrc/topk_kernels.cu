@@ -14,22 +14,24 @@
 //            a = [y not in S](w(y) + 1), C = L_S + P_S + a,
 //            L_S = sum_S p_s w, P_S = sum_S p_s.
 //
-// Forward, one CTA per trainable row:
-//   pass A  streams z_s and z_t once: online log-sum-exp of both sides.  For
-//           k <= 256 (every thread owning logits) each thread's running
-//           maximum comes for free; the k-th largest of the 256 maxima, tau,
-//           is a lower bound of the k-th largest logit (k distinct logits
-//           reach it).  Otherwise pass A also builds a 4096-bin histogram of
-//           the top 12 bits of an order-preserving integer key of z_s, and a
-//           block scan from the top finds the bin of the k-th largest key.
-//   pass B  streams z_s once more.  Threshold path: keys >= tau go to a
-//           candidate list (key, token id) in shared memory; about 70 for
-//           k = 64 on i.i.d. logits.  Histogram path: keys above the bin are
-//           members of S (z_t is gathered at them), keys in the bin are
-//           candidates.  A bitonic sort orders the list by key, lower token id
-//           first, and its first r entries (r = k - members found in pass B)
-//           complete S, fixing the k-th key K* and v_last, the last token id
-//           of key K* taken.
+// Forward, one CTA per trainable row (256 threads, at most 40 registers so
+// that six CTAs share an SM):
+//   Threshold path (k <= 256, every thread owning logits).  z_s and z_t
+//   stream once for both log-sum-exps, two 16-byte vectors of each per step.
+//   After a first slice of the row, the k-th largest of the 256 threads'
+//   running maxima, tau, bounds the k-th largest logit from below (k distinct
+//   logits reach it).  The slice is read a second time (from L2) and the rest
+//   of the row as it streams, listing the logits whose keys reach tau
+//   (key, token id) in shared memory.  The slice is sized for ~256 entries
+//   on i.i.d. logits.
+//   Histogram path (k > 256).  Pass A streams both rows for the log-sum-exps
+//   and a 4096-bin histogram of the top 12 bits of an order-preserving key of
+//   z_s; a block scan from the top finds the bin of the k-th largest key.
+//   Pass B streams z_s again: keys above the bin are members of S (z_t is
+//   gathered at them), keys in the bin are listed.
+//   Either way a bitonic sort orders the list by key, lower token id first,
+//   and its first r entries (r = k - members found before) complete S,
+//   fixing the k-th key K* and v_last, the last token id of key K* taken.
 //   If the list would exceed 4096 entries (long runs of tied logits), the
 //   selection finishes exactly instead: radix passes over the key bits not
 //   yet fixed give K*, and an index-ordered pass ranks the ties of key K* by
@@ -53,6 +55,16 @@ constexpr int kTkThreads = 256;
 __device__ __forceinline__ uint4 tk_ldg_v4(const void* p) {
   uint4 r;
   asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+// The forward's streaming loads bypass L1 (its only reuse, the second read of
+// the first slice, comes from L2).
+__device__ __forceinline__ uint4 tk_ldg_stream_v4(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
                : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
                : "l"(p));
   return r;
@@ -181,6 +193,7 @@ __device__ __forceinline__ void pick_bin(const int* hist, int need, int* bin, in
 constexpr int kTopShift = 20;            // first-level histogram: the top 12 key bits
 constexpr int kTopBins = 1 << (32 - kTopShift);
 constexpr int kCap = 4096;               // candidates sorted in shared memory
+constexpr float kListTarget = 256.f;     // expected candidates on the threshold path
 
 // Descending bitonic sort of n (a power of two, <= kCap) 64-bit entries in
 // shared memory by the whole block.
@@ -188,7 +201,7 @@ __device__ __forceinline__ void bitonic_desc(unsigned long long* a, int n) {
   for (int size = 2; size <= n; size <<= 1) {
     for (int stride = size >> 1; stride > 0; stride >>= 1) {
       for (int i = threadIdx.x; i < n / 2; i += kTkThreads) {
-        const int lo = 2 * stride * (i / stride) + (i % stride);
+        const int lo = ((i & ~(stride - 1)) << 1) | (i & (stride - 1));  // stride is a power of two
         const int hi = lo + stride;
         const unsigned long long x = a[lo], y = a[hi];
         if ((x < y) == ((lo & size) == 0)) {
@@ -211,29 +224,84 @@ __device__ __forceinline__ void add_member(float zs_v, const T* zt, int v, float
   P_S += p;
 }
 
-// Pass B's decision for one logit (key, value x, token id v): on the threshold
-// path keys >= tau become candidates; on the histogram path keys above the
-// bin are members and keys in the bin candidates.
+__device__ __forceinline__ void list_append(uint32_t key, int v, unsigned long long* cand, int* ncand) {
+  const int slot = atomicAdd(ncand, 1);
+  if (slot < kCap) cand[slot] = (static_cast<unsigned long long>(key) << 32) | (~static_cast<uint32_t>(v));
+}
+
+// Histogram path, pass B's decision for one logit (key, value x, token id v):
+// keys above the bin are members, keys in the bin are candidates.
 template <typename T>
-__device__ __forceinline__ void classify(bool thr, uint32_t key, float x, int v, uint32_t tau, uint32_t bin,
-                                         const T* zt, float lse_s, float lse_t, float& L_S, float& P_S,
-                                         unsigned long long* cand, int* ncand) {
-  bool take = false;
-  if (thr) {
-    take = key >= tau;
+__device__ __forceinline__ void classify(uint32_t key, float x, int v, uint32_t bin, const T* zt, float lse_s,
+                                         float lse_t, float& L_S, float& P_S, unsigned long long* cand,
+                                         int* ncand) {
+  const uint32_t kb = key >> kTopShift;
+  if (kb > bin) add_member<T>(x, zt, v, lse_s, lse_t, L_S, P_S);
+  if (kb == bin) list_append(key, v, cand, ncand);
+}
+
+// Threshold path: the logits of one vector of z_s (token ids v0, v0 + 1, ...)
+// whose keys reach the bound tau go to the candidate list.
+template <typename T>
+__device__ __forceinline__ void list_vec(const uint4& ws, int v0, uint32_t tau, unsigned long long* cand,
+                                         int* ncand) {
+  if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+    // 16-bit keys sit in the top half: a low-half key reaches tau iff it is
+    // >= tau >> 16, a high-half key iff the pair key is >= tau
+    const uint32_t wz[4] = {ws.x, ws.y, ws.z, ws.w};
+    uint32_t kp[4];
+    bool any = false;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      kp[q] = bf16_pair_keys(wz[q]);
+      any |= (kp[q] & 0xFFFFu) >= (tau >> 16) || kp[q] >= tau;
+    }
+    if (!any) return;  // the common case
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      if ((kp[q] << 16) >= tau) list_append(kp[q] << 16, v0 + 2 * q, cand, ncand);
+      if ((kp[q] & 0xFFFF0000u) >= tau) list_append(kp[q] & 0xFFFF0000u, v0 + 2 * q + 1, cand, ncand);
+    }
   } else {
-    const uint32_t kb = key >> kTopShift;
-    if (kb > bin) add_member<T>(x, zt, v, lse_s, lse_t, L_S, P_S);
-    take = kb == bin;
+    float x[4];
+    TkIo<float>::unpack(ws, x);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t key = fkey_raw(x[j]);
+      if (key >= tau) list_append(key, v0 + j, cand, ncand);
+    }
   }
-  if (take) {
-    const int slot = atomicAdd(ncand, 1);
-    if (slot < kCap) cand[slot] = (static_cast<unsigned long long>(key) << 32) | (~static_cast<uint32_t>(v));
+}
+
+// One vector of each row into the running log-sum-exps (maximum m, sum S of
+// exp(x - m)).
+template <int VEC>
+__device__ __forceinline__ void lse_vec(const float* xs, const float* xt, float& m_s, float& S_s, float& m_t,
+                                        float& S_t) {
+  float cs = xs[0], ct = xt[0];
+#pragma unroll
+  for (int j = 1; j < VEC; ++j) {
+    cs = fmaxf(cs, xs[j]);
+    ct = fmaxf(ct, xt[j]);
+  }
+  if (cs > m_s) {
+    S_s *= ex2((m_s - cs) * kLog2e);
+    m_s = cs;
+  }
+  if (ct > m_t) {
+    S_t *= ex2((m_t - ct) * kLog2e);
+    m_t = ct;
+  }
+  const float ms2 = m_s * kLog2e, mt2 = m_t * kLog2e;
+#pragma unroll
+  for (int j = 0; j < VEC; ++j) {
+    S_s += ex2(fmaf(xs[j], kLog2e, -ms2));
+    S_t += ex2(fmaf(xt[j], kLog2e, -mt2));
   }
 }
 
 template <typename T>
-__global__ void __launch_bounds__(kTkThreads) topk_fwd_kernel(const T* __restrict__ zs_all,
+__global__ void __launch_bounds__(kTkThreads, 6) topk_fwd_kernel(const T* __restrict__ zs_all,
                                                               const T* __restrict__ zt_all,
                                                               const int32_t* __restrict__ row_idx,
                                                               const int32_t* __restrict__ targets, int N, int V,
@@ -279,13 +347,25 @@ __global__ void __launch_bounds__(kTkThreads) topk_fwd_kernel(const T* __restric
   }
   __syncthreads();
 
-  // ---- pass A: both log-sum-exps and the 12-bit histogram of the z_s keys
+  // ---- pass A: both log-sum-exps, and the 12-bit histogram of the z_s keys
+  // or (threshold path) the candidate list
   float m_s = -INFINITY, S_s = 0.f, m_t = -INFINITY, S_t = 0.f;
-  for (int i = tid; i < nvec; i += kTkThreads) {
+  // Threshold path: vectors [0, i1) stream by before the bound is known and
+  // are listed by a second read while they are still in L2; the rest of the
+  // row is listed as it streams.  The bound is about the (1 - k/256) quantile
+  // of a thread's maximum over its e logits of [0, i1), so about
+  // V ln(256 / (256 - k)) / e logits reach it: e is sized for kListTarget.
+  int i1 = nvec;
+  if (thr) {
+    const float e = static_cast<float>(V) * __logf(256.f / (256.5f - static_cast<float>(k_sel))) / kListTarget;
+    const int j1 = max(1, static_cast<int>(ceilf(e / VEC)));
+    i1 = j1 >= nvec / kTkThreads ? nvec : j1 * kTkThreads;
+  }
+  for (int i = tid; i < i1; i += kTkThreads) {
     float xs[VEC], xt[VEC];
-    const uint4 ws = tk_ldg_v4(vs + i);
+    const uint4 ws = tk_ldg_stream_v4(vs + i);
     Io::unpack(ws, xs);
-    Io::unpack(tk_ldg_v4(vt + i), xt);
+    Io::unpack(tk_ldg_stream_v4(vt + i), xt);
     if (mode == 2 && !thr) {
       if constexpr (std::is_same<T, __nv_bfloat16>::value) {
         const uint32_t wz[4] = {ws.x, ws.y, ws.z, ws.w};
@@ -300,34 +380,58 @@ __global__ void __launch_bounds__(kTkThreads) topk_fwd_kernel(const T* __restric
         for (int j = 0; j < VEC; ++j) atomicAdd(&hist[(Io::KMASK & fkey_raw(xs[j])) >> kTopShift], 1);
       }
     }
-    float cs = xs[0], ct = xt[0];
-#pragma unroll
-    for (int j = 1; j < VEC; ++j) {
-      cs = fmaxf(cs, xs[j]);
-      ct = fmaxf(ct, xt[j]);
+    lse_vec<VEC>(xs, xt, m_s, S_s, m_t, S_t);
+  }
+  uint32_t tau = 0u;
+  if (thr) {
+    // tau = the k-th largest of the threads' maximum keys so far: k distinct
+    // logits reach it, so every logit of the row's top k does too
+    buf[tid] = (static_cast<unsigned long long>(Io::KMASK & fkey_raw(m_s)) << 32) | tid;
+    __syncthreads();
+    bitonic_desc(buf, kTkThreads);
+    if (tid == 0) {
+      s_tau = static_cast<uint32_t>(buf[k_sel - 1] >> 32);
+      s_need = static_cast<int>(k_sel);
     }
-    if (cs > m_s) {
-      S_s *= ex2((m_s - cs) * kLog2e);
-      m_s = cs;
+    __syncthreads();
+    tau = s_tau;
+    for (int i = tid; i < i1; i += kTkThreads) list_vec<T>(tk_ldg_stream_v4(vs + i), i * VEC, tau, buf, &s_ncand);
+    int i = i1 + tid;
+    // two vectors of each row per step, all four loads issued first
+    for (; i + kTkThreads < nvec; i += 2 * kTkThreads) {
+      const uint4 a0 = tk_ldg_stream_v4(vs + i), b0 = tk_ldg_stream_v4(vt + i);
+      const uint4 a1 = tk_ldg_stream_v4(vs + i + kTkThreads), b1 = tk_ldg_stream_v4(vt + i + kTkThreads);
+      float xs[VEC], xt[VEC];
+      list_vec<T>(a0, i * VEC, tau, buf, &s_ncand);
+      Io::unpack(a0, xs);
+      Io::unpack(b0, xt);
+      lse_vec<VEC>(xs, xt, m_s, S_s, m_t, S_t);
+      list_vec<T>(a1, (i + kTkThreads) * VEC, tau, buf, &s_ncand);
+      Io::unpack(a1, xs);
+      Io::unpack(b1, xt);
+      lse_vec<VEC>(xs, xt, m_s, S_s, m_t, S_t);
     }
-    if (ct > m_t) {
-      S_t *= ex2((m_t - ct) * kLog2e);
-      m_t = ct;
-    }
-    const float ms2 = m_s * kLog2e, mt2 = m_t * kLog2e;
-#pragma unroll
-    for (int j = 0; j < VEC; ++j) {
-      S_s += ex2(fmaf(xs[j], kLog2e, -ms2));
-      S_t += ex2(fmaf(xt[j], kLog2e, -mt2));
+    for (; i < nvec; i += kTkThreads) {
+      float xs[VEC], xt[VEC];
+      const uint4 ws = tk_ldg_stream_v4(vs + i);
+      list_vec<T>(ws, i * VEC, tau, buf, &s_ncand);
+      Io::unpack(ws, xs);
+      Io::unpack(tk_ldg_stream_v4(vt + i), xt);
+      lse_vec<VEC>(xs, xt, m_s, S_s, m_t, S_t);
     }
   }
   for (int v = nvec * VEC + tid; v < V; v += kTkThreads) {
     const float xs = Io::one(zs, v), xt = Io::one(zt, v);
     lse_add(m_s, S_s, xs);
     lse_add(m_t, S_t, xt);
-    if (mode == 2 && !thr) atomicAdd(&hist[(Io::KMASK & fkey_raw(xs)) >> kTopShift], 1);
+    if (mode == 2) {
+      const uint32_t key = Io::KMASK & fkey_raw(xs);
+      if (!thr)
+        atomicAdd(&hist[key >> kTopShift], 1);
+      else if (key >= tau)
+        list_append(key, v, buf, &s_ncand);
+    }
   }
-  const float thread_max = m_s;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     lse_join(m_s, S_s, __shfl_xor_sync(0xffffffffu, m_s, o), __shfl_xor_sync(0xffffffffu, S_s, o));
@@ -349,17 +453,7 @@ __global__ void __launch_bounds__(kTkThreads) topk_fwd_kernel(const T* __restric
     s_lse[0] = a + logf(b);
     s_lse[1] = c + logf(d);
   }
-  if (thr) {
-    // tau = the k-th largest of the threads' maximum keys: k distinct logits
-    // reach it, so every logit of the top k does too
-    buf[tid] = (static_cast<unsigned long long>(Io::KMASK & fkey_raw(thread_max)) << 32) | tid;
-    __syncthreads();
-    bitonic_desc(buf, kTkThreads);
-    if (tid == 0) {
-      s_tau = static_cast<uint32_t>(buf[k_sel - 1] >> 32);
-      s_need = static_cast<int>(k_sel);
-    }
-  } else if (mode == 2) {
+  if (mode == 2 && !thr) {
     // the bin of the k-th largest key: thread tid owns bins [16 g, 16 g + 16),
     // g = 255 - tid, so an inclusive scan in thread order counts from the top
     constexpr int PER = kTopBins / kTkThreads;
@@ -391,8 +485,8 @@ __global__ void __launch_bounds__(kTkThreads) topk_fwd_kernel(const T* __restric
     // ---- the whole row is the support
     for (int i = tid; i < nvec; i += kTkThreads) {
       float xs[VEC], xt[VEC];
-      Io::unpack(tk_ldg_v4(vs + i), xs);
-      Io::unpack(tk_ldg_v4(vt + i), xt);
+      Io::unpack(tk_ldg_stream_v4(vs + i), xs);
+      Io::unpack(tk_ldg_stream_v4(vt + i), xt);
 #pragma unroll
       for (int j = 0; j < VEC; ++j) {
         const float ls = xs[j] - lse_s;
@@ -403,47 +497,48 @@ __global__ void __launch_bounds__(kTkThreads) topk_fwd_kernel(const T* __restric
     }
     for (int v = nvec * VEC + tid; v < V; v += kTkThreads) add_member<T>(Io::one(zs, v), zt, v, lse_s, lse_t, L_S, P_S);
   } else if (mode == 2) {
-    // ---- pass B.  Histogram path: keys above the bin are members, keys in
-    // the bin are candidates.  Threshold path: keys >= tau are candidates.
+    // ---- pass B (histogram path): keys above the bin are members, keys in
+    // the bin are candidates; the threshold path has its list already
     const uint32_t bin = static_cast<uint32_t>(s_bin);
-    const uint32_t tau = s_tau;
     const int need = s_need;
-    // 16-bit (bf16) keys sit in the top half: a low-half key reaches the
-    // bound iff it is >= lo_thr, a high-half key iff the pair key is >= hi_thr
-    const uint32_t lo_thr = thr ? tau >> 16 : bin << (kTopShift - 16);
-    const uint32_t hi_thr = thr ? tau : bin << kTopShift;
-    for (int i = tid; i < nvec; i += kTkThreads) {
-      float xs[VEC];
-      const uint4 ws = tk_ldg_v4(vs + i);
-      uint32_t keys[VEC];
-      if constexpr (std::is_same<T, __nv_bfloat16>::value) {
-        const uint32_t wz[4] = {ws.x, ws.y, ws.z, ws.w};
-        uint32_t kp[4];
-        bool any = false;
+    if (!thr) {
+      // 16-bit (bf16) keys sit in the top half: a low-half key is in a bin
+      // >= bin iff it is >= bin << 4, a high-half key iff the pair key is
+      // >= bin << 20
+      const uint32_t lo_thr = bin << (kTopShift - 16), hi_thr = bin << kTopShift;
+      for (int i = tid; i < nvec; i += kTkThreads) {
+        float xs[VEC];
+        const uint4 ws = tk_ldg_stream_v4(vs + i);
+        uint32_t keys[VEC];
+        if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+          const uint32_t wz[4] = {ws.x, ws.y, ws.z, ws.w};
+          uint32_t kp[4];
+          bool any = false;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          kp[q] = bf16_pair_keys(wz[q]);
-          any |= (kp[q] & 0xFFFFu) >= lo_thr || kp[q] >= hi_thr;
+          for (int q = 0; q < 4; ++q) {
+            kp[q] = bf16_pair_keys(wz[q]);
+            any |= (kp[q] & 0xFFFFu) >= lo_thr || kp[q] >= hi_thr;
+          }
+          if (!any) continue;  // no key of these 8 reaches the bin (the common case)
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            keys[2 * q] = kp[q] << 16;
+            keys[2 * q + 1] = kp[q] & 0xFFFF0000u;
+          }
+          Io::unpack(ws, xs);
+        } else {
+          Io::unpack(ws, xs);
+#pragma unroll
+          for (int j = 0; j < VEC; ++j) keys[j] = Io::KMASK & fkey_raw(xs[j]);
         }
-        if (!any) continue;  // no key of these 8 reaches the bound (the common case)
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          keys[2 * q] = kp[q] << 16;
-          keys[2 * q + 1] = kp[q] & 0xFFFF0000u;
-        }
-        Io::unpack(ws, xs);
-      } else {
-        Io::unpack(ws, xs);
-#pragma unroll
-        for (int j = 0; j < VEC; ++j) keys[j] = Io::KMASK & fkey_raw(xs[j]);
+        for (int j = 0; j < VEC; ++j)
+          classify<T>(keys[j], xs[j], i * VEC + j, bin, zt, lse_s, lse_t, L_S, P_S, buf, &s_ncand);
       }
-#pragma unroll
-      for (int j = 0; j < VEC; ++j)
-        classify<T>(thr, keys[j], xs[j], i * VEC + j, tau, bin, zt, lse_s, lse_t, L_S, P_S, buf, &s_ncand);
-    }
-    for (int v = nvec * VEC + tid; v < V; v += kTkThreads) {
-      const float x = Io::one(zs, v);
-      classify<T>(thr, Io::KMASK & fkey_raw(x), x, v, tau, bin, zt, lse_s, lse_t, L_S, P_S, buf, &s_ncand);
+      for (int v = nvec * VEC + tid; v < V; v += kTkThreads) {
+        const float x = Io::one(zs, v);
+        classify<T>(Io::KMASK & fkey_raw(x), x, v, bin, zt, lse_s, lse_t, L_S, P_S, buf, &s_ncand);
+      }
     }
     __syncthreads();
     const int nc = s_ncand;

@@ -184,6 +184,11 @@ _ZERO_MIXES = [
     (9000, [0.55, 0.2, 0.2, 0.01, 0.03, 0.005, 0.005], 250),
     # k <= 256 with ~5570 logits at or above the bound (exact path from the top)
     (9000, [0.35, 0.3, 0.3, 0.01, 0.03, 0.005, 0.005], 250),
+    # small k: the bound comes from the first slice of the row only, the rest
+    # is listed as it streams (~3650 candidates)
+    (9000, [0.556, 0.2, 0.2, 0.002, 0.038, 0.001, 0.003], 90),
+    # the same with ~4570 logits at or above the bound (exact path from the top)
+    (9000, [0.456, 0.25, 0.25, 0.002, 0.036, 0.001, 0.005], 110),
 ]
 
 
