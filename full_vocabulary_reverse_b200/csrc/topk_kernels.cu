@@ -20,7 +20,7 @@
 //   stream once for both log-sum-exps, two 16-byte vectors of each per step.
 //   After a first slice of the row, the k-th largest of the 256 threads'
 //   running maxima, tau, bounds the k-th largest logit from below (k distinct
-//   logits reach it).  The slice is read a second time (from L2) and the rest
+//   logits reach it).  The slice is read a second time and the rest
 //   of the row as it streams, listing the logits whose keys reach tau
 //   (key, token id) in shared memory.  The slice is sized for ~256 entries
 //   on i.i.d. logits.
@@ -60,8 +60,8 @@ __device__ __forceinline__ uint4 tk_ldg_v4(const void* p) {
   return r;
 }
 
-// The forward's streaming loads bypass L1 (its only reuse, the second read of
-// the first slice, comes from L2).
+// The forward's streaming loads bypass L1 (nothing it streams is reused
+// from L1).
 __device__ __forceinline__ uint4 tk_ldg_stream_v4(const void* p) {
   uint4 r;
   asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
@@ -310,7 +310,8 @@ __global__ void __launch_bounds__(kTkThreads, 6) topk_fwd_kernel(const T* __rest
                                                               int local) {
   using Io = TkIo<T>;
   constexpr int VEC = Io::VEC;
-  // 32 KB: the 4096-bin histogram of pass A, then the candidate list
+  // 32 KB: the 4096-bin histogram of pass A (histogram path) or the sort of
+  // the threads' maxima (threshold path), then the candidate list
   __shared__ unsigned long long buf[kCap];
   int* hist = reinterpret_cast<int*>(buf);
   __shared__ int hist2[256];
@@ -351,8 +352,8 @@ __global__ void __launch_bounds__(kTkThreads, 6) topk_fwd_kernel(const T* __rest
   // or (threshold path) the candidate list
   float m_s = -INFINITY, S_s = 0.f, m_t = -INFINITY, S_t = 0.f;
   // Threshold path: vectors [0, i1) stream by before the bound is known and
-  // are listed by a second read while they are still in L2; the rest of the
-  // row is listed as it streams.  The bound is about the (1 - k/256) quantile
+  // are read a second time to be listed; the rest of the row is listed as it
+  // streams.  The bound is about the (1 - k/256) quantile
   // of a thread's maximum over its e logits of [0, i1), so about
   // V ln(256 / (256 - k)) / e logits reach it: e is sized for kListTarget.
   int i1 = nvec;
