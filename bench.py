@@ -125,7 +125,9 @@ class Problem:
         self.multi = "teacher_idx" in inp
         self.n_teachers = inp["W_t"].shape[0] if self.multi else 1
         self.topk = self.pair and "targets" in inp
-        self.topk_hidden = (not self.pair) and "targets" in inp
+        # per-token student entropy and target log-prob from the same forward
+        self.stats = bool(self.cfg.get("stats"))
+        self.topk_hidden = (not self.pair) and "targets" in inp and not self.stats
         self.k = int(self.cfg.get("k", 0)) if (self.topk or self.topk_hidden) else None
         self.student = inp["student_logits"] if self.pair else inp["h_s"]
         self.H = 0 if self.pair else inp["h_s"].shape[1]
@@ -152,6 +154,9 @@ class Problem:
         self.loss_tok = torch.empty((self.B, self.Sm1), dtype=torch.float32, device=device)
         self.loss = torch.empty(1, dtype=torch.float32, device=device)
         self.saved = torch.empty(7 * self.T, dtype=torch.float32, device=device)
+        if self.stats:
+            self.entropy = torch.empty((self.B, self.Sm1), dtype=torch.float32, device=device)
+            self.target_logprob = torch.empty((self.B, self.Sm1), dtype=torch.float32, device=device)
         if self.pair:
             self.dz = torch.empty_like(self.student)
         else:
@@ -168,7 +173,7 @@ class Problem:
         out = [self.student, self.teacher, self.inp["mask"]]
         if self.multi:
             out.append(self.inp["teacher_idx"])
-        if self.topk or self.topk_hidden:
+        if self.topk or self.topk_hidden or self.stats:
             out.append(self.inp["targets"])
         return out
 
@@ -221,6 +226,13 @@ class Problem:
             rb._check(L.rkl_forward_logits(p(h_s), p(self.inp["W_s"]), p(teacher), self.dt, self.B, self.Sm1, self.H,
                                            self.V, p(self.row_idx), N, self.reduction, p(self.loss_tok), p(self.loss),
                                            p(self.saved), p(self.ws), self.ws.numel(), s))
+        elif self.stats:
+            tg = self.inp["targets"] if extra is None else extra
+            rb._check(L.rkl_forward_hidden_ex(p(h_s), p(teacher), p(self.inp["W_s"]), p(self.W_t), self.dt, self.B,
+                                              self.Sm1, self.H, self.V, p(self.row_idx), N, self.reduction,
+                                              p(self.loss_tok), p(self.loss), p(self.saved), p(tg),
+                                              p(self.entropy), p(self.target_logprob), p(self.ws),
+                                              self.ws.numel(), s))
         else:
             rb._check(L.rkl_forward_hidden(p(h_s), p(teacher), p(self.inp["W_s"]), p(self.W_t), self.dt, self.B,
                                            self.Sm1, self.H, self.V, p(self.row_idx), N, self.reduction,
@@ -369,10 +381,14 @@ def cpu_oracle_sample(inp, reduction, name, rows=CPU_SAMPLE_ROWS, k=None):
             tid = inp["teacher_idx"].cpu().numpy()
             O.forward_multi(h_s, W_s, teacher, W_t, tid, sub, reduction)
             O.backward_multi(h_s, W_s, teacher, W_t, tid, sub, reduction)
-        elif "targets" in inp:
+        elif "targets" in inp and k is not None:
             y = inp["targets"].cpu().numpy()
             O.forward_topk_hidden(h_s, W_s, teacher, W_t, y, k, sub, reduction)
             O.backward_topk_hidden(h_s, W_s, teacher, W_t, y, k, sub, reduction)
+        elif "targets" in inp:  # the loss plus the student's per-token statistics
+            O.forward(h_s, W_s, teacher, W_t, sub, reduction)
+            O.student_stats(h_s, W_s, sub, targets=inp["targets"].cpu().numpy())
+            O.backward(h_s, W_s, teacher, W_t, sub, reduction)
         else:
             O.forward(h_s, W_s, teacher, W_t, sub, reduction)
             O.backward(h_s, W_s, teacher, W_t, sub, reduction)
@@ -533,6 +549,7 @@ def run_gpu(args, rank, world, dist):
                    "trainable_rows": N, "tokens_T": prob.T,
                    "payload": ("logits_pair, top-k estimator k=%d" % prob.k if prob.topk else "logits_pair")
                    if prob.pair else ("hidden, top-k estimator k=%d" % prob.k if prob.topk_hidden else
+                                      "hidden, with student entropy and target log-prob" if prob.stats else
                                       "logits" if prob.logits else
                                                                  ("hidden, %d teachers" % prob.n_teachers
                                                                   if prob.multi else "hidden")),

@@ -29,6 +29,9 @@ Named workloads:
   topk_hidden     qwen_hidden inputs, top-k estimator with k = 64 and a
                   sampled token per position drawn uniformly (the estimator's
                   cost does not depend on how the tokens were drawn).
+  qwen_hidden_stats  qwen_hidden inputs, the forward also returning the
+                  student's per-token entropy and the log-probability of a
+                  target token per position (drawn uniformly).
   multi_teacher   qwen_hidden shapes and mask with two teacher heads
                   W_t[g] = W_s + N(0, 0.004^2) (independent draws), teacher
                   of sequence b = b mod 2; token mean.
@@ -65,6 +68,9 @@ WORKLOADS = {
     "topk_hidden": dict(dtype="bf16", B=4, Sm1=2048, H=2048, V=151936, payload="hidden",
                         reduction=REDUCE_TOKEN_MEAN, mask="prefix", weights="perturbed", seed=1236,
                         targets="uniform", k=64),
+    "qwen_hidden_stats": dict(dtype="bf16", B=4, Sm1=2048, H=2048, V=151936, payload="hidden",
+                              reduction=REDUCE_TOKEN_MEAN, mask="prefix", weights="perturbed", seed=1236,
+                              targets="uniform", stats=True),
     "multi_teacher": dict(dtype="bf16", B=4, Sm1=2048, H=2048, V=151936, payload="hidden_multi",
                           reduction=REDUCE_TOKEN_MEAN, mask="prefix", weights="perturbed", seed=1241,
                           mask_seed=1236, n_teachers=2, teacher_assign="sequence"),
