@@ -107,6 +107,26 @@ class ClockSampler:
                 "reasons": sorted(self.reasons), "samples": len(self.samples)}
 
 
+PATHS = ("hidden", "stats", "topk_hidden", "multi", "logits", "pair", "topk_pair")
+
+
+def path_of(cfg):
+    """The entry points a workload's step goes through, from its config:
+    hidden (rkl_forward_hidden), stats (rkl_forward_hidden_ex with targets),
+    topk_hidden, multi (a teacher per row), logits (shipped teacher logits),
+    pair (both sides as logits) or topk_pair."""
+    payload = cfg["payload"]
+    if payload == "logits_pair":
+        return "topk_pair" if cfg.get("k") is not None else "pair"
+    if payload == "logits":
+        return "logits"
+    if payload == "hidden_multi":
+        return "multi"
+    if cfg.get("k") is not None:
+        return "topk_hidden"
+    return "stats" if cfg.get("stats") else "hidden"
+
+
 class Problem:
     """One batch of a workload, resident on the device, driven through the C ABI."""
 
@@ -120,14 +140,15 @@ class Problem:
         self.dev = device
         self.B, self.Sm1 = inp["mask"].shape
         self.T = self.B * self.Sm1
-        self.pair = "student_logits" in inp
-        self.logits = "teacher_logits" in inp and not self.pair
-        self.multi = "teacher_idx" in inp
+        path = path_of(self.cfg)
+        self.pair = path in ("pair", "topk_pair")
+        self.logits = path == "logits"
+        self.multi = path == "multi"
         self.n_teachers = inp["W_t"].shape[0] if self.multi else 1
-        self.topk = self.pair and "targets" in inp
+        self.topk = path == "topk_pair"
         # per-token student entropy and target log-prob from the same forward
-        self.stats = bool(self.cfg.get("stats"))
-        self.topk_hidden = (not self.pair) and "targets" in inp and not self.stats
+        self.stats = path == "stats"
+        self.topk_hidden = path == "topk_hidden"
         self.k = int(self.cfg.get("k", 0)) if (self.topk or self.topk_hidden) else None
         self.student = inp["student_logits"] if self.pair else inp["h_s"]
         self.H = 0 if self.pair else inp["h_s"].shape[1]
@@ -359,10 +380,11 @@ def cpu_oracle_sample(inp, reduction, name, rows=CPU_SAMPLE_ROWS, k=None):
     sub[flat] = 1
     sub = sub.reshape(mask.shape)
     f64 = lambda t: None if t is None else t.float().cpu().numpy()  # noqa: E731
-    if "student_logits" in inp:
+    path = path_of(WORKLOADS[name])
+    if path in ("pair", "topk_pair"):
         zs, zt = f64(inp["student_logits"]), f64(inp["teacher_logits"])
         t0 = time.perf_counter()
-        if "targets" in inp:
+        if path == "topk_pair":
             y = inp["targets"].cpu().numpy()
             O.forward_topk_pair(zs, zt, y, k, sub, reduction)
             O.backward_topk_pair(zs, zt, y, k, sub, reduction)
@@ -372,20 +394,20 @@ def cpu_oracle_sample(inp, reduction, name, rows=CPU_SAMPLE_ROWS, k=None):
         dt = time.perf_counter() - t0
     else:
         h_s, W_s = f64(inp["h_s"]), f64(inp["W_s"])
-        if "teacher_logits" in inp:
+        if path == "logits":
             teacher, W_t = f64(inp["teacher_logits"]), None
         else:
             teacher, W_t = f64(inp["h_t"]), f64(inp["W_t"])
         t0 = time.perf_counter()
-        if "teacher_idx" in inp:
+        if path == "multi":
             tid = inp["teacher_idx"].cpu().numpy()
             O.forward_multi(h_s, W_s, teacher, W_t, tid, sub, reduction)
             O.backward_multi(h_s, W_s, teacher, W_t, tid, sub, reduction)
-        elif "targets" in inp and k is not None:
+        elif path == "topk_hidden":
             y = inp["targets"].cpu().numpy()
             O.forward_topk_hidden(h_s, W_s, teacher, W_t, y, k, sub, reduction)
             O.backward_topk_hidden(h_s, W_s, teacher, W_t, y, k, sub, reduction)
-        elif "targets" in inp:  # the loss plus the student's per-token statistics
+        elif path == "stats":  # the loss plus the student's per-token statistics
             O.forward(h_s, W_s, teacher, W_t, sub, reduction)
             O.student_stats(h_s, W_s, sub, targets=inp["targets"].cpu().numpy())
             O.backward(h_s, W_s, teacher, W_t, sub, reduction)

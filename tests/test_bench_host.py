@@ -38,3 +38,15 @@ def test_traffic_withheld_when_sources_change(monkeypatch):
     assert bench.traffic_for(kernel, workload) == d["kernels"][key]["dram_bytes_per_launch"]
     monkeypatch.setattr(bench, "source_sha", lambda g: "changed" if g == group else d["source_sha"][g])
     assert bench.traffic_for(kernel, workload) is None
+
+
+def test_every_workload_takes_one_path():
+    expected = {"tiny_fp32": "hidden", "qwen_hidden": "hidden", "self_distill": "hidden", "long_prompt": "hidden",
+                "teacher_logits": "logits", "logits_pair": "pair", "logits_pair_topk": "topk_pair",
+                "topk_hidden": "topk_hidden", "multi_teacher": "multi", "qwen_hidden_stats": "stats"}
+    assert set(expected) == set(bench.WORKLOADS)
+    for name, cfg in bench.WORKLOADS.items():
+        path = bench.path_of(cfg)
+        assert path in bench.PATHS and path == expected[name], (name, path)
+        # sampled tokens are drawn exactly for the paths that read them
+        assert (cfg.get("targets") is not None) == (path in ("topk_pair", "topk_hidden", "stats")), name
