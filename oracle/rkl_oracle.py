@@ -214,6 +214,38 @@ def backward(h_s, W_s, teacher, W_t, mask, reduction, grad_loss=1.0, grad_tok=No
     return dH, dW
 
 
+def backward_dw_rows(h_s, W_s, teacher, W_t, mask, reduction, vocab_ids, grad_loss=1.0, grad_tok=None):
+    """Selected rows dW_s[vocab_ids] of the gradient that `backward` returns.
+
+    Same definition as `backward` (dz = g p_s (w - L) over every trainable
+    row, each row's log-softmaxes taken over the whole vocabulary), with the
+    product dz^T h_s[rows] formed only for the requested vocabulary columns
+    of dz.  Used where the full [V, H] float64 gradient is too large to
+    keep, e.g. to check single vocabulary rows of a full-size problem.
+    Returns [len(vocab_ids), H] float64.
+    """
+    mask = np.asarray(mask)
+    B, Sm1 = mask.shape
+    row_idx, N = compact_rows(mask)
+    W_s64 = _f64(W_s)
+    W_t64 = None if W_t is None else _f64(W_t)
+    vocab_ids = np.asarray(vocab_ids, dtype=np.int64)
+    H = np.asarray(h_s).shape[1]
+    g = row_weights(row_idx, B, Sm1, reduction, grad_loss, grad_tok)
+    out = np.zeros((vocab_ids.shape[0], H))
+    for c0 in range(0, N, _ROW_CHUNK):
+        rows = row_idx[c0:c0 + _ROW_CHUNK]
+        z_s, z_t = _student_teacher_logits(rows, h_s, W_s64, teacher, W_t64)
+        lp_s = log_softmax(z_s)
+        lp_t = log_softmax(z_t)
+        p_s = np.exp(lp_s)
+        w = lp_s - lp_t
+        L = np.sum(p_s * w, axis=1)
+        dz_sel = g[c0:c0 + len(rows), None] * p_s[:, vocab_ids] * (w[:, vocab_ids] - L[:, None])
+        out += dz_sel.T @ _f64(h_s[rows])
+    return out
+
+
 def dz_rows(z_s, z_t, g):
     """dLoss/dz_s for given logit rows and row weights (for small pins)."""
     lp_s = log_softmax(_f64(z_s))
@@ -508,6 +540,55 @@ def backward_topk_hidden(h_s, W_s, h_t, W_t, targets, k, mask, reduction, grad_l
     for c0 in range(0, N, _ROW_CHUNK):
         rows = row_idx[c0:c0 + _ROW_CHUNK]
         z_s, z_t = _student_teacher_logits(rows, h_s, W_s64, h_t, W_t64)
+        _, dz = topk_rows(z_s, z_t, yflat[rows], k, g[c0:c0 + len(rows)])
+        dH[rows] = dz @ W_s64
+        dW += dz.T @ _f64(h_s[rows])
+    return dH, dW
+
+
+# ---------------------------------------------------------------------------
+# Top-k estimator on the logits payload.  NeMo RL PR #3978, description (the
+# exact objective is the K = V limit of top-k MOPD) and payload bullet 2 (the
+# teacher ships its full-vocabulary logits).  The student's logits come from
+# its own hidden states and LM head, z_s = h_s W_s^T; the teacher's logits
+# are the shipped [T, V] rows.  Same estimator as the other two forms
+# (`topk_rows`), same chain rule back to h_s and W_s.
+# ---------------------------------------------------------------------------
+
+def forward_topk_logits(h_s, W_s, teacher_logits, targets, k, mask, reduction):
+    """Top-k estimate with z_s = h_s W_s^T and shipped teacher logits
+    [T, V]; targets [B, S-1] are the sampled tokens."""
+    mask = np.asarray(mask)
+    B, Sm1 = mask.shape
+    row_idx, N = compact_rows(mask)
+    W_s64 = _f64(W_s)
+    yflat = np.asarray(targets).reshape(-1)
+    L = np.zeros(N)
+    for c0 in range(0, N, _ROW_CHUNK):
+        rows = row_idx[c0:c0 + _ROW_CHUNK]
+        z_s, z_t = _student_teacher_logits(rows, h_s, W_s64, teacher_logits, None)
+        L[c0:c0 + len(rows)], _ = topk_rows(z_s, z_t, yflat[rows], k)
+    loss_tok = np.zeros(B * Sm1)
+    loss_tok[row_idx] = L
+    loss = reduce_loss(L, row_idx, B, Sm1, reduction)
+    return {"loss_tok": loss_tok.reshape(B, Sm1), "loss": loss, "L": L, "row_idx": row_idx, "N": N}
+
+
+def backward_topk_logits(h_s, W_s, teacher_logits, targets, k, mask, reduction, grad_loss=1.0, grad_tok=None):
+    """(dH_s [T, H], dW_s [V, H]) of the top-k estimate on the logits
+    payload: its z_s-gradient (`topk_rows`) through z_s = h_s W_s^T."""
+    mask = np.asarray(mask)
+    B, Sm1 = mask.shape
+    row_idx, N = compact_rows(mask)
+    W_s64 = _f64(W_s)
+    g = row_weights(row_idx, B, Sm1, reduction, grad_loss, grad_tok)
+    yflat = np.asarray(targets).reshape(-1)
+    T, H = np.asarray(h_s).shape
+    dH = np.zeros((T, H))
+    dW = np.zeros(W_s64.shape)
+    for c0 in range(0, N, _ROW_CHUNK):
+        rows = row_idx[c0:c0 + _ROW_CHUNK]
+        z_s, z_t = _student_teacher_logits(rows, h_s, W_s64, teacher_logits, None)
         _, dz = topk_rows(z_s, z_t, yflat[rows], k, g[c0:c0 + len(rows)])
         dH[rows] = dz @ W_s64
         dW += dz.T @ _f64(h_s[rows])

@@ -519,3 +519,82 @@ def topk_hidden_finite_differences(O, rs):
             num_W[i, j] = (f(h_s, wp) - f(h_s, wm)) / (2 * eps)
     return max(float(np.max(np.abs(dH - num_H))) / float(np.max(np.abs(num_H))),
                float(np.max(np.abs(dW - num_W))) / float(np.max(np.abs(num_W))))
+
+
+def dw_rows_vs_backward(O, rs):
+    """The selected-vocabulary-rows gradient equals those rows of the full
+    dW_s of `backward` (itself pinned by finite differences), on both
+    payloads, both reductions and with a per-token upstream gradient, for
+    sorted, unsorted and repeated vocabulary ids."""
+    worst = 0.0
+    for payload in ("hidden", "logits"):
+        for red in (1, 2):
+            h_s, W_s, teacher, W_t, mask = rand_problem(rs, B=3, Sm1=5, H=6, V=19, payload=payload)
+            gt = rs.normal(size=mask.shape)
+            ids = np.array([0, 18, 7, 7, 3, 12])
+            _, dW = O.backward(h_s, W_s, teacher, W_t, mask, red, grad_loss=0.8, grad_tok=gt)
+            sel = O.backward_dw_rows(h_s, W_s, teacher, W_t, mask, red, ids, grad_loss=0.8, grad_tok=gt)
+            worst = max(worst, float(np.max(np.abs(sel - dW[ids]))) / float(np.max(np.abs(dW))))
+    return worst
+
+
+def topk_logits_chain_rule(O, rs):
+    """The logits-payload top-k estimate equals the logits-pair one on
+    z_s = h_s W_s^T and the shipped teacher rows, and its gradients are
+    dz W_s and dz^T h_s (chain rule)."""
+    h_s, W_s, teacher, _, mask = rand_problem(rs, B=2, Sm1=4, H=3, V=11, payload="logits")
+    y = rs.randint(0, 11, size=mask.shape)
+    z_s = h_s @ W_s.T
+    worst = 0.0
+    for k in (0, 3, 11):
+        a = O.forward_topk_logits(h_s, W_s, teacher, y, k, mask, 2)
+        b = O.forward_topk_pair(z_s, teacher, y, k, mask, 2)
+        dH, dW = O.backward_topk_logits(h_s, W_s, teacher, y, k, mask, 2)
+        dz = O.backward_topk_pair(z_s, teacher, y, k, mask, 2)
+        worst = max(worst, float(np.max(np.abs(a["loss_tok"] - b["loss_tok"]))), abs(a["loss"] - b["loss"]),
+                    float(np.max(np.abs(dH - dz @ W_s))), float(np.max(np.abs(dW - dz.T @ h_s))))
+    return worst
+
+
+def topk_logits_exact_limit(O, rs):
+    """k >= V on the logits payload gives the exact objective of `forward` /
+    `backward` with shipped teacher logits (pinned by scipy and finite
+    differences)."""
+    h_s, W_s, teacher, _, mask = rand_problem(rs, B=2, Sm1=5, H=4, V=13, payload="logits")
+    y = rs.randint(0, 13, size=mask.shape)
+    a = O.forward_topk_logits(h_s, W_s, teacher, y, 13, mask, 1)
+    b = O.forward(h_s, W_s, teacher, None, mask, 1)
+    dHa, dWa = O.backward_topk_logits(h_s, W_s, teacher, y, 20, mask, 1)
+    dHb, dWb = O.backward(h_s, W_s, teacher, None, mask, 1)
+    return max(float(np.max(np.abs(a["loss_tok"] - b["loss_tok"]))), abs(a["loss"] - b["loss"]),
+               float(np.max(np.abs(dHa - dHb))), float(np.max(np.abs(dWa - dWb))))
+
+
+def topk_logits_finite_differences(O, rs):
+    """Central differences of the logits-payload top-k objective w.r.t. h_s
+    and W_s, with sampled tokens inside the support and a support that does
+    not move under the perturbation."""
+    H, V, k = 3, 9, 4
+    h_s = rs.normal(size=(3, H))
+    W_s = rs.normal(size=(V, H)) * 2
+    zt = rs.normal(size=(3, V)) * 2
+    mask = np.ones((1, 3), np.uint8)
+    S = O.topk_support(h_s @ W_s.T, k)
+    y = np.array([[int(np.flatnonzero(S[i])[-1]) for i in range(3)]])
+    f = lambda hs, ws: O.forward_topk_logits(hs, ws, zt, y, k, mask, 1)["loss"]  # noqa: E731
+    dH, dW = O.backward_topk_logits(h_s, W_s, zt, y, k, mask, 1)
+    eps = 1e-6
+    num_H = np.zeros_like(h_s)
+    for i in range(h_s.shape[0]):
+        for j in range(H):
+            hp = h_s.copy(); hp[i, j] += eps
+            hm = h_s.copy(); hm[i, j] -= eps
+            num_H[i, j] = (f(hp, W_s) - f(hm, W_s)) / (2 * eps)
+    num_W = np.zeros_like(W_s)
+    for i in range(V):
+        for j in range(H):
+            wp = W_s.copy(); wp[i, j] += eps
+            wm = W_s.copy(); wm[i, j] -= eps
+            num_W[i, j] = (f(h_s, wp) - f(h_s, wm)) / (2 * eps)
+    return max(float(np.max(np.abs(dH - num_H))) / float(np.max(np.abs(num_H))),
+               float(np.max(np.abs(dW - num_W))) / float(np.max(np.abs(num_W))))

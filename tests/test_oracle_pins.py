@@ -378,3 +378,53 @@ def test_topk_hidden_chain_rule(rs):
 
 def test_topk_hidden_finite_differences(rs):
     assert pins.topk_hidden_finite_differences(O, rs) < 1e-6
+
+
+# ------------------------------------------------------------ selected dW rows
+
+def test_backward_dw_rows_equal_full_backward(rs):
+    assert pins.dw_rows_vs_backward(O, rs) < 1e-12
+
+
+@pytest.mark.parametrize("old,new", [
+    # dz columns taken from the wrong vocabulary ids
+    ("p_s[:, vocab_ids] * (w[:, vocab_ids] - L[:, None])", "p_s[:, vocab_ids] * (w[:, vocab_ids - 1] - L[:, None])"),
+    # the -L term dropped in the selected columns
+    ("p_s[:, vocab_ids] * (w[:, vocab_ids] - L[:, None])", "p_s[:, vocab_ids] * (w[:, vocab_ids])"),
+])
+def test_dw_rows_pin_catches_planted_mistakes(old, new):
+    M = _mutant(old, new)
+    assert pins.dw_rows_vs_backward(M, np.random.RandomState(3)) > 1e-6
+
+
+# ------------------------------------------------------------ top-k on the logits payload
+
+def test_topk_logits_chain_rule(rs):
+    assert pins.topk_logits_chain_rule(O, rs) < 1e-12
+
+
+def test_topk_logits_exact_limit(rs):
+    assert pins.topk_logits_exact_limit(O, rs) < 1e-12
+
+
+def test_topk_logits_finite_differences(rs):
+    assert pins.topk_logits_finite_differences(O, rs) < 1e-6
+
+
+@pytest.mark.parametrize("old,new", [
+    # the student's logits taken for the teacher's as well
+    ("        z_s, z_t = _student_teacher_logits(rows, h_s, W_s64, teacher_logits, None)\n"
+     "        L[c0:c0 + len(rows)], _ = topk_rows(z_s, z_t, yflat[rows], k)",
+     "        z_s, z_t = _student_teacher_logits(rows, h_s, W_s64, teacher_logits, None)\n"
+     "        L[c0:c0 + len(rows)], _ = topk_rows(z_s, z_s, yflat[rows], k)"),
+    # dW from the teacher's logits instead of the student's hidden rows
+    ("        _, dz = topk_rows(z_s, z_t, yflat[rows], k, g[c0:c0 + len(rows)])\n"
+     "        dH[rows] = dz @ W_s64\n        dW += dz.T @ _f64(h_s[rows])\n    return dH, dW\n",
+     "        _, dz = topk_rows(z_s, z_t, yflat[rows], k, g[c0:c0 + len(rows)])\n"
+     "        dH[rows] = dz @ W_s64\n        dW += dz.T @ _f64(h_s[rows][::-1])\n    return dH, dW\n"),
+])
+def test_topk_logits_pins_catch_planted_mistakes(old, new):
+    M = _mutant(old, new)
+    rs = np.random.RandomState(17)
+    assert (pins.topk_logits_chain_rule(M, rs) > 1e-6 or pins.topk_logits_exact_limit(M, rs) > 1e-6
+            or pins.topk_logits_finite_differences(M, rs) > 1e-4)
