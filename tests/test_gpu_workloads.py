@@ -20,7 +20,11 @@ from tests.gpu_cases import GRAD_RTOL, TOK_ATOL, TOK_RTOL, to_np
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 
-SAMPLE = 12
+SAMPLE = 24
+
+# vocabulary rows of dW_s at the edges of the three backward chunks of V = 151936
+# (50688 columns each), of 256-row gradient tiles, and the ragged last tile
+VOCAB_EDGES = np.array([0, 1, 255, 256, 50687, 50688, 101375, 101376, 151807, 151808, 151935])
 
 
 def _run(inp, reduction, mask=None, grad_tok=None, grad_loss=1.0):
@@ -83,12 +87,19 @@ def _row_weights(out, inp, reduction, rows):
     return np.array([1.0 / (b_eff * counts[r // Sm1]) for r in rows])
 
 
+def _tile_edges(n):
+    """Compact-row indices at the edges of 128-row CTA tiles and 256-row pair
+    tiles, and the last row."""
+    e = [0, 127, 128, 255, 256, 511, 512, n - 1]
+    return np.array([k for k in e if 0 <= k < n])
+
+
 def _check_sampled(inp, out, reduction, seed):
     rs = np.random.RandomState(seed)
     ridx = out["row_idx"].cpu().numpy()
     pick = np.sort(rs.choice(len(ridx), size=min(SAMPLE, len(ridx)), replace=False))
-    # always include the first and last trainable rows (tile edges)
-    pick = np.unique(np.concatenate([[0, len(ridx) - 1], pick]))
+    # always include the rows at tile edges and the last trainable row
+    pick = np.unique(np.concatenate([_tile_edges(len(ridx)), pick]))
     rows = ridx[pick]
     fw, dH_ref = _oracle_rows(inp, rows, _row_weights(out, inp, reduction, rows))
     g_tok = to_np(out["loss_tok"].reshape(-1)[torch.as_tensor(rows, device=out["loss_tok"].device)])
@@ -100,6 +111,28 @@ def _check_sampled(inp, out, reduction, seed):
     g_dH = to_np(out["dH"][torch.as_tensor(rows, device=out["dH"].device)])
     r_dH = np.stack([dH_ref[int(r)] for r in rows])
     assert np.max(np.abs(g_dH - r_dH)) / np.max(np.abs(r_dH)) < GRAD_RTOL
+
+
+def _check_dw_rows(inp, out, reduction, seed, grad_tok=None):
+    """Sampled vocabulary rows of the full dW_s against the oracle, whose dz
+    comes from its own forward statistics over every trainable row."""
+    V = inp["W_s"].shape[0]
+    rs = np.random.RandomState(seed)
+    ids = np.unique(np.concatenate([VOCAB_EDGES[VOCAB_EDGES < V], rs.choice(V, 8, replace=False)]))
+    f = lambda t: None if t is None else t.float().cpu().numpy()  # noqa: E731
+    if "teacher_logits" in inp:
+        teacher, W_t = f(inp["teacher_logits"]), None
+    else:
+        teacher, W_t = f(inp["h_t"]), f(inp["W_t"])
+    ref = O.backward_dw_rows(f(inp["h_s"]), f(inp["W_s"]), teacher, W_t, inp["mask"].cpu().numpy(), reduction, ids,
+                             grad_tok=None if grad_tok is None else grad_tok.cpu().numpy())
+    got = to_np(out["dW"][torch.as_tensor(ids, device=out["dW"].device)])
+    err = np.max(np.abs(got - ref)) / np.max(np.abs(ref))
+    assert err < GRAD_RTOL, (err, ids)
+    # and row by row, each on its own scale
+    for i, v in enumerate(ids):
+        e = np.max(np.abs(got[i] - ref[i])) / np.max(np.abs(ref[i]))
+        assert e < GRAD_RTOL, (int(v), e)
 
 
 def _check_identities(inp, out):
@@ -125,6 +158,7 @@ def test_qwen_hidden_full_size():
     assert out["N"] == int(inp["mask"].sum())
     _check_sampled(inp, out, red, seed=1)
     _check_identities(inp, out)
+    _check_dw_rows(inp, out, red, seed=11)
     lt = out["loss_tok"].reshape(-1)
     off = ~inp["mask"].reshape(-1).bool()
     assert float(torch.count_nonzero(lt[off])) == 0
@@ -147,6 +181,7 @@ def test_teacher_logits_full_size():
     assert out["N"] == 8192
     _check_sampled(inp, out, red, seed=2)
     _check_identities(inp, out)
+    _check_dw_rows(inp, out, red, seed=12)
 
 
 def test_long_prompt_compact_equals_full():
@@ -165,6 +200,8 @@ def test_long_prompt_compact_equals_full():
     rel = ((comp["dW"] - full["dW"]).abs().max() / full["dW"].abs().max()).item()
     assert rel < 1e-3
     del full
+    # sampled vocabulary rows of dW_s (H = 4096: eight 512-column blocks)
+    _check_dw_rows(inp, comp, 0, seed=13, grad_tok=torch.full(mask.shape, 1.0 / 2048, dtype=torch.float64))
     # sampled rows against the oracle (row weights 1/2048 on the compact run)
     out = dict(comp)
     rs = np.random.RandomState(5)
