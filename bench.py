@@ -192,6 +192,12 @@ class Problem:
     def _p(self, t):
         return None if t is None else ctypes.c_void_p(t.data_ptr())
 
+    def trainable_rows(self):
+        """N of the last step's batch (a host read of the device count; only
+        outside the timed regions)."""
+        torch.cuda.synchronize()
+        return self.N if self.multi else int(self.n_dev.item())
+
     def inputs(self):
         """The per-batch input tensors (what a data loader would deliver each step)."""
         out = [self.student, self.teacher, self.inp["mask"]]
@@ -202,7 +208,10 @@ class Problem:
         return out
 
     def step(self, h_s=None, teacher=None, mask=None, extra=None):
-        """S1..S7 for one batch; returns N.  Inputs default to the resident ones."""
+        """S1..S7 for one batch.  Inputs default to the resident ones.  The
+        trainable-row count stays on the device (the kernels read it), so the
+        step is enqueued without any host synchronisation; the teacher-per-row
+        path reads N and the per-teacher counts back to plan its row layout."""
         L, p = self.L, self._p
         h_s = self.student if h_s is None else h_s
         teacher = self.teacher if teacher is None else teacher
@@ -212,61 +221,55 @@ class Problem:
             tid = self.inp["teacher_idx"] if extra is None else extra
             return self._step_multi(h_s, teacher, mask, tid, s)
         rb._check(L.rkl_compact_rows(p(mask), self.B, self.Sm1, p(self.row_idx), p(self.n_dev), s))
-        self.n_host.copy_(self.n_dev, non_blocking=True)
-        torch.cuda.current_stream().synchronize()
-        N = int(self.n_host[0])
+        N, nd = self.T, p(self.n_dev)  # bound and device count
         if self.topk:
             tg = self.inp["targets"] if extra is None else extra
-            rb._check(L.rkl_forward_topk_pair(p(h_s), p(teacher), self.dt, self.B, self.Sm1, self.V, p(self.row_idx), N,
+            rb._check(L.rkl_forward_topk_pair(p(h_s), p(teacher), self.dt, self.B, self.Sm1, self.V, p(self.row_idx), N, nd,
                                               self.k, p(tg), self.reduction, p(self.loss_tok), p(self.loss),
                                               p(self.saved), p(self.ws), self.ws.numel(), s))
             rb._check(L.rkl_backward_topk_pair(p(h_s), p(teacher), self.dt, self.B, self.Sm1, self.V, p(self.row_idx),
-                                               N, p(tg), self.reduction, p(self.saved), p(self.grad_loss), None,
+                                               N, nd, p(tg), self.reduction, p(self.saved), p(self.grad_loss), None,
                                                p(self.dz), p(self.ws), self.ws.numel(), s))
-            self.N = N
-            return N
+            return None
         if self.pair:
             rb._check(L.rkl_forward_logits_pair(p(h_s), p(teacher), self.dt, self.B, self.Sm1, self.V,
-                                                p(self.row_idx), N, self.reduction, p(self.loss_tok), p(self.loss),
+                                                p(self.row_idx), N, nd, self.reduction, p(self.loss_tok), p(self.loss),
                                                 p(self.saved), p(self.ws), self.ws.numel(), s))
             rb._check(L.rkl_backward_logits_pair(p(h_s), p(teacher), self.dt, self.B, self.Sm1, self.V,
-                                                 p(self.row_idx), N, self.reduction, p(self.saved),
+                                                 p(self.row_idx), N, nd, self.reduction, p(self.saved),
                                                  p(self.grad_loss), None, p(self.dz), p(self.ws), self.ws.numel(), s))
-            self.N = N
-            return N
+            return None
         if self.topk_hidden:
             tg = self.inp["targets"] if extra is None else extra
             rb._check(L.rkl_forward_topk_hidden(p(h_s), p(teacher), p(self.inp["W_s"]), p(self.W_t), self.dt, self.B,
-                                                self.Sm1, self.H, self.V, p(self.row_idx), N, self.k, p(tg),
+                                                self.Sm1, self.H, self.V, p(self.row_idx), N, nd, self.k, p(tg),
                                                 self.reduction, p(self.loss_tok), p(self.loss), p(self.saved),
                                                 p(self.ws), self.ws.numel(), s))
             rb._check(L.rkl_backward_topk_hidden(p(h_s), p(teacher), p(self.inp["W_s"]), p(self.W_t), self.dt,
-                                                 self.B, self.Sm1, self.H, self.V, p(self.row_idx), N, p(tg),
+                                                 self.B, self.Sm1, self.H, self.V, p(self.row_idx), N, nd, p(tg),
                                                  self.reduction, p(self.saved), p(self.grad_loss), None, p(self.dH),
                                                  p(self.dW), p(self.ws), self.ws.numel(), s))
-            self.N = N
-            return N
+            return None
         if self.logits:
             rb._check(L.rkl_forward_logits(p(h_s), p(self.inp["W_s"]), p(teacher), self.dt, self.B, self.Sm1, self.H,
-                                           self.V, p(self.row_idx), N, self.reduction, p(self.loss_tok), p(self.loss),
+                                           self.V, p(self.row_idx), N, nd, self.reduction, p(self.loss_tok), p(self.loss),
                                            p(self.saved), p(self.ws), self.ws.numel(), s))
         elif self.stats:
             tg = self.inp["targets"] if extra is None else extra
             rb._check(L.rkl_forward_hidden_ex(p(h_s), p(teacher), p(self.inp["W_s"]), p(self.W_t), self.dt, self.B,
-                                              self.Sm1, self.H, self.V, p(self.row_idx), N, self.reduction,
+                                              self.Sm1, self.H, self.V, p(self.row_idx), N, nd, self.reduction,
                                               p(self.loss_tok), p(self.loss), p(self.saved), p(tg),
                                               p(self.entropy), p(self.target_logprob), p(self.ws),
                                               self.ws.numel(), s))
         else:
             rb._check(L.rkl_forward_hidden(p(h_s), p(teacher), p(self.inp["W_s"]), p(self.W_t), self.dt, self.B,
-                                           self.Sm1, self.H, self.V, p(self.row_idx), N, self.reduction,
+                                           self.Sm1, self.H, self.V, p(self.row_idx), N, nd, self.reduction,
                                            p(self.loss_tok), p(self.loss), p(self.saved), p(self.ws),
                                            self.ws.numel(), s))
         rb._check(L.rkl_backward(self.payload, p(h_s), p(teacher), p(self.inp["W_s"]), p(self.W_t), self.dt, self.B,
-                                 self.Sm1, self.H, self.V, p(self.row_idx), N, self.reduction, p(self.saved),
+                                 self.Sm1, self.H, self.V, p(self.row_idx), N, nd, self.reduction, p(self.saved),
                                  p(self.grad_loss), None, p(self.dH), p(self.dW), p(self.ws), self.ws.numel(), s))
-        self.N = N
-        return N
+        return None
 
     def _step_multi(self, h_s, h_t, mask, tid, s):
         L, p = self.L, self._p
@@ -478,8 +481,7 @@ def run_gpu(args, rank, world, dist):
 
     for _ in range(args.warmup):
         prob.step()
-    torch.cuda.synchronize()
-    N = prob.N
+    N = prob.trainable_rows()
 
     # ---- device-timed region: inputs resident in HBM, no per-launch
     # instrumentation (the headline value)
@@ -563,11 +565,11 @@ def run_gpu(args, rank, world, dist):
     ms_e2e, _ = reduce_over_ranks(f0.elapsed_time(f1), 0, dist, dev)
     e2e_value = n_tot / (ms_e2e / 1000.0)
     h2d = sum(t.numel() * t.element_size() for t in pins)
-    # loss scalar + per-token losses [B, S-1] + N (the compaction count read
-    # back to size the launches) + the per-teacher row counts of the
-    # teacher-per-row mode.  The gradients stay on the device, where the
-    # optimizer step would consume them.
-    d2h = 4 + 4 * prob.T + 4 + (4 * (prob.n_teachers + 1) if prob.multi else 0)
+    # loss scalar + per-token losses [B, S-1], plus N and the per-teacher row
+    # counts in the teacher-per-row mode (read back to plan its row layout;
+    # the other paths keep N on the device).  The gradients stay on the
+    # device, where the optimizer step would consume them.
+    d2h = 4 + 4 * prob.T + (4 * (prob.n_teachers + 2) if prob.multi else 0)
 
     if rank != 0:
         return
@@ -636,7 +638,8 @@ def run_gpu(args, rank, world, dist):
                         "share": v["ms"] / total_ms} for k, v in sorted(prof.items(), key=lambda x: -x[1]["ms"])},
         "clocks": csum,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "read_back": "loss, loss_tok [B, S-1], N; gradients stay on the device for the optimizer"},
+                "read_back": "loss, loss_tok [B, S-1]%s; gradients stay on the device for the optimizer" % (
+                    ", N and per-teacher counts" if prob.multi else "")},
         "gpu_launches": int(launches),
     }
     if world == 1 and not args.no_cpu_baseline:

@@ -14,7 +14,8 @@ import os
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "librkl.so")
+# RKL_LIBRARY=debug selects the RKL_DEBUG build (device bounds checks)
+LIB_PATH = os.path.join(_HERE, "librkl_debug.so" if os.environ.get("RKL_LIBRARY") == "debug" else "librkl.so")
 
 REDUCE_NONE = 0
 REDUCE_TOKEN_MEAN = 1
@@ -48,20 +49,20 @@ _SIGS = {
     "rkl_last_error": ([], ctypes.c_char_p),
     "rkl_workspace_size": ([_i32, _i32, _i64, _i64, _i64, _i64, _i64, ctypes.POINTER(_sz)], _i32),
     "rkl_compact_rows": ([_vp, _i64, _i64, _vp, _vp, _vp], _i32),
-    "rkl_forward_hidden": ([_vp, _vp, _vp, _vp, _i32, _i64, _i64, _i64, _i64, _vp, _i32, _i32,
+    "rkl_forward_hidden": ([_vp, _vp, _vp, _vp, _i32, _i64, _i64, _i64, _i64, _vp, _i32, _vp, _i32,
                             _vp, _vp, _vp, _vp, _sz, _vp], _i32),
-    "rkl_forward_logits": ([_vp, _vp, _vp, _i32, _i64, _i64, _i64, _i64, _vp, _i32, _i32,
+    "rkl_forward_logits": ([_vp, _vp, _vp, _i32, _i64, _i64, _i64, _i64, _vp, _i32, _vp, _i32,
                             _vp, _vp, _vp, _vp, _sz, _vp], _i32),
-    "rkl_backward": ([_i32, _vp, _vp, _vp, _vp, _i32, _i64, _i64, _i64, _i64, _vp, _i32, _i32,
+    "rkl_backward": ([_i32, _vp, _vp, _vp, _vp, _i32, _i64, _i64, _i64, _i64, _vp, _i32, _vp, _i32,
                       _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp], _i32),
-    "rkl_forward_hidden_ex": ([_vp, _vp, _vp, _vp, _i32, _i64, _i64, _i64, _i64, _vp, _i32, _i32,
+    "rkl_forward_hidden_ex": ([_vp, _vp, _vp, _vp, _i32, _i64, _i64, _i64, _i64, _vp, _i32, _vp, _i32,
                                _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp], _i32),
-    "rkl_forward_logits_ex": ([_vp, _vp, _vp, _i32, _i64, _i64, _i64, _i64, _vp, _i32, _i32,
+    "rkl_forward_logits_ex": ([_vp, _vp, _vp, _i32, _i64, _i64, _i64, _i64, _vp, _i32, _vp, _i32,
                                _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp], _i32),
-    "rkl_forward_logits_pair": ([_vp, _vp, _i32, _i64, _i64, _i64, _vp, _i32, _i32, _vp, _vp, _vp, _vp, _sz, _vp],
-                                _i32),
-    "rkl_backward_logits_pair": ([_vp, _vp, _i32, _i64, _i64, _i64, _vp, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _sz,
-                                  _vp], _i32),
+    "rkl_forward_logits_pair": ([_vp, _vp, _i32, _i64, _i64, _i64, _vp, _i32, _vp, _i32, _vp, _vp, _vp, _vp, _sz,
+                                 _vp], _i32),
+    "rkl_backward_logits_pair": ([_vp, _vp, _i32, _i64, _i64, _i64, _vp, _i32, _vp, _i32, _vp, _vp, _vp, _vp, _vp,
+                                  _sz, _vp], _i32),
     "rkl_forward_hidden_noalloc": ([_vp, _vp, _vp, _vp, _i32, _i64, _i64, _i64, _i64, _vp, _i32, _i32,
                                     _vp, _vp, _vp, _vp], _i32),
     "rkl_compact_rows_multi": ([_vp, _vp, _i64, _i64, _i32, _vp, _vp, _vp, _vp], _i32),
@@ -70,14 +71,14 @@ _SIGS = {
                                   _vp, _vp, _vp, _vp, _sz, _vp], _i32),
     "rkl_backward_hidden_multi": ([_vp, _vp, _vp, _vp, _i32, _vp, _vp, _i32, _i64, _i64, _i64, _i64, _vp, _i32, _i32,
                                    _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp], _i32),
-    "rkl_forward_topk_pair": ([_vp, _vp, _i32, _i64, _i64, _i64, _vp, _i32, _i64, _vp, _i32, _vp, _vp, _vp, _vp, _sz,
-                               _vp], _i32),
-    "rkl_backward_topk_pair": ([_vp, _vp, _i32, _i64, _i64, _i64, _vp, _i32, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _sz,
-                                _vp], _i32),
-    "rkl_forward_topk_hidden": ([_vp, _vp, _vp, _vp, _i32, _i64, _i64, _i64, _i64, _vp, _i32, _i64, _vp, _i32, _vp,
-                                 _vp, _vp, _vp, _sz, _vp], _i32),
-    "rkl_backward_topk_hidden": ([_vp, _vp, _vp, _vp, _i32, _i64, _i64, _i64, _i64, _vp, _i32, _vp, _i32, _vp, _vp,
-                                  _vp, _vp, _vp, _vp, _sz, _vp], _i32),
+    "rkl_forward_topk_pair": ([_vp, _vp, _i32, _i64, _i64, _i64, _vp, _i32, _vp, _i64, _vp, _i32, _vp, _vp, _vp, _vp,
+                               _sz, _vp], _i32),
+    "rkl_backward_topk_pair": ([_vp, _vp, _i32, _i64, _i64, _i64, _vp, _i32, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _vp,
+                                _sz, _vp], _i32),
+    "rkl_forward_topk_hidden": ([_vp, _vp, _vp, _vp, _i32, _i64, _i64, _i64, _i64, _vp, _i32, _vp, _i64, _vp, _i32,
+                                 _vp, _vp, _vp, _vp, _sz, _vp], _i32),
+    "rkl_backward_topk_hidden": ([_vp, _vp, _vp, _vp, _i32, _i64, _i64, _i64, _i64, _vp, _i32, _vp, _vp, _i32, _vp,
+                                  _vp, _vp, _vp, _vp, _vp, _sz, _vp], _i32),
     "rkl_device_error": ([ctypes.POINTER(_i32)], _i32),
     "rkl_kernel_count": ([], _i32),
     "rkl_kernel_name": ([_i32], ctypes.c_char_p),
@@ -93,7 +94,8 @@ def lib():
     global _lib
     if _lib is None:
         if not os.path.exists(LIB_PATH):
-            raise RKLError(7, "librkl.so is not built (python -m full_vocabulary_reverse_b200.build)")
+            raise RKLError(7, "%s is not built (python -m full_vocabulary_reverse_b200.build)" %
+                           os.path.basename(LIB_PATH))
         L = ctypes.CDLL(LIB_PATH)
         for name, (args, res) in _SIGS.items():
             fn = getattr(L, name)
@@ -135,8 +137,11 @@ def _workspace(payload, dtype_code, n_max, B, Sm1, H, V, device):
     return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
 
 
-def compact_rows(mask):
-    """S1: (row_idx int32 [B*Sm1] device, N host int)."""
+def compact_rows(mask, on_device=False):
+    """S1: (row_idx int32 [B*Sm1] device, N).  N is a host int (read back
+    with one synchronising copy), or with on_device=True the 1-element int32
+    device tensor the kernels read themselves (no host synchronisation).
+    Every entry point below takes either form of N."""
     B, Sm1 = mask.shape
     mask = mask.contiguous()
     if mask.dtype != torch.uint8:
@@ -144,21 +149,34 @@ def compact_rows(mask):
     row_idx = torch.empty(B * Sm1, dtype=torch.int32, device=mask.device)
     n_dev = torch.empty(1, dtype=torch.int32, device=mask.device)
     _check(lib().rkl_compact_rows(_ptr(mask), B, Sm1, _ptr(row_idx), _ptr(n_dev), _stream(mask.device)))
+    if on_device:
+        return row_idx, n_dev
     return row_idx, int(n_dev.item())
+
+
+def _count(N, B, Sm1):
+    """(N argument, n_dev pointer) of a C call: a host count is exact; a
+    device count passes the capacity B*Sm1 as the bound."""
+    if isinstance(N, torch.Tensor):
+        if N.dtype != torch.int32 or N.numel() != 1 or not N.is_cuda:
+            raise RKLError(2, "a device row count must be a 1-element int32 CUDA tensor")
+        return B * Sm1, _ptr(N)
+    return int(N), None
 
 
 def forward_hidden(h_s, h_t, W_s, W_t, B, Sm1, row_idx, N, reduction, workspace=None):
     """S2-S4 on the hidden payload.  Returns (loss_tok [B,Sm1], loss [1], saved [N,3])."""
+    Nc, nd = _count(N, B, Sm1)
     dev = h_s.device
     T, H = h_s.shape
     V = W_s.shape[0]
     dt = _dtype_code(h_s)
     loss_tok = torch.empty((B, Sm1), dtype=torch.float32, device=dev)
     loss = torch.empty(1, dtype=torch.float32, device=dev)
-    saved = torch.empty((max(N, 1), 3), dtype=torch.float32, device=dev)
-    ws = workspace if workspace is not None else _workspace(PAYLOAD_HIDDEN, dt, max(N, 1), B, Sm1, H, V, dev)
+    saved = torch.empty((max(Nc, 1), 3), dtype=torch.float32, device=dev)
+    ws = workspace if workspace is not None else _workspace(PAYLOAD_HIDDEN, dt, max(Nc, 1), B, Sm1, H, V, dev)
     _check(lib().rkl_forward_hidden(_ptr(h_s), _ptr(h_t), _ptr(W_s), _ptr(W_t), dt, B, Sm1, H, V,
-                                    _ptr(row_idx), N, reduction, _ptr(loss_tok), _ptr(loss), _ptr(saved),
+                                    _ptr(row_idx), Nc, nd, reduction, _ptr(loss_tok), _ptr(loss), _ptr(saved),
                                     _ptr(ws), ws.numel(), _stream(dev)))
     return loss_tok, loss, saved
 
@@ -167,6 +185,7 @@ def forward_with_stats(h_s, teacher, W_s, W_t, B, Sm1, row_idx, N, reduction, ta
     """Forward of the hidden payload (W_t given) or the logits payload (W_t None)
     plus the student's per-token entropy and target log-prob.
     Returns (loss_tok, loss, saved, entropy [B,Sm1], target_logprob [B,Sm1] or None)."""
+    Nc, nd = _count(N, B, Sm1)
     dev = h_s.device
     T, H = h_s.shape
     V = W_s.shape[0]
@@ -174,18 +193,18 @@ def forward_with_stats(h_s, teacher, W_s, W_t, B, Sm1, row_idx, N, reduction, ta
     payload = PAYLOAD_HIDDEN if W_t is not None else PAYLOAD_LOGITS
     loss_tok = torch.empty((B, Sm1), dtype=torch.float32, device=dev)
     loss = torch.empty(1, dtype=torch.float32, device=dev)
-    saved = torch.empty((max(N, 1), 3), dtype=torch.float32, device=dev)
+    saved = torch.empty((max(Nc, 1), 3), dtype=torch.float32, device=dev)
     ent = torch.empty((B, Sm1), dtype=torch.float32, device=dev)
     tlp = torch.empty((B, Sm1), dtype=torch.float32, device=dev) if targets is not None else None
     if targets is not None:
         targets = targets.to(device=dev, dtype=torch.int32).contiguous()
-    ws = workspace if workspace is not None else _workspace(payload, dt, max(N, 1), B, Sm1, H, V, dev)
+    ws = workspace if workspace is not None else _workspace(payload, dt, max(Nc, 1), B, Sm1, H, V, dev)
     if payload == PAYLOAD_HIDDEN:
         st = lib().rkl_forward_hidden_ex(_ptr(h_s), _ptr(teacher), _ptr(W_s), _ptr(W_t), dt, B, Sm1, H, V,
-                                         _ptr(row_idx), N, reduction, _ptr(loss_tok), _ptr(loss), _ptr(saved),
+                                         _ptr(row_idx), Nc, nd, reduction, _ptr(loss_tok), _ptr(loss), _ptr(saved),
                                          _ptr(targets), _ptr(ent), _ptr(tlp), _ptr(ws), ws.numel(), _stream(dev))
     else:
-        st = lib().rkl_forward_logits_ex(_ptr(h_s), _ptr(W_s), _ptr(teacher), dt, B, Sm1, H, V, _ptr(row_idx), N,
+        st = lib().rkl_forward_logits_ex(_ptr(h_s), _ptr(W_s), _ptr(teacher), dt, B, Sm1, H, V, _ptr(row_idx), Nc, nd,
                                          reduction, _ptr(loss_tok), _ptr(loss), _ptr(saved), _ptr(targets),
                                          _ptr(ent), _ptr(tlp), _ptr(ws), ws.numel(), _stream(dev))
     _check(st)
@@ -194,16 +213,17 @@ def forward_with_stats(h_s, teacher, W_s, W_t, B, Sm1, row_idx, N, reduction, ta
 
 def forward_logits(h_s, W_s, teacher_logits, B, Sm1, row_idx, N, reduction, workspace=None):
     """S2-S4 + S8 on the logits payload.  Returns (loss_tok, loss, saved)."""
+    Nc, nd = _count(N, B, Sm1)
     dev = h_s.device
     T, H = h_s.shape
     V = W_s.shape[0]
     dt = _dtype_code(h_s)
     loss_tok = torch.empty((B, Sm1), dtype=torch.float32, device=dev)
     loss = torch.empty(1, dtype=torch.float32, device=dev)
-    saved = torch.empty((max(N, 1), 3), dtype=torch.float32, device=dev)
-    ws = workspace if workspace is not None else _workspace(PAYLOAD_LOGITS, dt, max(N, 1), B, Sm1, H, V, dev)
+    saved = torch.empty((max(Nc, 1), 3), dtype=torch.float32, device=dev)
+    ws = workspace if workspace is not None else _workspace(PAYLOAD_LOGITS, dt, max(Nc, 1), B, Sm1, H, V, dev)
     _check(lib().rkl_forward_logits(_ptr(h_s), _ptr(W_s), _ptr(teacher_logits), dt, B, Sm1, H, V,
-                                    _ptr(row_idx), N, reduction, _ptr(loss_tok), _ptr(loss), _ptr(saved),
+                                    _ptr(row_idx), Nc, nd, reduction, _ptr(loss_tok), _ptr(loss), _ptr(saved),
                                     _ptr(ws), ws.numel(), _stream(dev)))
     return loss_tok, loss, saved
 
@@ -211,6 +231,7 @@ def forward_logits(h_s, W_s, teacher_logits, B, Sm1, row_idx, N, reduction, work
 def backward(payload, h_s, teacher, W_s, W_t, B, Sm1, row_idx, N, reduction, saved,
              grad_loss=None, grad_tok=None, workspace=None, dH_s=None, dW_s=None):
     """S5-S7.  Returns (dH_s [T,H] fp32, dW_s [V,H] fp32)."""
+    Nc, nd = _count(N, B, Sm1)
     dev = h_s.device
     T, H = h_s.shape
     V = W_s.shape[0]
@@ -223,23 +244,24 @@ def backward(payload, h_s, teacher, W_s, W_t, B, Sm1, row_idx, N, reduction, sav
         grad_loss = grad_loss.reshape(1).to(device=dev, dtype=torch.float32).contiguous()
     if grad_tok is not None:
         grad_tok = grad_tok.to(device=dev, dtype=torch.float32).contiguous()
-    ws = workspace if workspace is not None else _workspace(payload, dt, max(N, 1), B, Sm1, H, V, dev)
+    ws = workspace if workspace is not None else _workspace(payload, dt, max(Nc, 1), B, Sm1, H, V, dev)
     _check(lib().rkl_backward(payload, _ptr(h_s), _ptr(teacher), _ptr(W_s), _ptr(W_t), dt, B, Sm1, H, V,
-                              _ptr(row_idx), N, reduction, _ptr(saved), _ptr(grad_loss), _ptr(grad_tok),
+                              _ptr(row_idx), Nc, nd, reduction, _ptr(saved), _ptr(grad_loss), _ptr(grad_tok),
                               _ptr(dH_s), _ptr(dW_s), _ptr(ws), ws.numel(), _stream(dev)))
     return dH_s, dW_s
 
 
 def forward_logits_pair(student_logits, teacher_logits, B, Sm1, row_idx, N, reduction, workspace=None):
     """Both sides as logits.  Returns (loss_tok [B,Sm1], loss [1], saved [N,3])."""
+    Nc, nd = _count(N, B, Sm1)
     dev = student_logits.device
     V = student_logits.shape[1]
     dt = _dtype_code(student_logits)
     loss_tok = torch.empty((B, Sm1), dtype=torch.float32, device=dev)
     loss = torch.empty(1, dtype=torch.float32, device=dev)
-    saved = torch.empty((max(N, 1), 3), dtype=torch.float32, device=dev)
-    ws = workspace if workspace is not None else _workspace(PAYLOAD_LOGITS_PAIR, dt, max(N, 1), B, Sm1, 64, V, dev)
-    _check(lib().rkl_forward_logits_pair(_ptr(student_logits), _ptr(teacher_logits), dt, B, Sm1, V, _ptr(row_idx), N,
+    saved = torch.empty((max(Nc, 1), 3), dtype=torch.float32, device=dev)
+    ws = workspace if workspace is not None else _workspace(PAYLOAD_LOGITS_PAIR, dt, max(Nc, 1), B, Sm1, 64, V, dev)
+    _check(lib().rkl_forward_logits_pair(_ptr(student_logits), _ptr(teacher_logits), dt, B, Sm1, V, _ptr(row_idx), Nc, nd,
                                          reduction, _ptr(loss_tok), _ptr(loss), _ptr(saved), _ptr(ws), ws.numel(),
                                          _stream(dev)))
     return loss_tok, loss, saved
@@ -248,6 +270,7 @@ def forward_logits_pair(student_logits, teacher_logits, B, Sm1, row_idx, N, redu
 def backward_logits_pair(student_logits, teacher_logits, B, Sm1, row_idx, N, reduction, saved, grad_loss=None,
                          grad_tok=None, workspace=None, dz=None):
     """dLoss/dz_s [T, V] in the dtype of the logits."""
+    Nc, nd = _count(N, B, Sm1)
     dev = student_logits.device
     V = student_logits.shape[1]
     dt = _dtype_code(student_logits)
@@ -257,9 +280,9 @@ def backward_logits_pair(student_logits, teacher_logits, B, Sm1, row_idx, N, red
         grad_loss = grad_loss.reshape(1).to(device=dev, dtype=torch.float32).contiguous()
     if grad_tok is not None:
         grad_tok = grad_tok.to(device=dev, dtype=torch.float32).contiguous()
-    ws = workspace if workspace is not None else _workspace(PAYLOAD_LOGITS_PAIR, dt, max(N, 1), B, Sm1, 64, V, dev)
+    ws = workspace if workspace is not None else _workspace(PAYLOAD_LOGITS_PAIR, dt, max(Nc, 1), B, Sm1, 64, V, dev)
     _check(lib().rkl_backward_logits_pair(_ptr(student_logits), _ptr(teacher_logits), dt, B, Sm1, V, _ptr(row_idx),
-                                          N, reduction, _ptr(saved), _ptr(grad_loss), _ptr(grad_tok), _ptr(dz),
+                                          Nc, nd, reduction, _ptr(saved), _ptr(grad_loss), _ptr(grad_tok), _ptr(dz),
                                           _ptr(ws), ws.numel(), _stream(dev)))
     return dz
 
@@ -269,15 +292,16 @@ def backward_logits_pair(student_logits, teacher_logits, B, Sm1, row_idx, N, red
 def forward_topk_pair(student_logits, teacher_logits, targets, k, B, Sm1, row_idx, N, reduction, workspace=None):
     """Top-k estimator with both sides as logits; targets [B, Sm1] are the
     sampled tokens.  Returns (loss_tok [B,Sm1], loss [1], saved [7N])."""
+    Nc, nd = _count(N, B, Sm1)
     dev = student_logits.device
     V = student_logits.shape[1]
     dt = _dtype_code(student_logits)
     tg = targets.to(device=dev, dtype=torch.int32).contiguous()
     loss_tok = torch.empty((B, Sm1), dtype=torch.float32, device=dev)
     loss = torch.empty(1, dtype=torch.float32, device=dev)
-    saved = torch.empty(7 * max(N, 1), dtype=torch.float32, device=dev)
-    ws = workspace if workspace is not None else _workspace(PAYLOAD_LOGITS_PAIR, dt, max(N, 1), B, Sm1, 64, V, dev)
-    _check(lib().rkl_forward_topk_pair(_ptr(student_logits), _ptr(teacher_logits), dt, B, Sm1, V, _ptr(row_idx), N,
+    saved = torch.empty(7 * max(Nc, 1), dtype=torch.float32, device=dev)
+    ws = workspace if workspace is not None else _workspace(PAYLOAD_LOGITS_PAIR, dt, max(Nc, 1), B, Sm1, 64, V, dev)
+    _check(lib().rkl_forward_topk_pair(_ptr(student_logits), _ptr(teacher_logits), dt, B, Sm1, V, _ptr(row_idx), Nc, nd,
                                        int(k), _ptr(tg), reduction, _ptr(loss_tok), _ptr(loss), _ptr(saved),
                                        _ptr(ws), ws.numel(), _stream(dev)))
     return loss_tok, loss, saved
@@ -286,6 +310,7 @@ def forward_topk_pair(student_logits, teacher_logits, targets, k, B, Sm1, row_id
 def backward_topk_pair(student_logits, teacher_logits, targets, B, Sm1, row_idx, N, reduction, saved,
                        grad_loss=None, grad_tok=None, workspace=None, dz=None):
     """Gradient estimate dLoss/dz_s [T, V] of the top-k estimator."""
+    Nc, nd = _count(N, B, Sm1)
     dev = student_logits.device
     V = student_logits.shape[1]
     dt = _dtype_code(student_logits)
@@ -296,8 +321,8 @@ def backward_topk_pair(student_logits, teacher_logits, targets, B, Sm1, row_idx,
         grad_loss = grad_loss.reshape(1).to(device=dev, dtype=torch.float32).contiguous()
     if grad_tok is not None:
         grad_tok = grad_tok.to(device=dev, dtype=torch.float32).contiguous()
-    ws = workspace if workspace is not None else _workspace(PAYLOAD_LOGITS_PAIR, dt, max(N, 1), B, Sm1, 64, V, dev)
-    _check(lib().rkl_backward_topk_pair(_ptr(student_logits), _ptr(teacher_logits), dt, B, Sm1, V, _ptr(row_idx), N,
+    ws = workspace if workspace is not None else _workspace(PAYLOAD_LOGITS_PAIR, dt, max(Nc, 1), B, Sm1, 64, V, dev)
+    _check(lib().rkl_backward_topk_pair(_ptr(student_logits), _ptr(teacher_logits), dt, B, Sm1, V, _ptr(row_idx), Nc, nd,
                                         _ptr(tg), reduction, _ptr(saved), _ptr(grad_loss), _ptr(grad_tok), _ptr(dz),
                                         _ptr(ws), ws.numel(), _stream(dev)))
     return dz
@@ -307,7 +332,7 @@ class _RKLTopkPair(torch.autograd.Function):
     @staticmethod
     def forward(ctx, student_logits, teacher_logits, targets, mask, k, reduction):
         B, Sm1 = mask.shape
-        row_idx, N = compact_rows(mask)
+        row_idx, N = compact_rows(mask, on_device=True)  # no host synchronisation
         loss_tok, loss, saved = forward_topk_pair(student_logits, teacher_logits, targets, k, B, Sm1, row_idx, N,
                                                   reduction)
         tg = targets.to(device=student_logits.device, dtype=torch.int32).contiguous()
@@ -335,6 +360,7 @@ PAYLOAD_TOPK_HIDDEN = 3
 
 def forward_topk_hidden(h_s, h_t, W_s, W_t, targets, k, B, Sm1, row_idx, N, reduction, workspace=None):
     """Top-k estimator on the hidden payload.  Returns (loss_tok, loss, saved [7N])."""
+    Nc, nd = _count(N, B, Sm1)
     dev = h_s.device
     T, H = h_s.shape
     V = W_s.shape[0]
@@ -342,10 +368,10 @@ def forward_topk_hidden(h_s, h_t, W_s, W_t, targets, k, B, Sm1, row_idx, N, redu
     tg = targets.to(device=dev, dtype=torch.int32).contiguous()
     loss_tok = torch.empty((B, Sm1), dtype=torch.float32, device=dev)
     loss = torch.empty(1, dtype=torch.float32, device=dev)
-    saved = torch.empty(7 * max(N, 1), dtype=torch.float32, device=dev)
-    ws = workspace if workspace is not None else _workspace(PAYLOAD_TOPK_HIDDEN, dt, max(N, 1), B, Sm1, H, V, dev)
+    saved = torch.empty(7 * max(Nc, 1), dtype=torch.float32, device=dev)
+    ws = workspace if workspace is not None else _workspace(PAYLOAD_TOPK_HIDDEN, dt, max(Nc, 1), B, Sm1, H, V, dev)
     _check(lib().rkl_forward_topk_hidden(_ptr(h_s), _ptr(h_t), _ptr(W_s), _ptr(W_t), dt, B, Sm1, H, V,
-                                         _ptr(row_idx), N, int(k), _ptr(tg), reduction, _ptr(loss_tok), _ptr(loss),
+                                         _ptr(row_idx), Nc, nd, int(k), _ptr(tg), reduction, _ptr(loss_tok), _ptr(loss),
                                          _ptr(saved), _ptr(ws), ws.numel(), _stream(dev)))
     return loss_tok, loss, saved
 
@@ -353,6 +379,7 @@ def forward_topk_hidden(h_s, h_t, W_s, W_t, targets, k, B, Sm1, row_idx, N, redu
 def backward_topk_hidden(h_s, h_t, W_s, W_t, targets, B, Sm1, row_idx, N, reduction, saved, grad_loss=None,
                          grad_tok=None, workspace=None, dH_s=None, dW_s=None):
     """(dH_s [T,H] fp32, dW_s [V,H] fp32) of the top-k estimator on the hidden payload."""
+    Nc, nd = _count(N, B, Sm1)
     dev = h_s.device
     T, H = h_s.shape
     V = W_s.shape[0]
@@ -366,9 +393,9 @@ def backward_topk_hidden(h_s, h_t, W_s, W_t, targets, B, Sm1, row_idx, N, reduct
         grad_loss = grad_loss.reshape(1).to(device=dev, dtype=torch.float32).contiguous()
     if grad_tok is not None:
         grad_tok = grad_tok.to(device=dev, dtype=torch.float32).contiguous()
-    ws = workspace if workspace is not None else _workspace(PAYLOAD_TOPK_HIDDEN, dt, max(N, 1), B, Sm1, H, V, dev)
+    ws = workspace if workspace is not None else _workspace(PAYLOAD_TOPK_HIDDEN, dt, max(Nc, 1), B, Sm1, H, V, dev)
     _check(lib().rkl_backward_topk_hidden(_ptr(h_s), _ptr(h_t), _ptr(W_s), _ptr(W_t), dt, B, Sm1, H, V,
-                                          _ptr(row_idx), N, _ptr(tg), reduction, _ptr(saved), _ptr(grad_loss),
+                                          _ptr(row_idx), Nc, nd, _ptr(tg), reduction, _ptr(saved), _ptr(grad_loss),
                                           _ptr(grad_tok), _ptr(dH_s), _ptr(dW_s), _ptr(ws), ws.numel(),
                                           _stream(dev)))
     return dH_s, dW_s
@@ -378,7 +405,7 @@ class _RKLTopkHidden(torch.autograd.Function):
     @staticmethod
     def forward(ctx, h_s, h_t, W_s, W_t, targets, mask, k, reduction):
         B, Sm1 = mask.shape
-        row_idx, N = compact_rows(mask)
+        row_idx, N = compact_rows(mask, on_device=True)  # no host synchronisation
         tg = targets.to(device=h_s.device, dtype=torch.int32).contiguous()
         loss_tok, loss, saved = forward_topk_hidden(h_s, h_t, W_s, W_t, tg, k, B, Sm1, row_idx, N, reduction)
         ctx.save_for_backward(h_s, h_t, W_s, W_t, tg, row_idx, saved)
@@ -521,7 +548,7 @@ class _RKLHidden(torch.autograd.Function):
     @staticmethod
     def forward(ctx, h_s, h_t, W_s, W_t, mask, reduction):
         B, Sm1 = mask.shape
-        row_idx, N = compact_rows(mask)
+        row_idx, N = compact_rows(mask, on_device=True)  # no host synchronisation
         loss_tok, loss, saved = forward_hidden(h_s, h_t, W_s, W_t, B, Sm1, row_idx, N, reduction)
         ctx.save_for_backward(h_s, h_t, W_s, W_t, row_idx, saved)
         ctx.meta = (B, Sm1, N, reduction)
@@ -540,7 +567,7 @@ class _RKLLogits(torch.autograd.Function):
     @staticmethod
     def forward(ctx, h_s, W_s, teacher_logits, mask, reduction):
         B, Sm1 = mask.shape
-        row_idx, N = compact_rows(mask)
+        row_idx, N = compact_rows(mask, on_device=True)  # no host synchronisation
         loss_tok, loss, saved = forward_logits(h_s, W_s, teacher_logits, B, Sm1, row_idx, N, reduction)
         ctx.save_for_backward(h_s, W_s, teacher_logits, row_idx, saved)
         ctx.meta = (B, Sm1, N, reduction)
@@ -559,7 +586,7 @@ class _RKLLogitsPair(torch.autograd.Function):
     @staticmethod
     def forward(ctx, student_logits, teacher_logits, mask, reduction):
         B, Sm1 = mask.shape
-        row_idx, N = compact_rows(mask)
+        row_idx, N = compact_rows(mask, on_device=True)  # no host synchronisation
         loss_tok, loss, saved = forward_logits_pair(student_logits, teacher_logits, B, Sm1, row_idx, N, reduction)
         ctx.save_for_backward(student_logits, teacher_logits, row_idx, saved)
         ctx.meta = (B, Sm1, N, reduction)

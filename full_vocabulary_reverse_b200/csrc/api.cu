@@ -15,10 +15,24 @@
 #include <string>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "rkl.h"
 #include "kernels.h"
 
 namespace rkl {
+
+// An NVTX range over one C-ABI call, named after the entry point.  Profilers
+// that listen to NVTX (Nsight Systems, Nsight Compute's range filters) show
+// each call with its kernels under it; without one attached a push/pop costs
+// a few nanoseconds.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
+#define RKL_NVTX_RANGE() ::rkl::NvtxRange rkl_nvtx_range_(__func__)
 
 // ------------------------------------------------------------------ errors
 static thread_local std::string g_last_error;
@@ -301,6 +315,13 @@ static rkl_status check_ptr(const void* p, const char* name, bool required = tru
   return RKL_OK;
 }
 
+// The optional device row count: one int32, 4-byte aligned.
+static rkl_status check_n_dev(const int32_t* n_dev) {
+  if (n_dev != nullptr && (reinterpret_cast<uintptr_t>(n_dev) & 3) != 0)
+    return fail(RKL_ERR_ALIGN, "n_dev is not 4-byte aligned");
+  return RKL_OK;
+}
+
 #define RKL_TRY(x)                   \
   do {                               \
     rkl_status s__ = (x);            \
@@ -312,12 +333,15 @@ static uint8_t* ws_at(void* ws, size_t off) { return static_cast<uint8_t*>(ws) +
 // ------------------------------------------------------------------ forward
 static rkl_status forward_impl(rkl_payload payload, const void* h_s, const void* teacher, const void* W_s,
                                const void* W_t, rkl_dtype dtype, int64_t B, int64_t Sm1, int64_t H, int64_t V,
-                               const int32_t* row_idx, int32_t N, rkl_reduction reduction, float* loss_tok,
-                               float* loss, float* saved, void* workspace, size_t workspace_bytes, void* stream_,
-                               bool forward_only_workspace = false, const int32_t* targets = nullptr,
+                               const int32_t* row_idx, int32_t N, const int32_t* n_dev, rkl_reduction reduction,
+                               float* loss_tok, float* loss, float* saved, void* workspace, size_t workspace_bytes,
+                               void* stream_, bool forward_only_workspace = false, const int32_t* targets = nullptr,
                                float* entropy = nullptr, float* target_logprob = nullptr,
                                const MultiTeacher* mt = nullptr) {
   RKL_TRY(check_common(payload, dtype, B, Sm1, H, V, N, reduction));
+  RKL_TRY(check_n_dev(n_dev));
+  if (mt && n_dev)
+    return fail(RKL_ERR_UNSUPPORTED, "a teacher per row needs the per-teacher counts on the host (n_dev must be NULL)");
   RKL_TRY(check_ptr(h_s, "h_s"));
   RKL_TRY(check_ptr(teacher, payload == RKL_PAYLOAD_HIDDEN ? "h_t" : "teacher_logits"));
   RKL_TRY(check_ptr(W_s, "W_s"));
@@ -365,17 +389,19 @@ static rkl_status forward_impl(rkl_payload payload, const void* h_s, const void*
       RKL_CUDA(launch_build_slots(row_idx, mt->teacher_idx, N, mt->ts, slot_k,
                                   reinterpret_cast<int32_t*>(ws_at(workspace, pl.off_kslot)), s));
     }
-    // S2: compact the rows (skipped when every row is trainable).
+    // S2: compact the rows (skipped when every row is known to be trainable).
+    const bool identity = N == T && !mt && !n_dev;
     const void* as = h_s;
     const void* at = teacher;
-    if (N < T || mt) {
+    if (!identity) {
       as = ws_at(workspace, pl.off_hcs);
       at = hidden ? ws_at(workspace, pl.off_hct) : nullptr;
       RKL_CUDA(launch_gather(h_s, hidden ? teacher : nullptr, const_cast<void*>(as), const_cast<void*>(at), row_idx,
-                             slot_k, n_rows, static_cast<int>(H * pl.es), s));
+                             slot_k, n_rows, n_dev, static_cast<int>(H * pl.es), T, s));
     }
     // S8: teacher log-sum-exp from the shipped logits.
-    if (!hidden) RKL_CUDA(launch_teacher_lse(teacher, bf16, row_idx, N, static_cast<int>(V), V, lse_ext, s));
+    if (!hidden)
+      RKL_CUDA(launch_teacher_lse(teacher, bf16, row_idx, N, n_dev, static_cast<int>(V), V, lse_ext, T, s));
     const int ng = hidden ? 2 : 1;
     if (bf16) {
       FusedArgs a;
@@ -391,7 +417,7 @@ static rkl_status forward_impl(rkl_payload payload, const void* h_s, const void*
         }
       } else {
         a.teacher = static_cast<const uint16_t*>(teacher);
-        a.teacher_rows = N < T ? row_idx : nullptr;
+        a.teacher_rows = identity ? nullptr : row_idx;
         a.teacher_pitch = V;
       }
       a.part = part;
@@ -399,6 +425,7 @@ static rkl_status forward_impl(rkl_payload payload, const void* h_s, const void*
       a.targets = targets;
       a.tlogit = tlogit;
       a.N = n_rows;
+      a.n_dev = n_dev;
       a.n_pad = pl.n_pad;
       a.H = static_cast<int>(H);
       a.V = static_cast<int>(V);
@@ -407,10 +434,8 @@ static rkl_status forward_impl(rkl_payload payload, const void* h_s, const void*
       a.vt_base = 0;
       a.GT = kGroupTiles;
       a.G = pl.S / 2;
-      const int MT = (n_rows + 2 * kBM - 1) / (2 * kBM);
-      a.MT = MT;
-      a.units_total = MT * a.G;
-      RKL_CUDA(launch_fused(ng, false, a, 2 * a.units_total < sms ? 2 * a.units_total : sms, s));
+      const int units = ((n_rows + 2 * kBM - 1) / (2 * kBM)) * a.G;  // at most; the kernel takes the live count
+      RKL_CUDA(launch_fused(ng, false, a, 2 * units < sms ? 2 * units : sms, s));
     } else {
       SimtArgs a;
       memset(&a, 0, sizeof(a));
@@ -425,7 +450,7 @@ static rkl_status forward_impl(rkl_payload payload, const void* h_s, const void*
         }
       } else {
         a.teacher = static_cast<const float*>(teacher);
-        a.teacher_rows = N < T ? row_idx : nullptr;
+        a.teacher_rows = identity ? nullptr : row_idx;
         a.teacher_pitch = V;
       }
       a.part = part;
@@ -433,6 +458,7 @@ static rkl_status forward_impl(rkl_payload payload, const void* h_s, const void*
       a.targets = targets;
       a.tlogit = tlogit;
       a.N = n_rows;
+      a.n_dev = n_dev;
       a.n_pad = pl.n_pad;
       a.H = static_cast<int>(H);
       a.V = static_cast<int>(V);
@@ -443,25 +469,28 @@ static rkl_status forward_impl(rkl_payload payload, const void* h_s, const void*
       RKL_CUDA(launch_simt_fused(false, a, dim3(MT, pl.S), s));
     }
     // S4
-    RKL_CUDA(launch_combine(part, pl.S, pl.n_pad, n_rows, hidden, lse_ext, tlogit, saved, ent_rows, lp_rows, slot_k,
-                            s));
+    RKL_CUDA(launch_combine(part, pl.S, pl.n_pad, n_rows, n_dev, hidden, lse_ext, tlogit, saved, ent_rows, lp_rows,
+                            slot_k, s));
   }
-  if (loss_tok) RKL_CUDA(launch_scatter_loss(saved, row_idx, N, T, loss_tok, s));
-  if (entropy) RKL_CUDA(launch_scatter_rows(ent_rows, row_idx, N, T, entropy, s));
-  if (target_logprob) RKL_CUDA(launch_scatter_rows(lp_rows, row_idx, N, T, target_logprob, s));
+  if (loss_tok) RKL_CUDA(launch_scatter_loss(saved, row_idx, N, n_dev, T, loss_tok, s));
+  if (entropy) RKL_CUDA(launch_scatter_rows(ent_rows, row_idx, N, n_dev, T, entropy, s));
+  if (target_logprob) RKL_CUDA(launch_scatter_rows(lp_rows, row_idx, N, n_dev, T, target_logprob, s));
   if (loss && reduction != RKL_REDUCE_NONE)
-    RKL_CUDA(launch_reduce(saved, row_idx, N, static_cast<int>(B), static_cast<int>(Sm1), reduction, loss, s));
+    RKL_CUDA(launch_reduce(saved, row_idx, N, n_dev, static_cast<int>(B), static_cast<int>(Sm1), reduction, loss, s));
   return RKL_OK;
 }
 
 // ------------------------------------------------------------------ backward
 static rkl_status backward_impl(rkl_payload payload, const void* h_s, const void* teacher, const void* W_s,
                                 const void* W_t, rkl_dtype dtype, int64_t B, int64_t Sm1, int64_t H, int64_t V,
-                                const int32_t* row_idx, int32_t N, rkl_reduction reduction, const float* saved,
-                                const float* grad_loss, const float* grad_tok, float* dH_s, float* dW_s,
-                                void* workspace, size_t workspace_bytes, void* stream_,
+                                const int32_t* row_idx, int32_t N, const int32_t* n_dev, rkl_reduction reduction,
+                                const float* saved, const float* grad_loss, const float* grad_tok, float* dH_s,
+                                float* dW_s, void* workspace, size_t workspace_bytes, void* stream_,
                                 const MultiTeacher* mt = nullptr, const int32_t* topk_targets = nullptr) {
   RKL_TRY(check_common(payload, dtype, B, Sm1, H, V, N, reduction));
+  RKL_TRY(check_n_dev(n_dev));
+  if (mt && n_dev)
+    return fail(RKL_ERR_UNSUPPORTED, "a teacher per row needs the per-teacher counts on the host (n_dev must be NULL)");
   RKL_TRY(check_ptr(h_s, "h_s"));
   RKL_TRY(check_ptr(teacher, payload != RKL_PAYLOAD_LOGITS ? "h_t" : "teacher_logits"));
   RKL_TRY(check_ptr(W_s, "W_s"));
@@ -490,7 +519,7 @@ static rkl_status backward_impl(rkl_payload payload, const void* h_s, const void
 
   if (N == 0) {
     RKL_CUDA(cudaMemsetAsync(dW_s, 0, size_t(V) * H * sizeof(float), s));
-    RKL_CUDA(launch_scatter_dh(dHc, row_idx, nullptr, 0, T, static_cast<int>(H), dH_s, s));
+    RKL_CUDA(launch_scatter_dh(dHc, row_idx, nullptr, 0, nullptr, T, static_cast<int>(H), dH_s, s));
     return RKL_OK;
   }
   // Teacher per row: rows regrouped by teacher into whole pair tiles.
@@ -504,21 +533,22 @@ static rkl_status backward_impl(rkl_payload payload, const void* h_s, const void
     RKL_CUDA(cudaMemsetAsync(slot_k, 0xFF, size_t(n_rows) * sizeof(int32_t), s));
     RKL_CUDA(launch_build_slots(row_idx, mt->teacher_idx, N, mt->ts, slot_k, k_slot, s));
   }
+  const bool identity = N == T && !mt && !n_dev;
   const void* as = h_s;
   const void* at = teacher;
-  if (N < T || mt) {
+  if (!identity) {
     as = ws_at(workspace, pl.off_hcs);
     at = hidden ? ws_at(workspace, pl.off_hct) : nullptr;
     RKL_CUDA(launch_gather(h_s, hidden ? teacher : nullptr, const_cast<void*>(as), const_cast<void*>(at), row_idx,
-                           slot_k, n_rows, static_cast<int>(H * pl.es), s));
+                           slot_k, n_rows, n_dev, static_cast<int>(H * pl.es), T, s));
   }
   float* rowc = reinterpret_cast<float*>(ws_at(workspace, pl.off_rowc));
-  RKL_CUDA(launch_row_weights(saved, row_idx, N, pl.n_pad, static_cast<int>(B), static_cast<int>(Sm1), reduction,
-                              grad_loss, grad_tok, rowc, slot_k, s));
+  RKL_CUDA(launch_row_weights(saved, row_idx, N, n_dev, pl.n_pad, static_cast<int>(B), static_cast<int>(Sm1),
+                              reduction, grad_loss, grad_tok, rowc, slot_k, s));
   float* rowk = nullptr;
   if (topk) {
     rowk = reinterpret_cast<float*>(ws_at(workspace, pl.off_rowk));
-    RKL_CUDA(launch_topk_rowk(saved, saved + 3 * size_t(N), row_idx, topk_targets, N, pl.n_pad, rowk, s));
+    RKL_CUDA(launch_topk_rowk(saved, saved + 3 * size_t(N), row_idx, topk_targets, N, n_dev, pl.n_pad, rowk, s));
   }
   void* dz = ws_at(workspace, pl.off_dz);
   const int ng = hidden ? 2 : 1;
@@ -538,18 +568,18 @@ static rkl_status backward_impl(rkl_payload payload, const void* h_s, const void
       }
     } else {
       a.teacher = static_cast<const uint16_t*>(teacher);
-      a.teacher_rows = N < T ? row_idx : nullptr;
+      a.teacher_rows = identity ? nullptr : row_idx;
       a.teacher_pitch = V;
     }
     a.rowc = rowc;
     a.rowk = rowk;
     a.N = n_rows;
+    a.n_dev = n_dev;
     a.n_pad = pl.n_pad;
     a.H = static_cast<int>(H);
     a.V = static_cast<int>(V);
     a.KB = static_cast<int>(H / kBK);
-    const int MT = (n_rows + 2 * kBM - 1) / (2 * kBM);
-    a.MT = MT;
+    const int MT = (n_rows + 2 * kBM - 1) / (2 * kBM);  // at most; the kernels take the live count
 
     int* counters = reinterpret_cast<int*>(ws_at(workspace, pl.off_cnt));
     RKL_CUDA(cudaMemsetAsync(counters, 0, size_t(nchunks) * sizeof(int), s));
@@ -560,11 +590,9 @@ static rkl_status backward_impl(rkl_payload payload, const void* h_s, const void
     RKL_TRY(make_map(&g.tm_dw, dW_s, true, H, V, H * 4, 32, 32));
     RKL_TRY(make_map(&g.tm_dh, dHc, true, H, n_rows, H * 4, 32, 32));
     g.N = n_rows;
+    g.n_dev = n_dev;
     g.H = static_cast<int>(H);
     g.NT = static_cast<int>(H / kGradBN) + (H % kGradBN ? 1 : 0);
-    g.MTH = (n_rows + 2 * kBM - 1) / (2 * kBM);  // 256-row pair tiles
-    g.nH = g.MTH * g.NT;
-    g.KBW = (n_rows + kBK - 1) / kBK;
 
     for (int c = 0; c < nchunks; ++c) {
       const int cv0 = c * pl.Vc;
@@ -576,8 +604,8 @@ static rkl_status backward_impl(rkl_payload payload, const void* h_s, const void
       a.chunk_v0 = cv0;
       a.GT = 1;
       a.G = a.IT;
-      a.units_total = MT * a.IT;
-      const int fgrid = 2 * a.units_total < sms ? 2 * a.units_total : sms;
+      const int units = MT * a.IT;
+      const int fgrid = 2 * units < sms ? 2 * units : sms;
       if (topk)
         RKL_CUDA(launch_fused_topk(2, a, fgrid, s));
       else
@@ -592,7 +620,7 @@ static rkl_status backward_impl(rkl_payload payload, const void* h_s, const void
       g.KBH = (cw + kBK - 1) / kBK;
       g.dh_accumulate = c > 0;
       g.tile_counter = counters + c;
-      const int pairs = g.nW + g.nH;
+      const int pairs = g.nW + MT * g.NT;  // at most
       RKL_CUDA(launch_grad(g, 2 * pairs < sms ? 2 * pairs : sms, s));
     }
   } else {
@@ -609,12 +637,13 @@ static rkl_status backward_impl(rkl_payload payload, const void* h_s, const void
       }
     } else {
       a.teacher = static_cast<const float*>(teacher);
-      a.teacher_rows = N < T ? row_idx : nullptr;
+      a.teacher_rows = identity ? nullptr : row_idx;
       a.teacher_pitch = V;
     }
     a.rowc = rowc;
     a.dz = static_cast<float*>(dz);
     a.N = n_rows;
+    a.n_dev = n_dev;
     a.n_pad = pl.n_pad;
     a.H = static_cast<int>(H);
     a.V = static_cast<int>(V);
@@ -632,13 +661,13 @@ static rkl_status backward_impl(rkl_payload payload, const void* h_s, const void
       const float* dzf = static_cast<const float*>(dz);
       // dW_s[cv0 + m, n] = sum_k dz[k, m] hc_s[k, n]
       RKL_CUDA(launch_simt_gemm(dzf, 1, cw, a.as, H, 1, dW_s + size_t(cv0) * H, H, cw, static_cast<int>(H), n_rows,
-                                0, s));
+                                0, n_dev, 2, s));
       // dHc[m, n] (+)= sum_k dz[m, k] W_s[cv0 + k, n]
       RKL_CUDA(launch_simt_gemm(dzf, cw, 1, a.bs + size_t(cv0) * H, H, 1, dHc, H, n_rows, static_cast<int>(H), cw,
-                                c > 0, s));
+                                c > 0, n_dev, 1, s));
     }
   }
-  RKL_CUDA(launch_scatter_dh(dHc, row_idx, k_slot, N, T, static_cast<int>(H), dH_s, s));
+  RKL_CUDA(launch_scatter_dh(dHc, row_idx, k_slot, N, n_dev, T, static_cast<int>(H), dH_s, s));
   return RKL_OK;
 }
 
@@ -649,7 +678,11 @@ using namespace rkl;
 
 extern "C" {
 
-const char* rkl_version(void) { return "rkl 0.1 (sm_100a)"; }
+#ifdef RKL_DEBUG
+const char* rkl_version(void) { return "rkl 0.2 (sm_100a, debug bounds checks)"; }
+#else
+const char* rkl_version(void) { return "rkl 0.2 (sm_100a)"; }
+#endif
 
 const char* rkl_last_error(void) { return g_last_error.c_str(); }
 
@@ -670,10 +703,12 @@ rkl_status rkl_workspace_size(rkl_payload payload, rkl_dtype dtype, int64_t n_ma
 }
 
 rkl_status rkl_forward_logits_pair(const void* student_logits, const void* teacher_logits, rkl_dtype dtype, int64_t B,
-                                   int64_t Sm1, int64_t V, const int32_t* row_idx, int32_t N, rkl_reduction reduction,
-                                   float* loss_tok, float* loss, float* saved, void* workspace,
-                                   size_t workspace_bytes, void* stream) {
+                                   int64_t Sm1, int64_t V, const int32_t* row_idx, int32_t N, const int32_t* n_dev,
+                                   rkl_reduction reduction, float* loss_tok, float* loss, float* saved,
+                                   void* workspace, size_t workspace_bytes, void* stream) {
+  RKL_NVTX_RANGE();
   RKL_TRY(check_common(RKL_PAYLOAD_LOGITS_PAIR, dtype, B, Sm1, 64, V, N, reduction));
+  RKL_TRY(check_n_dev(n_dev));
   RKL_TRY(check_ptr(student_logits, "student_logits"));
   RKL_TRY(check_ptr(teacher_logits, "teacher_logits"));
   RKL_TRY(check_ptr(row_idx, "row_idx"));
@@ -687,20 +722,22 @@ rkl_status rkl_forward_logits_pair(const void* student_logits, const void* teach
   RKL_TRY(device_setup(&sms));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const long long T = B * Sm1;
-  RKL_CUDA(launch_pair_fwd(student_logits, teacher_logits, dtype == RKL_BF16, row_idx, N, static_cast<int>(V), saved,
-                           s));
-  if (loss_tok) RKL_CUDA(launch_scatter_loss(saved, row_idx, N, T, loss_tok, s));
+  RKL_CUDA(launch_pair_fwd(student_logits, teacher_logits, dtype == RKL_BF16, row_idx, N, n_dev, static_cast<int>(V),
+                           saved, s));
+  if (loss_tok) RKL_CUDA(launch_scatter_loss(saved, row_idx, N, n_dev, T, loss_tok, s));
   if (loss && reduction != RKL_REDUCE_NONE)
-    RKL_CUDA(launch_reduce(saved, row_idx, N, static_cast<int>(B), static_cast<int>(Sm1), reduction, loss, s));
+    RKL_CUDA(launch_reduce(saved, row_idx, N, n_dev, static_cast<int>(B), static_cast<int>(Sm1), reduction, loss, s));
   return RKL_OK;
 }
 
 rkl_status rkl_backward_logits_pair(const void* student_logits, const void* teacher_logits, rkl_dtype dtype,
                                     int64_t B, int64_t Sm1, int64_t V, const int32_t* row_idx, int32_t N,
-                                    rkl_reduction reduction, const float* saved, const float* grad_loss,
-                                    const float* grad_tok, void* dz, void* workspace, size_t workspace_bytes,
-                                    void* stream) {
+                                    const int32_t* n_dev, rkl_reduction reduction, const float* saved,
+                                    const float* grad_loss, const float* grad_tok, void* dz, void* workspace,
+                                    size_t workspace_bytes, void* stream) {
+  RKL_NVTX_RANGE();
   RKL_TRY(check_common(RKL_PAYLOAD_LOGITS_PAIR, dtype, B, Sm1, 64, V, N, reduction));
+  RKL_TRY(check_n_dev(n_dev));
   RKL_TRY(check_ptr(student_logits, "student_logits"));
   RKL_TRY(check_ptr(teacher_logits, "teacher_logits"));
   RKL_TRY(check_ptr(row_idx, "row_idx"));
@@ -719,18 +756,19 @@ rkl_status rkl_backward_logits_pair(const void* student_logits, const void* teac
   const int n_pad = static_cast<int>(((n + 255) / 256) * 256);
   float* rowc = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + 256);
   if (N > 0)
-    RKL_CUDA(launch_row_weights(saved, row_idx, N, n_pad, static_cast<int>(B), static_cast<int>(Sm1), reduction,
-                                grad_loss, grad_tok, rowc, nullptr, s));
-  RKL_CUDA(launch_pair_bwd(student_logits, teacher_logits, dtype == RKL_BF16, row_idx, N, n_pad, T,
+    RKL_CUDA(launch_row_weights(saved, row_idx, N, n_dev, n_pad, static_cast<int>(B), static_cast<int>(Sm1),
+                                reduction, grad_loss, grad_tok, rowc, nullptr, s));
+  RKL_CUDA(launch_pair_bwd(student_logits, teacher_logits, dtype == RKL_BF16, row_idx, N, n_dev, n_pad, T,
                            static_cast<int>(V), rowc, dz, s));
   return RKL_OK;
 }
 
 // ---------------------------------------------------------------- top-k estimator
 static rkl_status check_topk(const void* zs, const void* zt, rkl_dtype dtype, int64_t B, int64_t Sm1, int64_t V,
-                             const int32_t* row_idx, int32_t N, int64_t k, const int32_t* targets, int reduction,
-                             void* workspace, size_t workspace_bytes) {
+                             const int32_t* row_idx, int32_t N, const int32_t* n_dev, int64_t k,
+                             const int32_t* targets, int reduction, void* workspace, size_t workspace_bytes) {
   RKL_TRY(check_common(RKL_PAYLOAD_LOGITS_PAIR, dtype, B, Sm1, 64, V, N, reduction));
+  RKL_TRY(check_n_dev(n_dev));
   RKL_TRY(check_ptr(zs, "student_logits"));
   RKL_TRY(check_ptr(zt, "teacher_logits"));
   RKL_TRY(check_ptr(row_idx, "row_idx"));
@@ -743,11 +781,12 @@ static rkl_status check_topk(const void* zs, const void* zt, rkl_dtype dtype, in
 }
 
 rkl_status rkl_forward_topk_pair(const void* student_logits, const void* teacher_logits, rkl_dtype dtype, int64_t B,
-                                 int64_t Sm1, int64_t V, const int32_t* row_idx, int32_t N, int64_t k,
-                                 const int32_t* targets, rkl_reduction reduction, float* loss_tok, float* loss,
-                                 float* saved, void* workspace, size_t workspace_bytes, void* stream) {
-  RKL_TRY(check_topk(student_logits, teacher_logits, dtype, B, Sm1, V, row_idx, N, k, targets, reduction, workspace,
-                     workspace_bytes));
+                                 int64_t Sm1, int64_t V, const int32_t* row_idx, int32_t N, const int32_t* n_dev,
+                                 int64_t k, const int32_t* targets, rkl_reduction reduction, float* loss_tok,
+                                 float* loss, float* saved, void* workspace, size_t workspace_bytes, void* stream) {
+  RKL_NVTX_RANGE();
+  RKL_TRY(check_topk(student_logits, teacher_logits, dtype, B, Sm1, V, row_idx, N, n_dev, k, targets, reduction,
+                     workspace, workspace_bytes));
   RKL_TRY(check_ptr(loss_tok, "loss_tok", false));
   RKL_TRY(check_ptr(loss, "loss", false));
   RKL_TRY(check_ptr(saved, "saved", N > 0));
@@ -755,21 +794,22 @@ rkl_status rkl_forward_topk_pair(const void* student_logits, const void* teacher
   RKL_TRY(device_setup(&sms));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const long long T = B * Sm1;
-  RKL_CUDA(launch_topk_fwd(student_logits, teacher_logits, dtype == RKL_BF16, row_idx, targets, N,
+  RKL_CUDA(launch_topk_fwd(student_logits, teacher_logits, dtype == RKL_BF16, row_idx, targets, N, n_dev, 0,
                            static_cast<int>(V), k, saved, saved + 3 * size_t(N), V, false, s));
-  if (loss_tok) RKL_CUDA(launch_scatter_loss(saved, row_idx, N, T, loss_tok, s));
+  if (loss_tok) RKL_CUDA(launch_scatter_loss(saved, row_idx, N, n_dev, T, loss_tok, s));
   if (loss && reduction != RKL_REDUCE_NONE)
-    RKL_CUDA(launch_reduce(saved, row_idx, N, static_cast<int>(B), static_cast<int>(Sm1), reduction, loss, s));
+    RKL_CUDA(launch_reduce(saved, row_idx, N, n_dev, static_cast<int>(B), static_cast<int>(Sm1), reduction, loss, s));
   return RKL_OK;
 }
 
 rkl_status rkl_backward_topk_pair(const void* student_logits, const void* teacher_logits, rkl_dtype dtype,
                                   int64_t B, int64_t Sm1, int64_t V, const int32_t* row_idx, int32_t N,
-                                  const int32_t* targets, rkl_reduction reduction, const float* saved,
-                                  const float* grad_loss, const float* grad_tok, void* dz, void* workspace,
-                                  size_t workspace_bytes, void* stream) {
-  RKL_TRY(check_topk(student_logits, teacher_logits, dtype, B, Sm1, V, row_idx, N, 0, targets, reduction, workspace,
-                     workspace_bytes));
+                                  const int32_t* n_dev, const int32_t* targets, rkl_reduction reduction,
+                                  const float* saved, const float* grad_loss, const float* grad_tok, void* dz,
+                                  void* workspace, size_t workspace_bytes, void* stream) {
+  RKL_NVTX_RANGE();
+  RKL_TRY(check_topk(student_logits, teacher_logits, dtype, B, Sm1, V, row_idx, N, n_dev, 0, targets, reduction,
+                     workspace, workspace_bytes));
   RKL_TRY(check_ptr(saved, "saved", N > 0));
   RKL_TRY(check_ptr(grad_loss, "grad_loss", false));
   RKL_TRY(check_ptr(grad_tok, "grad_tok", false));
@@ -782,9 +822,9 @@ rkl_status rkl_backward_topk_pair(const void* student_logits, const void* teache
   const int n_pad = static_cast<int>(((n + 255) / 256) * 256);
   float* rowc = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + 256);
   if (N > 0)
-    RKL_CUDA(launch_row_weights(saved, row_idx, N, n_pad, static_cast<int>(B), static_cast<int>(Sm1), reduction,
-                                grad_loss, grad_tok, rowc, nullptr, s));
-  RKL_CUDA(launch_topk_bwd(student_logits, teacher_logits, dtype == RKL_BF16, row_idx, targets, N, n_pad, T,
+    RKL_CUDA(launch_row_weights(saved, row_idx, N, n_dev, n_pad, static_cast<int>(B), static_cast<int>(Sm1),
+                                reduction, grad_loss, grad_tok, rowc, nullptr, s));
+  RKL_CUDA(launch_topk_bwd(student_logits, teacher_logits, dtype == RKL_BF16, row_idx, targets, N, n_dev, n_pad, T,
                            static_cast<int>(V), saved, N > 0 ? saved + 3 * size_t(N) : nullptr, rowc, dz, s));
   return RKL_OK;
 }
@@ -797,10 +837,12 @@ rkl_status rkl_backward_topk_pair(const void* student_logits, const void* teache
 // gradient GEMMs of the exact path.
 rkl_status rkl_forward_topk_hidden(const void* h_s, const void* h_t, const void* W_s, const void* W_t,
                                    rkl_dtype dtype, int64_t B, int64_t Sm1, int64_t H, int64_t V,
-                                   const int32_t* row_idx, int32_t N, int64_t k, const int32_t* targets,
-                                   rkl_reduction reduction, float* loss_tok, float* loss, float* saved,
-                                   void* workspace, size_t workspace_bytes, void* stream) {
+                                   const int32_t* row_idx, int32_t N, const int32_t* n_dev, int64_t k,
+                                   const int32_t* targets, rkl_reduction reduction, float* loss_tok, float* loss,
+                                   float* saved, void* workspace, size_t workspace_bytes, void* stream) {
+  RKL_NVTX_RANGE();
   RKL_TRY(check_common(RKL_PAYLOAD_TOPK_HIDDEN, dtype, B, Sm1, H, V, N, reduction));
+  RKL_TRY(check_n_dev(n_dev));
   if (dtype != RKL_BF16)
     return fail(RKL_ERR_UNSUPPORTED, "the top-k estimator on the hidden payload needs bf16 inputs");
   if (k < 0) return fail(RKL_ERR_SHAPE, "k = %lld is negative", (long long)k);
@@ -824,11 +866,11 @@ rkl_status rkl_forward_topk_hidden(const void* h_s, const void* h_t, const void*
   if (N > 0) {
     const uint8_t* as = static_cast<const uint8_t*>(h_s);
     const uint8_t* at = static_cast<const uint8_t*>(h_t);
-    if (N < T) {
+    if (N < T || n_dev) {
       as = ws_at(workspace, pl.off_hcs);
       at = ws_at(workspace, pl.off_hct);
-      RKL_CUDA(launch_gather(h_s, h_t, const_cast<uint8_t*>(as), const_cast<uint8_t*>(at), row_idx, nullptr, N,
-                             static_cast<int>(H * 2), s));
+      RKL_CUDA(launch_gather(h_s, h_t, const_cast<uint8_t*>(as), const_cast<uint8_t*>(at), row_idx, nullptr, N, n_dev,
+                             static_cast<int>(H * 2), T, s));
     }
     float* zs = reinterpret_cast<float*>(ws_at(workspace, pl.off_z));
     float* zt = zs + size_t(pl.zrows) * pl.zpitch;
@@ -843,6 +885,8 @@ rkl_status rkl_forward_topk_hidden(const void* h_s, const void* h_t, const void*
       RKL_TRY(make_map(&a.tm_zs, zs, true, V, nb, size_t(pl.zpitch) * 4, 32, 32));
       RKL_TRY(make_map(&a.tm_zt, zt, true, V, nb, size_t(pl.zpitch) * 4, 32, 32));
       a.N = nb;
+      a.n_dev = n_dev;
+      a.n_base = r0;
       a.n_pad = pl.n_pad;
       a.H = static_cast<int>(H);
       a.V = static_cast<int>(V);
@@ -851,31 +895,33 @@ rkl_status rkl_forward_topk_hidden(const void* h_s, const void* h_t, const void*
       a.vt_base = 0;
       a.GT = 1;
       a.G = pl.VT;
-      a.MT = (nb + 2 * kBM - 1) / (2 * kBM);
-      a.units_total = a.MT * a.G;
-      RKL_CUDA(launch_fused_topk(1, a, 2 * a.units_total < sms ? 2 * a.units_total : sms, s));
-      RKL_CUDA(launch_topk_fwd(zs, zt, false, row_idx + r0, targets, nb, static_cast<int>(V), k, saved + 3 * size_t(r0),
-                               saved + 3 * size_t(N) + 4 * size_t(r0), pl.zpitch, true, s));
+      const int units = ((nb + 2 * kBM - 1) / (2 * kBM)) * a.G;  // at most
+      RKL_CUDA(launch_fused_topk(1, a, 2 * units < sms ? 2 * units : sms, s));
+      RKL_CUDA(launch_topk_fwd(zs, zt, false, row_idx + r0, targets, nb, n_dev, r0, static_cast<int>(V), k,
+                               saved + 3 * size_t(r0), saved + 3 * size_t(N) + 4 * size_t(r0), pl.zpitch, true, s));
     }
   }
-  if (loss_tok) RKL_CUDA(launch_scatter_loss(saved, row_idx, N, T, loss_tok, s));
+  if (loss_tok) RKL_CUDA(launch_scatter_loss(saved, row_idx, N, n_dev, T, loss_tok, s));
   if (loss && reduction != RKL_REDUCE_NONE)
-    RKL_CUDA(launch_reduce(saved, row_idx, N, static_cast<int>(B), static_cast<int>(Sm1), reduction, loss, s));
+    RKL_CUDA(launch_reduce(saved, row_idx, N, n_dev, static_cast<int>(B), static_cast<int>(Sm1), reduction, loss, s));
   return RKL_OK;
 }
 
 rkl_status rkl_backward_topk_hidden(const void* h_s, const void* h_t, const void* W_s, const void* W_t,
                                     rkl_dtype dtype, int64_t B, int64_t Sm1, int64_t H, int64_t V,
-                                    const int32_t* row_idx, int32_t N, const int32_t* targets,
+                                    const int32_t* row_idx, int32_t N, const int32_t* n_dev, const int32_t* targets,
                                     rkl_reduction reduction, const float* saved, const float* grad_loss,
                                     const float* grad_tok, float* dH_s, float* dW_s, void* workspace,
                                     size_t workspace_bytes, void* stream) {
-  return backward_impl(RKL_PAYLOAD_TOPK_HIDDEN, h_s, h_t, W_s, W_t, dtype, B, Sm1, H, V, row_idx, N, reduction,
-                       saved, grad_loss, grad_tok, dH_s, dW_s, workspace, workspace_bytes, stream, nullptr, targets);
+  RKL_NVTX_RANGE();
+  return backward_impl(RKL_PAYLOAD_TOPK_HIDDEN, h_s, h_t, W_s, W_t, dtype, B, Sm1, H, V, row_idx, N, n_dev,
+                       reduction, saved, grad_loss, grad_tok, dH_s, dW_s, workspace, workspace_bytes, stream, nullptr,
+                       targets);
 }
 
 rkl_status rkl_compact_rows(const uint8_t* mask, int64_t B, int64_t Sm1, int32_t* row_idx, int32_t* n_dev,
                             void* stream) {
+  RKL_NVTX_RANGE();
   if (mask == nullptr || row_idx == nullptr || n_dev == nullptr)
     return fail(RKL_ERR_NULL, "mask, row_idx and n_dev must be non-NULL");
   if (!aligned16(row_idx)) return fail(RKL_ERR_ALIGN, "row_idx is not 16-byte aligned");
@@ -889,52 +935,59 @@ rkl_status rkl_compact_rows(const uint8_t* mask, int64_t B, int64_t Sm1, int32_t
 
 rkl_status rkl_forward_hidden(const void* h_s, const void* h_t, const void* W_s, const void* W_t, rkl_dtype dtype,
                               int64_t B, int64_t Sm1, int64_t H, int64_t V, const int32_t* row_idx, int32_t N,
-                              rkl_reduction reduction, float* loss_tok, float* loss, float* saved, void* workspace,
-                              size_t workspace_bytes, void* stream) {
-  return forward_impl(RKL_PAYLOAD_HIDDEN, h_s, h_t, W_s, W_t, dtype, B, Sm1, H, V, row_idx, N, reduction, loss_tok,
-                      loss, saved, workspace, workspace_bytes, stream);
+                              const int32_t* n_dev, rkl_reduction reduction, float* loss_tok, float* loss,
+                              float* saved, void* workspace, size_t workspace_bytes, void* stream) {
+  RKL_NVTX_RANGE();
+  return forward_impl(RKL_PAYLOAD_HIDDEN, h_s, h_t, W_s, W_t, dtype, B, Sm1, H, V, row_idx, N, n_dev, reduction,
+                      loss_tok, loss, saved, workspace, workspace_bytes, stream);
 }
 
 rkl_status rkl_forward_logits(const void* h_s, const void* W_s, const void* teacher_logits, rkl_dtype dtype,
                               int64_t B, int64_t Sm1, int64_t H, int64_t V, const int32_t* row_idx, int32_t N,
-                              rkl_reduction reduction, float* loss_tok, float* loss, float* saved, void* workspace,
-                              size_t workspace_bytes, void* stream) {
-  return forward_impl(RKL_PAYLOAD_LOGITS, h_s, teacher_logits, W_s, nullptr, dtype, B, Sm1, H, V, row_idx, N,
+                              const int32_t* n_dev, rkl_reduction reduction, float* loss_tok, float* loss,
+                              float* saved, void* workspace, size_t workspace_bytes, void* stream) {
+  RKL_NVTX_RANGE();
+  return forward_impl(RKL_PAYLOAD_LOGITS, h_s, teacher_logits, W_s, nullptr, dtype, B, Sm1, H, V, row_idx, N, n_dev,
                       reduction, loss_tok, loss, saved, workspace, workspace_bytes, stream);
 }
 
 rkl_status rkl_forward_hidden_ex(const void* h_s, const void* h_t, const void* W_s, const void* W_t, rkl_dtype dtype,
                                  int64_t B, int64_t Sm1, int64_t H, int64_t V, const int32_t* row_idx, int32_t N,
-                                 rkl_reduction reduction, float* loss_tok, float* loss, float* saved,
-                                 const int32_t* targets, float* entropy, float* target_logprob, void* workspace,
-                                 size_t workspace_bytes, void* stream) {
-  return forward_impl(RKL_PAYLOAD_HIDDEN, h_s, h_t, W_s, W_t, dtype, B, Sm1, H, V, row_idx, N, reduction, loss_tok,
-                      loss, saved, workspace, workspace_bytes, stream, false, targets, entropy, target_logprob);
+                                 const int32_t* n_dev, rkl_reduction reduction, float* loss_tok, float* loss,
+                                 float* saved, const int32_t* targets, float* entropy, float* target_logprob,
+                                 void* workspace, size_t workspace_bytes, void* stream) {
+  RKL_NVTX_RANGE();
+  return forward_impl(RKL_PAYLOAD_HIDDEN, h_s, h_t, W_s, W_t, dtype, B, Sm1, H, V, row_idx, N, n_dev, reduction,
+                      loss_tok, loss, saved, workspace, workspace_bytes, stream, false, targets, entropy,
+                      target_logprob);
 }
 
 rkl_status rkl_forward_logits_ex(const void* h_s, const void* W_s, const void* teacher_logits, rkl_dtype dtype,
                                  int64_t B, int64_t Sm1, int64_t H, int64_t V, const int32_t* row_idx, int32_t N,
-                                 rkl_reduction reduction, float* loss_tok, float* loss, float* saved,
-                                 const int32_t* targets, float* entropy, float* target_logprob, void* workspace,
-                                 size_t workspace_bytes, void* stream) {
-  return forward_impl(RKL_PAYLOAD_LOGITS, h_s, teacher_logits, W_s, nullptr, dtype, B, Sm1, H, V, row_idx, N,
+                                 const int32_t* n_dev, rkl_reduction reduction, float* loss_tok, float* loss,
+                                 float* saved, const int32_t* targets, float* entropy, float* target_logprob,
+                                 void* workspace, size_t workspace_bytes, void* stream) {
+  RKL_NVTX_RANGE();
+  return forward_impl(RKL_PAYLOAD_LOGITS, h_s, teacher_logits, W_s, nullptr, dtype, B, Sm1, H, V, row_idx, N, n_dev,
                       reduction, loss_tok, loss, saved, workspace, workspace_bytes, stream, false, targets, entropy,
                       target_logprob);
 }
 
 rkl_status rkl_backward(rkl_payload payload, const void* h_s, const void* teacher, const void* W_s, const void* W_t,
                         rkl_dtype dtype, int64_t B, int64_t Sm1, int64_t H, int64_t V, const int32_t* row_idx,
-                        int32_t N, rkl_reduction reduction, const float* saved, const float* grad_loss,
-                        const float* grad_tok, float* dH_s, float* dW_s, void* workspace, size_t workspace_bytes,
-                        void* stream) {
-  return backward_impl(payload, h_s, teacher, W_s, W_t, dtype, B, Sm1, H, V, row_idx, N, reduction, saved, grad_loss,
-                       grad_tok, dH_s, dW_s, workspace, workspace_bytes, stream);
+                        int32_t N, const int32_t* n_dev, rkl_reduction reduction, const float* saved,
+                        const float* grad_loss, const float* grad_tok, float* dH_s, float* dW_s, void* workspace,
+                        size_t workspace_bytes, void* stream) {
+  RKL_NVTX_RANGE();
+  return backward_impl(payload, h_s, teacher, W_s, W_t, dtype, B, Sm1, H, V, row_idx, N, n_dev, reduction, saved,
+                       grad_loss, grad_tok, dH_s, dW_s, workspace, workspace_bytes, stream);
 }
 
 // ---------------------------------------------------------------- teacher per row
 rkl_status rkl_compact_rows_multi(const uint8_t* mask, const int32_t* teacher_idx, int64_t B, int64_t Sm1,
                                   int32_t n_teachers, int32_t* row_idx, int32_t* n_dev, int32_t* counts,
                                   void* stream) {
+  RKL_NVTX_RANGE();
   if (mask == nullptr || teacher_idx == nullptr || row_idx == nullptr || n_dev == nullptr || counts == nullptr)
     return fail(RKL_ERR_NULL, "mask, teacher_idx, row_idx, n_dev and counts must be non-NULL");
   if (!aligned16(row_idx) || !aligned16(teacher_idx))
@@ -969,10 +1022,11 @@ rkl_status rkl_forward_hidden_multi(const void* h_s, const void* h_t, const void
                                    const int32_t* row_idx, int32_t N, rkl_reduction reduction, float* loss_tok,
                                    float* loss, float* saved, void* workspace, size_t workspace_bytes,
                                    void* stream) {
+  RKL_NVTX_RANGE();
   MultiTeacher mt;
   RKL_TRY(make_multi(n_teachers, teacher_idx, counts, N, &mt));
-  return forward_impl(RKL_PAYLOAD_HIDDEN, h_s, h_t, W_s, W_t, dtype, B, Sm1, H, V, row_idx, N, reduction, loss_tok,
-                      loss, saved, workspace, workspace_bytes, stream, false, nullptr, nullptr, nullptr,
+  return forward_impl(RKL_PAYLOAD_HIDDEN, h_s, h_t, W_s, W_t, dtype, B, Sm1, H, V, row_idx, N, nullptr, reduction,
+                      loss_tok, loss, saved, workspace, workspace_bytes, stream, false, nullptr, nullptr, nullptr,
                       n_teachers > 1 ? &mt : nullptr);
 }
 
@@ -982,19 +1036,28 @@ rkl_status rkl_backward_hidden_multi(const void* h_s, const void* h_t, const voi
                                     const int32_t* row_idx, int32_t N, rkl_reduction reduction, const float* saved,
                                     const float* grad_loss, const float* grad_tok, float* dH_s, float* dW_s,
                                     void* workspace, size_t workspace_bytes, void* stream) {
+  RKL_NVTX_RANGE();
   MultiTeacher mt;
   RKL_TRY(make_multi(n_teachers, teacher_idx, counts, N, &mt));
-  return backward_impl(RKL_PAYLOAD_HIDDEN, h_s, h_t, W_s, W_t, dtype, B, Sm1, H, V, row_idx, N, reduction, saved,
-                       grad_loss, grad_tok, dH_s, dW_s, workspace, workspace_bytes, stream,
+  return backward_impl(RKL_PAYLOAD_HIDDEN, h_s, h_t, W_s, W_t, dtype, B, Sm1, H, V, row_idx, N, nullptr, reduction,
+                       saved, grad_loss, grad_tok, dH_s, dW_s, workspace, workspace_bytes, stream,
                        n_teachers > 1 ? &mt : nullptr);
 }
 
 rkl_status rkl_device_error(int32_t* code) {
   if (code == nullptr) return fail(RKL_ERR_NULL, "code is NULL");
   RKL_CUDA(cudaDeviceSynchronize());
-  int v = 0;
+  int v = 0, line_tc = 0, line_small = 0;
   RKL_CUDA(read_and_clear_device_error(&v));
+  RKL_CUDA(read_and_clear_bounds_tc(&line_tc));
+  RKL_CUDA(read_and_clear_bounds_small(&line_small));
+  if (line_tc || line_small) v |= ERR_BOUNDS;
   *code = v;
+  if (line_tc || line_small)
+    return fail(RKL_ERR_DEVICE,
+                "a bounds check failed (tc_kernels.cu line %d, small_kernels.cu line %d; 0 = none); the access was "
+                "skipped and the outputs are invalid (bits 0x%x)",
+                line_tc, line_small, v);
   if (v != 0) return fail(RKL_ERR_DEVICE, "a kernel wait ran out (bits 0x%x); its outputs are invalid", v);
   return RKL_OK;
 }
@@ -1089,6 +1152,7 @@ extern "C" rkl_status rkl_forward_hidden_noalloc(const void* h_s, const void* h_
                                                  rkl_dtype dtype, int64_t B, int64_t Sm1, int64_t H, int64_t V,
                                                  const int32_t* row_idx, int32_t N, rkl_reduction reduction,
                                                  float* loss_tok, float* loss, float* saved, void* stream) {
+  RKL_NVTX_RANGE();
   // Size check first, from the same layout the workspace path uses; nothing
   // on the device is touched when the problem does not fit.
   RKL_TRY(check_common(RKL_PAYLOAD_HIDDEN, dtype, B, Sm1, H, V, N, reduction));
@@ -1102,6 +1166,6 @@ extern "C" rkl_status rkl_forward_hidden_noalloc(const void* h_s, const void* h_
   RKL_TRY(static_scratch_ptr(&scratch));
   // Every region of the scratch that the forward reads is written earlier in
   // the same call, so nothing needs clearing between calls.
-  return forward_impl(RKL_PAYLOAD_HIDDEN, h_s, h_t, W_s, W_t, dtype, B, Sm1, H, V, row_idx, N, reduction, loss_tok,
-                      loss, saved, scratch, kStaticScratchBytes, stream, /*forward_only_workspace=*/true);
+  return forward_impl(RKL_PAYLOAD_HIDDEN, h_s, h_t, W_s, W_t, dtype, B, Sm1, H, V, row_idx, N, nullptr, reduction,
+                      loss_tok, loss, saved, scratch, kStaticScratchBytes, stream, /*forward_only_workspace=*/true);
 }

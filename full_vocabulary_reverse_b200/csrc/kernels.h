@@ -41,6 +41,17 @@ enum KernelId : int {
 
 const char* kernel_name(int id);
 
+// Device error word bits (reported by rkl_device_error).
+enum : int {
+  ERR_WAIT_TMA_EMPTY = 1 << 0,   // producer waited too long for a free smem stage
+  ERR_WAIT_TMA_FULL = 1 << 1,    // MMA issuer waited too long for operands
+  ERR_WAIT_ACC_EMPTY = 1 << 2,   // MMA issuer waited too long for a free accumulator
+  ERR_WAIT_ACC_FULL = 1 << 3,    // epilogue waited too long for an accumulator
+  ERR_WAIT_AUX = 1 << 4,         // epilogue waited too long for an auxiliary tile
+  ERR_WAIT_TEARDOWN = 1 << 5,    // teardown wait for in-flight MMAs ran out
+  ERR_BOUNDS = 1 << 6,           // a bounds check of the RKL_DEBUG build failed
+};
+
 // Records (optionally timed) launches; implemented in api.cu.
 struct LaunchScope {
   LaunchScope(int id, cudaStream_t s);
@@ -49,6 +60,19 @@ struct LaunchScope {
   cudaStream_t stream;
   cudaEvent_t ev0 = nullptr, ev1 = nullptr;
 };
+
+// Trainable-row counts.  Every launcher takes the count as `n` (host) and an
+// optional device pointer `n_dev`.  Without n_dev, n is the exact count.
+// With n_dev, n is an upper bound (grids, tensor maps and workspace regions
+// are sized for it) and the kernels read the live count from *n_dev at run
+// time, clamped to [0, n], so that a step needs no host read of the count.
+#ifdef __CUDACC__
+__device__ __forceinline__ int live_rows(const int32_t* n_dev, int cap, int base = 0) {
+  if (n_dev == nullptr) return cap;
+  const int n = *n_dev - base;
+  return n < 0 ? 0 : (n > cap ? cap : n);
+}
+#endif
 
 constexpr int kBM = 128;       // rows per tile (TMEM lanes)
 constexpr int kFBN = 256;      // vocab columns per fused pair tile
@@ -72,12 +96,12 @@ struct FusedArgs {
   const int32_t* targets;            // stats: target token id per position (nullable)
   float* tlogit;                     // stats: z_s at the target column [n_pad]
   int N, n_pad, H, V, KB;
+  const int32_t* n_dev;              // live row count on the device (nullable: N exact)
+  int n_base;                        // first compacted row of this launch (count offset)
   int IT;                            // 256-column vocab tiles per row tile in this launch
   int vt_base;                       // first 256-column vocab tile of this launch
   int GT;                            // vocab tiles per unit (group)
   int G;                             // units per m-tile = ceil(IT / GT)
-  int MT;                            // row tiles (256 rows each, one per CTA pair)
-  int units_total;                   // MT * G
   int chunk_v0;                      // dz: first vocab column of the chunk
   // Teacher per row: tm_bt covers the stacked heads [tgroups * V, H] and the
   // rows of teacher g occupy [group_row_end[g-1], group_row_end[g]) (whole
@@ -101,7 +125,8 @@ struct GradArgs {
   CUtensorMap tm_dh;      // dHc [N, H] fp32 output (box {32, 32})
   int* tile_counter;      // zeroed before the launch; dynamic tile scheduler
   int N, H, cw, cv0;
-  int MTW, MTH, NT, nW, nH, KBW, KBH;
+  const int32_t* n_dev;   // live row count on the device (nullable: N exact)
+  int MTW, NT, nW, KBH;
   int dh_accumulate;
 };
 
@@ -114,31 +139,40 @@ cudaError_t launch_fused(int ng, bool dz, const FusedArgs& a, int grid, cudaStre
 cudaError_t launch_fused_topk(int variant, const FusedArgs& a, int grid, cudaStream_t s);
 cudaError_t launch_grad(const GradArgs& a, int grid, cudaStream_t s);
 cudaError_t read_and_clear_device_error(int* code);
+// RKL_DEBUG build: line of the first failed bounds check in each kernel file
+// since the last read (0: none), cleared by the read.
+cudaError_t read_and_clear_bounds_tc(int* line);
+cudaError_t read_and_clear_bounds_small(int* line);
 
 // ---------------------------------------------------------------- small kernels
 cudaError_t launch_compact(const uint8_t* mask, long long T, int32_t* row_idx, int32_t* n_dev, cudaStream_t s);
 // hc[p] = h[row_idx[k]] with k = slot_k[p] (slot_k nullptr: k = p); k < 0 gives a zero row.
+// With n_dev, rows [n, n rounded up to 256) of hc are zeroed (the padding of
+// the last pair tile, read by the tensor-core kernels).
+// T: rows of h (the debug build checks every row_idx entry against it).
 cudaError_t launch_gather(const void* h_s, const void* h_t, void* hc_s, void* hc_t, const int32_t* row_idx,
-                          const int32_t* slot_k, int n_rows, int row_bytes, cudaStream_t s);
-cudaError_t launch_teacher_lse(const void* logits, bool bf16, const int32_t* row_idx, int N, int V,
-                               long long pitch, float* lse_t, cudaStream_t s);
+                          const int32_t* slot_k, int n_rows, const int32_t* n_dev, int row_bytes, long long T,
+                          cudaStream_t s);
+// rows: rows of the logits (debug-build check of row_idx).
+cudaError_t launch_teacher_lse(const void* logits, bool bf16, const int32_t* row_idx, int N, const int32_t* n_dev,
+                               int V, long long pitch, float* lse_t, long long rows, cudaStream_t s);
 // Statistics rows p < n_rows are written to compact row slot_k[p] (nullptr: p; < 0: skipped).
-cudaError_t launch_combine(const float* part, int S, int n_pad, int n_rows, bool teacher_from_part,
-                           const float* lse_t_ext, const float* tlogit, float* saved, float* ent_rows,
-                           float* lp_rows, const int32_t* slot_k, cudaStream_t s);
-cudaError_t launch_scatter_loss(const float* saved, const int32_t* row_idx, int N, long long T, float* loss_tok,
-                                cudaStream_t s);
+cudaError_t launch_combine(const float* part, int S, int n_pad, int n_rows, const int32_t* n_dev,
+                           bool teacher_from_part, const float* lse_t_ext, const float* tlogit, float* saved,
+                           float* ent_rows, float* lp_rows, const int32_t* slot_k, cudaStream_t s);
+cudaError_t launch_scatter_loss(const float* saved, const int32_t* row_idx, int N, const int32_t* n_dev, long long T,
+                                float* loss_tok, cudaStream_t s);
 // out[t] = rows[k] where t = row_idx[k], else 0 (per-token [B, S-1] scatter)
-cudaError_t launch_scatter_rows(const float* rows, const int32_t* row_idx, int N, long long T, float* out,
-                                cudaStream_t s);
-cudaError_t launch_reduce(const float* saved, const int32_t* row_idx, int N, int B, int Sm1, int reduction,
-                          float* loss, cudaStream_t s);
-cudaError_t launch_row_weights(const float* saved, const int32_t* row_idx, int N, int n_pad, int B, int Sm1,
-                               int reduction, const float* grad_loss, const float* grad_tok, float* rowc,
-                               const int32_t* slot_k, cudaStream_t s);
+cudaError_t launch_scatter_rows(const float* rows, const int32_t* row_idx, int N, const int32_t* n_dev, long long T,
+                                float* out, cudaStream_t s);
+cudaError_t launch_reduce(const float* saved, const int32_t* row_idx, int N, const int32_t* n_dev, int B, int Sm1,
+                          int reduction, float* loss, cudaStream_t s);
+cudaError_t launch_row_weights(const float* saved, const int32_t* row_idx, int N, const int32_t* n_dev, int n_pad,
+                               int B, int Sm1, int reduction, const float* grad_loss, const float* grad_tok,
+                               float* rowc, const int32_t* slot_k, cudaStream_t s);
 // dH_s[row_idx[k]] = dHc[k_slot[k]] (k_slot nullptr: k), all other rows 0.
-cudaError_t launch_scatter_dh(const float* dHc, const int32_t* row_idx, const int32_t* k_slot, int N, long long T,
-                              int H, float* dH_s, cudaStream_t s);
+cudaError_t launch_scatter_dh(const float* dHc, const int32_t* row_idx, const int32_t* k_slot, int N,
+                              const int32_t* n_dev, long long T, int H, float* dH_s, cudaStream_t s);
 // Trainable rows per teacher: counts[g] for g < n_teachers, counts[n_teachers] =
 // trainable rows whose index is outside [0, n_teachers).  counts must be zeroed.
 cudaError_t launch_count_teachers(const uint8_t* mask, const int32_t* teacher_idx, long long T, int n_teachers,
@@ -152,23 +186,27 @@ struct TeacherSlots {
 // slot_k[p] = k (slot_k pre-filled with -1 for padding), k_slot[k] = p.
 cudaError_t launch_build_slots(const int32_t* row_idx, const int32_t* teacher_idx, int N, const TeacherSlots& ts,
                                int32_t* slot_k, int32_t* k_slot, cudaStream_t s);
-cudaError_t launch_pair_fwd(const void* zs, const void* zt, bool bf16, const int32_t* row_idx, int N, int V,
-                            float* saved, cudaStream_t s);
-cudaError_t launch_pair_bwd(const void* zs, const void* zt, bool bf16, const int32_t* row_idx, int N, int n_pad,
-                            long long T, int V, const float* rowc, void* dz, cudaStream_t s);
+cudaError_t launch_pair_fwd(const void* zs, const void* zt, bool bf16, const int32_t* row_idx, int N,
+                            const int32_t* n_dev, int V, float* saved, cudaStream_t s);
+cudaError_t launch_pair_bwd(const void* zs, const void* zt, bool bf16, const int32_t* row_idx, int N,
+                            const int32_t* n_dev, int n_pad, long long T, int V, const float* rowc, void* dz,
+                            cudaStream_t s);
 
 // Top-k estimator with both sides as logits (topk_kernels.cu).  saved [N, 3]
 // (lse_s, lse_t, estimate), saved_tk [N, 4] (C, a, K* bits, v_last bits).
 // Logit rows: zs + row * zpitch with row = row_idx[k] (local = false) or the
 // block-local k (local = true); the sampled token is targets[row_idx[k]].
+// The rows of this launch are compacted rows n_base .. n_base + N - 1 (with
+// n_dev: as many of them as are live).
 cudaError_t launch_topk_fwd(const void* zs, const void* zt, bool bf16, const int32_t* row_idx,
-                            const int32_t* targets, int N, int V, long long k, float* saved, float* saved_tk,
-                            long long zpitch, bool local, cudaStream_t s);
+                            const int32_t* targets, int N, const int32_t* n_dev, int n_base, int V, long long k,
+                            float* saved, float* saved_tk, long long zpitch, bool local, cudaStream_t s);
 cudaError_t launch_topk_rowk(const float* saved, const float* saved_tk, const int32_t* row_idx,
-                             const int32_t* targets, int N, int n_pad, float* rowk, cudaStream_t s);
+                             const int32_t* targets, int N, const int32_t* n_dev, int n_pad, float* rowk,
+                             cudaStream_t s);
 cudaError_t launch_topk_bwd(const void* zs, const void* zt, bool bf16, const int32_t* row_idx,
-                            const int32_t* targets, int N, int n_pad, long long T, int V, const float* saved,
-                            const float* saved_tk, const float* rowc, void* dz, cudaStream_t s);
+                            const int32_t* targets, int N, const int32_t* n_dev, int n_pad, long long T, int V,
+                            const float* saved, const float* saved_tk, const float* rowc, void* dz, cudaStream_t s);
 
 // ---------------------------------------------------------------- fp32 CUDA-core path
 struct SimtArgs {
@@ -181,15 +219,17 @@ struct SimtArgs {
   const int32_t* row_idx; const int32_t* targets; float* tlogit;
   float* dz;                          // dz chunk [N, cw] fp32
   int N, n_pad, H, V, S, IT, vt_base, chunk_v0, cw;
+  const int32_t* n_dev;               // live row count on the device (nullable: N exact)
   int ng;
   int tgroups;                        // > 1: bt is the stacked teacher heads [tgroups, V, H]
   int group_row_end[kMaxTeachers];    // rows of teacher g end here (multiples of 32)
 };
 constexpr int kSimtBN = 32;
 cudaError_t launch_simt_fused(bool dz, const SimtArgs& a, dim3 grid, cudaStream_t s);
-// C[M, Nc] (+)= sum_k A(m, k) B(k, n); A(m,k) = A[m*sam + k*sak], B(k,n) = B[k*sbk + n*sbn]
+// C[M, Nc] (+)= sum_k A(m, k) B(k, n); A(m,k) = A[m*sam + k*sak], B(k,n) = B[k*sbk + n*sbn].
+// With n_dev, the row count bounds M (live_dim = 1) or K (live_dim = 2).
 cudaError_t launch_simt_gemm(const float* A, long long sam, long long sak, const float* B, long long sbk,
                              long long sbn, float* C, long long ldc, int M, int Nc, int K, int accumulate,
-                             cudaStream_t s);
+                             const int32_t* n_dev, int live_dim, cudaStream_t s);
 
 }  // namespace rkl

@@ -19,15 +19,17 @@ __global__ void __launch_bounds__(256) simt_fused_kernel(const SimtArgs a) {
   __shared__ float As[TB][TB + 1], At[TB][TB + 1], Bs[TB][TB + 1], Bt[TB][TB + 1];
   __shared__ float Zs[TB][TB + 1], Zt[TB][TB + 1];
   const int tid = threadIdx.x, tx = tid & 31, ty = tid >> 5;  // ty in 0..7
+  const int N = live_rows(a.n_dev, a.N);  // rows in use (exact, or read from the device)
 
   int u0, u1, split = 0;
   if (!DZ) {
     const int mt = blockIdx.x;
+    if (mt * TB >= N) return;
     split = blockIdx.y;
     u0 = mt * a.IT + static_cast<int>((static_cast<long long>(split) * a.IT) / a.S);
     u1 = mt * a.IT + static_cast<int>((static_cast<long long>(split + 1) * a.IT) / a.S);
   } else {
-    const int MT = (a.N + TB - 1) / TB;
+    const int MT = (N + TB - 1) / TB;
     const int total = MT * a.IT;
     u0 = static_cast<int>((static_cast<long long>(blockIdx.x) * total) / gridDim.x);
     u1 = static_cast<int>((static_cast<long long>(blockIdx.x + 1) * total) / gridDim.x);
@@ -37,7 +39,7 @@ __global__ void __launch_bounds__(256) simt_fused_kernel(const SimtArgs a) {
   int tgt = -1;
   if (!DZ && tid < TB && a.targets != nullptr) {
     const int r = (u0 / a.IT) * TB + tid;
-    if (r < a.N) tgt = a.targets[a.row_idx[r]];
+    if (r < N) tgt = a.targets[a.row_idx[r]];
   }
   for (int u = u0; u < u1; ++u) {
     const int m0 = (u / a.IT) * TB;
@@ -54,10 +56,10 @@ __global__ void __launch_bounds__(256) simt_fused_kernel(const SimtArgs a) {
       for (int e = tid; e < TB * TB; e += 256) {
         const int r = e / TB, kk = e % TB;
         const bool kin = k0 + kk < a.H;
-        As[r][kk] = (m0 + r < a.N && kin) ? a.as[static_cast<long long>(m0 + r) * a.H + k0 + kk] : 0.f;
+        As[r][kk] = (m0 + r < N && kin) ? a.as[static_cast<long long>(m0 + r) * a.H + k0 + kk] : 0.f;
         Bs[r][kk] = (v0 + r < a.V && kin) ? a.bs[static_cast<long long>(v0 + r) * a.H + k0 + kk] : 0.f;
         if (a.ng == 2) {
-          At[r][kk] = (m0 + r < a.N && kin) ? a.at[static_cast<long long>(m0 + r) * a.H + k0 + kk] : 0.f;
+          At[r][kk] = (m0 + r < N && kin) ? a.at[static_cast<long long>(m0 + r) * a.H + k0 + kk] : 0.f;
           Bt[r][kk] = (v0 + r < a.V && kin) ? bt[static_cast<long long>(v0 + r) * a.H + k0 + kk] : 0.f;
         }
       }
@@ -82,7 +84,7 @@ __global__ void __launch_bounds__(256) simt_fused_kernel(const SimtArgs a) {
         Zt[r][tx] = ct[i];
       } else {
         float z = 0.f;
-        if (m0 + r < a.N && v0 + tx < a.V) {
+        if (m0 + r < N && v0 + tx < a.V) {
           const long long tr = a.teacher_rows ? a.teacher_rows[m0 + r] : (m0 + r);
           z = a.teacher[tr * a.teacher_pitch + v0 + tx];
         }
@@ -116,7 +118,7 @@ __global__ void __launch_bounds__(256) simt_fused_kernel(const SimtArgs a) {
         }
         const unsigned d = static_cast<unsigned>(tgt - v0);
         if (tgt >= 0 && d < static_cast<unsigned>(TB)) a.tlogit[m0 + r] = Zs[r][d];
-      } else if (m0 + r < a.N) {
+      } else if (m0 + r < N) {
         const float lse2 = a.rowc[m0 + r], cst = a.rowc[a.n_pad + m0 + r], g = a.rowc[2 * a.n_pad + m0 + r];
         float* out = a.dz + static_cast<long long>(m0 + r) * a.cw + (v0 - a.chunk_v0);
         for (int j = 0; j < TB && v0 - a.chunk_v0 + j < a.cw; ++j) {
@@ -142,10 +144,14 @@ __global__ void __launch_bounds__(256) simt_fused_kernel(const SimtArgs a) {
 __global__ void __launch_bounds__(256) simt_gemm_kernel(const float* __restrict__ A, long long sam, long long sak,
                                                         const float* __restrict__ B, long long sbk, long long sbn,
                                                         float* __restrict__ C, long long ldc, int M, int Nc, int K,
-                                                        int accumulate) {
+                                                        int accumulate, const int32_t* __restrict__ n_dev,
+                                                        int live_dim) {
   __shared__ float as[16][64 + 1], bs[16][64 + 1];
   const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
   const int m0 = blockIdx.y * 64, n0 = blockIdx.x * 64;
+  if (live_dim == 1) M = live_rows(n_dev, M);
+  if (live_dim == 2) K = live_rows(n_dev, K);
+  if (m0 >= M) return;
   float acc[4][4] = {};
   for (int k0 = 0; k0 < K; k0 += 16) {
     for (int e = tid; e < 16 * 64; e += 256) {
@@ -187,10 +193,10 @@ cudaError_t launch_simt_fused(bool dz, const SimtArgs& a, dim3 grid, cudaStream_
 
 cudaError_t launch_simt_gemm(const float* A, long long sam, long long sak, const float* B, long long sbk,
                              long long sbn, float* C, long long ldc, int M, int Nc, int K, int accumulate,
-                             cudaStream_t s) {
+                             const int32_t* n_dev, int live_dim, cudaStream_t s) {
   LaunchScope scope(K_GRAD_SIMT, s);
   dim3 grid((Nc + 63) / 64, (M + 63) / 64);
-  simt_gemm_kernel<<<grid, 256, 0, s>>>(A, sam, sak, B, sbk, sbn, C, ldc, M, Nc, K, accumulate);
+  simt_gemm_kernel<<<grid, 256, 0, s>>>(A, sam, sak, B, sbk, sbn, C, ldc, M, Nc, K, accumulate, n_dev, live_dim);
   return cudaGetLastError();
 }
 

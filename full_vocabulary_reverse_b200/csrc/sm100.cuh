@@ -9,17 +9,9 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
-namespace rkl {
+#include "kernels.h"  // device error word bits
 
-// Device error word bits (reported by rkl_device_error).
-enum : int {
-  ERR_WAIT_TMA_EMPTY = 1 << 0,   // producer waited too long for a free smem stage
-  ERR_WAIT_TMA_FULL = 1 << 1,    // MMA issuer waited too long for operands
-  ERR_WAIT_ACC_EMPTY = 1 << 2,   // MMA issuer waited too long for a free accumulator
-  ERR_WAIT_ACC_FULL = 1 << 3,    // epilogue waited too long for an accumulator
-  ERR_WAIT_AUX = 1 << 4,         // epilogue waited too long for an auxiliary tile
-  ERR_WAIT_TEARDOWN = 1 << 5,    // teardown wait for in-flight MMAs ran out
-};
+namespace rkl {
 
 // A wait gives up after this many nanoseconds of %globaltimer.
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s

@@ -11,10 +11,13 @@
 
 #include <cfloat>
 
+#include "bounds.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
 
 namespace rkl {
+RKL_DEFINE_BOUNDS_READER(read_and_clear_bounds_small)
+
 namespace {
 
 __device__ __forceinline__ int lower_bound_i32(const int32_t* a, int n, long long key) {
@@ -81,15 +84,21 @@ __global__ void __launch_bounds__(1024) compact_kernel(const uint8_t* __restrict
 // --------------------------------------------------------------------- S2
 // hc[p] = h[row_idx[k]] for p < n_rows, k = slot_k[p] (or p without a slot
 // map); a slot with k < 0 (padding between teacher groups) becomes a zero
-// row.  blockIdx.y selects student / teacher.
+// row.  With a device row count n, rows [n, n rounded up to 256) -- the rest
+// of the last pair tile, which the tensor-core kernels read -- become zero
+// rows too.  blockIdx.y selects student / teacher.
 __global__ void __launch_bounds__(256) gather_kernel(const uint8_t* __restrict__ h_s, const uint8_t* __restrict__ h_t,
                                                      uint8_t* __restrict__ hc_s, uint8_t* __restrict__ hc_t,
                                                      const int32_t* __restrict__ row_idx,
-                                                     const int32_t* __restrict__ slot_k, int n_rows, int row_bytes) {
+                                                     const int32_t* __restrict__ slot_k, int n_rows,
+                                                     const int32_t* __restrict__ n_dev, int row_bytes, long long T) {
   const uint8_t* src = blockIdx.y == 0 ? h_s : h_t;
   uint8_t* dst = blockIdx.y == 0 ? hc_s : hc_t;
-  for (int p = blockIdx.x; p < n_rows; p += gridDim.x) {
-    const int k = slot_k ? slot_k[p] : p;
+  const int n_live = live_rows(n_dev, n_rows);
+  const int n_end = n_dev ? ((n_live + 2 * kBM - 1) / (2 * kBM)) * (2 * kBM) : n_rows;
+  for (int p = blockIdx.x; p < n_end; p += gridDim.x) {
+    int k = p < n_live ? (slot_k ? slot_k[p] : p) : -1;
+    if (k >= 0 && !RKL_BOUNDS(row_idx[k] >= 0 && row_idx[k] < T)) k = -1;  // (debug build) a zero row instead
     uint8_t* d = dst + static_cast<long long>(p) * row_bytes;
     if (k < 0) {
       for (int i = threadIdx.x; i < row_bytes / 4; i += blockDim.x) reinterpret_cast<uint32_t*>(d)[i] = 0u;
@@ -157,13 +166,15 @@ __device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 x) { return _
 
 template <typename T>
 __global__ void __launch_bounds__(256) teacher_lse_kernel(const T* __restrict__ logits,
-                                                          const int32_t* __restrict__ row_idx, int N, int V,
-                                                          long long pitch, float* __restrict__ lse_t) {
+                                                          const int32_t* __restrict__ row_idx, int N,
+                                                          const int32_t* __restrict__ n_dev, int V, long long pitch,
+                                                          float* __restrict__ lse_t, long long rows) {
   constexpr int VEC = 16 / sizeof(T);
   constexpr int UNROLL = 4;
   const int k = blockIdx.x;
-  if (k >= N) return;
+  if (k >= live_rows(n_dev, N)) return;
   const long long r = row_idx ? row_idx[k] : k;
+  if (!RKL_BOUNDS(r >= 0 && r < rows)) return;
   const T* row = logits + r * pitch;
   float m = -INFINITY, s = 0.f;
   const bool vec_ok = ((reinterpret_cast<uintptr_t>(row) & 15) == 0);
@@ -262,15 +273,16 @@ __device__ __forceinline__ void merge3(Stat3& a, const Stat3& b) {
 // Statistics row k (a slot of the teacher-grouped layout when slot_k is
 // given) is written to compact row out = slot_k[k]; padding slots are skipped.
 __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ part, int S, int n_pad, int n_rows,
+                                                      const int32_t* __restrict__ n_dev,
                                                       int teacher_from_part, const float* __restrict__ lse_ext,
                                                       const float* __restrict__ tlogit, float* __restrict__ saved,
                                                       float* __restrict__ ent_rows, float* __restrict__ lp_rows,
                                                       const int32_t* __restrict__ slot_k) {
   const int lane = threadIdx.x & 31;
   const int k = blockIdx.x * 8 + (threadIdx.x >> 5);
-  if (k >= n_rows) return;
+  if (k >= live_rows(n_dev, n_rows)) return;
   const int out = slot_k ? slot_k[k] : k;
-  if (out < 0) return;
+  if (out < 0 || !RKL_BOUNDS(out < n_pad)) return;
   Stat3 s{-INFINITY, 0.f, 0.f, 0.f}, t{-INFINITY, 0.f, 0.f, 0.f};
   for (int g = lane; g < S; g += 32) {
     const float* b = part + static_cast<size_t>(g) * kStatVals * n_pad + k;
@@ -298,18 +310,20 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
 
 // out[t] = rows[k] if t = row_idx[k] else exactly 0.
 __global__ void scatter_rows_kernel(const float* __restrict__ rows, const int32_t* __restrict__ row_idx, int N,
-                                    long long T, float* __restrict__ out) {
+                                    const int32_t* __restrict__ n_dev, long long T, float* __restrict__ out) {
   const long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (t >= T) return;
+  N = live_rows(n_dev, N);
   const int k = lower_bound_i32(row_idx, N, t);
   out[t] = (k < N && row_idx[k] == t) ? rows[k] : 0.f;
 }
 
 // loss_tok[t] = L of t if t is trainable else exactly 0.
 __global__ void scatter_loss_kernel(const float* __restrict__ saved, const int32_t* __restrict__ row_idx, int N,
-                                    long long T, float* __restrict__ loss_tok) {
+                                    const int32_t* __restrict__ n_dev, long long T, float* __restrict__ loss_tok) {
   const long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (t >= T) return;
+  N = live_rows(n_dev, N);
   const int k = lower_bound_i32(row_idx, N, t);
   loss_tok[t] = (k < N && row_idx[k] == t) ? saved[3 * k + 2] : 0.f;
 }
@@ -330,9 +344,11 @@ __device__ __forceinline__ double block_sum_1024(double v, double* sh) {
 // Scalar loss: token mean sum_k L_k / N, or nested mean over sequences with
 // n_b > 0 of sum_{k in b} L_k / n_b.  Fixed summation order (deterministic).
 __global__ void __launch_bounds__(1024) reduce_kernel(const float* __restrict__ saved,
-                                                      const int32_t* __restrict__ row_idx, int N, int B, int Sm1,
+                                                      const int32_t* __restrict__ row_idx, int N,
+                                                      const int32_t* __restrict__ n_dev, int B, int Sm1,
                                                       int reduction, float* __restrict__ loss) {
   __shared__ double sh[32];
+  N = live_rows(n_dev, N);
   if (reduction == 1) {
     double acc = 0.0;
     for (int k = threadIdx.x; k < N; k += 1024) acc += saved[3 * k + 2];
@@ -361,13 +377,15 @@ __global__ void __launch_bounds__(1024) reduce_kernel(const float* __restrict__ 
 // rowc[1] = lse_t - lse_s - L, rowc[2] = g = dLoss/dL_k.  Padding rows get 0.
 // With a slot map, row p of rowc belongs to compact row slot_k[p].
 __global__ void __launch_bounds__(256) row_weights_kernel(const float* __restrict__ saved,
-                                                          const int32_t* __restrict__ row_idx, int N, int n_pad,
+                                                          const int32_t* __restrict__ row_idx, int N,
+                                                          const int32_t* __restrict__ n_dev, int n_pad,
                                                           int B, int Sm1, int reduction,
                                                           const float* __restrict__ grad_loss,
                                                           const float* __restrict__ grad_tok,
                                                           float* __restrict__ rowc,
                                                           const int32_t* __restrict__ slot_k) {
   __shared__ int b_eff_sh;
+  N = live_rows(n_dev, N);
   if (threadIdx.x == 0) b_eff_sh = 0;
   __syncthreads();
   if (reduction == 2) {
@@ -386,6 +404,7 @@ __global__ void __launch_bounds__(256) row_weights_kernel(const float* __restric
   float c0 = 0.f, c1 = 0.f, c2 = 0.f;
   if (k >= 0 && k < N) {
     const int row = row_idx[k];
+    if (!RKL_BOUNDS(row >= 0 && row < B * Sm1)) return;
     const float lse_s = saved[3 * k], lse_t = saved[3 * k + 1], L = saved[3 * k + 2];
     float w = 0.f;
     if (reduction == 1) {
@@ -412,8 +431,10 @@ __global__ void __launch_bounds__(256) row_weights_kernel(const float* __restric
 // else exact zeros.
 __global__ void __launch_bounds__(256) scatter_dh_kernel(const float* __restrict__ dHc,
                                                          const int32_t* __restrict__ row_idx,
-                                                         const int32_t* __restrict__ k_slot, int N, long long T,
-                                                         int H, float* __restrict__ dH_s) {
+                                                         const int32_t* __restrict__ k_slot, int N,
+                                                         const int32_t* __restrict__ n_dev, long long T, int H,
+                                                         float* __restrict__ dH_s) {
+  N = live_rows(n_dev, N);
   for (long long t = blockIdx.x; t < T; t += gridDim.x) {
     const int k = lower_bound_i32(row_idx, N, t);
     const int src = (k < N && row_idx[k] == t) ? (k_slot ? k_slot[k] : k) : -1;
@@ -581,11 +602,12 @@ __device__ __forceinline__ void pair_update(PairStat& st, const float* xs, const
 
 template <typename T>
 __global__ void __launch_bounds__(256) pair_fwd_kernel(const T* __restrict__ zs_all, const T* __restrict__ zt_all,
-                                                       const int32_t* __restrict__ row_idx, int N, int V,
+                                                       const int32_t* __restrict__ row_idx, int N,
+                                                       const int32_t* __restrict__ n_dev, int V,
                                                        float* __restrict__ saved) {
   constexpr int VEC = 16 / sizeof(T);
   const int k = blockIdx.x;
-  if (k >= N) return;
+  if (k >= live_rows(n_dev, N)) return;
   const long long r = row_idx[k];
   const T* zs = zs_all + r * V;
   const T* zt = zt_all + r * V;
@@ -665,10 +687,12 @@ __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) { return
 // dz[t, :] = g p_s ((z_s - z_t) + lse_t - lse_s - L) for trainable t, else 0.
 template <typename T>
 __global__ void __launch_bounds__(256) pair_bwd_kernel(const T* __restrict__ zs_all, const T* __restrict__ zt_all,
-                                                       const int32_t* __restrict__ row_idx, int N, int n_pad, int V,
+                                                       const int32_t* __restrict__ row_idx, int N,
+                                                       const int32_t* __restrict__ n_dev, int n_pad, int V,
                                                        const float* __restrict__ rowc, T* __restrict__ dz_all) {
   constexpr int VEC = 16 / sizeof(T);
   const long long t = blockIdx.x;
+  N = live_rows(n_dev, N);
   const int k = lower_bound_i32(row_idx, N, t);
   const bool hit = k < N && row_idx[k] == t;
   const T* zs = zs_all + t * V;
@@ -710,73 +734,76 @@ cudaError_t launch_compact(const uint8_t* mask, long long T, int32_t* row_idx, i
 }
 
 cudaError_t launch_gather(const void* h_s, const void* h_t, void* hc_s, void* hc_t, const int32_t* row_idx,
-                          const int32_t* slot_k, int n_rows, int row_bytes, cudaStream_t s) {
+                          const int32_t* slot_k, int n_rows, const int32_t* n_dev, int row_bytes, long long T,
+                          cudaStream_t s) {
   if (n_rows <= 0) return cudaSuccess;
   LaunchScope scope(K_GATHER, s);
-  dim3 grid(n_rows < 65535 ? n_rows : 65535, h_t ? 2 : 1);
+  const int span = n_dev ? ((n_rows + 2 * kBM - 1) / (2 * kBM)) * (2 * kBM) : n_rows;
+  dim3 grid(span < 65535 ? span : 65535, h_t ? 2 : 1);
   gather_kernel<<<grid, 256, 0, s>>>(static_cast<const uint8_t*>(h_s), static_cast<const uint8_t*>(h_t),
                                      static_cast<uint8_t*>(hc_s), static_cast<uint8_t*>(hc_t), row_idx, slot_k,
-                                     n_rows, row_bytes);
+                                     n_rows, n_dev, row_bytes, T);
   return cudaGetLastError();
 }
 
-cudaError_t launch_teacher_lse(const void* logits, bool bf16, const int32_t* row_idx, int N, int V, long long pitch,
-                               float* lse_t, cudaStream_t s) {
+cudaError_t launch_teacher_lse(const void* logits, bool bf16, const int32_t* row_idx, int N, const int32_t* n_dev,
+                               int V, long long pitch, float* lse_t, long long rows, cudaStream_t s) {
   if (N <= 0) return cudaSuccess;
   LaunchScope scope(K_TEACHER_LSE, s);
   if (bf16)
-    teacher_lse_kernel<__nv_bfloat16><<<N, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(logits), row_idx, N, V,
-                                                         pitch, lse_t);
+    teacher_lse_kernel<__nv_bfloat16><<<N, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(logits), row_idx, N, n_dev,
+                                                         V, pitch, lse_t, rows);
   else
-    teacher_lse_kernel<float><<<N, 256, 0, s>>>(static_cast<const float*>(logits), row_idx, N, V, pitch, lse_t);
+    teacher_lse_kernel<float><<<N, 256, 0, s>>>(static_cast<const float*>(logits), row_idx, N, n_dev, V, pitch,
+                                                lse_t, rows);
   return cudaGetLastError();
 }
 
-cudaError_t launch_combine(const float* part, int S, int n_pad, int n_rows, bool teacher_from_part,
-                           const float* lse_ext, const float* tlogit, float* saved, float* ent_rows, float* lp_rows,
-                           const int32_t* slot_k, cudaStream_t s) {
+cudaError_t launch_combine(const float* part, int S, int n_pad, int n_rows, const int32_t* n_dev,
+                           bool teacher_from_part, const float* lse_ext, const float* tlogit, float* saved,
+                           float* ent_rows, float* lp_rows, const int32_t* slot_k, cudaStream_t s) {
   if (n_rows <= 0) return cudaSuccess;
   LaunchScope scope(K_COMBINE, s);
-  combine_kernel<<<(n_rows + 7) / 8, 256, 0, s>>>(part, S, n_pad, n_rows, teacher_from_part ? 1 : 0, lse_ext, tlogit,
-                                                  saved, ent_rows, lp_rows, slot_k);
+  combine_kernel<<<(n_rows + 7) / 8, 256, 0, s>>>(part, S, n_pad, n_rows, n_dev, teacher_from_part ? 1 : 0, lse_ext,
+                                                  tlogit, saved, ent_rows, lp_rows, slot_k);
   return cudaGetLastError();
 }
 
-cudaError_t launch_scatter_rows(const float* rows, const int32_t* row_idx, int N, long long T, float* out,
-                                cudaStream_t s) {
+cudaError_t launch_scatter_rows(const float* rows, const int32_t* row_idx, int N, const int32_t* n_dev, long long T,
+                                float* out, cudaStream_t s) {
   LaunchScope scope(K_SCATTER_LOSS, s);
-  scatter_rows_kernel<<<static_cast<unsigned>((T + 255) / 256), 256, 0, s>>>(rows, row_idx, N, T, out);
+  scatter_rows_kernel<<<static_cast<unsigned>((T + 255) / 256), 256, 0, s>>>(rows, row_idx, N, n_dev, T, out);
   return cudaGetLastError();
 }
 
-cudaError_t launch_scatter_loss(const float* saved, const int32_t* row_idx, int N, long long T, float* loss_tok,
-                                cudaStream_t s) {
+cudaError_t launch_scatter_loss(const float* saved, const int32_t* row_idx, int N, const int32_t* n_dev, long long T,
+                                float* loss_tok, cudaStream_t s) {
   LaunchScope scope(K_SCATTER_LOSS, s);
-  scatter_loss_kernel<<<static_cast<unsigned>((T + 255) / 256), 256, 0, s>>>(saved, row_idx, N, T, loss_tok);
+  scatter_loss_kernel<<<static_cast<unsigned>((T + 255) / 256), 256, 0, s>>>(saved, row_idx, N, n_dev, T, loss_tok);
   return cudaGetLastError();
 }
 
-cudaError_t launch_reduce(const float* saved, const int32_t* row_idx, int N, int B, int Sm1, int reduction,
-                          float* loss, cudaStream_t s) {
+cudaError_t launch_reduce(const float* saved, const int32_t* row_idx, int N, const int32_t* n_dev, int B, int Sm1,
+                          int reduction, float* loss, cudaStream_t s) {
   LaunchScope scope(K_REDUCE, s);
-  reduce_kernel<<<1, 1024, 0, s>>>(saved, row_idx, N, B, Sm1, reduction, loss);
+  reduce_kernel<<<1, 1024, 0, s>>>(saved, row_idx, N, n_dev, B, Sm1, reduction, loss);
   return cudaGetLastError();
 }
 
-cudaError_t launch_row_weights(const float* saved, const int32_t* row_idx, int N, int n_pad, int B, int Sm1,
-                               int reduction, const float* grad_loss, const float* grad_tok, float* rowc,
-                               const int32_t* slot_k, cudaStream_t s) {
+cudaError_t launch_row_weights(const float* saved, const int32_t* row_idx, int N, const int32_t* n_dev, int n_pad,
+                               int B, int Sm1, int reduction, const float* grad_loss, const float* grad_tok,
+                               float* rowc, const int32_t* slot_k, cudaStream_t s) {
   LaunchScope scope(K_ROW_WEIGHTS, s);
-  row_weights_kernel<<<(n_pad + 255) / 256, 256, 0, s>>>(saved, row_idx, N, n_pad, B, Sm1, reduction, grad_loss,
-                                                         grad_tok, rowc, slot_k);
+  row_weights_kernel<<<(n_pad + 255) / 256, 256, 0, s>>>(saved, row_idx, N, n_dev, n_pad, B, Sm1, reduction,
+                                                         grad_loss, grad_tok, rowc, slot_k);
   return cudaGetLastError();
 }
 
-cudaError_t launch_scatter_dh(const float* dHc, const int32_t* row_idx, const int32_t* k_slot, int N, long long T,
-                              int H, float* dH_s, cudaStream_t s) {
+cudaError_t launch_scatter_dh(const float* dHc, const int32_t* row_idx, const int32_t* k_slot, int N,
+                              const int32_t* n_dev, long long T, int H, float* dH_s, cudaStream_t s) {
   LaunchScope scope(K_SCATTER_DH, s);
   const long long blocks = T < 65535 * 8 ? T : 65535 * 8;
-  scatter_dh_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(dHc, row_idx, k_slot, N, T, H, dH_s);
+  scatter_dh_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(dHc, row_idx, k_slot, N, n_dev, T, H, dH_s);
   return cudaGetLastError();
 }
 
@@ -801,31 +828,33 @@ cudaError_t launch_build_slots(const int32_t* row_idx, const int32_t* teacher_id
 
 namespace rkl {
 
-cudaError_t launch_pair_fwd(const void* zs, const void* zt, bool bf16, const int32_t* row_idx, int N, int V,
-                            float* saved, cudaStream_t s) {
+cudaError_t launch_pair_fwd(const void* zs, const void* zt, bool bf16, const int32_t* row_idx, int N,
+                            const int32_t* n_dev, int V, float* saved, cudaStream_t s) {
   if (N <= 0) return cudaSuccess;
   LaunchScope scope(K_PAIR_FWD, s);
   if (bf16)
     pair_fwd_kernel<__nv_bfloat16><<<N, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(zs),
-                                                      static_cast<const __nv_bfloat16*>(zt), row_idx, N, V, saved);
+                                                      static_cast<const __nv_bfloat16*>(zt), row_idx, N, n_dev, V,
+                                                      saved);
   else
     pair_fwd_kernel<float><<<N, 256, 0, s>>>(static_cast<const float*>(zs), static_cast<const float*>(zt), row_idx,
-                                             N, V, saved);
+                                             N, n_dev, V, saved);
   return cudaGetLastError();
 }
 
-cudaError_t launch_pair_bwd(const void* zs, const void* zt, bool bf16, const int32_t* row_idx, int N, int n_pad,
-                            long long T, int V, const float* rowc, void* dz, cudaStream_t s) {
+cudaError_t launch_pair_bwd(const void* zs, const void* zt, bool bf16, const int32_t* row_idx, int N,
+                            const int32_t* n_dev, int n_pad, long long T, int V, const float* rowc, void* dz,
+                            cudaStream_t s) {
   if (T <= 0) return cudaSuccess;
   LaunchScope scope(K_PAIR_BWD, s);
   if (bf16)
     pair_bwd_kernel<__nv_bfloat16><<<static_cast<unsigned>(T), 256, 0, s>>>(
-        static_cast<const __nv_bfloat16*>(zs), static_cast<const __nv_bfloat16*>(zt), row_idx, N, n_pad, V, rowc,
-        static_cast<__nv_bfloat16*>(dz));
+        static_cast<const __nv_bfloat16*>(zs), static_cast<const __nv_bfloat16*>(zt), row_idx, N, n_dev, n_pad, V,
+        rowc, static_cast<__nv_bfloat16*>(dz));
   else
     pair_bwd_kernel<float><<<static_cast<unsigned>(T), 256, 0, s>>>(static_cast<const float*>(zs),
-                                                                    static_cast<const float*>(zt), row_idx, N, n_pad,
-                                                                    V, rowc, static_cast<float*>(dz));
+                                                                    static_cast<const float*>(zt), row_idx, N, n_dev,
+                                                                    n_pad, V, rowc, static_cast<float*>(dz));
   return cudaGetLastError();
 }
 

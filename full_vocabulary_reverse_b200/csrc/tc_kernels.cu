@@ -28,12 +28,15 @@
 // columns).  Warp 2 also allocates / frees TMEM.
 #include <cuda_bf16.h>
 
+#include "bounds.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
 
 namespace rkl {
 
 __device__ int g_dev_err = 0;
+
+RKL_DEFINE_BOUNDS_READER(read_and_clear_bounds_tc)
 
 namespace {
 
@@ -215,6 +218,11 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_kernel(const __grid_co
   const bool leader = rank == 0;
   const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
   static_assert(Cfg::TMEM_COLS <= 512, "TMEM has 512 columns");
+  // Rows of this launch: exact, or read from the device (both CTAs of a pair
+  // read the same value, so they walk the same units).
+  const int n_rows = live_rows(p.n_dev, p.N, p.n_base);
+  const int MT = (n_rows + 2 * kBM - 1) / (2 * kBM);
+  const int units_total = MT * p.G;
 
   // Work of this pair: units u = pair, pair + npairs, ...
   // Unit u = (256-row tile u % MT, vocab group u / MT); group g covers the
@@ -262,9 +270,9 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_kernel(const __grid_co
       uint32_t armed = 0;  // bit i: stage i has been armed at least once
       uint32_t last_par = 0;
       bool ok = true;
-      for (int u = pair; u < p.units_total && ok; u += npairs) {
-        const int m0 = (u % p.MT) * 2 * kBM + rank * kBM;
-        const int g = u / p.MT;
+      for (int u = pair; u < units_total && ok; u += npairs) {
+        const int m0 = (u % MT) * 2 * kBM + rank * kBM;
+        const int g = u / MT;
         const int vt_end = min(g * p.GT + p.GT, p.IT);
         // Teacher per row: the head of this tile's teacher starts at row
         // teacher * V of the stacked heads.  Columns at or past V of a tile
@@ -272,7 +280,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_kernel(const __grid_co
         // uses them (statistics stop at V, the dz store is clipped at V).
         int tv_off = 0;
         if (NG == 2 && p.tgroups > 1) {
-          const int tile_row = (u % p.MT) * 2 * kBM;
+          const int tile_row = (u % MT) * 2 * kBM;
           int tg = 0;
           while (tg + 1 < p.tgroups && tile_row >= p.group_row_end[tg]) ++tg;
           tv_off = tg * p.V;
@@ -282,6 +290,15 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_kernel(const __grid_co
           for (int kb = 0; kb < p.KB; ++kb) {
             if (!mbar_wait_cluster(&empty[stage], phase ^ 1, abort_flag)) {
               raise_abort(abort_flag, ERR_WAIT_TMA_EMPTY);
+              ok = false;
+              break;
+            }
+            // TMA coordinates: x (the K offset) on a 16-byte boundary inside H,
+            // rows inside the padded row layout, vocab rows inside the launch
+            if (!RKL_BOUNDS(((kb * kBK) & 7) == 0 && kb * kBK < p.H && m0 >= 0 && m0 < p.n_pad && v0 >= 0 &&
+                            v0 < (p.vt_base + p.IT) * kFBN && tv_off >= 0 &&
+                            tv_off <= (p.tgroups > 1 ? (p.tgroups - 1) * p.V : 0))) {
+              raise_abort(abort_flag, ERR_BOUNDS);
               ok = false;
               break;
             }
@@ -319,8 +336,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_kernel(const __grid_co
       uint32_t phase = 0;
       bool ok = true;
       int it = 0;
-      for (int u = pair; u < p.units_total && ok; u += npairs) {
-        const int g = u / p.MT;
+      for (int u = pair; u < units_total && ok; u += npairs) {
+        const int g = u / MT;
         const int vt_end = min(g * p.GT + p.GT, p.IT);
         for (int vt = g * p.GT; vt < vt_end && ok; ++vt, ++it) {
           const int acc = it % Cfg::NUM_ACC;
@@ -386,9 +403,9 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_kernel(const __grid_co
     int box = 0;
     int it = 0;
     bool ok = true;
-    for (int u = pair; u < p.units_total && ok; u += npairs) {
-      const int m0 = (u % p.MT) * 2 * kBM + rank * kBM;  // this CTA's first row
-      const int g = u / p.MT;
+    for (int u = pair; u < units_total && ok; u += npairs) {
+      const int m0 = (u % MT) * 2 * kBM + rank * kBM;  // this CTA's first row
+      const int g = u / MT;
       const int vt_end = min(g * p.GT + p.GT, p.IT);
       if (m0 != cur_m0) {
         cur_m0 = m0;
@@ -407,11 +424,11 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_kernel(const __grid_co
           cst = p.rowc[p.n_pad + r];
           g_row = p.rowc[2 * p.n_pad + r];
         } else if (!DZ) {
-          tgt = (p.targets != nullptr && r < p.N) ? p.targets[p.row_idx[r]] : -1;
+          tgt = (p.targets != nullptr && r < n_rows) ? p.targets[p.row_idx[r]] : -1;
         }
         if (NG == 1) {
           trow = nullptr;
-          if (r < p.N) {
+          if (r < n_rows) {
             const long long tr = p.teacher_rows ? p.teacher_rows[r] : r;
             trow = p.teacher + tr * p.teacher_pitch;
           }
@@ -480,7 +497,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_kernel(const __grid_co
               stats_chunk(st, zs, zt);
             else if (nv > 0)
               stats_chunk_tail(st, zs, zt, nv);
-            if (tgt >= 0) pick_target(zs, tgt, v0 + c * 32, p.tlogit + m0 + row);
+            if (tgt >= 0 && RKL_BOUNDS(m0 + row < p.n_pad)) pick_target(zs, tgt, v0 + c * 32, p.tlogit + m0 + row);
           } else if (VAR == 1) {
             // z_s and z_t of this 32-column chunk, fp32, one 32 x 32 box each
             // (columns past V are clipped by the TMA store)
@@ -498,7 +515,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_kernel(const __grid_co
                              __float_as_uint(src[4 * e + 3]));
               fence_proxy_async_smem();
               __syncwarp();
-              if (lane == 0) {
+              if (lane == 0 && RKL_BOUNDS(v0 + c * 32 >= 0 && m0 + q * 32 >= 0)) {
                 tma_store_2d(which == 0 ? &p.tm_zs : &p.tm_zt, buf, v0 + c * 32, m0 + q * 32);
                 bulk_commit();
               }
@@ -551,8 +568,10 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_kernel(const __grid_co
             if (c & 1) {
               fence_proxy_async_smem();
               __syncwarp();
-              if (lane == 0) {
-                tma_store_2d(&p.tm_dz, buf, v0 - p.chunk_v0 + (c - 1) * 32, m0 + q * 32);
+              // a TMA store must not start at a negative coordinate; x (bf16) on a 16-byte boundary
+              const int dx = v0 - p.chunk_v0 + (c - 1) * 32;
+              if (lane == 0 && RKL_BOUNDS(dx >= 0 && (dx & 7) == 0 && m0 + q * 32 >= 0)) {
+                tma_store_2d(&p.tm_dz, buf, dx, m0 + q * 32);
                 bulk_commit();
               }
               ++box;
@@ -560,7 +579,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_kernel(const __grid_co
           }
         }
       }
-      if (!DZ && ok) {
+      if (!DZ && ok && RKL_BOUNDS(m0 + row < p.n_pad && g < p.G)) {
         // statistics slot (group, column half): 2 slots per group
         float* base = p.part + static_cast<size_t>(2 * g + half) * kStatVals * p.n_pad + m0 + row;
         base[0] = st.m_s;
@@ -635,7 +654,13 @@ __global__ void __launch_bounds__(kThreads, 1) grad_kernel(const __grid_constant
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
   const bool leader = rank == 0;
-  const int n_tiles = p.nW + p.nH;
+  // Row count (exact, or read from the device): dH tiles cover the rows in
+  // 256-row pair tiles, dW tiles reduce over them in 64-row K steps.  With no
+  // live row the dW tiles have K = 0 and store zeros.
+  const int n_rows = live_rows(p.n_dev, p.N);
+  const int nH = ((n_rows + 2 * kBM - 1) / (2 * kBM)) * p.NT;
+  const int KBW = (n_rows + kBK - 1) / kBK;
+  const int n_tiles = p.nW + nH;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kGStages; ++i) {
@@ -695,14 +720,21 @@ __global__ void __launch_bounds__(kThreads, 1) grad_kernel(const __grid_constant
           mbar_arrive_cluster(mapa_shared(smem_u32(&sched_empty[slot]), 0));
         }
         if (t < 0) break;
-        const bool is_h = t < p.nH;
-        const int tt = is_h ? t : t - p.nH;
+        const bool is_h = t < nH;
+        const int tt = is_h ? t : t - nH;
         // tile tt = (row / vocab block tt / NT, H block tt % NT): the H block is
         // the fast index, so the tiles running together share their A block
         // (a slice of dz) in L2 and each slice of dz is read from memory once.
         const int m0 = (tt / p.NT) * 2 * kBM + rank * kBM;   // this CTA's A rows
         const int nb = (tt % p.NT) * kGradBN + rank * 128;   // this CTA's first B piece
-        const int KB = is_h ? p.KBH : p.KBW;
+        const int KB = is_h ? p.KBH : KBW;
+        // tile index and TMA coordinates: x of every load on a 16-byte boundary
+        // (m0 is the x of the dz^T loads), no negative row of W_s
+        if (!RKL_BOUNDS(t < n_tiles && tt >= 0 && m0 >= 0 && (m0 & 7) == 0 && (nb & 7) == 0 &&
+                        nb < p.NT * kGradBN && p.cv0 >= 0)) {
+          raise_abort(abort_flag, ERR_BOUNDS);
+          break;
+        }
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait_cluster(&empty[stage], phase ^ 1, abort_flag)) {
             raise_abort(abort_flag, ERR_WAIT_TMA_EMPTY);
@@ -766,9 +798,19 @@ __global__ void __launch_bounds__(kThreads, 1) grad_kernel(const __grid_constant
         const int t = sched_tile[slot];
         mbar_arrive(&sched_empty[slot]);
         if (t < 0) break;
-        const bool is_h = t < p.nH;
-        const int KB = is_h ? p.KBH : p.KBW;
+        const bool is_h = t < nH;
+        const int KB = is_h ? p.KBH : KBW;
         const uint32_t ap = i & 1;  // the accumulator is drained once per tile
+        if (KB == 0) {
+          // No K step (no live row): no MMA, the epilogue stores zeros; the
+          // accumulator hand-off still waits for both halves to be drained.
+          for (int j = 0; j < 2 && ok; ++j)
+            if (!mbar_wait_cluster(&acc_empty[j], ap ^ 1, abort_flag)) {
+              raise_abort(abort_flag, ERR_WAIT_ACC_EMPTY);
+              ok = false;
+            }
+          tc_fence_after();
+        }
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(&full[stage], phase, abort_flag)) {
             raise_abort(abort_flag, ERR_WAIT_TMA_FULL);
@@ -838,8 +880,8 @@ __global__ void __launch_bounds__(kThreads, 1) grad_kernel(const __grid_constant
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(sched_empty0 + slot * 8);
       if (t < 0) break;
-      const bool is_h = t < p.nH;
-      const int tt = is_h ? t : t - p.nH;
+      const bool is_h = t < nH;
+      const int tt = is_h ? t : t - nH;
       const int mtile = tt / p.NT;
       const int n0 = (tt % p.NT) * kGradBN;
       ok = mbar_wait_cluster(acc_full, i & 1, abort_flag);
@@ -851,6 +893,7 @@ __global__ void __launch_bounds__(kThreads, 1) grad_kernel(const __grid_constant
       tc_fence_after();
       const int rows = mtile * 2 * kBM + rank * kBM + q * 32;
       const int row0 = is_h ? rows : p.cv0 + rows;
+      const bool zero_acc = !is_h && KBW == 0;  // no K step: the tile is zero
 #pragma unroll 1
       for (int j = 0; j < 2; ++j) {
         const int col = j * (kGradBN / 2) + sub * 128;  // first column of this warp in the tile
@@ -861,6 +904,12 @@ __global__ void __launch_bounds__(kThreads, 1) grad_kernel(const __grid_constant
 #pragma unroll
         for (int c = 0; c < 4; ++c) tmem_ld_32x32(tb + c * 32, vv[c]);
         tmem_wait_ld();
+        if (zero_acc) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int e = 0; e < 32; ++e) vv[c][e] = 0.f;
+        }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(acc_empty0 + j * 8);
@@ -876,8 +925,9 @@ __global__ void __launch_bounds__(kThreads, 1) grad_kernel(const __grid_constant
                          __float_as_uint(v[4 * e + 2]), __float_as_uint(v[4 * e + 3]));
           fence_proxy_async_smem();
           __syncwarp();
-          if (lane == 0) {
-            const int cx = n0 + col + c * 32;
+          const int cx = n0 + col + c * 32;
+          // fp32 TMA store / reduce: x on a 16-byte boundary, no negative coordinate
+          if (lane == 0 && RKL_BOUNDS(cx >= 0 && (cx & 3) == 0 && row0 >= 0)) {
             if (!is_h)
               tma_store_2d(&p.tm_dw, buf, cx, row0);
             else if (p.dh_accumulate)

@@ -304,7 +304,8 @@ template <typename T>
 __global__ void __launch_bounds__(kTkThreads, 6) topk_fwd_kernel(const T* __restrict__ zs_all,
                                                               const T* __restrict__ zt_all,
                                                               const int32_t* __restrict__ row_idx,
-                                                              const int32_t* __restrict__ targets, int N, int V,
+                                                              const int32_t* __restrict__ targets, int N,
+                                                              const int32_t* __restrict__ n_dev, int n_base, int V,
                                                               long long k_sel, float* __restrict__ saved,
                                                               float* __restrict__ saved_tk, long long zpitch,
                                                               int local) {
@@ -322,7 +323,7 @@ __global__ void __launch_bounds__(kTkThreads, 6) topk_fwd_kernel(const T* __rest
   __shared__ float s_lse[2];
 
   const int kr = blockIdx.x;
-  if (kr >= N) return;
+  if (kr >= live_rows(n_dev, N, n_base)) return;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const long long r = row_idx[kr];  // token position (sampled token)
   const long long zr = local ? kr : r;  // logit row: a block-local row, or the token position
@@ -675,13 +676,15 @@ template <typename T>
 __global__ void __launch_bounds__(kTkThreads) topk_bwd_kernel(const T* __restrict__ zs_all,
                                                               const T* __restrict__ zt_all,
                                                               const int32_t* __restrict__ row_idx,
-                                                              const int32_t* __restrict__ targets, int N, int n_pad,
+                                                              const int32_t* __restrict__ targets, int N,
+                                                              const int32_t* __restrict__ n_dev, int n_pad,
                                                               int V, const float* __restrict__ saved,
                                                               const float* __restrict__ saved_tk,
                                                               const float* __restrict__ rowc, T* __restrict__ dz_all) {
   using Io = TkIo<T>;
   constexpr int VEC = Io::VEC;
   const long long t = blockIdx.x;
+  N = live_rows(n_dev, N);
   int lo = 0, hi = N;
   while (lo < hi) {
     const int mid = (lo + hi) >> 1;
@@ -746,10 +749,12 @@ __global__ void __launch_bounds__(kTkThreads) topk_bwd_kernel(const T* __restric
 __global__ void __launch_bounds__(256) topk_rowk_kernel(const float* __restrict__ saved,
                                                         const float* __restrict__ saved_tk,
                                                         const int32_t* __restrict__ row_idx,
-                                                        const int32_t* __restrict__ targets, int N, int n_pad,
+                                                        const int32_t* __restrict__ targets, int N,
+                                                        const int32_t* __restrict__ n_dev, int n_pad,
                                                         float* __restrict__ rowk) {
   const int p = blockIdx.x * blockDim.x + threadIdx.x;
   if (p >= n_pad) return;
+  N = live_rows(n_dev, N);
   float v[6] = {0.f, 0.f, 0.f, __uint_as_float(0xFFFFFFFFu), __int_as_float(-1), __int_as_float(-1)};
   if (p < N) {
     v[0] = saved[3 * p + 1] - saved[3 * p];
@@ -766,41 +771,43 @@ __global__ void __launch_bounds__(256) topk_rowk_kernel(const float* __restrict_
 }  // namespace
 
 cudaError_t launch_topk_fwd(const void* zs, const void* zt, bool bf16, const int32_t* row_idx,
-                            const int32_t* targets, int N, int V, long long k, float* saved, float* saved_tk,
-                            long long zpitch, bool local, cudaStream_t s) {
+                            const int32_t* targets, int N, const int32_t* n_dev, int n_base, int V, long long k,
+                            float* saved, float* saved_tk, long long zpitch, bool local, cudaStream_t s) {
   if (N <= 0) return cudaSuccess;
   LaunchScope scope(K_TOPK_FWD, s);
   if (bf16)
     topk_fwd_kernel<__nv_bfloat16><<<N, kTkThreads, 0, s>>>(static_cast<const __nv_bfloat16*>(zs),
                                                             static_cast<const __nv_bfloat16*>(zt), row_idx, targets,
-                                                            N, V, k, saved, saved_tk, zpitch, local ? 1 : 0);
+                                                            N, n_dev, n_base, V, k, saved, saved_tk, zpitch,
+                                                            local ? 1 : 0);
   else
     topk_fwd_kernel<float><<<N, kTkThreads, 0, s>>>(static_cast<const float*>(zs), static_cast<const float*>(zt),
-                                                    row_idx, targets, N, V, k, saved, saved_tk, zpitch,
+                                                    row_idx, targets, N, n_dev, n_base, V, k, saved, saved_tk, zpitch,
                                                     local ? 1 : 0);
   return cudaGetLastError();
 }
 
 cudaError_t launch_topk_rowk(const float* saved, const float* saved_tk, const int32_t* row_idx,
-                             const int32_t* targets, int N, int n_pad, float* rowk, cudaStream_t s) {
+                             const int32_t* targets, int N, const int32_t* n_dev, int n_pad, float* rowk,
+                             cudaStream_t s) {
   LaunchScope scope(K_TOPK_ROWK, s);
-  topk_rowk_kernel<<<(n_pad + 255) / 256, 256, 0, s>>>(saved, saved_tk, row_idx, targets, N, n_pad, rowk);
+  topk_rowk_kernel<<<(n_pad + 255) / 256, 256, 0, s>>>(saved, saved_tk, row_idx, targets, N, n_dev, n_pad, rowk);
   return cudaGetLastError();
 }
 
 cudaError_t launch_topk_bwd(const void* zs, const void* zt, bool bf16, const int32_t* row_idx,
-                            const int32_t* targets, int N, int n_pad, long long T, int V, const float* saved,
-                            const float* saved_tk, const float* rowc, void* dz, cudaStream_t s) {
+                            const int32_t* targets, int N, const int32_t* n_dev, int n_pad, long long T, int V,
+                            const float* saved, const float* saved_tk, const float* rowc, void* dz, cudaStream_t s) {
   if (T <= 0) return cudaSuccess;
   LaunchScope scope(K_TOPK_BWD, s);
   if (bf16)
     topk_bwd_kernel<__nv_bfloat16><<<static_cast<unsigned>(T), kTkThreads, 0, s>>>(
-        static_cast<const __nv_bfloat16*>(zs), static_cast<const __nv_bfloat16*>(zt), row_idx, targets, N, n_pad, V,
-        saved, saved_tk, rowc, static_cast<__nv_bfloat16*>(dz));
+        static_cast<const __nv_bfloat16*>(zs), static_cast<const __nv_bfloat16*>(zt), row_idx, targets, N, n_dev,
+        n_pad, V, saved, saved_tk, rowc, static_cast<__nv_bfloat16*>(dz));
   else
     topk_bwd_kernel<float><<<static_cast<unsigned>(T), kTkThreads, 0, s>>>(
-        static_cast<const float*>(zs), static_cast<const float*>(zt), row_idx, targets, N, n_pad, V, saved, saved_tk,
-        rowc, static_cast<float*>(dz));
+        static_cast<const float*>(zs), static_cast<const float*>(zt), row_idx, targets, N, n_dev, n_pad, V, saved,
+        saved_tk, rowc, static_cast<float*>(dz));
   return cudaGetLastError();
 }
 

@@ -37,6 +37,20 @@
  *  - Results are deterministic: the same inputs give bitwise-equal outputs,
  *    and a row's loss and dH row do not depend on which other rows are in the
  *    batch.
+ *  - The trainable-row count.  Every entry point that takes `int32_t N` also
+ *    takes `const int32_t* n_dev` (device, 4-byte aligned, nullable):
+ *      n_dev == NULL: N is the exact count (a host value, e.g. read back
+ *                     from rkl_compact_rows);
+ *      n_dev != NULL: N is an upper bound (normally B*Sm1; the workspace and
+ *                     `saved` are sized for it) and the kernels read the
+ *                     count from *n_dev when they run, clamped to [0, N].
+ *    With n_dev a whole step (compaction, forward, backward) is enqueued with
+ *    no host synchronisation and no device-to-host copy; the mask may change
+ *    from step to step.  Outputs are the same in both modes; the device mode
+ *    always gathers the trainable rows (the host mode skips the gather when
+ *    N = B*Sm1).  `saved` offsets (the top-k entry points' second block) are
+ *    taken from N in both modes, so forward and backward must be given the
+ *    same N.
  */
 #ifndef RKL_H
 #define RKL_H
@@ -100,8 +114,10 @@ rkl_status rkl_workspace_size(rkl_payload payload, rkl_dtype dtype, int64_t n_ma
 /* S1, compaction (slime PR #2310, Summary: project only the N loss-masked
  * rows).  row_idx[k] = flattened index b*Sm1+t of the k-th nonzero entry of
  * mask [B, Sm1] (uint8, nonzero = trainable), strictly ascending; *n_dev = N.
- * row_idx must hold B*Sm1 int32.  Bit-exact, deterministic.  The caller
- * reads N back (one 4-byte device-to-host copy) to size the next calls. */
+ * row_idx must hold B*Sm1 int32.  Bit-exact, deterministic.  The next calls
+ * either take N from the host (one 4-byte device-to-host copy after this
+ * call) or read *n_dev on the device (pass n_dev to them, see the
+ * conventions above). */
 rkl_status rkl_compact_rows(const uint8_t* mask, int64_t B, int64_t Sm1,
                             int32_t* row_idx, int32_t* n_dev, void* stream);
 
@@ -116,7 +132,7 @@ rkl_status rkl_compact_rows(const uint8_t* mask, int64_t B, int64_t Sm1,
 rkl_status rkl_forward_hidden(const void* h_s, const void* h_t,
                               const void* W_s, const void* W_t, rkl_dtype dtype,
                               int64_t B, int64_t Sm1, int64_t H, int64_t V,
-                              const int32_t* row_idx, int32_t N,
+                              const int32_t* row_idx, int32_t N, const int32_t* n_dev,
                               rkl_reduction reduction,
                               float* loss_tok, float* loss, float* saved,
                               void* workspace, size_t workspace_bytes, void* stream);
@@ -128,7 +144,7 @@ rkl_status rkl_forward_hidden(const void* h_s, const void* h_t,
 rkl_status rkl_forward_logits(const void* h_s, const void* W_s,
                               const void* teacher_logits, rkl_dtype dtype,
                               int64_t B, int64_t Sm1, int64_t H, int64_t V,
-                              const int32_t* row_idx, int32_t N,
+                              const int32_t* row_idx, int32_t N, const int32_t* n_dev,
                               rkl_reduction reduction,
                               float* loss_tok, float* loss, float* saved,
                               void* workspace, size_t workspace_bytes, void* stream);
@@ -146,7 +162,7 @@ rkl_status rkl_forward_logits(const void* h_s, const void* W_s,
 rkl_status rkl_forward_hidden_ex(const void* h_s, const void* h_t,
                                  const void* W_s, const void* W_t, rkl_dtype dtype,
                                  int64_t B, int64_t Sm1, int64_t H, int64_t V,
-                                 const int32_t* row_idx, int32_t N,
+                                 const int32_t* row_idx, int32_t N, const int32_t* n_dev,
                                  rkl_reduction reduction,
                                  float* loss_tok, float* loss, float* saved,
                                  const int32_t* targets, float* entropy, float* target_logprob,
@@ -154,7 +170,7 @@ rkl_status rkl_forward_hidden_ex(const void* h_s, const void* h_t,
 rkl_status rkl_forward_logits_ex(const void* h_s, const void* W_s,
                                  const void* teacher_logits, rkl_dtype dtype,
                                  int64_t B, int64_t Sm1, int64_t H, int64_t V,
-                                 const int32_t* row_idx, int32_t N,
+                                 const int32_t* row_idx, int32_t N, const int32_t* n_dev,
                                  rkl_reduction reduction,
                                  float* loss_tok, float* loss, float* saved,
                                  const int32_t* targets, float* entropy, float* target_logprob,
@@ -176,7 +192,7 @@ rkl_status rkl_backward(rkl_payload payload,
                         const void* h_s, const void* teacher,
                         const void* W_s, const void* W_t, rkl_dtype dtype,
                         int64_t B, int64_t Sm1, int64_t H, int64_t V,
-                        const int32_t* row_idx, int32_t N,
+                        const int32_t* row_idx, int32_t N, const int32_t* n_dev,
                         rkl_reduction reduction, const float* saved,
                         const float* grad_loss, const float* grad_tok,
                         float* dH_s, float* dW_s,
@@ -191,7 +207,7 @@ rkl_status rkl_backward(rkl_payload payload,
  * (H is ignored). */
 rkl_status rkl_forward_logits_pair(const void* student_logits, const void* teacher_logits,
                                    rkl_dtype dtype, int64_t B, int64_t Sm1, int64_t V,
-                                   const int32_t* row_idx, int32_t N,
+                                   const int32_t* row_idx, int32_t N, const int32_t* n_dev,
                                    rkl_reduction reduction,
                                    float* loss_tok, float* loss, float* saved,
                                    void* workspace, size_t workspace_bytes, void* stream);
@@ -202,7 +218,7 @@ rkl_status rkl_forward_logits_pair(const void* student_logits, const void* teach
  * elements. */
 rkl_status rkl_backward_logits_pair(const void* student_logits, const void* teacher_logits,
                                     rkl_dtype dtype, int64_t B, int64_t Sm1, int64_t V,
-                                    const int32_t* row_idx, int32_t N,
+                                    const int32_t* row_idx, int32_t N, const int32_t* n_dev,
                                     rkl_reduction reduction, const float* saved,
                                     const float* grad_loss, const float* grad_tok, void* dz,
                                     void* workspace, size_t workspace_bytes, void* stream);
@@ -236,7 +252,7 @@ rkl_status rkl_backward_logits_pair(const void* student_logits, const void* teac
  * rkl_workspace_size(RKL_PAYLOAD_LOGITS_PAIR, ...). */
 rkl_status rkl_forward_topk_pair(const void* student_logits, const void* teacher_logits,
                                  rkl_dtype dtype, int64_t B, int64_t Sm1, int64_t V,
-                                 const int32_t* row_idx, int32_t N, int64_t k,
+                                 const int32_t* row_idx, int32_t N, const int32_t* n_dev, int64_t k,
                                  const int32_t* targets, rkl_reduction reduction,
                                  float* loss_tok, float* loss, float* saved,
                                  void* workspace, size_t workspace_bytes, void* stream);
@@ -254,7 +270,7 @@ rkl_status rkl_forward_topk_pair(const void* student_logits, const void* teacher
 rkl_status rkl_forward_topk_hidden(const void* h_s, const void* h_t,
                                    const void* W_s, const void* W_t, rkl_dtype dtype,
                                    int64_t B, int64_t Sm1, int64_t H, int64_t V,
-                                   const int32_t* row_idx, int32_t N, int64_t k,
+                                   const int32_t* row_idx, int32_t N, const int32_t* n_dev, int64_t k,
                                    const int32_t* targets, rkl_reduction reduction,
                                    float* loss_tok, float* loss, float* saved,
                                    void* workspace, size_t workspace_bytes, void* stream);
@@ -262,7 +278,8 @@ rkl_status rkl_forward_topk_hidden(const void* h_s, const void* h_t,
 rkl_status rkl_backward_topk_hidden(const void* h_s, const void* h_t,
                                     const void* W_s, const void* W_t, rkl_dtype dtype,
                                     int64_t B, int64_t Sm1, int64_t H, int64_t V,
-                                    const int32_t* row_idx, int32_t N, const int32_t* targets,
+                                    const int32_t* row_idx, int32_t N, const int32_t* n_dev,
+                                    const int32_t* targets,
                                     rkl_reduction reduction, const float* saved,
                                     const float* grad_loss, const float* grad_tok,
                                     float* dH_s, float* dW_s,
@@ -273,7 +290,8 @@ rkl_status rkl_backward_topk_hidden(const void* h_s, const void* h_t,
  * and targets from the matching forward call. */
 rkl_status rkl_backward_topk_pair(const void* student_logits, const void* teacher_logits,
                                   rkl_dtype dtype, int64_t B, int64_t Sm1, int64_t V,
-                                  const int32_t* row_idx, int32_t N, const int32_t* targets,
+                                  const int32_t* row_idx, int32_t N, const int32_t* n_dev,
+                                  const int32_t* targets,
                                   rkl_reduction reduction, const float* saved,
                                   const float* grad_loss, const float* grad_tok, void* dz,
                                   void* workspace, size_t workspace_bytes, void* stream);
@@ -291,6 +309,8 @@ rkl_status rkl_backward_topk_pair(const void* student_logits, const void* teache
  * Internally the compacted rows are regrouped by teacher into whole 256-row
  * tiles (padding rows between groups cost at most 255 rows per teacher of
  * extra tensor-core work), so every tile projects with one teacher head.
+ * That layout is planned on the host from the per-teacher counts, so these
+ * entry points take the exact N and counts from the host (no n_dev).
  * ------------------------------------------------------------------------ */
 
 /* S1 with teacher counts.  teacher_idx [B, Sm1] int32 (device; entries at

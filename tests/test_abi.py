@@ -58,13 +58,14 @@ GOOD = 0x10000  # 16-byte aligned fake device address (never dereferenced)
 
 
 def _fwd(L, **kw):
-    a = dict(h_s=GOOD, h_t=GOOD, W_s=GOOD, W_t=GOOD, dtype=0, B=2, Sm1=3, H=64, V=100, row_idx=GOOD, N=4,
+    a = dict(h_s=GOOD, h_t=GOOD, W_s=GOOD, W_t=GOOD, dtype=0, B=2, Sm1=3, H=64, V=100, row_idx=GOOD, N=4, n_dev=0,
              red=1, loss_tok=GOOD, loss=GOOD, saved=GOOD, ws=GOOD, ws_bytes=1 << 40)
     a.update(kw)
     return L.rkl_forward_hidden(_fake(a["h_s"]) if a["h_s"] else None, _fake(a["h_t"]) if a["h_t"] else None,
                                 _fake(a["W_s"]), _fake(a["W_t"]), a["dtype"], a["B"], a["Sm1"], a["H"], a["V"],
-                                _fake(a["row_idx"]), a["N"], a["red"], _fake(a["loss_tok"]), _fake(a["loss"]),
-                                _fake(a["saved"]), _fake(a["ws"]), a["ws_bytes"], None)
+                                _fake(a["row_idx"]), a["N"], _fake(a["n_dev"]) if a["n_dev"] else None, a["red"],
+                                _fake(a["loss_tok"]), _fake(a["loss"]), _fake(a["saved"]), _fake(a["ws"]),
+                                a["ws_bytes"], None)
 
 
 def test_forward_argument_errors(L):
@@ -79,10 +80,13 @@ def test_forward_argument_errors(L):
     assert _fwd(L, W_s=GOOD + 4) == 4               # misaligned
     assert _fwd(L, ws_bytes=1000) == 5              # workspace too small
     assert b"workspace" in L.rkl_last_error()
+    assert _fwd(L, n_dev=GOOD + 2) == 4             # device row count not 4-byte aligned
+    assert b"n_dev" in L.rkl_last_error()
+    assert _fwd(L, N=7, n_dev=GOOD) == 2            # the bound is still checked against B*Sm1
 
 
 def test_logits_payload_needs_v_multiple_of_8_in_bf16(L):
-    st = L.rkl_forward_logits(_fake(GOOD), _fake(GOOD), _fake(GOOD), 0, 2, 3, 64, 100 + 3, _fake(GOOD), 4, 1,
+    st = L.rkl_forward_logits(_fake(GOOD), _fake(GOOD), _fake(GOOD), 0, 2, 3, 64, 100 + 3, _fake(GOOD), 4, None, 1,
                               _fake(GOOD), _fake(GOOD), _fake(GOOD), _fake(GOOD), 1 << 40, None)
     assert st == 2
 
@@ -92,7 +96,7 @@ def test_backward_argument_errors(L):
         a = dict(payload=0, W_t=GOOD, dH=GOOD, dW=GOOD, saved=GOOD, gl=GOOD, N=4, ws_bytes=1 << 40)
         a.update(kw)
         return L.rkl_backward(a["payload"], _fake(GOOD), _fake(GOOD), _fake(GOOD),
-                              _fake(a["W_t"]) if a["W_t"] else None, 0, 2, 3, 64, 128, _fake(GOOD), a["N"], 1,
+                              _fake(a["W_t"]) if a["W_t"] else None, 0, 2, 3, 64, 128, _fake(GOOD), a["N"], None, 1,
                               _fake(a["saved"]) if a["saved"] else None, _fake(a["gl"]) if a["gl"] else None, None,
                               _fake(a["dH"]) if a["dH"] else None, _fake(a["dW"]), _fake(GOOD), a["ws_bytes"], None)
     assert bwd(payload=5) == 3
@@ -157,7 +161,7 @@ def test_multi_teacher_argument_errors(L):
 
 def test_topk_argument_errors(L):
     def fwd_pair(k=8, targets=GOOD, ws_bytes=1 << 40):
-        return L.rkl_forward_topk_pair(_fake(GOOD), _fake(GOOD), 0, 2, 3, 1000, _fake(GOOD), 4, k,
+        return L.rkl_forward_topk_pair(_fake(GOOD), _fake(GOOD), 0, 2, 3, 1000, _fake(GOOD), 4, None, k,
                                        _fake(targets) if targets else None, 1, _fake(GOOD), _fake(GOOD), _fake(GOOD),
                                        _fake(GOOD), ws_bytes, None)
     assert fwd_pair(k=-1) == 2
@@ -167,7 +171,7 @@ def test_topk_argument_errors(L):
 
     def fwd_hidden(dtype=0, k=8, targets=GOOD, H=64):
         return L.rkl_forward_topk_hidden(_fake(GOOD), _fake(GOOD), _fake(GOOD), _fake(GOOD), dtype, 2, 3, H, 1000,
-                                         _fake(GOOD), 4, k, _fake(targets) if targets else None, 1, _fake(GOOD),
+                                         _fake(GOOD), 4, None, k, _fake(targets) if targets else None, 1, _fake(GOOD),
                                          _fake(GOOD), _fake(GOOD), _fake(GOOD), 1 << 40, None)
     assert fwd_hidden(dtype=1) == 6          # fp32: unsupported on this path
     assert fwd_hidden(k=-3) == 2

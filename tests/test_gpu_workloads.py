@@ -27,10 +27,12 @@ SAMPLE = 24
 VOCAB_EDGES = np.array([0, 1, 255, 256, 50687, 50688, 101375, 101376, 151807, 151808, 151935])
 
 
-def _run(inp, reduction, mask=None, grad_tok=None, grad_loss=1.0):
+def _run(inp, reduction, mask=None, grad_tok=None, grad_loss=1.0, on_device=True):
+    """One step as bench.py times it: the row count stays on the device
+    (on_device=False: read back to the host first)."""
     mask = inp["mask"] if mask is None else mask
     B, Sm1 = mask.shape
-    row_idx, N = rb.compact_rows(mask.cuda())
+    row_idx, N = rb.compact_rows(mask.cuda(), on_device=on_device)
     logits = "teacher_logits" in inp
     if logits:
         lt, loss, saved = rb.forward_logits(inp["h_s"], inp["W_s"], inp["teacher_logits"], B, Sm1, row_idx, N,
@@ -46,6 +48,7 @@ def _run(inp, reduction, mask=None, grad_tok=None, grad_loss=1.0):
                          grad_loss=gl, grad_tok=gt)
     torch.cuda.synchronize()
     assert rb.device_error() == 0
+    N = N if isinstance(N, int) else int(N.item())
     return {"N": N, "row_idx": row_idx[:N], "loss_tok": lt, "loss": loss, "saved": saved[:N], "dH": dH, "dW": dW}
 
 
@@ -163,6 +166,10 @@ def test_qwen_hidden_full_size():
     off = ~inp["mask"].reshape(-1).bool()
     assert float(torch.count_nonzero(lt[off])) == 0
     assert float(torch.count_nonzero(out["dH"][off])) == 0
+    # the host-count mode gives bitwise the same results
+    host = _run(inp, red, on_device=False)
+    for k in ("loss_tok", "loss", "saved", "dH", "dW"):
+        assert torch.equal(out[k], host[k]), k
 
 
 def test_self_distill_full_size_exact_zero():

@@ -6,7 +6,9 @@ array inside the library instead of a caller workspace.
 The GPU test drives it through the C ABI (ctypes, raw pointers) and compares
 it with rkl_forward_hidden, which takes a caller workspace, on two calls in a
 row with different problems, so that whatever the first call left in the
-shared array cannot leak into the second.  This file is collected last."""
+shared array cannot leak into the second.  A second test checks it against
+the float64 oracle on a small bf16 and a small fp32 problem, so that a fault
+shared with the workspace path would show too.  This file is collected last."""
 
 import ctypes
 
@@ -25,8 +27,8 @@ def _p(t):
     return ctypes.c_void_p(t.data_ptr())
 
 
-def _problem(B, Sm1, H, V, seed):
-    inp = make_inputs(B, Sm1, H, V, dtype="bf16", payload="hidden", mask="random", weights="perturbed",
+def _problem(B, Sm1, H, V, seed, dtype="bf16"):
+    inp = make_inputs(B, Sm1, H, V, dtype=dtype, payload="hidden", mask="random", weights="perturbed",
                       seed=seed, device="cuda", teacher_noise=0.05)
     return inp
 
@@ -43,15 +45,17 @@ def _forward(L, inp, use_static):
     loss_tok = torch.full((B, Sm1), float("nan"), device="cuda")
     loss = torch.full((1,), float("nan"), device="cuda")
     saved = torch.full((max(N, 1), 3), float("nan"), device="cuda")
-    args = (_p(inp["h_s"]), _p(inp["h_t"]), _p(inp["W_s"]), _p(inp["W_t"]), 0, B, Sm1, H, V, _p(row_idx), N, 1,
+    dt = 0 if inp["h_s"].dtype == torch.bfloat16 else 1
+    args = (_p(inp["h_s"]), _p(inp["h_t"]), _p(inp["W_s"]), _p(inp["W_t"]), dt, B, Sm1, H, V, _p(row_idx), N, 1,
             _p(loss_tok), _p(loss), _p(saved))
     if use_static:
         st = L.rkl_forward_hidden_noalloc(*args, s)
     else:
         nbytes = ctypes.c_size_t(0)
-        assert L.rkl_workspace_size(0, 0, N, B, Sm1, H, V, ctypes.byref(nbytes)) == 0
+        assert L.rkl_workspace_size(0, dt, N, B, Sm1, H, V, ctypes.byref(nbytes)) == 0
         ws = torch.empty(nbytes.value, dtype=torch.uint8, device="cuda")
-        st = L.rkl_forward_hidden(*args, _p(ws), nbytes.value, s)
+        # the workspace entry point takes an optional device row count after N
+        st = L.rkl_forward_hidden(*args[:11], None, *args[11:], _p(ws), nbytes.value, s)
     assert st == 0, L.rkl_last_error().decode()
     torch.cuda.synchronize()
     return loss_tok, loss, saved[:N]
@@ -71,6 +75,25 @@ def test_noalloc_forward_matches_workspace_forward_twice():
         assert np.all(np.abs(g - r) <= TOK_ATOL + TOK_RTOL * np.abs(r))
         assert abs(float(loss) - float(ref_loss)) <= TOK_ATOL + TOK_RTOL * abs(float(ref_loss))
         assert torch.allclose(saved, ref_saved, atol=TOK_ATOL, rtol=TOK_RTOL)
+    code = ctypes.c_int32(0)
+    assert L.rkl_device_error(ctypes.byref(code)) == 0 and code.value == 0
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_noalloc_forward_matches_the_oracle(dtype):
+    from oracle import rkl_oracle as O
+
+    build()
+    L = rb.lib()
+    H = 128 if dtype == "bf16" else 40
+    inp = _problem(2, 300, H, 3000, 21, dtype=dtype)
+    tok, loss, saved = _forward(L, inp, use_static=True)
+    f = lambda t: t.double().cpu().numpy()  # noqa: E731
+    ref = O.forward(f(inp["h_s"]), f(inp["W_s"]), f(inp["h_t"]), f(inp["W_t"]), inp["mask"].cpu().numpy(), 1)
+    g = tok.double().cpu().numpy()
+    assert np.all(np.abs(g - ref["loss_tok"]) <= TOK_ATOL + TOK_RTOL * np.abs(ref["loss_tok"]))
+    assert abs(float(loss) - ref["loss"]) <= TOK_ATOL + TOK_RTOL * abs(ref["loss"])
     code = ctypes.c_int32(0)
     assert L.rkl_device_error(ctypes.byref(code)) == 0 and code.value == 0
 
