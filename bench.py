@@ -110,19 +110,19 @@ class ClockSampler:
                 "reasons": sorted(self.reasons), "samples": len(self.samples)}
 
 
-PATHS = ("hidden", "stats", "topk_hidden", "multi", "logits", "pair", "topk_pair")
+PATHS = ("hidden", "stats", "topk_hidden", "multi", "logits", "topk_logits", "pair", "topk_pair")
 
 
 def path_of(cfg):
     """The entry points a workload's step goes through, from its config:
     hidden (rkl_forward_hidden), stats (rkl_forward_hidden_ex with targets),
     topk_hidden, multi (a teacher per row), logits (shipped teacher logits),
-    pair (both sides as logits) or topk_pair."""
+    topk_logits, pair (both sides as logits) or topk_pair."""
     payload = cfg["payload"]
     if payload == "logits_pair":
         return "topk_pair" if cfg.get("k") is not None else "pair"
     if payload == "logits":
-        return "logits"
+        return "topk_logits" if cfg.get("k") is not None else "logits"
     if payload == "hidden_multi":
         return "multi"
     if cfg.get("k") is not None:
@@ -145,14 +145,15 @@ class Problem:
         self.T = self.B * self.Sm1
         path = path_of(self.cfg)
         self.pair = path in ("pair", "topk_pair")
-        self.logits = path == "logits"
+        self.topk_logits = path == "topk_logits"
+        self.logits = path in ("logits", "topk_logits")
         self.multi = path == "multi"
         self.n_teachers = inp["W_t"].shape[0] if self.multi else 1
         self.topk = path == "topk_pair"
         # per-token student entropy and target log-prob from the same forward
         self.stats = path == "stats"
         self.topk_hidden = path == "topk_hidden"
-        self.k = int(self.cfg.get("k", 0)) if (self.topk or self.topk_hidden) else None
+        self.k = int(self.cfg.get("k", 0)) if (self.topk or self.topk_hidden or self.topk_logits) else None
         self.student = inp["student_logits"] if self.pair else inp["h_s"]
         self.H = 0 if self.pair else inp["h_s"].shape[1]
         self.V = inp["student_logits"].shape[1] if self.pair else inp["W_s"].shape[0]
@@ -172,6 +173,8 @@ class Problem:
             self.counts_host = torch.empty(self.n_teachers + 1, dtype=torch.int32).pin_memory()
         elif self.topk_hidden:
             nbytes = rb.workspace_size(rb.PAYLOAD_TOPK_HIDDEN, self.dt, self.T, self.B, self.Sm1, self.H, self.V)
+        elif self.topk_logits:
+            nbytes = rb.workspace_size(rb.PAYLOAD_TOPK_LOGITS, self.dt, self.T, self.B, self.Sm1, self.H, self.V)
         else:
             nbytes = rb.workspace_size(self.payload, self.dt, self.T, self.B, self.Sm1, max(self.H, 64), self.V)
         self.ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
@@ -203,7 +206,7 @@ class Problem:
         out = [self.student, self.teacher, self.inp["mask"]]
         if self.multi:
             out.append(self.inp["teacher_idx"])
-        if self.topk or self.topk_hidden or self.stats:
+        if self.topk or self.topk_hidden or self.topk_logits or self.stats:
             out.append(self.inp["targets"])
         return out
 
@@ -249,6 +252,17 @@ class Problem:
                                                  self.B, self.Sm1, self.H, self.V, p(self.row_idx), N, nd, p(tg),
                                                  self.reduction, p(self.saved), p(self.grad_loss), None, p(self.dH),
                                                  p(self.dW), p(self.ws), self.ws.numel(), s))
+            return None
+        if self.topk_logits:
+            tg = self.inp["targets"] if extra is None else extra
+            rb._check(L.rkl_forward_topk_logits(p(h_s), p(self.inp["W_s"]), p(teacher), self.dt, self.B, self.Sm1,
+                                                self.H, self.V, p(self.row_idx), N, nd, self.k, p(tg),
+                                                self.reduction, p(self.loss_tok), p(self.loss), p(self.saved),
+                                                p(self.ws), self.ws.numel(), s))
+            rb._check(L.rkl_backward_topk_logits(p(h_s), p(self.inp["W_s"]), p(teacher), self.dt, self.B, self.Sm1,
+                                                 self.H, self.V, p(self.row_idx), N, nd, p(tg), self.reduction,
+                                                 p(self.saved), p(self.grad_loss), None, p(self.dH), p(self.dW),
+                                                 p(self.ws), self.ws.numel(), s))
             return None
         if self.logits:
             rb._check(L.rkl_forward_logits(p(h_s), p(self.inp["W_s"]), p(teacher), self.dt, self.B, self.Sm1, self.H,
@@ -324,6 +338,13 @@ def algorithmic_work(prob, N):
     if prob.pair:
         return {"pair_fwd": ("hbm", 4.0 * N * V + 16.0 * N),
                 "pair_bwd": ("hbm", 4.0 * N * V + 2.0 * prob.T * V)}
+    if prob.topk_logits:
+        # writer 2 N H V (z_s; the shipped z_t is copied beside it), the
+        # teacher rows read once (2 N V bytes) there, selection / estimate
+        # over the written fp32 block (2 x 4 N V bytes), dz recompute 2 N H V
+        # (+ the teacher rows again), grad 4 N H V
+        return {"zw_single_tc": ("tensor", 2.0 * N * H * V), "topk_fwd": ("hbm", 8.0 * N * V),
+                "dz_topk_single_tc": ("tensor", 2.0 * N * H * V), "grad_dw_dh_tc": ("tensor", 4.0 * N * H * V)}
     if prob.topk_hidden:
         # writer 4 N H V (z_s and z_t), selection/estimate over the written fp32
         # logits (read 2 x 4 N V bytes once), dz recompute 4 N H V, grad 4 N H V
@@ -412,12 +433,16 @@ def _cpu_oracle_sample(O, inp, reduction, name, rows, k):
         dt = time.perf_counter() - t0
     else:
         h_s, W_s = f64(inp["h_s"]), f64(inp["W_s"])
-        if path == "logits":
+        if path in ("logits", "topk_logits"):
             teacher, W_t = f64(inp["teacher_logits"]), None
         else:
             teacher, W_t = f64(inp["h_t"]), f64(inp["W_t"])
         t0 = time.perf_counter()
-        if path == "multi":
+        if path == "topk_logits":
+            y = inp["targets"].cpu().numpy()
+            O.forward_topk_logits(h_s, W_s, teacher, y, k, sub, reduction)
+            O.backward_topk_logits(h_s, W_s, teacher, y, k, sub, reduction)
+        elif path == "multi":
             tid = inp["teacher_idx"].cpu().numpy()
             O.forward_multi(h_s, W_s, teacher, W_t, tid, sub, reduction)
             O.backward_multi(h_s, W_s, teacher, W_t, tid, sub, reduction)
@@ -612,6 +637,7 @@ def run_gpu(args, rank, world, dist):
                    "payload": ("logits_pair, top-k estimator k=%d" % prob.k if prob.topk else "logits_pair")
                    if prob.pair else ("hidden, top-k estimator k=%d" % prob.k if prob.topk_hidden else
                                       "hidden, with student entropy and target log-prob" if prob.stats else
+                                      "logits, top-k estimator k=%d" % prob.k if prob.topk_logits else
                                       "logits" if prob.logits else
                                                                  ("hidden, %d teachers" % prob.n_teachers
                                                                   if prob.multi else "hidden")),

@@ -79,6 +79,10 @@ _SIGS = {
                                  _vp, _vp, _vp, _vp, _sz, _vp], _i32),
     "rkl_backward_topk_hidden": ([_vp, _vp, _vp, _vp, _i32, _i64, _i64, _i64, _i64, _vp, _i32, _vp, _vp, _i32, _vp,
                                   _vp, _vp, _vp, _vp, _vp, _sz, _vp], _i32),
+    "rkl_forward_topk_logits": ([_vp, _vp, _vp, _i32, _i64, _i64, _i64, _i64, _vp, _i32, _vp, _i64, _vp, _i32,
+                                 _vp, _vp, _vp, _vp, _sz, _vp], _i32),
+    "rkl_backward_topk_logits": ([_vp, _vp, _vp, _i32, _i64, _i64, _i64, _i64, _vp, _i32, _vp, _vp, _i32, _vp,
+                                  _vp, _vp, _vp, _vp, _vp, _sz, _vp], _i32),
     "rkl_device_error": ([ctypes.POINTER(_i32)], _i32),
     "rkl_kernel_count": ([], _i32),
     "rkl_kernel_name": ([_i32], ctypes.c_char_p),
@@ -426,6 +430,81 @@ def topk_estimator_hidden(h_s, h_t, W_s, W_t, targets, mask, k, reduction=REDUCE
     payload (targets = sampled tokens); grads to h_s and W_s."""
     return _RKLTopkHidden.apply(h_s.contiguous(), h_t.contiguous(), W_s.contiguous(), W_t.contiguous(), targets,
                                 mask, int(k), reduction)
+
+
+# ------------------------------------------------------------ top-k on the logits payload
+PAYLOAD_TOPK_LOGITS = 4
+
+
+def forward_topk_logits(h_s, W_s, teacher_logits, targets, k, B, Sm1, row_idx, N, reduction, workspace=None):
+    """Top-k estimator on the logits payload (student hidden states and LM
+    head, shipped bf16 teacher logits).  Returns (loss_tok, loss, saved [7N])."""
+    Nc, nd = _count(N, B, Sm1)
+    dev = h_s.device
+    T, H = h_s.shape
+    V = W_s.shape[0]
+    dt = _dtype_code(h_s)
+    tg = targets.to(device=dev, dtype=torch.int32).contiguous()
+    loss_tok = torch.empty((B, Sm1), dtype=torch.float32, device=dev)
+    loss = torch.empty(1, dtype=torch.float32, device=dev)
+    saved = torch.empty(7 * max(Nc, 1), dtype=torch.float32, device=dev)
+    ws = workspace if workspace is not None else _workspace(PAYLOAD_TOPK_LOGITS, dt, max(Nc, 1), B, Sm1, H, V, dev)
+    _check(lib().rkl_forward_topk_logits(_ptr(h_s), _ptr(W_s), _ptr(teacher_logits), dt, B, Sm1, H, V,
+                                         _ptr(row_idx), Nc, nd, int(k), _ptr(tg), reduction, _ptr(loss_tok),
+                                         _ptr(loss), _ptr(saved), _ptr(ws), ws.numel(), _stream(dev)))
+    return loss_tok, loss, saved
+
+
+def backward_topk_logits(h_s, W_s, teacher_logits, targets, B, Sm1, row_idx, N, reduction, saved, grad_loss=None,
+                         grad_tok=None, workspace=None, dH_s=None, dW_s=None):
+    """(dH_s [T,H] fp32, dW_s [V,H] fp32) of the top-k estimator on the logits payload."""
+    Nc, nd = _count(N, B, Sm1)
+    dev = h_s.device
+    T, H = h_s.shape
+    V = W_s.shape[0]
+    dt = _dtype_code(h_s)
+    tg = targets.to(device=dev, dtype=torch.int32).contiguous()
+    if dH_s is None:
+        dH_s = torch.empty((T, H), dtype=torch.float32, device=dev)
+    if dW_s is None:
+        dW_s = torch.empty((V, H), dtype=torch.float32, device=dev)
+    if grad_loss is not None:
+        grad_loss = grad_loss.reshape(1).to(device=dev, dtype=torch.float32).contiguous()
+    if grad_tok is not None:
+        grad_tok = grad_tok.to(device=dev, dtype=torch.float32).contiguous()
+    ws = workspace if workspace is not None else _workspace(PAYLOAD_TOPK_LOGITS, dt, max(Nc, 1), B, Sm1, H, V, dev)
+    _check(lib().rkl_backward_topk_logits(_ptr(h_s), _ptr(W_s), _ptr(teacher_logits), dt, B, Sm1, H, V,
+                                          _ptr(row_idx), Nc, nd, _ptr(tg), reduction, _ptr(saved), _ptr(grad_loss),
+                                          _ptr(grad_tok), _ptr(dH_s), _ptr(dW_s), _ptr(ws), ws.numel(),
+                                          _stream(dev)))
+    return dH_s, dW_s
+
+
+class _RKLTopkLogits(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, h_s, W_s, teacher_logits, targets, mask, k, reduction):
+        B, Sm1 = mask.shape
+        row_idx, N = compact_rows(mask, on_device=True)  # no host synchronisation
+        tg = targets.to(device=h_s.device, dtype=torch.int32).contiguous()
+        loss_tok, loss, saved = forward_topk_logits(h_s, W_s, teacher_logits, tg, k, B, Sm1, row_idx, N, reduction)
+        ctx.save_for_backward(h_s, W_s, teacher_logits, tg, row_idx, saved)
+        ctx.meta = (B, Sm1, N, reduction)
+        return loss.reshape(()), loss_tok
+
+    @staticmethod
+    def backward(ctx, g_loss, g_tok):
+        h_s, W_s, logits, tg, row_idx, saved = ctx.saved_tensors
+        B, Sm1, N, reduction = ctx.meta
+        dH, dW = backward_topk_logits(h_s, W_s, logits, tg, B, Sm1, row_idx, N, reduction, saved,
+                                      grad_loss=g_loss, grad_tok=g_tok)
+        return dH.to(h_s.dtype), dW.to(W_s.dtype), None, None, None, None, None
+
+
+def topk_estimator_logits(h_s, W_s, teacher_logits, targets, mask, k, reduction=REDUCE_TOKEN_MEAN):
+    """Differentiable (loss, loss_tok) of the top-k estimator on the logits
+    payload (targets = sampled tokens); grads to h_s and W_s."""
+    return _RKLTopkLogits.apply(h_s.contiguous(), W_s.contiguous(), teacher_logits.contiguous(), targets, mask,
+                                int(k), reduction)
 
 
 # ------------------------------------------------------------ teacher per row

@@ -58,7 +58,8 @@ static const char* const kKernelNames[K_COUNT] = {
     "compact_rows", "gather_rows",   "fwd_dual_tc",  "fwd_single_tc", "teacher_lse", "combine_splits",
     "scatter_loss", "reduce_loss",   "row_weights",  "dz_dual_tc",    "dz_single_tc", "grad_dw_dh_tc",
     "scatter_dh",   "fwd_simt_fp32", "dz_simt_fp32", "grad_simt_fp32", "pair_fwd",   "pair_bwd",
-    "count_teachers", "build_slots", "topk_fwd", "topk_bwd", "zw_dual_tc", "dz_topk_tc", "topk_rowk"};
+    "count_teachers", "build_slots", "topk_fwd", "topk_bwd", "zw_dual_tc", "dz_topk_tc", "topk_rowk",
+    "zw_single_tc", "dz_topk_single_tc"};
 
 const char* kernel_name(int id) { return (id >= 0 && id < K_COUNT) ? kKernelNames[id] : nullptr; }
 
@@ -192,8 +193,10 @@ static Plan make_plan(rkl_payload payload, rkl_dtype dtype, int64_t n_max, int64
   p.n_pad = static_cast<int>(((n + 2 * kBM - 1) / (2 * kBM)) * (2 * kBM));  // whole 256-row pair tiles
   if (n_teachers > 1) p.n_pad += 2 * kBM * (n_teachers - 1);
   p.VT = static_cast<int>((V + tile_v - 1) / tile_v);
-  // tensor-core path: two statistics slots (column halves) per group
-  p.S = bf16 ? 2 * ((p.VT + kGroupTiles - 1) / kGroupTiles) : (p.VT < kSimtSplits ? p.VT : kSimtSplits);
+  // tensor-core path: fwd_slots statistics slots (column parts) per group of
+  // the forward kernel of this payload (two GEMMs on the hidden payloads)
+  const int ng = (payload == RKL_PAYLOAD_HIDDEN || payload == RKL_PAYLOAD_TOPK_HIDDEN) ? 2 : 1;
+  p.S = bf16 ? fwd_slots(ng) * ((p.VT + kGroupTiles - 1) / kGroupTiles) : (p.VT < kSimtSplits ? p.VT : kSimtSplits);
   // Backward vocab chunks: as few as the widest chunk allows, of equal width
   // (a multiple of the 256-column tile), so that every gradient launch has the
   // same work and the tails of the persistent kernels are paid few times.
@@ -231,7 +234,7 @@ static Plan make_plan(rkl_payload payload, rkl_dtype dtype, int64_t n_max, int64
     p.off_kslot = off;
     off = align256(off + size_t(n) * sizeof(int32_t));
   }
-  if (payload == RKL_PAYLOAD_TOPK_HIDDEN) {
+  if (payload == RKL_PAYLOAD_TOPK_HIDDEN || payload == RKL_PAYLOAD_TOPK_LOGITS) {
     // per-row constants of the top-k dz pass, and z_s, z_t (fp32) of one
     // block of rows: never more than kTopkBlockRows rows of logits at a time
     p.off_rowk = off;
@@ -292,7 +295,7 @@ static rkl_status check_common(rkl_payload payload, rkl_dtype dtype, int64_t B, 
                                int32_t N, int reduction) {
   if (dtype != RKL_BF16 && dtype != RKL_FP32) return fail(RKL_ERR_DTYPE, "unknown dtype %d", (int)dtype);
   if (payload != RKL_PAYLOAD_HIDDEN && payload != RKL_PAYLOAD_LOGITS && payload != RKL_PAYLOAD_LOGITS_PAIR &&
-      payload != RKL_PAYLOAD_TOPK_HIDDEN)
+      payload != RKL_PAYLOAD_TOPK_HIDDEN && payload != RKL_PAYLOAD_TOPK_LOGITS)
     return fail(RKL_ERR_DTYPE, "unknown payload %d", (int)payload);
   if (payload == RKL_PAYLOAD_LOGITS_PAIR) H = 64;  // no hidden dimension in this mode
   if (reduction < 0 || reduction > 2) return fail(RKL_ERR_DTYPE, "unknown reduction %d", reduction);
@@ -303,7 +306,7 @@ static rkl_status check_common(rkl_payload payload, rkl_dtype dtype, int64_t B, 
   if (N < 0 || N > B * Sm1) return fail(RKL_ERR_SHAPE, "N = %d outside [0, B*Sm1]", N);
   if (dtype == RKL_BF16) {
     if (H % 64 != 0) return fail(RKL_ERR_SHAPE, "bf16 requires H %% 64 == 0 (H = %lld)", (long long)H);
-    if (payload == RKL_PAYLOAD_LOGITS && V % 8 != 0)
+    if ((payload == RKL_PAYLOAD_LOGITS || payload == RKL_PAYLOAD_TOPK_LOGITS) && V % 8 != 0)
       return fail(RKL_ERR_SHAPE, "bf16 logits payload requires V %% 8 == 0 (V = %lld)", (long long)V);
   }
   return RKL_OK;
@@ -433,7 +436,7 @@ static rkl_status forward_impl(rkl_payload payload, const void* h_s, const void*
       a.IT = pl.VT;
       a.vt_base = 0;
       a.GT = kGroupTiles;
-      a.G = pl.S / 2;
+      a.G = pl.S / fwd_slots(ng);
       const int units = ((n_rows + 2 * kBM - 1) / (2 * kBM)) * a.G;  // at most; the kernel takes the live count
       RKL_CUDA(launch_fused(ng, false, a, 2 * units < sms ? 2 * units : sms, s));
     } else {
@@ -491,13 +494,14 @@ static rkl_status backward_impl(rkl_payload payload, const void* h_s, const void
   RKL_TRY(check_n_dev(n_dev));
   if (mt && n_dev)
     return fail(RKL_ERR_UNSUPPORTED, "a teacher per row needs the per-teacher counts on the host (n_dev must be NULL)");
+  const bool topk = payload == RKL_PAYLOAD_TOPK_HIDDEN || payload == RKL_PAYLOAD_TOPK_LOGITS;
+  const bool hidden = payload == RKL_PAYLOAD_HIDDEN || payload == RKL_PAYLOAD_TOPK_HIDDEN;
   RKL_TRY(check_ptr(h_s, "h_s"));
-  RKL_TRY(check_ptr(teacher, payload != RKL_PAYLOAD_LOGITS ? "h_t" : "teacher_logits"));
+  RKL_TRY(check_ptr(teacher, hidden ? "h_t" : "teacher_logits"));
   RKL_TRY(check_ptr(W_s, "W_s"));
-  if (payload != RKL_PAYLOAD_LOGITS) RKL_TRY(check_ptr(W_t, "W_t"));
-  const bool topk = payload == RKL_PAYLOAD_TOPK_HIDDEN;
+  if (hidden) RKL_TRY(check_ptr(W_t, "W_t"));
   if (topk && dtype != RKL_BF16)
-    return fail(RKL_ERR_UNSUPPORTED, "the top-k estimator on the hidden payload needs bf16 inputs");
+    return fail(RKL_ERR_UNSUPPORTED, "the top-k estimator on the tensor-core payloads needs bf16 inputs");
   if (topk) RKL_TRY(check_ptr(topk_targets, "targets"));
   RKL_TRY(check_ptr(row_idx, "row_idx"));
   RKL_TRY(check_ptr(saved, "saved", N > 0));
@@ -514,7 +518,6 @@ static rkl_status backward_impl(rkl_payload payload, const void* h_s, const void
   cudaStream_t s = static_cast<cudaStream_t>(stream_);
   const long long T = B * Sm1;
   const bool bf16 = dtype == RKL_BF16;
-  const bool hidden = payload != RKL_PAYLOAD_LOGITS;
   float* dHc = reinterpret_cast<float*>(ws_at(workspace, pl.off_dh));
 
   if (N == 0) {
@@ -591,6 +594,10 @@ static rkl_status backward_impl(rkl_payload payload, const void* h_s, const void
     RKL_TRY(make_map(&g.tm_dh, dHc, true, H, n_rows, H * 4, 32, 32));
     g.N = n_rows;
     g.n_dev = n_dev;
+    g.dw = dW_s;
+    g.dh = dHc;
+    g.dw_rows = static_cast<int>(V);
+    g.dh_rows = n_rows;
     g.H = static_cast<int>(H);
     g.NT = static_cast<int>(H / kGradBN) + (H % kGradBN ? 1 : 0);
 
@@ -607,7 +614,7 @@ static rkl_status backward_impl(rkl_payload payload, const void* h_s, const void
       const int units = MT * a.IT;
       const int fgrid = 2 * units < sms ? 2 * units : sms;
       if (topk)
-        RKL_CUDA(launch_fused_topk(2, a, fgrid, s));
+        RKL_CUDA(launch_fused_topk(2, ng, a, fgrid, s));
       else
         RKL_CUDA(launch_fused(ng, true, a, fgrid, s));
       // S7: dW_s[chunk] = dz^T hc_s and dHc (+)= dz W_s[chunk].
@@ -835,28 +842,34 @@ rkl_status rkl_backward_topk_pair(const void* student_logits, const void* teache
 // runs on those rows.  Backward: the recompute + dz kernel with the top-k
 // formula (membership from the same fp32 logits, bit for bit), then the
 // gradient GEMMs of the exact path.
-rkl_status rkl_forward_topk_hidden(const void* h_s, const void* h_t, const void* W_s, const void* W_t,
-                                   rkl_dtype dtype, int64_t B, int64_t Sm1, int64_t H, int64_t V,
-                                   const int32_t* row_idx, int32_t N, const int32_t* n_dev, int64_t k,
-                                   const int32_t* targets, rkl_reduction reduction, float* loss_tok, float* loss,
-                                   float* saved, void* workspace, size_t workspace_bytes, void* stream) {
-  RKL_NVTX_RANGE();
-  RKL_TRY(check_common(RKL_PAYLOAD_TOPK_HIDDEN, dtype, B, Sm1, H, V, N, reduction));
+// Top-k forward of both tensor-core payloads.  Per block of up to
+// kTopkBlockRows compacted rows, a tcgen05 kernel writes z_s and z_t (fp32)
+// of the block -- on the hidden payload both by the tensor core, on the
+// logits payload z_s by the tensor core and z_t copied (exactly) from the
+// shipped bf16 teacher rows -- and the selection / estimate kernel of the
+// logits-pair form runs on those rows.
+static rkl_status forward_topk_impl(rkl_payload payload, const void* h_s, const void* teacher, const void* W_s,
+                                    const void* W_t, rkl_dtype dtype, int64_t B, int64_t Sm1, int64_t H, int64_t V,
+                                    const int32_t* row_idx, int32_t N, const int32_t* n_dev, int64_t k,
+                                    const int32_t* targets, rkl_reduction reduction, float* loss_tok, float* loss,
+                                    float* saved, void* workspace, size_t workspace_bytes, void* stream) {
+  const bool hidden = payload == RKL_PAYLOAD_TOPK_HIDDEN;
+  RKL_TRY(check_common(payload, dtype, B, Sm1, H, V, N, reduction));
   RKL_TRY(check_n_dev(n_dev));
   if (dtype != RKL_BF16)
-    return fail(RKL_ERR_UNSUPPORTED, "the top-k estimator on the hidden payload needs bf16 inputs");
+    return fail(RKL_ERR_UNSUPPORTED, "the top-k estimator on the tensor-core payloads needs bf16 inputs");
   if (k < 0) return fail(RKL_ERR_SHAPE, "k = %lld is negative", (long long)k);
   RKL_TRY(check_ptr(h_s, "h_s"));
-  RKL_TRY(check_ptr(h_t, "h_t"));
+  RKL_TRY(check_ptr(teacher, hidden ? "h_t" : "teacher_logits"));
   RKL_TRY(check_ptr(W_s, "W_s"));
-  RKL_TRY(check_ptr(W_t, "W_t"));
+  if (hidden) RKL_TRY(check_ptr(W_t, "W_t"));
   RKL_TRY(check_ptr(row_idx, "row_idx"));
   RKL_TRY(check_ptr(targets, "targets"));
   RKL_TRY(check_ptr(loss_tok, "loss_tok", false));
   RKL_TRY(check_ptr(loss, "loss", false));
   RKL_TRY(check_ptr(saved, "saved", N > 0));
   RKL_TRY(check_ptr(workspace, "workspace"));
-  const Plan pl = make_plan(RKL_PAYLOAD_TOPK_HIDDEN, dtype, N, H, V);
+  const Plan pl = make_plan(payload, dtype, N, H, V);
   if (workspace_bytes < pl.total)
     return fail(RKL_ERR_WORKSPACE, "workspace is %zu bytes, %zu needed", workspace_bytes, pl.total);
   int sms = 0;
@@ -865,12 +878,12 @@ rkl_status rkl_forward_topk_hidden(const void* h_s, const void* h_t, const void*
   const long long T = B * Sm1;
   if (N > 0) {
     const uint8_t* as = static_cast<const uint8_t*>(h_s);
-    const uint8_t* at = static_cast<const uint8_t*>(h_t);
+    const uint8_t* at = hidden ? static_cast<const uint8_t*>(teacher) : nullptr;
     if (N < T || n_dev) {
       as = ws_at(workspace, pl.off_hcs);
-      at = ws_at(workspace, pl.off_hct);
-      RKL_CUDA(launch_gather(h_s, h_t, const_cast<uint8_t*>(as), const_cast<uint8_t*>(at), row_idx, nullptr, N, n_dev,
-                             static_cast<int>(H * 2), T, s));
+      at = hidden ? ws_at(workspace, pl.off_hct) : nullptr;
+      RKL_CUDA(launch_gather(h_s, hidden ? teacher : nullptr, const_cast<uint8_t*>(as), const_cast<uint8_t*>(at),
+                             row_idx, nullptr, N, n_dev, static_cast<int>(H * 2), T, s));
     }
     float* zs = reinterpret_cast<float*>(ws_at(workspace, pl.off_z));
     float* zt = zs + size_t(pl.zrows) * pl.zpitch;
@@ -879,9 +892,16 @@ rkl_status rkl_forward_topk_hidden(const void* h_s, const void* h_t, const void*
       FusedArgs a;
       memset(&a, 0, sizeof(a));
       RKL_TRY(make_map(&a.tm_as, as + size_t(r0) * H * 2, false, H, nb, H * 2, kBK, kBM));
-      RKL_TRY(make_map(&a.tm_at, at + size_t(r0) * H * 2, false, H, nb, H * 2, kBK, kBM));
       RKL_TRY(make_map(&a.tm_bs, W_s, false, H, V, H * 2, kBK, kFBN / 2));
-      RKL_TRY(make_map(&a.tm_bt, W_t, false, H, V, H * 2, kBK, kFBN / 2));
+      if (hidden) {
+        RKL_TRY(make_map(&a.tm_at, at + size_t(r0) * H * 2, false, H, nb, H * 2, kBK, kBM));
+        RKL_TRY(make_map(&a.tm_bt, W_t, false, H, V, H * 2, kBK, kFBN / 2));
+      } else {
+        // row p of the block is compacted row r0 + p: token row row_idx[r0 + p]
+        a.teacher = static_cast<const uint16_t*>(teacher);
+        a.teacher_rows = row_idx + r0;
+        a.teacher_pitch = V;
+      }
       RKL_TRY(make_map(&a.tm_zs, zs, true, V, nb, size_t(pl.zpitch) * 4, 32, 32));
       RKL_TRY(make_map(&a.tm_zt, zt, true, V, nb, size_t(pl.zpitch) * 4, 32, 32));
       a.N = nb;
@@ -896,7 +916,7 @@ rkl_status rkl_forward_topk_hidden(const void* h_s, const void* h_t, const void*
       a.GT = 1;
       a.G = pl.VT;
       const int units = ((nb + 2 * kBM - 1) / (2 * kBM)) * a.G;  // at most
-      RKL_CUDA(launch_fused_topk(1, a, 2 * units < sms ? 2 * units : sms, s));
+      RKL_CUDA(launch_fused_topk(1, hidden ? 2 : 1, a, 2 * units < sms ? 2 * units : sms, s));
       RKL_CUDA(launch_topk_fwd(zs, zt, false, row_idx + r0, targets, nb, n_dev, r0, static_cast<int>(V), k,
                                saved + 3 * size_t(r0), saved + 3 * size_t(N) + 4 * size_t(r0), pl.zpitch, true, s));
     }
@@ -905,6 +925,37 @@ rkl_status rkl_forward_topk_hidden(const void* h_s, const void* h_t, const void*
   if (loss && reduction != RKL_REDUCE_NONE)
     RKL_CUDA(launch_reduce(saved, row_idx, N, n_dev, static_cast<int>(B), static_cast<int>(Sm1), reduction, loss, s));
   return RKL_OK;
+}
+
+rkl_status rkl_forward_topk_hidden(const void* h_s, const void* h_t, const void* W_s, const void* W_t,
+                                   rkl_dtype dtype, int64_t B, int64_t Sm1, int64_t H, int64_t V,
+                                   const int32_t* row_idx, int32_t N, const int32_t* n_dev, int64_t k,
+                                   const int32_t* targets, rkl_reduction reduction, float* loss_tok, float* loss,
+                                   float* saved, void* workspace, size_t workspace_bytes, void* stream) {
+  RKL_NVTX_RANGE();
+  return forward_topk_impl(RKL_PAYLOAD_TOPK_HIDDEN, h_s, h_t, W_s, W_t, dtype, B, Sm1, H, V, row_idx, N, n_dev, k,
+                           targets, reduction, loss_tok, loss, saved, workspace, workspace_bytes, stream);
+}
+
+rkl_status rkl_forward_topk_logits(const void* h_s, const void* W_s, const void* teacher_logits, rkl_dtype dtype,
+                                   int64_t B, int64_t Sm1, int64_t H, int64_t V, const int32_t* row_idx, int32_t N,
+                                   const int32_t* n_dev, int64_t k, const int32_t* targets, rkl_reduction reduction,
+                                   float* loss_tok, float* loss, float* saved, void* workspace,
+                                   size_t workspace_bytes, void* stream) {
+  RKL_NVTX_RANGE();
+  return forward_topk_impl(RKL_PAYLOAD_TOPK_LOGITS, h_s, teacher_logits, W_s, nullptr, dtype, B, Sm1, H, V, row_idx,
+                           N, n_dev, k, targets, reduction, loss_tok, loss, saved, workspace, workspace_bytes, stream);
+}
+
+rkl_status rkl_backward_topk_logits(const void* h_s, const void* W_s, const void* teacher_logits, rkl_dtype dtype,
+                                    int64_t B, int64_t Sm1, int64_t H, int64_t V, const int32_t* row_idx, int32_t N,
+                                    const int32_t* n_dev, const int32_t* targets, rkl_reduction reduction,
+                                    const float* saved, const float* grad_loss, const float* grad_tok, float* dH_s,
+                                    float* dW_s, void* workspace, size_t workspace_bytes, void* stream) {
+  RKL_NVTX_RANGE();
+  return backward_impl(RKL_PAYLOAD_TOPK_LOGITS, h_s, teacher_logits, W_s, nullptr, dtype, B, Sm1, H, V, row_idx, N,
+                       n_dev, reduction, saved, grad_loss, grad_tok, dH_s, dW_s, workspace, workspace_bytes, stream,
+                       nullptr, targets);
 }
 
 rkl_status rkl_backward_topk_hidden(const void* h_s, const void* h_t, const void* W_s, const void* W_t,

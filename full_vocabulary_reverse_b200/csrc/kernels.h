@@ -36,6 +36,8 @@ enum KernelId : int {
   K_ZW_DUAL_TC,       // top-k, hidden payload: z_s and z_t of a row block written by tcgen05
   K_DZ_TOPK_TC,       // top-k, hidden payload: recompute + top-k dz chunk
   K_TOPK_ROWK,        // top-k, hidden payload: per-row constants of the dz pass
+  K_ZW_SINGLE_TC,     // top-k, logits payload: z_s of a row block by tcgen05, shipped z_t copied beside it
+  K_DZ_TOPK_SINGLE_TC,  // top-k, logits payload: recompute z_s + top-k dz chunk
   K_COUNT
 };
 
@@ -79,6 +81,15 @@ constexpr int kFBN = 256;      // vocab columns per fused pair tile
 constexpr int kBK = 64;        // K per pipeline stage (128 B of bf16)
 constexpr int kGradBN = 512;   // H columns per gradient pair tile (two N = 256 halves)
 constexpr int kGroupTiles = 4;  // 256-column vocab tiles per forward statistics group (1024 columns)
+// Epilogue warps of the forward statistics kernel with ng GEMMs (a multiple
+// of 4: each TMEM lane quarter is read by fwd_epi / 4 warps, each owning
+// 256 / (fwd_epi / 4) columns of the tile) and its statistics slots per
+// vocab group.  The hidden payload (ng = 2) drains each tile with 16 warps,
+// so that a warp holds two 32-column chunks and the accumulator is released
+// to the next tile after one chunk of statistics work; the logits payload
+// (ng = 1) keeps 8, whose registers also carry the prefetched teacher rows.
+__host__ __device__ constexpr int fwd_epi(int ng) { return ng == 2 ? 16 : 8; }
+__host__ __device__ constexpr int fwd_slots(int ng) { return fwd_epi(ng) / 4; }
 constexpr int kStatVals = 6;    // per slot: m_s, S_s, A, m_t, S_t, sum e^(z_s-m_s) z_s
 constexpr int kMaxTeachers = 16;  // teacher heads of the per-row-teacher mode
 
@@ -126,6 +137,9 @@ struct GradArgs {
   int* tile_counter;      // zeroed before the launch; dynamic tile scheduler
   int N, H, cw, cv0;
   const int32_t* n_dev;   // live row count on the device (nullable: N exact)
+  float* dw;              // dW_s [V, H] fp32 (the tm_dw tensor)
+  float* dh;              // dHc [dh_rows, H] fp32 (the tm_dh tensor)
+  int dw_rows, dh_rows;   // V and the rows of dHc
   int MTW, NT, nW, KBH;
   int dh_accumulate;
 };
@@ -134,9 +148,10 @@ size_t fused_smem_bytes(int ng, bool dz);
 size_t grad_smem_bytes();
 cudaError_t tc_setup(int device);  // one-time cudaFuncSetAttribute per device
 cudaError_t launch_fused(int ng, bool dz, const FusedArgs& a, int grid, cudaStream_t s);  // grid: CTAs, even
-// Hidden-payload top-k: write z_s and z_t (fp32) of the rows of a (variant 1),
-// or the top-k dz chunk (variant 2); both on the NG = 2 dz configuration.
-cudaError_t launch_fused_topk(int variant, const FusedArgs& a, int grid, cudaStream_t s);
+// Top-k estimator: write z_s and z_t (fp32) of the rows of a (variant 1), or
+// the top-k dz chunk (variant 2).  ng = 2: hidden payload (both logits by the
+// tensor core); ng = 1: logits payload (z_t read from the shipped logits).
+cudaError_t launch_fused_topk(int variant, int ng, const FusedArgs& a, int grid, cudaStream_t s);
 cudaError_t launch_grad(const GradArgs& a, int grid, cudaStream_t s);
 cudaError_t read_and_clear_device_error(int* code);
 // RKL_DEBUG build: line of the first failed bounds check in each kernel file

@@ -249,11 +249,15 @@ __global__ void __launch_bounds__(256) teacher_lse_kernel(const T* __restrict__ 
 }
 
 // --------------------------------------------------------------------- S4
-// Merge the per-group statistics of each row; L = A/S_s - lse_s + lse_t.
-// One warp per row: lane l merges groups l, l+32, ..., then a fixed
-// butterfly merges the lanes (same order on every run).  Student and teacher
-// statistics go through identical operations, so teacher == student gives
-// L = 0 exactly.
+// Merge the per-slot statistics of each row; L = A/S_s - lse_s + lse_t.
+// A block takes 32 consecutive rows (lane = row) and its 8 warps split the
+// slots into 8 contiguous ranges, so every load of a warp reads 32
+// consecutive rows of one slot (coalesced) and each warp has few slots to
+// chain.  Within a warp the slots are taken four at a time and merged by a
+// fixed tree, ((g, g+1), (g+2, g+3)), into the running result; the 8
+// partial results are then merged in warp order by warp 0.  The same order
+// on every run.  Student and teacher statistics go through identical
+// operations, so teacher == student gives L = 0 exactly.
 struct Stat3 {
   float m, S, A, Bz;
 };
@@ -268,44 +272,74 @@ __device__ __forceinline__ void merge3(Stat3& a, const Stat3& b) {
   a.m = nm;
 }
 
+__device__ __forceinline__ void load_slot(const float* __restrict__ part, int g, int n_pad, int k, bool teacher,
+                                          Stat3& s, Stat3& t) {
+  const float* b = part + static_cast<size_t>(g) * kStatVals * n_pad + k;
+  s = Stat3{b[0], b[n_pad], b[2 * n_pad], b[5 * n_pad]};
+  t = teacher ? Stat3{b[3 * n_pad], b[4 * n_pad], 0.f, 0.f} : Stat3{-INFINITY, 0.f, 0.f, 0.f};
+}
+
+constexpr int kCombineWarps = 8;
+
 // Optional student statistics of row k (nullable outputs): entropy
 // lse_s - sum p_s z_s = lse_s - Bz / S_s, and target log-prob tlogit - lse_s.
 // Statistics row k (a slot of the teacher-grouped layout when slot_k is
 // given) is written to compact row out = slot_k[k]; padding slots are skipped.
-__global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ part, int S, int n_pad, int n_rows,
-                                                      const int32_t* __restrict__ n_dev,
-                                                      int teacher_from_part, const float* __restrict__ lse_ext,
-                                                      const float* __restrict__ tlogit, float* __restrict__ saved,
-                                                      float* __restrict__ ent_rows, float* __restrict__ lp_rows,
-                                                      const int32_t* __restrict__ slot_k) {
-  const int lane = threadIdx.x & 31;
-  const int k = blockIdx.x * 8 + (threadIdx.x >> 5);
-  if (k >= live_rows(n_dev, n_rows)) return;
+__global__ void __launch_bounds__(32 * kCombineWarps) combine_kernel(
+    const float* __restrict__ part, int S, int n_pad, int n_rows, const int32_t* __restrict__ n_dev,
+    int teacher_from_part, const float* __restrict__ lse_ext, const float* __restrict__ tlogit,
+    float* __restrict__ saved, float* __restrict__ ent_rows, float* __restrict__ lp_rows,
+    const int32_t* __restrict__ slot_k) {
+  __shared__ Stat3 sh_s[kCombineWarps][32], sh_t[kCombineWarps][32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int k = blockIdx.x * 32 + lane;
+  const int n_live = live_rows(n_dev, n_rows);
+  const bool teacher = teacher_from_part != 0;
+  Stat3 s{-INFINITY, 0.f, 0.f, 0.f}, t{-INFINITY, 0.f, 0.f, 0.f};
+  if (k < n_live) {
+    const int g0 = static_cast<int>((static_cast<long long>(S) * warp) / kCombineWarps);
+    const int g1 = static_cast<int>((static_cast<long long>(S) * (warp + 1)) / kCombineWarps);
+    int g = g0;
+    for (; g + 4 <= g1; g += 4) {
+      Stat3 s0, t0, s1, t1, s2, t2, s3, t3;
+      load_slot(part, g, n_pad, k, teacher, s0, t0);
+      load_slot(part, g + 1, n_pad, k, teacher, s1, t1);
+      load_slot(part, g + 2, n_pad, k, teacher, s2, t2);
+      load_slot(part, g + 3, n_pad, k, teacher, s3, t3);
+      merge3(s0, s1);
+      merge3(t0, t1);
+      merge3(s2, s3);
+      merge3(t2, t3);
+      merge3(s0, s2);
+      merge3(t0, t2);
+      merge3(s, s0);
+      merge3(t, t0);
+    }
+    for (; g < g1; ++g) {
+      Stat3 s0, t0;
+      load_slot(part, g, n_pad, k, teacher, s0, t0);
+      merge3(s, s0);
+      merge3(t, t0);
+    }
+  }
+  sh_s[warp][lane] = s;
+  sh_t[warp][lane] = t;
+  __syncthreads();
+  if (warp != 0 || k >= n_live) return;
+  for (int w = 1; w < kCombineWarps; ++w) {
+    merge3(s, sh_s[w][lane]);
+    merge3(t, sh_t[w][lane]);
+  }
   const int out = slot_k ? slot_k[k] : k;
   if (out < 0 || !RKL_BOUNDS(out < n_pad)) return;
-  Stat3 s{-INFINITY, 0.f, 0.f, 0.f}, t{-INFINITY, 0.f, 0.f, 0.f};
-  for (int g = lane; g < S; g += 32) {
-    const float* b = part + static_cast<size_t>(g) * kStatVals * n_pad + k;
-    merge3(s, Stat3{b[0], b[n_pad], b[2 * n_pad], b[5 * n_pad]});
-    if (teacher_from_part) merge3(t, Stat3{b[3 * n_pad], b[4 * n_pad], 0.f, 0.f});
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    merge3(s, Stat3{__shfl_xor_sync(0xffffffffu, s.m, o), __shfl_xor_sync(0xffffffffu, s.S, o),
-                    __shfl_xor_sync(0xffffffffu, s.A, o), __shfl_xor_sync(0xffffffffu, s.Bz, o)});
-    merge3(t, Stat3{__shfl_xor_sync(0xffffffffu, t.m, o), __shfl_xor_sync(0xffffffffu, t.S, o),
-                    __shfl_xor_sync(0xffffffffu, t.A, o), __shfl_xor_sync(0xffffffffu, t.Bz, o)});
-  }
-  if (lane == 0) {
-    const float lse_s = s.m + logf(s.S);
-    const float lse_t = teacher_from_part ? t.m + logf(t.S) : lse_ext[k];
-    const float L = s.A / s.S - lse_s + lse_t;
-    saved[3 * out + 0] = lse_s;
-    saved[3 * out + 1] = lse_t;
-    saved[3 * out + 2] = L;
-    if (ent_rows) ent_rows[out] = lse_s - s.Bz / s.S;
-    if (lp_rows) lp_rows[out] = tlogit[k] - lse_s;
-  }
+  const float lse_s = s.m + logf(s.S);
+  const float lse_t = teacher ? t.m + logf(t.S) : lse_ext[k];
+  const float L = s.A / s.S - lse_s + lse_t;
+  saved[3 * out + 0] = lse_s;
+  saved[3 * out + 1] = lse_t;
+  saved[3 * out + 2] = L;
+  if (ent_rows) ent_rows[out] = lse_s - s.Bz / s.S;
+  if (lp_rows) lp_rows[out] = tlogit[k] - lse_s;
 }
 
 // out[t] = rows[k] if t = row_idx[k] else exactly 0.
@@ -764,8 +798,9 @@ cudaError_t launch_combine(const float* part, int S, int n_pad, int n_rows, cons
                            float* ent_rows, float* lp_rows, const int32_t* slot_k, cudaStream_t s) {
   if (n_rows <= 0) return cudaSuccess;
   LaunchScope scope(K_COMBINE, s);
-  combine_kernel<<<(n_rows + 7) / 8, 256, 0, s>>>(part, S, n_pad, n_rows, n_dev, teacher_from_part ? 1 : 0, lse_ext,
-                                                  tlogit, saved, ent_rows, lp_rows, slot_k);
+  combine_kernel<<<(n_rows + 31) / 32, 32 * kCombineWarps, 0, s>>>(part, S, n_pad, n_rows, n_dev,
+                                                                   teacher_from_part ? 1 : 0, lse_ext, tlogit,
+                                                                   saved, ent_rows, lp_rows, slot_k);
   return cudaGetLastError();
 }
 

@@ -41,8 +41,15 @@ RKL_DEFINE_BOUNDS_READER(read_and_clear_bounds_tc)
 namespace {
 
 constexpr int kThreads = 64 + 32 * 8;  // gradient kernel: producer, MMA, 8 epilogue warps
-constexpr int kFusedEpi = 8;        // fused kernels: 2 epilogue warps per TMEM lane quarter
-constexpr int kFusedThreads = 64 + 32 * kFusedEpi;
+constexpr int kFusedEpi = 8;        // dz / writer kernels: 2 epilogue warps per TMEM lane quarter
+
+// Epilogue warps of fused_kernel<NG, DZ>: the forward statistics kernel has
+// fwd_epi(NG), the kernels with a store epilogue kFusedEpi (their staging
+// boxes live in shared memory beside the pipeline stages).
+template <int NG, bool DZ>
+__host__ __device__ constexpr int fused_epi() { return DZ ? kFusedEpi : fwd_epi(NG); }
+template <int NG, bool DZ>
+__host__ __device__ constexpr int fused_threads() { return 64 + 32 * fused_epi<NG, DZ>(); }
 constexpr int kStgBoxBytes = 4096;  // one 32-row staging box per epilogue warp
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
@@ -193,12 +200,13 @@ __device__ __forceinline__ void prefetch_l2(const void* p) {
 // accumulator-empty barriers; both CTAs run the same producer and epilogue
 // code on their own rows.
 // ============================================================================
-// VAR (with NG = 2, DZ = true) selects the epilogue of the hidden-payload
-// top-k estimator: 1 writes the z_s and z_t tiles (fp32), 2 writes the top-k
-// dz  g (p_s ([v in S](w + 1) - C) + [v = y] a),  S = {key(z_s) > K*, or
+// VAR (with DZ = true) selects the epilogue of the top-k estimator: 1 writes
+// the z_s and z_t tiles (fp32; with NG = 1, z_t is the exact fp32 value of the
+// shipped bf16 teacher logit), 2 writes the top-k dz
+// g (p_s ([v in S](w + 1) - C) + [v = y] a),  S = {key(z_s) > K*, or
 // key(z_s) = K* and v <= v_last} with the order-preserving float key.
 template <int NG, bool DZ, int VAR = 0>
-__global__ void __launch_bounds__(kFusedThreads, 1) fused_kernel(const __grid_constant__ FusedArgs p) {
+__global__ void __launch_bounds__(fused_threads<NG, DZ>(), 1) fused_kernel(const __grid_constant__ FusedArgs p) {
   using Cfg = FusedCfg<NG>;
   constexpr int STAGES = Cfg::STAGES;
   extern __shared__ uint8_t smem_raw[];
@@ -240,7 +248,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_kernel(const __grid_co
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&acc_full[i], 1);
-      mbar_init(&acc_empty[i], 2 * kFusedEpi);  // every epilogue warp of both CTAs
+      mbar_init(&acc_empty[i], 2 * fused_epi<NG, DZ>());  // every epilogue warp of both CTAs
     }
     mbar_init(tear, 1);
     *abort_flag = 0;
@@ -389,6 +397,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_kernel(const __grid_co
     // Warp w reads TMEM lane quarter q = w % 4 (tile rows 32 q .. 32 q + 31)
     // and columns [128 h, 128 h + 128) of the 256-column tile, h = (w-2) / 4.
     const int q = warp & 3;
+    // Warp part p = (w - 2) / 4 owns columns [COLS p, COLS p + COLS).
+    constexpr int COLS = kFBN / (fused_epi<NG, DZ>() / 4);
     const int half = (warp - 2) >> 2;
     const int row = q * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
@@ -436,7 +446,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_kernel(const __grid_co
       }
       RowStats st{-INFINITY, 0.f, 0.f, -INFINITY, 0.f, 0.f};
       for (int vt = g * p.GT; vt < vt_end; ++vt, ++it) {
-        const int v0 = (p.vt_base + vt) * kFBN + half * (kFBN / 2);  // this warp's first column
+        const int v0 = (p.vt_base + vt) * kFBN + half * COLS;  // this warp's first column
         // Teacher logits of this row (logits payload): 32 bf16 per chunk,
         // loaded one chunk ahead.
         uint4 tcur[NG == 1 ? 4 : 1], tnxt[NG == 1 ? 4 : 1];
@@ -456,8 +466,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_kernel(const __grid_co
           break;
         }
         tc_fence_after();
-        const uint32_t tb = tmem_base + lane_off + acc * Cfg::ACC_COLS + half * (kFBN / 2);
-        constexpr int kChunks = kFBN / 2 / 32;
+        const uint32_t tb = tmem_base + lane_off + acc * Cfg::ACC_COLS + half * COLS;
+        constexpr int kChunks = COLS / 32;
 #pragma unroll
         for (int c = 0; c < kChunks; ++c) {
           float zs[32], zt[32];
@@ -580,8 +590,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_kernel(const __grid_co
         }
       }
       if (!DZ && ok && RKL_BOUNDS(m0 + row < p.n_pad && g < p.G)) {
-        // statistics slot (group, column half): 2 slots per group
-        float* base = p.part + static_cast<size_t>(2 * g + half) * kStatVals * p.n_pad + m0 + row;
+        // statistics slot (group, column part): fwd_slots(NG) slots per group
+        float* base = p.part + static_cast<size_t>(fwd_slots(NG) * g + half) * kStatVals * p.n_pad + m0 + row;
         base[0] = st.m_s;
         base[p.n_pad] = st.S_s;
         base[2 * p.n_pad] = st.A;
@@ -983,14 +993,20 @@ cudaError_t tc_setup(int /*device*/) {
   if ((e = cudaFuncSetAttribute(fused_kernel<2, true, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)fused_smem<2, true>())) != cudaSuccess)
     return e;
+  if ((e = cudaFuncSetAttribute(fused_kernel<1, true, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)fused_smem<1, true>())) != cudaSuccess)
+    return e;
+  if ((e = cudaFuncSetAttribute(fused_kernel<1, true, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)fused_smem<1, true>())) != cudaSuccess)
+    return e;
   return cudaFuncSetAttribute(grad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)grad_smem_bytes());
 }
 
 template <typename K>
-static cudaError_t launch_pair(K kernel, int grid, size_t smem, cudaStream_t s, const FusedArgs& a) {
+static cudaError_t launch_pair(K kernel, int grid, int threads, size_t smem, cudaStream_t s, const FusedArgs& a) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid & ~1);  // whole CTA pairs
-  cfg.blockDim = dim3(kFusedThreads);
+  cfg.blockDim = dim3(threads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
@@ -1007,16 +1023,21 @@ cudaError_t launch_fused(int ng, bool dz, const FusedArgs& a, int grid, cudaStre
   const size_t smem = fused_smem_bytes(ng, dz);
   const int id = ng == 2 ? (dz ? K_DZ_DUAL_TC : K_FWD_DUAL_TC) : (dz ? K_DZ_SINGLE_TC : K_FWD_SINGLE_TC);
   LaunchScope scope(id, s);
-  if (ng == 2) return dz ? launch_pair(fused_kernel<2, true>, grid, smem, s, a)
-                         : launch_pair(fused_kernel<2, false>, grid, smem, s, a);
-  return dz ? launch_pair(fused_kernel<1, true>, grid, smem, s, a) : launch_pair(fused_kernel<1, false>, grid, smem, s, a);
+  if (ng == 2) return dz ? launch_pair(fused_kernel<2, true>, grid, fused_threads<2, true>(), smem, s, a)
+                         : launch_pair(fused_kernel<2, false>, grid, fused_threads<2, false>(), smem, s, a);
+  return dz ? launch_pair(fused_kernel<1, true>, grid, fused_threads<1, true>(), smem, s, a) : launch_pair(fused_kernel<1, false>, grid, fused_threads<1, false>(), smem, s, a);
 }
 
-cudaError_t launch_fused_topk(int variant, const FusedArgs& a, int grid, cudaStream_t s) {
-  const size_t smem = fused_smem_bytes(2, true);
-  LaunchScope scope(variant == 1 ? K_ZW_DUAL_TC : K_DZ_TOPK_TC, s);
-  return variant == 1 ? launch_pair(fused_kernel<2, true, 1>, grid, smem, s, a)
-                      : launch_pair(fused_kernel<2, true, 2>, grid, smem, s, a);
+cudaError_t launch_fused_topk(int variant, int ng, const FusedArgs& a, int grid, cudaStream_t s) {
+  const size_t smem = fused_smem_bytes(ng, true);
+  if (ng == 2) {
+    LaunchScope scope(variant == 1 ? K_ZW_DUAL_TC : K_DZ_TOPK_TC, s);
+    return variant == 1 ? launch_pair(fused_kernel<2, true, 1>, grid, fused_threads<2, true>(), smem, s, a)
+                        : launch_pair(fused_kernel<2, true, 2>, grid, fused_threads<2, true>(), smem, s, a);
+  }
+  LaunchScope scope(variant == 1 ? K_ZW_SINGLE_TC : K_DZ_TOPK_SINGLE_TC, s);
+  return variant == 1 ? launch_pair(fused_kernel<1, true, 1>, grid, fused_threads<1, true>(), smem, s, a)
+                      : launch_pair(fused_kernel<1, true, 2>, grid, fused_threads<1, true>(), smem, s, a);
 }
 
 cudaError_t launch_grad(const GradArgs& a, int grid, cudaStream_t s) {

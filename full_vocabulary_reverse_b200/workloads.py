@@ -29,6 +29,9 @@ Named workloads:
   topk_hidden     qwen_hidden inputs, top-k estimator with k = 64 and a
                   sampled token per position drawn uniformly (the estimator's
                   cost does not depend on how the tokens were drawn).
+  topk_logits     teacher_logits inputs, top-k estimator with k = 64 on the
+                  teacher-logits payload and a sampled token per position
+                  drawn uniformly.
   qwen_hidden_stats  qwen_hidden inputs, the forward also returning the
                   student's per-token entropy and the log-probability of a
                   target token per position (drawn uniformly).
@@ -67,6 +70,9 @@ WORKLOADS = {
                              targets="sampled", k=64),
     "topk_hidden": dict(dtype="bf16", B=4, Sm1=2048, H=2048, V=151936, payload="hidden",
                         reduction=REDUCE_TOKEN_MEAN, mask="prefix", weights="perturbed", seed=1236,
+                        targets="uniform", k=64),
+    "topk_logits": dict(dtype="bf16", B=4, Sm1=2048, H=2048, V=151936, payload="logits",
+                        reduction=REDUCE_TOKEN_MEAN, mask="all", weights="perturbed", seed=1238,
                         targets="uniform", k=64),
     "qwen_hidden_stats": dict(dtype="bf16", B=4, Sm1=2048, H=2048, V=151936, payload="hidden",
                               reduction=REDUCE_TOKEN_MEAN, mask="prefix", weights="perturbed", seed=1236,

@@ -88,13 +88,15 @@ typedef enum rkl_reduction {
 
 /* PR #3978, payload bullets: full.teacher_payload = hidden_states | logits.
  * LOGITS_PAIR: the student's logits are given too (rkl_*_logits_pair).
- * TOPK_HIDDEN: only for rkl_workspace_size, the workspace of
- * rkl_forward_topk_hidden / rkl_backward_topk_hidden. */
+ * TOPK_HIDDEN / TOPK_LOGITS: only for rkl_workspace_size, the workspaces of
+ * rkl_forward_topk_hidden / rkl_backward_topk_hidden and
+ * rkl_forward_topk_logits / rkl_backward_topk_logits. */
 typedef enum rkl_payload {
   RKL_PAYLOAD_HIDDEN = 0,
   RKL_PAYLOAD_LOGITS = 1,
   RKL_PAYLOAD_LOGITS_PAIR = 2,
-  RKL_PAYLOAD_TOPK_HIDDEN = 3
+  RKL_PAYLOAD_TOPK_HIDDEN = 3,
+  RKL_PAYLOAD_TOPK_LOGITS = 4
 } rkl_payload;
 
 /* Library version string (static storage). */
@@ -281,6 +283,34 @@ rkl_status rkl_backward_topk_hidden(const void* h_s, const void* h_t,
                                     const int32_t* row_idx, int32_t N, const int32_t* n_dev,
                                     const int32_t* targets,
                                     rkl_reduction reduction, const float* saved,
+                                    const float* grad_loss, const float* grad_tok,
+                                    float* dH_s, float* dW_s,
+                                    void* workspace, size_t workspace_bytes, void* stream);
+
+/* The same estimator on the logits payload (PR #3978, payload bullet 2: the
+ * teacher ships its full-vocabulary logits), bf16 only: z_s = h_s W_s^T by
+ * the tensor core, z_t the shipped teacher_logits [T, V] (V a multiple of 8)
+ * as in rkl_forward_logits.  The forward writes the fp32 z_s of at most 2048
+ * compacted rows at a time into the workspace, beside an exact fp32 copy of
+ * those rows' teacher logits, and selects / estimates on them; the backward
+ * recomputes z_s tile by tile (bitwise the same fp32 values) and runs the
+ * gradient GEMMs of rkl_backward.  Arguments as rkl_forward_logits /
+ * rkl_backward (payload RKL_PAYLOAD_LOGITS) plus k and targets as
+ * rkl_forward_topk_pair; saved [7 N]; workspace:
+ * rkl_workspace_size(RKL_PAYLOAD_TOPK_LOGITS, ...). */
+rkl_status rkl_forward_topk_logits(const void* h_s, const void* W_s,
+                                   const void* teacher_logits, rkl_dtype dtype,
+                                   int64_t B, int64_t Sm1, int64_t H, int64_t V,
+                                   const int32_t* row_idx, int32_t N, const int32_t* n_dev, int64_t k,
+                                   const int32_t* targets, rkl_reduction reduction,
+                                   float* loss_tok, float* loss, float* saved,
+                                   void* workspace, size_t workspace_bytes, void* stream);
+
+rkl_status rkl_backward_topk_logits(const void* h_s, const void* W_s,
+                                    const void* teacher_logits, rkl_dtype dtype,
+                                    int64_t B, int64_t Sm1, int64_t H, int64_t V,
+                                    const int32_t* row_idx, int32_t N, const int32_t* n_dev,
+                                    const int32_t* targets, rkl_reduction reduction, const float* saved,
                                     const float* grad_loss, const float* grad_tok,
                                     float* dH_s, float* dW_s,
                                     void* workspace, size_t workspace_bytes, void* stream);

@@ -43,10 +43,11 @@ def test_traffic_withheld_when_sources_change(monkeypatch):
 def test_every_workload_takes_one_path():
     expected = {"tiny_fp32": "hidden", "qwen_hidden": "hidden", "self_distill": "hidden", "long_prompt": "hidden",
                 "teacher_logits": "logits", "logits_pair": "pair", "logits_pair_topk": "topk_pair",
-                "topk_hidden": "topk_hidden", "multi_teacher": "multi", "qwen_hidden_stats": "stats"}
+                "topk_hidden": "topk_hidden", "topk_logits": "topk_logits", "multi_teacher": "multi",
+                "qwen_hidden_stats": "stats"}
     assert set(expected) == set(bench.WORKLOADS)
     for name, cfg in bench.WORKLOADS.items():
         path = bench.path_of(cfg)
         assert path in bench.PATHS and path == expected[name], (name, path)
         # sampled tokens are drawn exactly for the paths that read them
-        assert (cfg.get("targets") is not None) == (path in ("topk_pair", "topk_hidden", "stats")), name
+        assert (cfg.get("targets") is not None) == (path in ("topk_pair", "topk_hidden", "topk_logits", "stats")), name

@@ -22,7 +22,7 @@ ENTRY_POINTS = [
     "rkl_forward_hidden_ex", "rkl_forward_logits_ex", "rkl_backward", "rkl_forward_logits_pair",
     "rkl_backward_logits_pair", "rkl_forward_topk_pair", "rkl_backward_topk_pair", "rkl_forward_topk_hidden",
     "rkl_backward_topk_hidden", "rkl_forward_hidden_multi", "rkl_backward_hidden_multi",
-    "rkl_forward_hidden_noalloc",
+    "rkl_forward_hidden_noalloc", "rkl_forward_topk_logits", "rkl_backward_topk_logits",
 ]
 
 CALLER = r'''
