@@ -811,6 +811,15 @@ __global__ void __launch_bounds__(kThreads, 1) grad_kernel(const __grid_constant
         const bool is_h = t < nH;
         const int KB = is_h ? p.KBH : KBW;
         const uint32_t ap = i & 1;  // the accumulator is drained once per tile
+        // The tile kind selects A's layout once per tile: dH tiles read dz
+        // K-major (a 16-deep K slice is 32 B along the swizzled row), dW tiles
+        // read dz^T MN-major (a slice is 16 rows of 128 B; the two 64-wide
+        // vocab blocks lie kGA / 2 apart).  Keeping the choice out of the K
+        // loop leaves the MMA issue free of branches: a per-MMA branch on the
+        // kind measured 1330 instead of 1113 SM cycles per 64-deep K step.
+        const uint32_t idesc = is_h ? idesc_h : idesc_w;
+        const uint32_t a_step = is_h ? 32u : 2048u;
+        const uint32_t a_lbo = is_h ? 16u : static_cast<uint32_t>(kGA / 2);
         if (KB == 0) {
           // No K step (no live row): no MMA, the epilogue stores zeros; the
           // accumulator hand-off still waits for both halves to be drained.
@@ -844,15 +853,9 @@ __global__ void __launch_bounds__(kThreads, 1) grad_kernel(const __grid_constant
             const uint32_t d = tmem_base + j * (kGradBN / 2);
             const uint32_t bj = sb + j * kGBP;
 #pragma unroll
-            for (int k = 0; k < kBK / 16; ++k) {
-              const uint32_t acc_flag = (kb | k) != 0;
-              if (!is_h)
-                umma_bf16_pair(d, sdesc_sw128(sa + 2048 * k, kGA / 2, 1024), sdesc_sw128(bj + 2048 * k, kGBP / 2, 1024),
-                               idesc_w, acc_flag);
-              else
-                umma_bf16_pair(d, sdesc_sw128(sa + 32 * k, 16, 1024), sdesc_sw128(bj + 2048 * k, kGBP / 2, 1024),
-                               idesc_h, acc_flag);
-            }
+            for (int k = 0; k < kBK / 16; ++k)
+              umma_bf16_pair(d, sdesc_sw128(sa + a_step * k, a_lbo, 1024), sdesc_sw128(bj + 2048 * k, kGBP / 2, 1024),
+                             idesc, (kb | k) != 0);
           }
           if (!ok) break;
           umma_commit_pair(&empty[stage], 0x3);
