@@ -235,14 +235,17 @@ static Plan make_plan(rkl_payload payload, rkl_dtype dtype, int64_t n_max, int64
     off = align256(off + size_t(n) * sizeof(int32_t));
   }
   if (payload == RKL_PAYLOAD_TOPK_HIDDEN || payload == RKL_PAYLOAD_TOPK_LOGITS) {
-    // per-row constants of the top-k dz pass, and z_s, z_t (fp32) of one
-    // block of rows: never more than kTopkBlockRows rows of logits at a time
+    // per-row constants of the top-k dz pass, and the fp32 z_s (hidden
+    // payload: and z_t) of one block of rows: never more than
+    // kTopkBlockRows rows of logits at a time.  The teacher-logits payload
+    // selects against the shipped bf16 teacher rows directly.
     p.off_rowk = off;
     off = align256(off + size_t(6) * p.n_pad * sizeof(float));
     p.zrows = p.n_pad < kTopkBlockRows ? p.n_pad : kTopkBlockRows;
     p.zpitch = ((V + 3) / 4) * 4;
     p.off_z = off;
-    off = align256(off + size_t(2) * p.zrows * p.zpitch * sizeof(float));
+    const size_t zblocks = payload == RKL_PAYLOAD_TOPK_HIDDEN ? 2 : 1;
+    off = align256(off + zblocks * p.zrows * p.zpitch * sizeof(float));
   }
   p.total = off;
   return p;
@@ -886,7 +889,7 @@ static rkl_status forward_topk_impl(rkl_payload payload, const void* h_s, const 
                              row_idx, nullptr, N, n_dev, static_cast<int>(H * 2), T, s));
     }
     float* zs = reinterpret_cast<float*>(ws_at(workspace, pl.off_z));
-    float* zt = zs + size_t(pl.zrows) * pl.zpitch;
+    float* zt = hidden ? zs + size_t(pl.zrows) * pl.zpitch : nullptr;
     for (int r0 = 0; r0 < N; r0 += pl.zrows) {
       const int nb = (N - r0) < pl.zrows ? (N - r0) : pl.zrows;
       FusedArgs a;
@@ -903,7 +906,7 @@ static rkl_status forward_topk_impl(rkl_payload payload, const void* h_s, const 
         a.teacher_pitch = V;
       }
       RKL_TRY(make_map(&a.tm_zs, zs, true, V, nb, size_t(pl.zpitch) * 4, 32, 32));
-      RKL_TRY(make_map(&a.tm_zt, zt, true, V, nb, size_t(pl.zpitch) * 4, 32, 32));
+      if (hidden) RKL_TRY(make_map(&a.tm_zt, zt, true, V, nb, size_t(pl.zpitch) * 4, 32, 32));
       a.N = nb;
       a.n_dev = n_dev;
       a.n_base = r0;
@@ -917,8 +920,13 @@ static rkl_status forward_topk_impl(rkl_payload payload, const void* h_s, const 
       a.G = pl.VT;
       const int units = ((nb + 2 * kBM - 1) / (2 * kBM)) * a.G;  // at most
       RKL_CUDA(launch_fused_topk(1, hidden ? 2 : 1, a, 2 * units < sms ? 2 * units : sms, s));
-      RKL_CUDA(launch_topk_fwd(zs, zt, false, row_idx + r0, targets, nb, n_dev, r0, static_cast<int>(V), k,
-                               saved + 3 * size_t(r0), saved + 3 * size_t(N) + 4 * size_t(r0), pl.zpitch, true, s));
+      if (hidden)
+        RKL_CUDA(launch_topk_fwd(zs, zt, false, row_idx + r0, targets, nb, n_dev, r0, static_cast<int>(V), k,
+                                 saved + 3 * size_t(r0), saved + 3 * size_t(N) + 4 * size_t(r0), pl.zpitch, true, s));
+      else
+        RKL_CUDA(launch_topk_fwd_tlogits(zs, static_cast<const uint16_t*>(teacher), V, row_idx + r0, targets, nb,
+                                         n_dev, r0, static_cast<int>(V), k, saved + 3 * size_t(r0),
+                                         saved + 3 * size_t(N) + 4 * size_t(r0), pl.zpitch, s));
     }
   }
   if (loss_tok) RKL_CUDA(launch_scatter_loss(saved, row_idx, N, n_dev, T, loss_tok, s));

@@ -216,6 +216,13 @@ cudaError_t launch_pair_bwd(const void* zs, const void* zt, bool bf16, const int
 cudaError_t launch_topk_fwd(const void* zs, const void* zt, bool bf16, const int32_t* row_idx,
                             const int32_t* targets, int N, const int32_t* n_dev, int n_base, int V, long long k,
                             float* saved, float* saved_tk, long long zpitch, bool local, cudaStream_t s);
+// Top-k forward on the teacher-logits payload: the block's fp32 student
+// logits (block-local rows, pitch zpitch) beside the shipped bf16 teacher
+// logits (token rows row_idx[kr], pitch tpitch).
+cudaError_t launch_topk_fwd_tlogits(const float* zs, const uint16_t* teacher, long long tpitch,
+                                    const int32_t* row_idx, const int32_t* targets, int N, const int32_t* n_dev,
+                                    int n_base, int V, long long k, float* saved, float* saved_tk, long long zpitch,
+                                    cudaStream_t s);
 cudaError_t launch_topk_rowk(const float* saved, const float* saved_tk, const int32_t* row_idx,
                              const int32_t* targets, int N, const int32_t* n_dev, int n_pad, float* rowk,
                              cudaStream_t s);

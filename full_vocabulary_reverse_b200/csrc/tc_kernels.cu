@@ -457,8 +457,10 @@ __global__ void __launch_bounds__(fused_threads<NG, DZ>(), 1) fused_kernel(const
           tgt = (p.targets != nullptr && r < n_rows) ? p.targets[p.row_idx[r]] : -1;
         }
         if (NG == 1) {
+          // the top-k writer of the logits payload stores z_s only (the
+          // selection reads the shipped teacher rows itself): no teacher row
           trow = nullptr;
-          if (r < n_rows) {
+          if (r < n_rows && !(DZ && VAR == 1)) {
             const long long tr = p.teacher_rows ? p.teacher_rows[r] : r;
             trow = p.teacher + tr * p.teacher_pitch;
           }
@@ -529,11 +531,11 @@ __global__ void __launch_bounds__(fused_threads<NG, DZ>(), 1) fused_kernel(const
               stats_chunk_tail(st, zs, zt, nv);
             if (tgt >= 0 && RKL_BOUNDS(m0 + row < p.n_pad)) pick_target(zs, tgt, v0 + c * 32, p.tlogit + m0 + row);
           } else if (VAR == 1) {
-            // z_s and z_t of this 32-column chunk, fp32, one 32 x 32 box each
-            // (columns past V are clipped by the TMA store)
+            // z_s (and, NG = 2, z_t) of this 32-column chunk, fp32, one 32 x 32
+            // box each (columns past V are clipped by the TMA store)
             uint8_t* buf = stg + (warp - 2) * kStgBoxBytes;  // one staging box per warp
 #pragma unroll
-            for (int which = 0; which < 2; ++which) {
+            for (int which = 0; which < NG; ++which) {
               const float* src = which == 0 ? zs : zt;
               if (lane == 0) bulk_wait_read<0>();
               __syncwarp();

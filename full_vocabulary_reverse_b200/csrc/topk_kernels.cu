@@ -70,6 +70,12 @@ __device__ __forceinline__ uint4 tk_ldg_stream_v4(const void* p) {
   return r;
 }
 
+__device__ __forceinline__ uint2 tk_ldg_stream_v2(const void* p) {
+  uint2 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];" : "=r"(r.x), "=r"(r.y) : "l"(p));
+  return r;
+}
+
 // Order-preserving unsigned key of a float: a < b  <=>  key(a) < key(b) for
 // non-NaN values, and -0 and +0 share one key (they are equal logits).  For a
 // bf16 value only the top 16 bits carry information (the kernels mask the low
@@ -231,12 +237,12 @@ __device__ __forceinline__ void list_append(uint32_t key, int v, unsigned long l
 
 // Histogram path, pass B's decision for one logit (key, value x, token id v):
 // keys above the bin are members, keys in the bin are candidates.
-template <typename T>
-__device__ __forceinline__ void classify(uint32_t key, float x, int v, uint32_t bin, const T* zt, float lse_s,
+template <typename TT>
+__device__ __forceinline__ void classify(uint32_t key, float x, int v, uint32_t bin, const TT* zt, float lse_s,
                                          float lse_t, float& L_S, float& P_S, unsigned long long* cand,
                                          int* ncand) {
   const uint32_t kb = key >> kTopShift;
-  if (kb > bin) add_member<T>(x, zt, v, lse_s, lse_t, L_S, P_S);
+  if (kb > bin) add_member<TT>(x, zt, v, lse_s, lse_t, L_S, P_S);
   if (kb == bin) list_append(key, v, cand, ncand);
 }
 
@@ -300,15 +306,37 @@ __device__ __forceinline__ void lse_vec(const float* xs, const float* xt, float&
   }
 }
 
-template <typename T>
+// The teacher values of one student vector (the VEC logits of type T from
+// index i * VEC): one uint4 when both rows have the same type; for an fp32
+// student row beside a bf16 teacher row, the four bf16 of one 8-byte load,
+// widened exactly.
+template <typename T, typename TT>
+__device__ __forceinline__ void load_teacher_vec(const TT* zt, int i, float* out) {
+  if constexpr (std::is_same<T, TT>::value) {
+    TkIo<T>::unpack(tk_ldg_stream_v4(reinterpret_cast<const uint4*>(zt) + i), out);
+  } else {
+    static_assert(std::is_same<T, float>::value && std::is_same<TT, __nv_bfloat16>::value,
+                  "mixed rows: fp32 student logits, bf16 teacher logits");
+    const uint2 w = tk_ldg_stream_v2(reinterpret_cast<const uint2*>(zt) + i);
+    out[0] = __uint_as_float(w.x << 16);
+    out[1] = __uint_as_float(w.x & 0xFFFF0000u);
+    out[2] = __uint_as_float(w.y << 16);
+    out[3] = __uint_as_float(w.y & 0xFFFF0000u);
+  }
+}
+
+// zs rows: block-local (local) or token rows; zt rows: block-local (t_local)
+// or token rows, of type TT with pitch tpitch.  The teacher-logits payload
+// pairs the block's fp32 student logits with the shipped bf16 teacher rows.
+template <typename T, typename TT = T>
 __global__ void __launch_bounds__(kTkThreads, 6) topk_fwd_kernel(const T* __restrict__ zs_all,
-                                                              const T* __restrict__ zt_all,
+                                                              const TT* __restrict__ zt_all,
                                                               const int32_t* __restrict__ row_idx,
                                                               const int32_t* __restrict__ targets, int N,
                                                               const int32_t* __restrict__ n_dev, int n_base, int V,
                                                               long long k_sel, float* __restrict__ saved,
                                                               float* __restrict__ saved_tk, long long zpitch,
-                                                              int local) {
+                                                              int local, long long tpitch, int t_local) {
   using Io = TkIo<T>;
   constexpr int VEC = Io::VEC;
   // 32 KB: the 4096-bin histogram of pass A (histogram path) or the sort of
@@ -328,11 +356,11 @@ __global__ void __launch_bounds__(kTkThreads, 6) topk_fwd_kernel(const T* __rest
   const long long r = row_idx[kr];  // token position (sampled token)
   const long long zr = local ? kr : r;  // logit row: a block-local row, or the token position
   const T* zs = zs_all + zr * zpitch;
-  const T* zt = zt_all + zr * zpitch;
-  const bool vec_ok = ((reinterpret_cast<uintptr_t>(zs) | reinterpret_cast<uintptr_t>(zt)) & 15) == 0;
+  const TT* zt = zt_all + (t_local ? kr : r) * tpitch;
+  const bool vec_ok = (reinterpret_cast<uintptr_t>(zs) & 15) == 0 &&
+                      (reinterpret_cast<uintptr_t>(zt) & (VEC * sizeof(TT) - 1)) == 0;
   const int nvec = vec_ok ? V / VEC : 0;
   const uint4* vs = reinterpret_cast<const uint4*>(zs);
-  const uint4* vt = reinterpret_cast<const uint4*>(zt);
   // 0: empty support, 1: the whole row, 2: a proper subset to select
   const int mode = k_sel <= 0 ? 0 : (k_sel >= V ? 1 : 2);
   // small k with every thread owning logits: the k-th largest of the
@@ -367,7 +395,7 @@ __global__ void __launch_bounds__(kTkThreads, 6) topk_fwd_kernel(const T* __rest
     float xs[VEC], xt[VEC];
     const uint4 ws = tk_ldg_stream_v4(vs + i);
     Io::unpack(ws, xs);
-    Io::unpack(tk_ldg_stream_v4(vt + i), xt);
+    load_teacher_vec<T, TT>(zt, i, xt);
     if (mode == 2 && !thr) {
       if constexpr (std::is_same<T, __nv_bfloat16>::value) {
         const uint32_t wz[4] = {ws.x, ws.y, ws.z, ws.w};
@@ -401,29 +429,44 @@ __global__ void __launch_bounds__(kTkThreads, 6) topk_fwd_kernel(const T* __rest
     int i = i1 + tid;
     // two vectors of each row per step, all four loads issued first
     for (; i + kTkThreads < nvec; i += 2 * kTkThreads) {
-      const uint4 a0 = tk_ldg_stream_v4(vs + i), b0 = tk_ldg_stream_v4(vt + i);
-      const uint4 a1 = tk_ldg_stream_v4(vs + i + kTkThreads), b1 = tk_ldg_stream_v4(vt + i + kTkThreads);
-      float xs[VEC], xt[VEC];
-      list_vec<T>(a0, i * VEC, tau, buf, &s_ncand);
-      Io::unpack(a0, xs);
-      Io::unpack(b0, xt);
-      lse_vec<VEC>(xs, xt, m_s, S_s, m_t, S_t);
-      list_vec<T>(a1, (i + kTkThreads) * VEC, tau, buf, &s_ncand);
-      Io::unpack(a1, xs);
-      Io::unpack(b1, xt);
-      lse_vec<VEC>(xs, xt, m_s, S_s, m_t, S_t);
+      if constexpr (std::is_same<T, TT>::value) {
+        const uint4* vt = reinterpret_cast<const uint4*>(zt);
+        const uint4 a0 = tk_ldg_stream_v4(vs + i), b0 = tk_ldg_stream_v4(vt + i);
+        const uint4 a1 = tk_ldg_stream_v4(vs + i + kTkThreads), b1 = tk_ldg_stream_v4(vt + i + kTkThreads);
+        float xs[VEC], xt[VEC];
+        list_vec<T>(a0, i * VEC, tau, buf, &s_ncand);
+        Io::unpack(a0, xs);
+        Io::unpack(b0, xt);
+        lse_vec<VEC>(xs, xt, m_s, S_s, m_t, S_t);
+        list_vec<T>(a1, (i + kTkThreads) * VEC, tau, buf, &s_ncand);
+        Io::unpack(a1, xs);
+        Io::unpack(b1, xt);
+        lse_vec<VEC>(xs, xt, m_s, S_s, m_t, S_t);
+      } else {
+        const uint4 a0 = tk_ldg_stream_v4(vs + i);
+        const uint4 a1 = tk_ldg_stream_v4(vs + i + kTkThreads);
+        float xs[VEC], xt[VEC], xt1[VEC];
+        load_teacher_vec<T, TT>(zt, i, xt);
+        load_teacher_vec<T, TT>(zt, i + kTkThreads, xt1);
+        list_vec<T>(a0, i * VEC, tau, buf, &s_ncand);
+        Io::unpack(a0, xs);
+        lse_vec<VEC>(xs, xt, m_s, S_s, m_t, S_t);
+        list_vec<T>(a1, (i + kTkThreads) * VEC, tau, buf, &s_ncand);
+        Io::unpack(a1, xs);
+        lse_vec<VEC>(xs, xt1, m_s, S_s, m_t, S_t);
+      }
     }
     for (; i < nvec; i += kTkThreads) {
       float xs[VEC], xt[VEC];
       const uint4 ws = tk_ldg_stream_v4(vs + i);
       list_vec<T>(ws, i * VEC, tau, buf, &s_ncand);
       Io::unpack(ws, xs);
-      Io::unpack(tk_ldg_stream_v4(vt + i), xt);
+      load_teacher_vec<T, TT>(zt, i, xt);
       lse_vec<VEC>(xs, xt, m_s, S_s, m_t, S_t);
     }
   }
   for (int v = nvec * VEC + tid; v < V; v += kTkThreads) {
-    const float xs = Io::one(zs, v), xt = Io::one(zt, v);
+    const float xs = Io::one(zs, v), xt = TkIo<TT>::one(zt, v);
     lse_add(m_s, S_s, xs);
     lse_add(m_t, S_t, xt);
     if (mode == 2) {
@@ -488,7 +531,7 @@ __global__ void __launch_bounds__(kTkThreads, 6) topk_fwd_kernel(const T* __rest
     for (int i = tid; i < nvec; i += kTkThreads) {
       float xs[VEC], xt[VEC];
       Io::unpack(tk_ldg_stream_v4(vs + i), xs);
-      Io::unpack(tk_ldg_stream_v4(vt + i), xt);
+      load_teacher_vec<T, TT>(zt, i, xt);
 #pragma unroll
       for (int j = 0; j < VEC; ++j) {
         const float ls = xs[j] - lse_s;
@@ -497,7 +540,7 @@ __global__ void __launch_bounds__(kTkThreads, 6) topk_fwd_kernel(const T* __rest
         P_S += p;
       }
     }
-    for (int v = nvec * VEC + tid; v < V; v += kTkThreads) add_member<T>(Io::one(zs, v), zt, v, lse_s, lse_t, L_S, P_S);
+    for (int v = nvec * VEC + tid; v < V; v += kTkThreads) add_member<TT>(Io::one(zs, v), zt, v, lse_s, lse_t, L_S, P_S);
   } else if (mode == 2) {
     // ---- pass B (histogram path): keys above the bin are members, keys in
     // the bin are candidates; the threshold path has its list already
@@ -535,11 +578,11 @@ __global__ void __launch_bounds__(kTkThreads, 6) topk_fwd_kernel(const T* __rest
         }
 #pragma unroll
         for (int j = 0; j < VEC; ++j)
-          classify<T>(keys[j], xs[j], i * VEC + j, bin, zt, lse_s, lse_t, L_S, P_S, buf, &s_ncand);
+          classify<TT>(keys[j], xs[j], i * VEC + j, bin, zt, lse_s, lse_t, L_S, P_S, buf, &s_ncand);
       }
       for (int v = nvec * VEC + tid; v < V; v += kTkThreads) {
         const float x = Io::one(zs, v);
-        classify<T>(Io::KMASK & fkey_raw(x), x, v, bin, zt, lse_s, lse_t, L_S, P_S, buf, &s_ncand);
+        classify<TT>(Io::KMASK & fkey_raw(x), x, v, bin, zt, lse_s, lse_t, L_S, P_S, buf, &s_ncand);
       }
     }
     __syncthreads();
@@ -554,7 +597,7 @@ __global__ void __launch_bounds__(kTkThreads, 6) topk_fwd_kernel(const T* __rest
       bitonic_desc(buf, n2);
       for (int j = tid; j < need; j += kTkThreads) {
         const int v = static_cast<int>(~static_cast<uint32_t>(buf[j]));
-        add_member<T>(Io::one(zs, v), zt, v, lse_s, lse_t, L_S, P_S);
+        add_member<TT>(Io::one(zs, v), zt, v, lse_s, lse_t, L_S, P_S);
       }
       if (tid == 0) {
         const unsigned long long e = buf[need - 1];
@@ -622,7 +665,7 @@ __global__ void __launch_bounds__(kTkThreads, 6) topk_fwd_kernel(const T* __rest
             if (rank == rem - 1) s_vlast = v;
             ++rank;
           }
-          if (in) add_member<T>(xs[j], zt, v, lse_s, lse_t, L_S, P_S);
+          if (in) add_member<TT>(xs[j], zt, v, lse_s, lse_t, L_S, P_S);
         }
         carry += total;
       }
@@ -657,7 +700,7 @@ __global__ void __launch_bounds__(kTkThreads, 6) topk_fwd_kernel(const T* __rest
       const float zy = Io::one(zs, y);
       const uint32_t ky = Io::KMASK & fkey_raw(zy);
       const bool y_in = ky > kstar || (ky == kstar && y <= vlast);
-      const float wy = (zy - lse_s) - (Io::one(zt, y) - lse_t);
+      const float wy = (zy - lse_s) - (TkIo<TT>::one(zt, y) - lse_t);
       Lh = ls + (y_in ? 0.f : wy);
       a = y_in ? 0.f : wy + 1.f;
     }
@@ -779,11 +822,23 @@ cudaError_t launch_topk_fwd(const void* zs, const void* zt, bool bf16, const int
     topk_fwd_kernel<__nv_bfloat16><<<N, kTkThreads, 0, s>>>(static_cast<const __nv_bfloat16*>(zs),
                                                             static_cast<const __nv_bfloat16*>(zt), row_idx, targets,
                                                             N, n_dev, n_base, V, k, saved, saved_tk, zpitch,
-                                                            local ? 1 : 0);
+                                                            local ? 1 : 0, zpitch, local ? 1 : 0);
   else
     topk_fwd_kernel<float><<<N, kTkThreads, 0, s>>>(static_cast<const float*>(zs), static_cast<const float*>(zt),
                                                     row_idx, targets, N, n_dev, n_base, V, k, saved, saved_tk, zpitch,
-                                                    local ? 1 : 0);
+                                                    local ? 1 : 0, zpitch, local ? 1 : 0);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_topk_fwd_tlogits(const float* zs, const uint16_t* teacher, long long tpitch,
+                                    const int32_t* row_idx, const int32_t* targets, int N, const int32_t* n_dev,
+                                    int n_base, int V, long long k, float* saved, float* saved_tk, long long zpitch,
+                                    cudaStream_t s) {
+  if (N <= 0) return cudaSuccess;
+  LaunchScope scope(K_TOPK_FWD, s);
+  topk_fwd_kernel<float, __nv_bfloat16><<<N, kTkThreads, 0, s>>>(
+      zs, reinterpret_cast<const __nv_bfloat16*>(teacher), row_idx, targets, N, n_dev, n_base, V, k, saved, saved_tk,
+      zpitch, 1, tpitch, 0);
   return cudaGetLastError();
 }
 
