@@ -81,6 +81,20 @@ def test_logits_payload(red):
     assert grad_rel_err(g["dW_s"], r["dW_s"]) < GRAD_RTOL
 
 
+@pytest.mark.parametrize("H", [192, 320])
+def test_logits_payload_odd_k_steps(H):
+    # H / 64 odd: the logits-payload kernels stage 128 of K at a time, so
+    # their last stage holds one 64-deep box of data and one zero-filled box
+    # past H (whose MMAs add zeros)
+    inp = small_case(B=2, Sm1=150, H=H, V=1500, payload="logits", mask="random", seed=H)
+    g = run_gpu(inp, 1)
+    r = run_oracle(inp, 1)
+    assert_tok_close(g["loss_tok"], r["loss_tok"])
+    assert abs(float(g["loss"]) - r["loss"]) <= 1e-4 + 1e-3 * abs(r["loss"])
+    assert grad_rel_err(g["dH_s"], r["dH_s"]) < GRAD_RTOL
+    assert grad_rel_err(g["dW_s"], r["dW_s"]) < GRAD_RTOL
+
+
 def test_logits_payload_all_rows():
     inp = small_case(B=2, Sm1=128, H=64, V=520, payload="logits", mask="all", seed=22)
     g = run_gpu(inp, 1)

@@ -109,6 +109,13 @@ def test_topk_logits_device_count_and_wide_hidden():
     _check(inp, y, 64, 1, on_device=True)
 
 
+def test_topk_logits_odd_k_steps():
+    # H = 192: the last 128-deep stage of the writer / dz kernels is half
+    # zero-filled; the selection reads the shipped teacher rows directly
+    inp, y = _case(2, 150, 192, 1500, seed=185)
+    _check(inp, y, 40, 1)
+
+
 def test_topk_logits_whole_row_equals_exact_loss():
     inp, y = _case(2, 120, 128, 776, seed=180)
     lt, loss, dH, dW, N = _run(inp, y, 776, 1)
