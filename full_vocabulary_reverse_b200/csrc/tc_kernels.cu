@@ -426,7 +426,7 @@ __global__ void __launch_bounds__(fused_threads<NG, DZ>(), 1) fused_kernel(const
     int cur_m0 = -1;
     float lse2 = 0.f, cst = 0.f, g_row = 0.f;
     float tk_C = 0.f, tk_ga = 0.f;     // top-k dz: C and g a
-    uint32_t tk_kstar = 0u;
+    float tk_thr = 0.f;  // top-k dz: the support bound K* as a float
     int tk_vlast = -1, tk_y = -1;
     int tgt = -1;  // target column of this row (forward with targets), else -1
     const uint16_t* trow = nullptr;
@@ -446,7 +446,13 @@ __global__ void __launch_bounds__(fused_threads<NG, DZ>(), 1) fused_kernel(const
           cst = p.rowk[r];
           tk_C = p.rowk[p.n_pad + r];
           tk_ga = g_row * p.rowk[2 * p.n_pad + r];
-          tk_kstar = __float_as_uint(p.rowk[3 * p.n_pad + r]);
+          // K* is an order-preserving key (-0 and +0 one key); as a float the
+          // test key(z) > K* is z > thr and key(z) = K* is z == thr (IEEE
+          // compares -0 == +0).  K* = 0 (below every key: the whole row) is
+          // -inf; K* = ~0 (above every key: no member) decodes to a NaN, which
+          // no compare passes.
+          const uint32_t kk = __float_as_uint(p.rowk[3 * p.n_pad + r]);
+          tk_thr = kk == 0u ? -INFINITY : __uint_as_float((kk & 0x80000000u) ? (kk & 0x7FFFFFFFu) : ~kk);
           tk_vlast = __float_as_int(p.rowk[4 * p.n_pad + r]);
           tk_y = __float_as_int(p.rowk[5 * p.n_pad + r]);
         } else if (DZ && VAR == 0) {
@@ -559,19 +565,17 @@ __global__ void __launch_bounds__(fused_threads<NG, DZ>(), 1) fused_kernel(const
             if (VAR == 2) {
               // top-k: dz = g p_s ([v in S](w + 1) - C) + [v = y] g a
               const int col0 = v0 + c * 32;
+              const int vl = tk_vlast - col0, yo = tk_y - col0;  // offsets in this chunk
 #pragma unroll
               for (int j = 0; j < 32; j += 2) {
                 float d[2];
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                   const float x = zs[j + h];
-                  const uint32_t u = x == 0.f ? 0u : __float_as_uint(x);
-                  const uint32_t key = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-                  const int v = col0 + j + h;
-                  const bool in = key > tk_kstar || (key == tk_kstar && v <= tk_vlast);
+                  const bool in = x > tk_thr || (x == tk_thr && j + h <= vl);
                   const float pr = ex2(fmaf(x, kLog2e, -lse2));
                   const float coef = (in ? (x - zt[j + h]) + cst + 1.f : 0.f) - tk_C;
-                  d[h] = g_row * pr * coef + (v == tk_y ? tk_ga : 0.f);
+                  d[h] = g_row * pr * coef + (j + h == yo ? tk_ga : 0.f);
                 }
                 pk[j / 2] = pack_bf16x2(d[0], d[1]);
               }
