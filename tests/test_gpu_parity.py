@@ -86,7 +86,7 @@ def test_logits_payload_odd_k_steps(H):
     # H / 64 odd: the logits-payload kernels stage 128 of K at a time, so
     # their last stage holds one 64-deep box of data and one zero-filled box
     # past H (whose MMAs add zeros)
-    inp = small_case(B=2, Sm1=150, H=H, V=1500, payload="logits", mask="random", seed=H)
+    inp = small_case(B=2, Sm1=150, H=H, V=1504, payload="logits", mask="random", seed=H)
     g = run_gpu(inp, 1)
     r = run_oracle(inp, 1)
     assert_tok_close(g["loss_tok"], r["loss_tok"])
