@@ -22,10 +22,12 @@
 //   accumulators in TMEM, TMA store / TMA reduce-add epilogue.
 //
 // All kernels run on 2-CTA clusters with tcgen05.mma.cta_group::2 issued by
-// one thread of the leader CTA.  Warp roles (320 threads): warp 0 = TMA
-// producer, warp 1 = MMA issuer, warps 2..9 = epilogue (warp w reads TMEM
-// lanes 32*(w%4) .. +31, i.e. one tile row per thread, and half of the
-// columns).  Warp 2 also allocates / frees TMEM.
+// one thread of the leader CTA.  Warp roles: warp 0 = TMA producer, warp 1 =
+// MMA issuer, warps 2.. = epilogue, 8 warps (320 threads) in the store
+// kernels and the logits-payload forward, 16 (576 threads) in the
+// hidden-payload forward.  Epilogue warp w reads TMEM lanes 32*(w%4) .. +31,
+// i.e. one tile row per thread, and 1 / (E / 4) of the columns for E
+// epilogue warps.  Warp 2 also allocates / frees TMEM.
 #include <cuda_bf16.h>
 
 #include "bounds.cuh"
