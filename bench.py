@@ -331,6 +331,14 @@ def kernel_profile():
 def algorithmic_work(prob, N):
     """Per-kernel algorithmic flops (tensor kernels) or bytes (bandwidth kernels) of one step."""
     H, V = prob.H, prob.V
+    if prob.dt != 0:
+        # fp32 inputs: the FFMA (SIMT) kernels, bound by the FP32 pipe
+        w = {"fwd_simt_fp32": ("alu", (2.0 if prob.logits else 4.0) * N * H * V),
+             "dz_simt_fp32": ("alu", (2.0 if prob.logits else 4.0) * N * H * V),
+             "grad_simt_fp32": ("alu", 4.0 * N * H * V)}
+        if prob.logits:
+            w["teacher_lse"] = ("hbm", 4.0 * N * V + 4.0 * N)
+        return w
     if prob.topk:
         # the estimator must read both logit rows once and write dz once
         return {"topk_fwd": ("hbm", 4.0 * N * V + 28.0 * N),
@@ -339,11 +347,10 @@ def algorithmic_work(prob, N):
         return {"pair_fwd": ("hbm", 4.0 * N * V + 16.0 * N),
                 "pair_bwd": ("hbm", 4.0 * N * V + 2.0 * prob.T * V)}
     if prob.topk_logits:
-        # writer 2 N H V (z_s; the shipped z_t is copied beside it), the
-        # teacher rows read once (2 N V bytes) there, selection / estimate
-        # over the written fp32 block (2 x 4 N V bytes), dz recompute 2 N H V
-        # (+ the teacher rows again), grad 4 N H V
-        return {"zw_single_tc": ("tensor", 2.0 * N * H * V), "topk_fwd": ("hbm", 8.0 * N * V),
+        # writer 2 N H V (z_s), selection / estimate over the written fp32 z_s
+        # block beside the shipped bf16 teacher rows (4 N V + 2 N V bytes),
+        # dz recompute 2 N H V (+ the teacher rows again), grad 4 N H V
+        return {"zw_single_tc": ("tensor", 2.0 * N * H * V), "topk_fwd": ("hbm", 6.0 * N * V),
                 "dz_topk_single_tc": ("tensor", 2.0 * N * H * V), "grad_dw_dh_tc": ("tensor", 4.0 * N * H * V)}
     if prob.topk_hidden:
         # writer 4 N H V (z_s and z_t), selection/estimate over the written fp32
@@ -611,18 +618,31 @@ def run_gpu(args, rank, world, dist):
         # roofline (the sustained one is for seconds-long runs)
         peak = pk["bf16_tflops"]
         unit = "TFLOP/s"
+    elif bound == "alu":
+        # FP32 FMA pipe: 148 SMs x 128 lanes x 2 flop per cycle at the max SM clock
+        achieved = per_launch / avg_launch_s / 1e12
+        peak = 148 * 128 * 2 * (pk.get("sm_max_mhz") or 1965.0) * 1e6 / 1e12
+        unit = "TFLOP/s"
     else:
         achieved = per_launch / avg_launch_s / 1e9
         peak = pk["hbm_gbs"]
         unit = "GB/s"
-    extra = {}
+    extra, extra_tc = {}, {}
     for k, (b, w) in work.items():
-        if b == "hbm" and k in prof:
-            per_l = w * args.steps / prof[k]["launches"]
-            ach = per_l / (prof[k]["ms"] / prof[k]["launches"] / 1000.0) / 1e9
+        if k not in prof:
+            continue
+        per_l = w * args.steps / prof[k]["launches"]
+        avg_s = prof[k]["ms"] / prof[k]["launches"] / 1000.0
+        if b == "hbm":
+            ach = per_l / avg_s / 1e9
             extra[k] = {"bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
                         "frac": ach / pk["hbm_gbs"], "traffic": traffic_for(k, prob.name)}
-    step_flops = sum(w for b, w in work.values() if b == "tensor")
+        elif b == "tensor":
+            # every tensor-core kernel of the step against the same burst peak
+            ach = per_l / avg_s / 1e12
+            extra_tc[k] = {"bound": "tensor", "achieved": ach, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                           "frac": ach / pk["bf16_tflops"], "traffic": traffic_for(k, prob.name)}
+    step_flops = sum(w for b, w in work.values() if b in ("tensor", "alu"))
     step_tflops = step_flops * args.steps / (ms / 1000.0) / 1e12
     csum = clk.summary()
     clock_ratio = (csum["sm_mhz"] / csum["sm_max_mhz"]) if (csum.get("sm_mhz") and csum.get("sm_max_mhz")) else None
@@ -648,13 +668,15 @@ def run_gpu(args, rank, world, dist):
                        / 1e9)},
         "roofline": {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
                      "frac": achieved / peak, "traffic": traffic_for(dom, prob.name),
-                     "peak_source": "%s %s" % (pk["source"], "bf16 burst" if bound == "tensor" else "hbm copy"),
+                     "peak_source": "%s %s" % (pk["source"], {"tensor": "bf16 burst", "hbm": "hbm copy"}.get(
+                         bound, "fp32 FMA pipe at the max SM clock")),
                      "frac_of_sustained": achieved / pk["bf16_tflops_sustained"] if bound == "tensor" else None,
-                     "frac_of_datasheet": achieved / (DATASHEET_BF16_TFLOPS if bound == "tensor"
-                                                      else DATASHEET_HBM_GBS),
+                     "frac_of_datasheet": (achieved / (DATASHEET_BF16_TFLOPS if bound == "tensor"
+                                                       else DATASHEET_HBM_GBS)) if bound != "alu" else None,
                      "sm_clock_ratio": clock_ratio,
                      "split_pass_ms_per_step": ms_prof / args.steps},
         "roofline_hbm_kernels": extra or None,
+        "roofline_tc_kernels": extra_tc or None,
         "step_tflops": step_tflops, "step_tc_frac_burst": step_tflops / pk["bf16_tflops"],
         "step_tc_frac_sustained": step_tflops / pk["bf16_tflops_sustained"],
         "step_tc_frac_datasheet": step_tflops / DATASHEET_BF16_TFLOPS,
